@@ -1,0 +1,335 @@
+"""Benchmark of the LVSA block-sparse attention path on B200.
+
+A step is one pass of the whole LVSA hot path over one batch of the Wan-2.1-
+1.3B-like 6x-length workload (B=1, 12 heads, D=128, grid 126x30x52 = 196,560
+tokens, C=21, T_per=12): lvsa_mask(s) -> reorder_fwd(Q,K,V) -> bsattn ->
+reorder_inv(O), with s = step mod T_per.  Inputs (1.8 GB) exceed the 126 MB
+L2, so no flush is needed between steps.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Under torchrun (N > 1) every rank runs its own batch (the path shards over
+batch x heads with no data exchange): weak scaling, max time over ranks.
+`--impl reference` times the CPU fp64 oracle on a bounded sample instead.
+Prints one JSON line (rank 0).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from synth import CONFIGS, make_qkv  # noqa: E402
+
+METRIC = "bsattn ms/call + attended TFLOP/s (% BF16 peak), Wan-1.3B-shape 6× length LVSA"
+
+
+def attended_flops(w) -> float:
+    # T*C*P^2 (query, key) pairs per head, 4*D flops each (QK and PV products)
+    return float(w.T * w.lvsa_C * w.P * w.P) * w.Hh * w.B * 4 * w.D
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return d, "measured"
+    except Exception:
+        return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}, "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled every 200 ms."""
+
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, dev: int):
+        self.proc = None
+        self.path = None
+        try:
+            uuid = str(torch.cuda.get_device_properties(dev).uuid)
+            ident = uuid if uuid.startswith("GPU-") else "GPU-" + uuid
+        except Exception:
+            ident = str(dev)
+        self.ident = ident
+
+    def start(self):
+        try:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", self.ident, f"--query-gpu={self.Q}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if not self.proc:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) >= 9:
+                    rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return None
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i] == "Active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons,
+                "samples": len(rows)}
+
+
+def cpu_baseline(w, q_h, k_h, v_h, budget_s: float, seed: int = 0):
+    """The oracle, as it stands, on a bounded sample of the same workload:
+    the LVSA mask of step 0 in full, then masked attention of sampled query
+    blocks of one head.  Returns (attended TFLOP/s, threads, description)."""
+    import oracle
+    nbf = -(-w.P // 128)
+    t0 = time.perf_counter()
+    A = oracle.lvsa_frame_sets(w.T, w.lvsa_C, w.lvsa_T_per, 0)
+    rp, ci = oracle.lvsa_block_csr(A, nbf)
+    perm, Np = oracle.frame_layout_perm(w.T, w.H, w.W, 128)
+    valid = oracle.slot_valid(perm, Np)
+    qs, ks, vs = (oracle.reorder_fwd(x, perm, Np) for x in (q_h, k_h, v_h))
+    setup = time.perf_counter() - t0
+    rng = np.random.default_rng(seed)
+    nb = w.T * nbf
+    done, flops, t_att = 0, 0.0, 0.0
+    while t_att < budget_s and done < nb:
+        qb = int(rng.integers(0, nb))
+        t1 = time.perf_counter()
+        oracle.masked_attention(qs, ks, vs, valid, 128, rp, ci, False, 1 / math.sqrt(w.D),
+                                q_blocks=[qb], heads=[(0, 0)])
+        t_att += time.perf_counter() - t1
+        nq = int(valid[qb * 128:(qb + 1) * 128].sum())
+        keys = sum(int(valid[c * 128:(c + 1) * 128].sum()) for c in ci[rp[qb]:rp[qb + 1]])
+        flops += 4.0 * w.D * nq * keys
+        done += 1
+    threads = torch.get_num_threads()
+    try:
+        import threadpoolctl
+        info = threadpoolctl.threadpool_info()
+        threads = max([i.get("num_threads", 1) for i in info] + [1])
+    except Exception:
+        pass
+    desc = (f"oracle masked attention on {done} random query blocks of head 0 (of "
+            f"{nb} x {w.Hh}), LVSA s=0; mask+layout set-up {setup:.1f}s excluded")
+    return flops / t_att / 1e12, threads, desc, t_att
+
+
+def run_reference(args, rank, world):
+    """Reference arm: the CPU fp64 oracle, timed on the host cores."""
+    if rank != 0:
+        return
+    w = CONFIGS[args.config]
+    q, k, v = make_qkv(w, device="cpu")
+    q_h, k_h, v_h = (x[:, :, :1].float().numpy().astype(np.float64) for x in (q, k, v))
+    del q, k, v
+    vals = []
+    desc, thr = "", 1
+    for i in range(args.warmup + args.steps):
+        val, thr, desc, _ = cpu_baseline(w, q_h, k_h, v_h, budget_s=args.ref_step_s, seed=i)
+        if i >= args.warmup:
+            vals.append(val)
+    value = statistics.mean(vals)
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": None, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": w.name, "global_batch": w.B, "seq_len": w.N,
+                   "parallelism": f"dp{world}"},
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": thr, "kind": "oracle",
+                         "sample": desc},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--config", type=int, default=3)
+    ap.add_argument("--e2e-steps", type=int, default=3)
+    ap.add_argument("--cpu-budget-s", type=float, default=12.0)
+    ap.add_argument("--ref-step-s", type=float, default=4.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+
+    rank = int(os.environ.get("RANK", 0))
+    world = int(os.environ.get("WORLD_SIZE", 1))
+    local = int(os.environ.get("LOCAL_RANK", 0))
+    if args.impl == "reference":
+        run_reference(args, rank, world)
+        return
+    if args.warmup < 3:
+        raise SystemExit("at least 3 warm-up steps")
+
+    import block_sparse_attention_49_b200 as bsa
+    from block_sparse_attention_49_b200.pipeline import LvsaAttention
+
+    torch.cuda.set_device(local)
+    dist = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+
+    w = CONFIGS[args.config]
+    flops_step = attended_flops(w)
+    q, k, v = make_qkv(w, device="cuda")
+    att = LvsaAttention(w.B, w.Hh, w.D, w.T, w.H, w.W, w.lvsa_C, w.lvsa_T_per, block=128)
+    out = torch.empty_like(q)
+    stream = torch.cuda.current_stream()
+    launches_per_step = 4  # lvsa_mask, reorder_fwd, bsattn, reorder_inv
+
+    ev = []
+
+    def step(i, record):
+        s = i % w.lvsa_T_per
+        att.mask(s)
+        att.gather(q, k, v)
+        if record:
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            att.attend(per_head=False)
+            e1.record(stream)
+            ev.append((e0, e1))
+        else:
+            att.attend(per_head=False)
+        att.scatter(out)
+
+    for i in range(args.warmup):
+        step(i, False)
+    bsa.bsa_poll_status(att.plan)
+    torch.cuda.synchronize()
+    if dist:
+        dist.barrier()
+    clocks = ClockSampler(local)
+    clocks.start()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    t0.record(stream)
+    for i in range(args.steps):
+        step(args.warmup + i, True)
+    t1.record(stream)
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    bsa.bsa_poll_status(att.plan)
+    ms = t0.elapsed_time(t1) / args.steps
+    attn_ms = statistics.mean(a.elapsed_time(b) for a, b in ev)
+    if dist:
+        tt = torch.tensor([ms, attn_ms], device="cuda")
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        ms, attn_ms = float(tt[0]), float(tt[1])
+
+    # end to end through the public API with host buffers: pinned H2D of the
+    # step's Q, K, V, the step, D2H of O
+    hq, hk, hv = (x.cpu().pin_memory() for x in (q, k, v))
+    ho = torch.empty_like(hq).pin_memory()
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    torch.cuda.synchronize()
+    if dist:
+        dist.barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for i in range(args.e2e_steps):
+        dq.copy_(hq, non_blocking=True)
+        dk.copy_(hk, non_blocking=True)
+        dv.copy_(hv, non_blocking=True)
+        s = i % w.lvsa_T_per
+        att.mask(s)
+        att.gather(dq, dk, dv)
+        att.attend(per_head=False)
+        att.scatter(out)
+        ho.copy_(out, non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = e0.elapsed_time(e1) / args.e2e_steps
+    if dist:
+        tt = torch.tensor([e2e_ms], device="cuda")
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        e2e_ms = float(tt[0])
+    bsa.bsa_poll_status(att.plan)
+
+    pk, pk_kind = peaks()
+    peak = pk.get("bf16_tflops_sustained", pk["bf16_tflops"])
+    attn_tflops = flops_step / (attn_ms * 1e-3) / 1e12
+    value = world * flops_step / (ms * 1e-3) / 1e12
+    line = {
+        "metric": METRIC,
+        "value": value,
+        "unit": "TFLOP/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": ms,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic",
+        "config": {"workload": w.name, "global_batch": w.B * world, "seq_len": w.N,
+                   "heads": w.Hh, "head_dim": w.D, "lvsa_C": w.lvsa_C,
+                   "lvsa_T_per": w.lvsa_T_per, "steps_s": "s = step mod T_per",
+                   "parallelism": f"dp{world}",
+                   "l2": "inputs (1.8 GB) larger than L2; no flush"},
+        "bsattn_ms_per_call": attn_ms,
+        "bsattn_attended_tflops": attn_tflops,
+        "bsattn_pct_bf16_peak": 100.0 * attn_tflops / peak,
+        "attended_tflop_per_call": flops_step / 1e12,
+        "roofline": {"bound": "tensor", "achieved": attn_tflops, "peak": peak,
+                     "unit": "TFLOP/s", "frac": attn_tflops / peak, "traffic": None,
+                     "peak_kind": f"{pk_kind} bf16 sustained (kernel timed inside a long step)"},
+        "gpu_launches": launches_per_step * args.steps,
+        "clocks": clk,
+        "e2e": {"value": world * flops_step / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+                "ms_per_step": e2e_ms,
+                "h2d_bytes_per_step": 3 * q.numel() * q.element_size(),
+                "d2h_bytes_per_step": out.numel() * out.element_size()},
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        q_h, k_h, v_h = (x[:, :, :1].float().cpu().numpy().astype(np.float64) for x in (q, k, v))
+        val, thr, desc, _ = cpu_baseline(w, q_h, k_h, v_h, budget_s=args.cpu_budget_s)
+        line["cpu_baseline"] = {"value": val, "unit": "TFLOP/s", "cores": thr, "kind": "oracle",
+                                "sample": desc}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if dist:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,223 @@
+"""Python binding of libbsattn.so: block-sparse attention over [t,h,w] video
+tokens on NVIDIA B200 (sm_100a).
+
+Argument marshalling only: every computation runs in the library's CUDA
+kernels.  The binding passes device pointers (`tensor.data_ptr()`) and the
+current torch CUDA stream, and raises BsaError on any non-OK status.  If the
+library is missing, importing the binding's functions raises; there is no
+fallback of any kind.
+
+Entry points keep the C names (bsa_plan_create, bsa_lvsa_mask,
+bsa_draft_mask, bsa_reorder_fwd, bsa_reorder_inv, bsa_attn_fwd,
+bsa_poll_status, ...); see include/bsattn.h for their exact contracts.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+__all__ = [
+    "BsaError", "Plan", "LAYOUT_FRAME", "LAYOUT_TILE", "lib_path", "load",
+    "bsa_plan_create", "bsa_plan_destroy", "bsa_padded_tokens", "bsa_num_blocks",
+    "bsa_block_size", "bsa_lvsa_mask", "bsa_lvsa_nnz", "bsa_draft_keep_count",
+    "bsa_draft_workspace_bytes", "bsa_draft_mask", "bsa_reorder_fwd", "bsa_reorder_inv",
+    "bsa_attn_fwd", "bsa_poll_status", "bsa_set_wait_limit_ns", "bsa_selftest_timeout",
+    "bsa_last_error", "bsa_version", "EXPORTED_SYMBOLS",
+]
+
+LAYOUT_FRAME = 0
+LAYOUT_TILE = 1
+
+STATUS = {0: "BSA_OK", 1: "BSA_ERR_INVALID_ARG", 2: "BSA_ERR_UNSUPPORTED",
+          3: "BSA_ERR_ALIGNMENT", 4: "BSA_ERR_CUDA", 5: "BSA_ERR_TIMEOUT",
+          6: "BSA_ERR_BAD_BLOCKLIST"}
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+lib_path = os.path.join(_HERE, "libbsattn.so")
+
+_c_int, _c_i64, _c_sz, _c_p, _c_u64 = (ctypes.c_int, ctypes.c_int64, ctypes.c_size_t,
+                                       ctypes.c_void_p, ctypes.c_uint64)
+
+# name -> (restype, argtypes)
+_SIGS = {
+    "bsa_plan_create": (_c_int, [ctypes.POINTER(_c_p)] + [_c_int] * 10),
+    "bsa_plan_destroy": (_c_int, [_c_p]),
+    "bsa_padded_tokens": (_c_i64, [_c_p]),
+    "bsa_num_blocks": (_c_i64, [_c_p]),
+    "bsa_block_size": (_c_int, [_c_p]),
+    "bsa_lvsa_mask": (_c_int, [_c_p, _c_int, _c_int, _c_int, _c_p, _c_p, _c_p, _c_p]),
+    "bsa_lvsa_nnz": (_c_i64, [_c_p, _c_int]),
+    "bsa_draft_keep_count": (_c_int, [_c_p, _c_int]),
+    "bsa_draft_workspace_bytes": (_c_sz, [_c_p]),
+    "bsa_draft_mask": (_c_int, [_c_p, _c_p, _c_p, _c_int, _c_p, _c_p, _c_p, _c_p, _c_sz, _c_p]),
+    "bsa_reorder_fwd": (_c_int, [_c_p] * 8),
+    "bsa_reorder_inv": (_c_int, [_c_p, _c_p, _c_p, _c_p]),
+    "bsa_attn_fwd": (_c_int, [_c_p, _c_p, _c_p, _c_p, _c_p, _c_p, _c_int, ctypes.c_float, _c_p,
+                              _c_p, _c_p]),
+    "bsa_poll_status": (_c_int, [_c_p, _c_p]),
+    "bsa_set_wait_limit_ns": (_c_int, [_c_p, _c_u64]),
+    "bsa_selftest_timeout": (_c_int, [_c_p, _c_u64, _c_p]),
+    "bsa_last_error": (ctypes.c_char_p, []),
+    "bsa_version": (ctypes.c_char_p, []),
+}
+EXPORTED_SYMBOLS = tuple(_SIGS)
+
+_lib = None
+
+
+class BsaError(RuntimeError):
+    def __init__(self, status: int, where: str, msg: str):
+        super().__init__(f"{where}: {STATUS.get(status, status)}: {msg}")
+        self.status = status
+
+
+def load():
+    """Load libbsattn.so (building nothing) and return the ctypes handle."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(lib_path):
+            raise ImportError(f"libbsattn.so not built ({lib_path}); run "
+                              "python -m block_sparse_attention_49_b200._build")
+        lib = ctypes.CDLL(lib_path)
+        for name, (res, args) in _SIGS.items():
+            fn = getattr(lib, name)
+            fn.restype = res
+            fn.argtypes = args
+        _lib = lib
+    return _lib
+
+
+def _check(st: int, where: str):
+    if st != 0:
+        raise BsaError(st, where, load().bsa_last_error().decode())
+
+
+def _ptr(t) -> Optional[int]:
+    """Device address of a tensor (or None)."""
+    if t is None:
+        return None
+    if isinstance(t, int):
+        return t
+    if not t.is_cuda:
+        raise ValueError("tensor must live on a CUDA device")
+    if not t.is_contiguous():
+        raise ValueError("tensor must be contiguous")
+    return t.data_ptr()
+
+
+def _stream(stream) -> Optional[int]:
+    if stream is not None:
+        return stream if isinstance(stream, int) else stream.cuda_stream
+    import torch
+    return torch.cuda.current_stream().cuda_stream
+
+
+class Plan:
+    """Owns a bsa_plan_t; geometry of one attention problem."""
+
+    def __init__(self, B, Hh, D, T, H, W, layout, pool_h=0, pool_w=0, block=128):
+        self.B, self.Hh, self.D, self.T, self.H, self.W = B, Hh, D, T, H, W
+        self.layout, self.pool_h, self.pool_w = layout, pool_h, pool_w
+        h = _c_p()
+        _check(load().bsa_plan_create(ctypes.byref(h), B, Hh, D, T, H, W, layout, pool_h,
+                                      pool_w, block), "bsa_plan_create")
+        self.handle = h
+        self.Npad = int(load().bsa_padded_tokens(h))
+        self.nblocks = int(load().bsa_num_blocks(h))
+        self.block = int(load().bsa_block_size(h))
+
+    def close(self):
+        if getattr(self, "handle", None):
+            _check(load().bsa_plan_destroy(self.handle), "bsa_plan_destroy")
+            self.handle = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+
+def bsa_plan_create(B, Hh, D, T, H, W, layout, pool_h=0, pool_w=0, block=128) -> Plan:
+    return Plan(B, Hh, D, T, H, W, layout, pool_h, pool_w, block)
+
+
+def bsa_plan_destroy(plan: Plan):
+    plan.close()
+
+
+def bsa_padded_tokens(plan: Plan) -> int:
+    return int(load().bsa_padded_tokens(plan.handle))
+
+
+def bsa_num_blocks(plan: Plan) -> int:
+    return int(load().bsa_num_blocks(plan.handle))
+
+
+def bsa_block_size(plan: Plan) -> int:
+    return int(load().bsa_block_size(plan.handle))
+
+
+def bsa_lvsa_nnz(plan: Plan, C: int) -> int:
+    return int(load().bsa_lvsa_nnz(plan.handle, C))
+
+
+def bsa_lvsa_mask(plan: Plan, C: int, T_per: int, s: int, frame_sets, row_ptr, col_idx,
+                  stream=None):
+    _check(load().bsa_lvsa_mask(plan.handle, C, T_per, s, _ptr(frame_sets), _ptr(row_ptr),
+                                _ptr(col_idx), _stream(stream)), "bsa_lvsa_mask")
+
+
+def bsa_draft_keep_count(plan: Plan, sparsity_pct: int) -> int:
+    return int(load().bsa_draft_keep_count(plan.handle, sparsity_pct))
+
+
+def bsa_draft_workspace_bytes(plan: Plan) -> int:
+    return int(load().bsa_draft_workspace_bytes(plan.handle))
+
+
+def bsa_draft_mask(plan: Plan, q_slots, k_slots, sparsity_pct: int, row_ptr, kv_idx,
+                   draft_map, workspace, stream=None):
+    nbytes = workspace.numel() * workspace.element_size()
+    _check(load().bsa_draft_mask(plan.handle, _ptr(q_slots), _ptr(k_slots), sparsity_pct,
+                                 _ptr(row_ptr), _ptr(kv_idx), _ptr(draft_map), _ptr(workspace),
+                                 nbytes, _stream(stream)), "bsa_draft_mask")
+
+
+def bsa_reorder_fwd(plan: Plan, x0, y0, x1=None, y1=None, x2=None, y2=None, stream=None):
+    _check(load().bsa_reorder_fwd(plan.handle, _ptr(x0), _ptr(y0), _ptr(x1), _ptr(y1),
+                                  _ptr(x2), _ptr(y2), _stream(stream)), "bsa_reorder_fwd")
+
+
+def bsa_reorder_inv(plan: Plan, x_slots, x_nat, stream=None):
+    _check(load().bsa_reorder_inv(plan.handle, _ptr(x_slots), _ptr(x_nat), _stream(stream)),
+           "bsa_reorder_inv")
+
+
+def bsa_attn_fwd(plan: Plan, q, k, v, row_ptr, col_idx, per_head_lists: bool, scale: float,
+                 o, lse=None, stream=None):
+    _check(load().bsa_attn_fwd(plan.handle, _ptr(q), _ptr(k), _ptr(v), _ptr(row_ptr),
+                               _ptr(col_idx), int(bool(per_head_lists)), float(scale), _ptr(o),
+                               _ptr(lse), _stream(stream)), "bsa_attn_fwd")
+
+
+def bsa_poll_status(plan: Plan, stream=None):
+    _check(load().bsa_poll_status(plan.handle, _stream(stream)), "bsa_poll_status")
+
+
+def bsa_set_wait_limit_ns(plan: Plan, ns: int):
+    _check(load().bsa_set_wait_limit_ns(plan.handle, int(ns)), "bsa_set_wait_limit_ns")
+
+
+def bsa_selftest_timeout(plan: Plan, limit_ns: int, stream=None):
+    _check(load().bsa_selftest_timeout(plan.handle, int(limit_ns), _stream(stream)),
+           "bsa_selftest_timeout")
+
+
+def bsa_last_error() -> str:
+    return load().bsa_last_error().decode()
+
+
+def bsa_version() -> str:
+    return load().bsa_version().decode()

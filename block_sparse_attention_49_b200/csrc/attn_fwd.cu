@@ -1,0 +1,539 @@
+// Block-sparse softmax attention forward on sm_100a tensor cores.
+//
+// What it computes ("LVSA: Training-Free Sparse Attention for Long Video
+// Diffusion", section 2: attention restricted to the blocks of the frame set
+// A(t); Draft Attention article: the sparse mask guides full-resolution
+// block-sparse attention): for every query slot, softmax(scale * q.k) over
+// the non-empty key slots of the key blocks its query block may attend,
+// weighted sum of their values; plus the log-sum-exp.
+//
+// How (one CTA per 128-slot query tile; 8 warps):
+//   warp 0     TMA producer: Q tile once, then K and V tiles of every listed
+//              key tile into an NS-deep shared-memory ring (128-byte swizzle).
+//   warp 1     MMA issuer (one thread): S = Q K^T into tensor memory (two S
+//              buffers so the next S overlaps the softmax of the current
+//              one), then O += P V with P read from tensor memory.
+//   warps 4-7  softmax, one query row per thread (= one TMEM lane): reads S,
+//              masks empty / disallowed keys, keeps the running max and sum,
+//              writes P as bf16 over the upper half of its S buffer, rescales
+//              O only when the running max grew by more than 2^8 (the stale
+//              max stays exact because numerator and denominator share it),
+//              and finally normalises O and stores it.
+// Every wait is bounded; a wait that runs out records a timeout in the
+// plan's status word and the CTA leaves without trapping.
+#include <cuda_bf16.h>
+#include <cudaTypedefs.h>
+
+#include <cmath>
+
+#include "bsa_internal.cuh"
+#include "ptx.cuh"
+
+namespace bsa {
+namespace {
+
+constexpr int kTile = 128;          // query / key tile (slots)
+constexpr int kThreads = 256;
+constexpr int kFineMaxTiles = 2048; // key tiles addressable by the sub-tile-block path
+constexpr uint32_t kFull = 0xffffffffu;
+
+template <int D, bool FINE>
+struct AttnCfg {
+  static constexpr int kChunks = D / 64;  // 64-column (128-byte) swizzle panels
+  static constexpr int kPanel = kTile * 128;
+  static constexpr int kQBytes = kTile * D * 2;
+  static constexpr int kKVBytes = kTile * D * 2;
+  static constexpr int NS = (D == 128) ? (FINE ? 2 : 3) : 4;
+  static constexpr int kOffQ = 0;
+  static constexpr int kOffK = kQBytes;
+  static constexpr int kOffV = kOffK + NS * kKVBytes;
+  static constexpr int kOffBar = kOffV + NS * kKVBytes;
+  static constexpr int kNumBars = 1 + 3 * NS + 2 + 2;
+  static constexpr int kOffMisc = kOffBar + kNumBars * 8;
+  static constexpr int kOffList = kOffMisc + 16;
+  static constexpr int kOffBitmap = kOffList + (FINE ? kFineMaxTiles * 2 : 0);
+  static constexpr int kBytes = kOffBitmap + (FINE ? kFineMaxTiles / 8 : 0);
+  static constexpr int kSmem = kBytes + 1024;  // room to align the base to 1024
+  static constexpr uint32_t kTmemCols = 512;   // S0 | S1 | O
+  static_assert(kSmem <= 232448, "shared memory budget");
+};
+
+struct AttnParams {
+  int Hh;
+  int block;          // slots per block of the block list
+  int64_t Npad;       // slots per (b, head)
+  int64_t nblocks;    // blocks per (b, head)
+  const int32_t* row_ptr;
+  const int32_t* col_idx;
+  int per_head;
+  int64_t nlists;     // block lists in the CSR: B*Hh if per_head else 1
+  float scale;        // softmax scale applied to q.k
+  float scale_log2;   // scale * log2(e)
+  __nv_bfloat16* o;
+  float* lse;
+  const uint32_t* tile_valid;  // [ntiles][4]
+  unsigned int* status;
+  uint64_t wait_limit_ns;
+};
+
+// Set bits [lo, lo+len) of a 128-bit mask; lo is a multiple of len, len | 128.
+__device__ __forceinline__ void set_bits(uint32_t (&m)[4], int lo, int len) {
+  if (len >= 32) {
+    for (int x = lo; x < lo + len; x += 32) m[x >> 5] = kFull;
+  } else {
+    m[lo >> 5] |= ((1u << len) - 1u) << (lo & 31);
+  }
+}
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+  __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&v);
+}
+
+template <int D, bool FINE>
+__global__ void __launch_bounds__(kThreads, 1)
+    attn_fwd_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmk,
+                    const __grid_constant__ CUtensorMap tmv, const AttnParams p) {
+  using Cfg = AttnCfg<D, FINE>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  uint8_t* sQ = smem + Cfg::kOffQ;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Cfg::kOffBar);
+  uint64_t* q_full = bars;
+  uint64_t* k_full = bars + 1;
+  uint64_t* v_full = k_full + Cfg::NS;
+  uint64_t* kv_empty = v_full + Cfg::NS;
+  uint64_t* s_full = kv_empty + Cfg::NS;  // [2]
+  uint64_t* p_ready = s_full + 2;
+  uint64_t* o_ready = p_ready + 1;
+  uint32_t* misc = reinterpret_cast<uint32_t*>(smem + Cfg::kOffMisc);  // tmem, abort, count, skip
+  uint16_t* tlist = reinterpret_cast<uint16_t*>(smem + Cfg::kOffList);
+  uint32_t* bitmap = reinterpret_cast<uint32_t*>(smem + Cfg::kOffBitmap);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int qt = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+  const int64_t bh_row = ((int64_t)b * p.Hh + h) * p.Npad;
+  const int64_t list = p.per_head ? (int64_t)b * p.Hh + h : 0;
+  const WaitCtx wc{p.status, reinterpret_cast<volatile int*>(&misc[1]), p.wait_limit_ns};
+
+  // ------------------------------------------------------------ set-up
+  if (threadIdx.x == 0) {
+    mbar_init(q_full, 1);
+    for (int i = 0; i < Cfg::NS; ++i) {
+      mbar_init(&k_full[i], 1);
+      mbar_init(&v_full[i], 1);
+      mbar_init(&kv_empty[i], 1);
+    }
+    mbar_init(&s_full[0], 1);
+    mbar_init(&s_full[1], 1);
+    mbar_init(p_ready, 128);
+    mbar_init(o_ready, 1);
+    misc[1] = 0;
+    misc[2] = 0;
+    fence_mbar_init();
+    prefetch_tmap(&tmq);
+    prefetch_tmap(&tmk);
+    prefetch_tmap(&tmv);
+  }
+  // a timeout recorded by an earlier CTA (or call) stops the rest of the grid
+  if (threadIdx.x == 0)
+    misc[3] = (*reinterpret_cast<volatile unsigned int*>(p.status) & kStatusTimeout) ? 1u : 0u;
+  __syncthreads();
+  if (misc[3]) return;
+  if (warp == 1) {
+    tmem_alloc(&misc[0], Cfg::kTmemCols);
+    tmem_relinquish();
+  }
+  if (FINE) {
+    for (int i = threadIdx.x; i < kFineMaxTiles / 32; i += kThreads) bitmap[i] = 0;
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tbase = misc[0];
+
+  // ------------------------------------------------ key tiles of this query tile
+  int64_t rs = 0;
+  int n = 0;
+  const int64_t nnz = p.row_ptr[p.nlists * p.nblocks];  // entries of col_idx
+  if (!FINE) {
+    const int64_t r = list * p.nblocks + qt;  // block == tile
+    rs = p.row_ptr[r];
+    const int64_t re = p.row_ptr[r + 1];
+    if (re < rs || rs < 0 || re > nnz) {
+      if (threadIdx.x == 0) atomicOr(p.status, kStatusBadBlocklist);
+    } else {
+      n = (int)(re - rs);
+    }
+  } else {
+    // union over the query blocks of this tile of the key tiles they touch
+    const int per = kTile / p.block;
+    const int64_t qb0 = (int64_t)qt * per;
+    const int64_t qb1 = min(qb0 + per, p.nblocks);
+    for (int64_t qb = qb0 + warp; qb < qb1; qb += kThreads / 32) {
+      const int64_t r = list * p.nblocks + qb;
+      const int64_t a = max(p.row_ptr[r], 0), e = min((int64_t)p.row_ptr[r + 1], nnz);
+      for (int64_t i = a + lane; i < e; i += 32) {
+        const int c = p.col_idx[i];
+        if (c >= 0 && c < p.nblocks) {
+          const int tile = (int)(((int64_t)c * p.block) >> 7);
+          atomicOr(&bitmap[tile >> 5], 1u << (tile & 31));
+        }
+      }
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      int cnt = 0;
+      for (int w = 0; w < kFineMaxTiles / 32; ++w) {
+        uint32_t bits = bitmap[w];
+        while (bits) {
+          const int bpos = __ffs(bits) - 1;
+          bits &= bits - 1;
+          tlist[cnt++] = (uint16_t)(w * 32 + bpos);
+        }
+      }
+      misc[2] = cnt;
+    }
+    __syncthreads();
+    n = (int)misc[2];
+  }
+
+  auto tile_of = [&](int j, bool& ok) -> int {
+    if (FINE) {
+      ok = true;
+      return tlist[j];
+    }
+    const int c = __ldg(p.col_idx + rs + j);
+    ok = (c >= 0 && (int64_t)c < p.nblocks);
+    return ok ? c : 0;
+  };
+
+  if (warp == 0) {
+    // ---------------------------------------------------------- TMA producer
+    if (lane == 0 && n > 0) {
+      mbar_arrive_expect_tx(q_full, Cfg::kQBytes);
+      for (int c = 0; c < Cfg::kChunks; ++c)
+        tma_load_2d(sQ + c * Cfg::kPanel, &tmq, q_full, c * 64, (int)(bh_row + (int64_t)qt * kTile));
+      int issued = 0;
+      for (int j = 0; j < n; ++j) {
+        const int st = j % Cfg::NS;
+        const uint32_t ph = (j / Cfg::NS) & 1;
+        if (!bounded_wait(&kv_empty[st], ph ^ 1, wc)) break;
+        bool ok;
+        const int kt = tile_of(j, ok);
+        if (!ok) atomicOr(p.status, kStatusBadBlocklist);
+        const int krow = (int)(bh_row + (int64_t)kt * kTile);
+        uint8_t* sK = smem + Cfg::kOffK + st * Cfg::kKVBytes;
+        uint8_t* sV = smem + Cfg::kOffV + st * Cfg::kKVBytes;
+        mbar_arrive_expect_tx(&k_full[st], Cfg::kKVBytes);
+        for (int c = 0; c < Cfg::kChunks; ++c)
+          tma_load_2d(sK + c * Cfg::kPanel, &tmk, &k_full[st], c * 64, krow);
+        mbar_arrive_expect_tx(&v_full[st], Cfg::kKVBytes);
+        for (int c = 0; c < Cfg::kChunks; ++c)
+          tma_load_2d(sV + c * Cfg::kPanel, &tmv, &v_full[st], c * 64, krow);
+        issued = j + 1;
+      }
+      if (*wc.abort) {
+        // leave no copy in flight: wait (bounded, ignoring the abort flag)
+        // for the loads still owned by the ring
+        volatile int no_abort = 0;
+        const WaitCtx drain{p.status, &no_abort, p.wait_limit_ns};
+        bounded_wait(q_full, 0, drain);
+        for (int j = max(0, issued - Cfg::NS); j < issued; ++j) {
+          bounded_wait(&k_full[j % Cfg::NS], (j / Cfg::NS) & 1, drain);
+          bounded_wait(&v_full[j % Cfg::NS], (j / Cfg::NS) & 1, drain);
+        }
+      }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // ---------------------------------------------------------- MMA issuer
+    if (lane == 0 && n > 0) {
+      constexpr uint32_t idesc_qk = idesc_bf16(128, 128, 0);
+      constexpr uint32_t idesc_pv = idesc_bf16(128, D, 1);
+      const uint32_t tO = tbase + 256;
+      const uint32_t qaddr = smem_u32(sQ);
+      auto issue_qk = [&](int st, uint32_t tdst) {
+        const uint32_t kaddr = smem_u32(smem + Cfg::kOffK + st * Cfg::kKVBytes);
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * Cfg::kPanel + (kk & 3) * 32;
+          mma_ss(tdst, sdesc_sw128(qaddr + off, 16, 1024), sdesc_sw128(kaddr + off, 16, 1024),
+                 idesc_qk, kk > 0);
+        }
+      };
+      auto issue_pv = [&](int st, uint32_t tP, uint32_t acc) {
+        const uint32_t vaddr = smem_u32(smem + Cfg::kOffV + st * Cfg::kKVBytes);
+#pragma unroll
+        for (int kk = 0; kk < kTile / 16; ++kk)
+          mma_ts(tO, tP + kk * 8, sdesc_sw128(vaddr + kk * 2048, Cfg::kPanel, 1024), idesc_pv,
+                 (acc | (uint32_t)kk) != 0);
+      };
+      bool alive = bounded_wait(q_full, 0, wc) && bounded_wait(&k_full[0], 0, wc);
+      if (alive) {
+        tc_fence_after();
+        issue_qk(0, tbase);
+        mma_commit(&s_full[0]);
+      }
+      for (int j = 0; alive && j < n; ++j) {
+        if (j + 1 < n) {
+          const int st1 = (j + 1) % Cfg::NS;
+          if (!bounded_wait(&k_full[st1], ((j + 1) / Cfg::NS) & 1, wc)) break;
+          tc_fence_after();
+          issue_qk(st1, tbase + ((j + 1) & 1) * 128);
+          mma_commit(&s_full[(j + 1) & 1]);
+        }
+        const int st = j % Cfg::NS;
+        if (!bounded_wait(p_ready, j & 1, wc)) break;
+        if (!bounded_wait(&v_full[st], (j / Cfg::NS) & 1, wc)) break;
+        tc_fence_after();
+        issue_pv(st, tbase + (j & 1) * 128 + 64, j > 0);
+        mma_commit(o_ready);
+        mma_commit(&kv_empty[st]);
+      }
+    }
+    __syncwarp();
+  } else if (warp >= 4) {
+    // ---------------------------------------------------------- softmax
+    const int q4 = warp & 3;
+    const int row = q4 * 32 + lane;
+    const uint32_t lane_off = (uint32_t)(q4 * 32) << 16;
+    const uint32_t tO = tbase + 256 + lane_off;
+    const float sl2 = p.scale_log2;
+    const float thr = 8.0f / sl2;  // rescale O when the max grows by more than 2^8
+    float m_run = -INFINITY, l_run = 0.f;
+    int64_t fptr = 0, fend = 0;
+    if (FINE) {
+      const int64_t qb = (int64_t)qt * (kTile / p.block) + row / p.block;
+      if (qb < p.nblocks) {
+        const int64_t r = list * p.nblocks + qb;
+        fptr = p.row_ptr[r];
+        fend = p.row_ptr[r + 1];
+        if (fend < fptr || fptr < 0 || fend > nnz) {
+          atomicOr(p.status, kStatusBadBlocklist);
+          fend = fptr;
+        }
+      }
+    }
+    bool alive = true;
+    for (int j = 0; j < n; ++j) {
+      bool ok;
+      const int kt = tile_of(j, ok);
+      uint32_t vm[4];
+      {
+        const uint4 tv = __ldg(reinterpret_cast<const uint4*>(p.tile_valid) + kt);
+        vm[0] = ok ? tv.x : 0u;
+        vm[1] = ok ? tv.y : 0u;
+        vm[2] = ok ? tv.z : 0u;
+        vm[3] = ok ? tv.w : 0u;
+      }
+      if (FINE) {
+        uint32_t am[4] = {0u, 0u, 0u, 0u};
+        while (fptr < fend) {
+          const int c = __ldg(p.col_idx + fptr);
+          if (c < 0 || c >= p.nblocks) {
+            atomicOr(p.status, kStatusBadBlocklist);
+            ++fptr;
+            continue;
+          }
+          const int64_t s0 = (int64_t)c * p.block;
+          const int ct = (int)(s0 >> 7);
+          if (ct > kt) break;
+          if (ct < kt) {  // row not ascending
+            atomicOr(p.status, kStatusBadBlocklist);
+            ++fptr;
+            continue;
+          }
+          set_bits(am, (int)(s0 & 127), p.block);
+          ++fptr;
+        }
+#pragma unroll
+        for (int w = 0; w < 4; ++w) vm[w] &= am[w];
+      }
+      if (!__all_sync(kFull, bounded_wait(&s_full[j & 1], (j >> 1) & 1, wc))) {
+        alive = false;
+        break;
+      }
+      tc_fence_after();
+      const uint32_t tS = tbase + (j & 1) * 128 + lane_off;
+      float s[128];
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        uint32_t r32[32];
+        tmem_ld32(tS + c * 32, r32);
+#pragma unroll
+        for (int i = 0; i < 32; ++i) s[c * 32 + i] = __uint_as_float(r32[i]);
+      }
+      if ((vm[0] & vm[1] & vm[2] & vm[3]) != kFull) {
+#pragma unroll
+        for (int w = 0; w < 4; ++w)
+#pragma unroll
+          for (int i = 0; i < 32; ++i)
+            if (!((vm[w] >> i) & 1u)) s[w * 32 + i] = -INFINITY;
+      }
+      float mx = s[0];
+#pragma unroll
+      for (int i = 1; i < 128; ++i) mx = fmaxf(mx, s[i]);
+      const float m_new = fmaxf(m_run, mx);
+      const bool need = m_new > m_run + thr;
+      float corr = 1.f;
+      if (need) {
+        corr = ex2_approx((m_run - m_new) * sl2);
+        m_run = m_new;
+        l_run *= corr;
+      }
+      const float ms = (m_run == -INFINITY) ? 0.f : m_run * sl2;
+      uint32_t pk[64];
+      float lsum = 0.f;
+#pragma unroll
+      for (int i = 0; i < 64; ++i) {
+        const float p0 = ex2_approx(fmaf(s[2 * i], sl2, -ms));
+        const float p1 = ex2_approx(fmaf(s[2 * i + 1], sl2, -ms));
+        lsum += p0 + p1;
+        pk[i] = pack_bf16x2(p0, p1);
+      }
+      l_run += lsum;
+      if (j > 0) {
+        // PV(j-1) must be in O before O is rescaled or PV(j) is issued
+        if (!__all_sync(kFull, bounded_wait(o_ready, (j - 1) & 1, wc))) {
+          alive = false;
+          break;
+        }
+        tc_fence_after();
+        if (__any_sync(kFull, need)) {
+#pragma unroll
+          for (int c = 0; c < D / 32; ++c) {
+            uint32_t o32[32];
+            tmem_ld32(tO + c * 32, o32);
+#pragma unroll
+            for (int i = 0; i < 32; ++i) o32[i] = __float_as_uint(__uint_as_float(o32[i]) * corr);
+            tmem_st32(tO + c * 32, o32);
+          }
+        }
+      }
+      const uint32_t tP = tS + 64;
+      tmem_st32(tP, *reinterpret_cast<uint32_t(*)[32]>(&pk[0]));
+      tmem_st32(tP + 32, *reinterpret_cast<uint32_t(*)[32]>(&pk[32]));
+      tc_fence_before();
+      mbar_arrive(p_ready);
+    }
+    // ---------------------------------------------------------- epilogue
+    if (alive && n > 0) {
+      alive = __all_sync(kFull, bounded_wait(o_ready, (n - 1) & 1, wc));
+      tc_fence_after();
+    }
+    const uint4 tq = __ldg(reinterpret_cast<const uint4*>(p.tile_valid) + qt);
+    const uint32_t qw = (row < 32) ? tq.x : (row < 64) ? tq.y : (row < 96) ? tq.z : tq.w;
+    const bool qvalid = (qw >> (row & 31)) & 1u;
+    const bool has = alive && n > 0 && qvalid && l_run > 0.f;
+    const float inv_l = has ? 1.f / l_run : 0.f;
+    const int64_t orow = bh_row + (int64_t)qt * kTile + row;
+    uint4* dst = reinterpret_cast<uint4*>(p.o + orow * D);
+#pragma unroll
+    for (int c = 0; c < D / 32; ++c) {
+      uint32_t o32[32];
+      if (alive && n > 0) {
+        tmem_ld32(tO + c * 32, o32);
+      } else {
+#pragma unroll
+        for (int i = 0; i < 32; ++i) o32[i] = 0u;
+      }
+      uint32_t w16[16];
+#pragma unroll
+      for (int i = 0; i < 16; ++i)
+        w16[i] = pack_bf16x2(__uint_as_float(o32[2 * i]) * inv_l,
+                             __uint_as_float(o32[2 * i + 1]) * inv_l);
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+        dst[c * 4 + i] = make_uint4(w16[4 * i], w16[4 * i + 1], w16[4 * i + 2], w16[4 * i + 3]);
+    }
+    if (p.lse) p.lse[orow] = has ? m_run * p.scale + logf(l_run) : -INFINITY;
+    tc_fence_before();
+  }
+
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tbase, Cfg::kTmemCols);
+  }
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (!fn) {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+  }
+  return fn;
+}
+
+// [rows, D] bf16 row-major, 64 x 128 boxes, 128-byte swizzle.
+bool make_tmap(CUtensorMap* m, const void* ptr, int64_t rows, int D) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {(cuuint64_t)D, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)D * 2};
+  cuuint32_t box[2] = {64, (cuuint32_t)kTile};
+  cuuint32_t estr[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides, box,
+            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int D, bool FINE>
+cudaError_t launch_t(const CUtensorMap& q, const CUtensorMap& k, const CUtensorMap& v,
+                     const AttnParams& p, dim3 grid, cudaStream_t st) {
+  using Cfg = AttnCfg<D, FINE>;
+  auto kern = attn_fwd_kernel<D, FINE>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::kSmem);
+  if (e != cudaSuccess) return e;
+  kern<<<grid, kThreads, Cfg::kSmem, st>>>(q, k, v, p);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+bsa_status launch_attn_fwd(const bsa_plan_s& plan, const void* q, const void* k, const void* v,
+                           const int32_t* row_ptr, const int32_t* col_idx, int per_head,
+                           float scale, void* o, float* lse, cudaStream_t st) {
+  const Geometry& g = plan.g;
+  const int64_t rows = (int64_t)g.B * g.Hh * g.Npad;
+  if (rows >= (1ll << 31)) return set_error(BSA_ERR_UNSUPPORTED, "B*Hh*Npad must be < 2^31");
+  const bool fine = g.block < kTile;
+  if (fine && g.ntiles > kFineMaxTiles)
+    return set_error(BSA_ERR_UNSUPPORTED, "blocks smaller than 128 slots need Npad <= 262144");
+  CUtensorMap tq, tk, tv;
+  if (!make_tmap(&tq, q, rows, g.D) || !make_tmap(&tk, k, rows, g.D) || !make_tmap(&tv, v, rows, g.D))
+    return set_error(BSA_ERR_CUDA, "cuTensorMapEncodeTiled failed");
+  AttnParams p;
+  p.Hh = g.Hh;
+  p.block = g.block;
+  p.Npad = g.Npad;
+  p.nblocks = g.nblocks;
+  p.row_ptr = row_ptr;
+  p.col_idx = col_idx;
+  p.per_head = per_head ? 1 : 0;
+  p.nlists = per_head ? (int64_t)g.B * g.Hh : 1;
+  p.scale = scale;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  p.o = reinterpret_cast<__nv_bfloat16*>(o);
+  p.lse = lse;
+  p.tile_valid = plan.d_tile_valid;
+  p.status = plan.d_status;
+  p.wait_limit_ns = plan.wait_limit_ns;
+  const dim3 grid((unsigned)g.ntiles, (unsigned)g.Hh, (unsigned)g.B);
+  cudaError_t e;
+  if (g.D == 128)
+    e = fine ? launch_t<128, true>(tq, tk, tv, p, grid, st) : launch_t<128, false>(tq, tk, tv, p, grid, st);
+  else
+    e = fine ? launch_t<64, true>(tq, tk, tv, p, grid, st) : launch_t<64, false>(tq, tk, tv, p, grid, st);
+  if (e != cudaSuccess) return cuda_error(e, "attention launch");
+  return BSA_OK;
+}
+
+}  // namespace bsa

@@ -1,0 +1,97 @@
+// Internal declarations shared by the library's translation units: the plan,
+// status bits, integer helpers and launch entry points of each kernel file.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include <string>
+
+#include "../../include/bsattn.h"
+
+namespace bsa {
+
+// Bits of the plan's device status word (set with atomicOr by kernels).
+enum : unsigned int {
+  kStatusBadBlocklist = 1u << 0,
+  kStatusTimeout = 1u << 1,
+};
+
+// Division of a 32-bit unsigned n < 2^31 by an invariant divisor d >= 1 with
+// one multiply-high, add and shift (Granlund & Montgomery, "Division by
+// Invariant Integers using Multiplication", PLDI 1994, section 4):
+// with l = ceil(log2 d) and m = floor(2^32 (2^l - d) / d) + 1,
+// q = (mulhi(m, n) + n) >> l.  The add cannot overflow because n < 2^31.
+struct FastDiv {
+  uint32_t d = 1, m = 0, l = 0;
+  FastDiv() = default;
+  explicit FastDiv(uint32_t div) : d(div) {
+    l = 0;
+    while ((1ull << l) < div) ++l;
+    m = (uint32_t)((((1ull << l) - div) << 32) / div + 1);
+  }
+  __host__ __device__ __forceinline__ uint32_t div(uint32_t n) const {
+#ifdef __CUDA_ARCH__
+    return (__umulhi(m, n) + n) >> l;
+#else
+    return (uint32_t)((((uint64_t)m * n) >> 32) + n) >> l;
+#endif
+  }
+  __host__ __device__ __forceinline__ void divmod(uint32_t n, uint32_t& q, uint32_t& r) const {
+    q = div(n);
+    r = n - q * d;
+  }
+};
+
+// Geometry of the token <-> slot maps, passed by value to kernels.
+struct Geometry {
+  int B, Hh, D, T, H, W;
+  int layout;           // bsa_layout
+  int ph, pw, block;
+  int nbf;              // frame layout: blocks per frame
+  int TH, TW;           // tile layout: tiles per column / row
+  int P;                // tokens per frame (H*W)
+  int64_t nblocks;      // blocks per (b, head)
+  int64_t Npad;         // slots per (b, head), multiple of 128
+  int64_t ntiles;       // Npad / 128
+};
+
+}  // namespace bsa
+
+struct bsa_plan_s {
+  bsa::Geometry g;
+  int device = 0;
+  uint32_t* d_tile_valid = nullptr;  // [ntiles][4] bit per slot: slot holds a token
+  unsigned int* d_status = nullptr;  // device status word
+  uint64_t wait_limit_ns = 2000000000ull;
+};
+
+namespace bsa {
+
+// Records a message for bsa_last_error() and returns `st`.
+bsa_status set_error(bsa_status st, const std::string& msg);
+bsa_status cuda_error(cudaError_t e, const char* what);
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Kernel launchers (each in its own translation unit).
+cudaError_t launch_lvsa_mask(const Geometry& g, int C, int T_per, int s, int32_t* frame_sets,
+                             int32_t* row_ptr, int32_t* col_idx, unsigned int* status,
+                             cudaStream_t st);
+cudaError_t launch_reorder_fwd(const Geometry& g, const void* const x[3], void* const y[3],
+                               int nt, cudaStream_t st);
+cudaError_t launch_reorder_inv(const Geometry& g, const void* x_slots, void* x_nat,
+                               cudaStream_t st);
+cudaError_t launch_draft_mask(const Geometry& g, const uint32_t* tile_valid, const void* q,
+                              const void* k, int keep, int32_t* row_ptr, int32_t* kv_idx,
+                              float* draft_map, double* ws, cudaStream_t st);
+bsa_status launch_attn_fwd(const bsa_plan_s& plan, const void* q, const void* k, const void* v,
+                           const int32_t* row_ptr, const int32_t* col_idx, int per_head,
+                           float scale, void* o, float* lse, cudaStream_t st);
+cudaError_t launch_selftest_timeout(unsigned int* status, uint64_t limit_ns, cudaStream_t st);
+
+// Size bookkeeping shared by the API and the draft kernels.
+size_t draft_workspace_bytes(const Geometry& g);
+int draft_rows_per_cta(int64_t nblocks);
+
+}  // namespace bsa

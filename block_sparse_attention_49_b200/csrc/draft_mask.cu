@@ -1,0 +1,223 @@
+// Draft mask (Draft Attention article: tokens reshaped to [t,h,w]; Q and K
+// average-pooled over pool_h x pool_w tiles into a low-resolution draft
+// attention map; the map yields a sparse mask that keeps only the important
+// block connections, at a stated sparsity; pool_h*pool_w equals the block
+// size of the block-sparse attention that follows).
+//
+// Two kernels, both on the tile-layout slot tensors (each block = one tile):
+//  pool:  qbar/kbar[b,h,blk,:] = mean of the block's non-empty slots, fp64.
+//         The sum runs sequentially over the block's slots in order (the
+//         tile's row-major order) and is divided once by the token count.
+//         16-byte loads; HBM bound.
+//  score_topk: for a group of query-block rows of one (b, head), the fp64
+//         logits L[i][j] = sum_c qbar_i[c]*kbar_j[c] (sequential over c, the
+//         product and the sum each rounded, no fused multiply-add), then per
+//         row the k largest, ties to the lower j, by k rounds of a warp-wide
+//         arg-max; written ascending.  Optionally the draft map
+//         softmax_j(L[i][j]/sqrt(D)) as fp32.
+// With this fixed evaluation order the selection is reproducible bit for bit
+// by any implementation that follows the same order.
+#include <cuda_bf16.h>
+
+#include <cfloat>
+
+#include "bsa_internal.cuh"
+
+namespace bsa {
+namespace {
+
+constexpr int kPoolThreads = 256;
+constexpr int kScoreThreads = 256;
+constexpr int kKeyChunk = 32;  // key blocks staged in shared memory per step
+
+// One group of D/8 threads per (which, b, h, block); each thread owns 8
+// channels.  which = 0: Q, 1: K.
+template <int D>
+__global__ void __launch_bounds__(kPoolThreads)
+    draft_pool_kernel(const uint4* __restrict__ q, const uint4* __restrict__ k,
+                      const uint32_t* __restrict__ tile_valid, int Hh, int64_t Npad,
+                      int64_t nblocks, int block, int64_t groups_per_tensor,
+                      double* __restrict__ ws) {
+  constexpr int kTPG = D / 8;  // threads per group
+  const int64_t gid = ((int64_t)blockIdx.x * kPoolThreads + threadIdx.x) / kTPG;
+  const int sub = threadIdx.x % kTPG;
+  if (gid >= 2 * groups_per_tensor) return;
+  const int which = gid >= groups_per_tensor;
+  const int64_t g = gid - which * groups_per_tensor;  // (b*Hh + h)*nblocks + blk
+  const int64_t bh = g / nblocks, blk = g - bh * nblocks;
+  const uint4* src = (which ? k : q) + ((bh * Npad + blk * block) * (D / 8)) + sub;
+  const int64_t s0 = blk * block;
+  double acc[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) acc[i] = 0.0;
+  int cnt = 0;
+  for (int e = 0; e < block; ++e) {
+    const int64_t s = s0 + e;
+    const uint32_t w = __ldg(tile_valid + (s >> 5));
+    if (!((w >> (s & 31)) & 1u)) continue;
+    const uint4 v = __ldg(src + (int64_t)e * (D / 8));
+    const __nv_bfloat162* pv = reinterpret_cast<const __nv_bfloat162*>(&v);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const float2 f = __bfloat1622float2(pv[i]);
+      acc[2 * i] = __dadd_rn(acc[2 * i], (double)f.x);
+      acc[2 * i + 1] = __dadd_rn(acc[2 * i + 1], (double)f.y);
+    }
+    ++cnt;
+  }
+  double* dst = ws + ((int64_t)which * groups_per_tensor + g) * D + sub * 8;
+  const double dc = (double)cnt;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) dst[i] = cnt ? __ddiv_rn(acc[i], dc) : 0.0;
+}
+
+// grid: (ceil(nblocks / R), Hh, B); R query rows per CTA.
+template <int D>
+__global__ void __launch_bounds__(kScoreThreads)
+    draft_score_topk_kernel(const double* __restrict__ qbar, const double* __restrict__ kbar,
+                            int Hh, int nblocks, int R, int keep, int32_t* __restrict__ row_ptr,
+                            int32_t* __restrict__ kv_idx, float* __restrict__ draft_map) {
+  extern __shared__ double shd[];
+  double* sq = shd;                         // [R][D]
+  double* sk = sq + R * D;                  // [kKeyChunk][D + 1]
+  double* sl = sk + kKeyChunk * (D + 1);    // [R][nblocks] logits
+  uint8_t* sel = reinterpret_cast<uint8_t*>(sl + (int64_t)R * nblocks);  // [R][nblocks]
+  const int h = blockIdx.y, b = blockIdx.z;
+  const int64_t bh = (int64_t)b * Hh + h;
+  const int r0 = blockIdx.x * R;
+  const int rows = min(R, nblocks - r0);
+  const double* qb = qbar + (bh * nblocks + r0) * D;
+  const double* kb = kbar + bh * nblocks * D;
+  for (int i = threadIdx.x; i < rows * D; i += kScoreThreads) sq[i] = qb[i];
+  for (int i = threadIdx.x; i < rows * nblocks; i += kScoreThreads) sel[i] = 0;
+
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  for (int j0 = 0; j0 < nblocks; j0 += kKeyChunk) {
+    const int nj = min(kKeyChunk, nblocks - j0);
+    __syncthreads();
+    for (int i = threadIdx.x; i < nj * D; i += kScoreThreads) {
+      const int jj = i / D, c = i - jj * D;
+      sk[jj * (D + 1) + c] = kb[(int64_t)(j0 + jj) * D + c];
+    }
+    __syncthreads();
+    // warp w handles rows w, w+8, ...; lane = key block within the chunk
+    if (lane < nj) {
+      for (int r = warp; r < rows; r += kScoreThreads / 32) {
+        const double* a = sq + r * D;
+        const double* kk = sk + lane * (D + 1);
+        double acc = 0.0;
+        for (int c = 0; c < D; ++c) acc = __dadd_rn(acc, __dmul_rn(a[c], kk[c]));
+        sl[(int64_t)r * nblocks + j0 + lane] = acc;
+      }
+    }
+  }
+  __syncthreads();
+
+  // top-k per row, one warp per row
+  for (int r = warp; r < rows; r += kScoreThreads / 32) {
+    const double* L = sl + (int64_t)r * nblocks;
+    uint8_t* sr = sel + (int64_t)r * nblocks;
+    for (int it = 0; it < keep; ++it) {
+      double best = -DBL_MAX;
+      int bidx = 0x7fffffff;
+      for (int j = lane; j < nblocks; j += 32) {
+        if (sr[j]) continue;
+        const double v = L[j];
+        if (bidx == 0x7fffffff || v > best || (v == best && j < bidx)) {
+          best = v;
+          bidx = j;
+        }
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+        const double ov = __shfl_xor_sync(0xffffffffu, best, o);
+        const int oi = __shfl_xor_sync(0xffffffffu, bidx, o);
+        const bool take = (oi != 0x7fffffff) &&
+                          (bidx == 0x7fffffff || ov > best || (ov == best && oi < bidx));
+        if (take) {
+          best = ov;
+          bidx = oi;
+        }
+      }
+      if (lane == 0 && bidx != 0x7fffffff) sr[bidx] = 1;
+      __syncwarp();
+    }
+    // ascending output
+    const int64_t grow = bh * nblocks + r0 + r;
+    int32_t* out = kv_idx + grow * keep;
+    int pos = 0;
+    for (int j0 = 0; j0 < nblocks; j0 += 32) {
+      const int j = j0 + lane;
+      const bool on = j < nblocks && sr[j];
+      const uint32_t bal = __ballot_sync(0xffffffffu, on);
+      if (on) {
+        const int at = pos + __popc(bal & ((1u << lane) - 1u));
+        if (at < keep) out[at] = j;
+      }
+      pos += __popc(bal);
+    }
+    if (row_ptr && lane == 0) {
+      row_ptr[grow] = (int32_t)(grow * keep);
+      if (grow == (int64_t)gridDim.z * Hh * nblocks - 1) row_ptr[grow + 1] = (int32_t)((grow + 1) * keep);
+    }
+    if (draft_map) {
+      double mx = -DBL_MAX;
+      for (int j = lane; j < nblocks; j += 32) mx = fmax(mx, L[j]);
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) mx = fmax(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+      const double inv_sqrt_d = 1.0 / sqrt((double)D);
+      double sum = 0.0;
+      for (int j = lane; j < nblocks; j += 32) sum += exp((L[j] - mx) * inv_sqrt_d);
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+      float* dm = draft_map + grow * nblocks;
+      for (int j = lane; j < nblocks; j += 32) dm[j] = (float)(exp((L[j] - mx) * inv_sqrt_d) / sum);
+    }
+  }
+}
+
+template <int D>
+cudaError_t launch_t(const Geometry& g, const uint32_t* tile_valid, const void* q, const void* k,
+                     int keep, int32_t* row_ptr, int32_t* kv_idx, float* draft_map, double* ws,
+                     cudaStream_t st) {
+  const int64_t groups = (int64_t)g.B * g.Hh * g.nblocks;
+  const int64_t threads = 2 * groups * (D / 8);
+  const unsigned pool_grid = (unsigned)((threads + kPoolThreads - 1) / kPoolThreads);
+  draft_pool_kernel<D><<<pool_grid, kPoolThreads, 0, st>>>(
+      reinterpret_cast<const uint4*>(q), reinterpret_cast<const uint4*>(k), tile_valid, g.Hh,
+      g.Npad, g.nblocks, g.block, groups, ws);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  const int R = draft_rows_per_cta(g.nblocks);
+  const size_t smem = (size_t)(R * D + kKeyChunk * (D + 1) + (int64_t)R * g.nblocks) * sizeof(double) +
+                      (size_t)R * g.nblocks;
+  auto kern = draft_score_topk_kernel<D>;
+  e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  const dim3 grid((unsigned)((g.nblocks + R - 1) / R), (unsigned)g.Hh, (unsigned)g.B);
+  kern<<<grid, kScoreThreads, smem, st>>>(ws, ws + groups * D, g.Hh, (int)g.nblocks, R, keep,
+                                          row_ptr, kv_idx, draft_map);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+int draft_rows_per_cta(int64_t nblocks) {
+  // logits + selection flags of R rows within ~150 KB of shared memory
+  int64_t R = 16;
+  while (R > 1 && R * nblocks * 9 > 150 * 1024) R >>= 1;
+  return (int)R;
+}
+
+size_t draft_workspace_bytes(const Geometry& g) {
+  return (size_t)2 * g.B * g.Hh * g.nblocks * g.D * sizeof(double);
+}
+
+cudaError_t launch_draft_mask(const Geometry& g, const uint32_t* tile_valid, const void* q,
+                              const void* k, int keep, int32_t* row_ptr, int32_t* kv_idx,
+                              float* draft_map, double* ws, cudaStream_t st) {
+  if (g.D == 128) return launch_t<128>(g, tile_valid, q, k, keep, row_ptr, kv_idx, draft_map, ws, st);
+  return launch_t<64>(g, tile_valid, q, k, keep, row_ptr, kv_idx, draft_map, ws, st);
+}
+
+}  // namespace bsa

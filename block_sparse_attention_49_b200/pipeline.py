@@ -1,0 +1,94 @@
+"""Ready-made call sequences over the C ABI, with buffers from torch.
+
+LVSA attention ("LVSA: Training-Free Sparse Attention for Long Video
+Diffusion", section 2): lvsa_mask(s) -> reorder_fwd(Q,K,V) -> attn_fwd ->
+reorder_inv(O).  Draft attention (Draft Attention article): reorder_fwd(Q,K,V)
+-> draft_mask -> attn_fwd -> reorder_inv(O).
+
+torch only allocates device memory and supplies the stream; every step runs
+in libbsattn.so.
+"""
+from __future__ import annotations
+
+import math
+
+import torch
+
+from . import (LAYOUT_FRAME, LAYOUT_TILE, Plan, bsa_attn_fwd, bsa_draft_keep_count,
+               bsa_draft_mask, bsa_draft_workspace_bytes, bsa_lvsa_mask, bsa_lvsa_nnz,
+               bsa_reorder_fwd, bsa_reorder_inv)
+
+
+class _Base:
+    def _alloc_slots(self, device):
+        p = self.plan
+        shape = (p.B, p.Hh, p.Npad, p.D)
+        mk = lambda: torch.empty(shape, dtype=torch.bfloat16, device=device)
+        self.q_s, self.k_s, self.v_s, self.o_s = mk(), mk(), mk(), mk()
+        self.lse = torch.empty((p.B, p.Hh, p.Npad), dtype=torch.float32, device=device)
+
+    def attend(self, per_head: bool):
+        bsa_attn_fwd(self.plan, self.q_s, self.k_s, self.v_s, self.row_ptr, self.col_idx,
+                     per_head, self.scale, self.o_s, self.lse)
+
+    def gather(self, q, k, v):
+        bsa_reorder_fwd(self.plan, q, self.q_s, k, self.k_s, v, self.v_s)
+
+    def scatter(self, out):
+        bsa_reorder_inv(self.plan, self.o_s, out)
+        return out
+
+
+class LvsaAttention(_Base):
+    """LVSA block-sparse attention on the frame layout."""
+
+    def __init__(self, B, Hh, D, T, H, W, C, T_per, block=128, device="cuda", scale=None):
+        self.plan = Plan(B, Hh, D, T, H, W, LAYOUT_FRAME, block=block)
+        self.C, self.T_per = C, T_per
+        self.scale = scale if scale is not None else 1.0 / math.sqrt(D)
+        nnz = bsa_lvsa_nnz(self.plan, C)
+        self.frame_sets = torch.empty(T * C, dtype=torch.int32, device=device)
+        self.row_ptr = torch.empty(self.plan.nblocks + 1, dtype=torch.int32, device=device)
+        self.col_idx = torch.empty(nnz, dtype=torch.int32, device=device)
+        self._alloc_slots(device)
+
+    def mask(self, s: int):
+        bsa_lvsa_mask(self.plan, self.C, self.T_per, s, self.frame_sets, self.row_ptr,
+                      self.col_idx)
+
+    def __call__(self, q, k, v, s: int, out=None):
+        out = torch.empty_like(q) if out is None else out
+        self.mask(s)
+        self.gather(q, k, v)
+        self.attend(per_head=False)
+        return self.scatter(out)
+
+
+class DraftAttention(_Base):
+    """Draft-mask block-sparse attention on the tile layout."""
+
+    def __init__(self, B, Hh, D, T, H, W, pool_h, pool_w, sparsity_pct, device="cuda",
+                 scale=None, want_map=False):
+        self.plan = Plan(B, Hh, D, T, H, W, LAYOUT_TILE, pool_h, pool_w, pool_h * pool_w)
+        self.sparsity = sparsity_pct
+        self.scale = scale if scale is not None else 1.0 / math.sqrt(D)
+        self.keep = bsa_draft_keep_count(self.plan, sparsity_pct)
+        rows = B * Hh * self.plan.nblocks
+        self.row_ptr = torch.empty(rows + 1, dtype=torch.int32, device=device)
+        self.col_idx = torch.empty(rows * self.keep, dtype=torch.int32, device=device)
+        self.draft_map = (torch.empty(rows * self.plan.nblocks, dtype=torch.float32,
+                                      device=device) if want_map else None)
+        nbytes = bsa_draft_workspace_bytes(self.plan)
+        self.workspace = torch.empty((nbytes + 7) // 8, dtype=torch.float64, device=device)
+        self._alloc_slots(device)
+
+    def mask(self):
+        bsa_draft_mask(self.plan, self.q_s, self.k_s, self.sparsity, self.row_ptr, self.col_idx,
+                       self.draft_map, self.workspace)
+
+    def __call__(self, q, k, v, out=None):
+        out = torch.empty_like(q) if out is None else out
+        self.gather(q, k, v)
+        self.mask()
+        self.attend(per_head=True)
+        return self.scatter(out)

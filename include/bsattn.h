@@ -1,0 +1,182 @@
+/*
+ * bsattn.h - C ABI of libbsattn.so: block-sparse softmax attention over video
+ * tokens laid out as a [t,h,w] latent grid, for NVIDIA B200 (sm_100a).
+ *
+ * The operations follow two methods described on the web:
+ *  - "LVSA: Training-Free Sparse Attention for Long Video Diffusion",
+ *    section 2 "Methodology", "Core mechanism": each query frame t attends
+ *    the frame set A(t) = G_s U W(t) (rotating global anchors G_s plus an
+ *    extended local window W(t)), with |A(t)| = C; "Complexity": the cost is
+ *    T*C*P^2*d, linear in the number of frames T.
+ *  - The Draft Attention article ("科学家提出视频扩散模型加速方法，在H100实现
+ *    一倍以上端到端加速", 163.com): tokens are reshaped to [t,h,w]; Q and K are
+ *    average-pooled over pool_h x pool_w tiles into a low-resolution draft
+ *    attention map, which yields a sparse block mask (pool_h*pool_w equals
+ *    the block size) guiding full-resolution block-sparse attention; a reorder
+ *    makes the selected blocks contiguous in memory.
+ *
+ * Conventions common to every entry point
+ *  - Tensors are owned by the caller: device pointers, contiguous, 16-byte
+ *    aligned.  Nothing is allocated per call; a plan owns only small index
+ *    data and a device status word, allocated by bsa_plan_create on the
+ *    device that is current at that time.
+ *  - Every call is asynchronous on `stream` (a cudaStream_t; NULL = legacy
+ *    default stream) and returns after enqueueing its kernel(s).  Argument
+ *    errors are detected on the host before anything is enqueued and
+ *    reported as a status code; bsa_last_error() then describes the error.
+ *  - Errors found on the device (a block list naming a block out of range,
+ *    a bounded wait that ran out) are recorded in the plan's status word and
+ *    reported by bsa_poll_status().  Kernels never trap.
+ *  - Natural layout: [B, N, Hh, D] bf16, token n = (t*H + y)*W + x.
+ *    Slot layout: [B, Hh, Npad, D] bf16 (Npad = bsa_padded_tokens()); the
+ *    token -> slot map is set by the plan's layout (below).  Slots that hold
+ *    no token are "empty"; attention never reads them as keys.
+ *  - Supported head dims: D = 64 or 128.  Block size: a divisor of 128.
+ */
+#ifndef BSATTN_H_
+#define BSATTN_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  BSA_OK = 0,
+  BSA_ERR_INVALID_ARG = 1,    /* bad sizes, null pointer, inconsistent plan      */
+  BSA_ERR_UNSUPPORTED = 2,    /* valid but not implemented (e.g. D = 96)         */
+  BSA_ERR_ALIGNMENT = 3,      /* a pointer is not 16-byte aligned                */
+  BSA_ERR_CUDA = 4,           /* a CUDA runtime/driver call failed               */
+  BSA_ERR_TIMEOUT = 5,        /* a bounded device wait ran out (see poll)        */
+  BSA_ERR_BAD_BLOCKLIST = 6   /* a block list named a block out of range, or a
+                                 row_ptr decreased, or (block < 128) a row was
+                                 not ascending; offending entries were skipped   */
+} bsa_status;
+
+/* Token -> slot maps (Draft Attention article, the reorder paragraph and its
+ * figure "Full Map" vs "Reordered Full Map").
+ *  BSA_LAYOUT_FRAME: each frame padded to nbf = ceil(H*W/block) whole blocks;
+ *      token (t,y,x) -> slot t*nbf*block + y*W + x.  Used by the LVSA mask.
+ *  BSA_LAYOUT_TILE:  each pool_h x pool_w tile of a frame is one block
+ *      (block = pool_h*pool_w); with TH = ceil(H/pool_h), TW = ceil(W/pool_w),
+ *      token (t, i*pool_h+a, j*pool_w+b) -> slot
+ *      ((t*TH + i)*TW + j)*block + a*pool_w + b.  Used by the draft mask.
+ * In both, Npad is the block count times block, rounded up to a multiple of
+ * 128 (the attention tile); slots past the last block are empty. */
+typedef enum { BSA_LAYOUT_FRAME = 0, BSA_LAYOUT_TILE = 1 } bsa_layout;
+
+typedef struct bsa_plan_s* bsa_plan_t;
+
+/* Create a plan for batch B, Hh heads, head dim D, latent grid T x H x W.
+ * layout FRAME: `block` tokens per block (pool_h, pool_w ignored).
+ * layout TILE:  block must equal pool_h*pool_w.
+ * Allocates the plan's device data (per-128-slot validity masks, status
+ * word) on the current device.  On error *plan is set to NULL. */
+bsa_status bsa_plan_create(bsa_plan_t* plan, int B, int Hh, int D, int T, int H, int W,
+                           int layout, int pool_h, int pool_w, int block);
+
+/* Free the plan and its device data.  No call using it may be in flight. */
+bsa_status bsa_plan_destroy(bsa_plan_t plan);
+
+/* Geometry queries (return -1 for a NULL plan). */
+int64_t bsa_padded_tokens(bsa_plan_t plan);   /* Npad                          */
+int64_t bsa_num_blocks(bsa_plan_t plan);      /* blocks per (b, head): Nb      */
+int     bsa_block_size(bsa_plan_t plan);
+
+/* LVSA frame mask for denoising step s ("LVSA", section 2, "Rotating global
+ * anchors" and "Extended adaptive window").
+ *   G_s = {f in [0,T) : (f - s) mod T_per == 0};
+ *   A(t) = G_s U {t} grown by t+1, t-1, t+2, t-2, ... (frames outside [0,T)
+ *   or already present are skipped) until |A(t)| = C.
+ * Requires a FRAME plan, 1 <= T_per, C <= T and |G_s U {t}| <= C for every t.
+ * Outputs (device):
+ *   frame_sets int32[T*C] (may be NULL): row t = A(t) ascending;
+ *   row_ptr    int32[Nb+1]: row r = query block r, r*C*nbf entries before it;
+ *   col_idx    int32[Nb*C*nbf]: for query block r in frame t = r / nbf, every
+ *              block f*nbf + i of every frame f in A(t), ascending.
+ * The block list is the same for every batch and head (per_head_lists = 0). */
+bsa_status bsa_lvsa_mask(bsa_plan_t plan, int C, int T_per, int s, int32_t* frame_sets,
+                         int32_t* row_ptr, int32_t* col_idx, void* stream);
+
+/* Number of col_idx entries bsa_lvsa_mask writes (Nb*C*nbf), or -1. */
+int64_t bsa_lvsa_nnz(bsa_plan_t plan, int C);
+
+/* Blocks kept per query-block row at `sparsity_pct` percent sparsity:
+ * k = ceil(Nb*(100 - sparsity_pct)/100), i.e. never sparser than asked. */
+int bsa_draft_keep_count(bsa_plan_t plan, int sparsity_pct);
+
+/* Scratch bytes bsa_draft_mask needs (the pooled Q and K in fp64). */
+size_t bsa_draft_workspace_bytes(bsa_plan_t plan);
+
+/* Draft mask (Draft Attention article: average pooling of Q and K over each
+ * pool_h x pool_w tile, low-resolution map softmax(Qbar Kbar^T / sqrt(D)),
+ * sparse mask keeping the important blocks at the stated sparsity).
+ * Requires a TILE plan.  q_slots, k_slots: slot layout (output of
+ * bsa_reorder_fwd).  For every (b, head, query block i):
+ *   qbar_i, kbar_j = mean over the tile's tokens inside the grid (fp64,
+ *     sequential sum in row-major tile order, one IEEE division);
+ *   L[i][j] = sum_c qbar_i[c]*kbar_j[c], sequential over c, each product and
+ *     sum rounded to fp64 (no fused multiply-add);
+ *   keep the k = bsa_draft_keep_count() blocks j with the largest L[i][j],
+ *     ties to the lower j, written ascending.
+ * Outputs (device): kv_idx int32[B*Hh*Nb*k]; row_ptr int32[B*Hh*Nb+1] (may be
+ * NULL; row r starts at r*k); draft_map float[B*Hh*Nb*Nb] (may be NULL) =
+ * softmax_j(L[i][j]/sqrt(D)).  Use with bsa_attn_fwd(per_head_lists = 1).
+ * workspace: device scratch of at least bsa_draft_workspace_bytes(); its
+ * contents on entry do not matter. */
+bsa_status bsa_draft_mask(bsa_plan_t plan, const void* q_slots, const void* k_slots,
+                          int sparsity_pct, int32_t* row_ptr, int32_t* kv_idx,
+                          float* draft_map, void* workspace, size_t workspace_bytes,
+                          void* stream);
+
+/* Reorder (Draft Attention article, reorder paragraph): gather natural-layout
+ * tensors into the plan's slot layout; empty slots are written as zero.
+ * Up to three tensors in one launch: x1/y1 and x2/y2 may be NULL. */
+bsa_status bsa_reorder_fwd(bsa_plan_t plan, const void* x0, void* y0, const void* x1,
+                           void* y1, const void* x2, void* y2, void* stream);
+
+/* Inverse reorder: slot layout -> natural layout; empty slots are dropped. */
+bsa_status bsa_reorder_inv(bsa_plan_t plan, const void* x_slots, void* x_nat, void* stream);
+
+/* Block-sparse attention forward (LVSA section 2 and the Draft Attention
+ * article: softmax attention restricted to the allowed blocks).
+ * q, k, v, o: slot layout [B, Hh, Npad, D] bf16.  lse: float[B*Hh*Npad] or
+ * NULL.  Block list: one CSR with rows r = list*Nb + qb, list = b*Hh + h if
+ * per_head_lists else 0; row r lists the key blocks (index < Nb) that query
+ * block qb may attend, without repeats (ascending when block < 128).
+ * For every non-empty query slot q:
+ *   O[q] = sum_k softmax_k(scale * <q, k>) v_k over the non-empty slots k of
+ *   the allowed blocks; LSE[q] = log sum_k exp(scale * <q, k>).
+ * fp32 accumulation; probabilities rounded to bf16 before the PV product.
+ * Empty query slots, and queries with no allowed key, get O = 0 and
+ * LSE = -inf.  Block lists are not modified. */
+bsa_status bsa_attn_fwd(bsa_plan_t plan, const void* q, const void* k, const void* v,
+                        const int32_t* row_ptr, const int32_t* col_idx, int per_head_lists,
+                        float scale, void* o, float* lse, void* stream);
+
+/* Synchronize `stream`, read and clear the plan's device status word.
+ * Returns BSA_OK, BSA_ERR_BAD_BLOCKLIST, BSA_ERR_TIMEOUT or BSA_ERR_CUDA. */
+bsa_status bsa_poll_status(bsa_plan_t plan, void* stream);
+
+/* Set the limit, in nanoseconds, of every bounded wait inside the plan's
+ * kernels (default 2e9).  A wait that runs out records BSA_ERR_TIMEOUT. */
+bsa_status bsa_set_wait_limit_ns(bsa_plan_t plan, uint64_t ns);
+
+/* Failure-detection self test: launches one CTA that waits on a barrier no
+ * one arrives on, for at most `limit_ns`; the wait runs out, the kernel
+ * records BSA_ERR_TIMEOUT in the plan's status word and returns normally. */
+bsa_status bsa_selftest_timeout(bsa_plan_t plan, uint64_t limit_ns, void* stream);
+
+/* Message describing the last error of the calling thread ("" if none). */
+const char* bsa_last_error(void);
+
+/* Library version string. */
+const char* bsa_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* BSATTN_H_ */
