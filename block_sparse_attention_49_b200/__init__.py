@@ -21,7 +21,8 @@ __all__ = [
     "BsaError", "Plan", "LAYOUT_FRAME", "LAYOUT_TILE", "lib_path", "load",
     "bsa_plan_create", "bsa_plan_destroy", "bsa_padded_tokens", "bsa_num_blocks",
     "bsa_block_size", "bsa_lvsa_mask", "bsa_lvsa_nnz", "bsa_draft_keep_count",
-    "bsa_draft_workspace_bytes", "bsa_draft_mask", "bsa_reorder_fwd", "bsa_reorder_inv",
+    "bsa_draft_workspace_bytes", "bsa_draft_mask", "bsa_draft_mask_noalloc",
+    "bsa_draft_noalloc_max_scratch_bytes", "bsa_reorder_fwd", "bsa_reorder_inv",
     "bsa_attn_fwd", "bsa_poll_status", "bsa_set_wait_limit_ns", "bsa_selftest_timeout",
     "bsa_last_error", "bsa_version", "EXPORTED_SYMBOLS",
 ]
@@ -51,6 +52,8 @@ _SIGS = {
     "bsa_draft_keep_count": (_c_int, [_c_p, _c_int]),
     "bsa_draft_workspace_bytes": (_c_sz, [_c_p]),
     "bsa_draft_mask": (_c_int, [_c_p, _c_p, _c_p, _c_int, _c_p, _c_p, _c_p, _c_p, _c_sz, _c_p]),
+    "bsa_draft_mask_noalloc": (_c_int, [_c_p, _c_p, _c_p, _c_int, _c_p, _c_p, _c_p, _c_p]),
+    "bsa_draft_noalloc_max_scratch_bytes": (_c_sz, []),
     "bsa_reorder_fwd": (_c_int, [_c_p] * 8),
     "bsa_reorder_inv": (_c_int, [_c_p, _c_p, _c_p, _c_p]),
     "bsa_attn_fwd": (_c_int, [_c_p, _c_p, _c_p, _c_p, _c_p, _c_p, _c_int, ctypes.c_float, _c_p,
@@ -183,6 +186,18 @@ def bsa_draft_mask(plan: Plan, q_slots, k_slots, sparsity_pct: int, row_ptr, kv_
     _check(load().bsa_draft_mask(plan.handle, _ptr(q_slots), _ptr(k_slots), sparsity_pct,
                                  _ptr(row_ptr), _ptr(kv_idx), _ptr(draft_map), _ptr(workspace),
                                  nbytes, _stream(stream)), "bsa_draft_mask")
+
+
+def bsa_draft_mask_noalloc(plan: Plan, q_slots, k_slots, sparsity_pct: int, row_ptr, kv_idx,
+                           draft_map, stream=None):
+    """bsa_draft_mask without a caller workspace (scratch inside the library)."""
+    _check(load().bsa_draft_mask_noalloc(plan.handle, _ptr(q_slots), _ptr(k_slots), sparsity_pct,
+                                         _ptr(row_ptr), _ptr(kv_idx), _ptr(draft_map),
+                                         _stream(stream)), "bsa_draft_mask_noalloc")
+
+
+def bsa_draft_noalloc_max_scratch_bytes() -> int:
+    return int(load().bsa_draft_noalloc_max_scratch_bytes())
 
 
 def bsa_reorder_fwd(plan: Plan, x0, y0, x1=None, y1=None, x2=None, y2=None, stream=None):

@@ -221,3 +221,90 @@ cudaError_t launch_draft_mask(const Geometry& g, const uint32_t* tile_valid, con
 }
 
 }  // namespace bsa
+
+// ---------------------------------------------------------------------------
+// Draft mask without any allocation by the caller.
+//
+// Some callers cannot allocate device memory of their own: for example a
+// plugin running inside a host program that owns every device allocation and
+// hands the plugin only its input and output buffers, or a caller held to a
+// fixed memory budget, where an extra allocation may fail or stall the device
+// in the middle of a step.  bsa_draft_mask_noalloc serves them: it computes
+// exactly what bsa_draft_mask computes, with its fp64 scratch (the pooled Q
+// and K) taken from the file-scope device array below instead of a caller
+// workspace.
+//
+// The array is kNoAllocScratchBytes (32 MiB) on every GPU that loads this
+// library, held until the process exits; problems whose scratch would exceed
+// it (2*B*Hh*Nb*D*8 bytes) are rejected.  Every call on a device shares the
+// one array, so calls whose kernels overlap on the GPU (on different streams,
+// or from different host threads) race on it; calls in order on one stream
+// are safe.  The array keeps the last call's contents: nothing needs clearing,
+// because the pooling kernel writes every element the scoring kernel reads.
+// ---------------------------------------------------------------------------
+#include <mutex>
+
+namespace bsa {
+namespace {
+
+constexpr size_t kNoAllocScratchBytes = 32u << 20;
+constexpr int kMaxDevices = 64;
+
+static __device__ __align__(256) double g_noalloc_scratch[kNoAllocScratchBytes / sizeof(double)];
+
+// Device address of g_noalloc_scratch on the current device.  Looked up once
+// per device, on the first call made with that device current.
+cudaError_t noalloc_scratch_address(double** out) {
+  static std::mutex mu;
+  static double* addr[kMaxDevices] = {};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lock(mu);
+  if (!addr[dev]) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if (e != cudaSuccess) return e;
+    addr[dev] = reinterpret_cast<double*>(p);
+  }
+  *out = addr[dev];
+  return cudaSuccess;
+}
+
+}  // namespace
+}  // namespace bsa
+
+extern "C" size_t bsa_draft_noalloc_max_scratch_bytes(void) { return bsa::kNoAllocScratchBytes; }
+
+extern "C" bsa_status bsa_draft_mask_noalloc(bsa_plan_t plan, const void* q_slots,
+                                             const void* k_slots, int sparsity_pct,
+                                             int32_t* row_ptr, int32_t* kv_idx, float* draft_map,
+                                             void* stream) {
+  using namespace bsa;
+  if (!plan) return set_error(BSA_ERR_INVALID_ARG, "plan is NULL");
+  const Geometry& g = plan->g;
+  if (g.layout != BSA_LAYOUT_TILE) return set_error(BSA_ERR_INVALID_ARG, "draft mask needs a TILE plan");
+  if (sparsity_pct < 0 || sparsity_pct >= 100)
+    return set_error(BSA_ERR_INVALID_ARG, "sparsity must be in [0, 100)");
+  if (!q_slots || !k_slots || !kv_idx)
+    return set_error(BSA_ERR_INVALID_ARG, "q_slots / k_slots / kv_idx is NULL");
+  if (!aligned16(q_slots) || !aligned16(k_slots))
+    return set_error(BSA_ERR_ALIGNMENT, "q_slots / k_slots not 16-byte aligned");
+  const size_t need = draft_workspace_bytes(g);
+  if (need > kNoAllocScratchBytes)
+    return set_error(BSA_ERR_UNSUPPORTED,
+                     "draft scratch of " + std::to_string(need) +
+                         " bytes exceeds the 32 MiB static scratch of bsa_draft_mask_noalloc; "
+                         "use bsa_draft_mask with a caller workspace");
+  if (g.nblocks > 18000) return set_error(BSA_ERR_UNSUPPORTED, "draft mask supports up to 18000 blocks");
+  const int keep = (int)((g.nblocks * (100 - sparsity_pct) + 99) / 100);
+  if ((int64_t)g.B * g.Hh * g.nblocks * keep >= (1ll << 31))
+    return set_error(BSA_ERR_UNSUPPORTED, "block list longer than 2^31 entries");
+  double* scratch = nullptr;
+  cudaError_t e = noalloc_scratch_address(&scratch);
+  if (e != cudaSuccess) return cuda_error(e, "cudaGetSymbolAddress(scratch)");
+  e = launch_draft_mask(g, plan->d_tile_valid, q_slots, k_slots, keep, row_ptr, kv_idx, draft_map,
+                        scratch, reinterpret_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? BSA_OK : cuda_error(e, "draft_mask_noalloc launch");
+}

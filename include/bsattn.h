@@ -131,6 +131,28 @@ bsa_status bsa_draft_mask(bsa_plan_t plan, const void* q_slots, const void* k_sl
                           float* draft_map, void* workspace, size_t workspace_bytes,
                           void* stream);
 
+/* bsa_draft_mask for callers that cannot allocate device memory (the paper
+ * has no counterpart; this is a convenience of this library).  Examples: a
+ * plugin inside a host program that owns every device allocation and passes
+ * only input and output buffers, or a caller held to a fixed memory budget
+ * where an extra allocation could fail or stall the device mid-step.
+ * Same arguments, outputs and results as bsa_draft_mask, minus the workspace:
+ * the fp64 scratch lives in a 32 MiB array inside the library
+ * (bsa_draft_noalloc_max_scratch_bytes()), held by every GPU that loads the
+ * library until the process exits.  Problems needing more scratch than that
+ * (2*B*Hh*Nb*D*8 bytes) return BSA_ERR_UNSUPPORTED.  The first call made on a
+ * device looks up that array's device address (one cudaGetSymbolAddress);
+ * make that first call before any stream capture.  All calls on a device
+ * share the array: calls whose kernels overlap on the GPU race on it, calls
+ * in order on one stream do not.  Nothing in it needs clearing between calls.
+ * The current device must be the plan's device. */
+bsa_status bsa_draft_mask_noalloc(bsa_plan_t plan, const void* q_slots, const void* k_slots,
+                                  int sparsity_pct, int32_t* row_ptr, int32_t* kv_idx,
+                                  float* draft_map, void* stream);
+
+/* Scratch capacity of bsa_draft_mask_noalloc, in bytes (32 MiB). */
+size_t bsa_draft_noalloc_max_scratch_bytes(void);
+
 /* Reorder (Draft Attention article, reorder paragraph): gather natural-layout
  * tensors into the plan's slot layout; empty slots are written as zero.
  * Up to three tensors in one launch: x1/y1 and x2/y2 may be NULL. */
