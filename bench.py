@@ -176,7 +176,7 @@ def run_reference(args, rank, world):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--steps", type=int, default=30)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--config", type=int, default=3)
@@ -184,6 +184,8 @@ def main():
     ap.add_argument("--cpu-budget-s", type=float, default=12.0)
     ap.add_argument("--ref-step-s", type=float, default=4.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--frames", type=int, default=0,
+                    help="use only the first T frames (small profiling case of the same kernels)")
     args = ap.parse_args()
 
     rank = int(os.environ.get("RANK", 0))
@@ -207,6 +209,11 @@ def main():
                                 device_id=torch.device("cuda", local))
 
     w = CONFIGS[args.config]
+    if args.frames:
+        from synth import small_workload
+        Tc, Hc, Wc = w.field_grid
+        w = small_workload(w, T=args.frames, field_grid=(args.frames, Hc, Wc),
+                           name=f"{w.name} (first {args.frames} frames)")
     flops_step = attended_flops(w)
     q, k, v = make_qkv(w, device="cuda")
     att = LvsaAttention(w.B, w.Hh, w.D, w.T, w.H, w.W, w.lvsa_C, w.lvsa_T_per, block=128)
@@ -214,21 +221,23 @@ def main():
     stream = torch.cuda.current_stream()
     launches_per_step = 4  # lvsa_mask, reorder_fwd, bsattn, reorder_inv
 
+    names = ("lvsa_mask", "reorder_fwd", "bsattn_fwd", "reorder_inv")
     ev = []
 
     def step(i, record):
         s = i % w.lvsa_T_per
-        att.mask(s)
-        att.gather(q, k, v)
-        if record:
-            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            e0.record(stream)
-            att.attend(per_head=False)
-            e1.record(stream)
-            ev.append((e0, e1))
-        else:
-            att.attend(per_head=False)
-        att.scatter(out)
+        calls = (lambda: att.mask(s), lambda: att.gather(q, k, v),
+                 lambda: att.attend(per_head=False), lambda: att.scatter(out))
+        if not record:
+            for c in calls:
+                c()
+            return
+        marks = [torch.cuda.Event(enable_timing=True) for _ in range(len(calls) + 1)]
+        marks[0].record(stream)
+        for j, c in enumerate(calls):
+            c()
+            marks[j + 1].record(stream)
+        ev.append(marks)
 
     for i in range(args.warmup):
         step(i, False)
@@ -248,7 +257,9 @@ def main():
     clk = clocks.stop()
     bsa.bsa_poll_status(att.plan)
     ms = t0.elapsed_time(t1) / args.steps
-    attn_ms = statistics.mean(a.elapsed_time(b) for a, b in ev)
+    kern_ms = {n: statistics.mean(m[j].elapsed_time(m[j + 1]) for m in ev)
+               for j, n in enumerate(names)}
+    attn_ms = kern_ms["bsattn_fwd"]
     if dist:
         tt = torch.tensor([ms, attn_ms], device="cuda")
         dist.all_reduce(tt, op=dist.ReduceOp.MAX)
@@ -283,6 +294,20 @@ def main():
         e2e_ms = float(tt[0])
     bsa.bsa_poll_status(att.plan)
 
+    # algorithmic bytes of the HBM-bound kernels (valid tokens read + written)
+    tok_bytes = w.B * w.N * w.Hh * w.D * 2
+    nnz = att.col_idx.numel()
+    algo_bytes = {"reorder_fwd": 3 * 2 * tok_bytes, "reorder_inv": 2 * tok_bytes,
+                  "lvsa_mask": 4 * (nnz + att.row_ptr.numel() + att.frame_sets.numel())}
+    kernels = {}
+    for n in names:
+        d = {"ms": kern_ms[n]}
+        if n in algo_bytes:
+            gbs = algo_bytes[n] / (kern_ms[n] * 1e-3) / 1e9
+            d.update({"algo_bytes": algo_bytes[n], "GB_s": gbs,
+                      "frac_hbm": gbs / peaks()[0]["hbm_gbs"]})
+        kernels[n] = d
+
     pk, pk_kind = peaks()
     peak = pk.get("bf16_tflops_sustained", pk["bf16_tflops"])
     attn_tflops = flops_step / (attn_ms * 1e-3) / 1e12
@@ -312,6 +337,7 @@ def main():
         "roofline": {"bound": "tensor", "achieved": attn_tflops, "peak": peak,
                      "unit": "TFLOP/s", "frac": attn_tflops / peak, "traffic": None,
                      "peak_kind": f"{pk_kind} bf16 sustained (kernel timed inside a long step)"},
+        "kernels": kernels,
         "gpu_launches": launches_per_step * args.steps,
         "clocks": clk,
         "e2e": {"value": world * flops_step / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",

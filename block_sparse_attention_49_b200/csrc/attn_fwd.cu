@@ -7,18 +7,23 @@
 // the non-empty key slots of the key blocks its query block may attend,
 // weighted sum of their values; plus the log-sum-exp.
 //
-// How (one CTA per 128-slot query tile; 8 warps):
-//   warp 0     TMA producer: Q tile once, then K and V tiles of every listed
-//              key tile into an NS-deep shared-memory ring (128-byte swizzle).
-//   warp 1     MMA issuer (one thread): S = Q K^T into tensor memory (two S
-//              buffers so the next S overlaps the softmax of the current
-//              one), then O += P V with P read from tensor memory.
-//   warps 4-7  softmax, one query row per thread (= one TMEM lane): reads S,
-//              masks empty / disallowed keys, keeps the running max and sum,
-//              writes P as bf16 over the upper half of its S buffer, rescales
-//              O only when the running max grew by more than 2^8 (the stale
-//              max stays exact because numerator and denominator share it),
-//              and finally normalises O and stores it.
+// How (one CTA per 128-slot query tile; 12 warps):
+//   warp 0      TMA producer: the Q tile once, then K and V of every listed
+//               key tile into an NS-deep shared-memory ring (128-byte swizzle).
+//   warp 1      MMA issuer (one thread): S = Q K^T into tensor memory, then
+//               O += P V with P read from tensor memory.
+//   warps 4-7   softmax group A: key tiles 0, 2, 4, ... of the list;
+//   warps 8-11  softmax group B: key tiles 1, 3, 5, ...
+// Each group owns one S buffer and one O accumulator in tensor memory
+// (S_A | S_B | O_A | O_B = 512 columns) and keeps its own running max and
+// sum, so the two groups never wait for each other inside the loop: while one
+// group's softmax runs, the tensor cores work on the other group's tiles.
+// Each thread owns one query row (one TMEM lane): it reads its S row, masks
+// empty or disallowed keys, writes P as bf16 over the upper half of its S
+// buffer, and rescales its O only when its running max grew by more than 2^8
+// (numerator and denominator share the stale max, so the result is exact).
+// At the end the two partial results are merged with their maxima and sums,
+// as in a split-key combine, normalised and stored.
 // Every wait is bounded; a wait that runs out records a timeout in the
 // plan's status word and the CTA leaves without trapping.
 #include <cuda_bf16.h>
@@ -33,7 +38,7 @@ namespace bsa {
 namespace {
 
 constexpr int kTile = 128;          // query / key tile (slots)
-constexpr int kThreads = 256;
+constexpr int kThreads = 384;
 constexpr int kFineMaxTiles = 2048; // key tiles addressable by the sub-tile-block path
 constexpr uint32_t kFull = 0xffffffffu;
 
@@ -48,14 +53,15 @@ struct AttnCfg {
   static constexpr int kOffK = kQBytes;
   static constexpr int kOffV = kOffK + NS * kKVBytes;
   static constexpr int kOffBar = kOffV + NS * kKVBytes;
-  static constexpr int kNumBars = 1 + 3 * NS + 2 + 2;
+  static constexpr int kNumBars = 1 + 3 * NS + 2 + 2 + 1;
   static constexpr int kOffMisc = kOffBar + kNumBars * 8;
   static constexpr int kOffList = kOffMisc + 16;
   static constexpr int kOffBitmap = kOffList + (FINE ? kFineMaxTiles * 2 : 0);
   static constexpr int kBytes = kOffBitmap + (FINE ? kFineMaxTiles / 8 : 0);
   static constexpr int kSmem = kBytes + 1024;  // room to align the base to 1024
-  static constexpr uint32_t kTmemCols = 512;   // S0 | S1 | O
+  static constexpr uint32_t kTmemCols = 512;   // S_A | S_B | O_A | O_B
   static_assert(kSmem <= 232448, "shared memory budget");
+  static_assert(4 * kTile * 4 <= kKVBytes, "epilogue statistics fit in a K stage");
 };
 
 struct AttnParams {
@@ -90,6 +96,15 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return *reinterpret_cast<uint32_t*>(&v);
 }
 
+__device__ __forceinline__ void softmax_groups_sync() {
+  asm volatile("bar.sync 1, 256;" ::: "memory");  // warps 4-11
+}
+
+// Final CTA barrier, reached by every warp from its own role branch.
+__device__ __forceinline__ void cta_end_sync() {
+  asm volatile("bar.sync 2, 384;" ::: "memory");
+}
+
 template <int D, bool FINE>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmk,
@@ -104,9 +119,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* k_full = bars + 1;
   uint64_t* v_full = k_full + Cfg::NS;
   uint64_t* kv_empty = v_full + Cfg::NS;
-  uint64_t* s_full = kv_empty + Cfg::NS;  // [2]
-  uint64_t* p_ready = s_full + 2;
-  uint64_t* o_ready = p_ready + 1;
+  uint64_t* s_full = kv_empty + Cfg::NS;  // [2]: S_A, S_B written
+  uint64_t* p_ready = s_full + 2;         // [2]: P_A, P_B written (128 arrivals each)
+  uint64_t* o_final = p_ready + 2;        // every MMA done
   uint32_t* misc = reinterpret_cast<uint32_t*>(smem + Cfg::kOffMisc);  // tmem, abort, count, skip
   uint16_t* tlist = reinterpret_cast<uint16_t*>(smem + Cfg::kOffList);
   uint32_t* bitmap = reinterpret_cast<uint32_t*>(smem + Cfg::kOffBitmap);
@@ -127,18 +142,18 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     mbar_init(&s_full[0], 1);
     mbar_init(&s_full[1], 1);
-    mbar_init(p_ready, 128);
-    mbar_init(o_ready, 1);
+    mbar_init(&p_ready[0], 128);
+    mbar_init(&p_ready[1], 128);
+    mbar_init(o_final, 1);
     misc[1] = 0;
     misc[2] = 0;
+    // a timeout recorded by an earlier CTA (or call) stops the rest of the grid
+    misc[3] = (*reinterpret_cast<volatile unsigned int*>(p.status) & kStatusTimeout) ? 1u : 0u;
     fence_mbar_init();
     prefetch_tmap(&tmq);
     prefetch_tmap(&tmk);
     prefetch_tmap(&tmv);
   }
-  // a timeout recorded by an earlier CTA (or call) stops the rest of the grid
-  if (threadIdx.x == 0)
-    misc[3] = (*reinterpret_cast<volatile unsigned int*>(p.status) & kStatusTimeout) ? 1u : 0u;
   __syncthreads();
   if (misc[3]) return;
   if (warp == 1) {
@@ -209,7 +224,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     return ok ? c : 0;
   };
 
-  if (warp == 0) {
+  if (warp < 4) {
+    // producer, MMA issuer and two idle warps: few registers
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 56;");
+    if (warp == 0) {
     // ---------------------------------------------------------- TMA producer
     if (lane == 0 && n > 0) {
       mbar_arrive_expect_tx(q_full, Cfg::kQBytes);
@@ -247,12 +265,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
     __syncwarp();
-  } else if (warp == 1) {
+    } else if (warp == 1) {
     // ---------------------------------------------------------- MMA issuer
     if (lane == 0 && n > 0) {
       constexpr uint32_t idesc_qk = idesc_bf16(128, 128, 0);
       constexpr uint32_t idesc_pv = idesc_bf16(128, D, 1);
-      const uint32_t tO = tbase + 256;
       const uint32_t qaddr = smem_u32(sQ);
       auto issue_qk = [&](int st, uint32_t tdst) {
         const uint32_t kaddr = smem_u32(smem + Cfg::kOffK + st * Cfg::kKVBytes);
@@ -263,7 +280,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                  idesc_qk, kk > 0);
         }
       };
-      auto issue_pv = [&](int st, uint32_t tP, uint32_t acc) {
+      auto issue_pv = [&](int st, uint32_t tP, uint32_t tO, uint32_t acc) {
         const uint32_t vaddr = smem_u32(smem + Cfg::kOffV + st * Cfg::kKVBytes);
 #pragma unroll
         for (int kk = 0; kk < kTile / 16; ++kk)
@@ -284,26 +301,37 @@ __global__ void __launch_bounds__(kThreads, 1)
           issue_qk(st1, tbase + ((j + 1) & 1) * 128);
           mma_commit(&s_full[(j + 1) & 1]);
         }
-        const int st = j % Cfg::NS;
-        if (!bounded_wait(p_ready, j & 1, wc)) break;
+        const int g = j & 1, st = j % Cfg::NS;
+        if (!bounded_wait(&p_ready[g], (j >> 1) & 1, wc)) break;
         if (!bounded_wait(&v_full[st], (j / Cfg::NS) & 1, wc)) break;
         tc_fence_after();
-        issue_pv(st, tbase + (j & 1) * 128 + 64, j > 0);
-        mma_commit(o_ready);
+        issue_pv(st, tbase + g * 128 + 64, tbase + 256 + g * 128, j >= 2);
         mma_commit(&kv_empty[st]);
       }
+      mma_commit(o_final);
     }
     __syncwarp();
-  } else if (warp >= 4) {
-    // ---------------------------------------------------------- softmax
+    }
+    cta_end_sync();
+    if (warp == 1) {
+      // every tensor-memory read of the softmax groups is done: free TMEM
+      tc_fence_after();
+      tmem_dealloc(tbase, Cfg::kTmemCols);
+    }
+  } else {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 224;");
+    // ---------------------------------------------------------- softmax groups
+    const int g = (warp >= 8) ? 1 : 0;
     const int q4 = warp & 3;
     const int row = q4 * 32 + lane;
     const uint32_t lane_off = (uint32_t)(q4 * 32) << 16;
-    const uint32_t tO = tbase + 256 + lane_off;
+    const uint32_t tS = tbase + g * 128 + lane_off;
+    const uint32_t tO = tbase + 256 + g * 128 + lane_off;
     const float sl2 = p.scale_log2;
     const float thr = 8.0f / sl2;  // rescale O when the max grows by more than 2^8
     float m_run = -INFINITY, l_run = 0.f;
     int64_t fptr = 0, fend = 0;
+    int fprev = -1;
     if (FINE) {
       const int64_t qb = (int64_t)qt * (kTile / p.block) + row / p.block;
       if (qb < p.nblocks) {
@@ -311,13 +339,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         fptr = p.row_ptr[r];
         fend = p.row_ptr[r + 1];
         if (fend < fptr || fptr < 0 || fend > nnz) {
-          atomicOr(p.status, kStatusBadBlocklist);
+          if (g == 0) atomicOr(p.status, kStatusBadBlocklist);
           fend = fptr;
         }
       }
     }
     bool alive = true;
-    for (int j = 0; j < n; ++j) {
+    for (int j = g; j < n; j += 2) {
       bool ok;
       const int kt = tile_of(j, ok);
       uint32_t vm[4];
@@ -329,10 +357,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         vm[3] = ok ? tv.w : 0u;
       }
       if (FINE) {
+        // this row's allowed blocks inside key tile kt (entries of tiles
+        // handled by the other group are passed over)
         uint32_t am[4] = {0u, 0u, 0u, 0u};
         while (fptr < fend) {
           const int c = __ldg(p.col_idx + fptr);
-          if (c < 0 || c >= p.nblocks) {
+          if (c < 0 || c >= p.nblocks || c <= fprev) {  // out of range or not ascending
             atomicOr(p.status, kStatusBadBlocklist);
             ++fptr;
             continue;
@@ -340,30 +370,24 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int64_t s0 = (int64_t)c * p.block;
           const int ct = (int)(s0 >> 7);
           if (ct > kt) break;
-          if (ct < kt) {  // row not ascending
-            atomicOr(p.status, kStatusBadBlocklist);
-            ++fptr;
-            continue;
-          }
-          set_bits(am, (int)(s0 & 127), p.block);
+          if (ct == kt) set_bits(am, (int)(s0 & 127), p.block);
+          fprev = c;
           ++fptr;
         }
 #pragma unroll
         for (int w = 0; w < 4; ++w) vm[w] &= am[w];
       }
-      if (!__all_sync(kFull, bounded_wait(&s_full[j & 1], (j >> 1) & 1, wc))) {
+      if (!__all_sync(kFull, bounded_wait(&s_full[g], (j >> 1) & 1, wc))) {
         alive = false;
         break;
       }
       tc_fence_after();
-      const uint32_t tS = tbase + (j & 1) * 128 + lane_off;
       float s[128];
+      {
+        uint32_t r128[128];
+        tmem_ld128(tS, r128);
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        uint32_t r32[32];
-        tmem_ld32(tS + c * 32, r32);
-#pragma unroll
-        for (int i = 0; i < 32; ++i) s[c * 32 + i] = __uint_as_float(r32[i]);
+        for (int i = 0; i < 128; ++i) s[i] = __uint_as_float(r128[i]);
       }
       if ((vm[0] & vm[1] & vm[2] & vm[3]) != kFull) {
 #pragma unroll
@@ -372,9 +396,18 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int i = 0; i < 32; ++i)
             if (!((vm[w] >> i) & 1u)) s[w * 32 + i] = -INFINITY;
       }
-      float mx = s[0];
+      // row max: 8 independent chains of 3-input max, then a small tree
+      float m8[8];
 #pragma unroll
-      for (int i = 1; i < 128; ++i) mx = fmaxf(mx, s[i]);
+      for (int c = 0; c < 8; ++c) m8[c] = fmax3f(s[c], s[c + 8], s[c + 16]);
+#pragma unroll
+      for (int i = 24; i < 120; i += 16)
+#pragma unroll
+        for (int c = 0; c < 8; ++c) m8[c] = fmax3f(m8[c], s[i + c], s[i + 8 + c]);
+#pragma unroll
+      for (int c = 0; c < 8; ++c) m8[c] = fmaxf(m8[c], s[120 + c]);
+      const float mx = fmax3f(fmax3f(m8[0], m8[1], m8[2]), fmax3f(m8[3], m8[4], m8[5]),
+                              fmaxf(m8[6], m8[7]));
       const float m_new = fmaxf(m_run, mx);
       const bool need = m_new > m_run + thr;
       float corr = 1.f;
@@ -385,77 +418,82 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       const float ms = (m_run == -INFINITY) ? 0.f : m_run * sl2;
       uint32_t pk[64];
-      float lsum = 0.f;
+      float l8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};  // independent partial sums
 #pragma unroll
       for (int i = 0; i < 64; ++i) {
         const float p0 = ex2_approx(fmaf(s[2 * i], sl2, -ms));
         const float p1 = ex2_approx(fmaf(s[2 * i + 1], sl2, -ms));
-        lsum += p0 + p1;
+        l8[i & 7] += p0 + p1;
         pk[i] = pack_bf16x2(p0, p1);
       }
-      l_run += lsum;
-      if (j > 0) {
-        // PV(j-1) must be in O before O is rescaled or PV(j) is issued
-        if (!__all_sync(kFull, bounded_wait(o_ready, (j - 1) & 1, wc))) {
-          alive = false;
-          break;
-        }
-        tc_fence_after();
-        if (__any_sync(kFull, need)) {
+      l_run += ((l8[0] + l8[1]) + (l8[2] + l8[3])) + ((l8[4] + l8[5]) + (l8[6] + l8[7]));
+      // O of this group holds every earlier PV of the group: S(j) was written
+      // after the group's previous PV in the tensor cores' issue order.
+      if (j >= 2 && __any_sync(kFull, need)) {
 #pragma unroll
-          for (int c = 0; c < D / 32; ++c) {
-            uint32_t o32[32];
-            tmem_ld32(tO + c * 32, o32);
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t o32[32];
+          tmem_ld32(tO + c * 32, o32);
 #pragma unroll
-            for (int i = 0; i < 32; ++i) o32[i] = __float_as_uint(__uint_as_float(o32[i]) * corr);
-            tmem_st32(tO + c * 32, o32);
-          }
+          for (int i = 0; i < 32; ++i) o32[i] = __float_as_uint(__uint_as_float(o32[i]) * corr);
+          tmem_st32(tO + c * 32, o32);
         }
       }
-      const uint32_t tP = tS + 64;
-      tmem_st32(tP, *reinterpret_cast<uint32_t(*)[32]>(&pk[0]));
-      tmem_st32(tP + 32, *reinterpret_cast<uint32_t(*)[32]>(&pk[32]));
+      tmem_st32(tS + 64, *reinterpret_cast<uint32_t(*)[32]>(&pk[0]));
+      tmem_st32(tS + 96, *reinterpret_cast<uint32_t(*)[32]>(&pk[32]));
       tc_fence_before();
-      mbar_arrive(p_ready);
+      mbar_arrive(&p_ready[g]);
     }
     // ---------------------------------------------------------- epilogue
     if (alive && n > 0) {
-      alive = __all_sync(kFull, bounded_wait(o_ready, (n - 1) & 1, wc));
+      alive = __all_sync(kFull, bounded_wait(o_final, 0, wc));
       tc_fence_after();
     }
+    // exchange (max, sum) of the two groups through a free K stage
+    float* stats = reinterpret_cast<float*>(smem + Cfg::kOffK);  // [4][128]: mA lA mB lB
+    stats[(2 * g) * kTile + row] = m_run;
+    stats[(2 * g + 1) * kTile + row] = l_run;
+    softmax_groups_sync();
+    const float mA = stats[row], lA = stats[kTile + row];
+    const float mB = stats[2 * kTile + row], lB = stats[3 * kTile + row];
+    const int nA = (n + 1) / 2, nB = n / 2;  // tiles each group processed
+    const float m = fmaxf(mA, mB);
+    const float a = (nA > 0 && mA != -INFINITY) ? ex2_approx((mA - m) * sl2) : 0.f;
+    const float bb = (nB > 0 && mB != -INFINITY) ? ex2_approx((mB - m) * sl2) : 0.f;
+    const float l = lA * a + lB * bb;
     const uint4 tq = __ldg(reinterpret_cast<const uint4*>(p.tile_valid) + qt);
     const uint32_t qw = (row < 32) ? tq.x : (row < 64) ? tq.y : (row < 96) ? tq.z : tq.w;
     const bool qvalid = (qw >> (row & 31)) & 1u;
-    const bool has = alive && n > 0 && qvalid && l_run > 0.f;
-    const float inv_l = has ? 1.f / l_run : 0.f;
+    const bool has = alive && n > 0 && qvalid && l > 0.f;
+    const float inv_l = has ? 1.f / l : 0.f;
+    const float wa = a * inv_l, wb = bb * inv_l;
     const int64_t orow = bh_row + (int64_t)qt * kTile + row;
-    uint4* dst = reinterpret_cast<uint4*>(p.o + orow * D);
+    // group g stores columns [g*D/2, (g+1)*D/2) of its rows
+    uint4* dst = reinterpret_cast<uint4*>(p.o + orow * D + g * (D / 2));
+    const uint32_t oA = tbase + 256 + lane_off + g * (D / 2);
+    const uint32_t oB = tbase + 384 + lane_off + g * (D / 2);
 #pragma unroll
-    for (int c = 0; c < D / 32; ++c) {
-      uint32_t o32[32];
-      if (alive && n > 0) {
-        tmem_ld32(tO + c * 32, o32);
-      } else {
+    for (int c = 0; c < D / 64; ++c) {
+      uint32_t xa[32], xb[32];
 #pragma unroll
-        for (int i = 0; i < 32; ++i) o32[i] = 0u;
-      }
+      for (int i = 0; i < 32; ++i) xa[i] = xb[i] = 0u;
+      if (alive && nA > 0) tmem_ld32(oA + c * 32, xa);
+      if (alive && nB > 0) tmem_ld32(oB + c * 32, xb);
       uint32_t w16[16];
 #pragma unroll
-      for (int i = 0; i < 16; ++i)
-        w16[i] = pack_bf16x2(__uint_as_float(o32[2 * i]) * inv_l,
-                             __uint_as_float(o32[2 * i + 1]) * inv_l);
+      for (int i = 0; i < 16; ++i) {
+        const float v0 = has ? __uint_as_float(xa[2 * i]) * wa + __uint_as_float(xb[2 * i]) * wb : 0.f;
+        const float v1 =
+            has ? __uint_as_float(xa[2 * i + 1]) * wa + __uint_as_float(xb[2 * i + 1]) * wb : 0.f;
+        w16[i] = pack_bf16x2(v0, v1);
+      }
 #pragma unroll
       for (int i = 0; i < 4; ++i)
         dst[c * 4 + i] = make_uint4(w16[4 * i], w16[4 * i + 1], w16[4 * i + 2], w16[4 * i + 3]);
     }
-    if (p.lse) p.lse[orow] = has ? m_run * p.scale + logf(l_run) : -INFINITY;
+    if (g == 0 && p.lse) p.lse[orow] = has ? m * p.scale + logf(l) : -INFINITY;
     tc_fence_before();
-  }
-
-  __syncthreads();
-  if (warp == 1) {
-    tc_fence_after();
-    tmem_dealloc(tbase, Cfg::kTmemCols);
+    cta_end_sync();
   }
 }
 

@@ -8,7 +8,7 @@
 
 #include <string>
 
-#include "../../include/bsattn.h"
+#include "bsattn.h"
 
 namespace bsa {
 
