@@ -23,7 +23,7 @@ __all__ = [
     "bsa_block_size", "bsa_lvsa_mask", "bsa_lvsa_nnz", "bsa_draft_keep_count",
     "bsa_draft_workspace_bytes", "bsa_draft_mask", "bsa_draft_mask_noalloc",
     "bsa_draft_noalloc_max_scratch_bytes", "bsa_reorder_fwd", "bsa_reorder_inv",
-    "bsa_attn_fwd", "bsa_poll_status", "bsa_set_wait_limit_ns", "bsa_selftest_timeout",
+    "bsa_attn_fwd", "bsa_lvsa_attn_fwd", "bsa_poll_status", "bsa_set_wait_limit_ns", "bsa_selftest_timeout",
     "bsa_last_error", "bsa_version", "EXPORTED_SYMBOLS",
 ]
 
@@ -58,6 +58,8 @@ _SIGS = {
     "bsa_reorder_inv": (_c_int, [_c_p, _c_p, _c_p, _c_p]),
     "bsa_attn_fwd": (_c_int, [_c_p, _c_p, _c_p, _c_p, _c_p, _c_p, _c_int, ctypes.c_float, _c_p,
                               _c_p, _c_p]),
+    "bsa_lvsa_attn_fwd": (_c_int, [_c_p, _c_int, _c_int, _c_int, _c_p, _c_p, _c_p, ctypes.c_float,
+                                   _c_p, _c_p, _c_p]),
     "bsa_poll_status": (_c_int, [_c_p, _c_p]),
     "bsa_set_wait_limit_ns": (_c_int, [_c_p, _c_u64]),
     "bsa_selftest_timeout": (_c_int, [_c_p, _c_u64, _c_p]),
@@ -215,6 +217,13 @@ def bsa_attn_fwd(plan: Plan, q, k, v, row_ptr, col_idx, per_head_lists: bool, sc
     _check(load().bsa_attn_fwd(plan.handle, _ptr(q), _ptr(k), _ptr(v), _ptr(row_ptr),
                                _ptr(col_idx), int(bool(per_head_lists)), float(scale), _ptr(o),
                                _ptr(lse), _stream(stream)), "bsa_attn_fwd")
+
+
+def bsa_lvsa_attn_fwd(plan: Plan, C: int, T_per: int, s: int, q, k, v, scale: float, o,
+                      lse=None, stream=None):
+    _check(load().bsa_lvsa_attn_fwd(plan.handle, C, T_per, s, _ptr(q), _ptr(k), _ptr(v),
+                                    float(scale), _ptr(o), _ptr(lse), _stream(stream)),
+           "bsa_lvsa_attn_fwd")
 
 
 def bsa_poll_status(plan: Plan, stream=None):

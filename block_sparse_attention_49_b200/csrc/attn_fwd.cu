@@ -227,29 +227,35 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp < 4) {
     // producer, MMA issuer and two idle warps: few registers
     asm volatile("setmaxnreg.dec.sync.aligned.u32 56;");
-    if (warp == 0) {
-    // ---------------------------------------------------------- TMA producer
-    if (lane == 0 && n > 0) {
-      mbar_arrive_expect_tx(q_full, Cfg::kQBytes);
-      for (int c = 0; c < Cfg::kChunks; ++c)
-        tma_load_2d(sQ + c * Cfg::kPanel, &tmq, q_full, c * 64, (int)(bh_row + (int64_t)qt * kTile));
+    if (warp == 0 && n > 0) {
+      // -------------------------------------------------------- TMA producer
+      // the whole warp runs the loop (warp-uniform operands); one lane issues
+      if (elect_one()) {
+        mbar_arrive_expect_tx(q_full, Cfg::kQBytes);
+        for (int c = 0; c < Cfg::kChunks; ++c)
+          tma_load_2d(sQ + c * Cfg::kPanel, &tmq, q_full, c * 64, (int)(bh_row + (int64_t)qt * kTile));
+      }
+      __syncwarp();
       int issued = 0;
       for (int j = 0; j < n; ++j) {
         const int st = j % Cfg::NS;
         const uint32_t ph = (j / Cfg::NS) & 1;
-        if (!bounded_wait(&kv_empty[st], ph ^ 1, wc)) break;
+        if (!__all_sync(kFull, bounded_wait(&kv_empty[st], ph ^ 1, wc))) break;
         bool ok;
         const int kt = tile_of(j, ok);
-        if (!ok) atomicOr(p.status, kStatusBadBlocklist);
         const int krow = (int)(bh_row + (int64_t)kt * kTile);
-        uint8_t* sK = smem + Cfg::kOffK + st * Cfg::kKVBytes;
-        uint8_t* sV = smem + Cfg::kOffV + st * Cfg::kKVBytes;
-        mbar_arrive_expect_tx(&k_full[st], Cfg::kKVBytes);
-        for (int c = 0; c < Cfg::kChunks; ++c)
-          tma_load_2d(sK + c * Cfg::kPanel, &tmk, &k_full[st], c * 64, krow);
-        mbar_arrive_expect_tx(&v_full[st], Cfg::kKVBytes);
-        for (int c = 0; c < Cfg::kChunks; ++c)
-          tma_load_2d(sV + c * Cfg::kPanel, &tmv, &v_full[st], c * 64, krow);
+        if (elect_one()) {
+          if (!ok) atomicOr(p.status, kStatusBadBlocklist);
+          uint8_t* sK = smem + Cfg::kOffK + st * Cfg::kKVBytes;
+          uint8_t* sV = smem + Cfg::kOffV + st * Cfg::kKVBytes;
+          mbar_arrive_expect_tx(&k_full[st], Cfg::kKVBytes);
+          for (int c = 0; c < Cfg::kChunks; ++c)
+            tma_load_2d(sK + c * Cfg::kPanel, &tmk, &k_full[st], c * 64, krow);
+          mbar_arrive_expect_tx(&v_full[st], Cfg::kKVBytes);
+          for (int c = 0; c < Cfg::kChunks; ++c)
+            tma_load_2d(sV + c * Cfg::kPanel, &tmv, &v_full[st], c * 64, krow);
+        }
+        __syncwarp();
         issued = j + 1;
       }
       if (*wc.abort) {
@@ -263,54 +269,64 @@ __global__ void __launch_bounds__(kThreads, 1)
           bounded_wait(&v_full[j % Cfg::NS], (j / Cfg::NS) & 1, drain);
         }
       }
-    }
-    __syncwarp();
-    } else if (warp == 1) {
-    // ---------------------------------------------------------- MMA issuer
-    if (lane == 0 && n > 0) {
+      __syncwarp();
+    } else if (warp == 1 && n > 0) {
+      // -------------------------------------------------------- MMA issuer
+      // the whole warp runs the loop (descriptors stay warp-uniform); the
+      // elected lane issues the tcgen05 instructions
       constexpr uint32_t idesc_qk = idesc_bf16(128, 128, 0);
       constexpr uint32_t idesc_pv = idesc_bf16(128, D, 1);
-      const uint32_t qaddr = smem_u32(sQ);
+      const uint64_t qd = sdesc_sw128(smem_u32(sQ), 16, 1024);
+      const uint64_t kd0 = sdesc_sw128(smem_u32(smem + Cfg::kOffK), 16, 1024);
+      const uint64_t vd0 = sdesc_sw128(smem_u32(smem + Cfg::kOffV), Cfg::kPanel, 1024);
       auto issue_qk = [&](int st, uint32_t tdst) {
-        const uint32_t kaddr = smem_u32(smem + Cfg::kOffK + st * Cfg::kKVBytes);
+        const uint64_t kd = sdesc_add(kd0, st * Cfg::kKVBytes);
+        if (elect_one()) {
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * Cfg::kPanel + (kk & 3) * 32;
-          mma_ss(tdst, sdesc_sw128(qaddr + off, 16, 1024), sdesc_sw128(kaddr + off, 16, 1024),
-                 idesc_qk, kk > 0);
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint32_t off = (kk >> 2) * Cfg::kPanel + (kk & 3) * 32;
+            mma_ss(tdst, sdesc_add(qd, off), sdesc_add(kd, off), idesc_qk, kk > 0);
+          }
         }
+        __syncwarp();
       };
       auto issue_pv = [&](int st, uint32_t tP, uint32_t tO, uint32_t acc) {
-        const uint32_t vaddr = smem_u32(smem + Cfg::kOffV + st * Cfg::kKVBytes);
+        const uint64_t vd = sdesc_add(vd0, st * Cfg::kKVBytes);
+        if (elect_one()) {
 #pragma unroll
-        for (int kk = 0; kk < kTile / 16; ++kk)
-          mma_ts(tO, tP + kk * 8, sdesc_sw128(vaddr + kk * 2048, Cfg::kPanel, 1024), idesc_pv,
-                 (acc | (uint32_t)kk) != 0);
+          for (int kk = 0; kk < kTile / 16; ++kk)
+            mma_ts(tO, tP + kk * 8, sdesc_add(vd, kk * 2048), idesc_pv, (acc | (uint32_t)kk) != 0);
+        }
+        __syncwarp();
       };
-      bool alive = bounded_wait(q_full, 0, wc) && bounded_wait(&k_full[0], 0, wc);
+      auto commit = [&](uint64_t* bar) {
+        if (elect_one()) mma_commit(bar);
+        __syncwarp();
+      };
+      auto wait = [&](uint64_t* bar, uint32_t parity) {
+        return __all_sync(kFull, bounded_wait(bar, parity, wc));
+      };
+      bool alive = wait(q_full, 0) && wait(&k_full[0], 0);
       if (alive) {
         tc_fence_after();
         issue_qk(0, tbase);
-        mma_commit(&s_full[0]);
+        commit(&s_full[0]);
       }
       for (int j = 0; alive && j < n; ++j) {
         if (j + 1 < n) {
           const int st1 = (j + 1) % Cfg::NS;
-          if (!bounded_wait(&k_full[st1], ((j + 1) / Cfg::NS) & 1, wc)) break;
+          if (!wait(&k_full[st1], ((j + 1) / Cfg::NS) & 1)) break;
           tc_fence_after();
           issue_qk(st1, tbase + ((j + 1) & 1) * 128);
-          mma_commit(&s_full[(j + 1) & 1]);
+          commit(&s_full[(j + 1) & 1]);
         }
         const int g = j & 1, st = j % Cfg::NS;
-        if (!bounded_wait(&p_ready[g], (j >> 1) & 1, wc)) break;
-        if (!bounded_wait(&v_full[st], (j / Cfg::NS) & 1, wc)) break;
+        if (!wait(&p_ready[g], (j >> 1) & 1) || !wait(&v_full[st], (j / Cfg::NS) & 1)) break;
         tc_fence_after();
         issue_pv(st, tbase + g * 128 + 64, tbase + 256 + g * 128, j >= 2);
-        mma_commit(&kv_empty[st]);
+        commit(&kv_empty[st]);
       }
-      mma_commit(o_final);
-    }
-    __syncwarp();
+      commit(o_final);
     }
     cta_end_sync();
     if (warp == 1) {

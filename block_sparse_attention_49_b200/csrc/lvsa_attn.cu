@@ -1,0 +1,543 @@
+// LVSA attention in one kernel, on the natural token layout.
+//
+// What it computes ("LVSA: Training-Free Sparse Attention for Long Video
+// Diffusion", section 2 "Core mechanism"): every query token of frame t
+// attends, with softmax(scale * q.k), exactly the key tokens of the frames in
+// A(t) = G_s U W(t) - rotating anchors G_s = {f : (f - s) mod T_per = 0} and
+// a window around t grown t+1, t-1, t+2, ... past the frames already present
+// until |A(t)| = C.  The result equals bsa_lvsa_mask + bsa_reorder_fwd +
+// bsa_attn_fwd + bsa_reorder_inv; the reorder of the Draft Attention article
+// is fused into the tile loads (a 3-D tensor map reads [B*N, Hh, D] rows of
+// one head directly), so no padded copy of Q, K, V or O is ever made.
+//
+// Work unit (one CTA, 12 warps): 256 consecutive query tokens of one
+// (b, head) = two 128-row query tiles that share every key tile.
+//  * set-up: A(t) for the (at most 8) frames of the 256 queries, as bitmaps
+//    over frames; their union U; the key tiles = 128-token pieces of each run
+//    of consecutive frames of U.  Membership uses a closed form: a frame f
+//    outside G_s U {t} joins iff fewer than C - |G_s U {t}| such frames come
+//    before it in the growth order; anchors in a range are counted
+//    arithmetically (they are periodic).
+//  * warp 0: TMA producer (both query tiles, then K and V of every key tile
+//    into a 2-deep ring).  warp 1: MMA issuer.  warps 4-7 / 8-11: softmax of
+//    query tile 0 / 1, one row per thread, masking keys whose frame is not in
+//    the row's own A(t).
+//  * tensor memory: S0 | S1 | O0 | O1; P aliases the upper half of its S.
+//    MMA order per key tile j: PV0(j), QK0(j+1), PV1(j), QK1(j+1), so the
+//    tensor cores run one tile's products while the other tile's softmax runs.
+// Every wait is bounded (see bounded_wait).
+#include <cuda_bf16.h>
+#include <cudaTypedefs.h>
+
+#include <algorithm>
+#include <cmath>
+
+#include "attn_common.cuh"
+#include "bsa_internal.cuh"
+#include "ptx.cuh"
+
+namespace bsa {
+namespace {
+
+constexpr int kTile = 128;
+constexpr int kPair = 2 * kTile;
+constexpr int kThreads = 384;
+constexpr int kMaxRowFrames = 8;   // frames a 256-token query pair may touch
+constexpr int kMaxFrames = 4096;
+constexpr int kSetWords = kMaxFrames / 32;
+constexpr int kMaxTiles = 4096;    // key tiles per query pair
+
+template <int D>
+struct LvsaCfg {
+  static constexpr int kChunks = D / 64;
+  static constexpr int kPanel = kTile * 128;
+  static constexpr int kQBytes = kTile * D * 2;
+  static constexpr int kKVBytes = kTile * D * 2;
+  static constexpr int NS = (D == 128) ? 2 : 4;
+  static constexpr int kOffQ = 0;
+  static constexpr int kOffK = 2 * kQBytes;
+  static constexpr int kOffV = kOffK + NS * kKVBytes;
+  static constexpr int kOffBar = kOffV + NS * kKVBytes;
+  static constexpr int kNumBars = 1 + 3 * NS + 2 + 2 + 1;
+  static constexpr int kOffMisc = kOffBar + kNumBars * 8;
+  static constexpr int kOffTiles = kOffMisc + 16;
+  static constexpr int kOffSets = kOffTiles + kMaxTiles * 4;
+  static constexpr int kBytes = kOffSets + (kMaxRowFrames + 1) * kSetWords * 4;
+  static constexpr int kSmem = kBytes + 1024;
+  static constexpr uint32_t kTmemCols = 512;
+  static_assert(kSmem <= 232448, "shared memory budget");
+};
+
+struct LvsaParams {
+  int B, Hh, T, P, N, C, T_per, s_mod;
+  FastDiv divP;
+  float scale, scale_log2;
+  __nv_bfloat16* o;  // natural layout
+  float* lse;        // [B, Hh, N] or null
+  unsigned int* status;
+  uint64_t wait_limit_ns;
+};
+
+__device__ __forceinline__ int floordiv(int a, int b) {
+  int q = a / b;
+  if ((a % b != 0) && (a < 0)) --q;  // b > 0
+  return q;
+}
+
+// anchors in [a, b] (frames f with f = s_mod mod T_per)
+__device__ __forceinline__ int anchors_in(int a, int b, int s_mod, int T_per) {
+  return b < a ? 0 : floordiv(b - s_mod, T_per) - floordiv(a - 1 - s_mod, T_per);
+}
+
+__device__ __forceinline__ bool is_anchor(int f, int s_mod, int T_per) {
+  int r = (f - s_mod) % T_per;
+  if (r < 0) r += T_per;
+  return r == 0;
+}
+
+// f in A(t)?
+__device__ bool lvsa_member(int t, int f, const LvsaParams& p) {
+  const bool t_anchor = is_anchor(t, p.s_mod, p.T_per);
+  if (f == t || is_anchor(f, p.s_mod, p.T_per)) return true;
+  const int base = anchors_in(0, p.T - 1, p.s_mod, p.T_per) + (t_anchor ? 0 : 1);
+  const int need = p.C - base;
+  const int d = f > t ? f - t : t - f;
+  // frames outside the base strictly nearer than d (t itself is in the base)
+  const int lo = max(t - d + 1, 0), hi = min(t + d - 1, p.T - 1);
+  int before = (hi - lo + 1) - anchors_in(lo, hi, p.s_mod, p.T_per) - (t_anchor ? 0 : 1);
+  // at equal distance the right-hand frame comes first
+  if (f < t && t + d < p.T && !is_anchor(t + d, p.s_mod, p.T_per)) ++before;
+  return before < need;
+}
+
+__device__ __forceinline__ bool bit_of(const uint32_t* set, int f) {
+  return (set[f >> 5] >> (f & 31)) & 1u;
+}
+
+// first f' >= f (f' < T) with bit value `v` in `set`, else T
+__device__ int next_with(const uint32_t* set, int f, int T, bool v) {
+  while (f < T) {
+    uint32_t w = set[f >> 5];
+    if (!v) w = ~w;
+    w &= kFullMask << (f & 31);
+    if (w) {
+      const int g = (f & ~31) + __ffs(w) - 1;
+      return g < T ? g : T;
+    }
+    f = (f & ~31) + 32;
+  }
+  return T;
+}
+
+__device__ __forceinline__ void cta_end_sync() { asm volatile("bar.sync 2, 384;" ::: "memory"); }
+
+__device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, uint64_t* bar, int x,
+                                            int y, int z) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(x), "r"(y), "r"(z)
+      : "memory");
+}
+
+template <int D>
+__global__ void __launch_bounds__(kThreads, 1)
+    lvsa_attn_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmk,
+                     const __grid_constant__ CUtensorMap tmv, const LvsaParams p) {
+  using Cfg = LvsaCfg<D>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  uint8_t* sQ = smem + Cfg::kOffQ;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Cfg::kOffBar);
+  uint64_t* q_full = bars;
+  uint64_t* k_full = bars + 1;
+  uint64_t* v_full = k_full + Cfg::NS;
+  uint64_t* kv_empty = v_full + Cfg::NS;
+  uint64_t* s_full = kv_empty + Cfg::NS;  // [2]
+  uint64_t* p_ready = s_full + 2;         // [2]
+  uint64_t* o_final = p_ready + 2;
+  uint32_t* misc = reinterpret_cast<uint32_t*>(smem + Cfg::kOffMisc);  // tmem, abort, ntiles, skip
+  int32_t* tiles = reinterpret_cast<int32_t*>(smem + Cfg::kOffTiles);  // (k0 << 7) | (count - 1)
+  uint32_t* sets = reinterpret_cast<uint32_t*>(smem + Cfg::kOffSets);  // [rf][kSetWords], union last
+  uint32_t* uset = sets + kMaxRowFrames * kSetWords;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int pair = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+  const int q0 = pair * kPair;
+  const int64_t brow = (int64_t)b * p.N;
+  const int q_last = min(q0 + kPair, p.N) - 1;
+  const int tf = (int)p.divP.div((uint32_t)q0);
+  const int nrf = (int)p.divP.div((uint32_t)q_last) - tf + 1;
+  const int words = (p.T + 31) >> 5;
+  const WaitCtx wc{p.status, reinterpret_cast<volatile int*>(&misc[1]), p.wait_limit_ns};
+
+  // ------------------------------------------------------------ set-up
+  if (threadIdx.x == 0) {
+    mbar_init(q_full, 1);
+    for (int i = 0; i < Cfg::NS; ++i) {
+      mbar_init(&k_full[i], 1);
+      mbar_init(&v_full[i], 1);
+      mbar_init(&kv_empty[i], 1);
+    }
+    mbar_init(&s_full[0], 1);
+    mbar_init(&s_full[1], 1);
+    mbar_init(&p_ready[0], 128);
+    mbar_init(&p_ready[1], 128);
+    mbar_init(o_final, 1);
+    misc[1] = 0;
+    misc[2] = 0;
+    misc[3] = (*reinterpret_cast<volatile unsigned int*>(p.status) & kStatusTimeout) ? 1u : 0u;
+    fence_mbar_init();
+    prefetch_tmap(&tmq);
+    prefetch_tmap(&tmk);
+    prefetch_tmap(&tmv);
+  }
+  __syncthreads();
+  if (misc[3]) return;
+  if (warp == 1) {
+    tmem_alloc(&misc[0], Cfg::kTmemCols);
+    tmem_relinquish();
+  }
+  // frame sets of the query frames tf .. tf+nrf-1 (one 32-frame word per step)
+  for (int idx = threadIdx.x; idx < nrf * words; idx += kThreads) {
+    const int rf = idx / words, w = idx - rf * words;
+    uint32_t bits = 0u;
+    for (int i = 0; i < 32; ++i) {
+      const int f = 32 * w + i;
+      if (f < p.T && lvsa_member(tf + rf, f, p)) bits |= 1u << i;
+    }
+    sets[rf * kSetWords + w] = bits;
+  }
+  __syncthreads();
+  for (int w = threadIdx.x; w < words; w += kThreads) {
+    uint32_t u = 0u;
+    for (int rf = 0; rf < nrf; ++rf) u |= sets[rf * kSetWords + w];
+    uset[w] = u;
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    // key tiles: 128-token pieces of each run of consecutive frames of U
+    int cnt = 0;
+    bool overflow = false;
+    for (int f = next_with(uset, 0, p.T, true); f < p.T;) {
+      const int e = next_with(uset, f, p.T, false);  // run [f, e)
+      const int tok0 = f * p.P, tok1 = e * p.P;
+      for (int k = tok0; k < tok1; k += kTile) {
+        // first key token and number of this run's keys in the tile: the
+        // tile's overhang past the run is masked, so a key that also starts
+        // the next run is never counted twice
+        if (cnt < kMaxTiles) tiles[cnt++] = (k << 7) | (min(kTile, tok1 - k) - 1);
+        else overflow = true;
+      }
+      f = next_with(uset, e, p.T, true);
+    }
+    if (overflow) atomicOr(p.status, kStatusBadBlocklist);
+    misc[2] = cnt;
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tbase = misc[0];
+  const int n = (int)misc[2];
+
+  if (warp < 4) {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 56;");
+    if (warp == 0 && n > 0) {
+      // -------------------------------------------------------- TMA producer
+      // the whole warp runs the loop (warp-uniform operands); one lane issues
+      if (elect_one()) {
+        mbar_arrive_expect_tx(q_full, 2 * Cfg::kQBytes);
+        for (int g = 0; g < 2; ++g)
+          for (int c = 0; c < Cfg::kChunks; ++c)
+            tma_load_3d(sQ + g * Cfg::kQBytes + c * Cfg::kPanel, &tmq, q_full, c * 64, h,
+                        (int)(brow + q0 + g * kTile));
+      }
+      __syncwarp();
+      int issued = 0;
+      for (int j = 0; j < n; ++j) {
+        const int st = j % Cfg::NS;
+        if (!__all_sync(kFullMask, bounded_wait(&kv_empty[st], ((j / Cfg::NS) & 1) ^ 1, wc))) break;
+        const int krow = (int)(brow + (tiles[j] >> 7));
+        if (elect_one()) {
+          uint8_t* sK = smem + Cfg::kOffK + st * Cfg::kKVBytes;
+          uint8_t* sV = smem + Cfg::kOffV + st * Cfg::kKVBytes;
+          mbar_arrive_expect_tx(&k_full[st], Cfg::kKVBytes);
+          for (int c = 0; c < Cfg::kChunks; ++c)
+            tma_load_3d(sK + c * Cfg::kPanel, &tmk, &k_full[st], c * 64, h, krow);
+          mbar_arrive_expect_tx(&v_full[st], Cfg::kKVBytes);
+          for (int c = 0; c < Cfg::kChunks; ++c)
+            tma_load_3d(sV + c * Cfg::kPanel, &tmv, &v_full[st], c * 64, h, krow);
+        }
+        __syncwarp();
+        issued = j + 1;
+      }
+      if (*wc.abort) {
+        // leave no copy in flight: wait (bounded, ignoring the abort flag)
+        // for the loads still owned by the ring
+        volatile int no_abort = 0;
+        const WaitCtx drain{p.status, &no_abort, p.wait_limit_ns};
+        bounded_wait(q_full, 0, drain);
+        for (int j = max(0, issued - Cfg::NS); j < issued; ++j) {
+          bounded_wait(&k_full[j % Cfg::NS], (j / Cfg::NS) & 1, drain);
+          bounded_wait(&v_full[j % Cfg::NS], (j / Cfg::NS) & 1, drain);
+        }
+      }
+      __syncwarp();
+    } else if (warp == 1 && n > 0) {
+      // -------------------------------------------------------- MMA issuer
+      // the whole warp runs the loop (descriptors stay warp-uniform); the
+      // elected lane issues the tcgen05 instructions
+      constexpr uint32_t idesc_qk = idesc_bf16(128, 128, 0);
+      constexpr uint32_t idesc_pv = idesc_bf16(128, D, 1);
+      const uint64_t qd0 = sdesc_sw128(smem_u32(sQ), 16, 1024);
+      const uint64_t kd0 = sdesc_sw128(smem_u32(smem + Cfg::kOffK), 16, 1024);
+      const uint64_t vd0 = sdesc_sw128(smem_u32(smem + Cfg::kOffV), Cfg::kPanel, 1024);
+      auto issue_qk = [&](int g, int st) {
+        const uint32_t dst = tbase + g * 128;
+        const uint64_t qd = sdesc_add(qd0, g * Cfg::kQBytes);
+        const uint64_t kd = sdesc_add(kd0, st * Cfg::kKVBytes);
+        if (elect_one()) {
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint32_t off = (kk >> 2) * Cfg::kPanel + (kk & 3) * 32;
+            mma_ss(dst, sdesc_add(qd, off), sdesc_add(kd, off), idesc_qk, kk > 0);
+          }
+          mma_commit(&s_full[g]);
+        }
+        __syncwarp();
+      };
+      auto issue_pv = [&](int g, int st, uint32_t acc) {
+        const uint32_t dst = tbase + 256 + g * 128, pa = tbase + g * 128 + 64;
+        const uint64_t vd = sdesc_add(vd0, st * Cfg::kKVBytes);
+        if (elect_one()) {
+#pragma unroll
+          for (int kk = 0; kk < kTile / 16; ++kk)
+            mma_ts(dst, pa + kk * 8, sdesc_add(vd, kk * 2048), idesc_pv, (acc | (uint32_t)kk) != 0);
+        }
+        __syncwarp();
+      };
+      auto commit = [&](uint64_t* bar) {
+        if (elect_one()) mma_commit(bar);
+        __syncwarp();
+      };
+      auto wait = [&](uint64_t* bar, uint32_t parity) {
+        return __all_sync(kFullMask, bounded_wait(bar, parity, wc));
+      };
+      bool alive = wait(q_full, 0) && wait(&k_full[0], 0);
+      if (alive) {
+        tc_fence_after();
+        issue_qk(0, 0);
+        issue_qk(1, 0);
+      }
+      for (int j = 0; alive && j < n; ++j) {
+        const int st = j % Cfg::NS, st1 = (j + 1) % Cfg::NS;
+        if (!wait(&p_ready[0], j & 1) || !wait(&v_full[st], (j / Cfg::NS) & 1)) break;
+        tc_fence_after();
+        issue_pv(0, st, j > 0);
+        if (j + 1 < n) {
+          if (!wait(&k_full[st1], ((j + 1) / Cfg::NS) & 1)) break;
+          tc_fence_after();
+          issue_qk(0, st1);
+        }
+        if (!wait(&p_ready[1], j & 1)) break;
+        tc_fence_after();
+        issue_pv(1, st, j > 0);
+        commit(&kv_empty[st]);
+        if (j + 1 < n) issue_qk(1, st1);
+      }
+      commit(o_final);
+    }
+    cta_end_sync();
+    if (warp == 1) {
+      tc_fence_after();
+      tmem_dealloc(tbase, Cfg::kTmemCols);
+    }
+  } else {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 224;");
+    // ---------------------------------------------------------- softmax
+    const int g = (warp >= 8) ? 1 : 0;
+    const int q4 = warp & 3;
+    const int row = q4 * 32 + lane;
+    const uint32_t lane_off = (uint32_t)(q4 * 32) << 16;
+    const uint32_t tS = tbase + g * 128 + lane_off;
+    const uint32_t tO = tbase + 256 + g * 128 + lane_off;
+    const int qn = q0 + g * kTile + row;  // query token within the batch
+    const bool qvalid = qn < p.N;
+    const int tq = qvalid ? (int)p.divP.div((uint32_t)qn) : 0;
+    const uint32_t* myset = sets + (tq - tf) * kSetWords;
+    const float sl2 = p.scale_log2;
+    const float thr = 8.0f / sl2;
+    RowState st;
+    bool alive = true;
+    for (int j = 0; j < n; ++j) {
+      // keys of tile j allowed for this row: those whose frame is in A(tq)
+      uint32_t vm[4] = {0u, 0u, 0u, 0u};
+      if (qvalid) {
+        const int k0 = tiles[j] >> 7, kn = (tiles[j] & 127) + 1;  // keys [k0, k0 + kn)
+        int f = (int)p.divP.div((uint32_t)k0);
+        int lo = 0, fend = (f + 1) * p.P - k0;
+        while (lo < kn) {
+          const int hi = min(kn, fend);
+          if (f < p.T && bit_of(myset, f)) set_range(vm, lo, hi);
+          lo = hi;
+          ++f;
+          fend += p.P;
+        }
+      }
+      if (!__all_sync(kFullMask, bounded_wait(&s_full[g], j & 1, wc))) {
+        alive = false;
+        break;
+      }
+      tc_fence_after();
+      float s[128];
+      {
+        uint32_t r128[128];
+        tmem_ld128(tS, r128);
+#pragma unroll
+        for (int i = 0; i < 128; ++i) s[i] = __uint_as_float(r128[i]);
+      }
+      uint32_t pk[64];
+      float corr;
+      const bool need = softmax_tile(s, vm, st, sl2, thr, pk, corr);
+      // S of tile j was written after PV of tile j-1: O is complete here
+      if (j > 0 && __any_sync(kFullMask, need)) tmem_scale<D>(tO, corr);
+      tmem_st32(tS + 64, *reinterpret_cast<uint32_t(*)[32]>(&pk[0]));
+      tmem_st32(tS + 96, *reinterpret_cast<uint32_t(*)[32]>(&pk[32]));
+      tc_fence_before();
+      mbar_arrive(&p_ready[g]);
+    }
+    if (alive && n > 0) {
+      alive = __all_sync(kFullMask, bounded_wait(o_final, 0, wc));
+      tc_fence_after();
+    }
+    const bool has = alive && n > 0 && qvalid && st.l > 0.f;
+    const float inv_l = has ? 1.f / st.l : 0.f;
+    uint4* dst = reinterpret_cast<uint4*>(p.o + ((brow + qn) * p.Hh + h) * D);
+#pragma unroll
+    for (int c = 0; c < D / 32; ++c) {
+      uint32_t o32[32];
+      if (alive && n > 0) {
+        tmem_ld32(tO + c * 32, o32);
+      } else {
+#pragma unroll
+        for (int i = 0; i < 32; ++i) o32[i] = 0u;
+      }
+      uint32_t w16[16];
+#pragma unroll
+      for (int i = 0; i < 16; ++i)
+        w16[i] = pack_bf16x2(__uint_as_float(o32[2 * i]) * inv_l,
+                             __uint_as_float(o32[2 * i + 1]) * inv_l);
+      if (qvalid) {
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+          dst[c * 4 + i] = make_uint4(w16[4 * i], w16[4 * i + 1], w16[4 * i + 2], w16[4 * i + 3]);
+      }
+    }
+    if (qvalid && p.lse)
+      p.lse[((int64_t)b * p.Hh + h) * p.N + qn] = has ? st.m * p.scale + logf(st.l) : -INFINITY;
+    tc_fence_before();
+    cta_end_sync();
+  }
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn3() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (!fn) {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+  }
+  return fn;
+}
+
+// Natural layout [B*N, Hh, D] bf16: boxes of 64 channels x 1 head x 128 tokens.
+bool make_tmap_natural(CUtensorMap* m, const void* ptr, int64_t tokens, int Hh, int D) {
+  auto fn = encode_fn3();
+  if (!fn) return false;
+  cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)Hh, (cuuint64_t)tokens};
+  cuuint64_t strides[2] = {(cuuint64_t)D * 2, (cuuint64_t)Hh * D * 2};
+  cuuint32_t box[3] = {64, 1, (cuuint32_t)kTile};
+  cuuint32_t estr[3] = {1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims, strides, box,
+            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int D>
+cudaError_t launch_lvsa_t(const CUtensorMap& q, const CUtensorMap& k, const CUtensorMap& v,
+                          const LvsaParams& p, dim3 grid, cudaStream_t st) {
+  auto kern = lvsa_attn_kernel<D>;
+  cudaError_t e =
+      cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, LvsaCfg<D>::kSmem);
+  if (e != cudaSuccess) return e;
+  kern<<<grid, kThreads, LvsaCfg<D>::kSmem, st>>>(q, k, v, p);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+}  // namespace bsa
+
+using namespace bsa;
+
+extern "C" bsa_status bsa_lvsa_attn_fwd(bsa_plan_t plan, int C, int T_per, int s, const void* q,
+                                        const void* k, const void* v, float scale, void* o,
+                                        float* lse, void* stream) {
+  if (!plan) return set_error(BSA_ERR_INVALID_ARG, "plan is NULL");
+  const Geometry& g = plan->g;
+  if (g.layout != BSA_LAYOUT_FRAME) return set_error(BSA_ERR_INVALID_ARG, "LVSA attention needs a FRAME plan");
+  if (T_per < 1) return set_error(BSA_ERR_INVALID_ARG, "T_per must be >= 1");
+  if (C < 1 || C > g.T) return set_error(BSA_ERR_INVALID_ARG, "C must be in [1, T]");
+  if (!(scale > 0.f)) return set_error(BSA_ERR_INVALID_ARG, "scale must be positive");
+  for (const void* ptr : {q, k, v, (const void*)o}) {
+    if (!ptr) return set_error(BSA_ERR_INVALID_ARG, "q / k / v / o is NULL");
+    if (!aligned16(ptr)) return set_error(BSA_ERR_ALIGNMENT, "q / k / v / o not 16-byte aligned");
+  }
+  if (lse && (reinterpret_cast<uintptr_t>(lse) & 3u))
+    return set_error(BSA_ERR_ALIGNMENT, "lse is not 4-byte aligned");
+  const int sm = ((s % T_per) + T_per) % T_per;
+  int anchors = 0;
+  for (int f = 0; f < g.T; ++f) anchors += ((f - sm) % T_per + T_per) % T_per == 0;
+  if (anchors + (anchors < g.T ? 1 : 0) > C)
+    return set_error(BSA_ERR_INVALID_ARG, "budget C is smaller than the anchors plus the query frame");
+  if (g.T > kMaxFrames) return set_error(BSA_ERR_UNSUPPORTED, "fused LVSA attention supports T <= 4096");
+  if (g.P < 37) return set_error(BSA_ERR_UNSUPPORTED, "fused LVSA attention needs >= 37 tokens per frame");
+  const int64_t N = (int64_t)g.T * g.P;
+  if ((int64_t)g.B * N >= (1ll << 31)) return set_error(BSA_ERR_UNSUPPORTED, "B*N must be < 2^31");
+  if (N >= (1 << 24)) return set_error(BSA_ERR_UNSUPPORTED, "fused LVSA attention needs N < 2^24");
+  // key tiles of a query pair: at most |U| frames, |U| <= min(T, rows' frames * C)
+  const int64_t u_frames = std::min<int64_t>(g.T, (int64_t)kMaxRowFrames * C);
+  if ((u_frames * g.P + kTile - 1) / kTile + u_frames > kMaxTiles)
+    return set_error(BSA_ERR_UNSUPPORTED, "fused LVSA attention: too many key tiles per query pair");
+  CUtensorMap tq, tk, tv;
+  const int64_t tokens = (int64_t)g.B * N;
+  if (!make_tmap_natural(&tq, q, tokens, g.Hh, g.D) || !make_tmap_natural(&tk, k, tokens, g.Hh, g.D) ||
+      !make_tmap_natural(&tv, v, tokens, g.Hh, g.D))
+    return set_error(BSA_ERR_CUDA, "cuTensorMapEncodeTiled failed");
+  LvsaParams p;
+  p.B = g.B;
+  p.Hh = g.Hh;
+  p.T = g.T;
+  p.P = g.P;
+  p.N = (int)N;
+  p.C = C;
+  p.T_per = T_per;
+  p.s_mod = sm;
+  p.divP = FastDiv((uint32_t)g.P);
+  p.scale = scale;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  p.o = reinterpret_cast<__nv_bfloat16*>(o);
+  p.lse = lse;
+  p.status = plan->d_status;
+  p.wait_limit_ns = plan->wait_limit_ns;
+  const dim3 grid((unsigned)((N + kPair - 1) / kPair), (unsigned)g.Hh, (unsigned)g.B);
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const cudaError_t e = g.D == 128 ? launch_lvsa_t<128>(tq, tk, tv, p, grid, st)
+                                   : launch_lvsa_t<64>(tq, tk, tv, p, grid, st);
+  return e == cudaSuccess ? BSA_OK : cuda_error(e, "lvsa_attn launch");
+}
+

@@ -12,6 +12,19 @@ __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
 
+// One lane of the (converged) warp returns true.  Code that issues
+// tcgen05/TMA instructions runs on the whole warp, so that its operands are
+// warp-uniform, and only the elected lane issues.
+__device__ __forceinline__ bool elect_one() {
+  uint32_t pred = 0;
+  asm volatile(
+      "{\n\t.reg .pred P;\n\t"
+      "elect.sync _|P, 0xffffffff;\n\t"
+      "selp.b32 %0, 1, 0, P;\n\t}"
+      : "=r"(pred));
+  return pred != 0;
+}
+
 // ---------------------------------------------------------------- mbarrier
 __device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
   asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count)
@@ -40,6 +53,21 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
+// As mbar_try_wait, but the thread may be suspended (issuing nothing) for up
+// to `hint_ns` nanoseconds while the phase is incomplete; it resumes as soon
+// as the phase completes.
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t* bar, uint32_t parity, uint32_t hint_ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.b32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity), "r"(hint_ns)
+      : "memory");
+  return ok != 0;
+}
+
 __device__ __forceinline__ uint64_t global_timer_ns() {
   uint64_t t;
   asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
@@ -57,12 +85,15 @@ struct WaitCtx {
 
 // Waits for the phase of parity `parity` of `bar` to complete.  Returns false
 // (and records a timeout) when the wait exceeds the limit or another role of
-// the CTA already gave up.
+// the CTA, or another CTA, already gave up.  A waiting thread sleeps inside
+// mbarrier.try_wait (suspend-time hint 200 us) instead of spinning, so it
+// takes no issue slots from the warps doing work on the same sub-partition;
+// between sleeps it checks the abort flag, the status word and the clock.
 __device__ __forceinline__ bool bounded_wait(uint64_t* bar, uint32_t parity, const WaitCtx& w) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = global_timer_ns();
   while (true) {
-    if (mbar_try_wait(bar, parity)) return true;
+    if (mbar_try_wait_sleep(bar, parity, 200000u)) return true;
     if (*w.abort) return false;
     if (*reinterpret_cast<volatile unsigned int*>(w.status) & 2u) {
       *w.abort = 1;  // another CTA already ran out: stop waiting
@@ -156,6 +187,13 @@ __host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, int b_mn) {
 __device__ __forceinline__ uint64_t sdesc_sw128(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
   return (uint64_t)((saddr >> 4) & 0x3FFFu) | ((uint64_t)((lbo >> 4) & 0x3FFFu) << 16) |
          ((uint64_t)((sbo >> 4) & 0x3FFFu) << 32) | (1ull << 46) | (2ull << 61);
+}
+
+// Advance a descriptor's start address by `bytes` (a multiple of 16).  The
+// address field is the low 14 bits in 16-byte units; shared memory offsets
+// stay below 256 KB, so the add never carries into the other fields.
+__device__ __forceinline__ uint64_t sdesc_add(uint64_t d, uint32_t bytes) {
+  return d + (uint64_t)(bytes >> 4);
 }
 
 // 32 lanes x 32 columns of 32-bit from tensor memory, waited on in the same

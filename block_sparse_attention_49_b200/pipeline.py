@@ -15,8 +15,8 @@ import math
 import torch
 
 from . import (LAYOUT_FRAME, LAYOUT_TILE, Plan, bsa_attn_fwd, bsa_draft_keep_count,
-               bsa_draft_mask, bsa_draft_workspace_bytes, bsa_lvsa_mask, bsa_lvsa_nnz,
-               bsa_reorder_fwd, bsa_reorder_inv)
+               bsa_draft_mask, bsa_draft_workspace_bytes, bsa_lvsa_attn_fwd, bsa_lvsa_mask,
+               bsa_lvsa_nnz, bsa_reorder_fwd, bsa_reorder_inv)
 
 
 class _Base:
@@ -62,6 +62,12 @@ class LvsaAttention(_Base):
         self.gather(q, k, v)
         self.attend(per_head=False)
         return self.scatter(out)
+
+    def fused(self, q, k, v, s: int, out=None, lse=None):
+        """The same attention in one kernel on the natural layout."""
+        out = torch.empty_like(q) if out is None else out
+        bsa_lvsa_attn_fwd(self.plan, self.C, self.T_per, s, q, k, v, self.scale, out, lse)
+        return out
 
 
 class DraftAttention(_Base):

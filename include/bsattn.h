@@ -178,6 +178,23 @@ bsa_status bsa_attn_fwd(bsa_plan_t plan, const void* q, const void* k, const voi
                         const int32_t* row_ptr, const int32_t* col_idx, int per_head_lists,
                         float scale, void* o, float* lse, void* stream);
 
+/* LVSA attention in one pass on the natural layout ("LVSA", section 2 "Core
+ * mechanism"; the reorder of the Draft Attention article is fused into the
+ * tile loads, so no padded copies are made).
+ * Requires a FRAME plan (its block size is not used), D = 64 or 128,
+ * T <= 4096 and H*W >= 37; C, T_per and s as for bsa_lvsa_mask.
+ * q, k, v, o: natural layout [B, N, Hh, D] bf16, o written for every token.
+ * lse: float[B*Hh*N] at (b*Hh + h)*N + n, or NULL.
+ * Every query token of frame t attends exactly the key tokens of the frames
+ * in A(t):  O[n] = sum_m softmax_m(scale * <q_n, k_m>) v_m over those keys;
+ * LSE[n] = log sum_m exp(scale * <q_n, k_m>).  The result is that of
+ * bsa_lvsa_mask + bsa_reorder_fwd + bsa_attn_fwd + bsa_reorder_inv, up to the
+ * order of fp32 summation.  fp32 accumulation; probabilities rounded to bf16
+ * before the PV product. */
+bsa_status bsa_lvsa_attn_fwd(bsa_plan_t plan, int C, int T_per, int s, const void* q,
+                             const void* k, const void* v, float scale, void* o, float* lse,
+                             void* stream);
+
 /* Synchronize `stream`, read and clear the plan's device status word.
  * Returns BSA_OK, BSA_ERR_BAD_BLOCKLIST, BSA_ERR_TIMEOUT or BSA_ERR_CUDA. */
 bsa_status bsa_poll_status(bsa_plan_t plan, void* stream);
