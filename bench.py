@@ -1,10 +1,13 @@
 """Benchmark of the LVSA block-sparse attention path on B200.
 
-A step is one pass of the whole LVSA hot path over one batch of the Wan-2.1-
-1.3B-like 6x-length workload (B=1, 12 heads, D=128, grid 126x30x52 = 196,560
-tokens, C=21, T_per=12): lvsa_mask(s) -> reorder_fwd(Q,K,V) -> bsattn ->
-reorder_inv(O), with s = step mod T_per.  Inputs (1.8 GB) exceed the 126 MB
-L2, so no flush is needed between steps.
+A step is one pass of the LVSA hot path over one batch of the Wan-2.1-1.3B-
+like 6x-length workload (B=1, 12 heads, D=128, grid 126x30x52 = 196,560
+tokens, C=21, T_per=12), with s = step mod T_per: natural-layout Q, K, V in,
+natural-layout O out.  The step runs bsa_lvsa_attn_fwd, the one-kernel path
+(frame sets computed in the kernel, the reorder fused into its tile loads).
+The four-kernel path over the same data (lvsa_mask -> reorder_fwd ->
+attn_fwd on the block list -> reorder_inv) is timed too and reported per
+kernel.  Inputs (1.8 GB) exceed the 126 MB L2, so no flush is needed.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
@@ -34,6 +37,12 @@ sys.path.insert(0, ROOT)
 from synth import CONFIGS, make_qkv  # noqa: E402
 
 METRIC = "bsattn ms/call + attended TFLOP/s (% BF16 peak), Wan-1.3B-shape 6× length LVSA"
+
+# DRAM bytes per launch of the step kernel at the full workload, from the ncu
+# capture summarised in profiles/lvsa_attn_fwd_wan13b_6x_first24frames.md
+# (24-frame case, scaled by the number of query pairs).  Set to None whenever
+# the kernel changes until it is captured again.
+STEP_KERNEL_DRAM_BYTES = 449.8e6 * 126 / 24
 
 
 def attended_flops(w) -> float:
@@ -103,6 +112,23 @@ class ClockSampler:
         return {"sm_mhz": statistics.median(sm) if sm else None,
                 "sm_max_mhz": max(mx) if mx else None, "reasons": reasons,
                 "samples": len(rows)}
+
+
+def max_over_ranks(values, dist=None, device="cpu"):
+    """Element-wise maximum of per-rank timings (the whole job is as slow as
+    its slowest rank).  Works with any torch.distributed backend; without a
+    process group it returns the values unchanged."""
+    vals = [float(v) for v in values]
+    if dist is None or not dist.is_available() or not dist.is_initialized():
+        return vals
+    t = torch.tensor(vals, dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(x) for x in t.tolist()]
+
+
+def weak_scaling_value(flops_per_rank: float, world: int, ms_max: float) -> float:
+    """Whole-job attended TFLOP/s: every rank ran its own batch in ms_max."""
+    return world * flops_per_rank / (ms_max * 1e-3) / 1e12
 
 
 def cpu_baseline(w, q_h, k_h, v_h, budget_s: float, seed: int = 0):
@@ -219,51 +245,53 @@ def main():
     att = LvsaAttention(w.B, w.Hh, w.D, w.T, w.H, w.W, w.lvsa_C, w.lvsa_T_per, block=128)
     out = torch.empty_like(q)
     stream = torch.cuda.current_stream()
-    launches_per_step = 4  # lvsa_mask, reorder_fwd, bsattn, reorder_inv
+    ev = lambda: torch.cuda.Event(enable_timing=True)
 
-    names = ("lvsa_mask", "reorder_fwd", "bsattn_fwd", "reorder_inv")
-    ev = []
-
-    def step(i, record):
-        s = i % w.lvsa_T_per
-        calls = (lambda: att.mask(s), lambda: att.gather(q, k, v),
-                 lambda: att.attend(per_head=False), lambda: att.scatter(out))
-        if not record:
-            for c in calls:
-                c()
-            return
-        marks = [torch.cuda.Event(enable_timing=True) for _ in range(len(calls) + 1)]
-        marks[0].record(stream)
-        for j, c in enumerate(calls):
-            c()
-            marks[j + 1].record(stream)
-        ev.append(marks)
+    def step(i):
+        att.fused(q, k, v, i % w.lvsa_T_per, out)
 
     for i in range(args.warmup):
-        step(i, False)
+        step(i)
     bsa.bsa_poll_status(att.plan)
     torch.cuda.synchronize()
     if dist:
         dist.barrier()
     clocks = ClockSampler(local)
     clocks.start()
-    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    marks = [ev() for _ in range(args.steps + 1)]
     torch.cuda.synchronize()
-    t0.record(stream)
+    marks[0].record(stream)
     for i in range(args.steps):
-        step(args.warmup + i, True)
-    t1.record(stream)
+        step(args.warmup + i)
+        marks[i + 1].record(stream)
     torch.cuda.synchronize()
     clk = clocks.stop()
     bsa.bsa_poll_status(att.plan)
-    ms = t0.elapsed_time(t1) / args.steps
-    kern_ms = {n: statistics.mean(m[j].elapsed_time(m[j + 1]) for m in ev)
-               for j, n in enumerate(names)}
-    attn_ms = kern_ms["bsattn_fwd"]
-    if dist:
-        tt = torch.tensor([ms, attn_ms], device="cuda")
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        ms, attn_ms = float(tt[0]), float(tt[1])
+    per_call = [marks[i].elapsed_time(marks[i + 1]) for i in range(args.steps)]
+    ms = marks[0].elapsed_time(marks[-1]) / args.steps
+    attn_ms = statistics.mean(per_call)  # the step is the one attention launch
+    ms, attn_ms = max_over_ranks([ms, attn_ms], dist, "cuda")
+
+    # the four-kernel path on the same data, per kernel (secondary numbers)
+    names = ("lvsa_mask", "reorder_fwd", "attn_fwd_blocklist", "reorder_inv")
+    unf = {n: [] for n in names}
+    n_unf = max(3, min(args.steps, 10))
+    for i in range(args.warmup + n_unf):
+        s_i = i % w.lvsa_T_per
+        calls = (lambda: att.mask(s_i), lambda: att.gather(q, k, v),
+                 lambda: att.attend(per_head=False), lambda: att.scatter(out))
+        m = [ev() for _ in range(len(calls) + 1)]
+        m[0].record(stream)
+        for j, c in enumerate(calls):
+            c()
+            m[j + 1].record(stream)
+        if i >= args.warmup:
+            torch.cuda.synchronize()
+            for j, n in enumerate(names):
+                unf[n].append(m[j].elapsed_time(m[j + 1]))
+    torch.cuda.synchronize()
+    bsa.bsa_poll_status(att.plan)
+    unf_ms = max_over_ranks([statistics.mean(unf[n]) for n in names], dist, "cuda")
 
     # end to end through the public API with host buffers: pinned H2D of the
     # step's Q, K, V, the step, D2H of O
@@ -273,48 +301,37 @@ def main():
     torch.cuda.synchronize()
     if dist:
         dist.barrier()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0, e1 = ev(), ev()
     e0.record(stream)
     for i in range(args.e2e_steps):
         dq.copy_(hq, non_blocking=True)
         dk.copy_(hk, non_blocking=True)
         dv.copy_(hv, non_blocking=True)
-        s = i % w.lvsa_T_per
-        att.mask(s)
-        att.gather(dq, dk, dv)
-        att.attend(per_head=False)
-        att.scatter(out)
+        att.fused(dq, dk, dv, i % w.lvsa_T_per, out)
         ho.copy_(out, non_blocking=True)
     e1.record(stream)
     torch.cuda.synchronize()
-    e2e_ms = e0.elapsed_time(e1) / args.e2e_steps
-    if dist:
-        tt = torch.tensor([e2e_ms], device="cuda")
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        e2e_ms = float(tt[0])
+    (e2e_ms,) = max_over_ranks([e0.elapsed_time(e1) / args.e2e_steps], dist, "cuda")
     bsa.bsa_poll_status(att.plan)
-
-    # algorithmic bytes of the HBM-bound kernels (valid tokens read + written)
-    tok_bytes = w.B * w.N * w.Hh * w.D * 2
-    nnz = att.col_idx.numel()
-    algo_bytes = {"reorder_fwd": 3 * 2 * tok_bytes, "reorder_inv": 2 * tok_bytes,
-                  "lvsa_mask": 4 * (nnz + att.row_ptr.numel() + att.frame_sets.numel())}
-    kernels = {}
-    for n in names:
-        d = {"ms": kern_ms[n]}
-        if n in algo_bytes:
-            gbs = algo_bytes[n] / (kern_ms[n] * 1e-3) / 1e9
-            d.update({"algo_bytes": algo_bytes[n], "GB_s": gbs,
-                      "frac_hbm": gbs / peaks()[0]["hbm_gbs"]})
-        kernels[n] = d
 
     pk, pk_kind = peaks()
     peak = pk.get("bf16_tflops_sustained", pk["bf16_tflops"])
     attn_tflops = flops_step / (attn_ms * 1e-3) / 1e12
-    value = world * flops_step / (ms * 1e-3) / 1e12
+    tok_bytes = w.B * w.N * w.Hh * w.D * 2
+    algo_bytes = {"lvsa_mask": 4 * (att.col_idx.numel() + att.row_ptr.numel() + att.frame_sets.numel()),
+                  "reorder_fwd": 3 * 2 * tok_bytes, "reorder_inv": 2 * tok_bytes}
+    four = {}
+    for n, t in zip(names, unf_ms):
+        d = {"ms": t}
+        if n in algo_bytes:
+            gbs = algo_bytes[n] / (t * 1e-3) / 1e9
+            d.update({"algo_bytes": algo_bytes[n], "GB_s": gbs, "frac_hbm": gbs / pk["hbm_gbs"]})
+        else:
+            d["attended_tflops"] = flops_step / (t * 1e-3) / 1e12
+        four[n] = d
     line = {
         "metric": METRIC,
-        "value": value,
+        "value": weak_scaling_value(flops_step, world, ms),
         "unit": "TFLOP/s",
         "n_gpus": world,
         "steps": args.steps,
@@ -328,6 +345,7 @@ def main():
         "config": {"workload": w.name, "global_batch": w.B * world, "seq_len": w.N,
                    "heads": w.Hh, "head_dim": w.D, "lvsa_C": w.lvsa_C,
                    "lvsa_T_per": w.lvsa_T_per, "steps_s": "s = step mod T_per",
+                   "path": "bsa_lvsa_attn_fwd (one kernel, natural layout)",
                    "parallelism": f"dp{world}",
                    "l2": "inputs (1.8 GB) larger than L2; no flush"},
         "bsattn_ms_per_call": attn_ms,
@@ -335,12 +353,14 @@ def main():
         "bsattn_pct_bf16_peak": 100.0 * attn_tflops / peak,
         "attended_tflop_per_call": flops_step / 1e12,
         "roofline": {"bound": "tensor", "achieved": attn_tflops, "peak": peak,
-                     "unit": "TFLOP/s", "frac": attn_tflops / peak, "traffic": None,
+                     "unit": "TFLOP/s", "frac": attn_tflops / peak,
+                     "traffic": (STEP_KERNEL_DRAM_BYTES * w.T / 126
+                                 if STEP_KERNEL_DRAM_BYTES and args.config == 3 else None),
                      "peak_kind": f"{pk_kind} bf16 sustained (kernel timed inside a long step)"},
-        "kernels": kernels,
-        "gpu_launches": launches_per_step * args.steps,
+        "four_kernel_path": {"ms_per_step": sum(unf_ms), "kernels": four},
+        "gpu_launches": args.steps,
         "clocks": clk,
-        "e2e": {"value": world * flops_step / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+        "e2e": {"value": weak_scaling_value(flops_step, world, e2e_ms), "unit": "TFLOP/s",
                 "ms_per_step": e2e_ms,
                 "h2d_bytes_per_step": 3 * q.numel() * q.element_size(),
                 "d2h_bytes_per_step": out.numel() * out.element_size()},
