@@ -1,5 +1,5 @@
 // Device helpers shared by the attention kernels: key masks and the online
-// softmax step of one query row over one 128-key tile.
+// softmax step of one query row over one tile of keys.
 #pragma once
 
 #include <cuda_bf16.h>
@@ -56,18 +56,23 @@ struct RowState {
   float l = 0.f;
 };
 
-// One online-softmax step over a 128-key tile.  s: the row's raw scores
-// (masked keys become -inf); vm: keys allowed.  Writes P = 2^(s*sl2 - m*sl2)
-// as packed bf16 pairs, adds their sum to st.l, and returns true when the
-// row's reference max moved (then O must be multiplied by *corr).  Scaling
-// and summing use packed fp32x2 arithmetic (half the instructions).
-__device__ __forceinline__ bool softmax_tile(float (&s)[128], const uint32_t (&vm)[4], RowState& st,
-                                             float sl2, float thr, uint32_t (&pk)[64],
-                                             float& corr) {
-  const bool full = (vm[0] & vm[1] & vm[2] & vm[3]) == kFullMask;
-  if (!full) {
+// First half of an online-softmax step over NC keys (NC = 64 or 128): mask
+// the keys not allowed (vm) to -inf, take the row max and decide whether the
+// row's reference max moves (it does only when the max grows by more than
+// `thr`, so P stays below 2^(thr*sl2)).  On a move st.m and st.l are updated
+// and *corr is the factor O must be multiplied by.  *ms2 receives the packed
+// pair (-m*sl2, -m*sl2) for softmax_exp.
+template <int NC>
+__device__ __forceinline__ bool softmax_max(float (&s)[NC], const uint32_t (&vm)[NC / 32],
+                                            RowState& st, float sl2, float thr, float& corr,
+                                            uint64_t& neg_ms2) {
+  static_assert(NC == 64 || NC == 128, "column count");
+  uint32_t all = kFullMask;
 #pragma unroll
-    for (int w = 0; w < 4; ++w)
+  for (int w = 0; w < NC / 32; ++w) all &= vm[w];
+  if (all != kFullMask) {
+#pragma unroll
+    for (int w = 0; w < NC / 32; ++w)
 #pragma unroll
       for (int i = 0; i < 32; ++i)
         if (!((vm[w] >> i) & 1u)) s[w * 32 + i] = -INFINITY;
@@ -75,13 +80,16 @@ __device__ __forceinline__ bool softmax_tile(float (&s)[128], const uint32_t (&v
   // row max: 8 independent chains of 3-input max, then a small tree
   float m8[8];
 #pragma unroll
-  for (int c = 0; c < 8; ++c) m8[c] = fmax3f(s[c], s[c + 8], s[c + 16]);
+  for (int c = 0; c < 8; ++c) m8[c] = s[c];
+  constexpr int kTail = 8 + ((NC - 8) / 16) * 16;
 #pragma unroll
-  for (int i = 24; i < 120; i += 16)
+  for (int i = 8; i + 16 <= NC; i += 16)
 #pragma unroll
     for (int c = 0; c < 8; ++c) m8[c] = fmax3f(m8[c], s[i + c], s[i + 8 + c]);
+  if constexpr (kTail < NC) {
 #pragma unroll
-  for (int c = 0; c < 8; ++c) m8[c] = fmaxf(m8[c], s[120 + c]);
+    for (int c = 0; c < 8; ++c) m8[c] = fmaxf(m8[c], s[kTail + c]);
+  }
   const float mx = fmax3f(fmax3f(m8[0], m8[1], m8[2]), fmax3f(m8[3], m8[4], m8[5]),
                           fmaxf(m8[6], m8[7]));
   const float m_new = fmaxf(st.m, mx);
@@ -93,20 +101,47 @@ __device__ __forceinline__ bool softmax_tile(float (&s)[128], const uint32_t (&v
     st.l *= corr;
   }
   const float ms = (st.m == -INFINITY) ? 0.f : st.m * sl2;
-  const uint64_t scale2 = f2(sl2, sl2), neg_ms2 = f2(-ms, -ms);
-  uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};  // packed partial sums
+  neg_ms2 = f2(-ms, -ms);
+  return need;
+}
+
+// Second half, for keys [OFF, OFF + NK) of the row: P = 2^(s*sl2 - m*sl2)
+// written as packed bf16 pairs to pk[0 .. NK/2), their sum added to the
+// packed partial sums acc.  Scaling and summing use packed fp32x2
+// arithmetic (half the instructions).
+template <int OFF, int NK, int NC>
+__device__ __forceinline__ void softmax_exp(const float (&s)[NC], float sl2, uint64_t neg_ms2,
+                                            uint32_t (&pk)[NK / 2], uint64_t (&acc)[4]) {
+  const uint64_t scale2 = f2(sl2, sl2);
 #pragma unroll
-  for (int i = 0; i < 64; ++i) {
+  for (int i = 0; i < NK / 2; ++i) {
     float x0, x1;
-    unf2(ffma2(f2(s[2 * i], s[2 * i + 1]), scale2, neg_ms2), x0, x1);
+    unf2(ffma2(f2(s[OFF + 2 * i], s[OFF + 2 * i + 1]), scale2, neg_ms2), x0, x1);
     const float p0 = ex2_approx(x0), p1 = ex2_approx(x1);
     acc[i & 3] = fadd2(acc[i & 3], f2(p0, p1));
     pk[i] = pack_bf16x2(p0, p1);
   }
+}
+
+// Adds the packed partial sums to the row's running sum.
+__device__ __forceinline__ void softmax_sum(RowState& st, const uint64_t (&acc)[4]) {
   const uint64_t a = fadd2(fadd2(acc[0], acc[1]), fadd2(acc[2], acc[3]));
   float a0, a1;
   unf2(a, a0, a1);
   st.l += a0 + a1;
+}
+
+// One whole online-softmax step over NC keys: softmax_max, then P for all
+// NC keys.  Returns true when O must be multiplied by *corr.
+template <int NC>
+__device__ __forceinline__ bool softmax_tile(float (&s)[NC], const uint32_t (&vm)[NC / 32],
+                                             RowState& st, float sl2, float thr,
+                                             uint32_t (&pk)[NC / 2], float& corr) {
+  uint64_t neg_ms2;
+  const bool need = softmax_max(s, vm, st, sl2, thr, corr, neg_ms2);
+  uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};
+  softmax_exp<0, NC>(s, sl2, neg_ms2, pk, acc);
+  softmax_sum(st, acc);
   return need;
 }
 

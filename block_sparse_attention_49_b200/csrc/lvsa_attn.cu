@@ -19,12 +19,15 @@
 //    before it in the growth order; anchors in a range are counted
 //    arithmetically (they are periodic).
 //  * warp 0: TMA producer (both query tiles, then K and V of every key tile
-//    into a 2-deep ring).  warp 1: MMA issuer.  warps 4-7 / 8-11: softmax of
+//    into 2-deep rings; a K slot is refilled as soon as its last QK product
+//    is done, a V slot after its last PV product).  warp 1: MMA issuer.  warps 4-7 / 8-11: softmax of
 //    query tile 0 / 1, one row per thread, masking keys whose frame is not in
 //    the row's own A(t).
 //  * tensor memory: S0 | S1 | O0 | O1; P aliases the upper half of its S.
 //    MMA order per key tile j: PV0(j), QK0(j+1), PV1(j), QK1(j+1), so the
 //    tensor cores run one tile's products while the other tile's softmax runs.
+//    A softmax group hands P over in two 64-key halves: the PV product of the
+//    first half runs while the exponentials of the second are computed.
 // Every wait is bounded (see bounded_wait).
 #include <cuda_bf16.h>
 #include <cudaTypedefs.h>
@@ -58,7 +61,9 @@ struct LvsaCfg {
   static constexpr int kOffK = 2 * kQBytes;
   static constexpr int kOffV = kOffK + NS * kKVBytes;
   static constexpr int kOffBar = kOffV + NS * kKVBytes;
-  static constexpr int kNumBars = 1 + 3 * NS + 2 + 2 + 1;
+  // q_full, k_full[NS], v_full[NS], k_empty[NS], v_empty[NS], s_full[2],
+  // p_half[2], p_ready[2], o_final
+  static constexpr int kNumBars = 1 + 4 * NS + 2 + 2 + 2 + 1;
   static constexpr int kOffMisc = kOffBar + kNumBars * 8;
   static constexpr int kOffTiles = kOffMisc + 16;
   static constexpr int kOffSets = kOffTiles + kMaxTiles * 4;
@@ -153,9 +158,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* q_full = bars;
   uint64_t* k_full = bars + 1;
   uint64_t* v_full = k_full + Cfg::NS;
-  uint64_t* kv_empty = v_full + Cfg::NS;
-  uint64_t* s_full = kv_empty + Cfg::NS;  // [2]
-  uint64_t* p_ready = s_full + 2;         // [2]
+  uint64_t* k_empty = v_full + Cfg::NS;
+  uint64_t* v_empty = k_empty + Cfg::NS;
+  uint64_t* s_full = v_empty + Cfg::NS;   // [2]
+  uint64_t* p_half = s_full + 2;          // [2]: keys 0..63 of P stored
+  uint64_t* p_ready = p_half + 2;         // [2]: all of P stored
   uint64_t* o_final = p_ready + 2;
   uint32_t* misc = reinterpret_cast<uint32_t*>(smem + Cfg::kOffMisc);  // tmem, abort, ntiles, skip
   int32_t* tiles = reinterpret_cast<int32_t*>(smem + Cfg::kOffTiles);  // (k0 << 7) | (count - 1)
@@ -178,10 +185,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int i = 0; i < Cfg::NS; ++i) {
       mbar_init(&k_full[i], 1);
       mbar_init(&v_full[i], 1);
-      mbar_init(&kv_empty[i], 1);
+      mbar_init(&k_empty[i], 1);
+      mbar_init(&v_empty[i], 1);
     }
     mbar_init(&s_full[0], 1);
     mbar_init(&s_full[1], 1);
+    mbar_init(&p_half[0], 128);
+    mbar_init(&p_half[1], 128);
     mbar_init(&p_ready[0], 128);
     mbar_init(&p_ready[1], 128);
     mbar_init(o_final, 1);
@@ -241,8 +251,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tbase = misc[0];
   const int n = (int)misc[2];
 
+  // register split: 128 threads x 72 + 256 threads x 216 = 64512, the 384 x
+  // 168 registers the block is launched with (fewer for the issuing warps
+  // made them spill, and each reload delayed an MMA batch)
   if (warp < 4) {
-    asm volatile("setmaxnreg.dec.sync.aligned.u32 56;");
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 72;");
     if (warp == 0 && n > 0) {
       // -------------------------------------------------------- TMA producer
       // the whole warp runs the loop (warp-uniform operands); one lane issues
@@ -254,34 +267,40 @@ __global__ void __launch_bounds__(kThreads, 1)
                         (int)(brow + q0 + g * kTile));
       }
       __syncwarp();
-      int issued = 0;
+      int issued_k = 0, issued_v = 0;
       for (int j = 0; j < n; ++j) {
         const int st = j % Cfg::NS;
-        if (!__all_sync(kFullMask, bounded_wait(&kv_empty[st], ((j / Cfg::NS) & 1) ^ 1, wc))) break;
+        const uint32_t par = ((j / Cfg::NS) & 1) ^ 1;
         const int krow = (int)(brow + (tiles[j] >> 7));
+        if (!__all_sync(kFullMask, bounded_wait(&k_empty[st], par, wc))) break;
         if (elect_one()) {
           uint8_t* sK = smem + Cfg::kOffK + st * Cfg::kKVBytes;
-          uint8_t* sV = smem + Cfg::kOffV + st * Cfg::kKVBytes;
           mbar_arrive_expect_tx(&k_full[st], Cfg::kKVBytes);
           for (int c = 0; c < Cfg::kChunks; ++c)
             tma_load_3d(sK + c * Cfg::kPanel, &tmk, &k_full[st], c * 64, h, krow);
+        }
+        __syncwarp();
+        issued_k = j + 1;
+        if (!__all_sync(kFullMask, bounded_wait(&v_empty[st], par, wc))) break;
+        if (elect_one()) {
+          uint8_t* sV = smem + Cfg::kOffV + st * Cfg::kKVBytes;
           mbar_arrive_expect_tx(&v_full[st], Cfg::kKVBytes);
           for (int c = 0; c < Cfg::kChunks; ++c)
             tma_load_3d(sV + c * Cfg::kPanel, &tmv, &v_full[st], c * 64, h, krow);
         }
         __syncwarp();
-        issued = j + 1;
+        issued_v = j + 1;
       }
       if (*wc.abort) {
         // leave no copy in flight: wait (bounded, ignoring the abort flag)
-        // for the loads still owned by the ring
+        // for the loads still owned by the rings
         volatile int no_abort = 0;
         const WaitCtx drain{p.status, &no_abort, p.wait_limit_ns};
         bounded_wait(q_full, 0, drain);
-        for (int j = max(0, issued - Cfg::NS); j < issued; ++j) {
+        for (int j = max(0, issued_k - Cfg::NS); j < issued_k; ++j)
           bounded_wait(&k_full[j % Cfg::NS], (j / Cfg::NS) & 1, drain);
+        for (int j = max(0, issued_v - Cfg::NS); j < issued_v; ++j)
           bounded_wait(&v_full[j % Cfg::NS], (j / Cfg::NS) & 1, drain);
-        }
       }
       __syncwarp();
     } else if (warp == 1 && n > 0) {
@@ -290,30 +309,34 @@ __global__ void __launch_bounds__(kThreads, 1)
       // elected lane issues the tcgen05 instructions
       constexpr uint32_t idesc_qk = idesc_bf16(128, 128, 0);
       constexpr uint32_t idesc_pv = idesc_bf16(128, D, 1);
-      const uint64_t qd0 = sdesc_sw128(smem_u32(sQ), 16, 1024);
-      const uint64_t kd0 = sdesc_sw128(smem_u32(smem + Cfg::kOffK), 16, 1024);
-      const uint64_t vd0 = sdesc_sw128(smem_u32(smem + Cfg::kOffV), Cfg::kPanel, 1024);
+      // shared-memory descriptors: constant high word, 32-bit low words
+      constexpr uint32_t dhi = sdesc_sw128_hi(1024);
+      const uint32_t q_lo = sdesc_sw128_lo(smem_u32(sQ), 16);
+      const uint32_t k_lo = sdesc_sw128_lo(smem_u32(smem + Cfg::kOffK), 16);
+      const uint32_t v_lo = sdesc_sw128_lo(smem_u32(smem + Cfg::kOffV), Cfg::kPanel);
       auto issue_qk = [&](int g, int st) {
         const uint32_t dst = tbase + g * 128;
-        const uint64_t qd = sdesc_add(qd0, g * Cfg::kQBytes);
-        const uint64_t kd = sdesc_add(kd0, st * Cfg::kKVBytes);
+        const uint32_t qd = q_lo + ((g * Cfg::kQBytes) >> 4);
+        const uint32_t kd = k_lo + ((st * Cfg::kKVBytes) >> 4);
         if (elect_one()) {
 #pragma unroll
           for (int kk = 0; kk < D / 16; ++kk) {
-            const uint32_t off = (kk >> 2) * Cfg::kPanel + (kk & 3) * 32;
-            mma_ss(dst, sdesc_add(qd, off), sdesc_add(kd, off), idesc_qk, kk > 0);
+            const uint32_t off = ((kk >> 2) * Cfg::kPanel + (kk & 3) * 32) >> 4;
+            mma_ss(dst, sdesc_join(dhi, qd + off), sdesc_join(dhi, kd + off), idesc_qk, kk > 0);
           }
           mma_commit(&s_full[g]);
         }
         __syncwarp();
       };
-      auto issue_pv = [&](int g, int st, uint32_t acc) {
-        const uint32_t dst = tbase + 256 + g * 128, pa = tbase + g * 128 + 64;
-        const uint64_t vd = sdesc_add(vd0, st * Cfg::kKVBytes);
+      // O_g += P(keys 64 * half .. + 63) . V(same keys)
+      auto issue_pv = [&](int g, int st, int half, uint32_t acc) {
+        const uint32_t dst = tbase + 256 + g * 128, pa = tbase + g * 128 + 64 + half * 32;
+        const uint32_t vd = v_lo + ((st * Cfg::kKVBytes + half * 8192) >> 4);
         if (elect_one()) {
 #pragma unroll
-          for (int kk = 0; kk < kTile / 16; ++kk)
-            mma_ts(dst, pa + kk * 8, sdesc_add(vd, kk * 2048), idesc_pv, (acc | (uint32_t)kk) != 0);
+          for (int kk = 0; kk < 4; ++kk)
+            mma_ts(dst, pa + kk * 8, sdesc_join(dhi, vd + kk * (2048 >> 4)), idesc_pv,
+                   (acc | (uint32_t)half | (uint32_t)kk) != 0);
         }
         __syncwarp();
       };
@@ -329,22 +352,32 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_after();
         issue_qk(0, 0);
         issue_qk(1, 0);
+        commit(&k_empty[0]);
       }
       for (int j = 0; alive && j < n; ++j) {
         const int st = j % Cfg::NS, st1 = (j + 1) % Cfg::NS;
-        if (!wait(&p_ready[0], j & 1) || !wait(&v_full[st], (j / Cfg::NS) & 1)) break;
+        if (!wait(&p_half[0], j & 1) || !wait(&v_full[st], (j / Cfg::NS) & 1)) break;
         tc_fence_after();
-        issue_pv(0, st, j > 0);
+        issue_pv(0, st, 0, j > 0);
+        if (!wait(&p_ready[0], j & 1)) break;
+        tc_fence_after();
+        issue_pv(0, st, 1, 1);
         if (j + 1 < n) {
           if (!wait(&k_full[st1], ((j + 1) / Cfg::NS) & 1)) break;
           tc_fence_after();
           issue_qk(0, st1);
         }
+        if (!wait(&p_half[1], j & 1)) break;
+        tc_fence_after();
+        issue_pv(1, st, 0, j > 0);
         if (!wait(&p_ready[1], j & 1)) break;
         tc_fence_after();
-        issue_pv(1, st, j > 0);
-        commit(&kv_empty[st]);
-        if (j + 1 < n) issue_qk(1, st1);
+        issue_pv(1, st, 1, 1);
+        commit(&v_empty[st]);
+        if (j + 1 < n) {
+          issue_qk(1, st1);
+          commit(&k_empty[st1]);
+        }
       }
       commit(o_final);
     }
@@ -354,7 +387,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       tmem_dealloc(tbase, Cfg::kTmemCols);
     }
   } else {
-    asm volatile("setmaxnreg.inc.sync.aligned.u32 224;");
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 216;");
     // ---------------------------------------------------------- softmax
     const int g = (warp >= 8) ? 1 : 0;
     const int q4 = warp & 3;
@@ -397,13 +430,25 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int i = 0; i < 128; ++i) s[i] = __uint_as_float(r128[i]);
       }
-      uint32_t pk[64];
       float corr;
-      const bool need = softmax_tile(s, vm, st, sl2, thr, pk, corr);
+      uint64_t neg_ms2;
+      const bool need = softmax_max(s, vm, st, sl2, thr, corr, neg_ms2);
       // S of tile j was written after PV of tile j-1: O is complete here
       if (j > 0 && __any_sync(kFullMask, need)) tmem_scale<D>(tO, corr);
-      tmem_st32(tS + 64, *reinterpret_cast<uint32_t(*)[32]>(&pk[0]));
-      tmem_st32(tS + 96, *reinterpret_cast<uint32_t(*)[32]>(&pk[32]));
+      uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};
+      {
+        uint32_t pk[32];
+        softmax_exp<0, 64>(s, sl2, neg_ms2, pk, acc);
+        tmem_st32(tS + 64, pk);
+      }
+      tc_fence_before();
+      mbar_arrive(&p_half[g]);
+      {
+        uint32_t pk[32];
+        softmax_exp<64, 64>(s, sl2, neg_ms2, pk, acc);
+        tmem_st32(tS + 96, pk);
+      }
+      softmax_sum(st, acc);
       tc_fence_before();
       mbar_arrive(&p_ready[g]);
     }
