@@ -20,11 +20,15 @@ All floating point is fp64.  bf16 inputs convert to fp64 exactly.
 
 Readings of points the pages leave open (each listed in the design notes):
 * window extension order: offsets +1, -1, +2, -2, ... around t, skipping
-  frames outside [0,T) and frames already in the set, until |A(t)| = C;
-* anchors G_s = {f : (f - s) mod T_per == 0};
+  frames outside [0,T) and frames already in the set, until |A(t)| = C
+  (reading A, the default); reading B, alternating right and left pointers,
+  is available as order="alternate";
+* anchors G_s = {f : (f - s) mod T_per == 0}; the fixed-grid and window-only
+  variants take {f : f mod T_per == 0} and the empty set;
 * draft pooling averages the valid tokens of a tile only (grid-edge tiles are
   partially filled); sums run sequentially in row-major (a, then b) order and
-  the mean is one IEEE division;
+  the mean is one IEEE division; max pooling takes the maximum over the same
+  tokens;
 * draft logits are a sequential multiply-then-add chain over the channels,
   each operation rounded to fp64 (no fused multiply-add);
 * top-k per query-block row keeps k = ceil(Nb*(100-p)/100) blocks ranked by
@@ -46,42 +50,81 @@ import numpy as np
 # ---------------------------------------------------------------------------
 
 
-def lvsa_anchors(T: int, T_per: int, s: int) -> list[int]:
-    """Rotating global anchors G_s at denoising step s.
+ANCHOR_MODES = ("rotating", "fixed", "none")
+WINDOW_ORDERS = ("distance", "alternate")
 
-    The anchor grid has period T_per and is shifted by s mod T_per, so that
-    over T_per consecutive steps every frame is an anchor exactly once
-    (LVSA, section 2, "Rotating global anchors").
+
+def lvsa_anchors(T: int, T_per: int, s: int, anchors: str = "rotating") -> list[int]:
+    """Global anchor frames at denoising step s.
+
+    "rotating" (LVSA, section 2, "Rotating global anchors"): the grid of
+    period T_per is shifted by s mod T_per, so over T_per consecutive steps
+    every frame is an anchor exactly once.  "fixed": the fixed-grid global
+    frames the same section contrasts it with, {f : f mod T_per == 0} at every
+    step.  "none": no global frames, the sliding-window pattern the page's
+    introduction lists among earlier approaches.
     """
-    return [f for f in range(T) if (f - s) % T_per == 0]
+    if anchors == "rotating":
+        return [f for f in range(T) if (f - s) % T_per == 0]
+    if anchors == "fixed":
+        return [f for f in range(T) if f % T_per == 0]
+    if anchors == "none":
+        return []
+    raise ValueError(f"unknown anchor mode {anchors!r}")
 
 
-def lvsa_frame_set(t: int, T: int, C: int, T_per: int, s: int) -> list[int]:
+def lvsa_frame_set(t: int, T: int, C: int, T_per: int, s: int, anchors: str = "rotating",
+                   order: str = "distance") -> list[int]:
     """A(t) = G_s U W(t) for query frame t, with |A(t)| = C exactly.
 
     W(t) is a local window centred on t that grows past anchors it overlaps so
     that the budget C is always met (LVSA, section 2, "Extended adaptive
-    window").  Growth order: t+1, t-1, t+2, t-2, ...; frames outside [0, T)
-    and frames already in the set are skipped and cost no budget.
+    window").  The page does not fix the growth order; two readings:
+
+    * "distance": t+1, t-1, t+2, t-2, ...; frames outside [0, T) and frames
+      already in the set are skipped and cost no budget;
+    * "alternate": a right pointer and a left pointer take turns, right
+      first; each turn moves its pointer past frames already in the set and
+      adds the next frame on its side; a side that runs off the grid stops
+      and the other side continues.
     """
-    if not (0 <= t < T) or T_per <= 0 or C > T:
+    if not (0 <= t < T) or C > T or (anchors != "none" and T_per <= 0):
         raise ValueError("bad LVSA arguments")
-    A = set(lvsa_anchors(T, T_per, s))
+    if order not in WINDOW_ORDERS:
+        raise ValueError(f"unknown window order {order!r}")
+    A = set(lvsa_anchors(T, T_per, s, anchors))
     A.add(t)
     if len(A) > C:
         raise ValueError("budget C smaller than anchors + own frame")
-    d = 1
-    while len(A) < C:
-        for f in (t + d, t - d):
-            if len(A) < C and 0 <= f < T and f not in A:
-                A.add(f)
-        d += 1
+    if order == "distance":
+        d = 1
+        while len(A) < C:
+            for f in (t + d, t - d):
+                if len(A) < C and 0 <= f < T and f not in A:
+                    A.add(f)
+            d += 1
+    else:
+        r, l = t + 1, t - 1
+        while len(A) < C:
+            while r < T and r in A:
+                r += 1
+            if r < T:
+                A.add(r)
+                r += 1
+            if len(A) == C:
+                break
+            while l >= 0 and l in A:
+                l -= 1
+            if l >= 0:
+                A.add(l)
+                l -= 1
     return sorted(A)
 
 
-def lvsa_frame_sets(T: int, C: int, T_per: int, s: int) -> np.ndarray:
+def lvsa_frame_sets(T: int, C: int, T_per: int, s: int, anchors: str = "rotating",
+                    order: str = "distance") -> np.ndarray:
     """int32 [T, C]: row t is A(t) in ascending order."""
-    return np.array([lvsa_frame_set(t, T, C, T_per, s) for t in range(T)],
+    return np.array([lvsa_frame_set(t, T, C, T_per, s, anchors, order) for t in range(T)],
                     dtype=np.int32).reshape(T, C)
 
 
@@ -191,18 +234,27 @@ def draft_keep_count(Nb: int, sparsity_pct: int) -> int:
     return (Nb * (100 - sparsity_pct) + 99) // 100
 
 
-def draft_pool(x_nat: np.ndarray, T: int, H: int, W: int, ph: int, pw: int) -> np.ndarray:
-    """Average pooling of Q or K over ph x pw tiles of each frame.
+def draft_pool(x_nat: np.ndarray, T: int, H: int, W: int, ph: int, pw: int,
+               mode: str = "mean") -> np.ndarray:
+    """Pooling of Q or K over ph x pw tiles of each frame.
+
+    "mean" (the article's average pooling): only tokens inside the grid
+    count; the sum runs over them in row-major (a, then b) order and is
+    divided once by their count.  "max" (the max pooling the article's
+    authors tried first, before preferring the average at high sparsity):
+    the channel-wise maximum over the same tokens, exact in any order.
 
     x_nat: [B, N, Hh, D] (any float dtype; converted exactly to fp64).
     Returns fp64 [B, Hh, Nb, D], Nb = T*ceil(H/ph)*ceil(W/pw), block index
-    (t*TH + i)*TW + j.  Only tokens inside the grid count; the sum runs over
-    them in row-major (a, then b) order and is divided once by their count.
+    (t*TH + i)*TW + j.
     """
+    if mode not in ("mean", "max"):
+        raise ValueError(f"unknown pooling {mode!r}")
     B, N, Hh, D = x_nat.shape
     TH, TW = -(-H // ph), -(-W // pw)
     x = np.asarray(x_nat, dtype=np.float64).reshape(B, T, H, W, Hh, D)
-    acc = np.zeros((B, T, TH, TW, Hh, D), dtype=np.float64)
+    init = 0.0 if mode == "mean" else -np.inf
+    acc = np.full((B, T, TH, TW, Hh, D), init, dtype=np.float64)
     cnt = np.zeros((TH, TW), dtype=np.int64)
     for a in range(ph):
         for b in range(pw):
@@ -214,12 +266,15 @@ def draft_pool(x_nat: np.ndarray, T: int, H: int, W: int, ph: int, pw: int) -> n
                     xx = j * pw + b
                     if xx >= W:
                         continue
-                    acc[:, :, i, j] = acc[:, :, i, j] + x[:, :, y, xx]
+                    if mode == "mean":
+                        acc[:, :, i, j] = acc[:, :, i, j] + x[:, :, y, xx]
+                    else:
+                        acc[:, :, i, j] = np.maximum(acc[:, :, i, j], x[:, :, y, xx])
                     cnt[i, j] += 1
-    mean = acc / cnt[None, None, :, :, None, None].astype(np.float64)
+    pooled = acc / cnt[None, None, :, :, None, None].astype(np.float64) if mode == "mean" else acc
     # [B, T, TH, TW, Hh, D] -> [B, Hh, Nb, D]
     return np.ascontiguousarray(
-        np.transpose(mean, (0, 4, 1, 2, 3, 5)).reshape(B, Hh, T * TH * TW, D))
+        np.transpose(pooled, (0, 4, 1, 2, 3, 5)).reshape(B, Hh, T * TH * TW, D))
 
 
 def draft_logits(qbar: np.ndarray, kbar: np.ndarray) -> np.ndarray:
@@ -261,10 +316,10 @@ def draft_topk(logits: np.ndarray, k: int) -> np.ndarray:
     return out.reshape(*lead, Nq, k)
 
 
-def draft_blocks(q_nat, k_nat, T, H, W, ph, pw, sparsity_pct):
+def draft_blocks(q_nat, k_nat, T, H, W, ph, pw, sparsity_pct, mode: str = "mean"):
     """Full draft-mask pipeline: pool -> logits -> top-k.  int32 [B,Hh,Nb,k]."""
-    qbar = draft_pool(q_nat, T, H, W, ph, pw)
-    kbar = draft_pool(k_nat, T, H, W, ph, pw)
+    qbar = draft_pool(q_nat, T, H, W, ph, pw, mode)
+    kbar = draft_pool(k_nat, T, H, W, ph, pw, mode)
     L = draft_logits(qbar, kbar)
     return draft_topk(L, draft_keep_count(L.shape[-1], sparsity_pct))
 

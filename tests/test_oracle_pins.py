@@ -436,3 +436,109 @@ def test_output_does_not_depend_on_layout():
                                        valid, blk, rp, ci, False, 0.35)
         outs.append(oracle.reorder_inv(O, perm))
     np.testing.assert_allclose(outs[0], outs[1], rtol=1e-13, atol=1e-14)
+
+
+# ---------------------------------------------------------------------------
+# Mask variants: fixed-grid anchors and the sliding window (LVSA, section 2:
+# the fixed grid that rotating anchors replace; the introduction's sliding
+# window), window growth reading B, max pooling (Draft Attention article: the
+# max pooling tried before average pooling)
+# ---------------------------------------------------------------------------
+
+
+def test_fixed_grid_anchors_do_not_move_with_the_step():
+    for T, C, T_per in LVSA_CFGS:
+        G = [f for f in range(0, T, T_per)]          # every T_per-th frame from 0
+        for s in range(T_per):
+            assert oracle.lvsa_anchors(T, T_per, s, "fixed") == G
+        A0 = oracle.lvsa_frame_sets(T, C, T_per, 0, anchors="fixed")
+        for s in (1, T_per - 1):
+            assert (oracle.lvsa_frame_sets(T, C, T_per, s, anchors="fixed") == A0).all()
+
+
+@pytest.mark.parametrize("order", ["distance", "alternate"])
+def test_window_only_is_a_clamped_interval(order):
+    # with no anchors the C frames nearest t (ties to the right) are the
+    # interval [lo, lo + C - 1], lo = t - floor((C - 1) / 2) clamped into
+    # [0, T - C]; both growth orders give it (the sides alternate either way)
+    for T in range(1, 14):
+        for C in range(1, T + 1):
+            for t in range(T):
+                lo = min(max(t - (C - 1) // 2, 0), T - C)
+                got = oracle.lvsa_frame_set(t, T, C, 1, 0, anchors="none", order=order)
+                assert got == list(range(lo, lo + C)), (T, C, t)
+
+
+def test_alternate_order_hand_case():
+    # T = 8, C = 4, T_per = 4, s = 0, t = 3: G = {0, 4}, one frame to add.
+    # distance order tries +1 = 4 (already there), then -1 = 2;
+    # alternate order moves the right pointer past 4 and takes 5.
+    assert oracle.lvsa_frame_set(3, 8, 4, 4, 0) == [0, 2, 3, 4]
+    assert oracle.lvsa_frame_set(3, 8, 4, 4, 0, order="alternate") == [0, 3, 4, 5]
+
+
+def test_alternate_order_closed_form():
+    # reading B as a count: with need = C - |G U {t}| frames to add and nR / nL
+    # frames outside G U {t} right / left of t, the right side takes
+    # kR = min(nR, max(ceil(need/2), need - nL)) of its nearest frames and the
+    # left side the remaining need - kR of its own
+    for T in range(1, 13):
+        for T_per in range(1, T + 2):
+            for s in range(T_per):
+                for anchors in ("rotating", "none"):
+                    G = set(oracle.lvsa_anchors(T, T_per, s, anchors))
+                    for t in range(T):
+                        base = G | {t}
+                        right = [f for f in range(t + 1, T) if f not in base]
+                        left = [f for f in range(t - 1, -1, -1) if f not in base]
+                        for C in range(len(base), T + 1):
+                            need = C - len(base)
+                            kR = min(len(right), max((need + 1) // 2, need - len(left)))
+                            want = sorted(base | set(right[:kR]) | set(left[:need - kR]))
+                            got = oracle.lvsa_frame_set(t, T, C, T_per, s, anchors, "alternate")
+                            assert got == want, (T, T_per, s, t, C, anchors)
+
+
+@pytest.mark.parametrize("anchors", ["fixed", "none"])
+def test_variant_invariants(anchors):
+    for T, C, T_per in LVSA_CFGS:
+        for s in (0, 1):
+            G = set(oracle.lvsa_anchors(T, T_per, s, anchors))
+            for order in ("distance", "alternate"):
+                A = oracle.lvsa_frame_sets(T, C, T_per, s, anchors, order)
+                for t in range(T):
+                    row = list(A[t])
+                    assert row == sorted(set(row)) and len(row) == C
+                    assert G <= set(row) and t in row
+
+
+def test_max_pool_closed_forms():
+    T, H, W, ph, pw = 1, 30, 52, 8, 16
+    # constant: the constant; ramp: the largest coordinate inside the grid
+    x = np.full((1, T * H * W, 1, 3), -2.25)
+    assert (oracle.draft_pool(x, T, H, W, ph, pw, "max") == -2.25).all()
+    yy, xx = np.meshgrid(np.arange(H), np.arange(W), indexing="ij")
+    r = np.stack([yy, xx], -1).reshape(1, H * W, 1, 2).astype(np.float64)
+    p = oracle.draft_pool(r, T, H, W, ph, pw, "max")[0, 0]
+    for i in range(4):
+        for j in range(4):
+            assert p[i * 4 + j, 0] == min(H, (i + 1) * ph) - 1
+            assert p[i * 4 + j, 1] == min(W, (j + 1) * pw) - 1
+
+
+def test_max_pool_brute_force_and_bounds_mean():
+    w = small_workload(CONFIGS[2], T=2, Hh=2, D=8, field_grid=(2, 4, 7))
+    q, _, _ = make_qkv(w)
+    x = q.float().numpy().astype(np.float64)
+    mx = oracle.draft_pool(x, w.T, w.H, w.W, 8, 16, "max")
+    mean = oracle.draft_pool(x, w.T, w.H, w.W, 8, 16, "mean")
+    assert (mx >= mean).all()
+    xr = x.reshape(1, w.T, w.H, w.W, w.Hh, w.D)
+    for t in range(w.T):
+        for i in range(4):
+            for j in range(4):
+                tile = xr[0, t, i * 8:(i + 1) * 8, j * 16:(j + 1) * 16]
+                for h in range(w.Hh):
+                    for c in range(w.D):
+                        vals = sorted(tile[:, :, h, c].reshape(-1).tolist())
+                        assert mx[0, h, (t * 4 + i) * 4 + j, c] == vals[-1]
