@@ -10,6 +10,7 @@ attn_fwd on the block list -> reorder_inv) is timed too and reported per
 kernel.  Inputs (1.8 GB) exceed the 126 MB L2, so no flush is needed.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+    python bench.py --kernel-table      # every kernel on every workload, one JSON line each
 
 Under torchrun (N > 1) every rank runs its own batch (the path shards over
 batch x heads with no data exchange): weak scaling, max time over ranks.
@@ -199,6 +200,121 @@ def run_reference(args, rank, world):
     print(json.dumps(line), flush=True)
 
 
+def draft_attended_flops(w, kv_idx_host: np.ndarray, keep: int) -> float:
+    """4*D flops per (valid query, valid key) pair of every kept block pair.
+    Blocks are the ph x pw tiles of the tile layout, in (t, i, j) order."""
+    ph, pw = w.draft_ph, w.draft_pw
+    TH, TW = -(-w.H // ph), -(-w.W // pw)
+    vi = np.minimum(ph, w.H - np.arange(TH) * ph)
+    vj = np.minimum(pw, w.W - np.arange(TW) * pw)
+    nv = np.tile(np.outer(vi, vj).ravel(), w.T).astype(np.int64)
+    nb = nv.size
+    idx = kv_idx_host.reshape(-1, nb, keep)
+    pairs = int((nv[None, :, None] * nv[idx]).sum())
+    return 4.0 * w.D * pairs
+
+
+def kernel_table(args):
+    """ms per call of every kernel of both paths on every workload, with the
+    algorithmic bytes (HBM-bound kernels) or attended flops (attention).  L2
+    is flushed (a 256 MB write) before every timed call."""
+    import block_sparse_attention_49_b200 as bsa
+    from block_sparse_attention_49_b200.pipeline import DraftAttention, LvsaAttention
+
+    pk, pk_kind = peaks()
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+    stream = torch.cuda.current_stream()
+
+    def timed(fn, reps=args.table_reps):
+        for _ in range(3):
+            fn()
+        ts = []
+        for _ in range(reps):
+            flush.zero_()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            fn()
+            e1.record(stream)
+            torch.cuda.synchronize()
+            ts.append(e0.elapsed_time(e1))
+        return statistics.median(ts)
+
+    def emit(cid, kernel, ms, algo_bytes=None, flops=None, note=None):
+        d = {"config": cid, "workload": CONFIGS[cid].name, "kernel": kernel, "ms": round(ms, 4)}
+        if algo_bytes is not None:
+            gbs = algo_bytes / (ms * 1e-3) / 1e9
+            d.update({"algo_bytes": int(algo_bytes), "GB_s": round(gbs, 1),
+                      "frac_hbm": round(gbs / pk["hbm_gbs"], 3)})
+        if flops is not None:
+            tf = flops / (ms * 1e-3) / 1e12
+            d.update({"attended_tflop": round(flops / 1e12, 4), "TFLOP_s": round(tf, 1),
+                      "frac_bf16_burst": round(tf / pk["bf16_tflops"], 3)})
+        if note:
+            d["note"] = note
+        print(json.dumps(d), flush=True)
+
+    for cid in sorted(CONFIGS):
+        w = CONFIGS[cid]
+        q, k, v = make_qkv(w, device="cuda")
+        out = torch.empty_like(q)
+        tok_bytes = w.B * w.N * w.Hh * w.D * 2
+        scale = 1.0 / math.sqrt(w.D)
+        if w.lvsa_C:
+            blk = w.lvsa_block or 128
+            att = LvsaAttention(w.B, w.Hh, w.D, w.T, w.H, w.W, w.lvsa_C, w.lvsa_T_per, block=blk)
+            ms = timed(lambda: att.mask(0))
+            emit(cid, "lvsa_mask", ms, 4 * (att.col_idx.numel() + att.row_ptr.numel() +
+                                            att.frame_sets.numel()),
+                 note="launch-latency bound: output is a few MB")
+            emit(cid, "reorder_fwd (frame layout, Q K V)", timed(lambda: att.gather(q, k, v)),
+                 3 * 2 * tok_bytes)
+            flops = attended_flops(w)
+            emit(cid, f"attn_fwd (LVSA block list, {blk}-token blocks)",
+                 timed(lambda: att.attend(per_head=False)), flops=flops)
+            emit(cid, "reorder_inv (frame layout, O)", timed(lambda: att.scatter(out)),
+                 2 * tok_bytes)
+            fused = att if blk == 128 else LvsaAttention(w.B, w.Hh, w.D, w.T, w.H, w.W,
+                                                         w.lvsa_C, w.lvsa_T_per, block=128)
+            emit(cid, "lvsa_attn_fwd (fused, natural layout)",
+                 timed(lambda: fused.fused(q, k, v, 0, out)), flops=flops)
+            bsa.bsa_poll_status(att.plan)
+            del att, fused
+        if w.dense:
+            plan = bsa.Plan(w.B, w.Hh, w.D, w.T, w.H, w.W, bsa.LAYOUT_FRAME, block=w.dense_block)
+            nb = plan.nblocks
+            rp = torch.arange(0, nb + 1, dtype=torch.int32, device="cuda") * nb
+            ci = torch.arange(nb, dtype=torch.int32, device="cuda").repeat(nb)
+            shape = (w.B, w.Hh, plan.Npad, w.D)
+            qs, ks, vs, os_ = (torch.empty(shape, dtype=torch.bfloat16, device="cuda")
+                               for _ in range(4))
+            bsa.bsa_reorder_fwd(plan, q, qs, k, ks, v, vs)
+            emit(cid, "attn_fwd (dense block list)",
+                 timed(lambda: bsa.bsa_attn_fwd(plan, qs, ks, vs, rp, ci, False, scale, os_, None)),
+                 flops=4.0 * w.D * w.N * w.N * w.Hh * w.B)
+            bsa.bsa_poll_status(plan)
+            del qs, ks, vs, os_, plan
+        if w.draft_ph:
+            att = DraftAttention(w.B, w.Hh, w.D, w.T, w.H, w.W, w.draft_ph, w.draft_pw,
+                                 w.draft_sparsity)
+            emit(cid, "reorder_fwd (tile layout, Q K V)", timed(lambda: att.gather(q, k, v)),
+                 3 * 2 * tok_bytes)
+            nb = att.plan.nblocks
+            pooled = 2 * w.B * w.Hh * nb * w.D * 8
+            emit(cid, "draft_mask (pool + score/top-k)", timed(att.mask),
+                 2 * tok_bytes + 2 * pooled + 4 * att.col_idx.numel(),
+                 note=f"k = {att.keep} of {nb} blocks per row")
+            kv_host = att.col_idx.cpu().numpy()
+            emit(cid, "attn_fwd (draft, per-head block lists)",
+                 timed(lambda: att.attend(per_head=True)),
+                 flops=draft_attended_flops(w, kv_host, att.keep))
+            emit(cid, "reorder_inv (tile layout, O)", timed(lambda: att.scatter(out)),
+                 2 * tok_bytes)
+            bsa.bsa_poll_status(att.plan)
+            del att
+        del q, k, v, out
+        torch.cuda.empty_cache()
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -212,7 +328,14 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--frames", type=int, default=0,
                     help="use only the first T frames (small profiling case of the same kernels)")
+    ap.add_argument("--kernel-table", action="store_true",
+                    help="time every kernel on every workload instead of the step")
+    ap.add_argument("--table-reps", type=int, default=10)
     args = ap.parse_args()
+    if args.kernel_table:
+        torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", 0)))
+        kernel_table(args)
+        return
 
     rank = int(os.environ.get("RANK", 0))
     world = int(os.environ.get("WORLD_SIZE", 1))

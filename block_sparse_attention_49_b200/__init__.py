@@ -19,7 +19,10 @@ from typing import Optional
 
 __all__ = [
     "BsaError", "Plan", "LAYOUT_FRAME", "LAYOUT_TILE", "lib_path", "load",
-    "bsa_plan_create", "bsa_plan_destroy", "bsa_padded_tokens", "bsa_num_blocks",
+    "ANCHORS_ROTATING", "ANCHORS_FIXED", "ANCHORS_NONE", "WINDOW_DISTANCE", "WINDOW_ALTERNATE",
+    "POOL_MEAN", "POOL_MAX",
+    "bsa_plan_create", "bsa_plan_destroy", "bsa_plan_set_lvsa_variant",
+    "bsa_plan_set_draft_pooling", "bsa_padded_tokens", "bsa_num_blocks",
     "bsa_block_size", "bsa_lvsa_mask", "bsa_lvsa_nnz", "bsa_draft_keep_count",
     "bsa_draft_workspace_bytes", "bsa_draft_mask", "bsa_draft_mask_noalloc",
     "bsa_draft_noalloc_max_scratch_bytes", "bsa_reorder_fwd", "bsa_reorder_inv",
@@ -29,6 +32,9 @@ __all__ = [
 
 LAYOUT_FRAME = 0
 LAYOUT_TILE = 1
+ANCHORS_ROTATING, ANCHORS_FIXED, ANCHORS_NONE = 0, 1, 2
+WINDOW_DISTANCE, WINDOW_ALTERNATE = 0, 1
+POOL_MEAN, POOL_MAX = 0, 1
 
 STATUS = {0: "BSA_OK", 1: "BSA_ERR_INVALID_ARG", 2: "BSA_ERR_UNSUPPORTED",
           3: "BSA_ERR_ALIGNMENT", 4: "BSA_ERR_CUDA", 5: "BSA_ERR_TIMEOUT",
@@ -44,6 +50,8 @@ _c_int, _c_i64, _c_sz, _c_p, _c_u64 = (ctypes.c_int, ctypes.c_int64, ctypes.c_si
 _SIGS = {
     "bsa_plan_create": (_c_int, [ctypes.POINTER(_c_p)] + [_c_int] * 10),
     "bsa_plan_destroy": (_c_int, [_c_p]),
+    "bsa_plan_set_lvsa_variant": (_c_int, [_c_p, _c_int, _c_int]),
+    "bsa_plan_set_draft_pooling": (_c_int, [_c_p, _c_int]),
     "bsa_padded_tokens": (_c_i64, [_c_p]),
     "bsa_num_blocks": (_c_i64, [_c_p]),
     "bsa_block_size": (_c_int, [_c_p]),
@@ -228,6 +236,16 @@ def bsa_lvsa_attn_fwd(plan: Plan, C: int, T_per: int, s: int, q, k, v, scale: fl
 
 def bsa_poll_status(plan: Plan, stream=None):
     _check(load().bsa_poll_status(plan.handle, _stream(stream)), "bsa_poll_status")
+
+
+def bsa_plan_set_lvsa_variant(plan: Plan, anchors: int, window_order: int):
+    _check(load().bsa_plan_set_lvsa_variant(plan.handle, int(anchors), int(window_order)),
+           "bsa_plan_set_lvsa_variant")
+
+
+def bsa_plan_set_draft_pooling(plan: Plan, pooling: int):
+    _check(load().bsa_plan_set_draft_pooling(plan.handle, int(pooling)),
+           "bsa_plan_set_draft_pooling")
 
 
 def bsa_set_wait_limit_ns(plan: Plan, ns: int):

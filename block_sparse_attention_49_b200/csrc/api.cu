@@ -10,6 +10,21 @@
 
 namespace bsa {
 
+int lvsa_effective_anchors(const bsa_plan_s* plan, int T_per, int s, int* T_per_eff, int* s_eff) {
+  const int T = plan->g.T;
+  if (plan->lvsa_anchors == BSA_ANCHORS_NONE) {
+    *T_per_eff = 0;
+    *s_eff = 0;
+    return 0;
+  }
+  *T_per_eff = T_per;
+  *s_eff = plan->lvsa_anchors == BSA_ANCHORS_FIXED ? 0 : ((s % T_per) + T_per) % T_per;
+  int n = 0;
+  for (int f = 0; f < T; ++f) n += ((f - *s_eff) % T_per + T_per) % T_per == 0;
+  return n;
+}
+
+
 static thread_local std::string g_last_error;
 
 bsa_status set_error(bsa_status st, const std::string& msg) {
@@ -174,14 +189,14 @@ bsa_status bsa_lvsa_mask(bsa_plan_t plan, int C, int T_per, int s, int32_t* fram
   if (!row_ptr || !col_idx) return set_error(BSA_ERR_INVALID_ARG, "row_ptr / col_idx is NULL");
   if ((int64_t)g.nblocks * C * g.nbf >= (1ll << 31))
     return set_error(BSA_ERR_UNSUPPORTED, "block list longer than 2^31 entries");
-  // |G_s U {t}| <= C for every t
-  const int sm = ((s % T_per) + T_per) % T_per;
-  int anchors = 0;
-  for (int f = 0; f < g.T; ++f) anchors += ((f - sm) % T_per + T_per) % T_per == 0;
+  // |G U {t}| <= C for every t
+  int tp = 0, sm = 0;
+  const int anchors = lvsa_effective_anchors(plan, T_per, s, &tp, &sm);
   const int worst = anchors + (anchors < g.T ? 1 : 0);
   if (worst > C)
     return set_error(BSA_ERR_INVALID_ARG, "budget C is smaller than the anchors plus the query frame");
-  cudaError_t e = launch_lvsa_mask(g, C, T_per, s, frame_sets, row_ptr, col_idx, plan->d_status,
+  cudaError_t e = launch_lvsa_mask(g, C, tp, sm, plan->lvsa_window == BSA_WINDOW_ALTERNATE,
+                                   frame_sets, row_ptr, col_idx, plan->d_status,
                                    reinterpret_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? BSA_OK : cuda_error(e, "lvsa_mask launch");
 }
@@ -215,8 +230,9 @@ bsa_status bsa_draft_mask(bsa_plan_t plan, const void* q_slots, const void* k_sl
   const int keep = bsa_draft_keep_count(plan, sparsity_pct);
   if ((int64_t)g.B * g.Hh * g.nblocks * keep >= (1ll << 31))
     return set_error(BSA_ERR_UNSUPPORTED, "block list longer than 2^31 entries");
-  cudaError_t e = launch_draft_mask(g, plan->d_tile_valid, q_slots, k_slots, keep, row_ptr, kv_idx,
-                                    draft_map, reinterpret_cast<double*>(workspace),
+  cudaError_t e = launch_draft_mask(g, plan->d_tile_valid, q_slots, k_slots, keep,
+                                    plan->draft_pooling, row_ptr, kv_idx, draft_map,
+                                    reinterpret_cast<double*>(workspace),
                                     reinterpret_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? BSA_OK : cuda_error(e, "draft_mask launch");
 }
@@ -274,6 +290,25 @@ bsa_status bsa_poll_status(bsa_plan_t plan, void* stream) {
   if (h & kStatusTimeout) return set_error(BSA_ERR_TIMEOUT, "a bounded device wait ran out");
   if (h & kStatusBadBlocklist)
     return set_error(BSA_ERR_BAD_BLOCKLIST, "a block list named a block out of range or was not ordered");
+  return BSA_OK;
+}
+
+bsa_status bsa_plan_set_lvsa_variant(bsa_plan_t plan, int anchors, int window_order) {
+  if (!plan) return set_error(BSA_ERR_INVALID_ARG, "plan is NULL");
+  if (anchors < BSA_ANCHORS_ROTATING || anchors > BSA_ANCHORS_NONE)
+    return set_error(BSA_ERR_INVALID_ARG, "unknown anchor mode");
+  if (window_order != BSA_WINDOW_DISTANCE && window_order != BSA_WINDOW_ALTERNATE)
+    return set_error(BSA_ERR_INVALID_ARG, "unknown window order");
+  plan->lvsa_anchors = anchors;
+  plan->lvsa_window = window_order;
+  return BSA_OK;
+}
+
+bsa_status bsa_plan_set_draft_pooling(bsa_plan_t plan, int pooling) {
+  if (!plan) return set_error(BSA_ERR_INVALID_ARG, "plan is NULL");
+  if (pooling != BSA_POOL_MEAN && pooling != BSA_POOL_MAX)
+    return set_error(BSA_ERR_INVALID_ARG, "unknown pooling");
+  plan->draft_pooling = pooling;
   return BSA_OK;
 }
 

@@ -65,6 +65,9 @@ struct bsa_plan_s {
   uint32_t* d_tile_valid = nullptr;  // [ntiles][4] bit per slot: slot holds a token
   unsigned int* d_status = nullptr;  // device status word
   uint64_t wait_limit_ns = 2000000000ull;
+  int lvsa_anchors = BSA_ANCHORS_ROTATING;  // bsa_plan_set_lvsa_variant
+  int lvsa_window = BSA_WINDOW_DISTANCE;
+  int draft_pooling = BSA_POOL_MEAN;        // bsa_plan_set_draft_pooling
 };
 
 namespace bsa {
@@ -75,16 +78,21 @@ bsa_status cuda_error(cudaError_t e, const char* what);
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 // Kernel launchers (each in its own translation unit).
-cudaError_t launch_lvsa_mask(const Geometry& g, int C, int T_per, int s, int32_t* frame_sets,
-                             int32_t* row_ptr, int32_t* col_idx, unsigned int* status,
-                             cudaStream_t st);
+// T_per = 0: no anchors; alternate != 0: alternating window growth.
+cudaError_t launch_lvsa_mask(const Geometry& g, int C, int T_per, int s, int alternate,
+                             int32_t* frame_sets, int32_t* row_ptr, int32_t* col_idx,
+                             unsigned int* status, cudaStream_t st);
 cudaError_t launch_reorder_fwd(const Geometry& g, const void* const x[3], void* const y[3],
                                int nt, cudaStream_t st);
 cudaError_t launch_reorder_inv(const Geometry& g, const void* x_slots, void* x_nat,
                                cudaStream_t st);
 cudaError_t launch_draft_mask(const Geometry& g, const uint32_t* tile_valid, const void* q,
-                              const void* k, int keep, int32_t* row_ptr, int32_t* kv_idx,
-                              float* draft_map, double* ws, cudaStream_t st);
+                              const void* k, int keep, int pooling, int32_t* row_ptr,
+                              int32_t* kv_idx, float* draft_map, double* ws, cudaStream_t st);
+
+// Anchor grid actually used for (plan variant, T_per, s): *T_per_eff = 0
+// means no anchors; also returns |G| over the plan's T frames.
+int lvsa_effective_anchors(const bsa_plan_s* plan, int T_per, int s, int* T_per_eff, int* s_eff);
 bsa_status launch_attn_fwd(const bsa_plan_s& plan, const void* q, const void* k, const void* v,
                            const int32_t* row_ptr, const int32_t* col_idx, int per_head,
                            float scale, void* o, float* lse, cudaStream_t st);

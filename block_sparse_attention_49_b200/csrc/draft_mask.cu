@@ -8,7 +8,9 @@
 //  pool:  qbar/kbar[b,h,blk,:] = mean of the block's non-empty slots, fp64.
 //         The sum runs sequentially over the block's slots in order (the
 //         tile's row-major order) and is divided once by the token count.
-//         16-byte loads; HBM bound.
+//         With max pooling (which the article's authors tried before
+//         settling on the average) it is the channel-wise maximum instead,
+//         exact in any order.  16-byte loads; HBM bound.
 //  score_topk: for a group of query-block rows of one (b, head), the fp64
 //         logits L[i][j] = sum_c qbar_i[c]*kbar_j[c] (sequential over c, the
 //         product and the sum each rounded, no fused multiply-add), then per
@@ -36,7 +38,7 @@ template <int D>
 __global__ void __launch_bounds__(kPoolThreads)
     draft_pool_kernel(const uint4* __restrict__ q, const uint4* __restrict__ k,
                       const uint32_t* __restrict__ tile_valid, int Hh, int64_t Npad,
-                      int64_t nblocks, int block, int64_t groups_per_tensor,
+                      int64_t nblocks, int block, int64_t groups_per_tensor, int use_max,
                       double* __restrict__ ws) {
   constexpr int kTPG = D / 8;  // threads per group
   const int64_t gid = ((int64_t)blockIdx.x * kPoolThreads + threadIdx.x) / kTPG;
@@ -49,7 +51,7 @@ __global__ void __launch_bounds__(kPoolThreads)
   const int64_t s0 = blk * block;
   double acc[8];
 #pragma unroll
-  for (int i = 0; i < 8; ++i) acc[i] = 0.0;
+  for (int i = 0; i < 8; ++i) acc[i] = use_max ? -INFINITY : 0.0;
   int cnt = 0;
   for (int e = 0; e < block; ++e) {
     const int64_t s = s0 + e;
@@ -57,18 +59,27 @@ __global__ void __launch_bounds__(kPoolThreads)
     if (!((w >> (s & 31)) & 1u)) continue;
     const uint4 v = __ldg(src + (int64_t)e * (D / 8));
     const __nv_bfloat162* pv = reinterpret_cast<const __nv_bfloat162*>(&v);
+    if (use_max) {
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const float2 f = __bfloat1622float2(pv[i]);
-      acc[2 * i] = __dadd_rn(acc[2 * i], (double)f.x);
-      acc[2 * i + 1] = __dadd_rn(acc[2 * i + 1], (double)f.y);
+      for (int i = 0; i < 4; ++i) {
+        const float2 f = __bfloat1622float2(pv[i]);
+        acc[2 * i] = fmax(acc[2 * i], (double)f.x);
+        acc[2 * i + 1] = fmax(acc[2 * i + 1], (double)f.y);
+      }
+    } else {
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const float2 f = __bfloat1622float2(pv[i]);
+        acc[2 * i] = __dadd_rn(acc[2 * i], (double)f.x);
+        acc[2 * i + 1] = __dadd_rn(acc[2 * i + 1], (double)f.y);
+      }
     }
     ++cnt;
   }
   double* dst = ws + ((int64_t)which * groups_per_tensor + g) * D + sub * 8;
   const double dc = (double)cnt;
 #pragma unroll
-  for (int i = 0; i < 8; ++i) dst[i] = cnt ? __ddiv_rn(acc[i], dc) : 0.0;
+  for (int i = 0; i < 8; ++i) dst[i] = cnt ? (use_max ? acc[i] : __ddiv_rn(acc[i], dc)) : 0.0;
 }
 
 // grid: (ceil(nblocks / R), Hh, B); R query rows per CTA.
@@ -178,14 +189,14 @@ __global__ void __launch_bounds__(kScoreThreads)
 
 template <int D>
 cudaError_t launch_t(const Geometry& g, const uint32_t* tile_valid, const void* q, const void* k,
-                     int keep, int32_t* row_ptr, int32_t* kv_idx, float* draft_map, double* ws,
-                     cudaStream_t st) {
+                     int keep, int pooling, int32_t* row_ptr, int32_t* kv_idx, float* draft_map,
+                     double* ws, cudaStream_t st) {
   const int64_t groups = (int64_t)g.B * g.Hh * g.nblocks;
   const int64_t threads = 2 * groups * (D / 8);
   const unsigned pool_grid = (unsigned)((threads + kPoolThreads - 1) / kPoolThreads);
   draft_pool_kernel<D><<<pool_grid, kPoolThreads, 0, st>>>(
       reinterpret_cast<const uint4*>(q), reinterpret_cast<const uint4*>(k), tile_valid, g.Hh,
-      g.Npad, g.nblocks, g.block, groups, ws);
+      g.Npad, g.nblocks, g.block, groups, pooling == BSA_POOL_MAX ? 1 : 0, ws);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   const int R = draft_rows_per_cta(g.nblocks);
@@ -214,10 +225,11 @@ size_t draft_workspace_bytes(const Geometry& g) {
 }
 
 cudaError_t launch_draft_mask(const Geometry& g, const uint32_t* tile_valid, const void* q,
-                              const void* k, int keep, int32_t* row_ptr, int32_t* kv_idx,
-                              float* draft_map, double* ws, cudaStream_t st) {
-  if (g.D == 128) return launch_t<128>(g, tile_valid, q, k, keep, row_ptr, kv_idx, draft_map, ws, st);
-  return launch_t<64>(g, tile_valid, q, k, keep, row_ptr, kv_idx, draft_map, ws, st);
+                              const void* k, int keep, int pooling, int32_t* row_ptr,
+                              int32_t* kv_idx, float* draft_map, double* ws, cudaStream_t st) {
+  if (g.D == 128)
+    return launch_t<128>(g, tile_valid, q, k, keep, pooling, row_ptr, kv_idx, draft_map, ws, st);
+  return launch_t<64>(g, tile_valid, q, k, keep, pooling, row_ptr, kv_idx, draft_map, ws, st);
 }
 
 }  // namespace bsa
@@ -304,7 +316,7 @@ extern "C" bsa_status bsa_draft_mask_noalloc(bsa_plan_t plan, const void* q_slot
   double* scratch = nullptr;
   cudaError_t e = noalloc_scratch_address(&scratch);
   if (e != cudaSuccess) return cuda_error(e, "cudaGetSymbolAddress(scratch)");
-  e = launch_draft_mask(g, plan->d_tile_valid, q_slots, k_slots, keep, row_ptr, kv_idx, draft_map,
-                        scratch, reinterpret_cast<cudaStream_t>(stream));
+  e = launch_draft_mask(g, plan->d_tile_valid, q_slots, k_slots, keep, plan->draft_pooling, row_ptr,
+                        kv_idx, draft_map, scratch, reinterpret_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? BSA_OK : cuda_error(e, "draft_mask_noalloc launch");
 }

@@ -5,10 +5,12 @@
 // attends, with softmax(scale * q.k), exactly the key tokens of the frames in
 // A(t) = G_s U W(t) - rotating anchors G_s = {f : (f - s) mod T_per = 0} and
 // a window around t grown t+1, t-1, t+2, ... past the frames already present
-// until |A(t)| = C.  The result equals bsa_lvsa_mask + bsa_reorder_fwd +
-// bsa_attn_fwd + bsa_reorder_inv; the reorder of the Draft Attention article
-// is fused into the tile loads (a 3-D tensor map reads [B*N, Hh, D] rows of
-// one head directly), so no padded copy of Q, K, V or O is ever made.
+// until |A(t)| = C (or a variant chosen on the plan: fixed-grid or no
+// anchors, alternating window growth).  The result equals bsa_lvsa_mask +
+// bsa_reorder_fwd + bsa_attn_fwd + bsa_reorder_inv; the reorder of the Draft
+// Attention article is fused into the tile loads (a 3-D tensor map reads
+// [B*N, Hh, D] rows of one head directly), so no padded copy of Q, K, V or O
+// is ever made.
 //
 // Work unit (one CTA, 12 warps): 256 consecutive query tokens of one
 // (b, head) = two 128-row query tiles that share every key tile.
@@ -20,9 +22,9 @@
 //    arithmetically (they are periodic).
 //  * warp 0: TMA producer (both query tiles, then K and V of every key tile
 //    into 2-deep rings; a K slot is refilled as soon as its last QK product
-//    is done, a V slot after its last PV product).  warp 1: MMA issuer.  warps 4-7 / 8-11: softmax of
-//    query tile 0 / 1, one row per thread, masking keys whose frame is not in
-//    the row's own A(t).
+//    is done, a V slot after its last PV product).  warp 1: MMA issuer.
+//    warps 4-7 / 8-11: softmax of query tile 0 / 1, one row per thread,
+//    masking keys whose frame is not in the row's own A(t).
 //  * tensor memory: S0 | S1 | O0 | O1; P aliases the upper half of its S.
 //    MMA order per key tile j: PV0(j), QK0(j+1), PV1(j), QK1(j+1), so the
 //    tensor cores run one tile's products while the other tile's softmax runs.
@@ -74,7 +76,8 @@ struct LvsaCfg {
 };
 
 struct LvsaParams {
-  int B, Hh, T, P, N, C, T_per, s_mod;
+  int B, Hh, T, P, N, C, T_per, s_mod;  // T_per = 0: no anchors
+  int alternate;                        // alternating window growth
   FastDiv divP;
   float scale, scale_log2;
   __nv_bfloat16* o;  // natural layout
@@ -89,12 +92,14 @@ __device__ __forceinline__ int floordiv(int a, int b) {
   return q;
 }
 
-// anchors in [a, b] (frames f with f = s_mod mod T_per)
+// anchors in [a, b] (frames f with f = s_mod mod T_per; none when T_per = 0)
 __device__ __forceinline__ int anchors_in(int a, int b, int s_mod, int T_per) {
-  return b < a ? 0 : floordiv(b - s_mod, T_per) - floordiv(a - 1 - s_mod, T_per);
+  return (b < a || T_per == 0) ? 0
+                               : floordiv(b - s_mod, T_per) - floordiv(a - 1 - s_mod, T_per);
 }
 
 __device__ __forceinline__ bool is_anchor(int f, int s_mod, int T_per) {
+  if (T_per == 0) return false;
   int r = (f - s_mod) % T_per;
   if (r < 0) r += T_per;
   return r == 0;
@@ -106,6 +111,15 @@ __device__ bool lvsa_member(int t, int f, const LvsaParams& p) {
   if (f == t || is_anchor(f, p.s_mod, p.T_per)) return true;
   const int base = anchors_in(0, p.T - 1, p.s_mod, p.T_per) + (t_anchor ? 0 : 1);
   const int need = p.C - base;
+  if (p.alternate) {
+    // right and left pointers take turns (right first): the right side takes
+    // kR of its nR frames outside the base, nearest first, the left the rest
+    const int nR = (p.T - 1 - t) - anchors_in(t + 1, p.T - 1, p.s_mod, p.T_per);
+    const int nL = t - anchors_in(0, t - 1, p.s_mod, p.T_per);
+    const int kR = min(nR, max((need + 1) / 2, need - nL)), kL = need - kR;
+    if (f > t) return (f - t) - anchors_in(t + 1, f, p.s_mod, p.T_per) <= kR;
+    return (t - f) - anchors_in(f, t - 1, p.s_mod, p.T_per) <= kL;
+  }
   const int d = f > t ? f - t : t - f;
   // frames outside the base strictly nearer than d (t itself is in the base)
   const int lo = max(t - d + 1, 0), hi = min(t + d - 1, p.T - 1);
@@ -544,9 +558,8 @@ extern "C" bsa_status bsa_lvsa_attn_fwd(bsa_plan_t plan, int C, int T_per, int s
   }
   if (lse && (reinterpret_cast<uintptr_t>(lse) & 3u))
     return set_error(BSA_ERR_ALIGNMENT, "lse is not 4-byte aligned");
-  const int sm = ((s % T_per) + T_per) % T_per;
-  int anchors = 0;
-  for (int f = 0; f < g.T; ++f) anchors += ((f - sm) % T_per + T_per) % T_per == 0;
+  int tp = 0, sm = 0;
+  const int anchors = lvsa_effective_anchors(plan, T_per, s, &tp, &sm);
   if (anchors + (anchors < g.T ? 1 : 0) > C)
     return set_error(BSA_ERR_INVALID_ARG, "budget C is smaller than the anchors plus the query frame");
   if (g.T > kMaxFrames) return set_error(BSA_ERR_UNSUPPORTED, "fused LVSA attention supports T <= 4096");
@@ -570,8 +583,9 @@ extern "C" bsa_status bsa_lvsa_attn_fwd(bsa_plan_t plan, int C, int T_per, int s
   p.P = g.P;
   p.N = (int)N;
   p.C = C;
-  p.T_per = T_per;
+  p.T_per = tp;
   p.s_mod = sm;
+  p.alternate = plan->lvsa_window == BSA_WINDOW_ALTERNATE ? 1 : 0;
   p.divP = FastDiv((uint32_t)g.P);
   p.scale = scale;
   p.scale_log2 = scale * 1.4426950408889634f;

@@ -15,6 +15,14 @@
 // same distance on the right).  Each thread evaluates that count for its
 // frames in O(1) from a prefix sum, so the set needs no serial loop.
 //
+// Variants (chosen by the caller): T_per = 0 means no anchors (the sliding
+// window); fixed-grid anchors are the rotating ones at s = 0.  With the
+// alternating growth order (a right and a left pointer taking turns, right
+// first, each skipping frames already present; a side that runs off the
+// grid stops) the right side takes kR = min(nR, max(ceil(need/2), need - nL))
+// of its nR frames outside base, nearest first, and the left side the other
+// need - kR of its nL; membership is again a prefix-sum rank.
+//
 // One CTA per query block (grid nbf x T); each writes its CSR row.
 #include "bsa_internal.cuh"
 
@@ -51,7 +59,8 @@ __device__ int block_exclusive_scan(int* a, int n, int* warp_tot) {
 }
 
 __global__ void __launch_bounds__(kThreads)
-    lvsa_mask_kernel(int T, int C, int T_per, int s, int nbf, int32_t* __restrict__ frame_sets,
+    lvsa_mask_kernel(int T, int C, int T_per, int s, int alternate, int nbf,
+                     int32_t* __restrict__ frame_sets,
                      int32_t* __restrict__ row_ptr, int32_t* __restrict__ col_idx,
                      unsigned int* status) {
   extern __shared__ int sh[];
@@ -60,12 +69,16 @@ __global__ void __launch_bounds__(kThreads)
   int* members = incl + T + 1;  // [C]
   __shared__ int warp_tot[kThreads / 32];
   const int i = blockIdx.x, t = blockIdx.y;
-  const int sm = ((s % T_per) + T_per) % T_per;
+  const int sm = T_per > 0 ? ((s % T_per) + T_per) % T_per : 0;
 
   for (int f = threadIdx.x; f < T; f += kThreads) {
-    int r = (f - sm) % T_per;
-    if (r < 0) r += T_per;
-    out[f] = (r == 0 || f == t) ? 0 : 1;
+    bool anchor = false;
+    if (T_per > 0) {
+      int r = (f - sm) % T_per;
+      if (r < 0) r += T_per;
+      anchor = r == 0;
+    }
+    out[f] = (anchor || f == t) ? 0 : 1;
   }
   __syncthreads();
   const int n_out = block_exclusive_scan(out, T, warp_tot);
@@ -78,10 +91,16 @@ __global__ void __launch_bounds__(kThreads)
     const int lo = max(a + 1, 0), hi = min(b, T);
     return hi > lo ? out[hi] - out[lo] : 0;
   };
+  // alternating order: frames outside base right / left of t, and each side's share
+  const int nR = out[T] - out[t + 1], nL = out[t];
+  const int kR = min(nR, max((need + 1) / 2, need - nL)), kL = need - kR;
   for (int f = threadIdx.x; f < T; f += kThreads) {
     const bool is_out = (out[f + 1] - out[f]) != 0;
     int in = 1;
-    if (is_out) {
+    if (is_out && alternate) {
+      // rank of f among its side's frames outside base, nearest first (1-based)
+      in = f > t ? (out[f + 1] - out[t + 1] <= kR) : (out[t] - out[f] <= kL);
+    } else if (is_out) {
       const int d = f > t ? f - t : t - f;
       int before = between(t, t + d) + between(t - d, t);
       if (f < t && t + d < T && (out[t + d + 1] - out[t + d]) != 0) ++before;
@@ -117,13 +136,13 @@ __global__ void __launch_bounds__(kThreads)
 
 }  // namespace
 
-cudaError_t launch_lvsa_mask(const Geometry& g, int C, int T_per, int s, int32_t* frame_sets,
-                             int32_t* row_ptr, int32_t* col_idx, unsigned int* status,
-                             cudaStream_t st) {
+cudaError_t launch_lvsa_mask(const Geometry& g, int C, int T_per, int s, int alternate,
+                             int32_t* frame_sets, int32_t* row_ptr, int32_t* col_idx,
+                             unsigned int* status, cudaStream_t st) {
   const size_t smem = (size_t)(2 * (g.T + 1) + C) * sizeof(int);
   const dim3 grid((unsigned)g.nbf, (unsigned)g.T);
-  lvsa_mask_kernel<<<grid, kThreads, smem, st>>>(g.T, C, T_per, s, g.nbf, frame_sets, row_ptr,
-                                                  col_idx, status);
+  lvsa_mask_kernel<<<grid, kThreads, smem, st>>>(g.T, C, T_per, s, alternate, g.nbf, frame_sets,
+                                                  row_ptr, col_idx, status);
   return cudaGetLastError();
 }
 

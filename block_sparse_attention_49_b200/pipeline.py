@@ -14,9 +14,10 @@ import math
 
 import torch
 
-from . import (LAYOUT_FRAME, LAYOUT_TILE, Plan, bsa_attn_fwd, bsa_draft_keep_count,
-               bsa_draft_mask, bsa_draft_workspace_bytes, bsa_lvsa_attn_fwd, bsa_lvsa_mask,
-               bsa_lvsa_nnz, bsa_reorder_fwd, bsa_reorder_inv)
+from . import (ANCHORS_ROTATING, LAYOUT_FRAME, LAYOUT_TILE, POOL_MEAN, WINDOW_DISTANCE, Plan,
+               bsa_attn_fwd, bsa_draft_keep_count, bsa_draft_mask, bsa_draft_workspace_bytes,
+               bsa_lvsa_attn_fwd, bsa_lvsa_mask, bsa_lvsa_nnz, bsa_plan_set_draft_pooling,
+               bsa_plan_set_lvsa_variant, bsa_reorder_fwd, bsa_reorder_inv)
 
 
 class _Base:
@@ -40,10 +41,13 @@ class _Base:
 
 
 class LvsaAttention(_Base):
-    """LVSA block-sparse attention on the frame layout."""
+    """LVSA block-sparse attention on the frame layout.  `anchors` and
+    `window_order` select a mask variant (bsa_plan_set_lvsa_variant)."""
 
-    def __init__(self, B, Hh, D, T, H, W, C, T_per, block=128, device="cuda", scale=None):
+    def __init__(self, B, Hh, D, T, H, W, C, T_per, block=128, device="cuda", scale=None,
+                 anchors=ANCHORS_ROTATING, window_order=WINDOW_DISTANCE):
         self.plan = Plan(B, Hh, D, T, H, W, LAYOUT_FRAME, block=block)
+        bsa_plan_set_lvsa_variant(self.plan, anchors, window_order)
         self.C, self.T_per = C, T_per
         self.scale = scale if scale is not None else 1.0 / math.sqrt(D)
         nnz = bsa_lvsa_nnz(self.plan, C)
@@ -71,11 +75,13 @@ class LvsaAttention(_Base):
 
 
 class DraftAttention(_Base):
-    """Draft-mask block-sparse attention on the tile layout."""
+    """Draft-mask block-sparse attention on the tile layout.  `pooling`:
+    POOL_MEAN (the article's average) or POOL_MAX."""
 
     def __init__(self, B, Hh, D, T, H, W, pool_h, pool_w, sparsity_pct, device="cuda",
-                 scale=None, want_map=False):
+                 scale=None, want_map=False, pooling=POOL_MEAN):
         self.plan = Plan(B, Hh, D, T, H, W, LAYOUT_TILE, pool_h, pool_w, pool_h * pool_w)
+        bsa_plan_set_draft_pooling(self.plan, pooling)
         self.sparsity = sparsity_pct
         self.scale = scale if scale is not None else 1.0 / math.sqrt(D)
         self.keep = bsa_draft_keep_count(self.plan, sparsity_pct)

@@ -67,6 +67,20 @@ typedef enum {
  * 128 (the attention tile); slots past the last block are empty. */
 typedef enum { BSA_LAYOUT_FRAME = 0, BSA_LAYOUT_TILE = 1 } bsa_layout;
 
+/* LVSA mask variants (bsa_plan_set_lvsa_variant). */
+typedef enum {
+  BSA_ANCHORS_ROTATING = 0, /* G_s = {f : (f - s) mod T_per == 0} (LVSA)       */
+  BSA_ANCHORS_FIXED = 1,    /* G = {f : f mod T_per == 0} at every step         */
+  BSA_ANCHORS_NONE = 2      /* no global frames: the sliding window alone       */
+} bsa_anchor_mode;
+typedef enum {
+  BSA_WINDOW_DISTANCE = 0,  /* grow t+1, t-1, t+2, t-2, ... (default)          */
+  BSA_WINDOW_ALTERNATE = 1  /* right and left pointers take turns, right first */
+} bsa_window_order;
+
+/* Draft pooling (bsa_plan_set_draft_pooling). */
+typedef enum { BSA_POOL_MEAN = 0, BSA_POOL_MAX = 1 } bsa_pooling;
+
 typedef struct bsa_plan_s* bsa_plan_t;
 
 /* Create a plan for batch B, Hh heads, head dim D, latent grid T x H x W.
@@ -80,6 +94,24 @@ bsa_status bsa_plan_create(bsa_plan_t* plan, int B, int Hh, int D, int T, int H,
 /* Free the plan and its device data.  No call using it may be in flight. */
 bsa_status bsa_plan_destroy(bsa_plan_t plan);
 
+/* Choose the LVSA mask variant used by bsa_lvsa_mask and bsa_lvsa_attn_fwd
+ * with this plan (default ROTATING, DISTANCE).  "LVSA", section 2 "Core
+ * mechanism", contrasts its rotating anchors with fixed-grid global frames,
+ * and the page's introduction lists plain sliding windows; FIXED and NONE
+ * give those patterns under the same budget C.  The page leaves the growth
+ * order of the extended window open: DISTANCE adds the nearest frame not yet
+ * present (ties to the right), ALTERNATE lets a right and a left pointer take
+ * turns (right first), each moving past frames already present; a side that
+ * runs off [0, T) stops and the other continues.  Takes effect for calls
+ * issued after it; returns BSA_ERR_INVALID_ARG for unknown values. */
+bsa_status bsa_plan_set_lvsa_variant(bsa_plan_t plan, int anchors, int window_order);
+
+/* Choose the pooling of bsa_draft_mask / bsa_draft_mask_noalloc with this
+ * plan (default MEAN).  MAX takes the channel-wise maximum over the tile's
+ * tokens inside the grid: the Draft Attention article reports trying max
+ * pooling first and preferring the average at high sparsity. */
+bsa_status bsa_plan_set_draft_pooling(bsa_plan_t plan, int pooling);
+
 /* Geometry queries (return -1 for a NULL plan). */
 int64_t bsa_padded_tokens(bsa_plan_t plan);   /* Npad                          */
 int64_t bsa_num_blocks(bsa_plan_t plan);      /* blocks per (b, head): Nb      */
@@ -90,6 +122,7 @@ int     bsa_block_size(bsa_plan_t plan);
  *   G_s = {f in [0,T) : (f - s) mod T_per == 0};
  *   A(t) = G_s U {t} grown by t+1, t-1, t+2, t-2, ... (frames outside [0,T)
  *   or already present are skipped) until |A(t)| = C.
+ * (Other anchor grids and growth orders: bsa_plan_set_lvsa_variant.)
  * Requires a FRAME plan, 1 <= T_per, C <= T and |G_s U {t}| <= C for every t.
  * Outputs (device):
  *   frame_sets int32[T*C] (may be NULL): row t = A(t) ascending;
@@ -116,7 +149,8 @@ size_t bsa_draft_workspace_bytes(bsa_plan_t plan);
  * Requires a TILE plan.  q_slots, k_slots: slot layout (output of
  * bsa_reorder_fwd).  For every (b, head, query block i):
  *   qbar_i, kbar_j = mean over the tile's tokens inside the grid (fp64,
- *     sequential sum in row-major tile order, one IEEE division);
+ *     sequential sum in row-major tile order, one IEEE division), or their
+ *     maximum with bsa_plan_set_draft_pooling(BSA_POOL_MAX);
  *   L[i][j] = sum_c qbar_i[c]*kbar_j[c], sequential over c, each product and
  *     sum rounded to fp64 (no fused multiply-add);
  *   keep the k = bsa_draft_keep_count() blocks j with the largest L[i][j],

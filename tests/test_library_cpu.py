@@ -65,6 +65,8 @@ def test_null_plan_is_rejected(lib):
     assert lib.bsa_lvsa_mask(None, 4, 4, 0, None, None, None, None) == 1
     assert lib.bsa_attn_fwd(None, None, None, None, None, None, 0, 1.0, None, None, None) == 1
     assert lib.bsa_poll_status(None, None) == 1
+    assert lib.bsa_plan_set_lvsa_variant(None, 0, 0) == 1
+    assert lib.bsa_plan_set_draft_pooling(None, 0) == 1
 
 
 def test_no_cpu_fallback_path():
