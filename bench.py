@@ -43,7 +43,7 @@ METRIC = "bsattn ms/call + attended TFLOP/s (% BF16 peak), Wan-1.3B-shape 6× le
 # capture summarised in profiles/lvsa_attn_fwd_wan13b_6x_first24frames.md
 # (24-frame case, scaled by the number of query pairs).  Set to None whenever
 # the kernel changes until it is captured again.
-STEP_KERNEL_DRAM_BYTES = 449.8e6 * 126 / 24
+STEP_KERNEL_DRAM_BYTES = 447.9e6 * 126 / 24
 
 
 def attended_flops(w) -> float:
