@@ -26,7 +26,7 @@ __all__ = [
     "bsa_block_size", "bsa_lvsa_mask", "bsa_lvsa_nnz", "bsa_draft_keep_count",
     "bsa_draft_workspace_bytes", "bsa_draft_mask", "bsa_draft_mask_noalloc",
     "bsa_draft_noalloc_max_scratch_bytes", "bsa_reorder_fwd", "bsa_reorder_inv",
-    "bsa_attn_fwd", "bsa_lvsa_attn_fwd", "bsa_poll_status", "bsa_set_wait_limit_ns", "bsa_selftest_timeout",
+    "bsa_attn_fwd", "bsa_attn_fwd_natural", "bsa_draft_mask_natural", "bsa_lvsa_attn_fwd", "bsa_poll_status", "bsa_set_wait_limit_ns", "bsa_selftest_timeout",
     "bsa_last_error", "bsa_version", "EXPORTED_SYMBOLS",
 ]
 
@@ -66,6 +66,9 @@ _SIGS = {
     "bsa_reorder_inv": (_c_int, [_c_p, _c_p, _c_p, _c_p]),
     "bsa_attn_fwd": (_c_int, [_c_p, _c_p, _c_p, _c_p, _c_p, _c_p, _c_int, ctypes.c_float, _c_p,
                               _c_p, _c_p]),
+    "bsa_attn_fwd_natural": (_c_int, [_c_p, _c_p, _c_p, _c_p, _c_p, _c_p, _c_int, ctypes.c_float, _c_p,
+                              _c_p, _c_p]),
+    "bsa_draft_mask_natural": (_c_int, [_c_p, _c_p, _c_p, _c_int, _c_p, _c_p, _c_p, _c_p, _c_sz, _c_p]),
     "bsa_lvsa_attn_fwd": (_c_int, [_c_p, _c_int, _c_int, _c_int, _c_p, _c_p, _c_p, ctypes.c_float,
                                    _c_p, _c_p, _c_p]),
     "bsa_poll_status": (_c_int, [_c_p, _c_p]),
@@ -225,6 +228,24 @@ def bsa_attn_fwd(plan: Plan, q, k, v, row_ptr, col_idx, per_head_lists: bool, sc
     _check(load().bsa_attn_fwd(plan.handle, _ptr(q), _ptr(k), _ptr(v), _ptr(row_ptr),
                                _ptr(col_idx), int(bool(per_head_lists)), float(scale), _ptr(o),
                                _ptr(lse), _stream(stream)), "bsa_attn_fwd")
+
+
+def bsa_attn_fwd_natural(plan: Plan, q, k, v, row_ptr, col_idx, per_head_lists: bool,
+                         scale: float, o, lse=None, stream=None):
+    """bsa_attn_fwd on natural-layout [B, N, Hh, D] tensors (TILE plan, 128-slot tiles)."""
+    _check(load().bsa_attn_fwd_natural(plan.handle, _ptr(q), _ptr(k), _ptr(v), _ptr(row_ptr),
+                                       _ptr(col_idx), int(bool(per_head_lists)), float(scale),
+                                       _ptr(o), _ptr(lse), _stream(stream)), "bsa_attn_fwd_natural")
+
+
+def bsa_draft_mask_natural(plan: Plan, q, k, sparsity_pct: int, row_ptr, kv_idx, draft_map,
+                           workspace, stream=None):
+    """bsa_draft_mask reading natural-layout q, k directly."""
+    nbytes = workspace.numel() * workspace.element_size()
+    _check(load().bsa_draft_mask_natural(plan.handle, _ptr(q), _ptr(k), sparsity_pct,
+                                         _ptr(row_ptr), _ptr(kv_idx), _ptr(draft_map),
+                                         _ptr(workspace), nbytes, _stream(stream)),
+           "bsa_draft_mask_natural")
 
 
 def bsa_lvsa_attn_fwd(plan: Plan, C: int, T_per: int, s: int, q, k, v, scale: float, o,

@@ -279,6 +279,49 @@ bsa_status bsa_attn_fwd(bsa_plan_t plan, const void* q, const void* k, const voi
                          reinterpret_cast<cudaStream_t>(stream));
 }
 
+bsa_status bsa_attn_fwd_natural(bsa_plan_t plan, const void* q, const void* k, const void* v,
+                                const int32_t* row_ptr, const int32_t* col_idx, int per_head_lists,
+                                float scale, void* o, float* lse, void* stream) {
+  if (!plan) return set_error(BSA_ERR_INVALID_ARG, "plan is NULL");
+  if (plan->g.layout != BSA_LAYOUT_TILE)
+    return set_error(BSA_ERR_INVALID_ARG, "natural-layout attention needs a TILE plan");
+  bsa_status st;
+  if ((st = check_ptr(q, "q")) != BSA_OK || (st = check_ptr(k, "k")) != BSA_OK ||
+      (st = check_ptr(v, "v")) != BSA_OK || (st = check_ptr(o, "o")) != BSA_OK)
+    return st;
+  if (!row_ptr || !col_idx) return set_error(BSA_ERR_INVALID_ARG, "row_ptr / col_idx is NULL");
+  if (lse && (reinterpret_cast<uintptr_t>(lse) & 3u))
+    return set_error(BSA_ERR_ALIGNMENT, "lse is not 4-byte aligned");
+  if (!(scale > 0.f)) return set_error(BSA_ERR_INVALID_ARG, "scale must be positive");
+  return launch_attn_fwd_natural(*plan, q, k, v, row_ptr, col_idx, per_head_lists, scale, o, lse,
+                                 reinterpret_cast<cudaStream_t>(stream));
+}
+
+bsa_status bsa_draft_mask_natural(bsa_plan_t plan, const void* q, const void* k, int sparsity_pct,
+                                  int32_t* row_ptr, int32_t* kv_idx, float* draft_map,
+                                  void* workspace, size_t workspace_bytes, void* stream) {
+  if (!plan) return set_error(BSA_ERR_INVALID_ARG, "plan is NULL");
+  const Geometry& g = plan->g;
+  if (g.layout != BSA_LAYOUT_TILE) return set_error(BSA_ERR_INVALID_ARG, "draft mask needs a TILE plan");
+  if (sparsity_pct < 0 || sparsity_pct >= 100)
+    return set_error(BSA_ERR_INVALID_ARG, "sparsity must be in [0, 100)");
+  bsa_status st;
+  if ((st = check_ptr(q, "q")) != BSA_OK) return st;
+  if ((st = check_ptr(k, "k")) != BSA_OK) return st;
+  if ((st = check_ptr(workspace, "workspace")) != BSA_OK) return st;
+  if (!kv_idx) return set_error(BSA_ERR_INVALID_ARG, "kv_idx is NULL");
+  if (workspace_bytes < draft_workspace_bytes(g))
+    return set_error(BSA_ERR_INVALID_ARG, "workspace too small");
+  if (g.nblocks > 18000) return set_error(BSA_ERR_UNSUPPORTED, "draft mask supports up to 18000 blocks");
+  const int keep = bsa_draft_keep_count(plan, sparsity_pct);
+  if ((int64_t)g.B * g.Hh * g.nblocks * keep >= (1ll << 31))
+    return set_error(BSA_ERR_UNSUPPORTED, "block list longer than 2^31 entries");
+  cudaError_t e = launch_draft_mask(g, plan->d_tile_valid, q, k, keep, plan->draft_pooling, row_ptr,
+                                    kv_idx, draft_map, reinterpret_cast<double*>(workspace),
+                                    reinterpret_cast<cudaStream_t>(stream), /*natural=*/true);
+  return e == cudaSuccess ? BSA_OK : cuda_error(e, "draft_mask_natural launch");
+}
+
 bsa_status bsa_poll_status(bsa_plan_t plan, void* stream) {
   if (!plan) return set_error(BSA_ERR_INVALID_ARG, "plan is NULL");
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);

@@ -80,6 +80,9 @@ struct AttnParams {
   const uint32_t* tile_valid;  // [ntiles][4]
   unsigned int* status;
   uint64_t wait_limit_ns;
+  // natural layout (NAT): [B, N, Hh, D] in and out; tile = one ph x pw tile
+  int T, H, W, N, TW, ph, pw;
+  FastDiv div_tile_frame, div_TW, div_pw;  // by TH*TW, TW, pw
 };
 
 // Set bits [lo, lo+len) of a 128-bit mask; lo is a multiple of len, len | 128.
@@ -105,7 +108,7 @@ __device__ __forceinline__ void cta_end_sync() {
   asm volatile("bar.sync 2, 384;" ::: "memory");
 }
 
-template <int D, bool FINE>
+template <int D, bool FINE, bool NAT>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmk,
                     const __grid_constant__ CUtensorMap tmv, const AttnParams p) {
@@ -127,8 +130,20 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint32_t* bitmap = reinterpret_cast<uint32_t*>(smem + Cfg::kOffBitmap);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  static_assert(!(NAT && FINE), "natural-layout tiles are whole ph x pw tiles");
   const int qt = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
   const int64_t bh_row = ((int64_t)b * p.Hh + h) * p.Npad;
+  // natural layout: tile kt of (b, h) is the ph x pw tile (t, i, j); TMA
+  // coordinates {channel, head, x0, y0, frame}; the part past the grid edge
+  // reads as zero (the empty slots of the tile layout)
+  auto nat_coords = [&](int kt, int& x0, int& y0, int& fr) {
+    const int t = (int)p.div_tile_frame.div((uint32_t)kt);
+    const int r = kt - t * (int)p.div_tile_frame.d;
+    const int i = (int)p.div_TW.div((uint32_t)r);
+    x0 = (r - i * p.TW) * p.pw;
+    y0 = i * p.ph;
+    fr = b * p.T + t;
+  };
   const int64_t list = p.per_head ? (int64_t)b * p.Hh + h : 0;
   const WaitCtx wc{p.status, reinterpret_cast<volatile int*>(&misc[1]), p.wait_limit_ns};
 
@@ -226,14 +241,22 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (warp < 4) {
     // producer, MMA issuer and two idle warps: few registers
-    asm volatile("setmaxnreg.dec.sync.aligned.u32 56;");
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 72;");
     if (warp == 0 && n > 0) {
       // -------------------------------------------------------- TMA producer
       // the whole warp runs the loop (warp-uniform operands); one lane issues
       if (elect_one()) {
         mbar_arrive_expect_tx(q_full, Cfg::kQBytes);
-        for (int c = 0; c < Cfg::kChunks; ++c)
-          tma_load_2d(sQ + c * Cfg::kPanel, &tmq, q_full, c * 64, (int)(bh_row + (int64_t)qt * kTile));
+        if constexpr (NAT) {
+          int x0, y0, fr;
+          nat_coords(qt, x0, y0, fr);
+          for (int c = 0; c < Cfg::kChunks; ++c)
+            tma_load_5d(sQ + c * Cfg::kPanel, &tmq, q_full, c * 64, h, x0, y0, fr);
+        } else {
+          for (int c = 0; c < Cfg::kChunks; ++c)
+            tma_load_2d(sQ + c * Cfg::kPanel, &tmq, q_full, c * 64,
+                        (int)(bh_row + (int64_t)qt * kTile));
+        }
       }
       __syncwarp();
       int issued = 0;
@@ -248,12 +271,23 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (!ok) atomicOr(p.status, kStatusBadBlocklist);
           uint8_t* sK = smem + Cfg::kOffK + st * Cfg::kKVBytes;
           uint8_t* sV = smem + Cfg::kOffV + st * Cfg::kKVBytes;
-          mbar_arrive_expect_tx(&k_full[st], Cfg::kKVBytes);
-          for (int c = 0; c < Cfg::kChunks; ++c)
-            tma_load_2d(sK + c * Cfg::kPanel, &tmk, &k_full[st], c * 64, krow);
-          mbar_arrive_expect_tx(&v_full[st], Cfg::kKVBytes);
-          for (int c = 0; c < Cfg::kChunks; ++c)
-            tma_load_2d(sV + c * Cfg::kPanel, &tmv, &v_full[st], c * 64, krow);
+          if constexpr (NAT) {
+            int x0, y0, fr;
+            nat_coords(kt, x0, y0, fr);
+            mbar_arrive_expect_tx(&k_full[st], Cfg::kKVBytes);
+            for (int c = 0; c < Cfg::kChunks; ++c)
+              tma_load_5d(sK + c * Cfg::kPanel, &tmk, &k_full[st], c * 64, h, x0, y0, fr);
+            mbar_arrive_expect_tx(&v_full[st], Cfg::kKVBytes);
+            for (int c = 0; c < Cfg::kChunks; ++c)
+              tma_load_5d(sV + c * Cfg::kPanel, &tmv, &v_full[st], c * 64, h, x0, y0, fr);
+          } else {
+            mbar_arrive_expect_tx(&k_full[st], Cfg::kKVBytes);
+            for (int c = 0; c < Cfg::kChunks; ++c)
+              tma_load_2d(sK + c * Cfg::kPanel, &tmk, &k_full[st], c * 64, krow);
+            mbar_arrive_expect_tx(&v_full[st], Cfg::kKVBytes);
+            for (int c = 0; c < Cfg::kChunks; ++c)
+              tma_load_2d(sV + c * Cfg::kPanel, &tmv, &v_full[st], c * 64, krow);
+          }
         }
         __syncwarp();
         issued = j + 1;
@@ -335,7 +369,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       tmem_dealloc(tbase, Cfg::kTmemCols);
     }
   } else {
-    asm volatile("setmaxnreg.inc.sync.aligned.u32 224;");
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 216;");
     // ---------------------------------------------------------- softmax groups
     const int g = (warp >= 8) ? 1 : 0;
     const int q4 = warp & 3;
@@ -483,7 +517,20 @@ __global__ void __launch_bounds__(kThreads, 1)
     const bool has = alive && n > 0 && qvalid && l > 0.f;
     const float inv_l = has ? 1.f / l : 0.f;
     const float wa = a * inv_l, wb = bb * inv_l;
-    const int64_t orow = bh_row + (int64_t)qt * kTile + row;
+    int64_t orow = bh_row + (int64_t)qt * kTile + row;  // slot row, or natural token row
+    int64_t lrow = orow;                                 // LSE index
+    if constexpr (NAT) {
+      // slot (a, c) of tile (t, i, j) is token (t, y0 + a, x0 + c); empty slots
+      // (past the grid edge) are not stored
+      int x0, y0, fr;
+      nat_coords(qt, x0, y0, fr);
+      const int a = (int)p.div_pw.div((uint32_t)row);
+      const int y = y0 + a, x = x0 + (row - a * p.pw);
+      const int t = fr - b * p.T;
+      const int64_t n = ((int64_t)t * p.H + y) * p.W + x;
+      orow = ((int64_t)b * p.N + n) * p.Hh + h;
+      lrow = ((int64_t)b * p.Hh + h) * p.N + n;
+    }
     // group g stores columns [g*D/2, (g+1)*D/2) of its rows
     uint4* dst = reinterpret_cast<uint4*>(p.o + orow * D + g * (D / 2));
     const uint32_t oA = tbase + 256 + lane_off + g * (D / 2);
@@ -503,11 +550,13 @@ __global__ void __launch_bounds__(kThreads, 1)
             has ? __uint_as_float(xa[2 * i + 1]) * wa + __uint_as_float(xb[2 * i + 1]) * wb : 0.f;
         w16[i] = pack_bf16x2(v0, v1);
       }
+      if (!NAT || qvalid) {
 #pragma unroll
-      for (int i = 0; i < 4; ++i)
-        dst[c * 4 + i] = make_uint4(w16[4 * i], w16[4 * i + 1], w16[4 * i + 2], w16[4 * i + 3]);
+        for (int i = 0; i < 4; ++i)
+          dst[c * 4 + i] = make_uint4(w16[4 * i], w16[4 * i + 1], w16[4 * i + 2], w16[4 * i + 3]);
+      }
     }
-    if (g == 0 && p.lse) p.lse[orow] = has ? m * p.scale + logf(l) : -INFINITY;
+    if (g == 0 && p.lse && (!NAT || qvalid)) p.lse[lrow] = has ? m * p.scale + logf(l) : -INFINITY;
     tc_fence_before();
     cta_end_sync();
   }
@@ -539,11 +588,11 @@ bool make_tmap(CUtensorMap* m, const void* ptr, int64_t rows, int D) {
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int D, bool FINE>
+template <int D, bool FINE, bool NAT = false>
 cudaError_t launch_t(const CUtensorMap& q, const CUtensorMap& k, const CUtensorMap& v,
                      const AttnParams& p, dim3 grid, cudaStream_t st) {
   using Cfg = AttnCfg<D, FINE>;
-  auto kern = attn_fwd_kernel<D, FINE>;
+  auto kern = attn_fwd_kernel<D, FINE, NAT>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::kSmem);
   if (e != cudaSuccess) return e;
   kern<<<grid, kThreads, Cfg::kSmem, st>>>(q, k, v, p);
@@ -552,18 +601,11 @@ cudaError_t launch_t(const CUtensorMap& q, const CUtensorMap& k, const CUtensorM
 
 }  // namespace
 
-bsa_status launch_attn_fwd(const bsa_plan_s& plan, const void* q, const void* k, const void* v,
-                           const int32_t* row_ptr, const int32_t* col_idx, int per_head,
-                           float scale, void* o, float* lse, cudaStream_t st) {
+namespace {
+
+AttnParams make_params(const bsa_plan_s& plan, const int32_t* row_ptr, const int32_t* col_idx,
+                       int per_head, float scale, void* o, float* lse) {
   const Geometry& g = plan.g;
-  const int64_t rows = (int64_t)g.B * g.Hh * g.Npad;
-  if (rows >= (1ll << 31)) return set_error(BSA_ERR_UNSUPPORTED, "B*Hh*Npad must be < 2^31");
-  const bool fine = g.block < kTile;
-  if (fine && g.ntiles > kFineMaxTiles)
-    return set_error(BSA_ERR_UNSUPPORTED, "blocks smaller than 128 slots need Npad <= 262144");
-  CUtensorMap tq, tk, tv;
-  if (!make_tmap(&tq, q, rows, g.D) || !make_tmap(&tk, k, rows, g.D) || !make_tmap(&tv, v, rows, g.D))
-    return set_error(BSA_ERR_CUDA, "cuTensorMapEncodeTiled failed");
   AttnParams p;
   p.Hh = g.Hh;
   p.block = g.block;
@@ -580,6 +622,52 @@ bsa_status launch_attn_fwd(const bsa_plan_s& plan, const void* q, const void* k,
   p.tile_valid = plan.d_tile_valid;
   p.status = plan.d_status;
   p.wait_limit_ns = plan.wait_limit_ns;
+  p.T = g.T;
+  p.H = g.H;
+  p.W = g.W;
+  p.N = g.T * g.P;
+  p.ph = g.ph > 0 ? g.ph : 1;
+  p.pw = g.pw > 0 ? g.pw : 1;
+  p.TW = (g.W + p.pw - 1) / p.pw;
+  const int TH = (g.H + p.ph - 1) / p.ph;
+  p.div_tile_frame = FastDiv((uint32_t)(TH * p.TW));
+  p.div_TW = FastDiv((uint32_t)p.TW);
+  p.div_pw = FastDiv((uint32_t)p.pw);
+  return p;
+}
+
+// Natural layout [B, N, Hh, D] bf16 seen as 5-D {D, Hh, W, H, B*T}; boxes of
+// 64 channels x 1 head x pw x ph x 1 frame (one pooling tile, 128 rows of
+// 128 bytes), 128-byte swizzle.  Boxes reaching past W or H read zeros.
+bool make_tmap_tiles(CUtensorMap* m, const void* ptr, const Geometry& g) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  const cuuint64_t row = (cuuint64_t)g.Hh * g.D * 2;  // bytes per token
+  cuuint64_t dims[5] = {(cuuint64_t)g.D, (cuuint64_t)g.Hh, (cuuint64_t)g.W, (cuuint64_t)g.H,
+                        (cuuint64_t)g.B * g.T};
+  cuuint64_t strides[4] = {(cuuint64_t)g.D * 2, row, row * g.W, row * g.W * g.H};
+  cuuint32_t box[5] = {64, 1, (cuuint32_t)g.pw, (cuuint32_t)g.ph, 1};
+  cuuint32_t estr[5] = {1, 1, 1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, const_cast<void*>(ptr), dims, strides, box,
+            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+}  // namespace
+
+bsa_status launch_attn_fwd(const bsa_plan_s& plan, const void* q, const void* k, const void* v,
+                           const int32_t* row_ptr, const int32_t* col_idx, int per_head,
+                           float scale, void* o, float* lse, cudaStream_t st) {
+  const Geometry& g = plan.g;
+  const int64_t rows = (int64_t)g.B * g.Hh * g.Npad;
+  if (rows >= (1ll << 31)) return set_error(BSA_ERR_UNSUPPORTED, "B*Hh*Npad must be < 2^31");
+  const bool fine = g.block < kTile;
+  if (fine && g.ntiles > kFineMaxTiles)
+    return set_error(BSA_ERR_UNSUPPORTED, "blocks smaller than 128 slots need Npad <= 262144");
+  CUtensorMap tq, tk, tv;
+  if (!make_tmap(&tq, q, rows, g.D) || !make_tmap(&tk, k, rows, g.D) || !make_tmap(&tv, v, rows, g.D))
+    return set_error(BSA_ERR_CUDA, "cuTensorMapEncodeTiled failed");
+  const AttnParams p = make_params(plan, row_ptr, col_idx, per_head, scale, o, lse);
   const dim3 grid((unsigned)g.ntiles, (unsigned)g.Hh, (unsigned)g.B);
   cudaError_t e;
   if (g.D == 128)
@@ -587,6 +675,28 @@ bsa_status launch_attn_fwd(const bsa_plan_s& plan, const void* q, const void* k,
   else
     e = fine ? launch_t<64, true>(tq, tk, tv, p, grid, st) : launch_t<64, false>(tq, tk, tv, p, grid, st);
   if (e != cudaSuccess) return cuda_error(e, "attention launch");
+  return BSA_OK;
+}
+
+bsa_status launch_attn_fwd_natural(const bsa_plan_s& plan, const void* q, const void* k,
+                                   const void* v, const int32_t* row_ptr, const int32_t* col_idx,
+                                   int per_head, float scale, void* o, float* lse,
+                                   cudaStream_t st) {
+  const Geometry& g = plan.g;
+  if (g.layout != BSA_LAYOUT_TILE || g.block != kTile)
+    return set_error(BSA_ERR_UNSUPPORTED,
+                     "natural-layout attention needs a TILE plan with pool_h * pool_w = 128");
+  if ((int64_t)g.B * g.T * g.P * g.Hh >= (1ll << 31))
+    return set_error(BSA_ERR_UNSUPPORTED, "B*N*Hh must be < 2^31");
+  if ((int64_t)g.B * g.T >= (1ll << 31)) return set_error(BSA_ERR_UNSUPPORTED, "B*T must be < 2^31");
+  CUtensorMap tq, tk, tv;
+  if (!make_tmap_tiles(&tq, q, g) || !make_tmap_tiles(&tk, k, g) || !make_tmap_tiles(&tv, v, g))
+    return set_error(BSA_ERR_CUDA, "cuTensorMapEncodeTiled (5-D) failed");
+  const AttnParams p = make_params(plan, row_ptr, col_idx, per_head, scale, o, lse);
+  const dim3 grid((unsigned)g.ntiles, (unsigned)g.Hh, (unsigned)g.B);
+  const cudaError_t e = g.D == 128 ? launch_t<128, false, true>(tq, tk, tv, p, grid, st)
+                                   : launch_t<64, false, true>(tq, tk, tv, p, grid, st);
+  if (e != cudaSuccess) return cuda_error(e, "natural-layout attention launch");
   return BSA_OK;
 }
 

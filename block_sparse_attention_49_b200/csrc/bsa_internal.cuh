@@ -88,7 +88,8 @@ cudaError_t launch_reorder_inv(const Geometry& g, const void* x_slots, void* x_n
                                cudaStream_t st);
 cudaError_t launch_draft_mask(const Geometry& g, const uint32_t* tile_valid, const void* q,
                               const void* k, int keep, int pooling, int32_t* row_ptr,
-                              int32_t* kv_idx, float* draft_map, double* ws, cudaStream_t st);
+                              int32_t* kv_idx, float* draft_map, double* ws, cudaStream_t st,
+                              bool natural = false);
 
 // Anchor grid actually used for (plan variant, T_per, s): *T_per_eff = 0
 // means no anchors; also returns |G| over the plan's T frames.
@@ -96,6 +97,12 @@ int lvsa_effective_anchors(const bsa_plan_s* plan, int T_per, int s, int* T_per_
 bsa_status launch_attn_fwd(const bsa_plan_s& plan, const void* q, const void* k, const void* v,
                            const int32_t* row_ptr, const int32_t* col_idx, int per_head,
                            float scale, void* o, float* lse, cudaStream_t st);
+// The same on natural-layout [B, N, Hh, D] tensors for a TILE plan whose
+// tiles are 128 slots (pool_h * pool_w = 128); LSE as [B, Hh, N].
+bsa_status launch_attn_fwd_natural(const bsa_plan_s& plan, const void* q, const void* k,
+                                   const void* v, const int32_t* row_ptr, const int32_t* col_idx,
+                                   int per_head, float scale, void* o, float* lse,
+                                   cudaStream_t st);
 cudaError_t launch_selftest_timeout(unsigned int* status, uint64_t limit_ns, cudaStream_t st);
 
 // Size bookkeeping shared by the API and the draft kernels.

@@ -31,6 +31,7 @@ namespace {
 constexpr int kPoolThreads = 256;
 constexpr int kScoreThreads = 256;
 constexpr int kKeyChunk = 32;  // key blocks staged in shared memory per step
+constexpr int kRegCand = 16;   // top-k candidates per lane held in registers (Nb <= 512)
 
 // One group of D/8 threads per (which, b, h, block); each thread owns 8
 // channels.  which = 0: Q, 1: K.
@@ -82,6 +83,72 @@ __global__ void __launch_bounds__(kPoolThreads)
   for (int i = 0; i < 8; ++i) dst[i] = cnt ? (use_max ? acc[i] : __ddiv_rn(acc[i], dc)) : 0.0;
 }
 
+// The same pooling read straight from the natural layout [B, N, Hh, D]: one
+// group of D/8 threads per (which, block, b, h), heads fastest, so the
+// groups of a warp read neighbouring 256-byte rows of one token.  The tile's
+// tokens inside the grid are visited in row-major (a, then b) order, loads
+// eight at a time ahead of the sequential fp64 additions.
+template <int D>
+__global__ void __launch_bounds__(kPoolThreads)
+    draft_pool_nat_kernel(const uint4* __restrict__ q, const uint4* __restrict__ k, int B, int Hh,
+                          int T, int H, int W, int ph, int pw, int TH, int TW, int64_t nblocks,
+                          int64_t groups_per_tensor, int use_max, double* __restrict__ ws) {
+  constexpr int kTPG = D / 8;
+  constexpr int kAhead = 8;
+  const int64_t gid = ((int64_t)blockIdx.x * kPoolThreads + threadIdx.x) / kTPG;
+  const int sub = threadIdx.x % kTPG;
+  if (gid >= 2 * groups_per_tensor) return;
+  const int which = gid >= groups_per_tensor;
+  const int64_t gg = gid - which * groups_per_tensor;  // (blk * B + b) * Hh + h
+  const int h = (int)(gg % Hh);
+  const int64_t rest = gg / Hh;
+  const int b = (int)(rest % B);
+  const int64_t blk = rest / B;
+  const int t = (int)(blk / ((int64_t)TH * TW));
+  const int r = (int)(blk - (int64_t)t * TH * TW);
+  const int i = r / TW, j = r - (r / TW) * TW;
+  const int y0 = i * ph, x0 = j * pw;
+  const int hn = min(ph, H - y0), wn = min(pw, W - x0);
+  const int64_t N = (int64_t)T * H * W;
+  const uint4* src = (which ? k : q) + (((int64_t)b * N + ((int64_t)t * H + y0) * W + x0) * Hh + h) *
+                                           (D / 8) + sub;
+  const int64_t row_step = (int64_t)Hh * (D / 8);  // one token
+  double acc[8];
+#pragma unroll
+  for (int e = 0; e < 8; ++e) acc[e] = use_max ? -INFINITY : 0.0;
+  for (int a = 0; a < hn; ++a) {
+    const uint4* rowp = src + (int64_t)a * W * row_step;
+    for (int c0 = 0; c0 < wn; c0 += kAhead) {
+      uint4 v[kAhead];
+#pragma unroll
+      for (int u = 0; u < kAhead; ++u)
+        if (c0 + u < wn) v[u] = __ldg(rowp + (int64_t)(c0 + u) * row_step);
+#pragma unroll
+      for (int u = 0; u < kAhead; ++u) {
+        if (c0 + u >= wn) break;
+        const __nv_bfloat162* pv = reinterpret_cast<const __nv_bfloat162*>(&v[u]);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float2 f = __bfloat1622float2(pv[e]);
+          if (use_max) {
+            acc[2 * e] = fmax(acc[2 * e], (double)f.x);
+            acc[2 * e + 1] = fmax(acc[2 * e + 1], (double)f.y);
+          } else {
+            acc[2 * e] = __dadd_rn(acc[2 * e], (double)f.x);
+            acc[2 * e + 1] = __dadd_rn(acc[2 * e + 1], (double)f.y);
+          }
+        }
+      }
+    }
+  }
+  const int cnt = max(hn, 0) * max(wn, 0);
+  double* dst = ws + ((int64_t)which * groups_per_tensor + ((int64_t)b * Hh + h) * nblocks + blk) * D +
+                sub * 8;
+  const double dc = (double)cnt;
+#pragma unroll
+  for (int e = 0; e < 8; ++e) dst[e] = cnt ? (use_max ? acc[e] : __ddiv_rn(acc[e], dc)) : 0.0;
+}
+
 // grid: (ceil(nblocks / R), Hh, B); R query rows per CTA.
 template <int D>
 __global__ void __launch_bounds__(kScoreThreads)
@@ -103,55 +170,126 @@ __global__ void __launch_bounds__(kScoreThreads)
   for (int i = threadIdx.x; i < rows * nblocks; i += kScoreThreads) sel[i] = 0;
 
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  constexpr int kWarps = kScoreThreads / 32;
+  // key chunks: the next chunk is loaded into registers while the current
+  // one is used, then stored to shared memory (padded stride: no conflicts)
+  constexpr int kPer = kKeyChunk * D / kScoreThreads;
+  double pre[kPer];
+  auto load_chunk = [&](int j0) {
+#pragma unroll
+    for (int u = 0; u < kPer; ++u) {
+      const int idx = threadIdx.x + u * kScoreThreads;
+      const int jj = idx / D, c = idx - jj * D;
+      pre[u] = (j0 + jj < nblocks) ? kb[(int64_t)(j0 + jj) * D + c] : 0.0;
+    }
+  };
+  load_chunk(0);
   for (int j0 = 0; j0 < nblocks; j0 += kKeyChunk) {
     const int nj = min(kKeyChunk, nblocks - j0);
     __syncthreads();
-    for (int i = threadIdx.x; i < nj * D; i += kScoreThreads) {
-      const int jj = i / D, c = i - jj * D;
-      sk[jj * (D + 1) + c] = kb[(int64_t)(j0 + jj) * D + c];
+#pragma unroll
+    for (int u = 0; u < kPer; ++u) {
+      const int idx = threadIdx.x + u * kScoreThreads;
+      const int jj = idx / D, c = idx - jj * D;
+      sk[jj * (D + 1) + c] = pre[u];
     }
     __syncthreads();
-    // warp w handles rows w, w+8, ...; lane = key block within the chunk
+    if (j0 + kKeyChunk < nblocks) load_chunk(j0 + kKeyChunk);
+    // warp w takes rows w and w + 8 together (two independent chains);
+    // lane = key block within the chunk.  Each logit is still the sequential
+    // multiply-then-add over c.
     if (lane < nj) {
-      for (int r = warp; r < rows; r += kScoreThreads / 32) {
-        const double* a = sq + r * D;
-        const double* kk = sk + lane * (D + 1);
-        double acc = 0.0;
-        for (int c = 0; c < D; ++c) acc = __dadd_rn(acc, __dmul_rn(a[c], kk[c]));
-        sl[(int64_t)r * nblocks + j0 + lane] = acc;
+      const double* kk = sk + lane * (D + 1);
+      for (int ra = warp; ra < rows; ra += 2 * kWarps) {
+        const int rb = ra + kWarps;
+        const bool has_b = rb < rows;
+        const double* qa = sq + ra * D;
+        const double* qb2 = sq + (has_b ? rb : ra) * D;
+        double acc_a = 0.0, acc_b = 0.0;
+#pragma unroll 8
+        for (int c = 0; c < D; ++c) {
+          const double kc = kk[c];
+          acc_a = __dadd_rn(acc_a, __dmul_rn(qa[c], kc));
+          acc_b = __dadd_rn(acc_b, __dmul_rn(qb2[c], kc));
+        }
+        sl[(int64_t)ra * nblocks + j0 + lane] = acc_a;
+        if (has_b) sl[(int64_t)rb * nblocks + j0 + lane] = acc_b;
       }
     }
   }
   __syncthreads();
 
-  // top-k per row, one warp per row
-  for (int r = warp; r < rows; r += kScoreThreads / 32) {
+  // top-k per row, one warp per row: k rounds of a warp-wide arg-max (larger
+  // logit first, then the lower block index)
+  for (int r = warp; r < rows; r += kWarps) {
     const double* L = sl + (int64_t)r * nblocks;
     uint8_t* sr = sel + (int64_t)r * nblocks;
-    for (int it = 0; it < keep; ++it) {
-      double best = -DBL_MAX;
-      int bidx = 0x7fffffff;
-      for (int j = lane; j < nblocks; j += 32) {
-        if (sr[j]) continue;
-        const double v = L[j];
-        if (bidx == 0x7fffffff || v > best || (v == best && j < bidx)) {
-          best = v;
-          bidx = j;
+    if (nblocks <= 32 * kRegCand) {
+      // candidates j = lane + 32u held in registers; `avail` marks the ones
+      // not yet taken
+      double v[kRegCand];
+      uint32_t avail = 0u;
+#pragma unroll
+      for (int u = 0; u < kRegCand; ++u) {
+        const int j = lane + 32 * u;
+        v[u] = j < nblocks ? L[j] : 0.0;
+        if (j < nblocks) avail |= 1u << u;
+      }
+      const uint32_t start = avail;
+      for (int it = 0; it < keep; ++it) {
+        double best = 0.0;
+        int bidx = 0x7fffffff;
+#pragma unroll
+        for (int u = 0; u < kRegCand; ++u)
+          if (((avail >> u) & 1u) && (bidx == 0x7fffffff || v[u] > best)) {
+            best = v[u];
+            bidx = lane + 32 * u;
+          }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+          const double ov = __shfl_xor_sync(0xffffffffu, best, o);
+          const int oi = __shfl_xor_sync(0xffffffffu, bidx, o);
+          const bool take = (oi != 0x7fffffff) &&
+                            (bidx == 0x7fffffff || ov > best || (ov == best && oi < bidx));
+          if (take) {
+            best = ov;
+            bidx = oi;
+          }
         }
+        if (bidx != 0x7fffffff && (bidx & 31) == lane) avail &= ~(1u << (bidx >> 5));
       }
 #pragma unroll
-      for (int o = 16; o > 0; o >>= 1) {
-        const double ov = __shfl_xor_sync(0xffffffffu, best, o);
-        const int oi = __shfl_xor_sync(0xffffffffu, bidx, o);
-        const bool take = (oi != 0x7fffffff) &&
-                          (bidx == 0x7fffffff || ov > best || (ov == best && oi < bidx));
-        if (take) {
-          best = ov;
-          bidx = oi;
-        }
+      for (int u = 0; u < kRegCand; ++u) {
+        const int j = lane + 32 * u;
+        if (j < nblocks) sr[j] = (((start & ~avail) >> u) & 1u) ? 1 : 0;
       }
-      if (lane == 0 && bidx != 0x7fffffff) sr[bidx] = 1;
       __syncwarp();
+    } else {
+      for (int it = 0; it < keep; ++it) {
+        double best = -DBL_MAX;
+        int bidx = 0x7fffffff;
+        for (int j = lane; j < nblocks; j += 32) {
+          if (sr[j]) continue;
+          const double v = L[j];
+          if (bidx == 0x7fffffff || v > best || (v == best && j < bidx)) {
+            best = v;
+            bidx = j;
+          }
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+          const double ov = __shfl_xor_sync(0xffffffffu, best, o);
+          const int oi = __shfl_xor_sync(0xffffffffu, bidx, o);
+          const bool take = (oi != 0x7fffffff) &&
+                            (bidx == 0x7fffffff || ov > best || (ov == best && oi < bidx));
+          if (take) {
+            best = ov;
+            bidx = oi;
+          }
+        }
+        if (lane == 0 && bidx != 0x7fffffff) sr[bidx] = 1;
+        __syncwarp();
+      }
     }
     // ascending output
     const int64_t grow = bh * nblocks + r0 + r;
@@ -189,14 +327,20 @@ __global__ void __launch_bounds__(kScoreThreads)
 
 template <int D>
 cudaError_t launch_t(const Geometry& g, const uint32_t* tile_valid, const void* q, const void* k,
-                     int keep, int pooling, int32_t* row_ptr, int32_t* kv_idx, float* draft_map,
-                     double* ws, cudaStream_t st) {
+                     int keep, int pooling, bool natural, int32_t* row_ptr, int32_t* kv_idx,
+                     float* draft_map, double* ws, cudaStream_t st) {
   const int64_t groups = (int64_t)g.B * g.Hh * g.nblocks;
   const int64_t threads = 2 * groups * (D / 8);
   const unsigned pool_grid = (unsigned)((threads + kPoolThreads - 1) / kPoolThreads);
-  draft_pool_kernel<D><<<pool_grid, kPoolThreads, 0, st>>>(
-      reinterpret_cast<const uint4*>(q), reinterpret_cast<const uint4*>(k), tile_valid, g.Hh,
-      g.Npad, g.nblocks, g.block, groups, pooling == BSA_POOL_MAX ? 1 : 0, ws);
+  const int use_max = pooling == BSA_POOL_MAX ? 1 : 0;
+  if (natural)
+    draft_pool_nat_kernel<D><<<pool_grid, kPoolThreads, 0, st>>>(
+        reinterpret_cast<const uint4*>(q), reinterpret_cast<const uint4*>(k), g.B, g.Hh, g.T, g.H,
+        g.W, g.ph, g.pw, g.TH, g.TW, g.nblocks, groups, use_max, ws);
+  else
+    draft_pool_kernel<D><<<pool_grid, kPoolThreads, 0, st>>>(
+        reinterpret_cast<const uint4*>(q), reinterpret_cast<const uint4*>(k), tile_valid, g.Hh,
+        g.Npad, g.nblocks, g.block, groups, use_max, ws);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   const int R = draft_rows_per_cta(g.nblocks);
@@ -226,10 +370,13 @@ size_t draft_workspace_bytes(const Geometry& g) {
 
 cudaError_t launch_draft_mask(const Geometry& g, const uint32_t* tile_valid, const void* q,
                               const void* k, int keep, int pooling, int32_t* row_ptr,
-                              int32_t* kv_idx, float* draft_map, double* ws, cudaStream_t st) {
+                              int32_t* kv_idx, float* draft_map, double* ws, cudaStream_t st,
+                              bool natural) {
   if (g.D == 128)
-    return launch_t<128>(g, tile_valid, q, k, keep, pooling, row_ptr, kv_idx, draft_map, ws, st);
-  return launch_t<64>(g, tile_valid, q, k, keep, pooling, row_ptr, kv_idx, draft_map, ws, st);
+    return launch_t<128>(g, tile_valid, q, k, keep, pooling, natural, row_ptr, kv_idx, draft_map,
+                         ws, st);
+  return launch_t<64>(g, tile_valid, q, k, keep, pooling, natural, row_ptr, kv_idx, draft_map, ws,
+                      st);
 }
 
 }  // namespace bsa

@@ -2,8 +2,9 @@
 
 LVSA attention ("LVSA: Training-Free Sparse Attention for Long Video
 Diffusion", section 2): lvsa_mask(s) -> reorder_fwd(Q,K,V) -> attn_fwd ->
-reorder_inv(O).  Draft attention (Draft Attention article): reorder_fwd(Q,K,V)
--> draft_mask -> attn_fwd -> reorder_inv(O).
+reorder_inv(O), or the one-kernel lvsa_attn_fwd.  Draft attention (Draft
+Attention article): reorder_fwd(Q,K,V) -> draft_mask -> attn_fwd ->
+reorder_inv(O), or draft_mask_natural -> attn_fwd_natural with no reorder.
 
 torch only allocates device memory and supplies the stream; every step runs
 in libbsattn.so.
@@ -15,7 +16,8 @@ import math
 import torch
 
 from . import (ANCHORS_ROTATING, LAYOUT_FRAME, LAYOUT_TILE, POOL_MEAN, WINDOW_DISTANCE, Plan,
-               bsa_attn_fwd, bsa_draft_keep_count, bsa_draft_mask, bsa_draft_workspace_bytes,
+               bsa_attn_fwd, bsa_attn_fwd_natural, bsa_draft_keep_count, bsa_draft_mask,
+               bsa_draft_mask_natural, bsa_draft_workspace_bytes,
                bsa_lvsa_attn_fwd, bsa_lvsa_mask, bsa_lvsa_nnz, bsa_plan_set_draft_pooling,
                bsa_plan_set_lvsa_variant, bsa_reorder_fwd, bsa_reorder_inv)
 
@@ -104,3 +106,14 @@ class DraftAttention(_Base):
         self.mask()
         self.attend(per_head=True)
         return self.scatter(out)
+
+    def fused(self, q, k, v, out=None, lse=None):
+        """The same attention with no reorder: the draft mask pools the
+        natural layout in place and the attention reads and writes it
+        through tile-shaped tensor maps (pool_h * pool_w must be 128)."""
+        out = torch.empty_like(q) if out is None else out
+        bsa_draft_mask_natural(self.plan, q, k, self.sparsity, self.row_ptr, self.col_idx,
+                               self.draft_map, self.workspace)
+        bsa_attn_fwd_natural(self.plan, q, k, v, self.row_ptr, self.col_idx, True, self.scale,
+                             out, lse)
+        return out

@@ -212,6 +212,28 @@ bsa_status bsa_attn_fwd(bsa_plan_t plan, const void* q, const void* k, const voi
                         const int32_t* row_ptr, const int32_t* col_idx, int per_head_lists,
                         float scale, void* o, float* lse, void* stream);
 
+/* Draft-path attention on the natural layout: bsa_attn_fwd with the reorder
+ * of the Draft Attention article fused into the tile loads and the stores.
+ * Requires a TILE plan with pool_h * pool_w = 128 (one pooling tile per
+ * 128-slot tile; otherwise BSA_ERR_UNSUPPORTED).  q, k, v, o: natural layout
+ * [B, N, Hh, D] bf16; block i of (b, head) is the pool_h x pool_w tile
+ * (t, i_h, i_w), read through a 5-D tensor map whose part past the grid edge
+ * reads as zero; o is written for every token (nothing else).  lse:
+ * float[B*Hh*N] at (b*Hh + h)*N + n, or NULL.  Block lists, per_head_lists
+ * and scale as for bsa_attn_fwd; the result equals bsa_reorder_fwd +
+ * bsa_attn_fwd + bsa_reorder_inv bit for bit. */
+bsa_status bsa_attn_fwd_natural(bsa_plan_t plan, const void* q, const void* k, const void* v,
+                                const int32_t* row_ptr, const int32_t* col_idx, int per_head_lists,
+                                float scale, void* o, float* lse, void* stream);
+
+/* bsa_draft_mask on natural-layout q, k [B, N, Hh, D] bf16 (no reorder
+ * first): the pooling reads each tile's tokens in place, in the same order,
+ * so every output is identical to bsa_draft_mask on the reordered tensors.
+ * Requires a TILE plan; workspace as for bsa_draft_mask. */
+bsa_status bsa_draft_mask_natural(bsa_plan_t plan, const void* q, const void* k, int sparsity_pct,
+                                  int32_t* row_ptr, int32_t* kv_idx, float* draft_map,
+                                  void* workspace, size_t workspace_bytes, void* stream);
+
 /* LVSA attention in one pass on the natural layout ("LVSA", section 2 "Core
  * mechanism"; the reorder of the Draft Attention article is fused into the
  * tile loads, so no padded copies are made).

@@ -1,0 +1,149 @@
+"""The draft path on the natural layout (no reorder): bsa_draft_mask_natural
+and bsa_attn_fwd_natural.
+
+Draft Attention article: pooled Q and K give the draft map and the kept
+blocks; the reorder that makes the kept blocks contiguous is fused into the
+attention's tile loads and stores here.  Pooled values and kept blocks:
+bit-exact against the oracle.  Attention: identical, bit for bit, to the
+reorder + attn_fwd + reorder_inv path on every token (the kernels do the
+same arithmetic on the same tiles), and within max-abs 2e-2 / mean-abs 2e-3
+of the fp64 oracle.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import block_sparse_attention_49_b200 as bsa
+import oracle
+from block_sparse_attention_49_b200 import _build
+from block_sparse_attention_49_b200.pipeline import DraftAttention
+from synth import CONFIGS, make_qkv, small_workload
+
+from gpu_util import MAX_ABS, MEAN_ABS, sample_blocks, to_np64
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib():
+    _build.build()
+    bsa.load()
+
+
+CASES = [
+    dict(cid=2),                                                        # 30 x 52 grid, 8 x 16 tiles
+    dict(cid=5, Hh=6),                                                  # 40-head workload, 6 heads
+    dict(cid=2, T=3, H=13, W=37, Hh=3, field_grid=(3, 4, 7)),          # ragged edges both ways
+    dict(cid=2, T=2, H=20, W=12, Hh=2, D=64, draft_ph=16, draft_pw=8,  # transposed tile, D = 64
+         field_grid=(2, 4, 7)),
+    dict(cid=2, T=2, H=9, W=70, Hh=2, draft_ph=4, draft_pw=32, draft_sparsity=70,
+         field_grid=(2, 4, 7)),
+]
+
+
+@pytest.mark.parametrize("over", CASES)
+@pytest.mark.parametrize("pooling", [bsa.POOL_MEAN, bsa.POOL_MAX])
+def test_draft_mask_natural_bit_exact(over, pooling):
+    over = dict(over)
+    w = small_workload(CONFIGS[over.pop("cid")], **over)
+    ph, pw, sp = w.draft_ph, w.draft_pw, w.draft_sparsity
+    q, k, _ = make_qkv(w, device="cuda")
+    plan = bsa.Plan(w.B, w.Hh, w.D, w.T, w.H, w.W, bsa.LAYOUT_TILE, ph, pw, ph * pw)
+    bsa.bsa_plan_set_draft_pooling(plan, pooling)
+    keep = bsa.bsa_draft_keep_count(plan, sp)
+    nb = plan.nblocks
+    rows = w.B * w.Hh * nb
+    rp = torch.empty(rows + 1, dtype=torch.int32, device="cuda")
+    kv = torch.empty(rows * keep, dtype=torch.int32, device="cuda")
+    ws = torch.full(((bsa.bsa_draft_workspace_bytes(plan) + 7) // 8,), float("nan"),
+                    dtype=torch.float64, device="cuda")
+    bsa.bsa_draft_mask_natural(plan, q, k, sp, rp, kv, None, ws)
+    bsa.bsa_poll_status(plan)
+    mode = "max" if pooling == bsa.POOL_MAX else "mean"
+    qbar = oracle.draft_pool(to_np64(q), w.T, w.H, w.W, ph, pw, mode)
+    kbar = oracle.draft_pool(to_np64(k), w.T, w.H, w.W, ph, pw, mode)
+    got = ws.cpu().numpy()[:2 * rows * w.D].reshape(2, w.B, w.Hh, nb, w.D)
+    np.testing.assert_array_equal(got[0], qbar)
+    np.testing.assert_array_equal(got[1], kbar)
+    ref = oracle.draft_topk(oracle.draft_logits(qbar, kbar), oracle.draft_keep_count(nb, sp))
+    np.testing.assert_array_equal(kv.cpu().numpy().reshape(w.B, w.Hh, nb, keep), ref)
+
+
+@pytest.mark.parametrize("over", CASES)
+def test_attn_natural_equals_reorder_path_bitwise(over):
+    over = dict(over)
+    w = small_workload(CONFIGS[over.pop("cid")], **over)
+    q, k, v = make_qkv(w, device="cuda")
+    att = DraftAttention(w.B, w.Hh, w.D, w.T, w.H, w.W, w.draft_ph, w.draft_pw, w.draft_sparsity)
+    a = att(q, k, v)
+    lse_slots = att.lse.clone()
+    kv_a = att.col_idx.clone()
+    b = torch.full_like(q, float("nan"))
+    lse_nat = torch.full((w.B, w.Hh, w.N), float("nan"), dtype=torch.float32, device="cuda")
+    att.fused(q, k, v, b, lse_nat)
+    bsa.bsa_poll_status(att.plan)
+    assert torch.equal(att.col_idx, kv_a)                        # same kept blocks
+    assert torch.equal(a.view(torch.int16), b.view(torch.int16))  # same bits, every token
+    perm, _ = oracle.tile_layout_perm(w.T, w.H, w.W, w.draft_ph, w.draft_pw)
+    idx = torch.from_numpy(perm).cuda()
+    assert torch.equal(lse_slots[:, :, idx], lse_nat)
+
+
+@pytest.mark.parametrize("cid", [2, 5])
+def test_attn_natural_full_size_sampled_vs_oracle(cid):
+    w = CONFIGS[cid]
+    q, k, v = make_qkv(w, device="cuda")
+    att = DraftAttention(w.B, w.Hh, w.D, w.T, w.H, w.W, w.draft_ph, w.draft_pw, w.draft_sparsity)
+    out = att.fused(q, k, v)
+    bsa.bsa_poll_status(att.plan)
+    ph, pw = w.draft_ph, w.draft_pw
+    perm, Np = oracle.tile_layout_perm(w.T, w.H, w.W, ph, pw)
+    valid = oracle.slot_valid(perm, Np)
+    nb = Np // (ph * pw)
+    heads = [0, w.Hh - 1]
+    qn, kn, vn = (to_np64(x[:, :, heads]) for x in (q, k, v))
+    kv = oracle.draft_blocks(qn, kn, w.T, w.H, w.W, ph, pw, w.draft_sparsity)
+    np.testing.assert_array_equal(att.col_idx.view(w.B, w.Hh, nb, -1)[:, heads].cpu().numpy(), kv)
+    rp, ci = oracle.fixed_k_csr(kv)
+    O, _ = oracle.masked_attention(*(oracle.reorder_fwd(x, perm, Np) for x in (qn, kn, vn)),
+                                   valid, ph * pw, rp, ci, True, 1 / math.sqrt(w.D),
+                                   q_blocks=sample_blocks(nb, 6, seed=cid))
+    ref = oracle.reorder_inv(np.nan_to_num(O, nan=np.inf), perm)
+    got = to_np64(out[:, :, heads])
+    m = np.isfinite(ref)
+    err = np.abs(got[m] - ref[m])
+    assert m.any() and err.max() <= MAX_ABS and err.mean() <= MEAN_ABS
+
+
+def test_attn_natural_rejects_unsupported_plans():
+    x = torch.zeros((1, 512, 1, 64), dtype=torch.bfloat16, device="cuda")
+    buf = torch.zeros(4096, dtype=torch.int32, device="cuda")
+    fplan = bsa.Plan(1, 1, 64, 8, 8, 8, bsa.LAYOUT_FRAME, block=64)
+    with pytest.raises(bsa.BsaError) as ei:
+        bsa.bsa_attn_fwd_natural(fplan, x, x, x, buf, buf, True, 0.125, x)
+    assert ei.value.status == 1
+    tplan = bsa.Plan(1, 1, 64, 8, 8, 8, bsa.LAYOUT_TILE, 2, 2, 4)     # 4-token tiles
+    with pytest.raises(bsa.BsaError) as ei:
+        bsa.bsa_attn_fwd_natural(tplan, x, x, x, buf, buf, True, 0.125, x)
+    assert ei.value.status == 2
+
+
+def test_draft_mask_many_blocks_takes_the_shared_memory_selection():
+    # 2 x 64 x 64 grid with 2 x 2 tiles: 2048 blocks per row, more than the
+    # register-held candidates of the top-k, so the other selection path runs
+    w = small_workload(CONFIGS[1], T=2, H=64, W=64, Hh=1, D=64, qk="iid", draft_ph=2, draft_pw=2,
+                       draft_sparsity=95)
+    q, k, _ = make_qkv(w, device="cuda")
+    plan = bsa.Plan(w.B, w.Hh, w.D, w.T, w.H, w.W, bsa.LAYOUT_TILE, 2, 2, 4)
+    nb = plan.nblocks
+    assert nb == 2048
+    keep = bsa.bsa_draft_keep_count(plan, 95)
+    kv = torch.empty(nb * keep, dtype=torch.int32, device="cuda")
+    ws = torch.empty(((bsa.bsa_draft_workspace_bytes(plan) + 7) // 8,), dtype=torch.float64,
+                     device="cuda")
+    bsa.bsa_draft_mask_natural(plan, q, k, 95, None, kv, None, ws)
+    bsa.bsa_poll_status(plan)
+    ref = oracle.draft_blocks(to_np64(q), to_np64(k), w.T, w.H, w.W, 2, 2, 95)
+    np.testing.assert_array_equal(kv.cpu().numpy().reshape(1, 1, nb, keep), ref)
