@@ -309,6 +309,23 @@ def kernel_table(args):
                  flops=draft_attended_flops(w, kv_host, att.keep))
             emit(cid, "reorder_inv (tile layout, O)", timed(lambda: att.scatter(out)),
                  2 * tok_bytes)
+            if w.draft_ph * w.draft_pw == 128:
+                # the same path with no reorder: pooling and attention on the natural layout
+                emit(cid, "draft_mask_natural (pool in place + score/top-k)",
+                     timed(lambda: bsa.bsa_draft_mask_natural(att.plan, q, k, att.sparsity,
+                                                              att.row_ptr, att.col_idx, None,
+                                                              att.workspace)),
+                     2 * tok_bytes + 2 * pooled + 4 * att.col_idx.numel())
+                emit(cid, "attn_fwd_natural (draft, 5-D tile loads, token-order stores)",
+                     timed(lambda: bsa.bsa_attn_fwd_natural(att.plan, q, k, v, att.row_ptr,
+                                                            att.col_idx, True, scale, out)),
+                     flops=draft_attended_flops(w, kv_host, att.keep))
+                emit(cid, "draft pipeline, reorder path (reorder, mask, attention, inverse)",
+                     timed(lambda: att(q, k, v, out)),
+                     flops=draft_attended_flops(w, kv_host, att.keep))
+                emit(cid, "draft pipeline, natural layout (mask, attention)",
+                     timed(lambda: att.fused(q, k, v, out)),
+                     flops=draft_attended_flops(w, kv_host, att.keep))
             bsa.bsa_poll_status(att.plan)
             del att
         del q, k, v, out
