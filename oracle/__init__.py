@@ -14,7 +14,8 @@ what the method computes, written from the pages:
   端到端加速", 163.com): tokens reshaped to [t,h,w], average-pooled Q and K give
   a low-resolution draft attention map, which yields a sparse mask that guides
   full-resolution block-sparse attention; pool_h x pool_w = block_size; a
-  reorder makes the selected blocks contiguous.
+  reorder makes the selected blocks contiguous; quantization is named as the
+  next step.
 
 All floating point is fp64.  bf16 inputs convert to fp64 exactly.
 
@@ -34,7 +35,10 @@ Readings of points the pages leave open (each listed in the design notes):
 * top-k per query-block row keeps k = ceil(Nb*(100-p)/100) blocks ranked by
   (logit descending, block index ascending), returned in ascending order;
 * a query with no allowed valid key gets O = 0 and LSE = -inf; pad query
-  slots likewise.
+  slots likewise;
+* fp8 (quantization, the Draft article's next step): e4m3 values, one scale
+  per (batch, head) and tensor, scale = fp32(amax)/448, x/scale in fp32
+  rounded to nearest even and saturated at +-448.
 
 Parity status: every function here is pinned by tests/test_oracle_pins.py.
 """
@@ -396,3 +400,49 @@ def attended_pairs(valid: np.ndarray, block: int, row_ptr, col_idx, nlists: int 
         qb = r % nb
         total += int(vcount[qb]) * int(vcount[ci[rp[r]:rp[r + 1]]].sum())
     return total
+
+
+# ---------------------------------------------------------------------------
+# FP8 (Draft Attention article, closing paragraph: the authors' next step is
+# to bring quantization into Draft Attention).  The article fixes no format;
+# the reading taken: Q, K, V in e4m3 (1 sign, 4 exponent bits with bias 7, 3
+# mantissa bits, no infinities, largest finite 448), one scale per
+# (batch, head) and tensor, scale = fp32(amax) / 448 in fp32 (1 when amax is
+# 0), values divided by the scale in fp32 and rounded to the nearest e4m3
+# value, ties to even, saturating at +-448.
+# ---------------------------------------------------------------------------
+
+E4M3_MAX = 448.0
+
+
+def e4m3_round(x) -> np.ndarray:
+    """Nearest e4m3 value (ties to even), saturating at +-448, as fp64.
+
+    Normal e4m3 values in [2^e, 2^(e+1)) (e >= -6) are spaced 2^(e-3);
+    below 2^-6 the subnormals are spaced 2^-9.
+    """
+    x = np.asarray(x, dtype=np.float64)
+    a = np.abs(x)
+    _, ex = np.frexp(np.where(a > 0, a, 1.0))       # a = m * 2^ex, m in [0.5, 1)
+    quantum = np.where(a >= 2.0 ** -6, np.ldexp(1.0, ex - 1 - 3), 2.0 ** -9)
+    r = np.round(a / quantum) * quantum              # np.round: ties to even
+    r = np.minimum(r, E4M3_MAX)
+    return np.copysign(r, x)
+
+
+def fp8_scales(x_nat: np.ndarray) -> np.ndarray:
+    """fp32 [B, Hh]: fp32(max |x| over tokens and channels) / 448 (fp32 division)."""
+    amax = np.abs(np.asarray(x_nat, dtype=np.float64)).max(axis=(1, 3)).astype(np.float32)
+    s = amax / np.float32(E4M3_MAX)
+    return np.where(amax == 0, np.float32(1.0), s).astype(np.float32)
+
+
+def fp8_quantize(x_nat: np.ndarray, scales: np.ndarray) -> np.ndarray:
+    """e4m3 codes' values (fp64) of x / scale, the division in fp32: [B, N, Hh, D]."""
+    y = np.asarray(x_nat, dtype=np.float32) / scales[:, None, :, None]
+    return e4m3_round(y.astype(np.float64))
+
+
+def fp8_dequantize(q_vals: np.ndarray, scales: np.ndarray) -> np.ndarray:
+    """The values the fp8 attention computes with: q * scale, fp64 [B, N, Hh, D]."""
+    return q_vals * scales.astype(np.float64)[:, None, :, None]

@@ -542,3 +542,58 @@ def test_max_pool_brute_force_and_bounds_mean():
                     for c in range(w.D):
                         vals = sorted(tile[:, :, h, c].reshape(-1).tolist())
                         assert mx[0, h, (t * 4 + i) * 4 + j, c] == vals[-1]
+
+
+# ---------------------------------------------------------------------------
+# FP8 e4m3 (Draft Attention article: quantization as the next step)
+# ---------------------------------------------------------------------------
+
+
+def test_e4m3_grid_is_every_finite_bit_pattern():
+    # torch's float8_e4m3fn decoding of all 256 codes is the library reference
+    codes = torch.arange(256, dtype=torch.int32).to(torch.uint8).view(torch.float8_e4m3fn)
+    vals = codes.to(torch.float64).numpy()
+    fin = np.isfinite(vals)
+    assert fin.sum() == 254                      # 0x7f and 0xff are NaN
+    assert np.array_equal(oracle.e4m3_round(vals[fin]), vals[fin])   # the grid maps to itself
+    assert vals[fin].max() == 448.0 and sorted(set(np.abs(vals[fin])))[1] == 2.0 ** -9
+
+
+def test_e4m3_round_matches_library_cast():
+    rng = np.random.default_rng(5)
+    x = np.concatenate([rng.normal(0, 1, 20000), rng.normal(0, 60, 20000),
+                        rng.uniform(-464, 464, 20000), rng.normal(0, 2.0 ** -8, 20000),
+                        np.ldexp(rng.integers(-64, 64, 4000) + 0.5, -10)])   # exact ties
+    ref = torch.from_numpy(x).to(torch.float8_e4m3fn).to(torch.float64).numpy()
+    np.testing.assert_array_equal(oracle.e4m3_round(x), ref)
+    # beyond the largest finite value the rounding saturates
+    assert (oracle.e4m3_round(np.array([480.0, 1e6, -1e9])) == [448.0, 448.0, -448.0]).all()
+
+
+def test_fp8_scales_and_quantize():
+    rng = np.random.default_rng(6)
+    x = rng.normal(0, 1, (2, 40, 3, 16)).astype(np.float32).astype(np.float64)
+    x[1, :, 2] = 0.0                                    # an all-zero head: scale 1
+    s = oracle.fp8_scales(x)
+    assert s.dtype == np.float32 and s[1, 2] == 1.0
+    amax = np.abs(x).max(axis=(1, 3)).astype(np.float32)
+    assert s[0, 0] == np.float32(amax[0, 0]) / np.float32(448.0)
+    q = oracle.fp8_quantize(x, s)
+    # the largest |x| of a head lands on +-448 (within the fp32 division's rounding)
+    qmax = np.abs(q).max(axis=(1, 3))
+    assert (qmax[s != 1.0] >= 416.0).all() and (qmax <= 448.0).all()
+    # values are on the e4m3 grid, and dequantized values are within half a step
+    assert np.array_equal(oracle.e4m3_round(q), q)
+    deq = oracle.fp8_dequantize(q, s)
+    step = np.maximum(np.ldexp(1.0, np.frexp(np.abs(q) + 1e-300)[1] - 4), 2.0 ** -9)
+    assert (np.abs(deq - x) <= 0.5 * step * s.astype(np.float64)[:, None, :, None] * (1 + 1e-6)
+            + 1e-12).all()
+
+
+def test_fp8_quantize_is_exact_for_values_on_the_grid_with_power_of_two_scales():
+    # amax 448 * 2^-5 gives scale 2^-5 exactly; e4m3 values times 2^-5 survive
+    grid = oracle.e4m3_round(np.linspace(-448, 448, 301))
+    x = (grid * 2.0 ** -5).reshape(1, 301, 1, 1)
+    s = oracle.fp8_scales(x)
+    assert s[0, 0] == np.float32(2.0 ** -5)
+    np.testing.assert_array_equal(oracle.fp8_dequantize(oracle.fp8_quantize(x, s), s), x)
