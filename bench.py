@@ -326,6 +326,18 @@ def kernel_table(args):
                 emit(cid, "draft pipeline, natural layout (mask, attention)",
                      timed(lambda: att.fused(q, k, v, out)),
                      flops=draft_attended_flops(w, kv_host, att.keep))
+                if w.D == 128:
+                    # 8-bit attention: e4m3 Q, K, V (read twice, written at 1 byte)
+                    emit(cid, "quantize_e4m3 (Q K V, per-head scales)",
+                         timed(lambda: att.quantize(q, k, v)), 3 * tok_bytes + 3 * tok_bytes // 2)
+                    emit(cid, "attn_fwd_natural_e4m3 (8-bit QK and PV)",
+                         timed(lambda: bsa.bsa_attn_fwd_natural_e4m3(
+                             att.plan, att.q8, att.k8, att.v8, att.fp8_scales, att.row_ptr,
+                             att.col_idx, True, scale, out)),
+                         flops=draft_attended_flops(w, kv_host, att.keep))
+                    emit(cid, "draft pipeline, 8-bit (mask, quantize, attention)",
+                         timed(lambda: att.fused_e4m3(q, k, v, out)),
+                         flops=draft_attended_flops(w, kv_host, att.keep))
             bsa.bsa_poll_status(att.plan)
             del att
         del q, k, v, out

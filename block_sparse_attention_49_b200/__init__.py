@@ -26,7 +26,8 @@ __all__ = [
     "bsa_block_size", "bsa_lvsa_mask", "bsa_lvsa_nnz", "bsa_draft_keep_count",
     "bsa_draft_workspace_bytes", "bsa_draft_mask", "bsa_draft_mask_noalloc",
     "bsa_draft_noalloc_max_scratch_bytes", "bsa_reorder_fwd", "bsa_reorder_inv",
-    "bsa_attn_fwd", "bsa_attn_fwd_natural", "bsa_draft_mask_natural", "bsa_lvsa_attn_fwd", "bsa_poll_status", "bsa_set_wait_limit_ns", "bsa_selftest_timeout",
+    "bsa_attn_fwd", "bsa_attn_fwd_natural", "bsa_draft_mask_natural", "bsa_quantize_e4m3",
+    "bsa_attn_fwd_natural_e4m3", "bsa_lvsa_attn_fwd", "bsa_poll_status", "bsa_set_wait_limit_ns", "bsa_selftest_timeout",
     "bsa_last_error", "bsa_version", "EXPORTED_SYMBOLS",
 ]
 
@@ -69,6 +70,9 @@ _SIGS = {
     "bsa_attn_fwd_natural": (_c_int, [_c_p, _c_p, _c_p, _c_p, _c_p, _c_p, _c_int, ctypes.c_float, _c_p,
                               _c_p, _c_p]),
     "bsa_draft_mask_natural": (_c_int, [_c_p, _c_p, _c_p, _c_int, _c_p, _c_p, _c_p, _c_p, _c_sz, _c_p]),
+    "bsa_quantize_e4m3": (_c_int, [_c_p] * 9),
+    "bsa_attn_fwd_natural_e4m3": (_c_int, [_c_p, _c_p, _c_p, _c_p, _c_p, _c_p, _c_p, _c_int,
+                                           ctypes.c_float, _c_p, _c_p, _c_p]),
     "bsa_lvsa_attn_fwd": (_c_int, [_c_p, _c_int, _c_int, _c_int, _c_p, _c_p, _c_p, ctypes.c_float,
                                    _c_p, _c_p, _c_p]),
     "bsa_poll_status": (_c_int, [_c_p, _c_p]),
@@ -246,6 +250,23 @@ def bsa_draft_mask_natural(plan: Plan, q, k, sparsity_pct: int, row_ptr, kv_idx,
                                          _ptr(row_ptr), _ptr(kv_idx), _ptr(draft_map),
                                          _ptr(workspace), nbytes, _stream(stream)),
            "bsa_draft_mask_natural")
+
+
+def bsa_quantize_e4m3(plan: Plan, q, k, v, q8, k8, v8, scales, stream=None):
+    """e4m3 copies of natural-layout q, k, v (uint8 tensors) and their
+    per-(tensor, batch, head) scales (float32 [3, B, Hh])."""
+    _check(load().bsa_quantize_e4m3(plan.handle, _ptr(q), _ptr(k), _ptr(v), _ptr(q8), _ptr(k8),
+                                    _ptr(v8), _ptr(scales), _stream(stream)), "bsa_quantize_e4m3")
+
+
+def bsa_attn_fwd_natural_e4m3(plan: Plan, q8, k8, v8, scales, row_ptr, col_idx,
+                              per_head_lists: bool, scale: float, o, lse=None, stream=None):
+    """bsa_attn_fwd_natural on e4m3 inputs from bsa_quantize_e4m3 (8-bit MMAs)."""
+    _check(load().bsa_attn_fwd_natural_e4m3(plan.handle, _ptr(q8), _ptr(k8), _ptr(v8),
+                                            _ptr(scales), _ptr(row_ptr), _ptr(col_idx),
+                                            int(bool(per_head_lists)), float(scale), _ptr(o),
+                                            _ptr(lse), _stream(stream)),
+           "bsa_attn_fwd_natural_e4m3")
 
 
 def bsa_lvsa_attn_fwd(plan: Plan, C: int, T_per: int, s: int, q, k, v, scale: float, o,

@@ -148,9 +148,11 @@ bsa_status bsa_plan_create(bsa_plan_t* plan, int B, int Hh, int D, int T, int H,
     e = cudaMemcpy(p->d_tile_valid, tv.data(), tv.size() * sizeof(uint32_t), cudaMemcpyHostToDevice);
   if (e == cudaSuccess) e = cudaMalloc(&p->d_status, sizeof(unsigned int));
   if (e == cudaSuccess) e = cudaMemset(p->d_status, 0, sizeof(unsigned int));
+  if (e == cudaSuccess) e = cudaMalloc(&p->d_amax, sizeof(uint32_t) * 3 * B * Hh);
   if (e != cudaSuccess) {
     if (p->d_tile_valid) cudaFree(p->d_tile_valid);
     if (p->d_status) cudaFree(p->d_status);
+    if (p->d_amax) cudaFree(p->d_amax);
     delete p;
     return cuda_error(e, "plan allocation");
   }
@@ -165,6 +167,7 @@ bsa_status bsa_plan_destroy(bsa_plan_t plan) {
   cudaSetDevice(plan->device);
   cudaFree(plan->d_tile_valid);
   cudaFree(plan->d_status);
+  cudaFree(plan->d_amax);
   cudaSetDevice(cur);
   delete plan;
   return BSA_OK;
@@ -320,6 +323,42 @@ bsa_status bsa_draft_mask_natural(bsa_plan_t plan, const void* q, const void* k,
                                     kv_idx, draft_map, reinterpret_cast<double*>(workspace),
                                     reinterpret_cast<cudaStream_t>(stream), /*natural=*/true);
   return e == cudaSuccess ? BSA_OK : cuda_error(e, "draft_mask_natural launch");
+}
+
+bsa_status bsa_quantize_e4m3(bsa_plan_t plan, const void* q, const void* k, const void* v, void* q8,
+                             void* k8, void* v8, float* scales, void* stream) {
+  if (!plan) return set_error(BSA_ERR_INVALID_ARG, "plan is NULL");
+  bsa_status st;
+  if ((st = check_ptr(q, "q")) != BSA_OK || (st = check_ptr(k, "k")) != BSA_OK ||
+      (st = check_ptr(v, "v")) != BSA_OK || (st = check_ptr(q8, "q8")) != BSA_OK ||
+      (st = check_ptr(k8, "k8")) != BSA_OK || (st = check_ptr(v8, "v8")) != BSA_OK)
+    return st;
+  if (!scales || (reinterpret_cast<uintptr_t>(scales) & 3u))
+    return set_error(BSA_ERR_ALIGNMENT, "scales is NULL or not 4-byte aligned");
+  cudaError_t e = launch_quantize_e4m3(plan->g, plan->d_amax, q, k, v, q8, k8, v8, scales,
+                                       reinterpret_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? BSA_OK : cuda_error(e, "quantize_e4m3 launch");
+}
+
+bsa_status bsa_attn_fwd_natural_e4m3(bsa_plan_t plan, const void* q8, const void* k8,
+                                     const void* v8, const float* scales, const int32_t* row_ptr,
+                                     const int32_t* col_idx, int per_head_lists, float scale,
+                                     void* o, float* lse, void* stream) {
+  if (!plan) return set_error(BSA_ERR_INVALID_ARG, "plan is NULL");
+  if (plan->g.layout != BSA_LAYOUT_TILE)
+    return set_error(BSA_ERR_INVALID_ARG, "e4m3 attention needs a TILE plan");
+  bsa_status st;
+  if ((st = check_ptr(q8, "q8")) != BSA_OK || (st = check_ptr(k8, "k8")) != BSA_OK ||
+      (st = check_ptr(v8, "v8")) != BSA_OK || (st = check_ptr(o, "o")) != BSA_OK)
+    return st;
+  if (!scales || (reinterpret_cast<uintptr_t>(scales) & 3u))
+    return set_error(BSA_ERR_ALIGNMENT, "scales is NULL or not 4-byte aligned");
+  if (!row_ptr || !col_idx) return set_error(BSA_ERR_INVALID_ARG, "row_ptr / col_idx is NULL");
+  if (lse && (reinterpret_cast<uintptr_t>(lse) & 3u))
+    return set_error(BSA_ERR_ALIGNMENT, "lse is not 4-byte aligned");
+  if (!(scale > 0.f)) return set_error(BSA_ERR_INVALID_ARG, "scale must be positive");
+  return launch_attn_fwd_natural_e4m3(*plan, q8, k8, v8, scales, row_ptr, col_idx, per_head_lists,
+                                      scale, o, lse, reinterpret_cast<cudaStream_t>(stream));
 }
 
 bsa_status bsa_poll_status(bsa_plan_t plan, void* stream) {

@@ -42,13 +42,16 @@ constexpr int kThreads = 384;
 constexpr int kFineMaxTiles = 2048; // key tiles addressable by the sub-tile-block path
 constexpr uint32_t kFull = 0xffffffffu;
 
-template <int D, bool FINE>
+template <int D, bool FINE, bool F8 = false>
 struct AttnCfg {
-  static constexpr int kChunks = D / 64;  // 64-column (128-byte) swizzle panels
+  static constexpr int kElem = F8 ? 1 : 2;           // bytes per element
+  static constexpr int kChunkElems = 128 / kElem;    // elements per 128-byte swizzle row
+  static constexpr int kChunks = D / kChunkElems;    // 128-byte-wide swizzle panels
   static constexpr int kPanel = kTile * 128;
-  static constexpr int kQBytes = kTile * D * 2;
-  static constexpr int kKVBytes = kTile * D * 2;
-  static constexpr int NS = (D == 128) ? (FINE ? 2 : 3) : 4;
+  static constexpr int kQBytes = kTile * D * kElem;
+  static constexpr int kKVBytes = kTile * D * kElem;
+  static constexpr int kKeysPerMma = 32 / kElem;     // K of one MMA: 16 (bf16) or 32 (e4m3)
+  static constexpr int NS = F8 ? 4 : (D == 128) ? (FINE ? 2 : 3) : 4;
   static constexpr int kOffQ = 0;
   static constexpr int kOffK = kQBytes;
   static constexpr int kOffV = kOffK + NS * kKVBytes;
@@ -81,7 +84,8 @@ struct AttnParams {
   unsigned int* status;
   uint64_t wait_limit_ns;
   // natural layout (NAT): [B, N, Hh, D] in and out; tile = one ph x pw tile
-  int T, H, W, N, TW, ph, pw;
+  int B, T, H, W, N, TW, ph, pw;
+  const float* fp8_scales;  // F8: [3][B][Hh] scales of Q, K, V
   FastDiv div_tile_frame, div_TW, div_pw;  // by TH*TW, TW, pw
 };
 
@@ -99,6 +103,14 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return *reinterpret_cast<uint32_t*>(&v);
 }
 
+// Two floats to two e4m3 bytes (nearest, ties to even, saturating at +-448),
+// lo in the low byte.
+__device__ __forceinline__ uint32_t pack_e4m3x2(float lo, float hi) {
+  uint16_t r;
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+
 __device__ __forceinline__ void softmax_groups_sync() {
   asm volatile("bar.sync 1, 256;" ::: "memory");  // warps 4-11
 }
@@ -108,11 +120,12 @@ __device__ __forceinline__ void cta_end_sync() {
   asm volatile("bar.sync 2, 384;" ::: "memory");
 }
 
-template <int D, bool FINE, bool NAT>
+template <int D, bool FINE, bool NAT, bool F8 = false>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmk,
                     const __grid_constant__ CUtensorMap tmv, const AttnParams p) {
-  using Cfg = AttnCfg<D, FINE>;
+  using Cfg = AttnCfg<D, FINE, F8>;
+  static_assert(!F8 || (NAT && D == 128), "the e4m3 path reads the natural layout, D = 128");
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
@@ -251,7 +264,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           int x0, y0, fr;
           nat_coords(qt, x0, y0, fr);
           for (int c = 0; c < Cfg::kChunks; ++c)
-            tma_load_5d(sQ + c * Cfg::kPanel, &tmq, q_full, c * 64, h, x0, y0, fr);
+            tma_load_5d(sQ + c * Cfg::kPanel, &tmq, q_full, c * Cfg::kChunkElems, h, x0, y0, fr);
         } else {
           for (int c = 0; c < Cfg::kChunks; ++c)
             tma_load_2d(sQ + c * Cfg::kPanel, &tmq, q_full, c * 64,
@@ -276,10 +289,12 @@ __global__ void __launch_bounds__(kThreads, 1)
             nat_coords(kt, x0, y0, fr);
             mbar_arrive_expect_tx(&k_full[st], Cfg::kKVBytes);
             for (int c = 0; c < Cfg::kChunks; ++c)
-              tma_load_5d(sK + c * Cfg::kPanel, &tmk, &k_full[st], c * 64, h, x0, y0, fr);
+              tma_load_5d(sK + c * Cfg::kPanel, &tmk, &k_full[st], c * Cfg::kChunkElems, h, x0, y0,
+                          fr);
             mbar_arrive_expect_tx(&v_full[st], Cfg::kKVBytes);
             for (int c = 0; c < Cfg::kChunks; ++c)
-              tma_load_5d(sV + c * Cfg::kPanel, &tmv, &v_full[st], c * 64, h, x0, y0, fr);
+              tma_load_5d(sV + c * Cfg::kPanel, &tmv, &v_full[st], c * Cfg::kChunkElems, h, x0, y0,
+                          fr);
           } else {
             mbar_arrive_expect_tx(&k_full[st], Cfg::kKVBytes);
             for (int c = 0; c < Cfg::kChunks; ++c)
@@ -308,8 +323,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       // -------------------------------------------------------- MMA issuer
       // the whole warp runs the loop (descriptors stay warp-uniform); the
       // elected lane issues the tcgen05 instructions
-      constexpr uint32_t idesc_qk = idesc_bf16(128, 128, 0);
-      constexpr uint32_t idesc_pv = idesc_bf16(128, D, 1);
+      constexpr uint32_t idesc_qk = F8 ? idesc_e4m3(128, 128, 0) : idesc_bf16(128, 128, 0);
+      constexpr uint32_t idesc_pv = F8 ? idesc_e4m3(128, D, 1) : idesc_bf16(128, D, 1);
       const uint64_t qd = sdesc_sw128(smem_u32(sQ), 16, 1024);
       const uint64_t kd0 = sdesc_sw128(smem_u32(smem + Cfg::kOffK), 16, 1024);
       const uint64_t vd0 = sdesc_sw128(smem_u32(smem + Cfg::kOffV), Cfg::kPanel, 1024);
@@ -317,9 +332,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint64_t kd = sdesc_add(kd0, st * Cfg::kKVBytes);
         if (elect_one()) {
 #pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
+          for (int kk = 0; kk < D / Cfg::kKeysPerMma; ++kk) {
+            // K step kk: 32 bytes along the 128-byte swizzle row, then the next panel
             const uint32_t off = (kk >> 2) * Cfg::kPanel + (kk & 3) * 32;
-            mma_ss(tdst, sdesc_add(qd, off), sdesc_add(kd, off), idesc_qk, kk > 0);
+            if constexpr (F8)
+              mma_ss_f8(tdst, sdesc_add(qd, off), sdesc_add(kd, off), idesc_qk, kk > 0);
+            else
+              mma_ss(tdst, sdesc_add(qd, off), sdesc_add(kd, off), idesc_qk, kk > 0);
           }
         }
         __syncwarp();
@@ -328,8 +347,16 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint64_t vd = sdesc_add(vd0, st * Cfg::kKVBytes);
         if (elect_one()) {
 #pragma unroll
-          for (int kk = 0; kk < kTile / 16; ++kk)
-            mma_ts(tO, tP + kk * 8, sdesc_add(vd, kk * 2048), idesc_pv, (acc | (uint32_t)kk) != 0);
+          for (int kk = 0; kk < kTile / Cfg::kKeysPerMma; ++kk) {
+            // K step kk: the next kKeysPerMma keys = 8 TMEM columns of P and
+            // kKeysPerMma 128-byte rows of V
+            if constexpr (F8)
+              mma_ts_f8(tO, tP + kk * 8, sdesc_add(vd, kk * Cfg::kKeysPerMma * 128), idesc_pv,
+                        (acc | (uint32_t)kk) != 0);
+            else
+              mma_ts(tO, tP + kk * 8, sdesc_add(vd, kk * Cfg::kKeysPerMma * 128), idesc_pv,
+                     (acc | (uint32_t)kk) != 0);
+          }
         }
         __syncwarp();
       };
@@ -377,7 +404,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t lane_off = (uint32_t)(q4 * 32) << 16;
     const uint32_t tS = tbase + g * 128 + lane_off;
     const uint32_t tO = tbase + 256 + g * 128 + lane_off;
-    const float sl2 = p.scale_log2;
+    // e4m3: S holds q8.k8; the scores are S * sq * sk
+    const float sqk = F8 ? p.fp8_scales[(int64_t)b * p.Hh + h] *
+                               p.fp8_scales[((int64_t)p.B + b) * p.Hh + h]
+                         : 1.f;
+    const float sl2 = p.scale_log2 * sqk;
     const float thr = 8.0f / sl2;  // rescale O when the max grows by more than 2^8
     float m_run = -INFINITY, l_run = 0.f;
     int64_t fptr = 0, fend = 0;
@@ -469,12 +500,25 @@ __global__ void __launch_bounds__(kThreads, 1)
       const float ms = (m_run == -INFINITY) ? 0.f : m_run * sl2;
       uint32_t pk[64];
       float l8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};  // independent partial sums
+      if constexpr (F8) {
+        // P as e4m3 bytes, four keys to a word (P <= 2^8 < 448)
 #pragma unroll
-      for (int i = 0; i < 64; ++i) {
-        const float p0 = ex2_approx(fmaf(s[2 * i], sl2, -ms));
-        const float p1 = ex2_approx(fmaf(s[2 * i + 1], sl2, -ms));
-        l8[i & 7] += p0 + p1;
-        pk[i] = pack_bf16x2(p0, p1);
+        for (int i = 0; i < 32; ++i) {
+          const float p0 = ex2_approx(fmaf(s[4 * i], sl2, -ms));
+          const float p1 = ex2_approx(fmaf(s[4 * i + 1], sl2, -ms));
+          const float p2 = ex2_approx(fmaf(s[4 * i + 2], sl2, -ms));
+          const float p3 = ex2_approx(fmaf(s[4 * i + 3], sl2, -ms));
+          l8[i & 7] += (p0 + p1) + (p2 + p3);
+          pk[i] = pack_e4m3x2(p0, p1) | (pack_e4m3x2(p2, p3) << 16);
+        }
+      } else {
+#pragma unroll
+        for (int i = 0; i < 64; ++i) {
+          const float p0 = ex2_approx(fmaf(s[2 * i], sl2, -ms));
+          const float p1 = ex2_approx(fmaf(s[2 * i + 1], sl2, -ms));
+          l8[i & 7] += p0 + p1;
+          pk[i] = pack_bf16x2(p0, p1);
+        }
       }
       l_run += ((l8[0] + l8[1]) + (l8[2] + l8[3])) + ((l8[4] + l8[5]) + (l8[6] + l8[7]));
       // O of this group holds every earlier PV of the group: S(j) was written
@@ -490,7 +534,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
       tmem_st32(tS + 64, *reinterpret_cast<uint32_t(*)[32]>(&pk[0]));
-      tmem_st32(tS + 96, *reinterpret_cast<uint32_t(*)[32]>(&pk[32]));
+      if constexpr (!F8) tmem_st32(tS + 96, *reinterpret_cast<uint32_t(*)[32]>(&pk[32]));
       tc_fence_before();
       mbar_arrive(&p_ready[g]);
     }
@@ -515,7 +559,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t qw = (row < 32) ? tq.x : (row < 64) ? tq.y : (row < 96) ? tq.z : tq.w;
     const bool qvalid = (qw >> (row & 31)) & 1u;
     const bool has = alive && n > 0 && qvalid && l > 0.f;
-    const float inv_l = has ? 1.f / l : 0.f;
+    // e4m3: O holds P.v8; the values are O * sv
+    const float sv = F8 ? p.fp8_scales[(2 * (int64_t)p.B + b) * p.Hh + h] : 1.f;
+    const float inv_l = has ? sv / l : 0.f;
     const float wa = a * inv_l, wb = bb * inv_l;
     int64_t orow = bh_row + (int64_t)qt * kTile + row;  // slot row, or natural token row
     int64_t lrow = orow;                                 // LSE index
@@ -588,11 +634,11 @@ bool make_tmap(CUtensorMap* m, const void* ptr, int64_t rows, int D) {
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int D, bool FINE, bool NAT = false>
+template <int D, bool FINE, bool NAT = false, bool F8 = false>
 cudaError_t launch_t(const CUtensorMap& q, const CUtensorMap& k, const CUtensorMap& v,
                      const AttnParams& p, dim3 grid, cudaStream_t st) {
-  using Cfg = AttnCfg<D, FINE>;
-  auto kern = attn_fwd_kernel<D, FINE, NAT>;
+  using Cfg = AttnCfg<D, FINE, F8>;
+  auto kern = attn_fwd_kernel<D, FINE, NAT, F8>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::kSmem);
   if (e != cudaSuccess) return e;
   kern<<<grid, kThreads, Cfg::kSmem, st>>>(q, k, v, p);
@@ -622,6 +668,8 @@ AttnParams make_params(const bsa_plan_s& plan, const int32_t* row_ptr, const int
   p.tile_valid = plan.d_tile_valid;
   p.status = plan.d_status;
   p.wait_limit_ns = plan.wait_limit_ns;
+  p.B = g.B;
+  p.fp8_scales = nullptr;
   p.T = g.T;
   p.H = g.H;
   p.W = g.W;
@@ -639,16 +687,18 @@ AttnParams make_params(const bsa_plan_s& plan, const int32_t* row_ptr, const int
 // Natural layout [B, N, Hh, D] bf16 seen as 5-D {D, Hh, W, H, B*T}; boxes of
 // 64 channels x 1 head x pw x ph x 1 frame (one pooling tile, 128 rows of
 // 128 bytes), 128-byte swizzle.  Boxes reaching past W or H read zeros.
-bool make_tmap_tiles(CUtensorMap* m, const void* ptr, const Geometry& g) {
+bool make_tmap_tiles(CUtensorMap* m, const void* ptr, const Geometry& g, bool e4m3 = false) {
   auto fn = encode_fn();
   if (!fn) return false;
-  const cuuint64_t row = (cuuint64_t)g.Hh * g.D * 2;  // bytes per token
+  const cuuint64_t esz = e4m3 ? 1 : 2;
+  const cuuint64_t row = (cuuint64_t)g.Hh * g.D * esz;  // bytes per token
   cuuint64_t dims[5] = {(cuuint64_t)g.D, (cuuint64_t)g.Hh, (cuuint64_t)g.W, (cuuint64_t)g.H,
                         (cuuint64_t)g.B * g.T};
-  cuuint64_t strides[4] = {(cuuint64_t)g.D * 2, row, row * g.W, row * g.W * g.H};
-  cuuint32_t box[5] = {64, 1, (cuuint32_t)g.pw, (cuuint32_t)g.ph, 1};
+  cuuint64_t strides[4] = {(cuuint64_t)g.D * esz, row, row * g.W, row * g.W * g.H};
+  cuuint32_t box[5] = {(cuuint32_t)(128 / esz), 1, (cuuint32_t)g.pw, (cuuint32_t)g.ph, 1};
   cuuint32_t estr[5] = {1, 1, 1, 1, 1};
-  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, const_cast<void*>(ptr), dims, strides, box,
+  return fn(m, e4m3 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5,
+            const_cast<void*>(ptr), dims, strides, box,
             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
@@ -697,6 +747,30 @@ bsa_status launch_attn_fwd_natural(const bsa_plan_s& plan, const void* q, const 
   const cudaError_t e = g.D == 128 ? launch_t<128, false, true>(tq, tk, tv, p, grid, st)
                                    : launch_t<64, false, true>(tq, tk, tv, p, grid, st);
   if (e != cudaSuccess) return cuda_error(e, "natural-layout attention launch");
+  return BSA_OK;
+}
+
+bsa_status launch_attn_fwd_natural_e4m3(const bsa_plan_s& plan, const void* q8, const void* k8,
+                                        const void* v8, const float* scales,
+                                        const int32_t* row_ptr, const int32_t* col_idx,
+                                        int per_head, float scale, void* o, float* lse,
+                                        cudaStream_t st) {
+  const Geometry& g = plan.g;
+  if (g.layout != BSA_LAYOUT_TILE || g.block != kTile)
+    return set_error(BSA_ERR_UNSUPPORTED,
+                     "e4m3 attention needs a TILE plan with pool_h * pool_w = 128");
+  if (g.D != 128) return set_error(BSA_ERR_UNSUPPORTED, "e4m3 attention supports D = 128");
+  if ((int64_t)g.B * g.T * g.P * g.Hh >= (1ll << 31))
+    return set_error(BSA_ERR_UNSUPPORTED, "B*N*Hh must be < 2^31");
+  CUtensorMap tq, tk, tv;
+  if (!make_tmap_tiles(&tq, q8, g, true) || !make_tmap_tiles(&tk, k8, g, true) ||
+      !make_tmap_tiles(&tv, v8, g, true))
+    return set_error(BSA_ERR_CUDA, "cuTensorMapEncodeTiled (5-D, e4m3) failed");
+  AttnParams p = make_params(plan, row_ptr, col_idx, per_head, scale, o, lse);
+  p.fp8_scales = scales;
+  const dim3 grid((unsigned)g.ntiles, (unsigned)g.Hh, (unsigned)g.B);
+  const cudaError_t e = launch_t<128, false, true, true>(tq, tk, tv, p, grid, st);
+  if (e != cudaSuccess) return cuda_error(e, "e4m3 attention launch");
   return BSA_OK;
 }
 

@@ -68,6 +68,7 @@ struct bsa_plan_s {
   int lvsa_anchors = BSA_ANCHORS_ROTATING;  // bsa_plan_set_lvsa_variant
   int lvsa_window = BSA_WINDOW_DISTANCE;
   int draft_pooling = BSA_POOL_MEAN;        // bsa_plan_set_draft_pooling
+  uint32_t* d_amax = nullptr;               // [3][B][Hh] scratch of bsa_quantize_e4m3
 };
 
 namespace bsa {
@@ -90,6 +91,17 @@ cudaError_t launch_draft_mask(const Geometry& g, const uint32_t* tile_valid, con
                               const void* k, int keep, int pooling, int32_t* row_ptr,
                               int32_t* kv_idx, float* draft_map, double* ws, cudaStream_t st,
                               bool natural = false);
+
+// e4m3 quantization of natural-layout Q, K, V (scales [3][B][Hh]).
+cudaError_t launch_quantize_e4m3(const Geometry& g, uint32_t* amax_ws, const void* q, const void* k,
+                                 const void* v, void* q8, void* k8, void* v8, float* scales,
+                                 cudaStream_t st);
+// Natural-layout attention on e4m3 Q, K, V (TILE plan, 128-slot tiles, D = 128).
+bsa_status launch_attn_fwd_natural_e4m3(const bsa_plan_s& plan, const void* q8, const void* k8,
+                                        const void* v8, const float* scales,
+                                        const int32_t* row_ptr, const int32_t* col_idx,
+                                        int per_head, float scale, void* o, float* lse,
+                                        cudaStream_t st);
 
 // Anchor grid actually used for (plan variant, T_per, s): *T_per_eff = 0
 // means no anchors; also returns |G| over the plan's T frames.

@@ -1,0 +1,139 @@
+// e4m3 quantization of Q, K, V for the 8-bit draft attention (Draft
+// Attention article, closing paragraph: quantization as the next step; the
+// article fixes no format).  One scale per (tensor, batch, head):
+//   scale = fp32(max |x|) / 448 (1 when the head is all zero),
+//   code  = e4m3 nearest to x / scale (fp32 division), ties to even,
+//           saturating at +-448.
+// Three kernels on natural-layout [B, N, Hh, D] tensors: the per-head
+// maximum (one atomicMax per CTA; |x| of a float orders like its bits), the
+// scales, and the conversion (8 values per thread, 16-byte loads).
+#include <cuda_bf16.h>
+
+#include <algorithm>
+
+#include "bsa_internal.cuh"
+
+namespace bsa {
+namespace {
+
+constexpr int kThreads = 256;
+constexpr int kTokPerCta = 512;
+
+template <int D>
+__global__ void __launch_bounds__(kThreads)
+    e4m3_amax_kernel(const uint4* __restrict__ q, const uint4* __restrict__ k,
+                     const uint4* __restrict__ v, int B, int Hh, int64_t N, uint32_t* amax) {
+  constexpr int kTPR = D / 8;                  // threads per token row of one head
+  constexpr int kRowsPerPass = kThreads / kTPR;
+  __shared__ float red[kThreads / 32];
+  const int which = blockIdx.z;
+  const int bh = blockIdx.y, b = bh / Hh, h = bh - b * Hh;
+  const uint4* x = which == 0 ? q : (which == 1 ? k : v);
+  const int64_t n0 = (int64_t)blockIdx.x * kTokPerCta;
+  const int sub = threadIdx.x % kTPR;
+  float m = 0.f;
+  for (int r = threadIdx.x / kTPR; r < kTokPerCta; r += kRowsPerPass) {
+    const int64_t n = n0 + r;
+    if (n >= N) break;
+    const uint4 u = __ldg(x + (((int64_t)b * N + n) * Hh + h) * (D / 8) + sub);
+    const __nv_bfloat162* pv = reinterpret_cast<const __nv_bfloat162*>(&u);
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const float2 f = __bfloat1622float2(pv[e]);
+      m = fmaxf(m, fmaxf(fabsf(f.x), fabsf(f.y)));
+    }
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = m;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    float t = 0.f;
+    for (int w = 0; w < kThreads / 32; ++w) t = fmaxf(t, red[w]);
+    atomicMax(amax + ((int64_t)which * B + b) * Hh + h, __float_as_uint(t));
+  }
+}
+
+__global__ void e4m3_scales_kernel(const uint32_t* __restrict__ amax, int n, float* scales) {
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i < n) {
+    const float a = __uint_as_float(amax[i]);
+    scales[i] = a > 0.f ? __fdiv_rn(a, 448.f) : 1.f;
+  }
+}
+
+__device__ __forceinline__ uint32_t e4m3x2(float lo, float hi) {
+  uint16_t r;
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+
+// grid-stride over the 8-value groups of the three tensors
+template <int D>
+__global__ void __launch_bounds__(kThreads)
+    e4m3_convert_kernel(const uint4* __restrict__ q, const uint4* __restrict__ k,
+                        const uint4* __restrict__ v, uint2* __restrict__ q8, uint2* __restrict__ k8,
+                        uint2* __restrict__ v8, int B, int Hh, int64_t N,
+                        const float* __restrict__ scales) {
+  const int64_t per = (int64_t)B * N * Hh * (D / 8);  // groups per tensor
+  const int64_t stride = (int64_t)gridDim.x * kThreads;
+  for (int64_t e = (int64_t)blockIdx.x * kThreads + threadIdx.x; e < 3 * per; e += stride) {
+    const int which = (int)(e / per);
+    const int64_t r = e - which * per;
+    const int h = (int)((r / (D / 8)) % Hh);
+    const int b = (int)(r / (N * Hh * (D / 8)));
+    const float s = __ldg(scales + ((int64_t)which * B + b) * Hh + h);
+    const uint4* x = which == 0 ? q : (which == 1 ? k : v);
+    uint2* y = which == 0 ? q8 : (which == 1 ? k8 : v8);
+    const uint4 u = __ldg(x + r);
+    const __nv_bfloat162* pv = reinterpret_cast<const __nv_bfloat162*>(&u);
+    uint32_t w[2];
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+      const float2 f0 = __bfloat1622float2(pv[2 * i]), f1 = __bfloat1622float2(pv[2 * i + 1]);
+      w[i] = e4m3x2(__fdiv_rn(f0.x, s), __fdiv_rn(f0.y, s)) |
+             (e4m3x2(__fdiv_rn(f1.x, s), __fdiv_rn(f1.y, s)) << 16);
+    }
+    y[r] = make_uint2(w[0], w[1]);
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_quantize_e4m3(const Geometry& g, uint32_t* amax_ws, const void* q, const void* k,
+                                 const void* v, void* q8, void* k8, void* v8, float* scales,
+                                 cudaStream_t st) {
+  const int64_t N = (int64_t)g.T * g.P;
+  const int nsc = 3 * g.B * g.Hh;
+  cudaError_t e = cudaMemsetAsync(amax_ws, 0, sizeof(uint32_t) * nsc, st);
+  if (e != cudaSuccess) return e;
+  const dim3 grid((unsigned)((N + kTokPerCta - 1) / kTokPerCta), (unsigned)(g.B * g.Hh), 3);
+  auto qq = reinterpret_cast<const uint4*>(q);
+  auto kk = reinterpret_cast<const uint4*>(k);
+  auto vv = reinterpret_cast<const uint4*>(v);
+  if (g.D == 128)
+    e4m3_amax_kernel<128><<<grid, kThreads, 0, st>>>(qq, kk, vv, g.B, g.Hh, N, amax_ws);
+  else
+    e4m3_amax_kernel<64><<<grid, kThreads, 0, st>>>(qq, kk, vv, g.B, g.Hh, N, amax_ws);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  e4m3_scales_kernel<<<(nsc + 255) / 256, 256, 0, st>>>(amax_ws, nsc, scales);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int64_t groups = 3 * (int64_t)g.B * N * g.Hh * (g.D / 8);
+  const unsigned blocks =
+      (unsigned)std::min<int64_t>((groups + kThreads - 1) / kThreads, (int64_t)sms * 16);
+  auto y0 = reinterpret_cast<uint2*>(q8);
+  auto y1 = reinterpret_cast<uint2*>(k8);
+  auto y2 = reinterpret_cast<uint2*>(v8);
+  if (g.D == 128)
+    e4m3_convert_kernel<128><<<blocks, kThreads, 0, st>>>(qq, kk, vv, y0, y1, y2, g.B, g.Hh, N,
+                                                          scales);
+  else
+    e4m3_convert_kernel<64><<<blocks, kThreads, 0, st>>>(qq, kk, vv, y0, y1, y2, g.B, g.Hh, N,
+                                                         scales);
+  return cudaGetLastError();
+}
+
+}  // namespace bsa

@@ -234,6 +234,30 @@ bsa_status bsa_draft_mask_natural(bsa_plan_t plan, const void* q, const void* k,
                                   int32_t* row_ptr, int32_t* kv_idx, float* draft_map,
                                   void* workspace, size_t workspace_bytes, void* stream);
 
+/* e4m3 quantization for the 8-bit draft attention (the Draft Attention
+ * article names quantization as its next step without fixing a format; this
+ * is the reading taken).  q, k, v: natural layout [B, N, Hh, D] bf16; q8, k8,
+ * v8: the same layout, one e4m3 byte per element; scales: float[3*B*Hh],
+ * entry (t*B + b)*Hh + h for tensor t = 0 (Q), 1 (K), 2 (V):
+ *   scale = fp32(max |x| over the head) / 448 (1 for an all-zero head),
+ *   code  = e4m3 nearest to x / scale (fp32 division), ties to even,
+ *           saturating at +-448.
+ * Uses a small buffer owned by the plan: calls on one plan must not overlap. */
+bsa_status bsa_quantize_e4m3(bsa_plan_t plan, const void* q, const void* k, const void* v, void* q8,
+                             void* k8, void* v8, float* scales, void* stream);
+
+/* bsa_attn_fwd_natural on e4m3 inputs (from bsa_quantize_e4m3): the QK and
+ * PV products are 8-bit tensor-core MMAs (kind::f8f6f4) with fp32
+ * accumulation; the scores are S * sq * sk; P is rounded to e4m3 (it stays
+ * below 2^8); O is multiplied by sv.  Requires D = 128 and a TILE plan with
+ * pool_h * pool_w = 128.  o: bf16 natural layout; lse as for
+ * bsa_attn_fwd_natural.  Result within the e4m3 rounding of Q, K, V and P
+ * of the exact attention (see the tests for the bound used). */
+bsa_status bsa_attn_fwd_natural_e4m3(bsa_plan_t plan, const void* q8, const void* k8,
+                                     const void* v8, const float* scales, const int32_t* row_ptr,
+                                     const int32_t* col_idx, int per_head_lists, float scale,
+                                     void* o, float* lse, void* stream);
+
 /* LVSA attention in one pass on the natural layout ("LVSA", section 2 "Core
  * mechanism"; the reorder of the Draft Attention article is fused into the
  * tile loads, so no padded copies are made).
