@@ -239,7 +239,7 @@ def kernel_table(args):
             ts.append(e0.elapsed_time(e1))
         return statistics.median(ts)
 
-    def emit(cid, kernel, ms, algo_bytes=None, flops=None, note=None):
+    def emit(cid, kernel, ms, algo_bytes=None, flops=None, note=None, e4m3=False):
         d = {"config": cid, "workload": CONFIGS[cid].name, "kernel": kernel, "ms": round(ms, 4)}
         if algo_bytes is not None:
             gbs = algo_bytes / (ms * 1e-3) / 1e9
@@ -249,6 +249,9 @@ def kernel_table(args):
             tf = flops / (ms * 1e-3) / 1e12
             d.update({"attended_tflop": round(flops / 1e12, 4), "TFLOP_s": round(tf, 1),
                       "frac_bf16_burst": round(tf / pk["bf16_tflops"], 3)})
+            if e4m3:
+                # 8-bit contraction: measured bf16 peak x the nominal e4m3 / bf16 ratio (2)
+                d["frac_e4m3_peak"] = round(tf / (2 * pk["bf16_tflops"]), 3)
         if note:
             d["note"] = note
         print(json.dumps(d), flush=True)
@@ -334,7 +337,7 @@ def kernel_table(args):
                          timed(lambda: bsa.bsa_attn_fwd_natural_e4m3(
                              att.plan, att.q8, att.k8, att.v8, att.fp8_scales, att.row_ptr,
                              att.col_idx, True, scale, out)),
-                         flops=draft_attended_flops(w, kv_host, att.keep))
+                         flops=draft_attended_flops(w, kv_host, att.keep), e4m3=True)
                     emit(cid, "draft pipeline, 8-bit (mask, quantize, attention)",
                          timed(lambda: att.fused_e4m3(q, k, v, out)),
                          flops=draft_attended_flops(w, kv_host, att.keep))
