@@ -149,6 +149,12 @@ __global__ void __launch_bounds__(kPoolThreads)
   for (int e = 0; e < 8; ++e) dst[e] = cnt ? (use_max ? acc[e] : __ddiv_rn(acc[e], dc)) : 0.0;
 }
 
+// Unsigned key with the order of the doubles (-0 and +0 equal; no NaN).
+__device__ __forceinline__ uint64_t order_key(double v) {
+  const uint64_t b = (uint64_t)__double_as_longlong(v + 0.0);  // -0 + 0 = +0
+  return (b >> 63) ? ~b : (b | 0x8000000000000000ull);
+}
+
 // grid: (ceil(nblocks / R), Hh, B); R query rows per CTA.
 template <int D>
 __global__ void __launch_bounds__(kScoreThreads)
@@ -225,38 +231,36 @@ __global__ void __launch_bounds__(kScoreThreads)
     const double* L = sl + (int64_t)r * nblocks;
     uint8_t* sr = sel + (int64_t)r * nblocks;
     if (nblocks <= 32 * kRegCand) {
-      // candidates j = lane + 32u held in registers; `avail` marks the ones
-      // not yet taken
-      double v[kRegCand];
+      // candidates j = lane + 32u held in registers as order-preserving
+      // 64-bit keys; `avail` marks the ones not yet taken.  A round takes
+      // the largest key by three warp reductions (high word, low word among
+      // equal high words, lowest index among equal keys).
+      uint64_t key[kRegCand];
       uint32_t avail = 0u;
 #pragma unroll
       for (int u = 0; u < kRegCand; ++u) {
         const int j = lane + 32 * u;
-        v[u] = j < nblocks ? L[j] : 0.0;
+        key[u] = j < nblocks ? order_key(L[j]) : 0ull;
         if (j < nblocks) avail |= 1u << u;
       }
       const uint32_t start = avail;
       for (int it = 0; it < keep; ++it) {
-        double best = 0.0;
-        int bidx = 0x7fffffff;
+        uint64_t bk = 0ull;
+        int bu = -1;
 #pragma unroll
         for (int u = 0; u < kRegCand; ++u)
-          if (((avail >> u) & 1u) && (bidx == 0x7fffffff || v[u] > best)) {
-            best = v[u];
-            bidx = lane + 32 * u;
+          if (((avail >> u) & 1u) && (bu < 0 || key[u] > bk)) {
+            bk = key[u];
+            bu = u;
           }
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) {
-          const double ov = __shfl_xor_sync(0xffffffffu, best, o);
-          const int oi = __shfl_xor_sync(0xffffffffu, bidx, o);
-          const bool take = (oi != 0x7fffffff) &&
-                            (bidx == 0x7fffffff || ov > best || (ov == best && oi < bidx));
-          if (take) {
-            best = ov;
-            bidx = oi;
-          }
-        }
-        if (bidx != 0x7fffffff && (bidx & 31) == lane) avail &= ~(1u << (bidx >> 5));
+        const uint32_t hi = bu < 0 ? 0u : (uint32_t)(bk >> 32);
+        const uint32_t top_hi = __reduce_max_sync(0xffffffffu, hi);
+        const bool at_hi = bu >= 0 && hi == top_hi;
+        const uint32_t lo = at_hi ? (uint32_t)bk : 0u;
+        const uint32_t top_lo = __reduce_max_sync(0xffffffffu, lo);
+        const uint32_t idx = (at_hi && lo == top_lo) ? (uint32_t)(lane + 32 * bu) : 0xffffffffu;
+        const uint32_t win = __reduce_min_sync(0xffffffffu, idx);
+        if (win != 0xffffffffu && (int)(win & 31u) == lane) avail &= ~(1u << (win >> 5));
       }
 #pragma unroll
       for (int u = 0; u < kRegCand; ++u) {

@@ -68,23 +68,27 @@ __device__ __forceinline__ uint32_t e4m3x2(float lo, float hi) {
   return r;
 }
 
-// grid-stride over the 8-value groups of the three tensors
+// grid-stride over the 8-value groups of one tensor (blockIdx.y); the group
+// count of a tensor is below 2^31 (the plan checks it), so 32-bit indices
+// and magic-number division give (b, h) of a group
 template <int D>
 __global__ void __launch_bounds__(kThreads)
     e4m3_convert_kernel(const uint4* __restrict__ q, const uint4* __restrict__ k,
                         const uint4* __restrict__ v, uint2* __restrict__ q8, uint2* __restrict__ k8,
-                        uint2* __restrict__ v8, int B, int Hh, int64_t N,
-                        const float* __restrict__ scales) {
-  const int64_t per = (int64_t)B * N * Hh * (D / 8);  // groups per tensor
-  const int64_t stride = (int64_t)gridDim.x * kThreads;
-  for (int64_t e = (int64_t)blockIdx.x * kThreads + threadIdx.x; e < 3 * per; e += stride) {
-    const int which = (int)(e / per);
-    const int64_t r = e - which * per;
-    const int h = (int)((r / (D / 8)) % Hh);
-    const int b = (int)(r / (N * Hh * (D / 8)));
-    const float s = __ldg(scales + ((int64_t)which * B + b) * Hh + h);
-    const uint4* x = which == 0 ? q : (which == 1 ? k : v);
-    uint2* y = which == 0 ? q8 : (which == 1 ? k8 : v8);
+                        uint2* __restrict__ v8, int B, int Hh, uint32_t per, FastDiv div_Hh,
+                        FastDiv div_batch, const float* __restrict__ scales) {
+  constexpr int kShift = D == 128 ? 4 : 3;  // log2(D / 8)
+  const int which = blockIdx.y;
+  const uint4* x = which == 0 ? q : (which == 1 ? k : v);
+  uint2* y = which == 0 ? q8 : (which == 1 ? k8 : v8);
+  const float* sc = scales + (int64_t)which * B * Hh;
+  const uint32_t stride = gridDim.x * kThreads;
+  for (uint32_t r = blockIdx.x * kThreads + threadIdx.x; r < per; r += stride) {
+    const uint32_t row = r >> kShift;                  // (b * N + n) * Hh + h
+    const uint32_t bn = div_Hh.div(row);
+    const int h = (int)(row - bn * (uint32_t)Hh);
+    const int b = (int)div_batch.div(r);               // r / (N * Hh * D / 8)
+    const float s = __ldg(sc + b * Hh + h);
     const uint4 u = __ldg(x + r);
     const __nv_bfloat162* pv = reinterpret_cast<const __nv_bfloat162*>(&u);
     uint32_t w[2];
@@ -121,18 +125,19 @@ cudaError_t launch_quantize_e4m3(const Geometry& g, uint32_t* amax_ws, const voi
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  const int64_t groups = 3 * (int64_t)g.B * N * g.Hh * (g.D / 8);
-  const unsigned blocks =
-      (unsigned)std::min<int64_t>((groups + kThreads - 1) / kThreads, (int64_t)sms * 16);
+  const int64_t per = (int64_t)g.B * N * g.Hh * (g.D / 8);  // groups per tensor (< 2^31)
+  const dim3 cgrid(
+      (unsigned)std::min<int64_t>((per + kThreads - 1) / kThreads, (int64_t)sms * 8), 3);
+  const FastDiv div_Hh((uint32_t)g.Hh), div_batch((uint32_t)(N * g.Hh * (g.D / 8)));
   auto y0 = reinterpret_cast<uint2*>(q8);
   auto y1 = reinterpret_cast<uint2*>(k8);
   auto y2 = reinterpret_cast<uint2*>(v8);
   if (g.D == 128)
-    e4m3_convert_kernel<128><<<blocks, kThreads, 0, st>>>(qq, kk, vv, y0, y1, y2, g.B, g.Hh, N,
-                                                          scales);
+    e4m3_convert_kernel<128><<<cgrid, kThreads, 0, st>>>(qq, kk, vv, y0, y1, y2, g.B, g.Hh,
+                                                         (uint32_t)per, div_Hh, div_batch, scales);
   else
-    e4m3_convert_kernel<64><<<blocks, kThreads, 0, st>>>(qq, kk, vv, y0, y1, y2, g.B, g.Hh, N,
-                                                         scales);
+    e4m3_convert_kernel<64><<<cgrid, kThreads, 0, st>>>(qq, kk, vv, y0, y1, y2, g.B, g.Hh,
+                                                        (uint32_t)per, div_Hh, div_batch, scales);
   return cudaGetLastError();
 }
 
