@@ -103,7 +103,7 @@ def _randn(shape, seed: int, device) -> torch.Tensor:
 def _field_tokens(w: Workload, seed: int, device, h0: int, h1: int) -> torch.Tensor:
     """Trilinear upsample of an N(0,1) field on the coarse grid, heads [h0,h1).
 
-    Returns float32 [N, h1-h0, D].  The coarse field for all heads is drawn at
+    Returns float32 [B, N, h1-h0, D].  The coarse field for all heads is drawn at
     once from the seed, so any head range gives the same values.
     """
     Tc, Hc, Wc = w.field_grid
