@@ -7,7 +7,10 @@ natural-layout O out.  The step runs bsa_lvsa_attn_fwd, the one-kernel path
 (frame sets computed in the kernel, the reorder fused into its tile loads).
 The four-kernel path over the same data (lvsa_mask -> reorder_fwd ->
 attn_fwd on the block list -> reorder_inv) is timed too and reported per
-kernel.  Inputs (1.8 GB) exceed the 126 MB L2, so no flush is needed.
+kernel.  Inputs (1.8 GB) exceed the 126 MB L2, so no flush is needed.  The
+end-to-end figure copies every step's Q, K, V in from pinned host memory
+and its O out, overlapped with the neighbouring steps' compute
+(pipeline.StreamedSteps).
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
     python bench.py --kernel-table      # every kernel on every workload, one JSON line each
@@ -354,7 +357,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--config", type=int, default=3)
-    ap.add_argument("--e2e-steps", type=int, default=3)
+    ap.add_argument("--e2e-steps", type=int, default=6)
     ap.add_argument("--cpu-budget-s", type=float, default=12.0)
     ap.add_argument("--ref-step-s", type=float, default=4.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -448,26 +451,23 @@ def main():
     bsa.bsa_poll_status(att.plan)
     unf_ms = max_over_ranks([statistics.mean(unf[n]) for n in names], dist, "cuda")
 
-    # end to end through the public API with host buffers: pinned H2D of the
-    # step's Q, K, V, the step, D2H of O
+    # end to end through the public API with host buffers: every step copies
+    # its Q, K, V in from pinned host memory and its O back out; the copies
+    # of neighbouring steps overlap this step's compute (StreamedSteps)
+    from block_sparse_attention_49_b200.pipeline import StreamedSteps
     hq, hk, hv = (x.cpu().pin_memory() for x in (q, k, v))
     ho = torch.empty_like(hq).pin_memory()
-    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    streamed = StreamedSteps(q.shape, q.dtype)
+    step_fn = lambda dq, dk, dv, dout, i: att.fused(dq, dk, dv, i % w.lvsa_T_per, dout)
+    streamed.run(step_fn, (hq, hk, hv), ho, 2)       # warm-up
     torch.cuda.synchronize()
     if dist:
         dist.barrier()
-    e0, e1 = ev(), ev()
-    e0.record(stream)
-    for i in range(args.e2e_steps):
-        dq.copy_(hq, non_blocking=True)
-        dk.copy_(hk, non_blocking=True)
-        dv.copy_(hv, non_blocking=True)
-        att.fused(dq, dk, dv, i % w.lvsa_T_per, out)
-        ho.copy_(out, non_blocking=True)
-    e1.record(stream)
+    e0, e1 = streamed.run(step_fn, (hq, hk, hv), ho, args.e2e_steps)
     torch.cuda.synchronize()
     (e2e_ms,) = max_over_ranks([e0.elapsed_time(e1) / args.e2e_steps], dist, "cuda")
     bsa.bsa_poll_status(att.plan)
+    del streamed
 
     pk, pk_kind = peaks()
     peak = pk.get("bf16_tflops_sustained", pk["bf16_tflops"])

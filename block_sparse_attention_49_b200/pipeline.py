@@ -138,3 +138,56 @@ class DraftAttention(_Base):
         bsa_attn_fwd_natural_e4m3(self.plan, self.q8, self.k8, self.v8, self.fp8_scales,
                                   self.row_ptr, self.col_idx, True, self.scale, out, lse)
         return out
+
+
+class StreamedSteps:
+    """Runs attention steps whose inputs and outputs live in pinned host
+    memory, overlapping transfers with compute: step i+1's host-to-device
+    copies and step i-1's device-to-host read run on their own streams while
+    step i computes.  Two device buffer sets; every step still moves all of
+    its inputs in and its output out.
+
+        steps = StreamedSteps(shape, torch.bfloat16)
+        steps.run(lambda q, k, v, out, i: att.fused(q, k, v, i, out),
+                  host_inputs=(hq, hk, hv), host_output=ho, n=10)
+    """
+
+    def __init__(self, shape, dtype, device="cuda"):
+        mk = lambda: torch.empty(shape, dtype=dtype, device=device)
+        self.bufs = [[mk() for _ in range(4)] for _ in range(2)]  # q, k, v, out per set
+        self.h2d = torch.cuda.Stream(device)
+        self.d2h = torch.cuda.Stream(device)
+
+    def run(self, fn, host_inputs, host_output, n: int):
+        """Enqueue n steps; returns (start, end) CUDA events around all of them.
+        host_inputs: pinned (q, k, v) copied in for every step; host_output:
+        pinned tensor that receives every step's output."""
+        compute = torch.cuda.current_stream()
+        start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        ev_in = [torch.cuda.Event() for _ in range(2)]     # inputs of a set copied
+        ev_done = [torch.cuda.Event() for _ in range(2)]   # step on a set computed
+        ev_out = [torch.cuda.Event() for _ in range(2)]    # output of a set read back
+        start.record(compute)
+        self.h2d.wait_event(start)
+        self.d2h.wait_event(start)
+        for i in range(n):
+            b = i % 2
+            q, k, v, out = self.bufs[b]
+            with torch.cuda.stream(self.h2d):
+                if i >= 2:
+                    self.h2d.wait_event(ev_done[b])        # inputs of step i-2 consumed
+                for dst, src in zip((q, k, v), host_inputs):
+                    dst.copy_(src, non_blocking=True)
+                ev_in[b].record(self.h2d)
+            compute.wait_event(ev_in[b])
+            if i >= 2:
+                compute.wait_event(ev_out[b])              # output of step i-2 read back
+            fn(q, k, v, out, i)
+            ev_done[b].record(compute)
+            with torch.cuda.stream(self.d2h):
+                self.d2h.wait_event(ev_done[b])
+                host_output.copy_(out, non_blocking=True)
+                ev_out[b].record(self.d2h)
+        compute.wait_stream(self.d2h)
+        end.record(compute)
+        return start, end

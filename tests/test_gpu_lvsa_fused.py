@@ -142,3 +142,21 @@ def test_fused_rejects_unsupported_geometry():
     with pytest.raises(bsa.BsaError) as ei:
         bsa.bsa_lvsa_attn_fwd(tplan, 3, 2, 0, y, y, y, 0.125, y)
     assert ei.value.status == 1
+
+
+def test_streamed_steps_match_direct_calls():
+    # host inputs copied in and the output read back every step, overlapped
+    # with the neighbouring steps' compute: the last step's output equals the
+    # direct call's, bit for bit
+    from block_sparse_attention_49_b200.pipeline import LvsaAttention, StreamedSteps
+    w = small_workload(CONFIGS[3], T=12, Hh=2, field_grid=(12, 4, 7))
+    q, k, v = make_qkv(w)
+    hq, hk, hv = (x.pin_memory() for x in (q, k, v))
+    ho = torch.empty_like(hq).pin_memory()
+    att = LvsaAttention(w.B, w.Hh, w.D, w.T, w.H, w.W, 5, 4, block=128)
+    streamed = StreamedSteps(q.shape, q.dtype)
+    streamed.run(lambda a, b, c, out, i: att.fused(a, b, c, i, out), (hq, hk, hv), ho, 3)
+    torch.cuda.synchronize()
+    direct = att.fused(q.cuda(), k.cuda(), v.cuda(), 2)
+    bsa.bsa_poll_status(att.plan)
+    assert torch.equal(ho.view(torch.int16), direct.cpu().view(torch.int16))
