@@ -131,20 +131,6 @@ __device__ __forceinline__ void softmax_sum(RowState& st, const uint64_t (&acc)[
   st.l += a0 + a1;
 }
 
-// One whole online-softmax step over NC keys: softmax_max, then P for all
-// NC keys.  Returns true when O must be multiplied by *corr.
-template <int NC>
-__device__ __forceinline__ bool softmax_tile(float (&s)[NC], const uint32_t (&vm)[NC / 32],
-                                             RowState& st, float sl2, float thr,
-                                             uint32_t (&pk)[NC / 2], float& corr) {
-  uint64_t neg_ms2;
-  const bool need = softmax_max(s, vm, st, sl2, thr, corr, neg_ms2);
-  uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};
-  softmax_exp<0, NC>(s, sl2, neg_ms2, pk, acc);
-  softmax_sum(st, acc);
-  return need;
-}
-
 // Multiply NCOLS fp32 accumulator columns of this thread's TMEM lane by f.
 template <int NCOLS>
 __device__ __forceinline__ void tmem_scale(uint32_t taddr, float f) {
