@@ -14,6 +14,8 @@ and its O out, overlapped with the neighbouring steps' compute
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
     python bench.py --kernel-table      # every kernel on every workload, one JSON line each
+    python bench.py --draft-pipelines H # the three draft pipelines, twice, on H heads
+                                        # of the 40-head draft workload (for profilers)
 
 Under torchrun (N > 1) every rank runs its own batch (the path shards over
 batch x heads with no data exchange): weak scaling, max time over ranks.
@@ -350,6 +352,27 @@ def kernel_table(args):
         torch.cuda.empty_cache()
 
 
+def draft_pipelines(heads: int):
+    """Runs the three draft pipelines (with reorders, on the natural layout,
+    8-bit) twice each on `heads` heads of the 40-head draft workload: a fixed
+    launch sequence for profilers.  Prints one line."""
+    import block_sparse_attention_49_b200 as bsa
+    from block_sparse_attention_49_b200.pipeline import DraftAttention
+    from synth import small_workload
+
+    w = small_workload(CONFIGS[5], Hh=heads)
+    q, k, v = make_qkv(w, device="cuda")
+    att = DraftAttention(w.B, w.Hh, w.D, w.T, w.H, w.W, w.draft_ph, w.draft_pw, w.draft_sparsity)
+    out = torch.empty_like(q)
+    for _ in range(2):
+        att(q, k, v, out)
+        att.fused(q, k, v, out)
+        att.fused_e4m3(q, k, v, out)
+    torch.cuda.synchronize()
+    bsa.bsa_poll_status(att.plan)
+    print(json.dumps({"draft_pipelines": w.name, "heads": heads}), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -366,7 +389,13 @@ def main():
     ap.add_argument("--kernel-table", action="store_true",
                     help="time every kernel on every workload instead of the step")
     ap.add_argument("--table-reps", type=int, default=10)
+    ap.add_argument("--draft-pipelines", type=int, default=0, metavar="HEADS",
+                    help="run the three draft pipelines on HEADS heads (profiling)")
     args = ap.parse_args()
+    if args.draft_pipelines:
+        torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", 0)))
+        draft_pipelines(args.draft_pipelines)
+        return
     if args.kernel_table:
         torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", 0)))
         kernel_table(args)
