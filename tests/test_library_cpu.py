@@ -67,6 +67,20 @@ def test_null_plan_is_rejected(lib):
     assert lib.bsa_poll_status(None, None) == 1
     assert lib.bsa_plan_set_lvsa_variant(None, 0, 0) == 1
     assert lib.bsa_plan_set_draft_pooling(None, 0) == 1
+    assert lib.bsa_lvsa_attn_fwd(None, 4, 4, 0, None, None, None, 1.0, None, None, None) == 1
+    assert lib.bsa_attn_fwd_natural(None, None, None, None, None, None, 1, 1.0, None, None,
+                                    None) == 1
+    assert lib.bsa_draft_mask(None, None, None, 90, None, None, None, None, 0, None) == 1
+    assert lib.bsa_draft_mask_natural(None, None, None, 90, None, None, None, None, 0, None) == 1
+    assert lib.bsa_draft_mask_noalloc(None, None, None, 90, None, None, None, None) == 1
+    assert lib.bsa_quantize_e4m3(None, None, None, None, None, None, None, None, None) == 1
+    assert lib.bsa_attn_fwd_natural_e4m3(None, None, None, None, None, None, None, 1, 1.0, None,
+                                         None, None) == 1
+    assert lib.bsa_reorder_fwd(None, None, None, None, None, None, None, None) == 1
+    assert lib.bsa_reorder_inv(None, None, None, None) == 1
+    assert lib.bsa_lvsa_nnz(None, 4) == -1
+    assert lib.bsa_draft_keep_count(None, 90) == -1
+    assert lib.bsa_draft_workspace_bytes(None) == 0
 
 
 def test_no_cpu_fallback_path():
