@@ -10,8 +10,9 @@
 // How (one CTA per 128-slot query tile; 12 warps):
 //   warp 0      TMA producer: the Q tile once, then K and V of every listed
 //               key tile into an NS-deep shared-memory ring (128-byte swizzle).
-//   warp 1      MMA issuer (one thread): S = Q K^T into tensor memory, then
-//               O += P V with P read from tensor memory.
+//   warp 1      MMA issuer (the whole warp runs the loop, an elected lane
+//               issues): S = Q K^T into tensor memory, then O += P V with P
+//               read from tensor memory.
 //   warps 4-7   softmax group A: key tiles 0, 2, 4, ... of the list;
 //   warps 8-11  softmax group B: key tiles 1, 3, 5, ...
 // Each group owns one S buffer and one O accumulator in tensor memory
@@ -26,6 +27,17 @@
 // as in a split-key combine, normalised and stored.
 // Every wait is bounded; a wait that runs out records a timeout in the
 // plan's status word and the CTA leaves without trapping.
+//
+// Variants of the same body (template flags):
+//   FINE  blocks smaller than 128 slots: each row walks its own CSR row;
+//   NAT   natural-layout [B, N, Hh, D] tensors of a TILE plan whose tiles are
+//         128 slots: each tile is read through a 5-D tensor map (one
+//         pool_h x pool_w tile per box, zero past the grid edge) and O rows
+//         are stored straight to their tokens (the reorder of the Draft
+//         Attention article fused into loads and stores);
+//   F8    (with NAT) e4m3 Q, K, V: 8-bit MMAs (kind::f8f6f4, K = 32), P
+//         rounded to e4m3 in tensor memory, per-(batch, head) scales folded
+//         into the exponent and the final normalisation.
 #include <cuda_bf16.h>
 #include <cudaTypedefs.h>
 
