@@ -161,22 +161,28 @@ __global__ void __launch_bounds__(kScoreThreads)
     draft_score_topk_kernel(const double* __restrict__ qbar, const double* __restrict__ kbar,
                             int Hh, int nblocks, int R, int keep, int32_t* __restrict__ row_ptr,
                             int32_t* __restrict__ kv_idx, float* __restrict__ draft_map) {
+  constexpr int kWarps = kScoreThreads / 32;
+  constexpr int kKStride = D + 2;  // even: 16-byte loads of two channels, no bank conflicts
   extern __shared__ double shd[];
-  double* sq = shd;                         // [R][D]
-  double* sk = sq + R * D;                  // [kKeyChunk][D + 1]
-  double* sl = sk + kKeyChunk * (D + 1);    // [R][nblocks] logits
+  double* sq = shd;                            // [kWarps][D][2]: rows w and w + kWarps
+  double* sk = sq + 2 * kWarps * D;            // [kKeyChunk][kKStride]
+  double* sl = sk + kKeyChunk * kKStride;      // [R][nblocks] logits
   uint8_t* sel = reinterpret_cast<uint8_t*>(sl + (int64_t)R * nblocks);  // [R][nblocks]
   const int h = blockIdx.y, b = blockIdx.z;
   const int64_t bh = (int64_t)b * Hh + h;
   const int r0 = blockIdx.x * R;
-  const int rows = min(R, nblocks - r0);
+  const int rows = min(R, nblocks - r0);  // R <= 2 * kWarps
   const double* qb = qbar + (bh * nblocks + r0) * D;
   const double* kb = kbar + bh * nblocks * D;
-  for (int i = threadIdx.x; i < rows * D; i += kScoreThreads) sq[i] = qb[i];
+  // warp w carries rows w and w + kWarps: their values at channel c sit side
+  // by side (one broadcast 16-byte load); missing rows read zeros
+  for (int i = threadIdx.x; i < 2 * kWarps * D; i += kScoreThreads) {
+    const int r = i / D, c = i - r * D;
+    sq[((r % kWarps) * D + c) * 2 + r / kWarps] = r < rows ? qb[i] : 0.0;
+  }
   for (int i = threadIdx.x; i < rows * nblocks; i += kScoreThreads) sel[i] = 0;
 
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  constexpr int kWarps = kScoreThreads / 32;
   // key chunks: the next chunk is loaded into registers while the current
   // one is used, then stored to shared memory (padded stride: no conflicts)
   constexpr int kPer = kKeyChunk * D / kScoreThreads;
@@ -197,30 +203,28 @@ __global__ void __launch_bounds__(kScoreThreads)
     for (int u = 0; u < kPer; ++u) {
       const int idx = threadIdx.x + u * kScoreThreads;
       const int jj = idx / D, c = idx - jj * D;
-      sk[jj * (D + 1) + c] = pre[u];
+      sk[jj * kKStride + c] = pre[u];
     }
     __syncthreads();
     if (j0 + kKeyChunk < nblocks) load_chunk(j0 + kKeyChunk);
-    // warp w takes rows w and w + 8 together (two independent chains);
+    // warp w takes rows w and w + kWarps together (two independent chains);
     // lane = key block within the chunk.  Each logit is still the sequential
     // multiply-then-add over c.
-    if (lane < nj) {
-      const double* kk = sk + lane * (D + 1);
-      for (int ra = warp; ra < rows; ra += 2 * kWarps) {
-        const int rb = ra + kWarps;
-        const bool has_b = rb < rows;
-        const double* qa = sq + ra * D;
-        const double* qb2 = sq + (has_b ? rb : ra) * D;
-        double acc_a = 0.0, acc_b = 0.0;
-#pragma unroll 8
-        for (int c = 0; c < D; ++c) {
-          const double kc = kk[c];
-          acc_a = __dadd_rn(acc_a, __dmul_rn(qa[c], kc));
-          acc_b = __dadd_rn(acc_b, __dmul_rn(qb2[c], kc));
-        }
-        sl[(int64_t)ra * nblocks + j0 + lane] = acc_a;
-        if (has_b) sl[(int64_t)rb * nblocks + j0 + lane] = acc_b;
+    if (lane < nj && warp < rows) {
+      const double2* kk = reinterpret_cast<const double2*>(sk + lane * kKStride);
+      const double2* qq = reinterpret_cast<const double2*>(sq) + warp * D;
+      double acc_a = 0.0, acc_b = 0.0;
+#pragma unroll 4
+      for (int c2 = 0; c2 < D / 2; ++c2) {
+        const double2 kc = kk[c2];
+        const double2 q0 = qq[2 * c2], q1 = qq[2 * c2 + 1];
+        acc_a = __dadd_rn(acc_a, __dmul_rn(q0.x, kc.x));
+        acc_b = __dadd_rn(acc_b, __dmul_rn(q0.y, kc.x));
+        acc_a = __dadd_rn(acc_a, __dmul_rn(q1.x, kc.y));
+        acc_b = __dadd_rn(acc_b, __dmul_rn(q1.y, kc.y));
       }
+      sl[(int64_t)warp * nblocks + j0 + lane] = acc_a;
+      if (warp + kWarps < rows) sl[(int64_t)(warp + kWarps) * nblocks + j0 + lane] = acc_b;
     }
   }
   __syncthreads();
@@ -348,7 +352,8 @@ cudaError_t launch_t(const Geometry& g, const uint32_t* tile_valid, const void* 
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   const int R = draft_rows_per_cta(g.nblocks);
-  const size_t smem = (size_t)(R * D + kKeyChunk * (D + 1) + (int64_t)R * g.nblocks) * sizeof(double) +
+  const size_t smem = (size_t)(2 * (kScoreThreads / 32) * D + kKeyChunk * (D + 2) +
+                               (int64_t)R * g.nblocks) * sizeof(double) +
                       (size_t)R * g.nblocks;
   auto kern = draft_score_topk_kernel<D>;
   e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
@@ -362,7 +367,9 @@ cudaError_t launch_t(const Geometry& g, const uint32_t* tile_valid, const void* 
 }  // namespace
 
 int draft_rows_per_cta(int64_t nblocks) {
-  // logits + selection flags of R rows within ~150 KB of shared memory
+  // logits + selection flags of R rows within ~150 KB of shared memory; at
+  // most two rows per warp of the scoring kernel
+  static_assert(2 * (kScoreThreads / 32) >= 16, "two rows per warp");
   int64_t R = 16;
   while (R > 1 && R * nblocks * 9 > 150 * 1024) R >>= 1;
   return (int)R;

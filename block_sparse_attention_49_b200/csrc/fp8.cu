@@ -6,7 +6,24 @@
 //           saturating at +-448.
 // Three kernels on natural-layout [B, N, Hh, D] tensors: the per-head
 // maximum (one atomicMax per CTA; |x| of a float orders like its bits), the
-// scales, and the conversion (8 values per thread, 16-byte loads).
+// scales (and their fp32 reciprocals, kept in the maximum's workspace), and
+// the conversion (8 values per thread, 16-byte loads).
+//
+// The conversion needs x / scale only to e4m3 precision, so it multiplies by
+// the reciprocal r = fp32(1 / scale) and divides only where that could give
+// another code.  With z = x / scale exactly, x * r carries two roundings of
+// relative size at most 2^-24 and fp32(z) one, so the two fp32 numbers are at
+// most 3 units in the last place apart (both in the binade of z).  Rounding to
+// e4m3 (3 mantissa bits) can then differ only if a rounding boundary of e4m3
+// -- the midpoint between two neighbouring codes, where the 20 fp32 mantissa
+// bits below the e4m3 ones read 0x80000 -- lies within 3 units of x * r.
+// Products at least 4 units from every midpoint, in e4m3's normal range
+// [2^-6, 448], are used as they are; all others take the fp32 division: the
+// subnormal range, and near-midpoint products, about 8 in 2^20 values when
+// the quotients are not short binary fractions (a head whose maximum has a
+// short mantissa, a power of two say, gives many exact quotients, and those
+// that are midpoints are ties the division must settle).  The codes are those
+// of the division everywhere.
 #include <cuda_bf16.h>
 
 #include <algorithm>
@@ -54,11 +71,15 @@ __global__ void __launch_bounds__(kThreads)
   }
 }
 
-__global__ void e4m3_scales_kernel(const uint32_t* __restrict__ amax, int n, float* scales) {
+// scale = max / 448 (1 for an all-zero head); the maximum's slot then holds
+// the fp32 reciprocal of the scale for the conversion
+__global__ void e4m3_scales_kernel(uint32_t* __restrict__ amax, int n, float* scales) {
   const int i = blockIdx.x * blockDim.x + threadIdx.x;
   if (i < n) {
     const float a = __uint_as_float(amax[i]);
-    scales[i] = a > 0.f ? __fdiv_rn(a, 448.f) : 1.f;
+    const float sc = a > 0.f ? __fdiv_rn(a, 448.f) : 1.f;
+    scales[i] = sc;
+    amax[i] = __float_as_uint(__frcp_rn(sc));
   }
 }
 
@@ -66,6 +87,15 @@ __device__ __forceinline__ uint32_t e4m3x2(float lo, float hi) {
   uint16_t r;
   asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
   return r;
+}
+
+// x / s to the precision e4m3 keeps (r = fp32(1 / s); see the file comment)
+__device__ __forceinline__ float quotient_for_e4m3(float x, float s, float r) {
+  const float y = x * r;
+  const uint32_t a = __float_as_uint(y) & 0x7fffffffu;
+  const int d = (int)(a & 0xfffffu) - 0x80000;  // units in the last place to the midpoint
+  const bool safe = a >= 0x3c800000u && a <= 0x43e00000u && (d >= 4 || d <= -4);  // [2^-6, 448]
+  return safe ? y : __fdiv_rn(x, s);
 }
 
 // grid-stride over the 8-value groups of one tensor (blockIdx.y); the group
@@ -76,27 +106,29 @@ __global__ void __launch_bounds__(kThreads)
     e4m3_convert_kernel(const uint4* __restrict__ q, const uint4* __restrict__ k,
                         const uint4* __restrict__ v, uint2* __restrict__ q8, uint2* __restrict__ k8,
                         uint2* __restrict__ v8, int B, int Hh, uint32_t per, FastDiv div_Hh,
-                        FastDiv div_batch, const float* __restrict__ scales) {
+                        FastDiv div_batch, const float* __restrict__ scales,
+                        const float* __restrict__ recips) {
   constexpr int kShift = D == 128 ? 4 : 3;  // log2(D / 8)
   const int which = blockIdx.y;
   const uint4* x = which == 0 ? q : (which == 1 ? k : v);
   uint2* y = which == 0 ? q8 : (which == 1 ? k8 : v8);
   const float* sc = scales + (int64_t)which * B * Hh;
+  const float* rc = recips + (int64_t)which * B * Hh;
   const uint32_t stride = gridDim.x * kThreads;
   for (uint32_t r = blockIdx.x * kThreads + threadIdx.x; r < per; r += stride) {
     const uint32_t row = r >> kShift;                  // (b * N + n) * Hh + h
     const uint32_t bn = div_Hh.div(row);
     const int h = (int)(row - bn * (uint32_t)Hh);
     const int b = (int)div_batch.div(r);               // r / (N * Hh * D / 8)
-    const float s = __ldg(sc + b * Hh + h);
+    const float s = __ldg(sc + b * Hh + h), rs = __ldg(rc + b * Hh + h);
     const uint4 u = __ldg(x + r);
     const __nv_bfloat162* pv = reinterpret_cast<const __nv_bfloat162*>(&u);
     uint32_t w[2];
 #pragma unroll
     for (int i = 0; i < 2; ++i) {
       const float2 f0 = __bfloat1622float2(pv[2 * i]), f1 = __bfloat1622float2(pv[2 * i + 1]);
-      w[i] = e4m3x2(__fdiv_rn(f0.x, s), __fdiv_rn(f0.y, s)) |
-             (e4m3x2(__fdiv_rn(f1.x, s), __fdiv_rn(f1.y, s)) << 16);
+      w[i] = e4m3x2(quotient_for_e4m3(f0.x, s, rs), quotient_for_e4m3(f0.y, s, rs)) |
+             (e4m3x2(quotient_for_e4m3(f1.x, s, rs), quotient_for_e4m3(f1.y, s, rs)) << 16);
     }
     y[r] = make_uint2(w[0], w[1]);
   }
@@ -134,10 +166,12 @@ cudaError_t launch_quantize_e4m3(const Geometry& g, uint32_t* amax_ws, const voi
   auto y2 = reinterpret_cast<uint2*>(v8);
   if (g.D == 128)
     e4m3_convert_kernel<128><<<cgrid, kThreads, 0, st>>>(qq, kk, vv, y0, y1, y2, g.B, g.Hh,
-                                                         (uint32_t)per, div_Hh, div_batch, scales);
+                                                         (uint32_t)per, div_Hh, div_batch, scales,
+                                                         reinterpret_cast<const float*>(amax_ws));
   else
     e4m3_convert_kernel<64><<<cgrid, kThreads, 0, st>>>(qq, kk, vv, y0, y1, y2, g.B, g.Hh,
-                                                        (uint32_t)per, div_Hh, div_batch, scales);
+                                                        (uint32_t)per, div_Hh, div_batch, scales,
+                                                        reinterpret_cast<const float*>(amax_ws));
   return cudaGetLastError();
 }
 
