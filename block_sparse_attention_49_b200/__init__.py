@@ -126,6 +126,42 @@ def _ptr(t) -> Optional[int]:
     return t.data_ptr()
 
 
+def _need(what: str, t, nbytes: int):
+    """Rejects a tensor smaller than the plan implies: the kernels take every
+    size from the plan, so a short buffer would be read or written past its
+    end.  None and raw integer addresses pass unchecked."""
+    if t is None or isinstance(t, int):
+        return
+    have = t.numel() * t.element_size()
+    if have < nbytes:
+        raise ValueError(f"{what}: {have} bytes, the plan needs {nbytes}")
+
+
+def _natural(plan, elem: int = 2) -> int:
+    """Bytes of one natural-layout tensor [B, N, Hh, D]."""
+    return plan.B * plan.T * plan.H * plan.W * plan.Hh * plan.D * elem
+
+
+def _slots(plan, elem: int = 2) -> int:
+    """Bytes of one slot-layout tensor [B, Hh, Npad, D]."""
+    return plan.B * plan.Hh * plan.Npad * plan.D * elem
+
+
+def _need_lists(plan, per_head_lists: bool, row_ptr):
+    lists = plan.B * plan.Hh if per_head_lists else 1
+    _need("row_ptr", row_ptr, (lists * plan.nblocks + 1) * 4)
+
+
+def _need_draft_outputs(plan, sparsity_pct: int, row_ptr, kv_idx, draft_map):
+    if not 0 <= sparsity_pct < 100:
+        return  # rejected by the library
+    rows = plan.B * plan.Hh * plan.nblocks
+    keep = -(-plan.nblocks * (100 - sparsity_pct) // 100)
+    _need("kv_idx", kv_idx, rows * keep * 4)
+    _need("row_ptr", row_ptr, (rows + 1) * 4)
+    _need("draft_map", draft_map, rows * plan.nblocks * 4)
+
+
 def _stream(stream) -> Optional[int]:
     if stream is not None:
         return stream if isinstance(stream, int) else stream.cuda_stream
@@ -185,6 +221,10 @@ def bsa_lvsa_nnz(plan: Plan, C: int) -> int:
 
 def bsa_lvsa_mask(plan: Plan, C: int, T_per: int, s: int, frame_sets, row_ptr, col_idx,
                   stream=None):
+    if C > 0:
+        _need("frame_sets", frame_sets, plan.T * C * 4)
+        _need("col_idx", col_idx, plan.nblocks * C * (plan.nblocks // plan.T) * 4)
+    _need("row_ptr", row_ptr, (plan.nblocks + 1) * 4)
     _check(load().bsa_lvsa_mask(plan.handle, C, T_per, s, _ptr(frame_sets), _ptr(row_ptr),
                                 _ptr(col_idx), _stream(stream)), "bsa_lvsa_mask")
 
@@ -199,6 +239,9 @@ def bsa_draft_workspace_bytes(plan: Plan) -> int:
 
 def bsa_draft_mask(plan: Plan, q_slots, k_slots, sparsity_pct: int, row_ptr, kv_idx,
                    draft_map, workspace, stream=None):
+    _need("q_slots", q_slots, _slots(plan))
+    _need("k_slots", k_slots, _slots(plan))
+    _need_draft_outputs(plan, sparsity_pct, row_ptr, kv_idx, draft_map)
     nbytes = workspace.numel() * workspace.element_size()
     _check(load().bsa_draft_mask(plan.handle, _ptr(q_slots), _ptr(k_slots), sparsity_pct,
                                  _ptr(row_ptr), _ptr(kv_idx), _ptr(draft_map), _ptr(workspace),
@@ -208,6 +251,9 @@ def bsa_draft_mask(plan: Plan, q_slots, k_slots, sparsity_pct: int, row_ptr, kv_
 def bsa_draft_mask_noalloc(plan: Plan, q_slots, k_slots, sparsity_pct: int, row_ptr, kv_idx,
                            draft_map, stream=None):
     """bsa_draft_mask without a caller workspace (scratch inside the library)."""
+    _need("q_slots", q_slots, _slots(plan))
+    _need("k_slots", k_slots, _slots(plan))
+    _need_draft_outputs(plan, sparsity_pct, row_ptr, kv_idx, draft_map)
     _check(load().bsa_draft_mask_noalloc(plan.handle, _ptr(q_slots), _ptr(k_slots), sparsity_pct,
                                          _ptr(row_ptr), _ptr(kv_idx), _ptr(draft_map),
                                          _stream(stream)), "bsa_draft_mask_noalloc")
@@ -218,17 +264,26 @@ def bsa_draft_noalloc_max_scratch_bytes() -> int:
 
 
 def bsa_reorder_fwd(plan: Plan, x0, y0, x1=None, y1=None, x2=None, y2=None, stream=None):
+    for i, (x, y) in enumerate(((x0, y0), (x1, y1), (x2, y2))):
+        _need(f"x{i}", x, _natural(plan))
+        _need(f"y{i}", y, _slots(plan))
     _check(load().bsa_reorder_fwd(plan.handle, _ptr(x0), _ptr(y0), _ptr(x1), _ptr(y1),
                                   _ptr(x2), _ptr(y2), _stream(stream)), "bsa_reorder_fwd")
 
 
 def bsa_reorder_inv(plan: Plan, x_slots, x_nat, stream=None):
+    _need("x_slots", x_slots, _slots(plan))
+    _need("x_nat", x_nat, _natural(plan))
     _check(load().bsa_reorder_inv(plan.handle, _ptr(x_slots), _ptr(x_nat), _stream(stream)),
            "bsa_reorder_inv")
 
 
 def bsa_attn_fwd(plan: Plan, q, k, v, row_ptr, col_idx, per_head_lists: bool, scale: float,
                  o, lse=None, stream=None):
+    for name, t in (("q", q), ("k", k), ("v", v), ("o", o)):
+        _need(name, t, _slots(plan))
+    _need("lse", lse, plan.B * plan.Hh * plan.Npad * 4)
+    _need_lists(plan, per_head_lists, row_ptr)
     _check(load().bsa_attn_fwd(plan.handle, _ptr(q), _ptr(k), _ptr(v), _ptr(row_ptr),
                                _ptr(col_idx), int(bool(per_head_lists)), float(scale), _ptr(o),
                                _ptr(lse), _stream(stream)), "bsa_attn_fwd")
@@ -237,6 +292,10 @@ def bsa_attn_fwd(plan: Plan, q, k, v, row_ptr, col_idx, per_head_lists: bool, sc
 def bsa_attn_fwd_natural(plan: Plan, q, k, v, row_ptr, col_idx, per_head_lists: bool,
                          scale: float, o, lse=None, stream=None):
     """bsa_attn_fwd on natural-layout [B, N, Hh, D] tensors (TILE plan, 128-slot tiles)."""
+    for name, t in (("q", q), ("k", k), ("v", v), ("o", o)):
+        _need(name, t, _natural(plan))
+    _need("lse", lse, _natural(plan, 4) // plan.D)
+    _need_lists(plan, per_head_lists, row_ptr)
     _check(load().bsa_attn_fwd_natural(plan.handle, _ptr(q), _ptr(k), _ptr(v), _ptr(row_ptr),
                                        _ptr(col_idx), int(bool(per_head_lists)), float(scale),
                                        _ptr(o), _ptr(lse), _stream(stream)), "bsa_attn_fwd_natural")
@@ -245,6 +304,9 @@ def bsa_attn_fwd_natural(plan: Plan, q, k, v, row_ptr, col_idx, per_head_lists: 
 def bsa_draft_mask_natural(plan: Plan, q, k, sparsity_pct: int, row_ptr, kv_idx, draft_map,
                            workspace, stream=None):
     """bsa_draft_mask reading natural-layout q, k directly."""
+    _need("q", q, _natural(plan))
+    _need("k", k, _natural(plan))
+    _need_draft_outputs(plan, sparsity_pct, row_ptr, kv_idx, draft_map)
     nbytes = workspace.numel() * workspace.element_size()
     _check(load().bsa_draft_mask_natural(plan.handle, _ptr(q), _ptr(k), sparsity_pct,
                                          _ptr(row_ptr), _ptr(kv_idx), _ptr(draft_map),
@@ -255,6 +317,11 @@ def bsa_draft_mask_natural(plan: Plan, q, k, sparsity_pct: int, row_ptr, kv_idx,
 def bsa_quantize_e4m3(plan: Plan, q, k, v, q8, k8, v8, scales, stream=None):
     """e4m3 copies of natural-layout q, k, v (uint8 tensors) and their
     per-(tensor, batch, head) scales (float32 [3, B, Hh])."""
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        _need(name, t, _natural(plan))
+    for name, t in (("q8", q8), ("k8", k8), ("v8", v8)):
+        _need(name, t, _natural(plan, 1))
+    _need("scales", scales, 3 * plan.B * plan.Hh * 4)
     _check(load().bsa_quantize_e4m3(plan.handle, _ptr(q), _ptr(k), _ptr(v), _ptr(q8), _ptr(k8),
                                     _ptr(v8), _ptr(scales), _stream(stream)), "bsa_quantize_e4m3")
 
@@ -262,6 +329,12 @@ def bsa_quantize_e4m3(plan: Plan, q, k, v, q8, k8, v8, scales, stream=None):
 def bsa_attn_fwd_natural_e4m3(plan: Plan, q8, k8, v8, scales, row_ptr, col_idx,
                               per_head_lists: bool, scale: float, o, lse=None, stream=None):
     """bsa_attn_fwd_natural on e4m3 inputs from bsa_quantize_e4m3 (8-bit MMAs)."""
+    for name, t in (("q8", q8), ("k8", k8), ("v8", v8)):
+        _need(name, t, _natural(plan, 1))
+    _need("o", o, _natural(plan))
+    _need("scales", scales, 3 * plan.B * plan.Hh * 4)
+    _need("lse", lse, _natural(plan, 4) // plan.D)
+    _need_lists(plan, per_head_lists, row_ptr)
     _check(load().bsa_attn_fwd_natural_e4m3(plan.handle, _ptr(q8), _ptr(k8), _ptr(v8),
                                             _ptr(scales), _ptr(row_ptr), _ptr(col_idx),
                                             int(bool(per_head_lists)), float(scale), _ptr(o),
@@ -271,6 +344,9 @@ def bsa_attn_fwd_natural_e4m3(plan: Plan, q8, k8, v8, scales, row_ptr, col_idx,
 
 def bsa_lvsa_attn_fwd(plan: Plan, C: int, T_per: int, s: int, q, k, v, scale: float, o,
                       lse=None, stream=None):
+    for name, t in (("q", q), ("k", k), ("v", v), ("o", o)):
+        _need(name, t, _natural(plan))
+    _need("lse", lse, _natural(plan, 4) // plan.D)
     _check(load().bsa_lvsa_attn_fwd(plan.handle, C, T_per, s, _ptr(q), _ptr(k), _ptr(v),
                                     float(scale), _ptr(o), _ptr(lse), _stream(stream)),
            "bsa_lvsa_attn_fwd")

@@ -2,6 +2,7 @@
 // entry point validates on the host, then enqueues its kernel(s) on the
 // caller's stream; nothing is allocated per call.
 #include <cstdio>
+#include <new>
 #include <string>
 #include <vector>
 
@@ -108,8 +109,8 @@ bsa_status bsa_plan_create(bsa_plan_t* plan, int B, int Hh, int D, int T, int H,
   g.W = W;
   g.layout = layout;
   g.block = block;
-  g.P = H * W;
   if ((int64_t)H * W >= (1ll << 31)) return set_error(BSA_ERR_UNSUPPORTED, "frame too large");
+  g.P = H * W;
   if (layout == BSA_LAYOUT_FRAME) {
     g.ph = g.pw = 0;
     g.nbf = (g.P + block - 1) / block;
@@ -118,7 +119,7 @@ bsa_status bsa_plan_create(bsa_plan_t* plan, int B, int Hh, int D, int T, int H,
   } else if (layout == BSA_LAYOUT_TILE) {
     if (pool_h <= 0 || pool_w <= 0)
       return set_error(BSA_ERR_INVALID_ARG, "pool_h and pool_w must be positive");
-    if (pool_h * pool_w != block)
+    if ((int64_t)pool_h * pool_w != block)
       return set_error(BSA_ERR_INVALID_ARG, "pool_h * pool_w must equal the block size");
     g.ph = pool_h;
     g.pw = pool_w;
@@ -136,11 +137,18 @@ bsa_status bsa_plan_create(bsa_plan_t* plan, int B, int Hh, int D, int T, int H,
   if (chunks >= (1ll << 31) || nat_chunks >= (1ll << 31) || g.nblocks >= (1ll << 30))
     return set_error(BSA_ERR_UNSUPPORTED, "problem too large (index range)");
 
-  std::vector<uint32_t> tv((size_t)g.ntiles * 4, 0u);
+  // no exception may cross the C ABI: host allocations are checked here
+  std::vector<uint32_t> tv;
+  try {
+    tv.assign((size_t)g.ntiles * 4, 0u);
+  } catch (const std::bad_alloc&) {
+    return set_error(BSA_ERR_INVALID_ARG, "host memory for the slot map");
+  }
   for (int64_t s = 0; s < g.Npad; ++s)
     if (slot_holds_token(g, s)) tv[(size_t)(s >> 5)] |= 1u << (s & 31);
 
-  auto* p = new bsa_plan_s;
+  auto* p = new (std::nothrow) bsa_plan_s;
+  if (!p) return set_error(BSA_ERR_INVALID_ARG, "host memory for the plan");
   p->g = g;
   cudaError_t e = cudaGetDevice(&p->device);
   if (e == cudaSuccess) e = cudaMalloc(&p->d_tile_valid, tv.size() * sizeof(uint32_t));
@@ -247,12 +255,16 @@ bsa_status bsa_reorder_fwd(bsa_plan_t plan, const void* x0, void* y0, const void
   if ((st = check_ptr(x0, "x0")) != BSA_OK || (st = check_ptr(y0, "y0")) != BSA_OK) return st;
   const void* xs[3] = {x0, x1, x2};
   void* ys[3] = {y0, y1, y2};
+  // pairs 1 and 2 are optional, in order: a pair after an absent one is an error
   int nt = 1;
   for (int i = 1; i < 3; ++i) {
     if (!xs[i] && !ys[i]) break;
     if ((st = check_ptr(xs[i], "x")) != BSA_OK || (st = check_ptr(ys[i], "y")) != BSA_OK) return st;
     nt = i + 1;
   }
+  for (int i = nt + 1; i < 3; ++i)
+    if (xs[i] || ys[i])
+      return set_error(BSA_ERR_INVALID_ARG, "tensor pair 2 given without pair 1");
   cudaError_t e = launch_reorder_fwd(plan->g, xs, ys, nt, reinterpret_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? BSA_OK : cuda_error(e, "reorder_fwd launch");
 }

@@ -189,7 +189,8 @@ size_t bsa_draft_noalloc_max_scratch_bytes(void);
 
 /* Reorder (Draft Attention article, reorder paragraph): gather natural-layout
  * tensors into the plan's slot layout; empty slots are written as zero.
- * Up to three tensors in one launch: x1/y1 and x2/y2 may be NULL. */
+ * Up to three tensors in one launch: x1/y1 and x2/y2 may be NULL (both of a
+ * pair), x2/y2 only together with x1/y1; otherwise BSA_ERR_INVALID_ARG. */
 bsa_status bsa_reorder_fwd(bsa_plan_t plan, const void* x0, void* y0, const void* x1,
                            void* y1, const void* x2, void* y2, void* stream);
 

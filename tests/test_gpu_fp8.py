@@ -119,9 +119,10 @@ def test_attn_e4m3_full_size_sampled(cid):
 
 def test_attn_e4m3_rejects_unsupported_plans():
     x = torch.zeros((1, 512, 1, 64), dtype=torch.uint8, device="cuda")
+    o = torch.zeros((1, 512, 1, 64), dtype=torch.bfloat16, device="cuda")
     sc = torch.ones(3, dtype=torch.float32, device="cuda")
     buf = torch.zeros(4096, dtype=torch.int32, device="cuda")
     p64 = bsa.Plan(1, 1, 64, 2, 16, 16, bsa.LAYOUT_TILE, 8, 16, 128)    # D = 64
     with pytest.raises(bsa.BsaError) as ei:
-        bsa.bsa_attn_fwd_natural_e4m3(p64, x, x, x, sc, buf, buf, True, 0.125, x)
+        bsa.bsa_attn_fwd_natural_e4m3(p64, x, x, x, sc, buf, buf, True, 0.125, o)
     assert ei.value.status == 2

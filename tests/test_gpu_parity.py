@@ -115,6 +115,21 @@ def test_reorder_bit_exact(over, layout, blk):
     assert torch.equal(back.cpu().view(torch.int16), k.view(torch.int16))
 
 
+def test_reorder_rejects_a_third_pair_without_the_second():
+    plan = bsa.Plan(1, 1, 64, 8, 8, 8, bsa.LAYOUT_FRAME, block=64)
+    x = torch.zeros((1, 512, 1, 64), dtype=torch.bfloat16, device="cuda")
+    y = [torch.full((1, 1, plan.Npad, 64), 7.0, dtype=torch.bfloat16, device="cuda")
+         for _ in range(3)]
+    with pytest.raises(bsa.BsaError) as ei:
+        bsa.bsa_reorder_fwd(plan, x, y[0], None, None, x, y[2])
+    assert ei.value.status == 1
+    # rejected on the host: nothing was written
+    assert all((t == 7.0).all() for t in y)
+    bsa.bsa_reorder_fwd(plan, x, y[0], x, y[1], x, y[2])
+    bsa.bsa_poll_status(plan)
+    assert all((t == 0).all() for t in y)
+
+
 @pytest.mark.parametrize("cid,layout", [(3, "frame"), (4, "frame"), (5, "tile")])
 def test_reorder_round_trip_full_size(cid, layout):
     w = CONFIGS[cid]

@@ -52,6 +52,9 @@ def _create(lib, *args):
     ((1, 2, 64, 8, 8, 8, 1, 0, 2, 4), 1),       # pool sizes must be positive
     ((0, 2, 64, 8, 8, 8, 0, 0, 0, 64), 1),      # empty batch
     ((1, 2, 64, 8, 8, 8, 7, 0, 0, 64), 1),      # unknown layout
+    ((1, 2, 64, 8, 65536, 65536, 0, 0, 0, 64), 2),        # H * W beyond 32 bits
+    ((1, 2, 64, 8, 8, 8, 1, 65536, 65536, 64), 1),        # pool_h * pool_w beyond 32 bits
+    ((1, 2, 64, 8, 8, 8, 1, 128, 33554433, 128), 1),      # product wraps to 128 in 32 bits
 ])
 def test_plan_create_rejects_bad_geometry_on_host(lib, args, status):
     st, h = _create(lib, *args)

@@ -75,7 +75,10 @@ def test_noalloc_rejects_problems_above_its_scratch():
     assert bsa.bsa_draft_workspace_bytes(plan) > cap
     buf = torch.empty(16, dtype=torch.int32, device="cuda")
     x = torch.empty(8, dtype=torch.bfloat16, device="cuda")
+    # raw addresses: the binding's size checks pass them through, so the
+    # library's own scratch-size check is the one that answers
     with pytest.raises(bsa.BsaError) as ei:
-        bsa.bsa_draft_mask_noalloc(plan, x, x, 90, buf, buf, None)
+        bsa.bsa_draft_mask_noalloc(plan, x.data_ptr(), x.data_ptr(), 90, buf.data_ptr(),
+                                   buf.data_ptr(), None)
     assert ei.value.status == 2
     assert "32 MiB" in bsa.bsa_last_error()
