@@ -185,8 +185,12 @@ def run_reference(args, rank, world):
     del q, k, v
     vals = []
     desc, thr = "", 1
-    for i in range(args.warmup + args.steps):
-        val, thr, desc, _ = cpu_baseline(w, q_h, k_h, v_h, budget_s=args.ref_step_s, seed=i)
+    # each step samples for at most ref_step_s, less when there are many
+    # steps, so the whole run stays near two minutes of host time
+    n_all = args.warmup + args.steps
+    budget = min(args.ref_step_s, max(0.25, 120.0 / n_all))
+    for i in range(n_all):
+        val, thr, desc, _ = cpu_baseline(w, q_h, k_h, v_h, budget_s=budget, seed=i)
         if i >= args.warmup:
             vals.append(val)
     value = statistics.mean(vals)
@@ -452,6 +456,8 @@ def main():
         step(args.warmup + i)
         marks[i + 1].record(stream)
     torch.cuda.synchronize()
+    if dist:
+        dist.barrier()
     clk = clocks.stop()
     bsa.bsa_poll_status(att.plan)
     per_call = [marks[i].elapsed_time(marks[i + 1]) for i in range(args.steps)]
