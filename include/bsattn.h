@@ -17,9 +17,12 @@
  *
  * Conventions common to every entry point
  *  - Tensors are owned by the caller: device pointers, contiguous, 16-byte
- *    aligned.  Nothing is allocated per call; a plan owns only small index
- *    data and a device status word, allocated by bsa_plan_create on the
- *    device that is current at that time.
+ *    aligned, and at least as large as the plan's geometry implies (given
+ *    with each entry point).  The library sees only pointers and cannot
+ *    check sizes; the Python binding checks them before every call.
+ *    Nothing is allocated per call; a plan owns only small index data and a
+ *    device status word, allocated by bsa_plan_create on the device that is
+ *    current at that time.
  *  - Every call is asynchronous on `stream` (a cudaStream_t; NULL = legacy
  *    default stream) and returns after enqueueing its kernel(s).  Argument
  *    errors are detected on the host before anything is enqueued and
@@ -106,8 +109,8 @@ bsa_status bsa_plan_destroy(bsa_plan_t plan);
  * issued after it; returns BSA_ERR_INVALID_ARG for unknown values. */
 bsa_status bsa_plan_set_lvsa_variant(bsa_plan_t plan, int anchors, int window_order);
 
-/* Choose the pooling of bsa_draft_mask / bsa_draft_mask_noalloc with this
- * plan (default MEAN).  MAX takes the channel-wise maximum over the tile's
+/* Choose the pooling of bsa_draft_mask, bsa_draft_mask_noalloc and
+ * bsa_draft_mask_natural with this plan (default MEAN).  MAX takes the channel-wise maximum over the tile's
  * tokens inside the grid: the Draft Attention article reports trying max
  * pooling first and preferring the average at high sparsity. */
 bsa_status bsa_plan_set_draft_pooling(bsa_plan_t plan, int pooling);
@@ -188,13 +191,15 @@ bsa_status bsa_draft_mask_noalloc(bsa_plan_t plan, const void* q_slots, const vo
 size_t bsa_draft_noalloc_max_scratch_bytes(void);
 
 /* Reorder (Draft Attention article, reorder paragraph): gather natural-layout
- * tensors into the plan's slot layout; empty slots are written as zero.
+ * tensors x [B, N, Hh, D] into the plan's slot layout y [B, Hh, Npad, D]
+ * (2-byte elements, copied bit for bit); empty slots are written as zero.
  * Up to three tensors in one launch: x1/y1 and x2/y2 may be NULL (both of a
  * pair), x2/y2 only together with x1/y1; otherwise BSA_ERR_INVALID_ARG. */
 bsa_status bsa_reorder_fwd(bsa_plan_t plan, const void* x0, void* y0, const void* x1,
                            void* y1, const void* x2, void* y2, void* stream);
 
-/* Inverse reorder: slot layout -> natural layout; empty slots are dropped. */
+/* Inverse reorder: slot layout [B, Hh, Npad, D] -> natural layout
+ * [B, N, Hh, D], bit for bit; empty slots are dropped. */
 bsa_status bsa_reorder_inv(bsa_plan_t plan, const void* x_slots, void* x_nat, void* stream);
 
 /* Block-sparse attention forward (LVSA section 2 and the Draft Attention
