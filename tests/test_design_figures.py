@@ -1,0 +1,109 @@
+"""Figures the design notes quote about the masks, recomputed from the oracle
+on the synthetic workloads (CPU).
+
+* Draft lists (Wan-1.3B-shape draft workload, 12 heads, 34 of 336 blocks
+  kept per row): a query block shares few kept blocks with its neighbours
+  (6.7 with the right one, 8.4 with the lower one, 10.3 with its best partner
+  in the frame), so two query tiles sharing K/V would execute far more MMAs.
+* The top-k favours partly empty edge blocks (57.5 % of the kept blocks
+  against 43.8 % of all blocks): a kept key block is 65 % full on average,
+  and 49.6 % of the executed attention work is attended.
+* The one-kernel LVSA tiling (256 queries per CTA; key tiles are the
+  128-token pieces of each run of consecutive frames of the union of the
+  CTA's frame sets) at the Wan-1.3B 6x workload: 96.0 % of the multiplied
+  pairs are attended at steps 0-5 and 96.4 % at steps 6-11; run tail tiles
+  take 3.4 and 3.0 points (11 and 10 anchors), CTAs straddling two frames
+  0.6.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from synth import CONFIGS, make_qkv
+
+
+@pytest.fixture(scope="module")
+def draft_case():
+    w = CONFIGS[2]
+    q, k, _ = make_qkv(w)
+    kv = oracle.draft_blocks(q.to(torch.float64).numpy(), k.to(torch.float64).numpy(), w.T, w.H,
+                             w.W, w.draft_ph, w.draft_pw, w.draft_sparsity)
+    return w, kv
+
+
+def _grid(w):
+    return -(-w.H // w.draft_ph), -(-w.W // w.draft_pw)
+
+
+def test_draft_lists_of_neighbouring_query_blocks_share_few_blocks(draft_case):
+    w, kv = draft_case
+    TH, TW = _grid(w)
+    _, Hh, nb, keep = kv.shape
+    assert keep == 34 and nb == 336
+    right, below, best = [], [], []
+    for h in range(Hh):
+        for blk in range(nb):
+            t, r = divmod(blk, TH * TW)
+            i, j = divmod(r, TW)
+            own = kv[0, h, blk]
+            if j + 1 < TW:
+                right.append(len(np.intersect1d(own, kv[0, h, blk + 1])))
+            if i + 1 < TH:
+                below.append(len(np.intersect1d(own, kv[0, h, blk + TW])))
+            f0 = t * TH * TW
+            best.append(max(len(np.intersect1d(own, kv[0, h, o]))
+                            for o in range(f0, f0 + TH * TW) if o != blk))
+    assert np.mean(right) == pytest.approx(6.7, abs=0.1)
+    assert np.mean(below) == pytest.approx(8.4, abs=0.1)
+    assert np.mean(best) == pytest.approx(10.3, abs=0.1)
+
+
+def test_top_k_favours_partly_empty_edge_blocks(draft_case):
+    w, kv = draft_case
+    TH, TW = _grid(w)
+    ph, pw = w.draft_ph, w.draft_pw
+    nvalid = np.array([min(ph, w.H - i * ph) * min(pw, w.W - j * pw)
+                       for _ in range(w.T) for i in range(TH) for j in range(TW)])
+    kept = nvalid[kv]
+    assert (kept < 128).mean() == pytest.approx(0.575, abs=0.005)
+    assert (nvalid < 128).mean() == pytest.approx(0.438, abs=0.001)
+    assert kept.mean() / 128 == pytest.approx(0.65, abs=0.005)
+    attended = (nvalid[None, None, :, None] * kept).sum()
+    assert attended / (128 * 128 * kv.size) == pytest.approx(0.496, abs=0.002)
+
+
+def _lvsa_tiling(w, s):
+    T, P = w.T, w.H * w.W
+    N = T * P
+    A = [set(int(f) for f in r) for r in oracle.lvsa_frame_sets(T, w.lvsa_C, w.lvsa_T_per, s)]
+    executed = attended = tails = straddle = 0
+    for q0 in range(0, N, 256):
+        rows = range(q0, min(q0 + 256, N))
+        U = set().union(*(A[t] for t in {n // P for n in rows}))
+        runs = []
+        for f in sorted(U):
+            if runs and runs[-1][1] == f - 1:
+                runs[-1][1] = f
+            else:
+                runs.append([f, f])
+        keys = sum(-(-((b - a + 1) * P) // 128) * 128 for a, b in runs)
+        executed += 256 * keys
+        attended += sum(len(A[n // P]) * P for n in rows)
+        tails += 256 * (keys - len(U) * P)
+        straddle += sum((len(U) - len(A[n // P])) * P for n in rows)
+    return attended / executed, tails / executed, straddle / executed
+
+
+def test_lvsa_one_kernel_tiling_attends_96_percent():
+    w = CONFIGS[3]
+    early = [_lvsa_tiling(w, s) for s in (0, 5)]
+    late = [_lvsa_tiling(w, s) for s in (6, 11)]
+    for frac, tails, straddle in early:                 # 11 anchors
+        assert frac == pytest.approx(0.960, abs=0.001)
+        assert tails == pytest.approx(0.034, abs=0.001)
+    for frac, tails, straddle in late:                  # 10 anchors
+        assert frac == pytest.approx(0.964, abs=0.001)
+        assert tails == pytest.approx(0.030, abs=0.001)
+    for frac, tails, straddle in early + late:
+        assert straddle == pytest.approx(0.006, abs=0.001)
