@@ -14,6 +14,9 @@ on the synthetic workloads (CPU).
   pairs are attended at steps 0-5 and 96.4 % at steps 6-11; run tail tiles
   take 3.4 and 3.0 points (11 and 10 anchors), CTAs straddling two frames
   0.6.
+* The two readings of the window's growth order differ on 5 of 32 rows of
+  the tiny workload, 570 of 1512 at Wan-1.3B 6x and 3 of 1040 at
+  HunyuanVideo 2x.
 """
 import numpy as np
 import pytest
@@ -107,3 +110,18 @@ def test_lvsa_one_kernel_tiling_attends_96_percent():
         assert tails == pytest.approx(0.030, abs=0.001)
     for frac, tails, straddle in early + late:
         assert straddle == pytest.approx(0.006, abs=0.001)
+
+
+def test_the_two_window_readings_differ_on_the_stated_rows():
+    # rows (t, s) where reading A (distance order) and reading B (alternating
+    # pointers) give different frame sets, over one anchor period
+    expect = {1: (5, 32), 3: (570, 1512), 4: (3, 1040)}
+    for cid, (n_diff, n_rows) in expect.items():
+        w = CONFIGS[cid]
+        diff = rows = 0
+        for s in range(w.lvsa_T_per):
+            a = oracle.lvsa_frame_sets(w.T, w.lvsa_C, w.lvsa_T_per, s)
+            b = oracle.lvsa_frame_sets(w.T, w.lvsa_C, w.lvsa_T_per, s, order="alternate")
+            diff += int((a != b).any(axis=1).sum())
+            rows += w.T
+        assert (diff, rows) == (n_diff, n_rows)
