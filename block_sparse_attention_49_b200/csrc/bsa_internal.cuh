@@ -66,7 +66,7 @@ struct bsa_plan_s {
   unsigned int* d_status = nullptr;  // device status word
   uint64_t wait_limit_ns = 2000000000ull;
   int lvsa_anchors = BSA_ANCHORS_ROTATING;  // bsa_plan_set_lvsa_variant
-  int lvsa_window = BSA_WINDOW_DISTANCE;
+  int lvsa_window = BSA_WINDOW_ALTERNATE;
   int draft_pooling = BSA_POOL_MEAN;        // bsa_plan_set_draft_pooling
   uint32_t* d_amax = nullptr;               // [3][B][Hh] scratch of bsa_quantize_e4m3
 };

@@ -8,20 +8,21 @@
 // then expanded to key blocks on the frame layout (every block of every frame
 // in A(t), ascending) for each query block of frame t.
 //
-// The window grows t+1, t-1, t+2, t-2, ..., skipping frames outside [0, T)
-// and frames already present.  Equivalently, with base = G_s U {t} and
-// need = C - |base|, a frame f outside base joins iff fewer than `need`
-// frames outside base come before it in that order (closer to t, or at the
-// same distance on the right).  Each thread evaluates that count for its
-// frames in O(1) from a prefix sum, so the set needs no serial loop.
+// Growth order.  By default a right and a left pointer take turns, right
+// first, each skipping frames already present (the anchors); a side that
+// runs off the grid stops and the other continues.  With base = G_s U {t},
+// need = C - |base| and nR / nL frames outside base right / left of t, the
+// right side then takes kR = min(nR, max(ceil(need/2), need - nL)) of its
+// frames outside base, nearest first, and the left side the other
+// need - kR of its own.  The other order (distance: t+1, t-1, t+2, t-2, ...,
+// skipping frames outside [0, T) and frames already present) admits a frame
+// f outside base iff fewer than `need` frames outside base come before it
+// (closer to t, or at the same distance on the right).  Either way each
+// thread decides membership for its frames in O(1) from a prefix-sum rank,
+// so the set needs no serial loop.
 //
 // Variants (chosen by the caller): T_per = 0 means no anchors (the sliding
-// window); fixed-grid anchors are the rotating ones at s = 0.  With the
-// alternating growth order (a right and a left pointer taking turns, right
-// first, each skipping frames already present; a side that runs off the
-// grid stops) the right side takes kR = min(nR, max(ceil(need/2), need - nL))
-// of its nR frames outside base, nearest first, and the left side the other
-// need - kR of its nL; membership is again a prefix-sum rank.
+// window); fixed-grid anchors are the rotating ones at s = 0.
 //
 // One CTA per query block (grid nbf x T); each writes its CSR row.
 #include "bsa_internal.cuh"

@@ -15,7 +15,7 @@ import math
 
 import torch
 
-from . import (ANCHORS_ROTATING, LAYOUT_FRAME, LAYOUT_TILE, POOL_MEAN, WINDOW_DISTANCE, Plan,
+from . import (ANCHORS_ROTATING, LAYOUT_FRAME, LAYOUT_TILE, POOL_MEAN, WINDOW_ALTERNATE, Plan,
                bsa_attn_fwd, bsa_attn_fwd_natural, bsa_attn_fwd_natural_e4m3,
                bsa_draft_keep_count, bsa_draft_mask, bsa_draft_mask_natural,
                bsa_draft_workspace_bytes, bsa_quantize_e4m3,
@@ -48,7 +48,7 @@ class LvsaAttention(_Base):
     `window_order` select a mask variant (bsa_plan_set_lvsa_variant)."""
 
     def __init__(self, B, Hh, D, T, H, W, C, T_per, block=128, device="cuda", scale=None,
-                 anchors=ANCHORS_ROTATING, window_order=WINDOW_DISTANCE):
+                 anchors=ANCHORS_ROTATING, window_order=WINDOW_ALTERNATE):
         self.plan = Plan(B, Hh, D, T, H, W, LAYOUT_FRAME, block=block)
         bsa_plan_set_lvsa_variant(self.plan, anchors, window_order)
         self.C, self.T_per = C, T_per

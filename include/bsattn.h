@@ -77,8 +77,9 @@ typedef enum {
   BSA_ANCHORS_NONE = 2      /* no global frames: the sliding window alone       */
 } bsa_anchor_mode;
 typedef enum {
-  BSA_WINDOW_DISTANCE = 0,  /* grow t+1, t-1, t+2, t-2, ... (default)          */
-  BSA_WINDOW_ALTERNATE = 1  /* right and left pointers take turns, right first */
+  BSA_WINDOW_DISTANCE = 0,  /* grow t+1, t-1, t+2, t-2, ...                     */
+  BSA_WINDOW_ALTERNATE = 1  /* right and left pointers take turns, right first
+                               (default)                                        */
 } bsa_window_order;
 
 /* Draft pooling (bsa_plan_set_draft_pooling). */
@@ -98,15 +99,18 @@ bsa_status bsa_plan_create(bsa_plan_t* plan, int B, int Hh, int D, int T, int H,
 bsa_status bsa_plan_destroy(bsa_plan_t plan);
 
 /* Choose the LVSA mask variant used by bsa_lvsa_mask and bsa_lvsa_attn_fwd
- * with this plan (default ROTATING, DISTANCE).  "LVSA", section 2 "Core
+ * with this plan (default ROTATING, ALTERNATE).  "LVSA", section 2 "Core
  * mechanism", contrasts its rotating anchors with fixed-grid global frames,
  * and the page's introduction lists plain sliding windows; FIXED and NONE
  * give those patterns under the same budget C.  The page leaves the growth
- * order of the extended window open: DISTANCE adds the nearest frame not yet
- * present (ties to the right), ALTERNATE lets a right and a left pointer take
- * turns (right first), each moving past frames already present; a side that
- * runs off [0, T) stops and the other continues.  Takes effect for calls
- * issued after it; returns BSA_ERR_INVALID_ARG for unknown values. */
+ * order of the extended window open: ALTERNATE lets a right and a left
+ * pointer take turns (right first), each moving past frames already present
+ * (the anchors); a side that runs off [0, T) stops and the other continues.
+ * That is the window "extended alternately right then left, skipping anchors,
+ * clamped at the edges" of the workloads these kernels are measured on, and
+ * the default.  DISTANCE adds the nearest frame not yet present (ties to the
+ * right).  Takes effect for calls issued after it; returns
+ * BSA_ERR_INVALID_ARG for unknown values. */
 bsa_status bsa_plan_set_lvsa_variant(bsa_plan_t plan, int anchors, int window_order);
 
 /* Choose the pooling of bsa_draft_mask, bsa_draft_mask_noalloc and

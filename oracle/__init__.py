@@ -19,11 +19,13 @@ what the method computes, written from the pages:
 
 All floating point is fp64.  bf16 inputs convert to fp64 exactly.
 
-Readings of points the pages leave open (each listed in the design notes):
-* window extension order: offsets +1, -1, +2, -2, ... around t, skipping
-  frames outside [0,T) and frames already in the set, until |A(t)| = C
-  (reading A, the default); reading B, alternating right and left pointers,
-  is available as order="alternate";
+Readings of points the pages leave open:
+* window extension order: a right and a left pointer take turns, right
+  first, each moving past frames already in the set (anchors) and stopping
+  at the grid's edge, until |A(t)| = C (reading B, the default: the tiny
+  workload's definition says the window is extended alternately right then
+  left, skipping anchors, clamped at the edges); reading A, offsets +1, -1,
+  +2, -2, ... around t, is available as order="distance";
 * anchors G_s = {f : (f - s) mod T_per == 0}; the fixed-grid and window-only
   variants take {f : f mod T_per == 0} and the empty set;
 * draft pooling averages the valid tokens of a tile only (grid-edge tiles are
@@ -55,7 +57,7 @@ import numpy as np
 
 
 ANCHOR_MODES = ("rotating", "fixed", "none")
-WINDOW_ORDERS = ("distance", "alternate")
+WINDOW_ORDERS = ("alternate", "distance")
 
 
 def lvsa_anchors(T: int, T_per: int, s: int, anchors: str = "rotating") -> list[int]:
@@ -78,19 +80,19 @@ def lvsa_anchors(T: int, T_per: int, s: int, anchors: str = "rotating") -> list[
 
 
 def lvsa_frame_set(t: int, T: int, C: int, T_per: int, s: int, anchors: str = "rotating",
-                   order: str = "distance") -> list[int]:
+                   order: str = "alternate") -> list[int]:
     """A(t) = G_s U W(t) for query frame t, with |A(t)| = C exactly.
 
     W(t) is a local window centred on t that grows past anchors it overlaps so
     that the budget C is always met (LVSA, section 2, "Extended adaptive
     window").  The page does not fix the growth order; two readings:
 
+    * "alternate" (the default): a right pointer and a left pointer take
+      turns, right first; each turn moves its pointer past frames already in
+      the set and adds the next frame on its side; a side that runs off the
+      grid stops and the other side continues;
     * "distance": t+1, t-1, t+2, t-2, ...; frames outside [0, T) and frames
-      already in the set are skipped and cost no budget;
-    * "alternate": a right pointer and a left pointer take turns, right
-      first; each turn moves its pointer past frames already in the set and
-      adds the next frame on its side; a side that runs off the grid stops
-      and the other side continues.
+      already in the set are skipped and cost no budget.
     """
     if not (0 <= t < T) or C > T or (anchors != "none" and T_per <= 0):
         raise ValueError("bad LVSA arguments")
@@ -126,7 +128,7 @@ def lvsa_frame_set(t: int, T: int, C: int, T_per: int, s: int, anchors: str = "r
 
 
 def lvsa_frame_sets(T: int, C: int, T_per: int, s: int, anchors: str = "rotating",
-                    order: str = "distance") -> np.ndarray:
+                    order: str = "alternate") -> np.ndarray:
     """int32 [T, C]: row t is A(t) in ascending order."""
     return np.array([lvsa_frame_set(t, T, C, T_per, s, anchors, order) for t in range(T)],
                     dtype=np.int32).reshape(T, C)

@@ -8,6 +8,7 @@ tables, constructed inputs with known answers) or a library routine
 import itertools
 import math
 import os
+from fractions import Fraction
 
 import numpy as np
 import pytest
@@ -78,16 +79,27 @@ def test_window_rule_equals_nearest_non_anchor_closed_form():
                         need = nanch + (0 if (t - s) % T_per == 0 else 1)
                         if need > C:
                             with pytest.raises(ValueError):
-                                oracle.lvsa_frame_set(t, T, C, T_per, s)
+                                oracle.lvsa_frame_set(t, T, C, T_per, s, order="distance")
                             continue
-                        assert oracle.lvsa_frame_set(t, T, C, T_per, s) == \
+                        assert oracle.lvsa_frame_set(t, T, C, T_per, s, order="distance") == \
                             _closed_form(t, T, C, T_per, s), (T, C, T_per, s, t)
                         n += 1
     assert n > 10000
 
 
-# Hand-derived from the rule for the tiny workload (T=8, C=4, T_per=4).
-HAND_C1 = {
+# Hand-derived from the two growth rules for the tiny workload (T=8, C=4,
+# T_per=4).  Reading B, the default, follows the workload's own wording: the
+# window is extended alternately right then left, skipping anchors, clamped
+# at the edges.  E.g. s=0, t=3: G={0,4}, one frame to add; the right pointer
+# skips anchor 4 and takes 5 (reading B), while the nearest frame not yet
+# present is 2 (reading A, distance order).
+HAND_C1_ALTERNATE = {
+    0: ["0124", "0124", "0234", "0345", "0345", "0456", "0467", "0467"],
+    1: ["0125", "0125", "1235", "1345", "1456", "1456", "1567", "1567"],
+    2: ["0126", "1236", "1236", "2346", "2456", "2567", "2567", "2567"],
+    3: ["0137", "1237", "2347", "2347", "3457", "3567", "3567", "3567"],
+}
+HAND_C1_DISTANCE = {
     0: ["0124", "0124", "0234", "0234", "0345", "0456", "0467", "0467"],
     1: ["0125", "0125", "1235", "1345", "1345", "1456", "1567", "1567"],
     2: ["0126", "0126", "1236", "2346", "2456", "2456", "2567", "2567"],
@@ -95,19 +107,31 @@ HAND_C1 = {
 }
 
 
-def test_tiny_case_hand_table_and_golden():
+def _read_golden(name):
     gold = {}
-    with open(os.path.join(GOLDEN, "lvsa_tiny_T8_C4_Tper4.txt")) as f:
+    with open(os.path.join(GOLDEN, name)) as f:
         for line in f:
             if line.startswith("#") or not line.strip():
                 continue
             s, t, *fr = map(int, line.split())
             gold[(s, t)] = fr
-    for s, rows in HAND_C1.items():
-        A = oracle.lvsa_frame_sets(8, 4, 4, s)
+    return gold
+
+
+@pytest.mark.parametrize("order,hand,golden", [
+    ("alternate", HAND_C1_ALTERNATE, "lvsa_tiny_T8_C4_Tper4.txt"),
+    ("distance", HAND_C1_DISTANCE, "lvsa_tiny_T8_C4_Tper4_distance.txt")])
+def test_tiny_case_hand_table_and_golden(order, hand, golden):
+    gold = _read_golden(golden)
+    for s, rows in hand.items():
+        A = oracle.lvsa_frame_sets(8, 4, 4, s, order=order)
         for t, r in enumerate(rows):
             assert list(A[t]) == [int(c) for c in r], (s, t)
             assert gold[(s, t)] == [int(c) for c in r]
+    if order == "alternate":                     # the default
+        for s in hand:
+            assert (oracle.lvsa_frame_sets(8, 4, 4, s) ==
+                    oracle.lvsa_frame_sets(8, 4, 4, s, order=order)).all()
 
 
 @pytest.mark.parametrize("cid", [1, 3, 4])
@@ -366,7 +390,7 @@ def test_lvsa_mask_attention_matches_sdpa_with_frame_mask():
         frame = np.arange(w.N) // w.P
         allowed = np.zeros((w.T, w.T), bool)
         for t in range(w.T):
-            allowed[t, HAND_C1_SETS[s][t]] = True
+            allowed[t, HAND_C1_SETS[s][t]] = True         # reading B, the default
         mask = allowed[frame[:, None], frame[None, :]]
         ref = _sdpa64(q[0].transpose(1, 0, 2), k[0].transpose(1, 0, 2),
                       v[0].transpose(1, 0, 2), mask, 1 / 8.0)
@@ -374,7 +398,7 @@ def test_lvsa_mask_attention_matches_sdpa_with_frame_mask():
                                    rtol=1e-12, atol=1e-12)
 
 
-HAND_C1_SETS = {s: [[int(c) for c in r] for r in rows] for s, rows in HAND_C1.items()}
+HAND_C1_SETS = {s: [[int(c) for c in r] for r in rows] for s, rows in HAND_C1_ALTERNATE.items()}
 
 
 def test_draft_mask_attention_matches_sdpa_with_block_mask():
@@ -473,8 +497,9 @@ def test_alternate_order_hand_case():
     # T = 8, C = 4, T_per = 4, s = 0, t = 3: G = {0, 4}, one frame to add.
     # distance order tries +1 = 4 (already there), then -1 = 2;
     # alternate order moves the right pointer past 4 and takes 5.
-    assert oracle.lvsa_frame_set(3, 8, 4, 4, 0) == [0, 2, 3, 4]
+    assert oracle.lvsa_frame_set(3, 8, 4, 4, 0, order="distance") == [0, 2, 3, 4]
     assert oracle.lvsa_frame_set(3, 8, 4, 4, 0, order="alternate") == [0, 3, 4, 5]
+    assert oracle.lvsa_frame_set(3, 8, 4, 4, 0) == [0, 3, 4, 5]          # the default
 
 
 def test_alternate_order_closed_form():
@@ -597,3 +622,124 @@ def test_fp8_quantize_is_exact_for_values_on_the_grid_with_power_of_two_scales()
     s = oracle.fp8_scales(x)
     assert s[0, 0] == np.float32(2.0 ** -5)
     np.testing.assert_array_equal(oracle.fp8_dequantize(oracle.fp8_quantize(x, s), s), x)
+
+
+# ---------------------------------------------------------------------------
+# The draft attention map (Draft Attention article: the low-resolution
+# attention map softmax(Qbar Kbar^T / sqrt(D)) of the pooled queries and
+# keys), the fp64 evaluation order the selection follows, and the LVSA block
+# list at several blocks per frame
+# ---------------------------------------------------------------------------
+
+
+def test_draft_map_matches_library_softmax_over_key_blocks():
+    rng = np.random.default_rng(23)
+    D = 64
+    L = rng.standard_normal((2, 3, 7, 11)) * 9.0
+    got = oracle.draft_map(L, D)
+    ref = torch.softmax(torch.from_numpy(L) / math.sqrt(D), dim=-1).numpy()
+    np.testing.assert_allclose(got, ref, rtol=1e-13, atol=1e-16)
+    # a distribution over key blocks for every query block, not over queries
+    np.testing.assert_allclose(got.sum(axis=-1), 1.0, rtol=0, atol=1e-14)
+    assert not np.allclose(got.sum(axis=-2), 1.0)
+
+
+def test_draft_map_hand_cases():
+    D = 128
+    # equal logits: uniform over the Nb key blocks
+    L = np.full((1, 1, 3, 5), 2.5)
+    np.testing.assert_allclose(oracle.draft_map(L, D), 0.2, rtol=0, atol=1e-16)
+    # one logit ahead by delta*sqrt(D): weight ratio exp(delta), so with Nb
+    # blocks the leader holds e^delta / (e^delta + Nb - 1)
+    for delta in (0.5, 1.0, 3.0):
+        row = np.zeros((1, 1, 1, 4))
+        row[..., 2] = delta * math.sqrt(D)
+        m = oracle.draft_map(row, D)[0, 0, 0]
+        assert m[2] / m[0] == pytest.approx(math.exp(delta), rel=1e-13)
+        assert m[2] == pytest.approx(math.exp(delta) / (math.exp(delta) + 3), rel=1e-13)
+    # a shift of a whole row changes nothing; scaling by sqrt(D) is applied once
+    L = np.array([[[[0.0, math.sqrt(D) * math.log(3.0)]]]])
+    np.testing.assert_allclose(oracle.draft_map(L, D)[0, 0, 0], [0.25, 0.75], rtol=1e-14)
+    np.testing.assert_allclose(oracle.draft_map(L + 1e3, D), oracle.draft_map(L, D), rtol=1e-12)
+
+
+def test_pool_sums_in_row_major_order():
+    # one 2 x 2 tile whose sum depends on the order: row-major (a, then b)
+    # adds 2^-53 + 2^-53 = 2^-52 before the 1, which then survives; the
+    # column-major order adds 2^-53 to 1 first, which rounds away.
+    T, H, W, ph, pw = 1, 2, 2, 2, 2
+    x = np.zeros((1, 4, 1, 1))
+    x[0, 0, 0, 0] = 2.0 ** -53        # (a, b) = (0, 0)
+    x[0, 1, 0, 0] = 2.0 ** -53        # (0, 1)
+    x[0, 2, 0, 0] = 1.0               # (1, 0)
+    x[0, 3, 0, 0] = 0.0               # (1, 1)
+    got = oracle.draft_pool(x, T, H, W, ph, pw)[0, 0, 0, 0]
+    assert got == (1.0 + 2.0 ** -52) / 4
+    assert ((2.0 ** -53 + 1.0) + 2.0 ** -53) / 4 != got     # the other order differs
+
+
+def test_logits_are_sequential_and_unfused():
+    # channel 0 first: acc = -(1 + 2^-29); channel 1 adds the rounded product
+    # x*x with x = 1 + 2^-30, i.e. 1 + 2^-29 (the exact square carries an
+    # extra 2^-60), so the sum is exactly 0.  A fused multiply-add would keep
+    # 2^-60; the reversed order would give the same 0 here, so a second
+    # case pins the order: 1, then 2^-53 twice, rounds back to 1 each time.
+    x = 1.0 + 2.0 ** -30
+    q = np.array([1.0, x]).reshape(1, 1, 1, 2)
+    k = np.array([-(1.0 + 2.0 ** -29), x]).reshape(1, 1, 1, 2)
+    assert oracle.draft_logits(q, k)[0, 0, 0, 0] == 0.0
+    # the exact value a fused multiply-add would round: 2^-60, not 0
+    assert Fraction(x) * Fraction(x) - Fraction(1.0 + 2.0 ** -29) == Fraction(1, 2 ** 60)
+    q = np.ones((1, 1, 1, 3))
+    k = np.array([1.0, 2.0 ** -53, 2.0 ** -53]).reshape(1, 1, 1, 3)
+    assert oracle.draft_logits(q, k)[0, 0, 0, 0] == 1.0                 # c = 0, 1, 2
+    assert (2.0 ** -53 + 2.0 ** -53) + 1.0 == 1.0 + 2.0 ** -52           # reversed differs
+
+
+def test_lvsa_block_csr_literal_table_two_blocks_per_frame():
+    # T=3, C=2, T_per=3, s=0: G={0}; A(0)={0,1}, A(1)={0,1}, A(2)={0,2}.
+    # Two blocks per frame: frame f owns blocks 2f and 2f+1, and both query
+    # blocks of a frame carry that frame's list.
+    A = oracle.lvsa_frame_sets(3, 2, 3, 0)
+    assert A.tolist() == [[0, 1], [0, 1], [0, 2]]
+    rp, ci = oracle.lvsa_block_csr(A, 2)
+    assert rp.tolist() == [0, 4, 8, 12, 16, 20, 24]
+    rows = [ci[rp[r]:rp[r + 1]].tolist() for r in range(6)]
+    assert rows == [[0, 1, 2, 3], [0, 1, 2, 3], [0, 1, 2, 3], [0, 1, 2, 3],
+                    [0, 1, 4, 5], [0, 1, 4, 5]]
+    # three blocks per frame, frame sets of a later step
+    A = oracle.lvsa_frame_sets(3, 2, 3, 2)          # G={2}: A = {0,2}, {1,2}, {1,2}
+    assert A.tolist() == [[0, 2], [1, 2], [1, 2]]
+    rp, ci = oracle.lvsa_block_csr(A, 3)
+    assert ci[rp[0]:rp[1]].tolist() == [0, 1, 2, 6, 7, 8]
+    assert ci[rp[5]:rp[6]].tolist() == [3, 4, 5, 6, 7, 8]
+    assert ci[rp[8]:rp[9]].tolist() == [3, 4, 5, 6, 7, 8]
+
+
+@pytest.mark.parametrize("order", ["alternate", "distance"])
+def test_lvsa_csr_attention_matches_sdpa_with_several_blocks_per_frame(order):
+    # frames of 15 tokens on 4-token blocks: 4 blocks per frame, the last one
+    # holding 3 tokens and one empty slot; the token mask comes straight from
+    # the frame sets, not from the block list
+    T, H, W, D, blk, C, T_per = 6, 3, 5, 8, 4, 3, 4
+    P = H * W
+    rng = np.random.default_rng(29)
+    q, k, v = (rng.standard_normal((1, T * P, 2, D)) for _ in range(3))
+    perm, Npad = oracle.frame_layout_perm(T, H, W, blk)
+    nbf = Npad // (T * blk)
+    assert nbf == 4
+    valid = oracle.slot_valid(perm, Npad)
+    for s in range(T_per):
+        A = oracle.lvsa_frame_sets(T, C, T_per, s, order=order)
+        rp, ci = oracle.lvsa_block_csr(A, nbf)
+        O, _ = oracle.masked_attention(*(oracle.reorder_fwd(x, perm, Npad) for x in (q, k, v)),
+                                       valid, blk, rp, ci, False, 0.35)
+        frame = np.arange(T * P) // P
+        allowed = np.zeros((T, T), bool)
+        for t in range(T):
+            allowed[t, A[t]] = True
+        mask = allowed[frame[:, None], frame[None, :]]
+        ref = _sdpa64(q[0].transpose(1, 0, 2), k[0].transpose(1, 0, 2),
+                      v[0].transpose(1, 0, 2), mask, 0.35)
+        np.testing.assert_allclose(oracle.reorder_inv(O, perm)[0].transpose(1, 0, 2), ref,
+                                   rtol=1e-12, atol=1e-12)
