@@ -16,6 +16,8 @@ and its O out, overlapped with the neighbouring steps' compute
     python bench.py --kernel-table      # every kernel on every workload, one JSON line each
     python bench.py --draft-pipelines H # the three draft pipelines, twice, on H heads
                                         # of the 40-head draft workload (for profilers)
+    python bench.py --hbm-kernels C     # every HBM-bound kernel, twice, on workload C
+                                        # (for DRAM-counter captures)
 
 Under torchrun (N > 1) every rank runs its own batch (the path shards over
 batch x heads with no data exchange): weak scaling, max time over ranks.
@@ -377,6 +379,53 @@ def draft_pipelines(heads: int):
     print(json.dumps({"draft_pipelines": w.name, "heads": heads}), flush=True)
 
 
+def hbm_kernels(cid: int):
+    """Runs every HBM-bound kernel twice on workload `cid`: the frame- and
+    tile-layout reorders (forward and inverse), both draft masks (pooling and
+    scoring) and the e4m3 quantization.  A fixed launch sequence for DRAM
+    counter captures.  Prints one line with the algorithmic bytes per launch
+    of each kernel."""
+    import block_sparse_attention_49_b200 as bsa
+    from block_sparse_attention_49_b200.pipeline import DraftAttention
+
+    w = CONFIGS[cid]
+    q, k, v = make_qkv(w, device="cuda")
+    out = torch.empty_like(q)
+    tok = w.B * w.N * w.Hh * w.D * 2
+    fr = bsa.Plan(w.B, w.Hh, w.D, w.T, w.H, w.W, bsa.LAYOUT_FRAME, block=128)
+    shape = (w.B, w.Hh, fr.Npad, w.D)
+    fq, fk, fv = (torch.empty(shape, dtype=torch.bfloat16, device="cuda") for _ in range(3))
+    att = DraftAttention(w.B, w.Hh, w.D, w.T, w.H, w.W, w.draft_ph or 8, w.draft_pw or 16,
+                         w.draft_sparsity or 90)
+    nb = att.plan.nblocks
+    pooled = 2 * w.B * w.Hh * nb * w.D * 8
+    for _ in range(2):
+        bsa.bsa_reorder_fwd(fr, q, fq, k, fk, v, fv)
+        bsa.bsa_reorder_inv(fr, fq, out)
+        att.gather(q, k, v)
+        bsa.bsa_reorder_inv(att.plan, att.q_s, out)
+        att.mask()
+        bsa.bsa_draft_mask_natural(att.plan, q, k, att.sparsity, att.row_ptr, att.col_idx,
+                                   None, att.workspace)
+        att.quantize(q, k, v)
+    torch.cuda.synchronize()
+    bsa.bsa_poll_status(fr)
+    bsa.bsa_poll_status(att.plan)
+    print(json.dumps({
+        "hbm_kernels": w.name, "tokens": w.N, "heads": w.Hh, "head_dim": w.D,
+        "algo_bytes_per_launch": {
+            "reorder_fwd_kernel (Q K V, either layout)": 3 * 2 * tok,
+            "reorder_inv_kernel (O, either layout)": 2 * tok,
+            "draft_pool_kernel (tile-layout Q K slots read, pooled fp64 written)":
+                2 * w.B * w.Hh * att.plan.Npad * w.D * 2 + pooled,
+            "draft_pool_nat_kernel (natural Q K read, pooled fp64 written)": 2 * tok + pooled,
+            "draft_score_topk_kernel (pooled fp64 read, lists written)":
+                pooled + 4 * att.col_idx.numel(),
+            "e4m3_amax_kernel (Q K V read)": 3 * tok,
+            "e4m3_convert_kernel (Q K V read, codes written)": 3 * tok + 3 * tok // 2},
+        "slots": {"frame_Npad": fr.Npad, "tile_Npad": att.plan.Npad}}), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -395,7 +444,13 @@ def main():
     ap.add_argument("--table-reps", type=int, default=10)
     ap.add_argument("--draft-pipelines", type=int, default=0, metavar="HEADS",
                     help="run the three draft pipelines on HEADS heads (profiling)")
+    ap.add_argument("--hbm-kernels", type=int, default=0, metavar="CONFIG",
+                    help="run every HBM-bound kernel twice on workload CONFIG (profiling)")
     args = ap.parse_args()
+    if args.hbm_kernels:
+        torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", 0)))
+        hbm_kernels(args.hbm_kernels)
+        return
     if args.draft_pipelines:
         torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", 0)))
         draft_pipelines(args.draft_pipelines)
