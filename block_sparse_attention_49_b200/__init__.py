@@ -27,7 +27,7 @@ __all__ = [
     "bsa_draft_workspace_bytes", "bsa_draft_mask", "bsa_draft_mask_noalloc",
     "bsa_draft_noalloc_max_scratch_bytes", "bsa_reorder_fwd", "bsa_reorder_inv",
     "bsa_attn_fwd", "bsa_attn_fwd_natural", "bsa_draft_mask_natural", "bsa_quantize_e4m3",
-    "bsa_attn_fwd_natural_e4m3", "bsa_lvsa_attn_fwd", "bsa_poll_status", "bsa_set_wait_limit_ns", "bsa_selftest_timeout",
+    "bsa_attn_fwd_natural_e4m3", "bsa_draft_mask_natural_e4m3", "bsa_lvsa_attn_fwd", "bsa_poll_status", "bsa_set_wait_limit_ns", "bsa_selftest_timeout",
     "bsa_last_error", "bsa_version", "EXPORTED_SYMBOLS",
 ]
 
@@ -71,6 +71,8 @@ _SIGS = {
                               _c_p, _c_p]),
     "bsa_draft_mask_natural": (_c_int, [_c_p, _c_p, _c_p, _c_int, _c_p, _c_p, _c_p, _c_p, _c_sz, _c_p]),
     "bsa_quantize_e4m3": (_c_int, [_c_p] * 9),
+    "bsa_draft_mask_natural_e4m3": (_c_int, [_c_p, _c_p, _c_p, _c_p, _c_int, _c_p, _c_p, _c_p, _c_p,
+                                             _c_sz, _c_p, _c_p, _c_p, _c_p, _c_p]),
     "bsa_attn_fwd_natural_e4m3": (_c_int, [_c_p, _c_p, _c_p, _c_p, _c_p, _c_p, _c_p, _c_int,
                                            ctypes.c_float, _c_p, _c_p, _c_p]),
     "bsa_lvsa_attn_fwd": (_c_int, [_c_p, _c_int, _c_int, _c_int, _c_p, _c_p, _c_p, ctypes.c_float,
@@ -156,7 +158,7 @@ def _need_draft_outputs(plan, sparsity_pct: int, row_ptr, kv_idx, draft_map):
     if not 0 <= sparsity_pct < 100:
         return  # rejected by the library
     rows = plan.B * plan.Hh * plan.nblocks
-    keep = -(-plan.nblocks * (100 - sparsity_pct) // 100)
+    keep = plan.keep_count(sparsity_pct)
     _need("kv_idx", kv_idx, rows * keep * 4)
     _need("row_ptr", row_ptr, (rows + 1) * 4)
     _need("draft_map", draft_map, rows * plan.nblocks * 4)
@@ -182,6 +184,13 @@ class Plan:
         self.Npad = int(load().bsa_padded_tokens(h))
         self.nblocks = int(load().bsa_num_blocks(h))
         self.block = int(load().bsa_block_size(h))
+
+    def keep_count(self, sparsity_pct: int) -> int:
+        """Blocks kept per draft row at `sparsity_pct` (bsa_draft_keep_count)."""
+        k = int(load().bsa_draft_keep_count(self.handle, int(sparsity_pct)))
+        if k < 0:
+            raise BsaError(1, "bsa_draft_keep_count", load().bsa_last_error().decode())
+        return k
 
     def close(self):
         if getattr(self, "handle", None):
@@ -324,6 +333,24 @@ def bsa_quantize_e4m3(plan: Plan, q, k, v, q8, k8, v8, scales, stream=None):
     _need("scales", scales, 3 * plan.B * plan.Hh * 4)
     _check(load().bsa_quantize_e4m3(plan.handle, _ptr(q), _ptr(k), _ptr(v), _ptr(q8), _ptr(k8),
                                     _ptr(v8), _ptr(scales), _stream(stream)), "bsa_quantize_e4m3")
+
+
+def bsa_draft_mask_natural_e4m3(plan: Plan, q, k, v, sparsity_pct: int, row_ptr, kv_idx,
+                                draft_map, workspace, q8, k8, v8, scales, stream=None):
+    """bsa_draft_mask_natural and bsa_quantize_e4m3 in one call (the pooling
+    also takes the maxima of q and k)."""
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        _need(name, t, _natural(plan))
+    for name, t in (("q8", q8), ("k8", k8), ("v8", v8)):
+        _need(name, t, _natural(plan, 1))
+    _need("scales", scales, 3 * plan.B * plan.Hh * 4)
+    _need_draft_outputs(plan, sparsity_pct, row_ptr, kv_idx, draft_map)
+    nbytes = workspace.numel() * workspace.element_size()
+    _check(load().bsa_draft_mask_natural_e4m3(plan.handle, _ptr(q), _ptr(k), _ptr(v), sparsity_pct,
+                                              _ptr(row_ptr), _ptr(kv_idx), _ptr(draft_map),
+                                              _ptr(workspace), nbytes, _ptr(q8), _ptr(k8), _ptr(v8),
+                                              _ptr(scales), _stream(stream)),
+           "bsa_draft_mask_natural_e4m3")
 
 
 def bsa_attn_fwd_natural_e4m3(plan: Plan, q8, k8, v8, scales, row_ptr, col_idx,

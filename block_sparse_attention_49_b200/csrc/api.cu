@@ -243,8 +243,8 @@ bsa_status bsa_draft_mask(bsa_plan_t plan, const void* q_slots, const void* k_sl
     return set_error(BSA_ERR_UNSUPPORTED, "block list longer than 2^31 entries");
   cudaError_t e = launch_draft_mask(g, plan->d_tile_valid, q_slots, k_slots, keep,
                                     plan->draft_pooling, row_ptr, kv_idx, draft_map,
-                                    reinterpret_cast<double*>(workspace),
-                                    reinterpret_cast<cudaStream_t>(stream));
+                                    reinterpret_cast<double*>(workspace), plan->d_status,
+                                    plan->wait_limit_ns, reinterpret_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? BSA_OK : cuda_error(e, "draft_mask launch");
 }
 
@@ -333,8 +333,47 @@ bsa_status bsa_draft_mask_natural(bsa_plan_t plan, const void* q, const void* k,
     return set_error(BSA_ERR_UNSUPPORTED, "block list longer than 2^31 entries");
   cudaError_t e = launch_draft_mask(g, plan->d_tile_valid, q, k, keep, plan->draft_pooling, row_ptr,
                                     kv_idx, draft_map, reinterpret_cast<double*>(workspace),
+                                    plan->d_status, plan->wait_limit_ns,
                                     reinterpret_cast<cudaStream_t>(stream), /*natural=*/true);
   return e == cudaSuccess ? BSA_OK : cuda_error(e, "draft_mask_natural launch");
+}
+
+bsa_status bsa_draft_mask_natural_e4m3(bsa_plan_t plan, const void* q, const void* k, const void* v,
+                                       int sparsity_pct, int32_t* row_ptr, int32_t* kv_idx,
+                                       float* draft_map, void* workspace, size_t workspace_bytes,
+                                       void* q8, void* k8, void* v8, float* scales, void* stream) {
+  if (!plan) return set_error(BSA_ERR_INVALID_ARG, "plan is NULL");
+  const Geometry& g = plan->g;
+  if (g.layout != BSA_LAYOUT_TILE) return set_error(BSA_ERR_INVALID_ARG, "draft mask needs a TILE plan");
+  if (sparsity_pct < 0 || sparsity_pct >= 100)
+    return set_error(BSA_ERR_INVALID_ARG, "sparsity must be in [0, 100)");
+  bsa_status st;
+  if ((st = check_ptr(q, "q")) != BSA_OK || (st = check_ptr(k, "k")) != BSA_OK ||
+      (st = check_ptr(v, "v")) != BSA_OK || (st = check_ptr(q8, "q8")) != BSA_OK ||
+      (st = check_ptr(k8, "k8")) != BSA_OK || (st = check_ptr(v8, "v8")) != BSA_OK ||
+      (st = check_ptr(workspace, "workspace")) != BSA_OK)
+    return st;
+  if (!scales || (reinterpret_cast<uintptr_t>(scales) & 3u))
+    return set_error(BSA_ERR_ALIGNMENT, "scales is NULL or not 4-byte aligned");
+  if (!kv_idx) return set_error(BSA_ERR_INVALID_ARG, "kv_idx is NULL");
+  if (workspace_bytes < draft_workspace_bytes(g))
+    return set_error(BSA_ERR_INVALID_ARG, "workspace too small");
+  if (g.nblocks > 18000) return set_error(BSA_ERR_UNSUPPORTED, "draft mask supports up to 18000 blocks");
+  const int keep = bsa_draft_keep_count(plan, sparsity_pct);
+  if ((int64_t)g.B * g.Hh * g.nblocks * keep >= (1ll << 31))
+    return set_error(BSA_ERR_UNSUPPORTED, "block list longer than 2^31 entries");
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  // the pooling reads Q and K once for the draft map and records their
+  // per-(batch, head) maxima on the way; the quantization then takes only V's
+  cudaError_t e = cudaMemsetAsync(plan->d_amax, 0, sizeof(uint32_t) * 3 * g.B * g.Hh, s);
+  if (e != cudaSuccess) return cuda_error(e, "amax reset");
+  bool recorded = false;
+  e = launch_draft_mask(g, plan->d_tile_valid, q, k, keep, plan->draft_pooling, row_ptr, kv_idx,
+                        draft_map, reinterpret_cast<double*>(workspace), plan->d_status,
+                        plan->wait_limit_ns, s, /*natural=*/true, plan->d_amax, &recorded);
+  if (e != cudaSuccess) return cuda_error(e, "draft_mask_natural_e4m3 launch");
+  e = launch_quantize_e4m3(g, plan->d_amax, q, k, v, q8, k8, v8, scales, s, recorded);
+  return e == cudaSuccess ? BSA_OK : cuda_error(e, "quantize_e4m3 launch");
 }
 
 bsa_status bsa_quantize_e4m3(bsa_plan_t plan, const void* q, const void* k, const void* v, void* q8,

@@ -89,13 +89,15 @@ cudaError_t launch_reorder_inv(const Geometry& g, const void* x_slots, void* x_n
                                cudaStream_t st);
 cudaError_t launch_draft_mask(const Geometry& g, const uint32_t* tile_valid, const void* q,
                               const void* k, int keep, int pooling, int32_t* row_ptr,
-                              int32_t* kv_idx, float* draft_map, double* ws, cudaStream_t st,
-                              bool natural = false);
+                              int32_t* kv_idx, float* draft_map, double* ws, unsigned int* status,
+                              uint64_t wait_limit_ns, cudaStream_t st, bool natural = false,
+                              uint32_t* amax = nullptr, bool* amax_recorded = nullptr);
 
 // e4m3 quantization of natural-layout Q, K, V (scales [3][B][Hh]).
+// qk_amax_ready: amax_ws already holds the maxima of Q and K (and zero for V).
 cudaError_t launch_quantize_e4m3(const Geometry& g, uint32_t* amax_ws, const void* q, const void* k,
                                  const void* v, void* q8, void* k8, void* v8, float* scales,
-                                 cudaStream_t st);
+                                 cudaStream_t st, bool qk_amax_ready = false);
 // Natural-layout attention on e4m3 Q, K, V (TILE plan, 128-slot tiles, D = 128).
 bsa_status launch_attn_fwd_natural_e4m3(const bsa_plan_s& plan, const void* q8, const void* k8,
                                         const void* v8, const float* scales,

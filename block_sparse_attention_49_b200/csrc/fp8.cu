@@ -39,11 +39,12 @@ constexpr int kTokPerCta = 512;
 template <int D>
 __global__ void __launch_bounds__(kThreads)
     e4m3_amax_kernel(const uint4* __restrict__ q, const uint4* __restrict__ k,
-                     const uint4* __restrict__ v, int B, int Hh, int64_t N, uint32_t* amax) {
+                     const uint4* __restrict__ v, int B, int Hh, int64_t N, int which0,
+                     uint32_t* amax) {
   constexpr int kTPR = D / 8;                  // threads per token row of one head
   constexpr int kRowsPerPass = kThreads / kTPR;
   __shared__ float red[kThreads / 32];
-  const int which = blockIdx.z;
+  const int which = which0 + blockIdx.z;
   const int bh = blockIdx.y, b = bh / Hh, h = bh - b * Hh;
   const uint4* x = which == 0 ? q : (which == 1 ? k : v);
   const int64_t n0 = (int64_t)blockIdx.x * kTokPerCta;
@@ -138,19 +139,26 @@ __global__ void __launch_bounds__(kThreads)
 
 cudaError_t launch_quantize_e4m3(const Geometry& g, uint32_t* amax_ws, const void* q, const void* k,
                                  const void* v, void* q8, void* k8, void* v8, float* scales,
-                                 cudaStream_t st) {
+                                 cudaStream_t st, bool qk_amax_ready) {
   const int64_t N = (int64_t)g.T * g.P;
   const int nsc = 3 * g.B * g.Hh;
-  cudaError_t e = cudaMemsetAsync(amax_ws, 0, sizeof(uint32_t) * nsc, st);
-  if (e != cudaSuccess) return e;
-  const dim3 grid((unsigned)((N + kTokPerCta - 1) / kTokPerCta), (unsigned)(g.B * g.Hh), 3);
+  cudaError_t e = cudaSuccess;
+  // qk_amax_ready: the maxima of Q and K are already in amax_ws (recorded by
+  // the draft pooling, which read both), so only V's are taken here
+  if (!qk_amax_ready) {
+    e = cudaMemsetAsync(amax_ws, 0, sizeof(uint32_t) * nsc, st);
+    if (e != cudaSuccess) return e;
+  }
+  const int which0 = qk_amax_ready ? 2 : 0;
+  const dim3 grid((unsigned)((N + kTokPerCta - 1) / kTokPerCta), (unsigned)(g.B * g.Hh),
+                  (unsigned)(3 - which0));
   auto qq = reinterpret_cast<const uint4*>(q);
   auto kk = reinterpret_cast<const uint4*>(k);
   auto vv = reinterpret_cast<const uint4*>(v);
   if (g.D == 128)
-    e4m3_amax_kernel<128><<<grid, kThreads, 0, st>>>(qq, kk, vv, g.B, g.Hh, N, amax_ws);
+    e4m3_amax_kernel<128><<<grid, kThreads, 0, st>>>(qq, kk, vv, g.B, g.Hh, N, which0, amax_ws);
   else
-    e4m3_amax_kernel<64><<<grid, kThreads, 0, st>>>(qq, kk, vv, g.B, g.Hh, N, amax_ws);
+    e4m3_amax_kernel<64><<<grid, kThreads, 0, st>>>(qq, kk, vv, g.B, g.Hh, N, which0, amax_ws);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   e4m3_scales_kernel<<<(nsc + 255) / 256, 256, 0, st>>>(amax_ws, nsc, scales);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;

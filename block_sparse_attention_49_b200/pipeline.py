@@ -18,6 +18,7 @@ import torch
 from . import (ANCHORS_ROTATING, LAYOUT_FRAME, LAYOUT_TILE, POOL_MEAN, WINDOW_ALTERNATE, Plan,
                bsa_attn_fwd, bsa_attn_fwd_natural, bsa_attn_fwd_natural_e4m3,
                bsa_draft_keep_count, bsa_draft_mask, bsa_draft_mask_natural,
+               bsa_draft_mask_natural_e4m3,
                bsa_draft_workspace_bytes, bsa_quantize_e4m3,
                bsa_lvsa_attn_fwd, bsa_lvsa_mask, bsa_lvsa_nnz, bsa_plan_set_draft_pooling,
                bsa_plan_set_lvsa_variant, bsa_reorder_fwd, bsa_reorder_inv)
@@ -119,22 +120,31 @@ class DraftAttention(_Base):
                              out, lse)
         return out
 
-    def quantize(self, q, k, v):
-        """e4m3 copies of q, k, v and their per-(tensor, batch, head) scales."""
+    def _e4m3_buffers(self, q):
         if getattr(self, "q8", None) is None or self.q8.shape != q.shape:
             self.q8, self.k8, self.v8 = (torch.empty(q.shape, dtype=torch.uint8, device=q.device)
                                          for _ in range(3))
             p = self.plan
             self.fp8_scales = torch.empty((3, p.B, p.Hh), dtype=torch.float32, device=q.device)
+
+    def quantize(self, q, k, v):
+        """e4m3 copies of q, k, v and their per-(tensor, batch, head) scales."""
+        self._e4m3_buffers(q)
         bsa_quantize_e4m3(self.plan, q, k, v, self.q8, self.k8, self.v8, self.fp8_scales)
+
+    def mask_and_quantize(self, q, k, v):
+        """The draft mask from the bf16 Q and K and the e4m3 copies of Q, K, V
+        in one call (the pooling also takes the maxima of Q and K)."""
+        self._e4m3_buffers(q)
+        bsa_draft_mask_natural_e4m3(self.plan, q, k, v, self.sparsity, self.row_ptr, self.col_idx,
+                                    self.draft_map, self.workspace, self.q8, self.k8, self.v8,
+                                    self.fp8_scales)
 
     def fused_e4m3(self, q, k, v, out=None, lse=None):
         """fused() with 8-bit attention: the draft mask from the bf16 Q and K,
-        then Q, K, V quantized to e4m3 and attended with 8-bit MMAs."""
+        Q, K, V quantized to e4m3, then attended with 8-bit MMAs."""
         out = torch.empty_like(q) if out is None else out
-        bsa_draft_mask_natural(self.plan, q, k, self.sparsity, self.row_ptr, self.col_idx,
-                               self.draft_map, self.workspace)
-        self.quantize(q, k, v)
+        self.mask_and_quantize(q, k, v)
         bsa_attn_fwd_natural_e4m3(self.plan, self.q8, self.k8, self.v8, self.fp8_scales,
                                   self.row_ptr, self.col_idx, True, self.scale, out, lse)
         return out

@@ -127,8 +127,9 @@ int     bsa_block_size(bsa_plan_t plan);
 /* LVSA frame mask for denoising step s ("LVSA", section 2, "Rotating global
  * anchors" and "Extended adaptive window").
  *   G_s = {f in [0,T) : (f - s) mod T_per == 0};
- *   A(t) = G_s U {t} grown by t+1, t-1, t+2, t-2, ... (frames outside [0,T)
- *   or already present are skipped) until |A(t)| = C.
+ *   A(t) = G_s U {t}, then grown until |A(t)| = C by a right and a left
+ *   pointer taking turns, right first, each skipping frames already present;
+ *   a side that runs off [0,T) stops and the other continues.
  * (Other anchor grids and growth orders: bsa_plan_set_lvsa_variant.)
  * Requires a FRAME plan, 1 <= T_per, C <= T and |G_s U {t}| <= C for every t.
  * Outputs (device):
@@ -186,7 +187,10 @@ bsa_status bsa_draft_mask(bsa_plan_t plan, const void* q_slots, const void* k_sl
  * make that first call before any stream capture.  All calls on a device
  * share the array: calls whose kernels overlap on the GPU race on it, calls
  * in order on one stream do not.  Nothing in it needs clearing between calls.
- * The current device must be the plan's device. */
+ * The current device must be the plan's device (BSA_ERR_INVALID_ARG
+ * otherwise).  The address is cached for the life of the process: after
+ * cudaDeviceReset on a device, do not call this entry point again in that
+ * process. */
 bsa_status bsa_draft_mask_noalloc(bsa_plan_t plan, const void* q_slots, const void* k_slots,
                                   int sparsity_pct, int32_t* row_ptr, int32_t* kv_idx,
                                   float* draft_map, void* stream);
@@ -256,6 +260,17 @@ bsa_status bsa_draft_mask_natural(bsa_plan_t plan, const void* q, const void* k,
 bsa_status bsa_quantize_e4m3(bsa_plan_t plan, const void* q, const void* k, const void* v, void* q8,
                              void* k8, void* v8, float* scales, void* stream);
 
+/* The front half of the 8-bit draft pipeline in one call: the draft mask of
+ * bsa_draft_mask_natural and the quantization of bsa_quantize_e4m3, with the
+ * same outputs bit for bit (arguments as there).  The pooling pass that
+ * reads Q and K for the draft map also takes their per-head maxima, so the
+ * quantization reads only V once more before converting all three tensors.
+ * Uses the plan's buffer as bsa_quantize_e4m3 does. */
+bsa_status bsa_draft_mask_natural_e4m3(bsa_plan_t plan, const void* q, const void* k, const void* v,
+                                       int sparsity_pct, int32_t* row_ptr, int32_t* kv_idx,
+                                       float* draft_map, void* workspace, size_t workspace_bytes,
+                                       void* q8, void* k8, void* v8, float* scales, void* stream);
+
 /* bsa_attn_fwd_natural on e4m3 inputs (from bsa_quantize_e4m3): the QK and
  * PV products are 8-bit tensor-core MMAs (kind::f8f6f4) with fp32
  * accumulation; the scores are S * sq * sk; P is rounded to e4m3 (it stays
@@ -286,7 +301,12 @@ bsa_status bsa_lvsa_attn_fwd(bsa_plan_t plan, int C, int T_per, int s, const voi
                              void* stream);
 
 /* Synchronize `stream`, read and clear the plan's device status word.
- * Returns BSA_OK, BSA_ERR_BAD_BLOCKLIST, BSA_ERR_TIMEOUT or BSA_ERR_CUDA. */
+ * Returns BSA_OK, BSA_ERR_BAD_BLOCKLIST, BSA_ERR_TIMEOUT or BSA_ERR_CUDA.
+ * A recorded timeout is sticky: until this call clears it, every later
+ * kernel of the plan sees it at start and returns at once without writing
+ * its outputs (so a plan whose wait ran out stops working instead of
+ * waiting again).  Callers that do not poll after each step get stale
+ * outputs in that state; poll at least once per step to detect it. */
 bsa_status bsa_poll_status(bsa_plan_t plan, void* stream);
 
 /* Set the limit, in nanoseconds, of every bounded wait inside the plan's

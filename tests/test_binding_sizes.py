@@ -23,7 +23,8 @@ def _lib():
 
 # FRAME-like geometry: 3 frames of 5 x 7 tokens, 32-token blocks -> 2 blocks
 # per frame, 6 blocks, 256 slots
-P = types.SimpleNamespace(B=2, Hh=3, D=64, T=3, H=5, W=7, Npad=256, nblocks=6, handle=None)
+P = types.SimpleNamespace(B=2, Hh=3, D=64, T=3, H=5, W=7, Npad=256, nblocks=6, handle=None,
+                         keep_count=lambda sp: -(-6 * (100 - sp) // 100))
 N = P.T * P.H * P.W
 NAT = (P.B, N, P.Hh, P.D)
 SLOT = (P.B, P.Hh, P.Npad, P.D)

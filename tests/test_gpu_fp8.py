@@ -4,6 +4,9 @@ scale per (tensor, batch, head), P rounded to e4m3 on the way into the PV
 product, fp32 accumulation).
 
 * bsa_quantize_e4m3: codes and scales bit-exact against the oracle.
+* bsa_draft_mask_natural_e4m3 (the draft mask and the quantization in one
+  call, the maxima of Q and K taken by the pooling): every output identical,
+  bit for bit, to the two separate calls.
 * bsa_attn_fwd_natural_e4m3: against the fp64 oracle run on the dequantized
   inputs.  What is left is mostly the e4m3 rounding of P: a relative error
   of at most 2^-4 per weight, of either sign, so it largely cancels in the
@@ -63,6 +66,47 @@ def test_quantize_e4m3_bit_exact(over):
         s_ref = oracle.fp8_scales(xn)
         np.testing.assert_array_equal(scales[i].cpu().numpy(), s_ref)
         np.testing.assert_array_equal(_codes_to_values(x8), oracle.fp8_quantize(xn, s_ref))
+
+
+@pytest.mark.parametrize("over", [dict(cid=5, Hh=4),
+                                  dict(cid=2, T=3, H=13, W=37, Hh=3, field_grid=(3, 4, 7)),
+                                  dict(cid=1, qk="iid", D=64),
+                                  # 16 x 32 tiles (512 tokens): pooled without TMA, so the
+                                  # maxima of Q and K come from the separate pass
+                                  dict(cid=2, T=2, H=32, W=64, Hh=2, draft_ph=16, draft_pw=32,
+                                       field_grid=(2, 4, 7))])
+@pytest.mark.parametrize("pooling", [bsa.POOL_MEAN, bsa.POOL_MAX])
+def test_draft_mask_and_quantize_in_one_call_equal_the_two_calls(over, pooling):
+    over = dict(over)
+    w = small_workload(CONFIGS[over.pop("cid")], **over)
+    q, k, v = make_qkv(w, device="cuda")
+    v = v * 3.0
+    ph, pw, sp = w.draft_ph, w.draft_pw, w.draft_sparsity
+    plan = bsa.Plan(w.B, w.Hh, w.D, w.T, w.H, w.W, bsa.LAYOUT_TILE, ph, pw, ph * pw)
+    bsa.bsa_plan_set_draft_pooling(plan, pooling)
+    keep = bsa.bsa_draft_keep_count(plan, sp)
+    rows = w.B * w.Hh * plan.nblocks
+
+    def outputs():
+        rp = torch.full((rows + 1,), -1, dtype=torch.int32, device="cuda")
+        kv = torch.full((rows * keep,), -1, dtype=torch.int32, device="cuda")
+        dm = torch.full((rows * plan.nblocks,), float("nan"), dtype=torch.float32, device="cuda")
+        ws = torch.empty(((bsa.bsa_draft_workspace_bytes(plan) + 7) // 8,), dtype=torch.float64,
+                         device="cuda")
+        x8 = [torch.full(x.shape, 0x7f, dtype=torch.uint8, device="cuda") for x in (q, k, v)]
+        sc = torch.full((3, w.B, w.Hh), float("nan"), dtype=torch.float32, device="cuda")
+        return rp, kv, dm, ws, x8, sc
+
+    rp, kv, dm, ws, x8, sc = outputs()
+    bsa.bsa_draft_mask_natural(plan, q, k, sp, rp, kv, dm, ws)
+    bsa.bsa_quantize_e4m3(plan, q, k, v, *x8, sc)
+    rp1, kv1, dm1, ws1, y8, sc1 = outputs()
+    bsa.bsa_draft_mask_natural_e4m3(plan, q, k, v, sp, rp1, kv1, dm1, ws1, *y8, sc1)
+    bsa.bsa_poll_status(plan)
+    assert torch.equal(rp, rp1) and torch.equal(kv, kv1) and torch.equal(dm, dm1)
+    assert torch.equal(sc, sc1)
+    for a, b in zip(x8, y8):
+        assert torch.equal(a, b)
 
 
 def _e4m3_case(w, q_blocks=None, heads=None):

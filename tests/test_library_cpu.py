@@ -77,6 +77,8 @@ def test_null_plan_is_rejected(lib):
     assert lib.bsa_draft_mask_natural(None, None, None, 90, None, None, None, None, 0, None) == 1
     assert lib.bsa_draft_mask_noalloc(None, None, None, 90, None, None, None, None) == 1
     assert lib.bsa_quantize_e4m3(None, None, None, None, None, None, None, None, None) == 1
+    assert lib.bsa_draft_mask_natural_e4m3(None, None, None, None, 90, None, None, None, None, 0,
+                                           None, None, None, None, None) == 1
     assert lib.bsa_attn_fwd_natural_e4m3(None, None, None, None, None, None, None, 1, 1.0, None,
                                          None, None) == 1
     assert lib.bsa_reorder_fwd(None, None, None, None, None, None, None, None) == 1
