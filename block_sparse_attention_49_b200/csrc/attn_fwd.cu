@@ -41,7 +41,9 @@
 #include <cuda_bf16.h>
 #include <cudaTypedefs.h>
 
+#include <algorithm>
 #include <cmath>
+#include <cstring>
 
 #include "bsa_internal.cuh"
 #include "ptx.cuh"
@@ -52,9 +54,11 @@ namespace {
 constexpr int kTile = 128;          // query / key tile (slots)
 constexpr int kThreads = 384;
 constexpr int kFineMaxTiles = 2048; // key tiles addressable by the sub-tile-block path
+constexpr int kPackMax = 768;       // key-list entries a CTA can pack (longer lists run unpacked)
+constexpr uint16_t kPackBad = 0xffffu;  // packed-list marker of an out-of-range entry
 constexpr uint32_t kFull = 0xffffffffu;
 
-template <int D, bool FINE, bool F8 = false>
+template <int D, bool FINE, bool F8 = false, bool PACK = false>
 struct AttnCfg {
   static constexpr int kElem = F8 ? 1 : 2;           // bytes per element
   static constexpr int kChunkElems = 128 / kElem;    // elements per 128-byte swizzle row
@@ -71,7 +75,9 @@ struct AttnCfg {
   static constexpr int kNumBars = 1 + 3 * NS + 2 + 2 + 1;
   static constexpr int kOffMisc = kOffBar + kNumBars * 8;
   static constexpr int kOffList = kOffMisc + 16;
-  static constexpr int kOffBitmap = kOffList + (FINE ? kFineMaxTiles * 2 : 0);
+  // FINE: the union of key tiles (uint16); PACK: the key list sorted by tile
+  // kind (uint16) followed by four counts
+  static constexpr int kOffBitmap = kOffList + (FINE ? kFineMaxTiles * 2 : PACK ? kPackMax * 2 + 16 : 0);
   static constexpr int kBytes = kOffBitmap + (FINE ? kFineMaxTiles / 8 : 0);
   static constexpr int kSmem = kBytes + 1024;  // room to align the base to 1024
   static constexpr uint32_t kTmemCols = 512;   // S_A | S_B | O_A | O_B
@@ -99,7 +105,40 @@ struct AttnParams {
   int B, T, H, W, N, TW, ph, pw;
   const float* fp8_scales;  // F8: [3][B][Hh] scales of Q, K, V
   FastDiv div_tile_frame, div_TW, div_pw;  // by TH*TW, TW, pw
+  // edge-tile packing (PACK): the partial tiles at the grid's right edge
+  // (kind 1), bottom edge (2) and corner (3), in decreasing size
+  int TH;
+  int pk_on;       // some edge kind exists and block indices fit 15 bits
+  int pk_kind[3];  // kind of each slot (0: absent)
+  int pk_rows[3];  // token rows of a tile of that kind
+  int pk_step[3];  // the same rounded up to 8 (row offset step inside a packed tile)
 };
+
+// Tensor maps of the edge kinds (boxes of their exact size), indexed kind - 1.
+struct EdgeMaps {
+  CUtensorMap k[3], v[3];
+};
+
+// Set bits [lo, hi) of a 128-bit mask (0 <= lo <= hi <= 128).
+__device__ __forceinline__ void set_rows(uint32_t (&m)[4], int lo, int hi) {
+#pragma unroll
+  for (int w = 0; w < 4; ++w) {
+    const int a = max(lo, 32 * w), e = min(hi, 32 * w + 32);
+    if (e > a) m[w] |= (e - a == 32 ? kFull : ((1u << (e - a)) - 1u)) << (a - 32 * w);
+  }
+}
+
+// Composition of the next packed tile of edge pieces: take as many pieces of
+// each kind as fit in 128 rows, largest kind first; r[] = pieces left.
+__device__ __forceinline__ void next_bin(const AttnParams& p, int (&r)[3], int (&a)[3]) {
+  int cap = kTile;
+#pragma unroll
+  for (int e = 0; e < 3; ++e) {
+    a[e] = p.pk_step[e] > 0 ? min(r[e], cap / p.pk_step[e]) : 0;
+    cap -= a[e] * p.pk_step[e];
+    r[e] -= a[e];
+  }
+}
 
 // Set bits [lo, lo+len) of a 128-bit mask; lo is a multiple of len, len | 128.
 __device__ __forceinline__ void set_bits(uint32_t (&m)[4], int lo, int len) {
@@ -132,11 +171,13 @@ __device__ __forceinline__ void cta_end_sync() {
   asm volatile("bar.sync 2, 384;" ::: "memory");
 }
 
-template <int D, bool FINE, bool NAT, bool F8 = false>
+template <int D, bool FINE, bool NAT, bool F8 = false, bool PACK = false>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmk,
-                    const __grid_constant__ CUtensorMap tmv, const AttnParams p) {
-  using Cfg = AttnCfg<D, FINE, F8>;
+                    const __grid_constant__ CUtensorMap tmv, const AttnParams p,
+                    const __grid_constant__ EdgeMaps em) {
+  using Cfg = AttnCfg<D, FINE, F8, PACK>;
+  static_assert(!PACK || (NAT && !FINE), "edge packing: natural-layout tiles");
   static_assert(!F8 || (NAT && D == 128), "the e4m3 path reads the natural layout, D = 128");
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -254,10 +295,102 @@ __global__ void __launch_bounds__(kThreads, 1)
     n = (int)misc[2];
   }
 
+  // ------------------------------------------- edge packing: sort the list by kind
+  // Full tiles first (list order), then the edge pieces grouped by kind in
+  // decreasing size; every role replays the same packing of those pieces
+  // (next_bin), so no per-tile schedule is stored.
+  uint16_t* plist = tlist;
+  int* pcnt = reinterpret_cast<int*>(smem + Cfg::kOffList + kPackMax * 2);  // nF, c0, c1, c2
+  bool packed = false;
+  int nF = 0, pc[3] = {0, 0, 0};
+  if constexpr (PACK) {
+    packed = p.pk_on && n > 0 && n <= kPackMax;
+    if (packed) {
+      if (warp == 2) {
+        const int TT = (int)p.div_tile_frame.d;
+        auto kind_of = [&](int c) {
+          const int rr = c % TT, i = rr / p.TW, jj = rr - i * p.TW;
+          const int right = (jj == p.TW - 1 && p.W - jj * p.pw < p.pw) ? 1 : 0;
+          const int bottom = (i == p.TH - 1 && p.H - i * p.ph < p.ph) ? 2 : 0;
+          return right | bottom;
+        };
+        int cF = 0, ce[3] = {0, 0, 0};
+        for (int base = 0; base < n; base += 32) {
+          const int i = base + lane;
+          int kind = -1;
+          if (i < n) {
+            const int c = __ldg(p.col_idx + rs + i);
+            kind = (c >= 0 && (int64_t)c < p.nblocks) ? kind_of(c) : 0;
+          }
+          cF += __popc(__ballot_sync(kFull, kind == 0));
+#pragma unroll
+          for (int e = 0; e < 3; ++e)
+            ce[e] += __popc(__ballot_sync(kFull, kind > 0 && kind == p.pk_kind[e]));
+        }
+        int wF = 0, we[3] = {0, 0, 0};
+        const int start[3] = {cF, cF + ce[0], cF + ce[0] + ce[1]};
+        const uint32_t lt = (1u << lane) - 1u;
+        bool bad = false;
+        for (int base = 0; base < n; base += 32) {
+          const int i = base + lane;
+          int kind = -1;
+          uint16_t val = 0;
+          if (i < n) {
+            const int c = __ldg(p.col_idx + rs + i);
+            const bool ok = c >= 0 && (int64_t)c < p.nblocks;
+            bad |= !ok;
+            kind = ok ? kind_of(c) : 0;
+            val = ok ? (uint16_t)c : kPackBad;
+          }
+          const uint32_t bF = __ballot_sync(kFull, kind == 0);
+          int pos = kind == 0 ? wF + __popc(bF & lt) : 0;
+          wF += __popc(bF);
+#pragma unroll
+          for (int e = 0; e < 3; ++e) {
+            const uint32_t be = __ballot_sync(kFull, kind > 0 && kind == p.pk_kind[e]);
+            if (kind > 0 && kind == p.pk_kind[e]) pos = start[e] + we[e] + __popc(be & lt);
+            we[e] += __popc(be);
+          }
+          if (i < n) plist[pos] = val;
+        }
+        if (__any_sync(kFull, bad) && lane == 0) atomicOr(p.status, kStatusBadBlocklist);
+        if (lane == 0) {
+          pcnt[0] = cF;
+          pcnt[1] = ce[0];
+          pcnt[2] = ce[1];
+          pcnt[3] = ce[2];
+        }
+      }
+      // stale rows of a packed tile are masked, but P = 0 times a value must
+      // stay 0: start every V stage at zero (finite)
+      for (int i = threadIdx.x; i < Cfg::NS * Cfg::kKVBytes / 16; i += kThreads)
+        reinterpret_cast<uint4*>(smem + Cfg::kOffV)[i] = make_uint4(0u, 0u, 0u, 0u);
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+      __syncthreads();
+      nF = pcnt[0];
+      pc[0] = pcnt[1];
+      pc[1] = pcnt[2];
+      pc[2] = pcnt[3];
+      // packed tiles: the full ones plus the bins of edge pieces
+      int r[3] = {pc[0], pc[1], pc[2]}, a[3];
+      int nb = 0;
+      while (r[0] + r[1] + r[2] > 0) {
+        next_bin(p, r, a);
+        ++nb;
+      }
+      n = nF + nb;
+    }
+  }
+
   auto tile_of = [&](int j, bool& ok) -> int {
     if (FINE) {
       ok = true;
       return tlist[j];
+    }
+    if (PACK && packed) {  // a full tile of the sorted list (j < nF)
+      const uint16_t c = plist[j];
+      ok = c != kPackBad;
+      return ok ? c : 0;
     }
     const int c = __ldg(p.col_idx + rs + j);
     ok = (c >= 0 && (int64_t)c < p.nblocks);
@@ -285,15 +418,61 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       __syncwarp();
       int issued = 0;
+      // packed bins: pieces left per kind, their region starts and cursors
+      int prem[3] = {pc[0], pc[1], pc[2]};
+      const int pstart[3] = {nF, nF + pc[0], nF + pc[0] + pc[1]};
+      int pptr[3] = {0, 0, 0};
+      (void)prem;
+      (void)pstart;
+      (void)pptr;
       for (int j = 0; j < n; ++j) {
         const int st = j % Cfg::NS;
         const uint32_t ph = (j / Cfg::NS) & 1;
         if (!__all_sync(kFull, bounded_wait(&kv_empty[st], ph ^ 1, wc))) break;
+        if constexpr (PACK) {
+          if (packed && j >= nF) {
+            // a bin of edge pieces: each piece's exact box at 8-row offsets
+            int a[3];
+            next_bin(p, prem, a);
+            if (elect_one()) {
+              uint8_t* sK = smem + Cfg::kOffK + st * Cfg::kKVBytes;
+              uint8_t* sV = smem + Cfg::kOffV + st * Cfg::kKVBytes;
+              uint32_t bytes = 0;
+#pragma unroll
+              for (int e = 0; e < 3; ++e) bytes += a[e] * p.pk_rows[e] * 128 * Cfg::kChunks;
+              mbar_arrive_expect_tx(&k_full[st], bytes);
+              mbar_arrive_expect_tx(&v_full[st], bytes);
+              int off = 0;
+#pragma unroll
+              for (int e = 0; e < 3; ++e) {
+                for (int m = 0; m < a[e]; ++m) {
+                  const int kt = plist[pstart[e] + pptr[e] + m];
+                  int x0, y0, fr;
+                  nat_coords(kt, x0, y0, fr);
+                  const CUtensorMap* mk = &em.k[p.pk_kind[e] - 1];
+                  const CUtensorMap* mv = &em.v[p.pk_kind[e] - 1];
+                  for (int c = 0; c < Cfg::kChunks; ++c) {
+                    tma_load_5d(sK + c * Cfg::kPanel + off * 128, mk, &k_full[st],
+                                c * Cfg::kChunkElems, h, x0, y0, fr);
+                    tma_load_5d(sV + c * Cfg::kPanel + off * 128, mv, &v_full[st],
+                                c * Cfg::kChunkElems, h, x0, y0, fr);
+                  }
+                  off += p.pk_step[e];
+                }
+              }
+            }
+#pragma unroll
+            for (int e = 0; e < 3; ++e) pptr[e] += a[e];
+            __syncwarp();
+            issued = j + 1;
+            continue;
+          }
+        }
         bool ok;
         const int kt = tile_of(j, ok);
         const int krow = (int)(bh_row + (int64_t)kt * kTile);
         if (elect_one()) {
-          if (!ok) atomicOr(p.status, kStatusBadBlocklist);
+          if (!ok && !PACK) atomicOr(p.status, kStatusBadBlocklist);
           uint8_t* sK = smem + Cfg::kOffK + st * Cfg::kKVBytes;
           uint8_t* sV = smem + Cfg::kOffV + st * Cfg::kKVBytes;
           if constexpr (NAT) {
@@ -438,11 +617,31 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
     bool alive = true;
+    int srem[3] = {pc[0], pc[1], pc[2]};  // packed bins: pieces left per kind
+    int scur = nF;                        // next bin index to replay
+    (void)srem;
+    (void)scur;
     for (int j = g; j < n; j += 2) {
-      bool ok;
-      const int kt = tile_of(j, ok);
-      uint32_t vm[4];
-      {
+      uint32_t vm[4] = {0u, 0u, 0u, 0u};
+      if (PACK && packed && j >= nF) {
+        // rows of this bin's pieces: [off, off + rows) of each
+        int a[3];
+        while (scur < j) {
+          next_bin(p, srem, a);
+          ++scur;
+        }
+        next_bin(p, srem, a);
+        ++scur;
+        int off = 0;
+#pragma unroll
+        for (int e = 0; e < 3; ++e)
+          for (int m = 0; m < a[e]; ++m) {
+            set_rows(vm, off, off + p.pk_rows[e]);
+            off += p.pk_step[e];
+          }
+      } else {
+        bool ok;
+        const int kt = tile_of(j, ok);
         const uint4 tv = __ldg(reinterpret_cast<const uint4*>(p.tile_valid) + kt);
         vm[0] = ok ? tv.x : 0u;
         vm[1] = ok ? tv.y : 0u;
@@ -450,6 +649,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         vm[3] = ok ? tv.w : 0u;
       }
       if (FINE) {
+        bool ok;
+        const int kt = tile_of(j, ok);
         // this row's allowed blocks inside key tile kt (entries of tiles
         // handled by the other group are passed over)
         uint32_t am[4] = {0u, 0u, 0u, 0u};
@@ -646,14 +847,17 @@ bool make_tmap(CUtensorMap* m, const void* ptr, int64_t rows, int D) {
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int D, bool FINE, bool NAT = false, bool F8 = false>
+template <int D, bool FINE, bool NAT = false, bool F8 = false, bool PACK = false>
 cudaError_t launch_t(const CUtensorMap& q, const CUtensorMap& k, const CUtensorMap& v,
-                     const AttnParams& p, dim3 grid, cudaStream_t st) {
-  using Cfg = AttnCfg<D, FINE, F8>;
-  auto kern = attn_fwd_kernel<D, FINE, NAT, F8>;
+                     const AttnParams& p, dim3 grid, cudaStream_t st,
+                     const EdgeMaps* em = nullptr) {
+  using Cfg = AttnCfg<D, FINE, F8, PACK>;
+  auto kern = attn_fwd_kernel<D, FINE, NAT, F8, PACK>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::kSmem);
   if (e != cudaSuccess) return e;
-  kern<<<grid, kThreads, Cfg::kSmem, st>>>(q, k, v, p);
+  EdgeMaps none;
+  memset(&none, 0, sizeof(none));
+  kern<<<grid, kThreads, Cfg::kSmem, st>>>(q, k, v, p, em ? *em : none);
   return cudaGetLastError();
 }
 
@@ -693,13 +897,44 @@ AttnParams make_params(const bsa_plan_s& plan, const int32_t* row_ptr, const int
   p.div_tile_frame = FastDiv((uint32_t)(TH * p.TW));
   p.div_TW = FastDiv((uint32_t)p.TW);
   p.div_pw = FastDiv((uint32_t)p.pw);
+  p.TH = TH;
+  p.pk_on = 0;
+  for (int e = 0; e < 3; ++e) p.pk_kind[e] = p.pk_rows[e] = p.pk_step[e] = 0;
   return p;
+}
+
+// Edge kinds of a TILE plan's grid: right (kind 1, the last tile column when
+// pool_w does not divide W), bottom (2) and corner (3), sorted by size
+// (rows), largest first; their box width and height.
+int edge_kinds(const Geometry& g, int kind[3], int rows[3], int bw[3], int bh[3]) {
+  const int wR = g.W - (g.TW - 1) * g.pw, hB = g.H - (g.TH - 1) * g.ph;
+  int n = 0;
+  auto add = [&](int k, int w, int h) {
+    kind[n] = k;
+    rows[n] = w * h;
+    bw[n] = w;
+    bh[n] = h;
+    ++n;
+  };
+  if (wR < g.pw) add(1, wR, g.ph);
+  if (hB < g.ph) add(2, g.pw, hB);
+  if (wR < g.pw && hB < g.ph) add(3, wR, hB);
+  for (int a = 0; a < n; ++a)  // by rows descending, then kind
+    for (int b = a + 1; b < n; ++b)
+      if (rows[b] > rows[a] || (rows[b] == rows[a] && kind[b] < kind[a])) {
+        std::swap(kind[a], kind[b]);
+        std::swap(rows[a], rows[b]);
+        std::swap(bw[a], bw[b]);
+        std::swap(bh[a], bh[b]);
+      }
+  return n;
 }
 
 // Natural layout [B, N, Hh, D] bf16 seen as 5-D {D, Hh, W, H, B*T}; boxes of
 // 64 channels x 1 head x pw x ph x 1 frame (one pooling tile, 128 rows of
 // 128 bytes), 128-byte swizzle.  Boxes reaching past W or H read zeros.
-bool make_tmap_tiles(CUtensorMap* m, const void* ptr, const Geometry& g, bool e4m3 = false) {
+bool make_tmap_tiles(CUtensorMap* m, const void* ptr, const Geometry& g, bool e4m3 = false,
+                     int box_w = 0, int box_h = 0) {
   auto fn = encode_fn();
   if (!fn) return false;
   const cuuint64_t esz = e4m3 ? 1 : 2;
@@ -707,7 +942,8 @@ bool make_tmap_tiles(CUtensorMap* m, const void* ptr, const Geometry& g, bool e4
   cuuint64_t dims[5] = {(cuuint64_t)g.D, (cuuint64_t)g.Hh, (cuuint64_t)g.W, (cuuint64_t)g.H,
                         (cuuint64_t)g.B * g.T};
   cuuint64_t strides[4] = {(cuuint64_t)g.D * esz, row, row * g.W, row * g.W * g.H};
-  cuuint32_t box[5] = {(cuuint32_t)(128 / esz), 1, (cuuint32_t)g.pw, (cuuint32_t)g.ph, 1};
+  cuuint32_t box[5] = {(cuuint32_t)(128 / esz), 1, (cuuint32_t)(box_w > 0 ? box_w : g.pw),
+                       (cuuint32_t)(box_h > 0 ? box_h : g.ph), 1};
   cuuint32_t estr[5] = {1, 1, 1, 1, 1};
   return fn(m, e4m3 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5,
             const_cast<void*>(ptr), dims, strides, box,
@@ -754,10 +990,31 @@ bsa_status launch_attn_fwd_natural(const bsa_plan_s& plan, const void* q, const 
   CUtensorMap tq, tk, tv;
   if (!make_tmap_tiles(&tq, q, g) || !make_tmap_tiles(&tk, k, g) || !make_tmap_tiles(&tv, v, g))
     return set_error(BSA_ERR_CUDA, "cuTensorMapEncodeTiled (5-D) failed");
-  const AttnParams p = make_params(plan, row_ptr, col_idx, per_head, scale, o, lse);
+  AttnParams p = make_params(plan, row_ptr, col_idx, per_head, scale, o, lse);
   const dim3 grid((unsigned)g.ntiles, (unsigned)g.Hh, (unsigned)g.B);
-  const cudaError_t e = g.D == 128 ? launch_t<128, false, true>(tq, tk, tv, p, grid, st)
-                                   : launch_t<64, false, true>(tq, tk, tv, p, grid, st);
+  // partial key tiles at the grid's edges are packed several to an MMA tile,
+  // each read with a box of its exact size
+  int kind[3] = {0, 0, 0}, rows[3] = {0, 0, 0}, bw[3] = {0, 0, 0}, bh[3] = {0, 0, 0};
+  const int nk = edge_kinds(g, kind, rows, bw, bh);
+  cudaError_t e;
+  if (nk > 0 && g.nblocks < 32768) {
+    EdgeMaps em;
+    memset(&em, 0, sizeof(em));
+    for (int i = 0; i < nk; ++i) {
+      p.pk_kind[i] = kind[i];
+      p.pk_rows[i] = rows[i];
+      p.pk_step[i] = (rows[i] + 7) / 8 * 8;
+      if (!make_tmap_tiles(&em.k[kind[i] - 1], k, g, false, bw[i], bh[i]) ||
+          !make_tmap_tiles(&em.v[kind[i] - 1], v, g, false, bw[i], bh[i]))
+        return set_error(BSA_ERR_CUDA, "cuTensorMapEncodeTiled (5-D edge boxes) failed");
+    }
+    p.pk_on = 1;
+    e = g.D == 128 ? launch_t<128, false, true, false, true>(tq, tk, tv, p, grid, st, &em)
+                   : launch_t<64, false, true, false, true>(tq, tk, tv, p, grid, st, &em);
+  } else {
+    e = g.D == 128 ? launch_t<128, false, true>(tq, tk, tv, p, grid, st)
+                   : launch_t<64, false, true>(tq, tk, tv, p, grid, st);
+  }
   if (e != cudaSuccess) return cuda_error(e, "natural-layout attention launch");
   return BSA_OK;
 }
@@ -781,7 +1038,25 @@ bsa_status launch_attn_fwd_natural_e4m3(const bsa_plan_s& plan, const void* q8, 
   AttnParams p = make_params(plan, row_ptr, col_idx, per_head, scale, o, lse);
   p.fp8_scales = scales;
   const dim3 grid((unsigned)g.ntiles, (unsigned)g.Hh, (unsigned)g.B);
-  const cudaError_t e = launch_t<128, false, true, true>(tq, tk, tv, p, grid, st);
+  int kind[3] = {0, 0, 0}, rows[3] = {0, 0, 0}, bw[3] = {0, 0, 0}, bh[3] = {0, 0, 0};
+  const int nk = edge_kinds(g, kind, rows, bw, bh);
+  cudaError_t e;
+  if (nk > 0 && g.nblocks < 32768) {
+    EdgeMaps em;
+    memset(&em, 0, sizeof(em));
+    for (int i = 0; i < nk; ++i) {
+      p.pk_kind[i] = kind[i];
+      p.pk_rows[i] = rows[i];
+      p.pk_step[i] = (rows[i] + 7) / 8 * 8;
+      if (!make_tmap_tiles(&em.k[kind[i] - 1], k8, g, true, bw[i], bh[i]) ||
+          !make_tmap_tiles(&em.v[kind[i] - 1], v8, g, true, bw[i], bh[i]))
+        return set_error(BSA_ERR_CUDA, "cuTensorMapEncodeTiled (5-D e4m3 edge boxes) failed");
+    }
+    p.pk_on = 1;
+    e = launch_t<128, false, true, true, true>(tq, tk, tv, p, grid, st, &em);
+  } else {
+    e = launch_t<128, false, true, true>(tq, tk, tv, p, grid, st);
+  }
   if (e != cudaSuccess) return cuda_error(e, "e4m3 attention launch");
   return BSA_OK;
 }

@@ -4,10 +4,11 @@ and bsa_attn_fwd_natural.
 Draft Attention article: pooled Q and K give the draft map and the kept
 blocks; the reorder that makes the kept blocks contiguous is fused into the
 attention's tile loads and stores here.  Pooled values and kept blocks:
-bit-exact against the oracle.  Attention: identical, bit for bit, to the
-reorder + attn_fwd + reorder_inv path on every token (the kernels do the
-same arithmetic on the same tiles), and within max-abs 2e-2 / mean-abs 2e-3
-of the fp64 oracle.
+bit-exact against the oracle.  Attention: within max-abs 2e-2 / mean-abs
+2e-3 of the fp64 oracle (LSE within 2e-3), on grids whose edges leave
+partial tiles (the kernel packs those key tiles several to an MMA tile) and
+on lists too long to pack; on a grid with no partial tiles it is identical,
+bit for bit, to the reorder + attn_fwd + reorder_inv path.
 """
 import math
 
@@ -71,24 +72,89 @@ def test_draft_mask_natural_bit_exact(over, pooling):
     np.testing.assert_array_equal(kv.cpu().numpy().reshape(w.B, w.Hh, nb, keep), ref)
 
 
+def _oracle_natural(w, q, k, v, kv_gpu, heads, q_blocks=None):
+    """fp64 oracle attention on the natural layout for the given heads (and
+    query blocks), with the kept blocks the GPU chose (checked separately)."""
+    ph, pw = w.draft_ph, w.draft_pw
+    perm, Np = oracle.tile_layout_perm(w.T, w.H, w.W, ph, pw)
+    valid = oracle.slot_valid(perm, Np)
+    qn, kn, vn = (to_np64(x[:, :, heads]) for x in (q, k, v))
+    rp, ci = oracle.fixed_k_csr(kv_gpu[:, heads])
+    O, LSE = oracle.masked_attention(*(oracle.reorder_fwd(x, perm, Np) for x in (qn, kn, vn)),
+                                     valid, ph * pw, rp, ci, True, 1 / math.sqrt(w.D),
+                                     q_blocks=q_blocks)
+    return (oracle.reorder_inv(np.nan_to_num(O, nan=np.inf), perm),
+            np.nan_to_num(LSE, nan=np.inf)[:, :, perm])
+
+
 @pytest.mark.parametrize("over", CASES)
-def test_attn_natural_equals_reorder_path_bitwise(over):
+def test_attn_natural_matches_oracle_and_reorder_path(over):
+    # grids with partial edge tiles: the natural-layout kernel packs the
+    # kept edge key tiles several to an MMA tile, so its key order differs
+    # from the reorder path's; both are within tolerance of the oracle
     over = dict(over)
     w = small_workload(CONFIGS[over.pop("cid")], **over)
     q, k, v = make_qkv(w, device="cuda")
     att = DraftAttention(w.B, w.Hh, w.D, w.T, w.H, w.W, w.draft_ph, w.draft_pw, w.draft_sparsity)
     a = att(q, k, v)
-    lse_slots = att.lse.clone()
     kv_a = att.col_idx.clone()
     b = torch.full_like(q, float("nan"))
     lse_nat = torch.full((w.B, w.Hh, w.N), float("nan"), dtype=torch.float32, device="cuda")
     att.fused(q, k, v, b, lse_nat)
     bsa.bsa_poll_status(att.plan)
     assert torch.equal(att.col_idx, kv_a)                        # same kept blocks
-    assert torch.equal(a.view(torch.int16), b.view(torch.int16))  # same bits, every token
-    perm, _ = oracle.tile_layout_perm(w.T, w.H, w.W, w.draft_ph, w.draft_pw)
-    idx = torch.from_numpy(perm).cuda()
-    assert torch.equal(lse_slots[:, :, idx], lse_nat)
+    nb = att.plan.nblocks
+    kv = att.col_idx.view(w.B, w.Hh, nb, -1).cpu().numpy()
+    heads = sorted({0, w.Hh - 1})
+    small = w.N * w.Hh <= 200_000
+    ref, ref_lse = _oracle_natural(w, q, k, v, kv, heads,
+                                   None if small else sample_blocks(nb, 6, seed=w.N))
+    got = to_np64(b[:, :, heads])
+    m = np.isfinite(ref)
+    err = np.abs(got[m] - ref[m])
+    assert m.any() and err.max() <= MAX_ABS and err.mean() <= MEAN_ABS
+    lse = lse_nat[:, heads].cpu().numpy().astype(np.float64)
+    ml = np.isfinite(ref_lse)
+    assert np.abs(lse[ml] - ref_lse[ml]).max() <= 2e-3
+    d = (a.float() - b.float()).abs()                             # the two GPU paths agree
+    assert d.max().item() <= MAX_ABS and d.mean().item() <= MEAN_ABS
+
+
+def test_attn_natural_equals_reorder_path_bitwise_without_edge_tiles():
+    # 8 x 16 tiles dividing a 16 x 32 grid: no partial tiles, nothing to
+    # pack, so the natural-layout kernel does the reorder path's arithmetic
+    # on the same tiles: the same bits on every token
+    w = small_workload(CONFIGS[2], T=3, H=16, W=32, Hh=2, field_grid=(3, 4, 7))
+    q, k, v = make_qkv(w, device="cuda")
+    att = DraftAttention(w.B, w.Hh, w.D, w.T, w.H, w.W, 8, 16, 50)
+    a = att(q, k, v)
+    lse_slots = att.lse.clone()
+    b = torch.full_like(q, float("nan"))
+    lse_nat = torch.full((w.B, w.Hh, w.N), float("nan"), dtype=torch.float32, device="cuda")
+    att.fused(q, k, v, b, lse_nat)
+    bsa.bsa_poll_status(att.plan)
+    assert torch.equal(a.view(torch.int16), b.view(torch.int16))
+    perm, _ = oracle.tile_layout_perm(w.T, w.H, w.W, 8, 16)
+    assert torch.equal(lse_slots[:, :, torch.from_numpy(perm).cuda()], lse_nat)
+
+
+def test_attn_natural_long_lists_run_unpacked():
+    # 792 key blocks, all kept (sparsity 0): lists longer than a CTA packs
+    # run tile by tile; sampled query blocks against the oracle
+    w = small_workload(CONFIGS[2], T=11, H=90, W=90, Hh=1, D=64, draft_sparsity=0,
+                       field_grid=(11, 4, 7))
+    q, k, v = make_qkv(w, device="cuda")
+    att = DraftAttention(w.B, w.Hh, w.D, w.T, w.H, w.W, 8, 16, 0)
+    assert att.plan.nblocks == 792 and att.keep == 792
+    out = att.fused(q, k, v)
+    bsa.bsa_poll_status(att.plan)
+    kv = att.col_idx.view(1, 1, 792, -1).cpu().numpy()
+    assert (kv == np.arange(792)).all()
+    ref, _ = _oracle_natural(w, q, k, v, kv, [0], q_blocks=[0, 71, 400, 791])
+    got = to_np64(out)
+    m = np.isfinite(ref)
+    err = np.abs(got[m] - ref[m])
+    assert m.any() and err.max() <= MAX_ABS and err.mean() <= MEAN_ABS
 
 
 @pytest.mark.parametrize("cid", [2, 5])
