@@ -46,11 +46,13 @@ from synth import CONFIGS, make_qkv  # noqa: E402
 
 METRIC = "bsattn ms/call + attended TFLOP/s (% BF16 peak), Wan-1.3B-shape 6× length LVSA"
 
-# DRAM bytes per launch of the step kernel at the full workload, from the ncu
-# capture summarised in profiles/lvsa_attn_fwd_wan13b_6x_first24frames.md
-# (24-frame case, scaled by the number of query pairs).  Set to None whenever
-# the kernel changes until it is captured again.
+# DRAM bytes per launch of the LVSA step kernel at the full Wan-1.3B 6x
+# workload: dram__bytes_read.sum + dram__bytes_write.sum of one ncu capture of
+# the same kernel on the first 24 frames (447.9 MB), scaled by the number of
+# query pairs (126 / 24).  None whenever the kernel has changed since.
 STEP_KERNEL_DRAM_BYTES = 447.9e6 * 126 / 24
+STEP_KERNEL_TRAFFIC_SOURCE = ("ncu capture of lvsa_attn_kernel on the first 24 frames "
+                              "(447.9 MB), scaled by 126/24; not measured by this run")
 
 
 def attended_flops(w) -> float:
@@ -65,6 +67,8 @@ def peaks():
             d = json.load(f)
         return d, "measured"
     except Exception:
+        # the profiling recipe's fallback for this machine's B200s (an earlier
+        # measurement: STREAM-style copy, cuBLAS bf16 burst and sustained)
         return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}, "fallback"
 
 
@@ -192,12 +196,18 @@ def run_reference(args, rank, world):
     n_all = args.warmup + args.steps
     budget = min(args.ref_step_s, max(0.25, 120.0 / n_all))
     for i in range(n_all):
-        val, thr, desc, _ = cpu_baseline(w, q_h, k_h, v_h, budget_s=budget, seed=i)
+        if w.lvsa_C:
+            val, thr, desc, _ = cpu_baseline(w, q_h, k_h, v_h, budget_s=budget, seed=i)
+        else:
+            val, thr, desc, _ = cpu_baseline_draft(w, q_h, k_h, v_h, budget, seed=i)
         if i >= args.warmup:
             vals.append(val)
     value = statistics.mean(vals)
     line = {
-        "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s",
+        "impl": "reference",
+        "metric": METRIC if w.lvsa_C else
+        f"bsattn ms/call + attended TFLOP/s (% BF16 peak), {w.name}, draft attention",
+        "value": value, "unit": "TFLOP/s",
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": None, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
@@ -267,7 +277,10 @@ def kernel_table(args):
             d["note"] = note
         print(json.dumps(d), flush=True)
 
+    only = {int(c) for c in args.table_configs.split(",")} if args.table_configs else None
     for cid in sorted(CONFIGS):
+        if only is not None and cid not in only:
+            continue
         w = CONFIGS[cid]
         q, k, v = make_qkv(w, device="cuda")
         out = torch.empty_like(q)
@@ -442,6 +455,8 @@ def main():
     ap.add_argument("--kernel-table", action="store_true",
                     help="time every kernel on every workload instead of the step")
     ap.add_argument("--table-reps", type=int, default=10)
+    ap.add_argument("--table-configs", default="",
+                    help="comma-separated workloads for --kernel-table (default: all)")
     ap.add_argument("--draft-pipelines", type=int, default=0, metavar="HEADS",
                     help="run the three draft pipelines on HEADS heads (profiling)")
     ap.add_argument("--hbm-kernels", type=int, default=0, metavar="CONFIG",
@@ -470,7 +485,7 @@ def main():
         raise SystemExit("at least 3 warm-up steps")
 
     import block_sparse_attention_49_b200 as bsa
-    from block_sparse_attention_49_b200.pipeline import LvsaAttention
+    bsa.load()  # fails loudly when the library is missing
 
     torch.cuda.set_device(local)
     dist = None
@@ -486,48 +501,47 @@ def main():
         Tc, Hc, Wc = w.field_grid
         w = small_workload(w, T=args.frames, field_grid=(args.frames, Hc, Wc),
                            name=f"{w.name} (first {args.frames} frames)")
-    flops_step = attended_flops(w)
     q, k, v = make_qkv(w, device="cuda")
-    att = LvsaAttention(w.B, w.Hh, w.D, w.T, w.H, w.W, w.lvsa_C, w.lvsa_T_per, block=128)
     out = torch.empty_like(q)
     stream = torch.cuda.current_stream()
     ev = lambda: torch.cuda.Event(enable_timing=True)
+    if w.lvsa_C:
+        step_setup = lvsa_step_setup(w, q, k, v, out)
+    else:
+        step_setup = draft_step_setup(w, q, k, v, out)
+    step, flops_step, dominant, extra = step_setup
 
-    def step(i):
-        att.fused(q, k, v, i % w.lvsa_T_per, out)
-
+    # warm-up, then exactly `steps` timed steps between barriers
     for i in range(args.warmup):
-        step(i)
-    bsa.bsa_poll_status(att.plan)
+        step(i, None)
+    extra["poll"]()
     torch.cuda.synchronize()
     if dist:
         dist.barrier()
     clocks = ClockSampler(local)
     clocks.start()
     marks = [ev() for _ in range(args.steps + 1)]
+    dom = [(ev(), ev()) for _ in range(args.steps)]
     torch.cuda.synchronize()
     marks[0].record(stream)
     for i in range(args.steps):
-        step(args.warmup + i)
+        step(args.warmup + i, dom[i])
         marks[i + 1].record(stream)
     torch.cuda.synchronize()
     if dist:
         dist.barrier()
     clk = clocks.stop()
-    bsa.bsa_poll_status(att.plan)
-    per_call = [marks[i].elapsed_time(marks[i + 1]) for i in range(args.steps)]
+    extra["poll"]()
     ms = marks[0].elapsed_time(marks[-1]) / args.steps
-    attn_ms = statistics.mean(per_call)  # the step is the one attention launch
-    ms, attn_ms = max_over_ranks([ms, attn_ms], dist, "cuda")
+    dom_ms = statistics.mean(a.elapsed_time(b) for a, b in dom)
+    ms, dom_ms = max_over_ranks([ms, dom_ms], dist, "cuda")
 
-    # the four-kernel path on the same data, per kernel (secondary numbers)
-    names = ("lvsa_mask", "reorder_fwd", "attn_fwd_blocklist", "reorder_inv")
-    unf = {n: [] for n in names}
-    n_unf = max(3, min(args.steps, 10))
-    for i in range(args.warmup + n_unf):
-        s_i = i % w.lvsa_T_per
-        calls = (lambda: att.mask(s_i), lambda: att.gather(q, k, v),
-                 lambda: att.attend(per_head=False), lambda: att.scatter(out))
+    # the same path as separate kernels (secondary numbers)
+    names, calls_of = extra["breakdown"]
+    per = {n: [] for n in names}
+    n_sep = max(3, min(args.steps, 10))
+    for i in range(args.warmup + n_sep):
+        calls = calls_of(i)
         m = [ev() for _ in range(len(calls) + 1)]
         m[0].record(stream)
         for j, c in enumerate(calls):
@@ -536,10 +550,10 @@ def main():
         if i >= args.warmup:
             torch.cuda.synchronize()
             for j, n in enumerate(names):
-                unf[n].append(m[j].elapsed_time(m[j + 1]))
+                per[n].append(m[j].elapsed_time(m[j + 1]))
     torch.cuda.synchronize()
-    bsa.bsa_poll_status(att.plan)
-    unf_ms = max_over_ranks([statistics.mean(unf[n]) for n in names], dist, "cuda")
+    extra["poll"]()
+    sep_ms = max_over_ranks([statistics.mean(per[n]) for n in names], dist, "cuda")
 
     # end to end through the public API with host buffers: every step copies
     # its Q, K, V in from pinned host memory and its O back out; the copies
@@ -548,7 +562,7 @@ def main():
     hq, hk, hv = (x.cpu().pin_memory() for x in (q, k, v))
     ho = torch.empty_like(hq).pin_memory()
     streamed = StreamedSteps(q.shape, q.dtype)
-    step_fn = lambda dq, dk, dv, dout, i: att.fused(dq, dk, dv, i % w.lvsa_T_per, dout)
+    step_fn = extra["host_step"]
     streamed.run(step_fn, (hq, hk, hv), ho, 2)       # warm-up
     torch.cuda.synchronize()
     if dist:
@@ -556,26 +570,39 @@ def main():
     e0, e1 = streamed.run(step_fn, (hq, hk, hv), ho, args.e2e_steps)
     torch.cuda.synchronize()
     (e2e_ms,) = max_over_ranks([e0.elapsed_time(e1) / args.e2e_steps], dist, "cuda")
-    bsa.bsa_poll_status(att.plan)
+    extra["poll"]()
     del streamed
 
     pk, pk_kind = peaks()
-    peak = pk.get("bf16_tflops_sustained", pk["bf16_tflops"])
-    attn_tflops = flops_step / (attn_ms * 1e-3) / 1e12
+    burst = pk["bf16_tflops"]
+    sustained = pk.get("bf16_tflops_sustained")
+    dom_tflops = flops_step / (dom_ms * 1e-3) / 1e12
     tok_bytes = w.B * w.N * w.Hh * w.D * 2
-    algo_bytes = {"lvsa_mask": 4 * (att.col_idx.numel() + att.row_ptr.numel() + att.frame_sets.numel()),
-                  "reorder_fwd": 3 * 2 * tok_bytes, "reorder_inv": 2 * tok_bytes}
-    four = {}
-    for n, t in zip(names, unf_ms):
+    sep = {}
+    for n, t in zip(names, sep_ms):
         d = {"ms": t}
-        if n in algo_bytes:
-            gbs = algo_bytes[n] / (t * 1e-3) / 1e9
-            d.update({"algo_bytes": algo_bytes[n], "GB_s": gbs, "frac_hbm": gbs / pk["hbm_gbs"]})
+        ab = extra["algo_bytes"].get(n)
+        if ab is not None:
+            gbs = ab / (t * 1e-3) / 1e9
+            d.update({"algo_bytes": ab, "GB_s": gbs, "frac_hbm": gbs / pk["hbm_gbs"]})
         else:
             d["attended_tflops"] = flops_step / (t * 1e-3) / 1e12
-        four[n] = d
+        sep[n] = d
+    roof = {"bound": "tensor", "achieved": dom_tflops, "peak": burst, "unit": "TFLOP/s",
+            "frac": dom_tflops / burst, "traffic": extra["traffic"],
+            "peak_kind": f"{pk_kind} bf16 burst (the kernel timed on its own)",
+            "kernel": dominant}
+    if extra.get("traffic_source"):
+        roof["traffic_source"] = extra["traffic_source"]
+    if sustained:
+        roof["frac_of_sustained"] = dom_tflops / sustained
+        peak_mhz = _peak_sm_mhz(pk)
+        if peak_mhz and clk and clk.get("sm_mhz"):
+            # the same ratio per clock: sustained peak and kernel each divided
+            # by the median SM clock seen while they ran
+            roof["frac_of_sustained_per_clock"] = (dom_tflops / clk["sm_mhz"]) / (sustained / peak_mhz)
     line = {
-        "metric": METRIC,
+        "metric": extra["metric"],
         "value": weak_scaling_value(flops_step, world, ms),
         "unit": "TFLOP/s",
         "n_gpus": world,
@@ -587,23 +614,18 @@ def main():
         "vs_baseline": None,
         "dtype": "bf16",
         "data": "synthetic",
-        "config": {"workload": w.name, "global_batch": w.B * world, "seq_len": w.N,
-                   "heads": w.Hh, "head_dim": w.D, "lvsa_C": w.lvsa_C,
-                   "lvsa_T_per": w.lvsa_T_per, "steps_s": "s = step mod T_per",
-                   "path": "bsa_lvsa_attn_fwd (one kernel, natural layout)",
-                   "parallelism": f"dp{world}",
-                   "l2": "inputs (1.8 GB) larger than L2; no flush"},
-        "bsattn_ms_per_call": attn_ms,
-        "bsattn_attended_tflops": attn_tflops,
-        "bsattn_pct_bf16_peak": 100.0 * attn_tflops / peak,
+        "config": dict(extra["config"], workload=w.name, global_batch=w.B * world, seq_len=w.N,
+                       heads=w.Hh, head_dim=w.D, parallelism=f"dp{world}",
+                       l2=f"inputs ({3 * tok_bytes / 1e9:.2f} GB) "
+                          + ("larger than L2; no flush" if 3 * tok_bytes > 126e6
+                             else "smaller than L2 (tiny case)")),
+        "bsattn_ms_per_call": dom_ms,
+        "bsattn_attended_tflops": dom_tflops,
+        "bsattn_pct_bf16_peak": 100.0 * dom_tflops / burst,
         "attended_tflop_per_call": flops_step / 1e12,
-        "roofline": {"bound": "tensor", "achieved": attn_tflops, "peak": peak,
-                     "unit": "TFLOP/s", "frac": attn_tflops / peak,
-                     "traffic": (STEP_KERNEL_DRAM_BYTES * w.T / 126
-                                 if STEP_KERNEL_DRAM_BYTES and args.config == 3 else None),
-                     "peak_kind": f"{pk_kind} bf16 sustained (kernel timed inside a long step)"},
-        "four_kernel_path": {"ms_per_step": sum(unf_ms), "kernels": four},
-        "gpu_launches": args.steps,
+        "roofline": roof,
+        extra["breakdown_key"]: {"ms_per_step": sum(sep_ms), "kernels": sep},
+        "gpu_launches": args.steps * extra["launches_per_step"],
         "clocks": clk,
         "e2e": {"value": weak_scaling_value(flops_step, world, e2e_ms), "unit": "TFLOP/s",
                 "ms_per_step": e2e_ms,
@@ -612,7 +634,7 @@ def main():
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         q_h, k_h, v_h = (x[:, :, :1].float().cpu().numpy().astype(np.float64) for x in (q, k, v))
-        val, thr, desc, _ = cpu_baseline(w, q_h, k_h, v_h, budget_s=args.cpu_budget_s)
+        val, thr, desc, _ = extra["cpu_baseline"](w, q_h, k_h, v_h, args.cpu_budget_s)
         line["cpu_baseline"] = {"value": val, "unit": "TFLOP/s", "cores": thr, "kind": "oracle",
                                 "sample": desc}
     if rank == 0:
@@ -621,6 +643,146 @@ def main():
         dist.barrier()
         dist.destroy_process_group()
 
+
+def _peak_sm_mhz(pk):
+    """Median SM clock of the sustained peak measurement, if the peaks file
+    records one."""
+    for key in ("clocks_under_load", "clocks", "sustained_clocks"):
+        c = pk.get(key)
+        if isinstance(c, dict):
+            for name, val in c.items():
+                if "sm" in name and isinstance(val, (int, float)) and val > 100:
+                    return float(val)
+        elif isinstance(c, (int, float)) and c > 100:
+            return float(c)
+    return None
+
+
+def lvsa_step_setup(w, q, k, v, out):
+    """The LVSA step: bsa_lvsa_attn_fwd (one kernel, natural layout) with
+    s = step mod T_per.  Returns (step, attended flops, kernel name, extras)."""
+    import block_sparse_attention_49_b200 as bsa
+    from block_sparse_attention_49_b200.pipeline import LvsaAttention
+    att = LvsaAttention(w.B, w.Hh, w.D, w.T, w.H, w.W, w.lvsa_C, w.lvsa_T_per, block=128)
+    stream = torch.cuda.current_stream()
+
+    def step(i, evs):
+        if evs:
+            evs[0].record(stream)
+        att.fused(q, k, v, i % w.lvsa_T_per, out)
+        if evs:
+            evs[1].record(stream)
+
+    def calls_of(i):
+        s_i = i % w.lvsa_T_per
+        return (lambda: att.mask(s_i), lambda: att.gather(q, k, v),
+                lambda: att.attend(per_head=False), lambda: att.scatter(out))
+
+    tok_bytes = w.B * w.N * w.Hh * w.D * 2
+    scaled = STEP_KERNEL_DRAM_BYTES is not None and w.name == CONFIGS[3].name
+    extra = {
+        "metric": METRIC,
+        "poll": lambda: bsa.bsa_poll_status(att.plan),
+        "breakdown": (("lvsa_mask", "reorder_fwd", "attn_fwd_blocklist", "reorder_inv"), calls_of),
+        "breakdown_key": "four_kernel_path",
+        "algo_bytes": {"lvsa_mask": 4 * (att.col_idx.numel() + att.row_ptr.numel() +
+                                         att.frame_sets.numel()),
+                       "reorder_fwd": 3 * 2 * tok_bytes, "reorder_inv": 2 * tok_bytes},
+        "host_step": lambda dq, dk, dv, dout, i: att.fused(dq, dk, dv, i % w.lvsa_T_per, dout),
+        "launches_per_step": 1,
+        "traffic": STEP_KERNEL_DRAM_BYTES if scaled else None,
+        "traffic_source": STEP_KERNEL_TRAFFIC_SOURCE if scaled else None,
+        "config": {"lvsa_C": w.lvsa_C, "lvsa_T_per": w.lvsa_T_per,
+                   "steps_s": "s = step mod T_per",
+                   "path": "bsa_lvsa_attn_fwd (one kernel, natural layout)",
+                   "window_growth": "alternating right/left pointers (plan default)",
+                   "lse": "not written (lse = NULL)"},
+        "cpu_baseline": lambda w_, qh, kh, vh, budget: cpu_baseline(w_, qh, kh, vh, budget_s=budget),
+    }
+    return step, attended_flops(w), "lvsa_attn_kernel", extra
+
+
+def draft_step_setup(w, q, k, v, out):
+    """The draft step: bsa_draft_mask_natural (pooling in place, scoring,
+    top-k) then bsa_attn_fwd_natural on the natural layout."""
+    import block_sparse_attention_49_b200 as bsa
+    from block_sparse_attention_49_b200.pipeline import DraftAttention
+    att = DraftAttention(w.B, w.Hh, w.D, w.T, w.H, w.W, w.draft_ph, w.draft_pw, w.draft_sparsity)
+    if w.draft_ph * w.draft_pw != 128:
+        raise SystemExit("the draft step on the natural layout needs pool_h * pool_w = 128")
+    stream = torch.cuda.current_stream()
+    scale = 1.0 / math.sqrt(w.D)
+
+    def mask():
+        bsa.bsa_draft_mask_natural(att.plan, q, k, att.sparsity, att.row_ptr, att.col_idx, None,
+                                   att.workspace)
+
+    def attend():
+        bsa.bsa_attn_fwd_natural(att.plan, q, k, v, att.row_ptr, att.col_idx, True, scale, out)
+
+    def step(i, evs):
+        mask()
+        if evs:
+            evs[0].record(stream)
+        attend()
+        if evs:
+            evs[1].record(stream)
+
+    mask()
+    torch.cuda.synchronize()
+    flops = draft_attended_flops(w, att.col_idx.cpu().numpy(), att.keep)
+    tok_bytes = w.B * w.N * w.Hh * w.D * 2
+    pooled = 2 * w.B * w.Hh * att.plan.nblocks * w.D * 8
+    extra = {
+        "metric": f"bsattn ms/call + attended TFLOP/s (% BF16 peak), {w.name}, draft attention",
+        "poll": lambda: bsa.bsa_poll_status(att.plan),
+        "breakdown": (("reorder_fwd", "draft_mask", "attn_fwd_blocklist", "reorder_inv"),
+                      lambda i: (lambda: att.gather(q, k, v), att.mask,
+                                 lambda: att.attend(per_head=True), lambda: att.scatter(out))),
+        "breakdown_key": "reorder_path",
+        "algo_bytes": {"reorder_fwd": 3 * 2 * tok_bytes, "reorder_inv": 2 * tok_bytes,
+                       "draft_mask": 2 * tok_bytes + 2 * pooled + 4 * att.col_idx.numel()},
+        "host_step": lambda dq, dk, dv, dout, i: att.fused(dq, dk, dv, dout),
+        "launches_per_step": 3,
+        "traffic": None,
+        "config": {"draft_pool": f"{w.draft_ph}x{w.draft_pw}", "sparsity_pct": w.draft_sparsity,
+                   "keep_per_row": att.keep, "blocks_per_head": att.plan.nblocks,
+                   "path": "bsa_draft_mask_natural + bsa_attn_fwd_natural (natural layout)",
+                   "lse": "not written (lse = NULL)"},
+        "cpu_baseline": cpu_baseline_draft,
+    }
+    return step, flops, "attn_fwd_kernel (natural layout, draft lists)", extra
+
+
+def cpu_baseline_draft(w, q_h, k_h, v_h, budget_s: float, seed: int = 0):
+    """The oracle on a bounded sample of the draft workload: head 0's draft
+    blocks in full, then masked attention of sampled query blocks."""
+    import oracle
+    t0 = time.perf_counter()
+    kv = oracle.draft_blocks(q_h, k_h, w.T, w.H, w.W, w.draft_ph, w.draft_pw, w.draft_sparsity)
+    rp, ci = oracle.fixed_k_csr(kv)
+    perm, Np = oracle.tile_layout_perm(w.T, w.H, w.W, w.draft_ph, w.draft_pw)
+    valid = oracle.slot_valid(perm, Np)
+    qs, ks, vs = (oracle.reorder_fwd(x, perm, Np) for x in (q_h, k_h, v_h))
+    setup = time.perf_counter() - t0
+    blk = w.draft_ph * w.draft_pw
+    nb = Np // blk
+    rng = np.random.default_rng(seed)
+    done, flops, t_att = 0, 0.0, 0.0
+    while t_att < budget_s and done < nb:
+        qb = int(rng.integers(0, nb))
+        t1 = time.perf_counter()
+        oracle.masked_attention(qs, ks, vs, valid, blk, rp, ci, True, 1 / math.sqrt(w.D),
+                                q_blocks=[qb], heads=[(0, 0)])
+        t_att += time.perf_counter() - t1
+        nq = int(valid[qb * blk:(qb + 1) * blk].sum())
+        keys = sum(int(valid[c * blk:(c + 1) * blk].sum()) for c in ci[rp[qb]:rp[qb + 1]])
+        flops += 4.0 * w.D * nq * keys
+        done += 1
+    threads = torch.get_num_threads()
+    desc = (f"oracle masked attention on {done} random query blocks of head 0 (of {nb} x {w.Hh}), "
+            f"draft lists of head 0; draft mask and layout set-up {setup:.1f}s excluded")
+    return flops / t_att / 1e12, threads, desc, t_att
 
 if __name__ == "__main__":
     main()
