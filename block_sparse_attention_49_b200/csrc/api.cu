@@ -238,6 +238,8 @@ bsa_status bsa_draft_mask(bsa_plan_t plan, const void* q_slots, const void* k_sl
   if (workspace_bytes < draft_workspace_bytes(g))
     return set_error(BSA_ERR_INVALID_ARG, "workspace too small");
   if (g.nblocks > 18000) return set_error(BSA_ERR_UNSUPPORTED, "draft mask supports up to 18000 blocks");
+  if ((int64_t)g.B * g.Hh * g.Npad >= (1ll << 31))
+    return set_error(BSA_ERR_UNSUPPORTED, "draft mask needs B*Hh*Npad < 2^31");
   const int keep = bsa_draft_keep_count(plan, sparsity_pct);
   if ((int64_t)g.B * g.Hh * g.nblocks * keep >= (1ll << 31))
     return set_error(BSA_ERR_UNSUPPORTED, "block list longer than 2^31 entries");
@@ -328,6 +330,8 @@ bsa_status bsa_draft_mask_natural(bsa_plan_t plan, const void* q, const void* k,
   if (workspace_bytes < draft_workspace_bytes(g))
     return set_error(BSA_ERR_INVALID_ARG, "workspace too small");
   if (g.nblocks > 18000) return set_error(BSA_ERR_UNSUPPORTED, "draft mask supports up to 18000 blocks");
+  if ((int64_t)g.B * g.Hh * g.Npad >= (1ll << 31))
+    return set_error(BSA_ERR_UNSUPPORTED, "draft mask needs B*Hh*Npad < 2^31");
   const int keep = bsa_draft_keep_count(plan, sparsity_pct);
   if ((int64_t)g.B * g.Hh * g.nblocks * keep >= (1ll << 31))
     return set_error(BSA_ERR_UNSUPPORTED, "block list longer than 2^31 entries");
@@ -359,6 +363,8 @@ bsa_status bsa_draft_mask_natural_e4m3(bsa_plan_t plan, const void* q, const voi
   if (workspace_bytes < draft_workspace_bytes(g))
     return set_error(BSA_ERR_INVALID_ARG, "workspace too small");
   if (g.nblocks > 18000) return set_error(BSA_ERR_UNSUPPORTED, "draft mask supports up to 18000 blocks");
+  if ((int64_t)g.B * g.Hh * g.Npad >= (1ll << 31))
+    return set_error(BSA_ERR_UNSUPPORTED, "draft mask needs B*Hh*Npad < 2^31");
   const int keep = bsa_draft_keep_count(plan, sparsity_pct);
   if ((int64_t)g.B * g.Hh * g.nblocks * keep >= (1ll << 31))
     return set_error(BSA_ERR_UNSUPPORTED, "block list longer than 2^31 entries");

@@ -4,13 +4,14 @@
 // block connections, at a stated sparsity; pool_h*pool_w equals the block
 // size of the block-sparse attention that follows).
 //
-// Two kernels, both on the tile-layout slot tensors (each block = one tile):
-//  pool:  qbar/kbar[b,h,blk,:] = mean of the block's non-empty slots, fp64.
-//         The sum runs sequentially over the block's slots in order (the
-//         tile's row-major order) and is divided once by the token count.
-//         With max pooling (which the article's authors tried before
-//         settling on the average) it is the channel-wise maximum instead,
-//         exact in any order.  16-byte loads; HBM bound.
+// Two kernels, on the tile-layout slot tensors or in place on the natural
+// layout (each block = one pool_h x pool_w tile):
+//  pool:  qbar/kbar[b,h,blk,:] = mean of the tile's tokens, fp64.  The sum
+//         runs sequentially over the tile's tokens in row-major order and is
+//         divided once by the token count.  With max pooling (which the
+//         article's authors tried before settling on the average) it is the
+//         channel-wise maximum instead, exact in any order.  16-byte
+//         loads, four rows ahead; HBM bound.
 //  score_topk: for a group of query-block rows of one (b, head), the fp64
 //         logits L[i][j] = sum_c qbar_i[c]*kbar_j[c] (sequential over c, the
 //         product and the sum each rounded, no fused multiply-add), then per
@@ -24,6 +25,7 @@
 
 #include <algorithm>
 #include <cfloat>
+#include <type_traits>
 
 #include "bsa_internal.cuh"
 #include "ptx.cuh"
@@ -31,105 +33,79 @@
 namespace bsa {
 namespace {
 
-constexpr int kPoolThreads = 256;
 constexpr int kScoreThreads = 256;
 constexpr int kKeyChunk = 32;  // key blocks staged in shared memory per step
 constexpr int kRegCand = 16;   // top-k candidates per lane held in registers (Nb <= 512)
 constexpr unsigned kFullMaskScore = 0xffffffffu;
 
-// One group of D/8 threads per (which, b, h, block); each thread owns 8
-// channels.  which = 0: Q, 1: K.
-template <int D>
-__global__ void __launch_bounds__(kPoolThreads)
-    draft_pool_kernel(const uint4* __restrict__ q, const uint4* __restrict__ k,
-                      const uint32_t* __restrict__ tile_valid, int Hh, int64_t Npad,
-                      int64_t nblocks, int block, int64_t groups_per_tensor, int use_max,
-                      double* __restrict__ ws) {
-  constexpr int kTPG = D / 8;  // threads per group
-  const int64_t gid = ((int64_t)blockIdx.x * kPoolThreads + threadIdx.x) / kTPG;
-  const int sub = threadIdx.x % kTPG;
-  if (gid >= 2 * groups_per_tensor) return;
-  const int which = gid >= groups_per_tensor;
-  const int64_t g = gid - which * groups_per_tensor;  // (b*Hh + h)*nblocks + blk
-  const int64_t bh = g / nblocks, blk = g - bh * nblocks;
-  const uint4* src = (which ? k : q) + ((bh * Npad + blk * block) * (D / 8)) + sub;
-  const int64_t s0 = blk * block;
-  double acc[8];
-#pragma unroll
-  for (int i = 0; i < 8; ++i) acc[i] = use_max ? -INFINITY : 0.0;
-  int cnt = 0;
-  for (int e = 0; e < block; ++e) {
-    const int64_t s = s0 + e;
-    const uint32_t w = __ldg(tile_valid + (s >> 5));
-    if (!((w >> (s & 31)) & 1u)) continue;
-    const uint4 v = __ldg(src + (int64_t)e * (D / 8));
-    const __nv_bfloat162* pv = reinterpret_cast<const __nv_bfloat162*>(&v);
-    if (use_max) {
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const float2 f = __bfloat1622float2(pv[i]);
-        acc[2 * i] = fmax(acc[2 * i], (double)f.x);
-        acc[2 * i + 1] = fmax(acc[2 * i + 1], (double)f.y);
-      }
-    } else {
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const float2 f = __bfloat1622float2(pv[i]);
-        acc[2 * i] = __dadd_rn(acc[2 * i], (double)f.x);
-        acc[2 * i + 1] = __dadd_rn(acc[2 * i + 1], (double)f.y);
-      }
-    }
-    ++cnt;
-  }
-  double* dst = ws + ((int64_t)which * groups_per_tensor + g) * D + sub * 8;
-  const double dc = (double)cnt;
-#pragma unroll
-  for (int i = 0; i < 8; ++i) dst[i] = cnt ? (use_max ? acc[i] : __ddiv_rn(acc[i], dc)) : 0.0;
-}
+// ---------------------------------------------------------------------------
+// Pooling.  One group of D/8 threads per unit (Q or K, tile, batch, head);
+// each thread owns 8 channels: eight independent fp64 chains, each the
+// sequential sum over the tile's tokens in row-major order.  Token rows are
+// read with 16-byte loads, four rows ahead of the additions.  Units are
+// ordered heads fastest, so the groups of a warp read neighbouring 256-byte
+// rows of one token.  At most 64 registers a thread: four 256-thread CTAs fit
+// on an SM, so a 12-head Wan-1.3B-like problem runs in one wave.
+//   natural layout [B, N, Hh, D]: the tokens of the pool_h x pool_w tile
+//     inside the grid, row by row;
+//   slot layout [B, Hh, Npad, D]: the block's non-empty slots in order (runs
+//     of consecutive slots, from the plan's validity bits).
+// Optionally records max |x| per (Q or K, batch, head) for the e4m3 scales.
+// ---------------------------------------------------------------------------
+constexpr int kPoolThreads = 256;
 
-// The same pooling read straight from the natural layout [B, N, Hh, D]: one
-// group of D/8 threads per (which, block, b, h), heads fastest, so the
-// groups of a warp read neighbouring 256-byte rows of one token.  The tile's
-// tokens inside the grid are visited in row-major (a, then b) order, loads
-// eight at a time ahead of the sequential fp64 additions.
-template <int D>
-__global__ void __launch_bounds__(kPoolThreads)
-    draft_pool_nat_kernel(const uint4* __restrict__ q, const uint4* __restrict__ k, int B, int Hh,
-                          int T, int H, int W, int ph, int pw, int TH, int TW, int64_t nblocks,
-                          int64_t groups_per_tensor, int use_max, double* __restrict__ ws) {
-  constexpr int kTPG = D / 8;
-  constexpr int kAhead = 8;
+struct PoolParams {
+  int B, Hh, T, H, W, ph, pw, TH, TW, block;
+  int64_t nblocks, Npad, groups_per_tensor;
+  int use_max;
+  const uint32_t* tile_valid;
+  uint32_t* amax;  // [3][B][Hh] float bits, or null
+  double* ws;
+};
+
+template <int D, bool NAT, bool MAXP, bool AMAX>
+__global__ void __launch_bounds__(kPoolThreads, 4)
+    draft_pool_kernel(const uint4* __restrict__ q, const uint4* __restrict__ k, const PoolParams p) {
+  constexpr int kTPG = D / 8;  // threads per group
+  constexpr int kAhead = 4;
   const int64_t gid = ((int64_t)blockIdx.x * kPoolThreads + threadIdx.x) / kTPG;
   const int sub = threadIdx.x % kTPG;
-  if (gid >= 2 * groups_per_tensor) return;
-  const int which = gid >= groups_per_tensor;
-  const int64_t gg = gid - which * groups_per_tensor;  // (blk * B + b) * Hh + h
-  const int h = (int)(gg % Hh);
-  const int64_t rest = gg / Hh;
-  const int b = (int)(rest % B);
-  const int64_t blk = rest / B;
-  const int t = (int)(blk / ((int64_t)TH * TW));
-  const int r = (int)(blk - (int64_t)t * TH * TW);
-  const int i = r / TW, j = r - (r / TW) * TW;
-  const int y0 = i * ph, x0 = j * pw;
-  const int hn = min(ph, H - y0), wn = min(pw, W - x0);
-  const int64_t N = (int64_t)T * H * W;
-  const uint4* src = (which ? k : q) + (((int64_t)b * N + ((int64_t)t * H + y0) * W + x0) * Hh + h) *
-                                           (D / 8) + sub;
-  const int64_t row_step = (int64_t)Hh * (D / 8);  // one token
+  const bool live = gid < 2 * p.groups_per_tensor;
+  const int which = live && gid >= p.groups_per_tensor;
+  const int64_t gg = live ? gid - which * p.groups_per_tensor : 0;  // (blk * B + b) * Hh + h
+  const int h = (int)(gg % p.Hh);
+  const int64_t rest = gg / p.Hh;
+  const int b = (int)(rest % p.B);
+  const int64_t blk = rest / p.B;
+  const int64_t row_step = NAT ? (int64_t)p.Hh * (D / 8) : (D / 8);  // one token / one slot
+  const uint4* base;
+  if (NAT) {
+    const int t = (int)(blk / ((int64_t)p.TH * p.TW));
+    const int r = (int)(blk - (int64_t)t * p.TH * p.TW);
+    const int i = r / p.TW, j = r - (r / p.TW) * p.TW;
+    const int64_t N = (int64_t)p.T * p.H * p.W;
+    base = (which ? k : q) +
+           (((int64_t)b * N + ((int64_t)t * p.H + i * p.ph) * p.W + j * p.pw) * p.Hh + h) * (D / 8) +
+           sub;
+  } else {
+    base = (which ? k : q) + (((int64_t)b * p.Hh + h) * p.Npad + blk * p.block) * (D / 8) + sub;
+  }
+  constexpr bool use_max = MAXP;
   double acc[8];
 #pragma unroll
   for (int e = 0; e < 8; ++e) acc[e] = use_max ? -INFINITY : 0.0;
-  for (int a = 0; a < hn; ++a) {
-    const uint4* rowp = src + (int64_t)a * W * row_step;
-    for (int c0 = 0; c0 < wn; c0 += kAhead) {
+  float mabs = 0.f;
+  int cnt = 0;
+  // rows [0, len) from `rowp`, in order, four loads ahead of the additions
+  auto run = [&](const uint4* rowp, int len) {
+    for (int c0 = 0; c0 < len; c0 += kAhead) {
       uint4 v[kAhead];
 #pragma unroll
       for (int u = 0; u < kAhead; ++u)
-        if (c0 + u < wn) v[u] = __ldg(rowp + (int64_t)(c0 + u) * row_step);
+        if (c0 + u < len) v[u] = __ldg(rowp + (int64_t)(c0 + u) * row_step);
 #pragma unroll
       for (int u = 0; u < kAhead; ++u) {
-        if (c0 + u >= wn) break;
+        if (c0 + u >= len) break;
         const __nv_bfloat162* pv = reinterpret_cast<const __nv_bfloat162*>(&v[u]);
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
@@ -141,266 +117,57 @@ __global__ void __launch_bounds__(kPoolThreads)
             acc[2 * e] = __dadd_rn(acc[2 * e], (double)f.x);
             acc[2 * e + 1] = __dadd_rn(acc[2 * e + 1], (double)f.y);
           }
+          if (AMAX) mabs = fmaxf(mabs, fmaxf(fabsf(f.x), fabsf(f.y)));
         }
       }
     }
-  }
-  const int cnt = max(hn, 0) * max(wn, 0);
-  double* dst = ws + ((int64_t)which * groups_per_tensor + ((int64_t)b * Hh + h) * nblocks + blk) * D +
-                sub * 8;
-  const double dc = (double)cnt;
-#pragma unroll
-  for (int e = 0; e < 8; ++e) dst[e] = cnt ? (use_max ? acc[e] : __ddiv_rn(acc[e], dc)) : 0.0;
-}
-
-// ---------------------------------------------------------------------------
-// Pooling fed by TMA (tiles of up to 256 tokens): a persistent CTA per SM.
-// Warp 0 streams units - (Q or K, tile, batch, head, 64-channel chunk) - into
-// a ring of shared-memory stages with one tensor-map load each; warps 1..4
-// take the units in turn, each lane summing two channels over the tile's
-// tokens in row-major order straight out of shared memory.  The deep ring
-// keeps many loads in flight per SM without holding them in registers, so
-// the pass runs at the memory's rate at any number of heads.
-//   natural layout: 5-D map {D, Hh, W, H, B*T}, box {64, 1, pw, ph, 1} (one
-//     pooling tile of one head; parts past the grid read as zero and are
-//     skipped);
-//   slot layout: 2-D map {D, B*Hh*Npad}, box {64, block} (one block; empty
-//     slots skipped by the plan's validity bits).
-// Optionally records max |x| per (Q or K, batch, head) for the e4m3 scales.
-// ---------------------------------------------------------------------------
-constexpr int kPoolTmaConsumers = 4;
-constexpr int kPoolTmaThreads = 32 * (1 + kPoolTmaConsumers);
-constexpr int kPoolTmaMaxStages = 8;
-constexpr int kPoolTmaSmemBudget = 160 * 1024;
-
-struct PoolTmaParams {
-  int B, Hh, T, H, W, ph, pw, TH, TW;
-  int64_t nblocks, Npad;
-  int rows;          // box rows: pw * ph (natural) or the block size (slots)
-  int nchunk;        // D / 64
-  int stages;
-  int64_t units;     // 2 * nblocks * B * Hh * nchunk
-  int use_max;
-  const uint32_t* tile_valid;
-  uint32_t* amax;    // [3][B][Hh] float bits, or null
-  double* ws;
-  unsigned int* status;
-  uint64_t wait_limit_ns;
-};
-
-template <int D, bool NAT>
-__global__ void __launch_bounds__(kPoolTmaThreads, 1)
-    draft_pool_tma_kernel(const __grid_constant__ CUtensorMap tmq,
-                          const __grid_constant__ CUtensorMap tmk, const PoolTmaParams p) {
-  extern __shared__ uint8_t pool_smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(pool_smem_raw) + 127) &
-                                             ~uintptr_t(127));
-  const int stage_bytes = p.rows * 128;
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + (size_t)p.stages * stage_bytes);
-  uint64_t* empty = full + kPoolTmaMaxStages;
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(empty + kPoolTmaMaxStages);
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  if (threadIdx.x == 0) {
-    for (int i = 0; i < p.stages; ++i) {
-      mbar_init(&full[i], 1);
-      mbar_init(&empty[i], 1);
-    }
-    *abort_flag = (*reinterpret_cast<volatile unsigned int*>(p.status) & kStatusTimeout) ? 1 : 0;
-    fence_mbar_init();
-    prefetch_tmap(&tmq);
-    prefetch_tmap(&tmk);
-  }
-  __syncthreads();
-  if (*abort_flag) return;
-  const WaitCtx wc{p.status, abort_flag, p.wait_limit_ns};
-  const int64_t per_which = p.units / 2;
-  const int64_t nbh = (int64_t)p.B * p.Hh;
-
-  if (warp == 0) {
-    // ------------------------------------------------------------ producer
-    int64_t k = 0, issued = 0;
-    for (int64_t u = blockIdx.x; u < p.units; u += gridDim.x, ++k) {
-      const int st = (int)(k % p.stages);
-      const uint32_t par = (uint32_t)((k / p.stages) & 1) ^ 1u;
-      if (!__all_sync(kFullMaskScore, bounded_wait(&empty[st], par, wc))) break;
-      const int which = u >= per_which;
-      const int64_t r = u - which * per_which;
-      const int chunk = (int)(r % p.nchunk);
-      const int64_t r2 = r / p.nchunk;
-      if (elect_one()) {
-        const CUtensorMap* m = which ? &tmk : &tmq;
-        mbar_arrive_expect_tx(&full[st], (uint32_t)stage_bytes);
-        uint8_t* dst = smem + (size_t)st * stage_bytes;
-        if (NAT) {
-          // r2 = (blk * B + b) * Hh + h
-          const int h = (int)(r2 % p.Hh);
-          const int64_t r3 = r2 / p.Hh;
-          const int b = (int)(r3 % p.B);
-          const int64_t blk = r3 / p.B;
-          const int t = (int)(blk / ((int64_t)p.TH * p.TW));
-          const int rr = (int)(blk - (int64_t)t * p.TH * p.TW);
-          const int i = rr / p.TW, j = rr - (rr / p.TW) * p.TW;
-          tma_load_5d(dst, m, &full[st], chunk * 64, h, j * p.pw, i * p.ph, b * p.T + t);
-        } else {
-          // r2 = (b * Hh + h) * nblocks + blk
-          const int64_t bh = r2 / p.nblocks, blk = r2 - bh * p.nblocks;
-          tma_load_2d(dst, m, &full[st], chunk * 64, (int)(bh * p.Npad + blk * p.rows));
-        }
-      }
-      __syncwarp();
-      issued = k + 1;
-    }
-    if (*wc.abort) {
-      // leave no copy in flight: wait (bounded, ignoring the abort flag) for
-      // the loads still owned by the ring
-      volatile int no_abort = 0;
-      const WaitCtx drain{p.status, &no_abort, p.wait_limit_ns};
-      for (int64_t q = std::max<int64_t>(0, issued - p.stages); q < issued; ++q)
-        bounded_wait(&full[q % p.stages], (uint32_t)((q / p.stages) & 1), drain);
-    }
-    return;
-  }
-  // -------------------------------------------------------------- consumers
-  const int cw = warp - 1;
-  int64_t k = cw;
-  for (int64_t u = blockIdx.x + (int64_t)cw * gridDim.x; u < p.units;
-       u += (int64_t)kPoolTmaConsumers * gridDim.x, k += kPoolTmaConsumers) {
-    const int st = (int)(k % p.stages);
-    if (!__all_sync(kFullMaskScore, bounded_wait(&full[st], (uint32_t)((k / p.stages) & 1), wc)))
-      return;
-    const int which = u >= per_which;
-    const int64_t r = u - which * per_which;
-    const int chunk = (int)(r % p.nchunk);
-    const int64_t r2 = r / p.nchunk;
-    int b, h;
-    int64_t blk;
-    int hn, wn;
+    cnt += len;
+  };
+  if (live) {
     if (NAT) {
-      h = (int)(r2 % p.Hh);
-      const int64_t r3 = r2 / p.Hh;
-      b = (int)(r3 % p.B);
-      blk = r3 / p.B;
-      const int rr = (int)(blk % ((int64_t)p.TH * p.TW));
-      const int i = rr / p.TW, j = rr - (rr / p.TW) * p.TW;
-      hn = min(p.ph, p.H - i * p.ph);
-      wn = min(p.pw, p.W - j * p.pw);
+      const int r = (int)(blk % ((int64_t)p.TH * p.TW));
+      const int i = r / p.TW, j = r - (r / p.TW) * p.TW;
+      const int hn = min(p.ph, p.H - i * p.ph), wn = min(p.pw, p.W - j * p.pw);
+      for (int a = 0; a < hn; ++a) run(base + (int64_t)a * p.W * row_step, wn);
     } else {
-      const int64_t bh = r2 / p.nblocks;
-      blk = r2 - bh * p.nblocks;
-      b = (int)(bh / p.Hh);
-      h = (int)(bh - (int64_t)b * p.Hh);
-      hn = 1;
-      wn = p.rows;
-    }
-    const uint32_t* src = reinterpret_cast<const uint32_t*>(smem + (size_t)st * stage_bytes) + lane;
-    const bool use_max = p.use_max != 0;
-    double a0 = use_max ? -INFINITY : 0.0, a1 = a0;
-    float mabs = 0.f;
-    int cnt = 0;
-    const int64_t s0 = blk * p.rows;  // first slot (slot layout)
-    for (int a = 0; a < hn; ++a) {
-      for (int c = 0; c < wn; ++c) {
-        const int e = a * p.pw * (NAT ? 1 : 0) + c;
-        if (!NAT) {
-          const int64_t sl = s0 + c;
-          if (!((__ldg(p.tile_valid + (sl >> 5)) >> (sl & 31)) & 1u)) continue;
+      // runs of consecutive non-empty slots, 32 validity bits at a time
+      const int64_t s0 = blk * p.block;
+      for (int w0 = 0; w0 < p.block; w0 += 32) {
+        const int64_t sl = s0 + w0;
+        const int nb = min(32, p.block - w0);
+        const int sh = (int)(sl & 31);
+        uint32_t bits = __ldg(p.tile_valid + (sl >> 5)) >> sh;
+        if (sh + nb > 32) bits |= __ldg(p.tile_valid + (sl >> 5) + 1) << (32 - sh);
+        if (nb < 32) bits &= (1u << nb) - 1u;
+        while (bits) {
+          const int lo = __ffs(bits) - 1;
+          const uint32_t rest_bits = ~(bits >> lo);
+          const int len = rest_bits ? __ffs(rest_bits) - 1 : 32 - lo;
+          run(base + (int64_t)(w0 + lo) * row_step, len);
+          bits = (lo + len >= 32) ? 0u : bits & (~0u << (lo + len));
         }
-        const uint32_t v = src[e * 32];
-        const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&v));
-        if (use_max) {
-          a0 = fmax(a0, (double)f.x);
-          a1 = fmax(a1, (double)f.y);
-        } else {
-          a0 = __dadd_rn(a0, (double)f.x);
-          a1 = __dadd_rn(a1, (double)f.y);
-        }
-        mabs = fmaxf(mabs, fmaxf(fabsf(f.x), fabsf(f.y)));
-        ++cnt;
       }
     }
-    __syncwarp();
-    if (lane == 0) mbar_arrive(&empty[st]);
+    double* dst = p.ws + ((int64_t)which * p.groups_per_tensor +
+                          ((int64_t)b * p.Hh + h) * p.nblocks + blk) * D + sub * 8;
     const double dc = (double)cnt;
-    double2 out;
-    out.x = cnt ? (use_max ? a0 : __ddiv_rn(a0, dc)) : 0.0;
-    out.y = cnt ? (use_max ? a1 : __ddiv_rn(a1, dc)) : 0.0;
-    const int64_t gidx = (int64_t)which * nbh * p.nblocks + ((int64_t)b * p.Hh + h) * p.nblocks + blk;
-    reinterpret_cast<double2*>(p.ws + gidx * D + chunk * 64)[lane] = out;
-    if (p.amax) {
 #pragma unroll
-      for (int o = 16; o > 0; o >>= 1) mabs = fmaxf(mabs, __shfl_xor_sync(kFullMaskScore, mabs, o));
-      if (lane == 0) atomicMax(p.amax + ((int64_t)which * p.B + b) * p.Hh + h, __float_as_uint(mabs));
-    }
+    for (int e = 0; e < 8; ++e) dst[e] = cnt ? (use_max ? acc[e] : __ddiv_rn(acc[e], dc)) : 0.0;
   }
-}
-
-PFN_cuTensorMapEncodeTiled_v12000 pool_encode_fn() {
-  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-  if (!fn) {
-    void* ptr = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
-            cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+  if (AMAX) {
+    // max |x| of the group's tile: lanes of a group are kTPG consecutive lanes
+#pragma unroll
+    for (int o = kTPG / 2; o > 0; o >>= 1)
+      mabs = fmaxf(mabs, __shfl_xor_sync(kFullMaskScore, mabs, o));
+    if (live && sub == 0)
+      atomicMax(p.amax + ((int64_t)which * p.B + b) * p.Hh + h, __float_as_uint(mabs));
   }
-  return fn;
-}
-
-// Unswizzled maps with 64-channel boxes: one pooling tile of one head
-// (natural layout) or one block of slots.
-bool make_pool_tmap(CUtensorMap* m, const void* ptr, const Geometry& g, bool natural) {
-  auto fn = pool_encode_fn();
-  if (!fn) return false;
-  cuuint32_t estr[5] = {1, 1, 1, 1, 1};
-  if (natural) {
-    const cuuint64_t row = (cuuint64_t)g.Hh * g.D * 2;
-    cuuint64_t dims[5] = {(cuuint64_t)g.D, (cuuint64_t)g.Hh, (cuuint64_t)g.W, (cuuint64_t)g.H,
-                          (cuuint64_t)g.B * g.T};
-    cuuint64_t strides[4] = {(cuuint64_t)g.D * 2, row, row * g.W, row * g.W * g.H};
-    cuuint32_t box[5] = {64, 1, (cuuint32_t)g.pw, (cuuint32_t)g.ph, 1};
-    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, const_cast<void*>(ptr), dims, strides, box,
-              estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
-              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-  }
-  cuuint64_t dims[2] = {(cuuint64_t)g.D, (cuuint64_t)g.B * g.Hh * g.Npad};
-  cuuint64_t strides[1] = {(cuuint64_t)g.D * 2};
-  cuuint32_t box[2] = {64, (cuuint32_t)g.block};
-  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides, box, estr,
-            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
-            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
-int sm_count() {
-  static int n[64] = {};
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
-  if (!n[dev]) {
-    int v = 0;
-    n[dev] = cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess && v > 0
-                 ? v
-                 : 148;
-  }
-  return n[dev];
-}
-
-// TMA pooling applies when a unit (box) is at most 256 token rows and the
-// 5-D / 2-D maps can address the tensors.
-bool pool_tma_applies(const Geometry& g, bool natural) {
-  const int rows = natural ? g.ph * g.pw : g.block;
-  if (rows < 1 || rows > 256 || (g.D % 64) != 0) return false;
-  if (natural) return g.pw <= 256 && g.ph <= 256;
-  return (int64_t)g.B * g.Hh * g.Npad < (1ll << 31);
 }
 
 template <int D>
-cudaError_t launch_pool_tma(const Geometry& g, const uint32_t* tile_valid, const void* q,
-                            const void* k, int use_max, bool natural, double* ws, uint32_t* amax,
-                            unsigned int* status, uint64_t wait_limit_ns, cudaStream_t st) {
-  CUtensorMap tq, tk;
-  if (!make_pool_tmap(&tq, q, g, natural) || !make_pool_tmap(&tk, k, g, natural))
-    return cudaErrorInvalidValue;
-  PoolTmaParams p;
+cudaError_t launch_pool(const Geometry& g, const uint32_t* tile_valid, const void* q, const void* k,
+                        int use_max, bool natural, double* ws, uint32_t* amax, cudaStream_t st) {
+  PoolParams p;
   p.B = g.B;
   p.Hh = g.Hh;
   p.T = g.T;
@@ -410,25 +177,26 @@ cudaError_t launch_pool_tma(const Geometry& g, const uint32_t* tile_valid, const
   p.pw = g.pw;
   p.TH = g.TH;
   p.TW = g.TW;
+  p.block = g.block;
   p.nblocks = g.nblocks;
   p.Npad = g.Npad;
-  p.rows = natural ? g.ph * g.pw : g.block;
-  p.nchunk = D / 64;
-  const int stage_bytes = p.rows * 128;
-  p.stages = std::max(2, std::min(kPoolTmaMaxStages, kPoolTmaSmemBudget / stage_bytes));
-  p.units = 2 * g.nblocks * g.B * g.Hh * p.nchunk;
+  p.groups_per_tensor = (int64_t)g.B * g.Hh * g.nblocks;
   p.use_max = use_max;
   p.tile_valid = tile_valid;
   p.amax = amax;
   p.ws = ws;
-  p.status = status;
-  p.wait_limit_ns = wait_limit_ns;
-  const size_t smem = 128 + (size_t)p.stages * stage_bytes + 2 * kPoolTmaMaxStages * 8 + 16;
-  auto kern = natural ? draft_pool_tma_kernel<D, true> : draft_pool_tma_kernel<D, false>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-  if (e != cudaSuccess) return e;
-  const int64_t grid = std::min<int64_t>(p.units, sm_count());
-  kern<<<(unsigned)grid, kPoolTmaThreads, smem, st>>>(tq, tk, p);
+  const int64_t threads = 2 * p.groups_per_tensor * (D / 8);
+  const unsigned grid = (unsigned)((threads + kPoolThreads - 1) / kPoolThreads);
+  auto qq = reinterpret_cast<const uint4*>(q);
+  auto kk = reinterpret_cast<const uint4*>(k);
+  auto pick = [&](auto nat) {
+    constexpr bool NAT = decltype(nat)::value;
+    if (use_max)
+      return amax ? draft_pool_kernel<D, NAT, true, true> : draft_pool_kernel<D, NAT, true, false>;
+    return amax ? draft_pool_kernel<D, NAT, false, true> : draft_pool_kernel<D, NAT, false, false>;
+  };
+  auto kern = natural ? pick(std::true_type{}) : pick(std::false_type{});
+  kern<<<grid, kPoolThreads, 0, st>>>(qq, kk, p);
   return cudaGetLastError();
 }
 
@@ -622,18 +390,24 @@ __global__ void __launch_bounds__(kScoreThreads)
 // A warp owns R whole query-block rows; lane l accumulates the logits of key
 // blocks j = l + 32u (u < U) of each row, so a row's top-k runs straight out
 // of registers and no logit ever goes to shared memory.  The CTA's 8 warps
-// share the pooled keys, staged CK channels at a time (transposed to
-// [channel][key], so a lane's loads are conflict-free) in a two-stage
-// cp.async ring; the pooled query values are broadcast reads.  Every logit
+// share the pooled keys, staged CK channels at a time in a two-stage cp.async
+// ring, as [channel pair][key][2] (16-byte copies that land side by side; a
+// lane reads one key's two channels at once); the pooled query values are
+// broadcast reads.  Every logit
 // is still the sequential multiply-then-add chain over c = 0..D-1, each
 // operation rounded: only the loop order around the chains changes.
 // ---------------------------------------------------------------------------
-constexpr int kRegScoreWarps = 8;
+constexpr int kRegScoreWarps = 4;
 constexpr int kRegScoreCK = 8;  // channels per stage
 
 __device__ __forceinline__ void cp_async8(void* dst, const void* src, bool valid) {
   asm volatile("cp.async.ca.shared.global [%0], [%1], 8, %2;" ::"r"(smem_u32(dst)), "l"(src),
                "r"(valid ? 8 : 0)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async16(void* dst, const void* src, bool valid) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(dst)), "l"(src),
+               "r"(valid ? 16 : 0)
                : "memory");
 }
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
@@ -654,7 +428,7 @@ struct RegScoreCfg {
 
 // grid: (ceil(nblocks / kRows), Hh, B)
 template <int D, int U>
-__global__ void __launch_bounds__(32 * kRegScoreWarps, 2)
+__global__ void __launch_bounds__(32 * kRegScoreWarps, 3)
     draft_score_reg_kernel(const double* __restrict__ qbar, const double* __restrict__ kbar,
                            int Hh, int nblocks, int keep, int32_t* __restrict__ row_ptr,
                            int32_t* __restrict__ kv_idx, float* __restrict__ draft_map) {
@@ -662,7 +436,7 @@ __global__ void __launch_bounds__(32 * kRegScoreWarps, 2)
   constexpr int R = Cfg::R, CK = kRegScoreCK, NK = Cfg::NK;
   constexpr int kThreads = 32 * kRegScoreWarps;
   extern __shared__ double shd[];
-  double* sK = shd;                   // [2][CK][NK]
+  double* sK = shd;                   // [2][CK/2][NK][2]
   double* sQ = shd + 2 * Cfg::kStageK;  // [2][CK][kRows]
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int h = blockIdx.y, b = blockIdx.z;
@@ -676,10 +450,10 @@ __global__ void __launch_bounds__(32 * kRegScoreWarps, 2)
   // passed: the copy reads 0 bytes from it)
   auto issue = [&](int st, int c0) {
     double* dk = sK + st * Cfg::kStageK;
-    for (int i = threadIdx.x; i < Cfg::kStageK; i += kThreads) {
-      const int j = i / CK, c = i - j * CK;
+    for (int i = threadIdx.x; i < Cfg::kStageK / 2; i += kThreads) {
+      const int c2 = i / NK, j = i - c2 * NK;
       const bool ok = j < nblocks;
-      cp_async8(dk + c * NK + j, kb + (int64_t)(ok ? j : 0) * D + c0 + c, ok);
+      cp_async16(dk + 2 * i, kb + (int64_t)(ok ? j : 0) * D + c0 + 2 * c2, ok);
     }
     double* dq = sQ + st * Cfg::kStageQ;
     for (int i = threadIdx.x; i < Cfg::kStageQ; i += kThreads) {
@@ -706,18 +480,23 @@ __global__ void __launch_bounds__(32 * kRegScoreWarps, 2)
       cp_async_wait<0>();
     }
     __syncthreads();
-    const double* ck = sK + (cs & 1) * Cfg::kStageK + lane;
+    const double2* ck = reinterpret_cast<const double2*>(sK + (cs & 1) * Cfg::kStageK) + lane;
     const double* cq = sQ + (cs & 1) * Cfg::kStageQ + warp * R;
 #pragma unroll
-    for (int c = 0; c < CK; ++c) {
-      double qv[R];
+    for (int c2 = 0; c2 < CK / 2; ++c2) {
+      double q0[R], q1[R];
 #pragma unroll
-      for (int r = 0; r < R; ++r) qv[r] = cq[c * Cfg::kRows + r];
+      for (int r = 0; r < R; ++r) {
+        q0[r] = cq[(2 * c2) * Cfg::kRows + r];
+        q1[r] = cq[(2 * c2 + 1) * Cfg::kRows + r];
+      }
 #pragma unroll
       for (int u = 0; u < U; ++u) {
-        const double kv = ck[c * NK + 32 * u];
+        const double2 kv = ck[c2 * NK + 32 * u];  // channels 2*c2 and 2*c2 + 1 of key lane + 32u
 #pragma unroll
-        for (int r = 0; r < R; ++r) acc[r][u] = __dadd_rn(acc[r][u], __dmul_rn(qv[r], kv));
+        for (int r = 0; r < R; ++r) acc[r][u] = __dadd_rn(acc[r][u], __dmul_rn(q0[r], kv.x));
+#pragma unroll
+        for (int r = 0; r < R; ++r) acc[r][u] = __dadd_rn(acc[r][u], __dmul_rn(q1[r], kv.y));
       }
     }
     __syncthreads();  // the next issue() overwrites this stage
@@ -819,26 +598,10 @@ cudaError_t launch_t(const Geometry& g, const uint32_t* tile_valid, const void* 
                      int keep, int pooling, bool natural, int32_t* row_ptr, int32_t* kv_idx,
                      float* draft_map, double* ws, unsigned int* status, uint64_t wait_limit_ns,
                      cudaStream_t st, uint32_t* amax, bool* amax_recorded) {
-  const int64_t groups = (int64_t)g.B * g.Hh * g.nblocks;
-  const int64_t threads = 2 * groups * (D / 8);
-  const unsigned pool_grid = (unsigned)((threads + kPoolThreads - 1) / kPoolThreads);
   const int use_max = pooling == BSA_POOL_MAX ? 1 : 0;
-  if (amax_recorded) *amax_recorded = false;
-  if (pool_tma_applies(g, natural)) {
-    cudaError_t e0 = launch_pool_tma<D>(g, tile_valid, q, k, use_max, natural, ws, amax, status,
-                                        wait_limit_ns, st);
-    if (e0 != cudaSuccess) return e0;
-    if (amax_recorded) *amax_recorded = amax != nullptr;
-  } else if (natural)
-    draft_pool_nat_kernel<D><<<pool_grid, kPoolThreads, 0, st>>>(
-        reinterpret_cast<const uint4*>(q), reinterpret_cast<const uint4*>(k), g.B, g.Hh, g.T, g.H,
-        g.W, g.ph, g.pw, g.TH, g.TW, g.nblocks, groups, use_max, ws);
-  else
-    draft_pool_kernel<D><<<pool_grid, kPoolThreads, 0, st>>>(
-        reinterpret_cast<const uint4*>(q), reinterpret_cast<const uint4*>(k), tile_valid, g.Hh,
-        g.Npad, g.nblocks, g.block, groups, use_max, ws);
-  cudaError_t e = cudaGetLastError();
+  cudaError_t e = launch_pool<D>(g, tile_valid, q, k, use_max, natural, ws, amax, st);
   if (e != cudaSuccess) return e;
+  if (amax_recorded) *amax_recorded = amax != nullptr;
   // rows of up to 512 key blocks: logits in registers
   if (g.nblocks <= 128) return launch_score_reg<D, 4>(g, ws, keep, row_ptr, kv_idx, draft_map, st);
   if (g.nblocks <= 256) return launch_score_reg<D, 8>(g, ws, keep, row_ptr, kv_idx, draft_map, st);
@@ -852,6 +615,7 @@ cudaError_t launch_t(const Geometry& g, const uint32_t* tile_valid, const void* 
   e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   const dim3 grid((unsigned)((g.nblocks + R - 1) / R), (unsigned)g.Hh, (unsigned)g.B);
+  const int64_t groups = (int64_t)g.B * g.Hh * g.nblocks;
   kern<<<grid, kScoreThreads, smem, st>>>(ws, ws + groups * D, g.Hh, (int)g.nblocks, R, keep,
                                           row_ptr, kv_idx, draft_map);
   return cudaGetLastError();
@@ -965,6 +729,8 @@ extern "C" bsa_status bsa_draft_mask_noalloc(bsa_plan_t plan, const void* q_slot
                          " bytes exceeds the 32 MiB static scratch of bsa_draft_mask_noalloc; "
                          "use bsa_draft_mask with a caller workspace");
   if (g.nblocks > 18000) return set_error(BSA_ERR_UNSUPPORTED, "draft mask supports up to 18000 blocks");
+  if ((int64_t)g.B * g.Hh * g.Npad >= (1ll << 31))
+    return set_error(BSA_ERR_UNSUPPORTED, "draft mask needs B*Hh*Npad < 2^31");
   const int keep = (int)((g.nblocks * (100 - sparsity_pct) + 99) / 100);
   if ((int64_t)g.B * g.Hh * g.nblocks * keep >= (1ll << 31))
     return set_error(BSA_ERR_UNSUPPORTED, "block list longer than 2^31 entries");

@@ -82,12 +82,18 @@ def test_draft_paths_batch_of_two():
     nat = att.fused(q, k, v)
     bsa.bsa_poll_status(att.plan)
     assert torch.equal(att.col_idx, kv_slots)
-    assert torch.equal(slots.view(torch.int16), nat.view(torch.int16))
     qn, kn, vn = (to_np64(x) for x in (q, k, v))
     kv = oracle.draft_blocks(qn, kn, w.T, w.H, w.W, w.draft_ph, w.draft_pw, w.draft_sparsity)
     nb = kv.shape[2]
     np.testing.assert_array_equal(att.col_idx.view(w.B, w.Hh, nb, -1).cpu().numpy(), kv)
-    _check(nat, _draft_ref(w, qn, kn, vn, kv))
+    ref = _draft_ref(w, qn, kn, vn, kv)
+    _check(nat, ref)
+    _check(slots, ref)
+    # batch 1 alone gives the same bits as inside the batch of two
+    one = DraftAttention(1, w.Hh, w.D, w.T, w.H, w.W, w.draft_ph, w.draft_pw, w.draft_sparsity)
+    nat1 = one.fused(q[1:].contiguous(), k[1:].contiguous(), v[1:].contiguous())
+    bsa.bsa_poll_status(one.plan)
+    assert torch.equal(nat1.view(torch.int16), nat[1:].view(torch.int16))
 
 
 def test_e4m3_path_batch_of_two():

@@ -71,10 +71,8 @@ def test_quantize_e4m3_bit_exact(over):
 @pytest.mark.parametrize("over", [dict(cid=5, Hh=4),
                                   dict(cid=2, T=3, H=13, W=37, Hh=3, field_grid=(3, 4, 7)),
                                   dict(cid=1, qk="iid", D=64),
-                                  # 16 x 32 tiles (512 tokens): pooled without TMA, so the
-                                  # maxima of Q and K come from the separate pass
-                                  dict(cid=2, T=2, H=32, W=64, Hh=2, draft_ph=16, draft_pw=32,
-                                       field_grid=(2, 4, 7))])
+                                  dict(cid=2, T=2, H=20, W=12, Hh=2, D=64, draft_ph=16,
+                                       draft_pw=8, field_grid=(2, 4, 7))])
 @pytest.mark.parametrize("pooling", [bsa.POOL_MEAN, bsa.POOL_MAX])
 def test_draft_mask_and_quantize_in_one_call_equal_the_two_calls(over, pooling):
     over = dict(over)
