@@ -903,6 +903,31 @@ AttnParams make_params(const bsa_plan_s& plan, const int32_t* row_ptr, const int
   return p;
 }
 
+
+
+// Natural layout [B, N, Hh, D] bf16 seen as 5-D {D, Hh, W, H, B*T}; boxes of
+// 64 channels x 1 head x pw x ph x 1 frame (one pooling tile, 128 rows of
+// 128 bytes), 128-byte swizzle.  Boxes reaching past W or H read zeros.
+bool make_tmap_tiles(CUtensorMap* m, const void* ptr, const Geometry& g, bool e4m3 = false,
+                     int box_w = 0, int box_h = 0) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  const cuuint64_t esz = e4m3 ? 1 : 2;
+  const cuuint64_t row = (cuuint64_t)g.Hh * g.D * esz;  // bytes per token
+  cuuint64_t dims[5] = {(cuuint64_t)g.D, (cuuint64_t)g.Hh, (cuuint64_t)g.W, (cuuint64_t)g.H,
+                        (cuuint64_t)g.B * g.T};
+  cuuint64_t strides[4] = {(cuuint64_t)g.D * esz, row, row * g.W, row * g.W * g.H};
+  cuuint32_t box[5] = {(cuuint32_t)(128 / esz), 1, (cuuint32_t)(box_w > 0 ? box_w : g.pw),
+                       (cuuint32_t)(box_h > 0 ? box_h : g.ph), 1};
+  cuuint32_t estr[5] = {1, 1, 1, 1, 1};
+  return fn(m, e4m3 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5,
+            const_cast<void*>(ptr), dims, strides, box,
+            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+}  // namespace
+
 // Edge kinds of a TILE plan's grid: right (kind 1, the last tile column when
 // pool_w does not divide W), bottom (2) and corner (3), sorted by size
 // (rows), largest first; their box width and height.
@@ -929,29 +954,6 @@ int edge_kinds(const Geometry& g, int kind[3], int rows[3], int bw[3], int bh[3]
       }
   return n;
 }
-
-// Natural layout [B, N, Hh, D] bf16 seen as 5-D {D, Hh, W, H, B*T}; boxes of
-// 64 channels x 1 head x pw x ph x 1 frame (one pooling tile, 128 rows of
-// 128 bytes), 128-byte swizzle.  Boxes reaching past W or H read zeros.
-bool make_tmap_tiles(CUtensorMap* m, const void* ptr, const Geometry& g, bool e4m3 = false,
-                     int box_w = 0, int box_h = 0) {
-  auto fn = encode_fn();
-  if (!fn) return false;
-  const cuuint64_t esz = e4m3 ? 1 : 2;
-  const cuuint64_t row = (cuuint64_t)g.Hh * g.D * esz;  // bytes per token
-  cuuint64_t dims[5] = {(cuuint64_t)g.D, (cuuint64_t)g.Hh, (cuuint64_t)g.W, (cuuint64_t)g.H,
-                        (cuuint64_t)g.B * g.T};
-  cuuint64_t strides[4] = {(cuuint64_t)g.D * esz, row, row * g.W, row * g.W * g.H};
-  cuuint32_t box[5] = {(cuuint32_t)(128 / esz), 1, (cuuint32_t)(box_w > 0 ? box_w : g.pw),
-                       (cuuint32_t)(box_h > 0 ? box_h : g.ph), 1};
-  cuuint32_t estr[5] = {1, 1, 1, 1, 1};
-  return fn(m, e4m3 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5,
-            const_cast<void*>(ptr), dims, strides, box,
-            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
-}  // namespace
 
 bsa_status launch_attn_fwd(const bsa_plan_s& plan, const void* q, const void* k, const void* v,
                            const int32_t* row_ptr, const int32_t* col_idx, int per_head,
@@ -980,43 +982,8 @@ bsa_status launch_attn_fwd_natural(const bsa_plan_s& plan, const void* q, const 
                                    const void* v, const int32_t* row_ptr, const int32_t* col_idx,
                                    int per_head, float scale, void* o, float* lse,
                                    cudaStream_t st) {
-  const Geometry& g = plan.g;
-  if (g.layout != BSA_LAYOUT_TILE || g.block != kTile)
-    return set_error(BSA_ERR_UNSUPPORTED,
-                     "natural-layout attention needs a TILE plan with pool_h * pool_w = 128");
-  if ((int64_t)g.B * g.T * g.P * g.Hh >= (1ll << 31))
-    return set_error(BSA_ERR_UNSUPPORTED, "B*N*Hh must be < 2^31");
-  if ((int64_t)g.B * g.T >= (1ll << 31)) return set_error(BSA_ERR_UNSUPPORTED, "B*T must be < 2^31");
-  CUtensorMap tq, tk, tv;
-  if (!make_tmap_tiles(&tq, q, g) || !make_tmap_tiles(&tk, k, g) || !make_tmap_tiles(&tv, v, g))
-    return set_error(BSA_ERR_CUDA, "cuTensorMapEncodeTiled (5-D) failed");
-  AttnParams p = make_params(plan, row_ptr, col_idx, per_head, scale, o, lse);
-  const dim3 grid((unsigned)g.ntiles, (unsigned)g.Hh, (unsigned)g.B);
-  // partial key tiles at the grid's edges are packed several to an MMA tile,
-  // each read with a box of its exact size
-  int kind[3] = {0, 0, 0}, rows[3] = {0, 0, 0}, bw[3] = {0, 0, 0}, bh[3] = {0, 0, 0};
-  const int nk = edge_kinds(g, kind, rows, bw, bh);
-  cudaError_t e;
-  if (nk > 0 && g.nblocks < 32768) {
-    EdgeMaps em;
-    memset(&em, 0, sizeof(em));
-    for (int i = 0; i < nk; ++i) {
-      p.pk_kind[i] = kind[i];
-      p.pk_rows[i] = rows[i];
-      p.pk_step[i] = (rows[i] + 7) / 8 * 8;
-      if (!make_tmap_tiles(&em.k[kind[i] - 1], k, g, false, bw[i], bh[i]) ||
-          !make_tmap_tiles(&em.v[kind[i] - 1], v, g, false, bw[i], bh[i]))
-        return set_error(BSA_ERR_CUDA, "cuTensorMapEncodeTiled (5-D edge boxes) failed");
-    }
-    p.pk_on = 1;
-    e = g.D == 128 ? launch_t<128, false, true, false, true>(tq, tk, tv, p, grid, st, &em)
-                   : launch_t<64, false, true, false, true>(tq, tk, tv, p, grid, st, &em);
-  } else {
-    e = g.D == 128 ? launch_t<128, false, true>(tq, tk, tv, p, grid, st)
-                   : launch_t<64, false, true>(tq, tk, tv, p, grid, st);
-  }
-  if (e != cudaSuccess) return cuda_error(e, "natural-layout attention launch");
-  return BSA_OK;
+  // bf16 tiles: the persistent kernel of attn_draft.cu
+  return launch_attn_draft(plan, q, k, v, row_ptr, col_idx, per_head, scale, o, lse, st);
 }
 
 bsa_status launch_attn_fwd_natural_e4m3(const bsa_plan_s& plan, const void* q8, const void* k8,

@@ -117,6 +117,13 @@ bsa_status launch_attn_fwd_natural(const bsa_plan_s& plan, const void* q, const 
                                    const void* v, const int32_t* row_ptr, const int32_t* col_idx,
                                    int per_head, float scale, void* o, float* lse,
                                    cudaStream_t st);
+// The same, persistent (one CTA per SM over all query tiles), bf16 tiles.
+bsa_status launch_attn_draft(const bsa_plan_s& plan, const void* q, const void* k, const void* v,
+                             const int32_t* row_ptr, const int32_t* col_idx, int per_head,
+                             float scale, void* o, float* lse, cudaStream_t st);
+// Partial-tile kinds at a TILE grid's right edge (1), bottom edge (2) and
+// corner (3), largest first, with their token rows and box width / height.
+int edge_kinds(const Geometry& g, int kind[3], int rows[3], int bw[3], int bh[3]);
 cudaError_t launch_selftest_timeout(unsigned int* status, uint64_t limit_ns, cudaStream_t st);
 
 // Size bookkeeping shared by the API and the draft kernels.
