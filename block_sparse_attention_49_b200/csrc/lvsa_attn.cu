@@ -36,6 +36,7 @@
 
 #include <algorithm>
 #include <cmath>
+#include <cstring>
 
 #include "attn_common.cuh"
 #include "bsa_internal.cuh"
@@ -50,7 +51,7 @@ constexpr int kThreads = 384;
 constexpr int kMaxRowFrames = 8;   // frames a 256-token query pair may touch
 constexpr int kMaxFrames = 4096;
 constexpr int kSetWords = kMaxFrames / 32;
-constexpr int kMaxTiles = 4096;    // key tiles per query pair
+constexpr int kMaxRuns = 1024;     // runs of consecutive frames in a query pair's union
 
 template <int D>
 struct LvsaCfg {
@@ -68,7 +69,7 @@ struct LvsaCfg {
   static constexpr int kNumBars = 1 + 4 * NS + 2 + 2 + 2 + 1;
   static constexpr int kOffMisc = kOffBar + kNumBars * 8;
   static constexpr int kOffTiles = kOffMisc + 16;
-  static constexpr int kOffSets = kOffTiles + kMaxTiles * 4;
+  static constexpr int kOffSets = kOffTiles + kMaxRuns * 12;  // run table: tok0, len, v0
   static constexpr int kBytes = kOffSets + (kMaxRowFrames + 1) * kSetWords * 4;
   static constexpr int kSmem = kBytes + 1024;
   static constexpr uint32_t kTmemCols = 512;
@@ -78,12 +79,19 @@ struct LvsaCfg {
 struct LvsaParams {
   int B, Hh, T, P, N, C, T_per, s_mod;  // T_per = 0: no anchors
   int alternate;                        // alternating window growth
+  int pack;                             // runs start on 8-row (1) or 128-row (0) boundaries
   FastDiv divP;
   float scale, scale_log2;
   __nv_bfloat16* o;  // natural layout
   float* lse;        // [B, Hh, N] or null
   unsigned int* status;
   uint64_t wait_limit_ns;
+};
+
+// Maps of the same tensors with boxes of 64, 32, 16 and 8 tokens (index 3..0):
+// the pieces of packed key tiles.
+struct RunMaps {
+  CUtensorMap k[4], v[4];
 };
 
 __device__ __forceinline__ int floordiv(int a, int b) {
@@ -162,7 +170,8 @@ __device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, u
 template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
     lvsa_attn_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmk,
-                     const __grid_constant__ CUtensorMap tmv, const LvsaParams p) {
+                     const __grid_constant__ CUtensorMap tmv, const LvsaParams p,
+                     const __grid_constant__ RunMaps rm) {
   using Cfg = LvsaCfg<D>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -179,7 +188,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* p_ready = p_half + 2;         // [2]: all of P stored
   uint64_t* o_final = p_ready + 2;
   uint32_t* misc = reinterpret_cast<uint32_t*>(smem + Cfg::kOffMisc);  // tmem, abort, ntiles, skip
-  int32_t* tiles = reinterpret_cast<int32_t*>(smem + Cfg::kOffTiles);  // (k0 << 7) | (count - 1)
+  // runs of consecutive frames of the union, laid end to end as a stream of
+  // key rows: run r = tokens [run_tok[r], + run_len[r]) at rows run_v[r]..
+  int32_t* run_tok = reinterpret_cast<int32_t*>(smem + Cfg::kOffTiles);
+  int32_t* run_len = run_tok + kMaxRuns;
+  int32_t* run_v = run_len + kMaxRuns;
   uint32_t* sets = reinterpret_cast<uint32_t*>(smem + Cfg::kOffSets);  // [rf][kSetWords], union last
   uint32_t* uset = sets + kMaxRowFrames * kSetWords;
 
@@ -217,6 +230,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     prefetch_tmap(&tmk);
     prefetch_tmap(&tmv);
   }
+  // packed key tiles leave rows between and after their pieces: masked, but
+  // P = 0 times a value must stay 0, so V stages start at zero
+  if (p.pack) {
+    for (int i = threadIdx.x; i < Cfg::NS * Cfg::kKVBytes / 16; i += kThreads)
+      reinterpret_cast<uint4*>(smem + Cfg::kOffV)[i] = make_uint4(0u, 0u, 0u, 0u);
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+  }
   __syncthreads();
   if (misc[3]) return;
   if (warp == 1) {
@@ -241,29 +261,42 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
   __syncthreads();
   if (threadIdx.x == 0) {
-    // key tiles: 128-token pieces of each run of consecutive frames of U
-    int cnt = 0;
+    // the runs of consecutive frames of U, end to end: a run starts on the
+    // next 8-row boundary after the previous one (the 128-byte swizzle
+    // atom) when frames are a multiple of 8 tokens, so the tail of one run
+    // shares its key tile with the head of the next; otherwise on the next
+    // 128-row boundary.  Key tile j = stream rows [128 j, 128 j + 128).
+    const int align = p.pack ? 8 : kTile;
+    int nr = 0, v = 0;
     bool overflow = false;
     for (int f = next_with(uset, 0, p.T, true); f < p.T;) {
       const int e = next_with(uset, f, p.T, false);  // run [f, e)
-      const int tok0 = f * p.P, tok1 = e * p.P;
-      for (int k = tok0; k < tok1; k += kTile) {
-        // first key token and number of this run's keys in the tile: the
-        // tile's overhang past the run is masked, so a key that also starts
-        // the next run is never counted twice
-        if (cnt < kMaxTiles) tiles[cnt++] = (k << 7) | (min(kTile, tok1 - k) - 1);
-        else overflow = true;
+      if (nr < kMaxRuns) {
+        run_tok[nr] = f * p.P;
+        run_len[nr] = (e - f) * p.P;
+        run_v[nr] = v;
+        v = (v + (e - f) * p.P + align - 1) / align * align;
+        ++nr;
+      } else {
+        overflow = true;
       }
       f = next_with(uset, e, p.T, true);
     }
     if (overflow) atomicOr(p.status, kStatusBadBlocklist);
-    misc[2] = cnt;
+    misc[2] = (v + kTile - 1) / kTile;
+    misc[3] = nr;
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tbase = misc[0];
   const int n = (int)misc[2];
+  const int nruns = (int)misc[3];
+  // pieces of key tile j: [row offset, first token, length] of each run it
+  // meets, walked with a cursor (tiles are visited in order)
+  auto first_run = [&](int j, int& r) {
+    while (r < nruns && run_v[r] + run_len[r] <= j * kTile) ++r;
+  };
 
   // register split: 128 threads x 72 + 256 threads x 216 = 64512, the 384 x
   // 168 registers the block is launched with (fewer for the issuing warps
@@ -282,26 +315,52 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       __syncwarp();
       int issued_k = 0, issued_v = 0;
+      int rcur = 0;
+      // one key tile into `dst`: a 128-token box at the tile's first token
+      // (128-row runs), or each run's piece with boxes of 128/64/32/16/8
+      // tokens at its row offset (packed runs, pieces of multiples of 8)
+      auto load_tile = [&](int j, int r0, uint8_t* dst, uint64_t* bar, const CUtensorMap* m128,
+                           const CUtensorMap* msmall) {
+        if (!p.pack) {
+          const int krow = (int)(brow + run_tok[r0] + (j * kTile - run_v[r0]));
+          mbar_arrive_expect_tx(bar, Cfg::kKVBytes);
+          for (int c = 0; c < Cfg::kChunks; ++c)
+            tma_load_3d(dst + c * Cfg::kPanel, m128, bar, c * 64, h, krow);
+          return;
+        }
+        uint32_t bytes = 0;
+        for (int r = r0; r < nruns && run_v[r] < (j + 1) * kTile; ++r) {
+          const int a = max(j * kTile, run_v[r]), e = min((j + 1) * kTile, run_v[r] + run_len[r]);
+          if (e > a) bytes += (uint32_t)(e - a) * 128u * Cfg::kChunks;
+        }
+        mbar_arrive_expect_tx(bar, bytes);
+        for (int r = r0; r < nruns && run_v[r] < (j + 1) * kTile; ++r) {
+          const int a = max(j * kTile, run_v[r]), e = min((j + 1) * kTile, run_v[r] + run_len[r]);
+          if (e <= a) continue;
+          int tok = run_tok[r] + (a - run_v[r]), row = a - j * kTile;
+          const int len8 = (e - a) >> 3;
+          for (int bsz = 4; bsz >= 0; --bsz) {
+            if (!((len8 >> bsz) & 1)) continue;
+            const CUtensorMap* m = bsz == 4 ? m128 : &msmall[bsz];
+            for (int c = 0; c < Cfg::kChunks; ++c)
+              tma_load_3d(dst + c * Cfg::kPanel + row * 128, m, bar, c * 64, h, (int)(brow + tok));
+            tok += 8 << bsz;
+            row += 8 << bsz;
+          }
+        }
+      };
       for (int j = 0; j < n; ++j) {
         const int st = j % Cfg::NS;
         const uint32_t par = ((j / Cfg::NS) & 1) ^ 1;
-        const int krow = (int)(brow + (tiles[j] >> 7));
+        first_run(j, rcur);
         if (!__all_sync(kFullMask, bounded_wait(&k_empty[st], par, wc))) break;
-        if (elect_one()) {
-          uint8_t* sK = smem + Cfg::kOffK + st * Cfg::kKVBytes;
-          mbar_arrive_expect_tx(&k_full[st], Cfg::kKVBytes);
-          for (int c = 0; c < Cfg::kChunks; ++c)
-            tma_load_3d(sK + c * Cfg::kPanel, &tmk, &k_full[st], c * 64, h, krow);
-        }
+        if (elect_one())
+          load_tile(j, rcur, smem + Cfg::kOffK + st * Cfg::kKVBytes, &k_full[st], &tmk, rm.k);
         __syncwarp();
         issued_k = j + 1;
         if (!__all_sync(kFullMask, bounded_wait(&v_empty[st], par, wc))) break;
-        if (elect_one()) {
-          uint8_t* sV = smem + Cfg::kOffV + st * Cfg::kKVBytes;
-          mbar_arrive_expect_tx(&v_full[st], Cfg::kKVBytes);
-          for (int c = 0; c < Cfg::kChunks; ++c)
-            tma_load_3d(sV + c * Cfg::kPanel, &tmv, &v_full[st], c * 64, h, krow);
-        }
+        if (elect_one())
+          load_tile(j, rcur, smem + Cfg::kOffV + st * Cfg::kKVBytes, &v_full[st], &tmv, rm.v);
         __syncwarp();
         issued_v = j + 1;
       }
@@ -417,19 +476,26 @@ __global__ void __launch_bounds__(kThreads, 1)
     const float thr = 8.0f / sl2;
     RowState st;
     bool alive = true;
+    int rcur = 0;
     for (int j = 0; j < n; ++j) {
-      // keys of tile j allowed for this row: those whose frame is in A(tq)
+      // keys of tile j allowed for this row: those whose frame is in A(tq);
+      // rows between and after the pieces stay masked
       uint32_t vm[4] = {0u, 0u, 0u, 0u};
+      first_run(j, rcur);
       if (qvalid) {
-        const int k0 = tiles[j] >> 7, kn = (tiles[j] & 127) + 1;  // keys [k0, k0 + kn)
-        int f = (int)p.divP.div((uint32_t)k0);
-        int lo = 0, fend = (f + 1) * p.P - k0;
-        while (lo < kn) {
-          const int hi = min(kn, fend);
-          if (f < p.T && bit_of(myset, f)) set_range(vm, lo, hi);
-          lo = hi;
-          ++f;
-          fend += p.P;
+        for (int r = rcur; r < nruns && run_v[r] < (j + 1) * kTile; ++r) {
+          const int a = max(j * kTile, run_v[r]), e = min((j + 1) * kTile, run_v[r] + run_len[r]);
+          if (e <= a) continue;
+          const int k0 = run_tok[r] + (a - run_v[r]), kn = e - a, o = a - j * kTile;
+          int f = (int)p.divP.div((uint32_t)k0);
+          int lo = 0, fend = (f + 1) * p.P - k0;
+          while (lo < kn) {
+            const int hi = min(kn, fend);
+            if (f < p.T && bit_of(myset, f)) set_range(vm, o + lo, o + hi);
+            lo = hi;
+            ++f;
+            fend += p.P;
+          }
         }
       }
       if (!__all_sync(kFullMask, bounded_wait(&s_full[g], j & 1, wc))) {
@@ -513,13 +579,15 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn3() {
   return fn;
 }
 
-// Natural layout [B*N, Hh, D] bf16: boxes of 64 channels x 1 head x 128 tokens.
-bool make_tmap_natural(CUtensorMap* m, const void* ptr, int64_t tokens, int Hh, int D) {
+// Natural layout [B*N, Hh, D] bf16: boxes of 64 channels x 1 head x `rows`
+// tokens.
+bool make_tmap_natural(CUtensorMap* m, const void* ptr, int64_t tokens, int Hh, int D,
+                       int rows = kTile) {
   auto fn = encode_fn3();
   if (!fn) return false;
   cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)Hh, (cuuint64_t)tokens};
   cuuint64_t strides[2] = {(cuuint64_t)D * 2, (cuuint64_t)Hh * D * 2};
-  cuuint32_t box[3] = {64, 1, (cuuint32_t)kTile};
+  cuuint32_t box[3] = {64, 1, (cuuint32_t)rows};
   cuuint32_t estr[3] = {1, 1, 1};
   return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims, strides, box,
             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -528,12 +596,12 @@ bool make_tmap_natural(CUtensorMap* m, const void* ptr, int64_t tokens, int Hh, 
 
 template <int D>
 cudaError_t launch_lvsa_t(const CUtensorMap& q, const CUtensorMap& k, const CUtensorMap& v,
-                          const LvsaParams& p, dim3 grid, cudaStream_t st) {
+                          const LvsaParams& p, const RunMaps& rm, dim3 grid, cudaStream_t st) {
   auto kern = lvsa_attn_kernel<D>;
   cudaError_t e =
       cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, LvsaCfg<D>::kSmem);
   if (e != cudaSuccess) return e;
-  kern<<<grid, kThreads, LvsaCfg<D>::kSmem, st>>>(q, k, v, p);
+  kern<<<grid, kThreads, LvsaCfg<D>::kSmem, st>>>(q, k, v, p, rm);
   return cudaGetLastError();
 }
 
@@ -567,10 +635,10 @@ extern "C" bsa_status bsa_lvsa_attn_fwd(bsa_plan_t plan, int C, int T_per, int s
   const int64_t N = (int64_t)g.T * g.P;
   if ((int64_t)g.B * N >= (1ll << 31)) return set_error(BSA_ERR_UNSUPPORTED, "B*N must be < 2^31");
   if (N >= (1 << 24)) return set_error(BSA_ERR_UNSUPPORTED, "fused LVSA attention needs N < 2^24");
-  // key tiles of a query pair: at most |U| frames, |U| <= min(T, rows' frames * C)
+  // runs of a query pair's union: at most |U| <= min(T, rows' frames * C)
   const int64_t u_frames = std::min<int64_t>(g.T, (int64_t)kMaxRowFrames * C);
-  if ((u_frames * g.P + kTile - 1) / kTile + u_frames > kMaxTiles)
-    return set_error(BSA_ERR_UNSUPPORTED, "fused LVSA attention: too many key tiles per query pair");
+  if (u_frames > kMaxRuns)
+    return set_error(BSA_ERR_UNSUPPORTED, "fused LVSA attention: too many frames per query pair");
   CUtensorMap tq, tk, tv;
   const int64_t tokens = (int64_t)g.B * N;
   if (!make_tmap_natural(&tq, q, tokens, g.Hh, g.D) || !make_tmap_natural(&tk, k, tokens, g.Hh, g.D) ||
@@ -586,6 +654,14 @@ extern "C" bsa_status bsa_lvsa_attn_fwd(bsa_plan_t plan, int C, int T_per, int s
   p.T_per = tp;
   p.s_mod = sm;
   p.alternate = plan->lvsa_window == BSA_WINDOW_ALTERNATE ? 1 : 0;
+  p.pack = (g.P % 8 == 0) ? 1 : 0;
+  RunMaps rm;
+  memset(&rm, 0, sizeof(rm));
+  if (p.pack)
+    for (int b = 0; b < 4; ++b)
+      if (!make_tmap_natural(&rm.k[b], k, tokens, g.Hh, g.D, 8 << b) ||
+          !make_tmap_natural(&rm.v[b], v, tokens, g.Hh, g.D, 8 << b))
+        return set_error(BSA_ERR_CUDA, "cuTensorMapEncodeTiled (3-D, small boxes) failed");
   p.divP = FastDiv((uint32_t)g.P);
   p.scale = scale;
   p.scale_log2 = scale * 1.4426950408889634f;
@@ -595,8 +671,8 @@ extern "C" bsa_status bsa_lvsa_attn_fwd(bsa_plan_t plan, int C, int T_per, int s
   p.wait_limit_ns = plan->wait_limit_ns;
   const dim3 grid((unsigned)((N + kPair - 1) / kPair), (unsigned)g.Hh, (unsigned)g.B);
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  const cudaError_t e = g.D == 128 ? launch_lvsa_t<128>(tq, tk, tv, p, grid, st)
-                                   : launch_lvsa_t<64>(tq, tk, tv, p, grid, st);
+  const cudaError_t e = g.D == 128 ? launch_lvsa_t<128>(tq, tk, tv, p, rm, grid, st)
+                                   : launch_lvsa_t<64>(tq, tk, tv, p, rm, grid, st);
   return e == cudaSuccess ? BSA_OK : cuda_error(e, "lvsa_attn launch");
 }
 

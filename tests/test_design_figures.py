@@ -9,12 +9,13 @@ attention kernels; they are not parity evidence.
 * The top-k favours partly empty edge blocks (57.5 % of the kept blocks
   against 43.8 % of all blocks): a kept key block is 65 % full on average,
   and 49.6 % of the executed attention work is attended.
-* The one-kernel LVSA tiling (256 queries per CTA; key tiles are the
-  128-token pieces of each run of consecutive frames of the union of the
-  CTA's frame sets) at the Wan-1.3B 6x workload: 96.0 % of the multiplied
-  pairs are attended at steps 0-5 and 96.4 % at steps 6-11; run tail tiles
-  take 3.4 and 3.0 points (11 and 10 anchors), CTAs straddling two frames
-  0.6.
+* The one-kernel LVSA tiling (256 queries per CTA; the runs of consecutive
+  frames of the union of the CTA's frame sets laid end to end at 8-row
+  boundaries and cut into 128-row key tiles) at the Wan-1.3B 6x workload:
+  99.3 % of the multiplied pairs are attended, CTAs straddling two frames
+  cost 0.6 points.  With each run starting on a whole key tile, the share
+  was 96.0 % at steps 0-5 and 96.4 % at steps 6-11 (run tail tiles 3.4 and
+  3.0 points with 11 and 10 anchors).
 * The two readings of the window's growth order (alternating pointers, the
   default, and distance order) differ on 5 of 32 rows of
   the tiny workload, 570 of 1512 at Wan-1.3B 6x and 3 of 1040 at
@@ -78,7 +79,11 @@ def test_top_k_favours_partly_empty_edge_blocks(draft_case):
     assert attended / (128 * 128 * kv.size) == pytest.approx(0.496, abs=0.002)
 
 
-def _lvsa_tiling(w, s):
+def _lvsa_tiling(w, s, pack=True):
+    """Multiplied and attended pairs of the one-kernel LVSA tiling: 256
+    queries per CTA; the runs of consecutive frames of the union of their
+    frame sets laid end to end, each starting on the next 8-row boundary
+    (pack) or on the next 128-row boundary, cut into 128-row key tiles."""
     T, P = w.T, w.H * w.W
     N = T * P
     A = [set(int(f) for f in r) for r in oracle.lvsa_frame_sets(T, w.lvsa_C, w.lvsa_T_per, s)]
@@ -92,7 +97,11 @@ def _lvsa_tiling(w, s):
                 runs[-1][1] = f
             else:
                 runs.append([f, f])
-        keys = sum(-(-((b - a + 1) * P) // 128) * 128 for a, b in runs)
+        align = 8 if pack else 128
+        v = 0
+        for a, b in runs:
+            v = -(-(v + (b - a + 1) * P) // align) * align
+        keys = -(-v // 128) * 128
         executed += 256 * keys
         attended += sum(len(A[n // P]) * P for n in rows)
         tails += 256 * (keys - len(U) * P)
@@ -100,18 +109,22 @@ def _lvsa_tiling(w, s):
     return attended / executed, tails / executed, straddle / executed
 
 
-def test_lvsa_one_kernel_tiling_attends_96_percent():
+def test_lvsa_one_kernel_tiling_attends_99_percent():
     w = CONFIGS[3]
-    early = [_lvsa_tiling(w, s) for s in (0, 5)]
-    late = [_lvsa_tiling(w, s) for s in (6, 11)]
-    for frac, tails, straddle in early:                 # 11 anchors
+    for s in (0, 5, 6, 11):
+        frac, tails, straddle = _lvsa_tiling(w, s)
+        assert frac == pytest.approx(0.993, abs=0.001)
+        assert tails == pytest.approx(0.0007, abs=0.0002)
+        assert straddle == pytest.approx(0.006, abs=0.001)
+    # runs starting on whole key tiles: each run's last tile is partly empty
+    early = [_lvsa_tiling(w, s, pack=False) for s in (0, 5)]   # 11 anchors
+    late = [_lvsa_tiling(w, s, pack=False) for s in (6, 11)]   # 10 anchors
+    for frac, tails, _ in early:
         assert frac == pytest.approx(0.960, abs=0.001)
         assert tails == pytest.approx(0.034, abs=0.001)
-    for frac, tails, straddle in late:                  # 10 anchors
+    for frac, tails, _ in late:
         assert frac == pytest.approx(0.964, abs=0.001)
         assert tails == pytest.approx(0.030, abs=0.001)
-    for frac, tails, straddle in early + late:
-        assert straddle == pytest.approx(0.006, abs=0.001)
 
 
 def test_the_two_window_readings_differ_on_the_stated_rows():
