@@ -959,6 +959,10 @@ bsa_status launch_attn_fwd(const bsa_plan_s& plan, const void* q, const void* k,
                            const int32_t* row_ptr, const int32_t* col_idx, int per_head,
                            float scale, void* o, float* lse, cudaStream_t st) {
   const Geometry& g = plan.g;
+  // one list for every (batch, head), 128-slot blocks: two query tiles per
+  // CTA share every key tile (attn_pair.cu)
+  if (attn_pair_applies(g, per_head))
+    return launch_attn_pair(plan, q, k, v, row_ptr, col_idx, scale, o, lse, st);
   const int64_t rows = (int64_t)g.B * g.Hh * g.Npad;
   if (rows >= (1ll << 31)) return set_error(BSA_ERR_UNSUPPORTED, "B*Hh*Npad must be < 2^31");
   const bool fine = g.block < kTile;

@@ -121,6 +121,12 @@ bsa_status launch_attn_fwd_natural(const bsa_plan_s& plan, const void* q, const 
 bsa_status launch_attn_draft(const bsa_plan_s& plan, const void* q, const void* k, const void* v,
                              const int32_t* row_ptr, const int32_t* col_idx, int per_head,
                              float scale, void* o, float* lse, cudaStream_t st);
+// Shared block lists (per_head = 0) with 128-slot blocks: two query tiles per
+// CTA over the union of their rows (attn_pair.cu).
+bool attn_pair_applies(const Geometry& g, int per_head);
+bsa_status launch_attn_pair(const bsa_plan_s& plan, const void* q, const void* k, const void* v,
+                            const int32_t* row_ptr, const int32_t* col_idx, float scale, void* o,
+                            float* lse, cudaStream_t st);
 // Partial-tile kinds at a TILE grid's right edge (1), bottom edge (2) and
 // corner (3), largest first, with their token rows and box width / height.
 int edge_kinds(const Geometry& g, int kind[3], int rows[3], int bw[3], int bh[3]);
