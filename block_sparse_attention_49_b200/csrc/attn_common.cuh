@@ -61,8 +61,9 @@ struct RowState {
 // row's reference max moves (it does only when the max grows by more than
 // `thr`, so P stays below 2^(thr*sl2)).  On a move st.m and st.l are updated
 // and *corr is the factor O must be multiplied by.  *ms2 receives the packed
-// pair (-m*sl2, -m*sl2) for softmax_exp.
-template <int NC>
+// pair (-m*sl2, -m*sl2) for softmax_exp.  MASK = false: the caller knows
+// every key is allowed, and the masking code is left out altogether.
+template <int NC, bool MASK = true>
 __device__ __forceinline__ bool softmax_max(float (&s)[NC], const uint32_t (&vm)[NC / 32],
                                             RowState& st, float sl2, float thr, float& corr,
                                             uint64_t& neg_ms2) {
@@ -70,7 +71,7 @@ __device__ __forceinline__ bool softmax_max(float (&s)[NC], const uint32_t (&vm)
   uint32_t all = kFullMask;
 #pragma unroll
   for (int w = 0; w < NC / 32; ++w) all &= vm[w];
-  if (all != kFullMask) {
+  if (MASK && all != kFullMask) {
 #pragma unroll
     for (int w = 0; w < NC / 32; ++w)
 #pragma unroll

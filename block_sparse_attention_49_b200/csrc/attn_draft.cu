@@ -48,6 +48,7 @@
 #include <cmath>
 #include <cstring>
 
+#include "attn_common.cuh"
 #include "bsa_internal.cuh"
 #include "ptx.cuh"
 
@@ -57,6 +58,7 @@ namespace {
 constexpr int kTile = 128;
 constexpr int kThreads = 384;
 constexpr int kListMax = 768;           // key-list entries a tile can pack
+constexpr int kMaxBins = 128;           // packed tiles of edge pieces a list can hold
 constexpr uint16_t kBad = 0xffffu;      // packed-list marker of an out-of-range entry
 constexpr uint32_t kAll = 0xffffffffu;
 
@@ -73,12 +75,18 @@ struct DraftCfg {
   static constexpr int kOffV = kOffK + NK * kTileBytes;
   static constexpr int kOffBar = kOffV + NV * kTileBytes;
   // q_full, q_empty, k_full[NK], k_empty[NK], v_full[NV], v_empty[NV],
-  // s_full[2], p_ready[2], o_final, o_free, list_full[2], list_empty[2]
-  static constexpr int kNumBars = 2 + 2 * NK + 2 * NV + 2 + 2 + 2 + 2 + 2;
+  // s_full[2], p_half[2], p_ready[2], o_final, o_free, list_full[2], list_empty[2]
+  static constexpr int kNumBars = 2 + 2 * NK + 2 * NV + 2 + 2 + 2 + 2 + 2 + 2;
   static constexpr int kOffMisc = kOffBar + kNumBars * 8;     // tmem, abort
-  static constexpr int kOffStats = kOffMisc + 16;             // [4][128] floats
-  static constexpr int kOffLists = kOffStats + 4 * kTile * 4;
-  static constexpr int kListBytes = kListMax * 2 + 32;        // entries + header
+  static constexpr int kOffStats = kOffMisc + 16;             // [2][4][128] floats
+  static constexpr int kOffLists = kOffStats + 2 * 4 * kTile * 4;
+  // a list buffer: bin row masks (uint4), bin piece counts (uint32), the
+  // entries (uint16), the header
+  static constexpr int kOffBinVm = 0;
+  static constexpr int kOffBinCnt = kMaxBins * 16;
+  static constexpr int kOffEnt = kOffBinCnt + kMaxBins * 4;
+  static constexpr int kOffHead = kOffEnt + kListMax * 2;
+  static constexpr int kListBytes = kOffHead + 32;
   static constexpr int kBytes = kOffLists + 2 * kListBytes;
   static constexpr int kSmem = kBytes + 1024;
   static_assert(kSmem <= 232448, "shared memory budget");
@@ -135,11 +143,6 @@ __device__ __forceinline__ void next_bin(const DraftParams& p, int (&r)[3], int 
   }
 }
 
-__device__ __forceinline__ uint32_t pack_bf16x2_d(float lo, float hi) {
-  __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
-  return *reinterpret_cast<uint32_t*>(&v);
-}
-
 __device__ __forceinline__ void softmax_sync() { asm volatile("bar.sync 1, 256;" ::: "memory"); }
 __device__ __forceinline__ void end_sync() { asm volatile("bar.sync 2, 384;" ::: "memory"); }
 
@@ -161,18 +164,25 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* v_full = k_empty + Cfg::NK;
   uint64_t* v_empty = v_full + Cfg::NV;
   uint64_t* s_full = v_empty + Cfg::NV;   // [2]
-  uint64_t* p_ready = s_full + 2;         // [2]
+  uint64_t* p_half = s_full + 2;          // [2]: keys 0..63 of P stored
+  uint64_t* p_ready = p_half + 2;         // [2]: all of P stored
   uint64_t* o_final = p_ready + 2;
   uint64_t* o_free = o_final + 1;
   uint64_t* list_full = o_free + 1;       // [2]
   uint64_t* list_empty = list_full + 2;   // [2]
   uint32_t* misc = reinterpret_cast<uint32_t*>(smem + Cfg::kOffMisc);  // tmem, abort, skip
   float* stats = reinterpret_cast<float*>(smem + Cfg::kOffStats);
+  auto list_base = [&](int buf) { return smem + Cfg::kOffLists + buf * Cfg::kListBytes; };
   auto list_entries = [&](int buf) {
-    return reinterpret_cast<uint16_t*>(smem + Cfg::kOffLists + buf * Cfg::kListBytes);
+    return reinterpret_cast<uint16_t*>(list_base(buf) + Cfg::kOffEnt);
   };
   auto list_head = [&](int buf) {
-    return reinterpret_cast<ListHead*>(smem + Cfg::kOffLists + buf * Cfg::kListBytes + kListMax * 2);
+    return reinterpret_cast<ListHead*>(list_base(buf) + Cfg::kOffHead);
+  };
+  // bin b of a packed list: its row mask and its pieces per kind (one byte each)
+  auto bin_vm = [&](int buf) { return reinterpret_cast<uint4*>(list_base(buf) + Cfg::kOffBinVm); };
+  auto bin_cnt = [&](int buf) {
+    return reinterpret_cast<uint32_t*>(list_base(buf) + Cfg::kOffBinCnt);
   };
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -211,6 +221,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     mbar_init(&s_full[0], 1);
     mbar_init(&s_full[1], 1);
+    mbar_init(&p_half[0], 128);
+    mbar_init(&p_half[1], 128);
     mbar_init(&p_ready[0], 128);
     mbar_init(&p_ready[1], 128);
     mbar_init(o_final, 1);
@@ -272,7 +284,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         ListHead* hd = list_head(buf);
         uint16_t* ent = list_entries(buf);
-        const bool packed = p.pk_on && n > 0 && n <= kListMax;
+        bool packed = p.pk_on && n > 0 && n <= kListMax;
         int cF = 0, ce[3] = {0, 0, 0};
         if (packed) {
           // counting sort by kind: full tiles first (list order), then the
@@ -319,13 +331,34 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         int npk = n;
         if (packed) {
+          // the bins of edge pieces, each with its row mask, computed once here
+          // for the producers and the softmax groups
           int rr[3] = {ce[0], ce[1], ce[2]}, a[3];
           int nb = 0;
-          while (rr[0] + rr[1] + rr[2] > 0) {
+          uint4* bvm = bin_vm(buf);
+          uint32_t* bcnt = bin_cnt(buf);
+          while (rr[0] + rr[1] + rr[2] > 0 && nb < kMaxBins) {
             next_bin(p, rr, a);
+            if (lane == 0) {
+              uint32_t vm[4] = {0u, 0u, 0u, 0u};
+              int off = 0;
+              for (int e = 0; e < 3; ++e)
+                for (int m = 0; m < a[e]; ++m) {
+                  set_rows(vm, off, off + p.pk_rows[e]);
+                  off += p.pk_step[e];
+                }
+              bvm[nb] = make_uint4(vm[0], vm[1], vm[2], vm[3]);
+              bcnt[nb] = (uint32_t)a[0] | ((uint32_t)a[1] << 8) | ((uint32_t)a[2] << 16);
+            }
             ++nb;
           }
-          npk = cF + nb;
+          if (rr[0] + rr[1] + rr[2] > 0) {
+            // more bins than the buffer holds: run this list unpacked (the
+            // entries are read from col_idx again, in list order)
+            packed = false;
+          } else {
+            npk = cF + nb;
+          }
         }
         if (lane == 0) {
           hd->rs = rs;
@@ -370,7 +403,6 @@ __global__ void __launch_bounds__(kThreads, 1)
           __syncwarp();
           issued_q = i + 1;
         }
-        int prem[3] = {hd.c[0], hd.c[1], hd.c[2]};
         const int pstart[3] = {hd.nF, hd.nF + hd.c[0], hd.nF + hd.c[0] + hd.c[1]};
         int pptr[3] = {0, 0, 0};
         for (int j = 0; j < hd.n; ++j, ++jj) {
@@ -382,8 +414,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           uint8_t* dst = smem + ring_off + st * Cfg::kTileBytes;
           if (hd.packed && j >= hd.nF) {
-            int a[3];
-            next_bin(p, prem, a);
+            const uint32_t cnt = bin_cnt(buf)[j - hd.nF];
+            const int a[3] = {(int)(cnt & 255u), (int)((cnt >> 8) & 255u), (int)(cnt >> 16)};
             if (elect_one()) {
               uint32_t bytes = 0;
 #pragma unroll
@@ -457,12 +489,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         __syncwarp();
       };
-      auto issue_pv = [&](int st, uint32_t tP, uint32_t tO, uint32_t acc) {
-        const uint64_t vd = sdesc_add(vd0, st * Cfg::kTileBytes);
+      // O_g (+)= P(keys 64 * half .. + 63) . V(same keys)
+      auto issue_pv = [&](int st, int g, int half, uint32_t acc) {
+        const uint64_t vd = sdesc_add(vd0, st * Cfg::kTileBytes + half * 64 * 128);
+        const uint32_t tP = tbase + g * 128 + 64 + half * 32, tO = tbase + 256 + g * 128;
         if (elect_one()) {
 #pragma unroll
-          for (int kk = 0; kk < kTile / 16; ++kk)
-            mma_ts(tO, tP + kk * 8, sdesc_add(vd, kk * 16 * 128), idesc_pv, (acc | (uint32_t)kk) != 0);
+          for (int kk = 0; kk < 4; ++kk)
+            mma_ts(tO, tP + kk * 8, sdesc_add(vd, kk * 16 * 128), idesc_pv,
+                   (acc | (uint32_t)half | (uint32_t)kk) != 0);
         }
         __syncwarp();
       };
@@ -476,6 +511,17 @@ __global__ void __launch_bounds__(kThreads, 1)
       int64_t jj = 0;             // key tiles consumed so far (ring position)
       int64_t pcount[2] = {0, 0};  // completed P hand-offs per group
       bool alive = true;
+      // QK of tile t (ring position jj + t) into the S buffer of its group
+      auto qk = [&](int t) {
+        const int64_t q = jj + t;
+        const int st = (int)(q % Cfg::NK);
+        if (!wait(&k_full[st], (uint32_t)((q / Cfg::NK) & 1))) return false;
+        tc_fence_after();
+        issue_qk(st, tbase + (t & 1) * 128);
+        commit(&s_full[t & 1]);
+        commit(&k_empty[st]);
+        return true;
+      };
       for (int64_t i = 0; alive && i < my_tiles; ++i) {
         const int buf = (int)(i & 1);
         if (!wait(&list_full[buf], (uint32_t)((i >> 1) & 1))) break;
@@ -484,41 +530,34 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (lane == 0) mbar_arrive(&list_empty[buf]);
         if (!wait(q_full, (uint32_t)(i & 1))) break;
         tc_fence_after();
-        if (n > 0) {
-          const int st0 = (int)(jj % Cfg::NK);
-          if (!wait(&k_full[st0], (uint32_t)((jj / Cfg::NK) & 1))) break;
-          tc_fence_after();
-          issue_qk(st0, tbase);
-          commit(&s_full[0]);
-          commit(&k_empty[st0]);
-        }
-        if (n <= 1) commit(q_empty);  // Q no longer read once that QK completes
+        // group g takes tiles g, g + 2, ...; each group's next QK follows its
+        // own PV, so S of tile j+2 is ready as soon as PV of tile j is done
+        if (n > 0 && !qk(0)) break;
+        if (n > 1 && !qk(1)) break;
+        if (n <= 2) commit(q_empty);  // Q no longer read once those QKs complete
         for (int j = 0; j < n; ++j) {
-          if (j + 1 < n) {
-            const int64_t q1 = jj + j + 1;
-            const int st1 = (int)(q1 % Cfg::NK);
-            if (!wait(&k_full[st1], (uint32_t)((q1 / Cfg::NK) & 1))) { alive = false; break; }
-            tc_fence_after();
-            issue_qk(st1, tbase + ((j + 1) & 1) * 128);
-            commit(&s_full[(j + 1) & 1]);
-            commit(&k_empty[st1]);
-            if (j + 2 == n) commit(q_empty);
-          }
           const int g = j & 1;
           const int64_t q0 = jj + j;
           const int st = (int)(q0 % Cfg::NV);
-          if (!wait(&p_ready[g], (uint32_t)(pcount[g] & 1)) ||
-              !wait(&v_full[st], (uint32_t)((q0 / Cfg::NV) & 1))) {
+          const uint32_t ph = (uint32_t)(pcount[g] & 1);
+          if (!wait(&p_half[g], ph) || !wait(&v_full[st], (uint32_t)((q0 / Cfg::NV) & 1))) {
             alive = false;
             break;
           }
-          ++pcount[g];
           // the previous tile's output must be out of tensor memory before
           // this tile's first PV overwrites O
           if (j == 0 && i > 0 && !wait(o_free, (uint32_t)((i - 1) & 1))) { alive = false; break; }
           tc_fence_after();
-          issue_pv(st, tbase + g * 128 + 64, tbase + 256 + g * 128, j >= 2);
+          issue_pv(st, g, 0, j >= 2);
+          if (!wait(&p_ready[g], ph)) { alive = false; break; }
+          ++pcount[g];
+          tc_fence_after();
+          issue_pv(st, g, 1, 1);
           commit(&v_empty[st]);
+          if (j + 2 < n) {
+            if (!qk(j + 2)) { alive = false; break; }
+            if (j + 3 == n) commit(q_empty);
+          }
         }
         jj += n;
         if (n == 0 && i > 0 && !wait(o_free, (uint32_t)((i - 1) & 1))) alive = false;
@@ -554,34 +593,23 @@ __global__ void __launch_bounds__(kThreads, 1)
       int qt, h, b;
       tile_of(i, qt, h, b);
       const int n = hd.n;
-      float m_run = -INFINITY, l_run = 0.f;
-      int srem[3] = {hd.c[0], hd.c[1], hd.c[2]};
-      int scur = hd.nF;
+      RowState rs;
       for (int j = g; j < n; j += 2) {
         uint32_t vm[4] = {0u, 0u, 0u, 0u};
         if (hd.packed && j >= hd.nF) {
-          int a[3];
-          while (scur < j) {
-            next_bin(p, srem, a);
-            ++scur;
-          }
-          next_bin(p, srem, a);
-          ++scur;
-          int off = 0;
-#pragma unroll
-          for (int e = 0; e < 3; ++e)
-            for (int m = 0; m < a[e]; ++m) {
-              set_rows(vm, off, off + p.pk_rows[e]);
-              off += p.pk_step[e];
-            }
+          const uint4 b = bin_vm(buf)[j - hd.nF];
+          vm[0] = b.x;
+          vm[1] = b.y;
+          vm[2] = b.z;
+          vm[3] = b.w;
+        } else if (hd.packed) {
+          // a full tile (every slot holds a token) unless the entry was out of range
+          const uint32_t f = ent[j] != kBad ? kAll : 0u;
+          vm[0] = vm[1] = vm[2] = vm[3] = f;
         } else {
           int kt;
           bool ok;
-          if (hd.packed) {
-            const uint16_t c = ent[j];
-            ok = c != kBad;
-            kt = ok ? c : 0;
-          } else {
+          {
             const int c = __ldg(p.col_idx + hd.rs + j);
             ok = c >= 0 && (int64_t)c < p.nblocks;
             kt = ok ? c : 0;
@@ -605,58 +633,31 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int e = 0; e < 128; ++e) s[e] = __uint_as_float(r128[e]);
         }
-        if ((vm[0] & vm[1] & vm[2] & vm[3]) != kAll) {
-#pragma unroll
-          for (int w = 0; w < 4; ++w)
-#pragma unroll
-            for (int e = 0; e < 32; ++e)
-              if (!((vm[w] >> e) & 1u)) s[w * 32 + e] = -INFINITY;
+        float corr;
+        uint64_t neg_ms2;
+        // most key tiles are full: they take a copy of the step without masking
+        const bool need = (vm[0] & vm[1] & vm[2] & vm[3]) == kAll
+                              ? softmax_max<128, false>(s, vm, rs, sl2, thr, corr, neg_ms2)
+                              : softmax_max<128, true>(s, vm, rs, sl2, thr, corr, neg_ms2);
+        uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};
+        {
+          uint32_t pk[32];
+          softmax_exp<0, 64>(s, sl2, neg_ms2, pk, acc);
+          tmem_st32(tS + 64, pk);
         }
-        // row max: 8 independent chains of 3-input max, then a small tree
-        float m8[8];
-#pragma unroll
-        for (int c = 0; c < 8; ++c) m8[c] = fmax3f(s[c], s[c + 8], s[c + 16]);
-#pragma unroll
-        for (int e = 24; e < 120; e += 16)
-#pragma unroll
-          for (int c = 0; c < 8; ++c) m8[c] = fmax3f(m8[c], s[e + c], s[e + 8 + c]);
-#pragma unroll
-        for (int c = 0; c < 8; ++c) m8[c] = fmaxf(m8[c], s[120 + c]);
-        const float mx = fmax3f(fmax3f(m8[0], m8[1], m8[2]), fmax3f(m8[3], m8[4], m8[5]),
-                                fmaxf(m8[6], m8[7]));
-        const float m_new = fmaxf(m_run, mx);
-        const bool need = m_new > m_run + thr;
-        float corr = 1.f;
-        if (need) {
-          corr = ex2_approx((m_run - m_new) * sl2);
-          m_run = m_new;
-          l_run *= corr;
+        // O of this group holds every earlier PV of the group in this query
+        // tile (S(j) was written after the group's previous PV); it is
+        // rescaled before this tile's first PV, once half of s is no longer
+        // live
+        if (j >= 2 && __any_sync(kAll, need)) tmem_scale<D>(tO, corr);
+        tc_fence_before();
+        mbar_arrive(&p_half[g]);
+        {
+          uint32_t pk[32];
+          softmax_exp<64, 64>(s, sl2, neg_ms2, pk, acc);
+          tmem_st32(tS + 96, pk);
         }
-        const float ms = (m_run == -INFINITY) ? 0.f : m_run * sl2;
-        uint32_t pk[64];
-        float l8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};  // independent partial sums
-#pragma unroll
-        for (int e = 0; e < 64; ++e) {
-          const float p0 = ex2_approx(fmaf(s[2 * e], sl2, -ms));
-          const float p1 = ex2_approx(fmaf(s[2 * e + 1], sl2, -ms));
-          l8[e & 7] += p0 + p1;
-          pk[e] = pack_bf16x2_d(p0, p1);
-        }
-        l_run += ((l8[0] + l8[1]) + (l8[2] + l8[3])) + ((l8[4] + l8[5]) + (l8[6] + l8[7]));
-        // O of this group holds every earlier PV of the group in this tile:
-        // S(j) was written after the group's previous PV
-        if (j >= 2 && __any_sync(kAll, need)) {
-#pragma unroll
-          for (int c = 0; c < D / 32; ++c) {
-            uint32_t o32[32];
-            tmem_ld32(tO + c * 32, o32);
-#pragma unroll
-            for (int e = 0; e < 32; ++e) o32[e] = __float_as_uint(__uint_as_float(o32[e]) * corr);
-            tmem_st32(tO + c * 32, o32);
-          }
-        }
-        tmem_st32(tS + 64, *reinterpret_cast<uint32_t(*)[32]>(&pk[0]));
-        tmem_st32(tS + 96, *reinterpret_cast<uint32_t(*)[32]>(&pk[32]));
+        softmax_sum(rs, acc);
         tc_fence_before();
         mbar_arrive(&p_ready[g]);
       }
@@ -668,28 +669,30 @@ __global__ void __launch_bounds__(kThreads, 1)
         break;
       }
       tc_fence_after();
-      stats[(2 * g) * kTile + row] = m_run;
-      stats[(2 * g + 1) * kTile + row] = l_run;
+      // statistics buffers alternate between query tiles: each group reads
+      // tile i's before it reaches tile i+1's barrier, so tile i+2 may
+      // overwrite them
+      float* st = stats + (i & 1) * 4 * kTile;
+      st[(2 * g) * kTile + row] = rs.m;
+      st[(2 * g + 1) * kTile + row] = rs.l;
       softmax_sync();
-      const float mA = stats[row], lA = stats[kTile + row];
-      const float mB = stats[2 * kTile + row], lB = stats[3 * kTile + row];
-      softmax_sync();  // the statistics are read before the next tile rewrites them
+      const float mA = st[row], lA = st[kTile + row];
+      const float mB = st[2 * kTile + row], lB = st[3 * kTile + row];
       const int nA = (n + 1) / 2, nB = n / 2;
       const float m = fmaxf(mA, mB);
       const float a = (nA > 0 && mA != -INFINITY) ? ex2_approx((mA - m) * sl2) : 0.f;
       const float bb = (nB > 0 && mB != -INFINITY) ? ex2_approx((mB - m) * sl2) : 0.f;
       const float l = lA * a + lB * bb;
-      const uint4 tq = __ldg(reinterpret_cast<const uint4*>(p.tile_valid) + qt);
-      const uint32_t qw = (row < 32) ? tq.x : (row < 64) ? tq.y : (row < 96) ? tq.z : tq.w;
-      const bool qvalid = (qw >> (row & 31)) & 1u;
-      const bool has = n > 0 && qvalid && l > 0.f;
-      const float inv_l = has ? 1.f / l : 0.f;
-      const float wa = a * inv_l, wb = bb * inv_l;
-      // slot (y, x) of tile (t, i, j) is token (t, y0 + y, x0 + x)
+      // slot (y, x) of tile (t, i, j) is token (t, y0 + y, x0 + x); slots
+      // past the grid's right or bottom edge hold no token
       int x0, y0, fr;
       nat_coords(qt, b, x0, y0, fr);
       const int ay = (int)p.div_pw.div((uint32_t)row);
       const int yy = y0 + ay, xx = x0 + (row - ay * p.pw);
+      const bool qvalid = ay < p.ph && yy < p.H && xx < p.W;
+      const bool has = n > 0 && qvalid && l > 0.f;
+      const float inv_l = has ? 1.f / l : 0.f;
+      const float wa = a * inv_l, wb = bb * inv_l;
       const int t = fr - b * p.T;
       const int64_t ntok = ((int64_t)t * p.H + yy) * p.W + xx;
       const int64_t orow = ((int64_t)b * p.N + ntok) * p.Hh + h;
@@ -711,7 +714,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           const float v0 = has ? __uint_as_float(xa[2 * e]) * wa + __uint_as_float(xb[2 * e]) * wb : 0.f;
           const float v1 =
               has ? __uint_as_float(xa[2 * e + 1]) * wa + __uint_as_float(xb[2 * e + 1]) * wb : 0.f;
-          w16[e] = pack_bf16x2_d(v0, v1);
+          w16[e] = pack_bf16x2(v0, v1);
         }
         if (qvalid) {
 #pragma unroll

@@ -45,6 +45,7 @@
 #include <cmath>
 #include <cstring>
 
+#include "attn_common.cuh"
 #include "bsa_internal.cuh"
 #include "ptx.cuh"
 
@@ -72,7 +73,7 @@ struct AttnCfg {
   static constexpr int kOffK = kQBytes;
   static constexpr int kOffV = kOffK + NS * kKVBytes;
   static constexpr int kOffBar = kOffV + NS * kKVBytes;
-  static constexpr int kNumBars = 1 + 3 * NS + 2 + 2 + 1;
+  static constexpr int kNumBars = 1 + 3 * NS + 2 + 2 + 2 + 1;
   static constexpr int kOffMisc = kOffBar + kNumBars * 8;
   static constexpr int kOffList = kOffMisc + 16;
   // FINE: the union of key tiles (uint16); PACK: the key list sorted by tile
@@ -149,11 +150,6 @@ __device__ __forceinline__ void set_bits(uint32_t (&m)[4], int lo, int len) {
   }
 }
 
-__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
-  __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
-  return *reinterpret_cast<uint32_t*>(&v);
-}
-
 // Two floats to two e4m3 bytes (nearest, ties to even, saturating at +-448),
 // lo in the low byte.
 __device__ __forceinline__ uint32_t pack_e4m3x2(float lo, float hi) {
@@ -189,7 +185,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* v_full = k_full + Cfg::NS;
   uint64_t* kv_empty = v_full + Cfg::NS;
   uint64_t* s_full = kv_empty + Cfg::NS;  // [2]: S_A, S_B written
-  uint64_t* p_ready = s_full + 2;         // [2]: P_A, P_B written (128 arrivals each)
+  uint64_t* p_half = s_full + 2;          // [2]: keys 0..63 of P_A, P_B written (bf16)
+  uint64_t* p_ready = p_half + 2;         // [2]: P_A, P_B written (128 arrivals each)
   uint64_t* o_final = p_ready + 2;        // every MMA done
   uint32_t* misc = reinterpret_cast<uint32_t*>(smem + Cfg::kOffMisc);  // tmem, abort, count, skip
   uint16_t* tlist = reinterpret_cast<uint16_t*>(smem + Cfg::kOffList);
@@ -223,6 +220,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     mbar_init(&s_full[0], 1);
     mbar_init(&s_full[1], 1);
+    mbar_init(&p_half[0], 128);
+    mbar_init(&p_half[1], 128);
     mbar_init(&p_ready[0], 128);
     mbar_init(&p_ready[1], 128);
     mbar_init(o_final, 1);
@@ -551,6 +550,18 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         __syncwarp();
       };
+      // bf16: O_g (+)= P(keys 64 * half .. + 63) . V(same keys)
+      auto issue_pv_half = [&](int st, int g, int half, uint32_t acc) {
+        const uint64_t vd = sdesc_add(vd0, st * Cfg::kKVBytes + half * 64 * 128);
+        const uint32_t tP = tbase + g * 128 + 64 + half * 32, tO = tbase + 256 + g * 128;
+        if (elect_one()) {
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)
+            mma_ts(tO, tP + kk * 8, sdesc_add(vd, kk * 16 * 128), idesc_pv,
+                   (acc | (uint32_t)half | (uint32_t)kk) != 0);
+        }
+        __syncwarp();
+      };
       auto commit = [&](uint64_t* bar) {
         if (elect_one()) mma_commit(bar);
         __syncwarp();
@@ -558,6 +569,32 @@ __global__ void __launch_bounds__(kThreads, 1)
       auto wait = [&](uint64_t* bar, uint32_t parity) {
         return __all_sync(kFull, bounded_wait(bar, parity, wc));
       };
+      if constexpr (!F8) {
+        // group g takes tiles g, g + 2, ...; QK of tile j+2 follows PV of
+        // tile j, so each group's next S is ready as soon as its PV is done;
+        // P is handed over in two halves
+        auto qk = [&](int t) {
+          const int st = t % Cfg::NS;
+          if (!wait(&k_full[st], (t / Cfg::NS) & 1)) return false;
+          tc_fence_after();
+          issue_qk(st, tbase + (t & 1) * 128);
+          commit(&s_full[t & 1]);
+          return true;
+        };
+        bool alive = wait(q_full, 0) && qk(0) && (n < 2 || qk(1));
+        for (int j = 0; alive && j < n; ++j) {
+          const int g = j & 1, st = j % Cfg::NS;
+          if (!wait(&p_half[g], (j >> 1) & 1) || !wait(&v_full[st], (j / Cfg::NS) & 1)) break;
+          tc_fence_after();
+          issue_pv_half(st, g, 0, j >= 2);
+          if (!wait(&p_ready[g], (j >> 1) & 1)) break;
+          tc_fence_after();
+          issue_pv_half(st, g, 1, 1);
+          commit(&kv_empty[st]);
+          if (j + 2 < n && !qk(j + 2)) break;
+        }
+        commit(o_final);
+      } else {
       bool alive = wait(q_full, 0) && wait(&k_full[0], 0);
       if (alive) {
         tc_fence_after();
@@ -579,6 +616,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         commit(&kv_empty[st]);
       }
       commit(o_final);
+      }
     }
     cta_end_sync();
     if (warp == 1) {
@@ -601,7 +639,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                          : 1.f;
     const float sl2 = p.scale_log2 * sqk;
     const float thr = 8.0f / sl2;  // rescale O when the max grows by more than 2^8
-    float m_run = -INFINITY, l_run = 0.f;
+    RowState rs;
     int64_t fptr = 0, fend = 0;
     int fprev = -1;
     if (FINE) {
@@ -683,37 +721,66 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int i = 0; i < 128; ++i) s[i] = __uint_as_float(r128[i]);
       }
-      if ((vm[0] & vm[1] & vm[2] & vm[3]) != kFull) {
+      if constexpr (!F8) {
+        float corr;
+        uint64_t neg_ms2;
+        // full key tiles take a copy of the step without masking
+        const bool need = (vm[0] & vm[1] & vm[2] & vm[3]) == kFull
+                              ? softmax_max<128, false>(s, vm, rs, sl2, thr, corr, neg_ms2)
+                              : softmax_max<128, true>(s, vm, rs, sl2, thr, corr, neg_ms2);
+        uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};
+        {
+          uint32_t pk[32];
+          softmax_exp<0, 64>(s, sl2, neg_ms2, pk, acc);
+          tmem_st32(tS + 64, pk);
+        }
+        // O of this group holds every earlier PV of the group (S(j) was
+        // written after the group's previous PV); it is rescaled before this
+        // tile's first PV, once half of s is no longer live
+        if (j >= 2 && __any_sync(kFull, need)) tmem_scale<D>(tO, corr);
+        tc_fence_before();
+        mbar_arrive(&p_half[g]);
+        {
+          uint32_t pk[32];
+          softmax_exp<64, 64>(s, sl2, neg_ms2, pk, acc);
+          tmem_st32(tS + 96, pk);
+        }
+        softmax_sum(rs, acc);
+        tc_fence_before();
+        mbar_arrive(&p_ready[g]);
+        continue;
+      } else {
+        // e4m3: P rounded to e4m3, four keys to a TMEM column, in one hand-off
+        if ((vm[0] & vm[1] & vm[2] & vm[3]) != kFull) {
 #pragma unroll
-        for (int w = 0; w < 4; ++w)
+          for (int w = 0; w < 4; ++w)
 #pragma unroll
-          for (int i = 0; i < 32; ++i)
-            if (!((vm[w] >> i) & 1u)) s[w * 32 + i] = -INFINITY;
-      }
-      // row max: 8 independent chains of 3-input max, then a small tree
-      float m8[8];
+            for (int i = 0; i < 32; ++i)
+              if (!((vm[w] >> i) & 1u)) s[w * 32 + i] = -INFINITY;
+        }
+        // row max: 8 independent chains of 3-input max, then a small tree
+        float m8[8];
 #pragma unroll
-      for (int c = 0; c < 8; ++c) m8[c] = fmax3f(s[c], s[c + 8], s[c + 16]);
+        for (int c = 0; c < 8; ++c) m8[c] = fmax3f(s[c], s[c + 8], s[c + 16]);
 #pragma unroll
-      for (int i = 24; i < 120; i += 16)
+        for (int i = 24; i < 120; i += 16)
 #pragma unroll
-        for (int c = 0; c < 8; ++c) m8[c] = fmax3f(m8[c], s[i + c], s[i + 8 + c]);
+          for (int c = 0; c < 8; ++c) m8[c] = fmax3f(m8[c], s[i + c], s[i + 8 + c]);
 #pragma unroll
-      for (int c = 0; c < 8; ++c) m8[c] = fmaxf(m8[c], s[120 + c]);
-      const float mx = fmax3f(fmax3f(m8[0], m8[1], m8[2]), fmax3f(m8[3], m8[4], m8[5]),
-                              fmaxf(m8[6], m8[7]));
-      const float m_new = fmaxf(m_run, mx);
-      const bool need = m_new > m_run + thr;
-      float corr = 1.f;
-      if (need) {
-        corr = ex2_approx((m_run - m_new) * sl2);
-        m_run = m_new;
-        l_run *= corr;
-      }
-      const float ms = (m_run == -INFINITY) ? 0.f : m_run * sl2;
-      uint32_t pk[64];
-      float l8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};  // independent partial sums
-      if constexpr (F8) {
+        for (int c = 0; c < 8; ++c) m8[c] = fmaxf(m8[c], s[120 + c]);
+        const float mx = fmax3f(fmax3f(m8[0], m8[1], m8[2]), fmax3f(m8[3], m8[4], m8[5]),
+                                fmaxf(m8[6], m8[7]));
+        const float m_new = fmaxf(rs.m, mx);
+        const bool need = m_new > rs.m + thr;
+        float corr = 1.f;
+        if (need) {
+          corr = ex2_approx((rs.m - m_new) * sl2);
+          rs.m = m_new;
+          rs.l *= corr;
+        }
+        const float ms = (rs.m == -INFINITY) ? 0.f : rs.m * sl2;
+        uint32_t pk[32];
+        float l8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};  // independent partial sums
         // P as e4m3 bytes, four keys to a word (P <= 2^8 < 448)
 #pragma unroll
         for (int i = 0; i < 32; ++i) {
@@ -724,32 +791,23 @@ __global__ void __launch_bounds__(kThreads, 1)
           l8[i & 7] += (p0 + p1) + (p2 + p3);
           pk[i] = pack_e4m3x2(p0, p1) | (pack_e4m3x2(p2, p3) << 16);
         }
-      } else {
+        rs.l += ((l8[0] + l8[1]) + (l8[2] + l8[3])) + ((l8[4] + l8[5]) + (l8[6] + l8[7]));
+        // O of this group holds every earlier PV of the group: S(j) was written
+        // after the group's previous PV in the tensor cores' issue order.
+        if (j >= 2 && __any_sync(kFull, need)) {
 #pragma unroll
-        for (int i = 0; i < 64; ++i) {
-          const float p0 = ex2_approx(fmaf(s[2 * i], sl2, -ms));
-          const float p1 = ex2_approx(fmaf(s[2 * i + 1], sl2, -ms));
-          l8[i & 7] += p0 + p1;
-          pk[i] = pack_bf16x2(p0, p1);
+          for (int c = 0; c < D / 32; ++c) {
+            uint32_t o32[32];
+            tmem_ld32(tO + c * 32, o32);
+#pragma unroll
+            for (int i = 0; i < 32; ++i) o32[i] = __float_as_uint(__uint_as_float(o32[i]) * corr);
+            tmem_st32(tO + c * 32, o32);
+          }
         }
+        tmem_st32(tS + 64, *reinterpret_cast<uint32_t(*)[32]>(&pk[0]));
+        tc_fence_before();
+        mbar_arrive(&p_ready[g]);
       }
-      l_run += ((l8[0] + l8[1]) + (l8[2] + l8[3])) + ((l8[4] + l8[5]) + (l8[6] + l8[7]));
-      // O of this group holds every earlier PV of the group: S(j) was written
-      // after the group's previous PV in the tensor cores' issue order.
-      if (j >= 2 && __any_sync(kFull, need)) {
-#pragma unroll
-        for (int c = 0; c < D / 32; ++c) {
-          uint32_t o32[32];
-          tmem_ld32(tO + c * 32, o32);
-#pragma unroll
-          for (int i = 0; i < 32; ++i) o32[i] = __float_as_uint(__uint_as_float(o32[i]) * corr);
-          tmem_st32(tO + c * 32, o32);
-        }
-      }
-      tmem_st32(tS + 64, *reinterpret_cast<uint32_t(*)[32]>(&pk[0]));
-      if constexpr (!F8) tmem_st32(tS + 96, *reinterpret_cast<uint32_t(*)[32]>(&pk[32]));
-      tc_fence_before();
-      mbar_arrive(&p_ready[g]);
     }
     // ---------------------------------------------------------- epilogue
     if (alive && n > 0) {
@@ -758,8 +816,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     // exchange (max, sum) of the two groups through a free K stage
     float* stats = reinterpret_cast<float*>(smem + Cfg::kOffK);  // [4][128]: mA lA mB lB
-    stats[(2 * g) * kTile + row] = m_run;
-    stats[(2 * g + 1) * kTile + row] = l_run;
+    stats[(2 * g) * kTile + row] = rs.m;
+    stats[(2 * g + 1) * kTile + row] = rs.l;
     softmax_groups_sync();
     const float mA = stats[row], lA = stats[kTile + row];
     const float mB = stats[2 * kTile + row], lB = stats[3 * kTile + row];
