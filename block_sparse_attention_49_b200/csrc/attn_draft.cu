@@ -75,8 +75,9 @@ struct DraftCfg {
   static constexpr int kOffV = kOffK + NK * kTileBytes;
   static constexpr int kOffBar = kOffV + NV * kTileBytes;
   // q_full, q_empty, k_full[NK], k_empty[NK], v_full[NV], v_empty[NV],
-  // s_full[2], p_half[2], p_ready[2], o_final, o_free, list_full[2], list_empty[2]
-  static constexpr int kNumBars = 2 + 2 * NK + 2 * NV + 2 + 2 + 2 + 2 + 2 + 2;
+  // s_full[2], p_half[2], p_ready[2], o_final, o_free, list_full[2], list_empty[2],
+  // stats_full[2]
+  static constexpr int kNumBars = 2 + 2 * NK + 2 * NV + 2 + 2 + 2 + 2 + 2 + 2 + 2;
   static constexpr int kOffMisc = kOffBar + kNumBars * 8;     // tmem, abort
   static constexpr int kOffStats = kOffMisc + 16;             // [2][4][128] floats
   static constexpr int kOffLists = kOffStats + 2 * 4 * kTile * 4;
@@ -143,7 +144,6 @@ __device__ __forceinline__ void next_bin(const DraftParams& p, int (&r)[3], int 
   }
 }
 
-__device__ __forceinline__ void softmax_sync() { asm volatile("bar.sync 1, 256;" ::: "memory"); }
 __device__ __forceinline__ void end_sync() { asm volatile("bar.sync 2, 384;" ::: "memory"); }
 
 template <int D>
@@ -170,6 +170,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* o_free = o_final + 1;
   uint64_t* list_full = o_free + 1;       // [2]
   uint64_t* list_empty = list_full + 2;   // [2]
+  uint64_t* stats_full = list_empty + 2;  // [2]: both groups' (max, sum) of a query tile
   uint32_t* misc = reinterpret_cast<uint32_t*>(smem + Cfg::kOffMisc);  // tmem, abort, skip
   float* stats = reinterpret_cast<float*>(smem + Cfg::kOffStats);
   auto list_base = [&](int buf) { return smem + Cfg::kOffLists + buf * Cfg::kListBytes; };
@@ -230,6 +231,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int i = 0; i < 2; ++i) {
       mbar_init(&list_full[i], 32);
       mbar_init(&list_empty[i], 2 + 1 + 256);  // producers, MMA warp, softmax threads
+      mbar_init(&stats_full[i], 256);
     }
     misc[1] = 0;
     misc[2] = (*reinterpret_cast<volatile unsigned int*>(p.status) & kStatusTimeout) ? 1u : 0u;
@@ -675,7 +677,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       float* st = stats + (i & 1) * 4 * kTile;
       st[(2 * g) * kTile + row] = rs.m;
       st[(2 * g + 1) * kTile + row] = rs.l;
-      softmax_sync();
+      // a bounded wait, not a named barrier: a group that gave up on an
+      // earlier wait must not leave the other one waiting for good
+      mbar_arrive(&stats_full[i & 1]);
+      if (!__all_sync(kAll, bounded_wait(&stats_full[i & 1], (uint32_t)((i >> 1) & 1), wc))) {
+        alive = false;
+        break;
+      }
       const float mA = st[row], lA = st[kTile + row];
       const float mB = st[2 * kTile + row], lB = st[3 * kTile + row];
       const int nA = (n + 1) / 2, nB = n / 2;

@@ -23,6 +23,9 @@
 //  * warp 0: TMA producer (both query tiles, then K and V of every key tile
 //    into 2-deep rings; a K slot is refilled as soon as its last QK product
 //    is done, a V slot after its last PV product).  warp 1: MMA issuer.
+//    warp 2: key masks - for each key tile and each query frame of the CTA,
+//    the rows whose frame is in that frame's A(t), computed a ring of tiles
+//    ahead (once per CTA instead of once per softmax warp).
 //    warps 4-7 / 8-11: softmax of query tile 0 / 1, one row per thread,
 //    masking keys whose frame is not in the row's own A(t).
 //  * tensor memory: S0 | S1 | O0 | O1; P aliases the upper half of its S.
@@ -52,6 +55,7 @@ constexpr int kMaxRowFrames = 8;   // frames a 256-token query pair may touch
 constexpr int kMaxFrames = 4096;
 constexpr int kSetWords = kMaxFrames / 32;
 constexpr int kMaxRuns = 1024;     // runs of consecutive frames in a query pair's union
+constexpr int kMaskRing = 16;      // key tiles whose row masks are computed ahead
 
 template <int D>
 struct LvsaCfg {
@@ -65,12 +69,14 @@ struct LvsaCfg {
   static constexpr int kOffV = kOffK + NS * kKVBytes;
   static constexpr int kOffBar = kOffV + NS * kKVBytes;
   // q_full, k_full[NS], v_full[NS], k_empty[NS], v_empty[NS], s_full[2],
-  // p_half[2], p_ready[2], o_final
-  static constexpr int kNumBars = 1 + 4 * NS + 2 + 2 + 2 + 1;
+  // p_half[2], p_ready[2], o_final, mask_full[kMaskRing], mask_empty[kMaskRing]
+  static constexpr int kNumBars = 1 + 4 * NS + 2 + 2 + 2 + 1 + 2 * kMaskRing;
   static constexpr int kOffMisc = kOffBar + kNumBars * 8;
   static constexpr int kOffTiles = kOffMisc + 16;
   static constexpr int kOffSets = kOffTiles + kMaxRuns * 12;  // run table: tok0, len, v0
-  static constexpr int kBytes = kOffSets + (kMaxRowFrames + 1) * kSetWords * 4;
+  static constexpr int kOffMasks = kOffSets + (kMaxRowFrames + 1) * kSetWords * 4;
+  // [kMaskRing][kMaxRowFrames] 128-bit key masks: tile j, query frame tf + slot
+  static constexpr int kBytes = kOffMasks + kMaskRing * kMaxRowFrames * 16;
   static constexpr int kSmem = kBytes + 1024;
   static constexpr uint32_t kTmemCols = 512;
   static_assert(kSmem <= 232448, "shared memory budget");
@@ -187,6 +193,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* p_half = s_full + 2;          // [2]: keys 0..63 of P stored
   uint64_t* p_ready = p_half + 2;         // [2]: all of P stored
   uint64_t* o_final = p_ready + 2;
+  uint64_t* mask_full = o_final + 1;            // [kMaskRing]: masks of a tile written
+  uint64_t* mask_empty = mask_full + kMaskRing;  // [kMaskRing]: read by the 8 softmax warps
+  uint4* masks = reinterpret_cast<uint4*>(smem + Cfg::kOffMasks);
   uint32_t* misc = reinterpret_cast<uint32_t*>(smem + Cfg::kOffMisc);  // tmem, abort, ntiles, skip
   // runs of consecutive frames of the union, laid end to end as a stream of
   // key rows: run r = tokens [run_tok[r], + run_len[r]) at rows run_v[r]..
@@ -222,6 +231,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(&p_ready[0], 128);
     mbar_init(&p_ready[1], 128);
     mbar_init(o_final, 1);
+    for (int i = 0; i < kMaskRing; ++i) {
+      mbar_init(&mask_full[i], 32);
+      mbar_init(&mask_empty[i], 8);
+    }
     misc[1] = 0;
     misc[2] = 0;
     misc[3] = (*reinterpret_cast<volatile unsigned int*>(p.status) & kStatusTimeout) ? 1u : 0u;
@@ -303,7 +316,39 @@ __global__ void __launch_bounds__(kThreads, 1)
   // made them spill, and each reload delayed an MMA batch)
   if (warp < 4) {
     asm volatile("setmaxnreg.dec.sync.aligned.u32 72;");
-    if (warp == 0 && n > 0) {
+    if (warp == 2 && n > 0) {
+      // ------------------------------------------------------ key masks
+      // lane rf computes, for key tile j, which of its 128 rows the queries
+      // of frame tf + rf attend: rows of frames in A(tf + rf); rows between
+      // and after the pieces stay masked.  The softmax warps read them from
+      // a ring of kMaskRing tiles.
+      int rcur = 0;
+      const uint32_t* myset = sets + min(lane, kMaxRowFrames - 1) * kSetWords;
+      for (int j = 0; j < n; ++j) {
+        const int r = j % kMaskRing;
+        if (!__all_sync(kFullMask, bounded_wait(&mask_empty[r], ((j / kMaskRing) & 1) ^ 1, wc)))
+          break;
+        first_run(j, rcur);
+        uint32_t vm[4] = {0u, 0u, 0u, 0u};
+        for (int rr = rcur; rr < nruns && run_v[rr] < (j + 1) * kTile; ++rr) {
+          const int a = max(j * kTile, run_v[rr]), e = min((j + 1) * kTile, run_v[rr] + run_len[rr]);
+          if (e <= a) continue;
+          const int k0 = run_tok[rr] + (a - run_v[rr]), kn = e - a, o = a - j * kTile;
+          int f = (int)p.divP.div((uint32_t)k0);
+          int lo = 0, fend = (f + 1) * p.P - k0;
+          while (lo < kn) {
+            const int hi = min(kn, fend);
+            if (f < p.T && bit_of(myset, f)) set_range(vm, o + lo, o + hi);
+            lo = hi;
+            ++f;
+            fend += p.P;
+          }
+        }
+        if (lane < nrf) masks[r * kMaxRowFrames + lane] = make_uint4(vm[0], vm[1], vm[2], vm[3]);
+        __syncwarp();
+        mbar_arrive(&mask_full[r]);
+      }
+    } else if (warp == 0 && n > 0) {
       // -------------------------------------------------------- TMA producer
       // the whole warp runs the loop (warp-uniform operands); one lane issues
       if (elect_one()) {
@@ -471,33 +516,24 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int qn = q0 + g * kTile + row;  // query token within the batch
     const bool qvalid = qn < p.N;
     const int tq = qvalid ? (int)p.divP.div((uint32_t)qn) : 0;
-    const uint32_t* myset = sets + (tq - tf) * kSetWords;
     const float sl2 = p.scale_log2;
     const float thr = 8.0f / sl2;
     RowState st;
     bool alive = true;
-    int rcur = 0;
+    const int slot = qvalid ? tq - tf : 0;
     for (int j = 0; j < n; ++j) {
-      // keys of tile j allowed for this row: those whose frame is in A(tq);
-      // rows between and after the pieces stay masked
-      uint32_t vm[4] = {0u, 0u, 0u, 0u};
-      first_run(j, rcur);
-      if (qvalid) {
-        for (int r = rcur; r < nruns && run_v[r] < (j + 1) * kTile; ++r) {
-          const int a = max(j * kTile, run_v[r]), e = min((j + 1) * kTile, run_v[r] + run_len[r]);
-          if (e <= a) continue;
-          const int k0 = run_tok[r] + (a - run_v[r]), kn = e - a, o = a - j * kTile;
-          int f = (int)p.divP.div((uint32_t)k0);
-          int lo = 0, fend = (f + 1) * p.P - k0;
-          while (lo < kn) {
-            const int hi = min(kn, fend);
-            if (f < p.T && bit_of(myset, f)) set_range(vm, o + lo, o + hi);
-            lo = hi;
-            ++f;
-            fend += p.P;
-          }
-        }
+      // keys of tile j allowed for this row (those whose frame is in A(tq)),
+      // from the mask warp
+      const int r = j % kMaskRing;
+      if (!__all_sync(kFullMask, bounded_wait(&mask_full[r], (j / kMaskRing) & 1, wc))) {
+        alive = false;
+        break;
       }
+      const uint4 mv = masks[r * kMaxRowFrames + slot];
+      const uint32_t vm[4] = {qvalid ? mv.x : 0u, qvalid ? mv.y : 0u, qvalid ? mv.z : 0u,
+                              qvalid ? mv.w : 0u};
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&mask_empty[r]);
       if (!__all_sync(kFullMask, bounded_wait(&s_full[g], j & 1, wc))) {
         alive = false;
         break;
