@@ -48,11 +48,11 @@ METRIC = "bsattn ms/call + attended TFLOP/s (% BF16 peak), Wan-1.3B-shape 6× le
 
 # DRAM bytes per launch of the LVSA step kernel at the full Wan-1.3B 6x
 # workload: dram__bytes_read.sum + dram__bytes_write.sum of one ncu capture of
-# the same kernel on the first 24 frames (450.6 MB), scaled by the number of
+# the same kernel on the first 24 frames (445.7 MB), scaled by the number of
 # query pairs (126 / 24).  None whenever the kernel has changed since.
-STEP_KERNEL_DRAM_BYTES = 450.6e6 * 126 / 24
-STEP_KERNEL_TRAFFIC_SOURCE = ("ncu capture of lvsa_attn_kernel (runs packed into key tiles) "
-                              "on the first 24 frames (450.6 MB), scaled by 126/24; not "
+STEP_KERNEL_DRAM_BYTES = 445.7e6 * 126 / 24
+STEP_KERNEL_TRAFFIC_SOURCE = ("ncu capture of lvsa_attn_kernel (key masks from the mask warp) "
+                              "on the first 24 frames (445.7 MB), scaled by 126/24; not "
                               "measured by this run")
 
 
