@@ -103,6 +103,8 @@ struct ListHead {
 };
 
 struct DraftParams {
+  int slot;       // 1: [B, Hh, Npad, D] slot tensors, tile kt = slots 128 kt ..
+  int64_t Npad;   //    (slot mode) slots per (b, head)
   int B, Hh, T, H, W, N, TW, TH, ph, pw;
   int64_t nblocks, ntiles, total_tiles;
   const int32_t* row_ptr;
@@ -396,11 +398,17 @@ __global__ void __launch_bounds__(kThreads, 1)
           // Q of this tile once the last QK of the previous one has completed
           if (!__all_sync(kAll, bounded_wait(q_empty, (uint32_t)(i & 1) ^ 1u, wc))) break;
           if (elect_one()) {
-            int x0, y0, fr;
-            nat_coords(qt, b, x0, y0, fr);
             mbar_arrive_expect_tx(q_full, Cfg::kTileBytes);
-            for (int c = 0; c < Cfg::kChunks; ++c)
-              tma_load_5d(sQ + c * Cfg::kPanel, &tmq, q_full, c * 64, h, x0, y0, fr);
+            if (p.slot) {
+              const int row0 = (int)(((int64_t)b * p.Hh + h) * p.Npad + (int64_t)qt * kTile);
+              for (int c = 0; c < Cfg::kChunks; ++c)
+                tma_load_2d(sQ + c * Cfg::kPanel, &tmq, q_full, c * 64, row0);
+            } else {
+              int x0, y0, fr;
+              nat_coords(qt, b, x0, y0, fr);
+              for (int c = 0; c < Cfg::kChunks; ++c)
+                tma_load_5d(sQ + c * Cfg::kPanel, &tmq, q_full, c * 64, h, x0, y0, fr);
+            }
           }
           __syncwarp();
           issued_q = i + 1;
@@ -451,11 +459,17 @@ __global__ void __launch_bounds__(kThreads, 1)
               kt = ok ? c : 0;
             }
             if (elect_one()) {
-              int x0, y0, fr;
-              nat_coords(kt, b, x0, y0, fr);
               mbar_arrive_expect_tx(&full[st], Cfg::kTileBytes);
-              for (int c = 0; c < Cfg::kChunks; ++c)
-                tma_load_5d(dst + c * Cfg::kPanel, tmx, &full[st], c * 64, h, x0, y0, fr);
+              if (p.slot) {
+                const int row0 = (int)(((int64_t)b * p.Hh + h) * p.Npad + (int64_t)kt * kTile);
+                for (int c = 0; c < Cfg::kChunks; ++c)
+                  tma_load_2d(dst + c * Cfg::kPanel, tmx, &full[st], c * 64, row0);
+              } else {
+                int x0, y0, fr;
+                nat_coords(kt, b, x0, y0, fr);
+                for (int c = 0; c < Cfg::kChunks; ++c)
+                  tma_load_5d(dst + c * Cfg::kPanel, tmx, &full[st], c * 64, h, x0, y0, fr);
+              }
             }
           }
           __syncwarp();
@@ -691,20 +705,33 @@ __global__ void __launch_bounds__(kThreads, 1)
       const float a = (nA > 0 && mA != -INFINITY) ? ex2_approx((mA - m) * sl2) : 0.f;
       const float bb = (nB > 0 && mB != -INFINITY) ? ex2_approx((mB - m) * sl2) : 0.f;
       const float l = lA * a + lB * bb;
-      // slot (y, x) of tile (t, i, j) is token (t, y0 + y, x0 + x); slots
-      // past the grid's right or bottom edge hold no token
-      int x0, y0, fr;
-      nat_coords(qt, b, x0, y0, fr);
-      const int ay = (int)p.div_pw.div((uint32_t)row);
-      const int yy = y0 + ay, xx = x0 + (row - ay * p.pw);
-      const bool qvalid = ay < p.ph && yy < p.H && xx < p.W;
+      bool qvalid;
+      int64_t orow, lrow;
+      if (p.slot) {
+        // slot tensors: row `row` of tile qt; an empty slot is written as 0
+        // (LSE -inf) like every slot of the layout
+        const uint4 tq = __ldg(reinterpret_cast<const uint4*>(p.tile_valid) + qt);
+        const uint32_t qw = (row < 32) ? tq.x : (row < 64) ? tq.y : (row < 96) ? tq.z : tq.w;
+        qvalid = (qw >> (row & 31)) & 1u;
+        orow = ((int64_t)b * p.Hh + h) * p.Npad + (int64_t)qt * kTile + row;
+        lrow = orow;
+      } else {
+        // slot (y, x) of tile (t, i, j) is token (t, y0 + y, x0 + x); slots
+        // past the grid's right or bottom edge hold no token
+        int x0, y0, fr;
+        nat_coords(qt, b, x0, y0, fr);
+        const int ay = (int)p.div_pw.div((uint32_t)row);
+        const int yy = y0 + ay, xx = x0 + (row - ay * p.pw);
+        qvalid = ay < p.ph && yy < p.H && xx < p.W;
+        const int t = fr - b * p.T;
+        const int64_t ntok = ((int64_t)t * p.H + yy) * p.W + xx;
+        orow = ((int64_t)b * p.N + ntok) * p.Hh + h;
+        lrow = ((int64_t)b * p.Hh + h) * p.N + ntok;
+      }
+      const bool write = qvalid || p.slot;
       const bool has = n > 0 && qvalid && l > 0.f;
       const float inv_l = has ? 1.f / l : 0.f;
       const float wa = a * inv_l, wb = bb * inv_l;
-      const int t = fr - b * p.T;
-      const int64_t ntok = ((int64_t)t * p.H + yy) * p.W + xx;
-      const int64_t orow = ((int64_t)b * p.N + ntok) * p.Hh + h;
-      const int64_t lrow = ((int64_t)b * p.Hh + h) * p.N + ntok;
       // group g stores columns [g*D/2, (g+1)*D/2) of its rows
       uint4* dst = reinterpret_cast<uint4*>(p.o + orow * D + g * (D / 2));
       const uint32_t oA = tbase + 256 + lane_off + g * (D / 2);
@@ -724,13 +751,13 @@ __global__ void __launch_bounds__(kThreads, 1)
               has ? __uint_as_float(xa[2 * e + 1]) * wa + __uint_as_float(xb[2 * e + 1]) * wb : 0.f;
           w16[e] = pack_bf16x2(v0, v1);
         }
-        if (qvalid) {
+        if (write) {
 #pragma unroll
           for (int e = 0; e < 4; ++e)
             dst[c * 4 + e] = make_uint4(w16[4 * e], w16[4 * e + 1], w16[4 * e + 2], w16[4 * e + 3]);
         }
       }
-      if (g == 0 && p.lse && qvalid) p.lse[lrow] = has ? m * p.scale + logf(l) : -INFINITY;
+      if (g == 0 && p.lse && write) p.lse[lrow] = has ? m * p.scale + logf(l) : -INFINITY;
       tc_fence_before();
       mbar_arrive(o_free);
     }
@@ -769,6 +796,20 @@ bool make_draft_tmap(CUtensorMap* m, const void* ptr, const Geometry& g, int box
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// Slot tensors [B, Hh, Npad, D] bf16 as a 2-D [B*Hh*Npad, D] tensor; boxes of
+// 64 channels x 128 slots, 128-byte swizzle.
+bool make_slot_tmap(CUtensorMap* m, const void* ptr, int64_t rows, int D) {
+  auto fn = draft_encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {(cuuint64_t)D, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)D * 2};
+  cuuint32_t box[2] = {64, (cuuint32_t)kTile};
+  cuuint32_t estr[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides, box,
+            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 int draft_sm_count() {
   static int n[64] = {};
   int dev = 0;
@@ -800,20 +841,33 @@ cudaError_t launch_draft_t(const CUtensorMap& q, const CUtensorMap& k, const CUt
 
 bsa_status launch_attn_draft(const bsa_plan_s& plan, const void* q, const void* k, const void* v,
                              const int32_t* row_ptr, const int32_t* col_idx, int per_head,
-                             float scale, void* o, float* lse, cudaStream_t st) {
+                             float scale, void* o, float* lse, cudaStream_t st, bool slot) {
   const Geometry& g = plan.g;
-  if (g.layout != BSA_LAYOUT_TILE || g.block != kTile)
-    return set_error(BSA_ERR_UNSUPPORTED,
-                     "natural-layout attention needs a TILE plan with pool_h * pool_w = 128");
-  if ((int64_t)g.B * g.T * g.P * g.Hh >= (1ll << 31))
-    return set_error(BSA_ERR_UNSUPPORTED, "B*N*Hh must be < 2^31");
-  if ((int64_t)g.B * g.T >= (1ll << 31)) return set_error(BSA_ERR_UNSUPPORTED, "B*T must be < 2^31");
   CUtensorMap tq, tk, tv;
-  if (!make_draft_tmap(&tq, q, g, g.pw, g.ph) || !make_draft_tmap(&tk, k, g, g.pw, g.ph) ||
-      !make_draft_tmap(&tv, v, g, g.pw, g.ph))
-    return set_error(BSA_ERR_CUDA, "cuTensorMapEncodeTiled (5-D) failed");
+  if (slot) {
+    if (g.block != kTile)
+      return set_error(BSA_ERR_UNSUPPORTED, "slot-layout persistent attention needs 128-slot blocks");
+    const int64_t rows = (int64_t)g.B * g.Hh * g.Npad;
+    if (rows >= (1ll << 31)) return set_error(BSA_ERR_UNSUPPORTED, "B*Hh*Npad must be < 2^31");
+    if (!make_slot_tmap(&tq, q, rows, g.D) || !make_slot_tmap(&tk, k, rows, g.D) ||
+        !make_slot_tmap(&tv, v, rows, g.D))
+      return set_error(BSA_ERR_CUDA, "cuTensorMapEncodeTiled (2-D) failed");
+  } else {
+    if (g.layout != BSA_LAYOUT_TILE || g.block != kTile)
+      return set_error(BSA_ERR_UNSUPPORTED,
+                       "natural-layout attention needs a TILE plan with pool_h * pool_w = 128");
+    if ((int64_t)g.B * g.T * g.P * g.Hh >= (1ll << 31))
+      return set_error(BSA_ERR_UNSUPPORTED, "B*N*Hh must be < 2^31");
+    if ((int64_t)g.B * g.T >= (1ll << 31))
+      return set_error(BSA_ERR_UNSUPPORTED, "B*T must be < 2^31");
+    if (!make_draft_tmap(&tq, q, g, g.pw, g.ph) || !make_draft_tmap(&tk, k, g, g.pw, g.ph) ||
+        !make_draft_tmap(&tv, v, g, g.pw, g.ph))
+      return set_error(BSA_ERR_CUDA, "cuTensorMapEncodeTiled (5-D) failed");
+  }
   DraftParams p;
   memset(&p, 0, sizeof(p));
+  p.slot = slot ? 1 : 0;
+  p.Npad = g.Npad;
   p.B = g.B;
   p.Hh = g.Hh;
   p.T = g.T;
@@ -838,11 +892,22 @@ bsa_status launch_attn_draft(const bsa_plan_s& plan, const void* q, const void* 
   p.tile_valid = plan.d_tile_valid;
   p.status = plan.d_status;
   p.wait_limit_ns = plan.wait_limit_ns;
+  DraftEdgeMaps em;
+  memset(&em, 0, sizeof(em));
+  if (slot) {
+    // key tiles as stored (empty slots masked), no packing; the tile-grid
+    // divisors are unused
+    p.div_tile_frame = FastDiv(1u);
+    p.div_TW = FastDiv(1u);
+    p.div_pw = FastDiv(1u);
+    const cudaError_t e = g.D == 128 ? launch_draft_t<128>(tq, tk, tv, p, em, st)
+                                     : launch_draft_t<64>(tq, tk, tv, p, em, st);
+    if (e != cudaSuccess) return cuda_error(e, "draft attention launch");
+    return BSA_OK;
+  }
   p.div_tile_frame = FastDiv((uint32_t)(g.TH * g.TW));
   p.div_TW = FastDiv((uint32_t)g.TW);
   p.div_pw = FastDiv((uint32_t)g.pw);
-  DraftEdgeMaps em;
-  memset(&em, 0, sizeof(em));
   int kind[3] = {0, 0, 0}, rows[3] = {0, 0, 0}, bw[3] = {0, 0, 0}, bh[3] = {0, 0, 0};
   const int nk = edge_kinds(g, kind, rows, bw, bh);
   if (nk > 0 && g.nblocks < 32768) {

@@ -1021,6 +1021,11 @@ bsa_status launch_attn_fwd(const bsa_plan_s& plan, const void* q, const void* k,
   // CTA share every key tile (attn_pair.cu)
   if (attn_pair_applies(g, per_head))
     return launch_attn_pair(plan, q, k, v, row_ptr, col_idx, scale, o, lse, st);
+  // a list per (batch, head), 128-slot blocks: the persistent kernel of
+  // attn_draft.cu, one CTA per SM over all query tiles
+  if (per_head && g.block == kTile)
+    return launch_attn_draft(plan, q, k, v, row_ptr, col_idx, per_head, scale, o, lse, st,
+                             /*slot=*/true);
   const int64_t rows = (int64_t)g.B * g.Hh * g.Npad;
   if (rows >= (1ll << 31)) return set_error(BSA_ERR_UNSUPPORTED, "B*Hh*Npad must be < 2^31");
   const bool fine = g.block < kTile;

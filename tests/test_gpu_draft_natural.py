@@ -157,6 +157,28 @@ def test_attn_natural_long_lists_run_unpacked():
     assert m.any() and err.max() <= MAX_ABS and err.mean() <= MEAN_ABS
 
 
+@pytest.mark.parametrize("T", [256, 300])
+def test_attn_natural_lists_at_and_past_the_bin_limit(T):
+    # a 6 x 10 frame is one corner tile of 60 tokens (8 x 16 tiles): two
+    # pieces fit a 128-row MMA tile, so a list keeping every block of T
+    # frames needs T / 2 packed tiles - 128 at T = 256, the most a list
+    # buffer holds, and 150 at T = 300, where the list runs unpacked
+    w = small_workload(CONFIGS[2], T=T, H=6, W=10, Hh=1, D=64, draft_sparsity=0,
+                       field_grid=(16, 2, 3))
+    q, k, v = make_qkv(w, device="cuda")
+    att = DraftAttention(w.B, w.Hh, w.D, w.T, w.H, w.W, 8, 16, 0)
+    assert att.plan.nblocks == T and att.keep == T
+    out = att.fused(q, k, v)
+    bsa.bsa_poll_status(att.plan)
+    kv = att.col_idx.view(1, 1, T, -1).cpu().numpy()
+    assert (kv == np.arange(T)).all()
+    ref, _ = _oracle_natural(w, q, k, v, kv, [0], q_blocks=[0, 1, T // 2, T - 1])
+    got = to_np64(out)
+    m = np.isfinite(ref)
+    err = np.abs(got[m] - ref[m])
+    assert m.any() and err.max() <= MAX_ABS and err.mean() <= MEAN_ABS
+
+
 @pytest.mark.parametrize("cid", [2, 5])
 def test_attn_natural_full_size_sampled_vs_oracle(cid):
     w = CONFIGS[cid]
