@@ -124,6 +124,33 @@ __device__ __forceinline__ void softmax_exp(const float (&s)[NC], float sl2, uin
   }
 }
 
+// Two floats to two e4m3 bytes (nearest, ties to even, saturating at +-448),
+// lo in the low byte.
+__device__ __forceinline__ uint32_t pack_e4m3x2(float lo, float hi) {
+  uint16_t r;
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+
+// softmax_exp for 8-bit P: keys [OFF, OFF + 64) as e4m3, four to a word
+// (P <= 2^8 < 448), into pk[0 .. 16); the sums take the unrounded values.
+template <int OFF, int NC>
+__device__ __forceinline__ void softmax_exp_e4m3(const float (&s)[NC], float sl2, uint64_t neg_ms2,
+                                                 uint32_t (&pk)[16], uint64_t (&acc)[4]) {
+  const uint64_t scale2 = f2(sl2, sl2);
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    float x0, x1, x2, x3;
+    unf2(ffma2(f2(s[OFF + 4 * i], s[OFF + 4 * i + 1]), scale2, neg_ms2), x0, x1);
+    unf2(ffma2(f2(s[OFF + 4 * i + 2], s[OFF + 4 * i + 3]), scale2, neg_ms2), x2, x3);
+    const float p0 = ex2_approx(x0), p1 = ex2_approx(x1);
+    const float p2 = ex2_approx(x2), p3 = ex2_approx(x3);
+    acc[(2 * i) & 3] = fadd2(acc[(2 * i) & 3], f2(p0, p1));
+    acc[(2 * i + 1) & 3] = fadd2(acc[(2 * i + 1) & 3], f2(p2, p3));
+    pk[i] = pack_e4m3x2(p0, p1) | (pack_e4m3x2(p2, p3) << 16);
+  }
+}
+
 // Adds the packed partial sums to the row's running sum.
 __device__ __forceinline__ void softmax_sum(RowState& st, const uint64_t (&acc)[4]) {
   const uint64_t a = fadd2(fadd2(acc[0], acc[1]), fadd2(acc[2], acc[3]));

@@ -62,14 +62,18 @@ constexpr int kMaxBins = 128;           // packed tiles of edge pieces a list ca
 constexpr uint16_t kBad = 0xffffu;      // packed-list marker of an out-of-range entry
 constexpr uint32_t kAll = 0xffffffffu;
 
-template <int D>
+template <int D, bool F8>
 struct DraftCfg {
-  static constexpr int kChunks = D / 64;          // 128-byte swizzle panels
+  static constexpr int kElem = F8 ? 1 : 2;         // bytes per element
+  static constexpr int kChunkElems = 128 / kElem;  // elements per 128-byte swizzle row
+  static constexpr int kChunks = D / kChunkElems;  // 128-byte swizzle panels
   static constexpr int kPanel = kTile * 128;
-  static constexpr int kTileBytes = kTile * D * 2;
-  // K and V have rings of their own: K is needed a softmax earlier than V
-  // (QK of the next tile is issued before PV of this one), so it runs deeper
-  static constexpr int NK = 3, NV = 2;
+  static constexpr int kTileBytes = kTile * D * kElem;
+  static constexpr int kKeysPerMma = 32 / kElem;   // K of one MMA: 16 (bf16) or 32 (e4m3)
+  static constexpr int kPHalfCols = 16 * kElem;    // TMEM columns of 64 keys of P
+  // K and V have rings of their own: K is needed a softmax earlier than V,
+  // so it runs deeper; 8-bit tiles are half the size and both run deeper
+  static constexpr int NK = F8 ? 4 : 3, NV = F8 ? 4 : 2;
   static constexpr int kOffQ = 0;
   static constexpr int kOffK = kTileBytes;
   static constexpr int kOffV = kOffK + NK * kTileBytes;
@@ -114,6 +118,7 @@ struct DraftParams {
   float scale, scale_log2;
   __nv_bfloat16* o;
   float* lse;
+  const float* fp8_scales;  // 8-bit tiles: [3][B][Hh] scales of Q, K, V
   const uint32_t* tile_valid;
   unsigned int* status;
   uint64_t wait_limit_ns;
@@ -148,12 +153,13 @@ __device__ __forceinline__ void next_bin(const DraftParams& p, int (&r)[3], int 
 
 __device__ __forceinline__ void end_sync() { asm volatile("bar.sync 2, 384;" ::: "memory"); }
 
-template <int D>
+template <int D, bool F8>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_draft_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmk,
                       const __grid_constant__ CUtensorMap tmv, const DraftParams p,
                       const __grid_constant__ DraftEdgeMaps em) {
-  using Cfg = DraftCfg<D>;
+  using Cfg = DraftCfg<D, F8>;
+  static_assert(!F8 || D == 128, "8-bit tiles: D = 128");
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
@@ -402,12 +408,12 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (p.slot) {
               const int row0 = (int)(((int64_t)b * p.Hh + h) * p.Npad + (int64_t)qt * kTile);
               for (int c = 0; c < Cfg::kChunks; ++c)
-                tma_load_2d(sQ + c * Cfg::kPanel, &tmq, q_full, c * 64, row0);
+                tma_load_2d(sQ + c * Cfg::kPanel, &tmq, q_full, c * Cfg::kChunkElems, row0);
             } else {
               int x0, y0, fr;
               nat_coords(qt, b, x0, y0, fr);
               for (int c = 0; c < Cfg::kChunks; ++c)
-                tma_load_5d(sQ + c * Cfg::kPanel, &tmq, q_full, c * 64, h, x0, y0, fr);
+                tma_load_5d(sQ + c * Cfg::kPanel, &tmq, q_full, c * Cfg::kChunkElems, h, x0, y0, fr);
             }
           }
           __syncwarp();
@@ -439,8 +445,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                   nat_coords(ent[pstart[e] + pptr[e] + m], b, x0, y0, fr);
                   const CUtensorMap* mx = isK ? &em.k[p.pk_kind[e] - 1] : &em.v[p.pk_kind[e] - 1];
                   for (int c = 0; c < Cfg::kChunks; ++c)
-                    tma_load_5d(dst + c * Cfg::kPanel + off * 128, mx, &full[st], c * 64, h, x0, y0,
-                                fr);
+                    tma_load_5d(dst + c * Cfg::kPanel + off * 128, mx, &full[st],
+                                c * Cfg::kChunkElems, h, x0, y0, fr);
                   off += p.pk_step[e];
                 }
               }
@@ -463,12 +469,12 @@ __global__ void __launch_bounds__(kThreads, 1)
               if (p.slot) {
                 const int row0 = (int)(((int64_t)b * p.Hh + h) * p.Npad + (int64_t)kt * kTile);
                 for (int c = 0; c < Cfg::kChunks; ++c)
-                  tma_load_2d(dst + c * Cfg::kPanel, tmx, &full[st], c * 64, row0);
+                  tma_load_2d(dst + c * Cfg::kPanel, tmx, &full[st], c * Cfg::kChunkElems, row0);
               } else {
                 int x0, y0, fr;
                 nat_coords(kt, b, x0, y0, fr);
                 for (int c = 0; c < Cfg::kChunks; ++c)
-                  tma_load_5d(dst + c * Cfg::kPanel, tmx, &full[st], c * 64, h, x0, y0, fr);
+                  tma_load_5d(dst + c * Cfg::kPanel, tmx, &full[st], c * Cfg::kChunkElems, h, x0, y0, fr);
               }
             }
           }
@@ -489,8 +495,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       __syncwarp();
     } else if (warp == 1) {
       // ------------------------------------------------------ MMA issuer
-      constexpr uint32_t idesc_qk = idesc_bf16(128, 128, 0);
-      constexpr uint32_t idesc_pv = idesc_bf16(128, D, 1);
+      constexpr uint32_t idesc_qk = F8 ? idesc_e4m3(128, 128, 0) : idesc_bf16(128, 128, 0);
+      constexpr uint32_t idesc_pv = F8 ? idesc_e4m3(128, D, 1) : idesc_bf16(128, D, 1);
       const uint64_t qd = sdesc_sw128(smem_u32(sQ), 16, 1024);
       const uint64_t kd0 = sdesc_sw128(smem_u32(smem + Cfg::kOffK), 16, 1024);
       const uint64_t vd0 = sdesc_sw128(smem_u32(smem + Cfg::kOffV), Cfg::kPanel, 1024);
@@ -498,9 +504,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint64_t kd = sdesc_add(kd0, st * Cfg::kTileBytes);  // K ring stage
         if (elect_one()) {
 #pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
+          for (int kk = 0; kk < D / Cfg::kKeysPerMma; ++kk) {
+            // K step kk: 32 bytes along the 128-byte swizzle row, then the next panel
             const uint32_t off = (kk >> 2) * Cfg::kPanel + (kk & 3) * 32;
-            mma_ss(tdst, sdesc_add(qd, off), sdesc_add(kd, off), idesc_qk, kk > 0);
+            if constexpr (F8)
+              mma_ss_f8(tdst, sdesc_add(qd, off), sdesc_add(kd, off), idesc_qk, kk > 0);
+            else
+              mma_ss(tdst, sdesc_add(qd, off), sdesc_add(kd, off), idesc_qk, kk > 0);
           }
         }
         __syncwarp();
@@ -508,12 +518,20 @@ __global__ void __launch_bounds__(kThreads, 1)
       // O_g (+)= P(keys 64 * half .. + 63) . V(same keys)
       auto issue_pv = [&](int st, int g, int half, uint32_t acc) {
         const uint64_t vd = sdesc_add(vd0, st * Cfg::kTileBytes + half * 64 * 128);
-        const uint32_t tP = tbase + g * 128 + 64 + half * 32, tO = tbase + 256 + g * 128;
+        const uint32_t tP = tbase + g * 128 + 64 + half * Cfg::kPHalfCols;
+        const uint32_t tO = tbase + 256 + g * 128;
         if (elect_one()) {
+          // K step kk: the next kKeysPerMma keys = 8 TMEM columns of P and
+          // kKeysPerMma 128-byte rows of V
 #pragma unroll
-          for (int kk = 0; kk < 4; ++kk)
-            mma_ts(tO, tP + kk * 8, sdesc_add(vd, kk * 16 * 128), idesc_pv,
-                   (acc | (uint32_t)half | (uint32_t)kk) != 0);
+          for (int kk = 0; kk < 64 / Cfg::kKeysPerMma; ++kk) {
+            const uint64_t bd = sdesc_add(vd, kk * Cfg::kKeysPerMma * 128);
+            const uint32_t on = (acc | (uint32_t)half | (uint32_t)kk) != 0;
+            if constexpr (F8)
+              mma_ts_f8(tO, tP + kk * 8, bd, idesc_pv, on);
+            else
+              mma_ts(tO, tP + kk * 8, bd, idesc_pv, on);
+          }
         }
         __syncwarp();
       };
@@ -594,8 +612,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t lane_off = (uint32_t)(q4 * 32) << 16;
     const uint32_t tS = tbase + g * 128 + lane_off;
     const uint32_t tO = tbase + 256 + g * 128 + lane_off;
-    const float sl2 = p.scale_log2;
-    const float thr = 8.0f / sl2;  // rescale O when the max grows by more than 2^8
+    float sl2 = p.scale_log2;
+    float thr = 8.0f / sl2;  // rescale O when the max grows by more than 2^8
     int64_t scount = 0;            // S buffers of this group consumed so far
     bool alive = true;
     for (int64_t i = 0; i < my_tiles; ++i) {
@@ -609,6 +627,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       int qt, h, b;
       tile_of(i, qt, h, b);
       const int n = hd.n;
+      // 8-bit tiles: S holds q8.k8, the scores are S * sq * sk; O holds
+      // P.v8, the values are O * sv
+      float sqk = 1.f, sv = 1.f;
+      if (F8) {
+        sqk = p.fp8_scales[(int64_t)b * p.Hh + h] * p.fp8_scales[((int64_t)p.B + b) * p.Hh + h];
+        sv = p.fp8_scales[(2 * (int64_t)p.B + b) * p.Hh + h];
+        sl2 = p.scale_log2 * sqk;
+        thr = 8.0f / sl2;
+      }
       RowState rs;
       for (int j = g; j < n; j += 2) {
         uint32_t vm[4] = {0u, 0u, 0u, 0u};
@@ -656,7 +683,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                               ? softmax_max<128, false>(s, vm, rs, sl2, thr, corr, neg_ms2)
                               : softmax_max<128, true>(s, vm, rs, sl2, thr, corr, neg_ms2);
         uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};
-        {
+        if constexpr (F8) {
+          uint32_t pk[16];
+          softmax_exp_e4m3<0, 128>(s, sl2, neg_ms2, pk, acc);
+          tmem_st16(tS + 64, pk);
+        } else {
           uint32_t pk[32];
           softmax_exp<0, 64>(s, sl2, neg_ms2, pk, acc);
           tmem_st32(tS + 64, pk);
@@ -668,10 +699,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (j >= 2 && __any_sync(kAll, need)) tmem_scale<D>(tO, corr);
         tc_fence_before();
         mbar_arrive(&p_half[g]);
-        {
+        if constexpr (F8) {
+          uint32_t pk[16];
+          softmax_exp_e4m3<64, 128>(s, sl2, neg_ms2, pk, acc);
+          tmem_st16(tS + 64 + Cfg::kPHalfCols, pk);
+        } else {
           uint32_t pk[32];
           softmax_exp<64, 64>(s, sl2, neg_ms2, pk, acc);
-          tmem_st32(tS + 96, pk);
+          tmem_st32(tS + 64 + Cfg::kPHalfCols, pk);
         }
         softmax_sum(rs, acc);
         tc_fence_before();
@@ -730,7 +765,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       const bool write = qvalid || p.slot;
       const bool has = n > 0 && qvalid && l > 0.f;
-      const float inv_l = has ? 1.f / l : 0.f;
+      const float inv_l = has ? sv / l : 0.f;
       const float wa = a * inv_l, wb = bb * inv_l;
       // group g stores columns [g*D/2, (g+1)*D/2) of its rows
       uint4* dst = reinterpret_cast<uint4*>(p.o + orow * D + g * (D / 2));
@@ -757,7 +792,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             dst[c * 4 + e] = make_uint4(w16[4 * e], w16[4 * e + 1], w16[4 * e + 2], w16[4 * e + 3]);
         }
       }
-      if (g == 0 && p.lse && write) p.lse[lrow] = has ? m * p.scale + logf(l) : -INFINITY;
+      if (g == 0 && p.lse && write) p.lse[lrow] = has ? m * (p.scale * sqk) + logf(l) : -INFINITY;
       tc_fence_before();
       mbar_arrive(o_free);
     }
@@ -779,21 +814,24 @@ PFN_cuTensorMapEncodeTiled_v12000 draft_encode_fn() {
   return fn;
 }
 
-// Natural layout [B, N, Hh, D] bf16 as 5-D {D, Hh, W, H, B*T}; boxes of 64
-// channels x 1 head x box_w x box_h x 1 frame, 128-byte swizzle; boxes
-// reaching past W or H read zeros.
-bool make_draft_tmap(CUtensorMap* m, const void* ptr, const Geometry& g, int box_w, int box_h) {
+// Natural layout [B, N, Hh, D] as 5-D {D, Hh, W, H, B*T}; boxes of one
+// 128-byte row of channels (64 bf16 or 128 e4m3) x 1 head x box_w x box_h x
+// 1 frame, 128-byte swizzle; boxes reaching past W or H read zeros.
+bool make_draft_tmap(CUtensorMap* m, const void* ptr, const Geometry& g, int box_w, int box_h,
+                     bool e4m3 = false) {
   auto fn = draft_encode_fn();
   if (!fn) return false;
-  const cuuint64_t row = (cuuint64_t)g.Hh * g.D * 2;
+  const cuuint64_t esz = e4m3 ? 1 : 2;
+  const cuuint64_t row = (cuuint64_t)g.Hh * g.D * esz;
   cuuint64_t dims[5] = {(cuuint64_t)g.D, (cuuint64_t)g.Hh, (cuuint64_t)g.W, (cuuint64_t)g.H,
                         (cuuint64_t)g.B * g.T};
-  cuuint64_t strides[4] = {(cuuint64_t)g.D * 2, row, row * g.W, row * g.W * g.H};
-  cuuint32_t box[5] = {64, 1, (cuuint32_t)box_w, (cuuint32_t)box_h, 1};
+  cuuint64_t strides[4] = {(cuuint64_t)g.D * esz, row, row * g.W, row * g.W * g.H};
+  cuuint32_t box[5] = {(cuuint32_t)(128 / esz), 1, (cuuint32_t)box_w, (cuuint32_t)box_h, 1};
   cuuint32_t estr[5] = {1, 1, 1, 1, 1};
-  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, const_cast<void*>(ptr), dims, strides, box, estr,
-            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+  return fn(m, e4m3 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5,
+            const_cast<void*>(ptr), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+            CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 // Slot tensors [B, Hh, Npad, D] bf16 as a 2-D [B*Hh*Npad, D] tensor; boxes of
@@ -823,15 +861,16 @@ int draft_sm_count() {
   return n[dev];
 }
 
-template <int D>
+template <int D, bool F8 = false>
 cudaError_t launch_draft_t(const CUtensorMap& q, const CUtensorMap& k, const CUtensorMap& v,
                            const DraftParams& p, const DraftEdgeMaps& em, cudaStream_t st) {
-  auto kern = attn_draft_kernel<D>;
+  using Cfg = DraftCfg<D, F8>;
+  auto kern = attn_draft_kernel<D, F8>;
   cudaError_t e =
-      cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, DraftCfg<D>::kSmem);
+      cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::kSmem);
   if (e != cudaSuccess) return e;
   const int64_t grid = std::min<int64_t>(p.total_tiles, draft_sm_count());
-  kern<<<(unsigned)grid, kThreads, DraftCfg<D>::kSmem, st>>>(q, k, v, p, em);
+  kern<<<(unsigned)grid, kThreads, Cfg::kSmem, st>>>(q, k, v, p, em);
   return cudaGetLastError();
 }
 
@@ -841,7 +880,9 @@ cudaError_t launch_draft_t(const CUtensorMap& q, const CUtensorMap& k, const CUt
 
 bsa_status launch_attn_draft(const bsa_plan_s& plan, const void* q, const void* k, const void* v,
                              const int32_t* row_ptr, const int32_t* col_idx, int per_head,
-                             float scale, void* o, float* lse, cudaStream_t st, bool slot) {
+                             float scale, void* o, float* lse, cudaStream_t st, bool slot,
+                             const float* fp8_scales) {
+  const bool f8 = fp8_scales != nullptr;
   const Geometry& g = plan.g;
   CUtensorMap tq, tk, tv;
   if (slot) {
@@ -856,18 +897,20 @@ bsa_status launch_attn_draft(const bsa_plan_s& plan, const void* q, const void* 
     if (g.layout != BSA_LAYOUT_TILE || g.block != kTile)
       return set_error(BSA_ERR_UNSUPPORTED,
                        "natural-layout attention needs a TILE plan with pool_h * pool_w = 128");
+    if (f8 && g.D != 128) return set_error(BSA_ERR_UNSUPPORTED, "e4m3 attention supports D = 128");
     if ((int64_t)g.B * g.T * g.P * g.Hh >= (1ll << 31))
       return set_error(BSA_ERR_UNSUPPORTED, "B*N*Hh must be < 2^31");
     if ((int64_t)g.B * g.T >= (1ll << 31))
       return set_error(BSA_ERR_UNSUPPORTED, "B*T must be < 2^31");
-    if (!make_draft_tmap(&tq, q, g, g.pw, g.ph) || !make_draft_tmap(&tk, k, g, g.pw, g.ph) ||
-        !make_draft_tmap(&tv, v, g, g.pw, g.ph))
+    if (!make_draft_tmap(&tq, q, g, g.pw, g.ph, f8) || !make_draft_tmap(&tk, k, g, g.pw, g.ph, f8) ||
+        !make_draft_tmap(&tv, v, g, g.pw, g.ph, f8))
       return set_error(BSA_ERR_CUDA, "cuTensorMapEncodeTiled (5-D) failed");
   }
   DraftParams p;
   memset(&p, 0, sizeof(p));
   p.slot = slot ? 1 : 0;
   p.Npad = g.Npad;
+  p.fp8_scales = fp8_scales;
   p.B = g.B;
   p.Hh = g.Hh;
   p.T = g.T;
@@ -915,14 +958,15 @@ bsa_status launch_attn_draft(const bsa_plan_s& plan, const void* q, const void* 
       p.pk_kind[i] = kind[i];
       p.pk_rows[i] = rows[i];
       p.pk_step[i] = (rows[i] + 7) / 8 * 8;
-      if (!make_draft_tmap(&em.k[kind[i] - 1], k, g, bw[i], bh[i]) ||
-          !make_draft_tmap(&em.v[kind[i] - 1], v, g, bw[i], bh[i]))
+      if (!make_draft_tmap(&em.k[kind[i] - 1], k, g, bw[i], bh[i], f8) ||
+          !make_draft_tmap(&em.v[kind[i] - 1], v, g, bw[i], bh[i], f8))
         return set_error(BSA_ERR_CUDA, "cuTensorMapEncodeTiled (5-D edge boxes) failed");
     }
     p.pk_on = 1;
   }
-  const cudaError_t e = g.D == 128 ? launch_draft_t<128>(tq, tk, tv, p, em, st)
-                                   : launch_draft_t<64>(tq, tk, tv, p, em, st);
+  const cudaError_t e = f8 ? launch_draft_t<128, true>(tq, tk, tv, p, em, st)
+                       : g.D == 128 ? launch_draft_t<128>(tq, tk, tv, p, em, st)
+                                    : launch_draft_t<64>(tq, tk, tv, p, em, st);
   if (e != cudaSuccess) return cuda_error(e, "draft attention launch");
   return BSA_OK;
 }

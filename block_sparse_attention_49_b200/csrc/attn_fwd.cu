@@ -150,14 +150,6 @@ __device__ __forceinline__ void set_bits(uint32_t (&m)[4], int lo, int len) {
   }
 }
 
-// Two floats to two e4m3 bytes (nearest, ties to even, saturating at +-448),
-// lo in the low byte.
-__device__ __forceinline__ uint32_t pack_e4m3x2(float lo, float hi) {
-  uint16_t r;
-  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
-  return r;
-}
-
 __device__ __forceinline__ void softmax_groups_sync() {
   asm volatile("bar.sync 1, 256;" ::: "memory");  // warps 4-11
 }
@@ -1063,36 +1055,9 @@ bsa_status launch_attn_fwd_natural_e4m3(const bsa_plan_s& plan, const void* q8, 
     return set_error(BSA_ERR_UNSUPPORTED,
                      "e4m3 attention needs a TILE plan with pool_h * pool_w = 128");
   if (g.D != 128) return set_error(BSA_ERR_UNSUPPORTED, "e4m3 attention supports D = 128");
-  if ((int64_t)g.B * g.T * g.P * g.Hh >= (1ll << 31))
-    return set_error(BSA_ERR_UNSUPPORTED, "B*N*Hh must be < 2^31");
-  CUtensorMap tq, tk, tv;
-  if (!make_tmap_tiles(&tq, q8, g, true) || !make_tmap_tiles(&tk, k8, g, true) ||
-      !make_tmap_tiles(&tv, v8, g, true))
-    return set_error(BSA_ERR_CUDA, "cuTensorMapEncodeTiled (5-D, e4m3) failed");
-  AttnParams p = make_params(plan, row_ptr, col_idx, per_head, scale, o, lse);
-  p.fp8_scales = scales;
-  const dim3 grid((unsigned)g.ntiles, (unsigned)g.Hh, (unsigned)g.B);
-  int kind[3] = {0, 0, 0}, rows[3] = {0, 0, 0}, bw[3] = {0, 0, 0}, bh[3] = {0, 0, 0};
-  const int nk = edge_kinds(g, kind, rows, bw, bh);
-  cudaError_t e;
-  if (nk > 0 && g.nblocks < 32768) {
-    EdgeMaps em;
-    memset(&em, 0, sizeof(em));
-    for (int i = 0; i < nk; ++i) {
-      p.pk_kind[i] = kind[i];
-      p.pk_rows[i] = rows[i];
-      p.pk_step[i] = (rows[i] + 7) / 8 * 8;
-      if (!make_tmap_tiles(&em.k[kind[i] - 1], k8, g, true, bw[i], bh[i]) ||
-          !make_tmap_tiles(&em.v[kind[i] - 1], v8, g, true, bw[i], bh[i]))
-        return set_error(BSA_ERR_CUDA, "cuTensorMapEncodeTiled (5-D e4m3 edge boxes) failed");
-    }
-    p.pk_on = 1;
-    e = launch_t<128, false, true, true, true>(tq, tk, tv, p, grid, st, &em);
-  } else {
-    e = launch_t<128, false, true, true>(tq, tk, tv, p, grid, st);
-  }
-  if (e != cudaSuccess) return cuda_error(e, "e4m3 attention launch");
-  return BSA_OK;
+  // e4m3 tiles: the persistent kernel of attn_draft.cu
+  return launch_attn_draft(plan, q8, k8, v8, row_ptr, col_idx, per_head, scale, o, lse, st,
+                           /*slot=*/false, scales);
 }
 
 }  // namespace bsa

@@ -120,9 +120,12 @@ bsa_status launch_attn_fwd_natural(const bsa_plan_s& plan, const void* q, const 
 // The same, persistent (one CTA per SM over all query tiles), bf16 tiles.
 // slot = true: the slot tensors [B, Hh, Npad, D] of any plan with 128-slot
 // blocks instead (LSE as [B, Hh, Npad]; empty slots written as 0 / -inf).
+// fp8_scales != null: natural-layout e4m3 tiles with those [3][B][Hh] scales
+// (8-bit MMAs, P rounded to e4m3; D = 128).
 bsa_status launch_attn_draft(const bsa_plan_s& plan, const void* q, const void* k, const void* v,
                              const int32_t* row_ptr, const int32_t* col_idx, int per_head,
-                             float scale, void* o, float* lse, cudaStream_t st, bool slot = false);
+                             float scale, void* o, float* lse, cudaStream_t st, bool slot = false,
+                             const float* fp8_scales = nullptr);
 // Shared block lists (per_head = 0) with 128-slot blocks: two query tiles per
 // CTA over the union of their rows (attn_pair.cu).
 bool attn_pair_applies(const Geometry& g, int per_head);

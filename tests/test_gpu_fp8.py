@@ -30,7 +30,7 @@ from block_sparse_attention_49_b200 import _build
 from block_sparse_attention_49_b200.pipeline import DraftAttention
 from synth import CONFIGS, make_qkv, small_workload
 
-from gpu_util import sample_blocks, to_np64
+from gpu_util import LSE_ABS, sample_blocks, to_np64
 
 pytestmark = pytest.mark.gpu
 
@@ -131,6 +131,13 @@ def _e4m3_case(w, q_blocks=None, heads=None):
     m = np.isfinite(ref)
     assert m.any()
     err = np.abs(got[m] - ref[m])
+    # the log-sum-exp of the scores on the dequantized values (S * sq * sk
+    # times the softmax scale): P's rounding does not enter it
+    lref = np.nan_to_num(L, nan=np.inf)[:, :, perm]
+    lgot = lse[:, heads].double().cpu().numpy()
+    ml = np.isfinite(lref)
+    assert ml.any()
+    assert np.abs(lgot[ml] - lref[ml]).max() <= LSE_ABS
     return q, k, v, att, out8, err
 
 
