@@ -28,16 +28,11 @@
 // Every wait is bounded; a wait that runs out records a timeout in the
 // plan's status word and the CTA leaves without trapping.
 //
-// Variants of the same body (template flags):
-//   FINE  blocks smaller than 128 slots: each row walks its own CSR row;
-//   NAT   natural-layout [B, N, Hh, D] tensors of a TILE plan whose tiles are
-//         128 slots: each tile is read through a 5-D tensor map (one
-//         pool_h x pool_w tile per box, zero past the grid edge) and O rows
-//         are stored straight to their tokens (the reorder of the Draft
-//         Attention article fused into loads and stores);
-//   F8    (with NAT) e4m3 Q, K, V: 8-bit MMAs (kind::f8f6f4, K = 32), P
-//         rounded to e4m3 in tensor memory, per-(batch, head) scales folded
-//         into the exponent and the final normalisation.
+// FINE (template flag): blocks smaller than 128 slots; each row walks its own
+// CSR row.  Lists of 128-slot blocks run elsewhere: per-head lists and the
+// natural-layout and 8-bit draft paths on the persistent kernel
+// (attn_draft.cu), lists shared by every head on the paired kernel
+// (attn_pair.cu); this kernel keeps shared lists too long for the latter.
 #include <cuda_bf16.h>
 #include <cudaTypedefs.h>
 
@@ -55,20 +50,16 @@ namespace {
 constexpr int kTile = 128;          // query / key tile (slots)
 constexpr int kThreads = 384;
 constexpr int kFineMaxTiles = 2048; // key tiles addressable by the sub-tile-block path
-constexpr int kPackMax = 768;       // key-list entries a CTA can pack (longer lists run unpacked)
-constexpr uint16_t kPackBad = 0xffffu;  // packed-list marker of an out-of-range entry
 constexpr uint32_t kFull = 0xffffffffu;
 
-template <int D, bool FINE, bool F8 = false, bool PACK = false>
+template <int D, bool FINE>
 struct AttnCfg {
-  static constexpr int kElem = F8 ? 1 : 2;           // bytes per element
-  static constexpr int kChunkElems = 128 / kElem;    // elements per 128-byte swizzle row
-  static constexpr int kChunks = D / kChunkElems;    // 128-byte-wide swizzle panels
+  static constexpr int kChunks = D / 64;             // 128-byte-wide swizzle panels
   static constexpr int kPanel = kTile * 128;
-  static constexpr int kQBytes = kTile * D * kElem;
-  static constexpr int kKVBytes = kTile * D * kElem;
-  static constexpr int kKeysPerMma = 32 / kElem;     // K of one MMA: 16 (bf16) or 32 (e4m3)
-  static constexpr int NS = F8 ? 4 : (D == 128) ? (FINE ? 2 : 3) : 4;
+  static constexpr int kQBytes = kTile * D * 2;
+  static constexpr int kKVBytes = kTile * D * 2;
+  static constexpr int kKeysPerMma = 16;             // K of one bf16 MMA
+  static constexpr int NS = (D == 128) ? (FINE ? 2 : 3) : 4;
   static constexpr int kOffQ = 0;
   static constexpr int kOffK = kQBytes;
   static constexpr int kOffV = kOffK + NS * kKVBytes;
@@ -76,9 +67,8 @@ struct AttnCfg {
   static constexpr int kNumBars = 1 + 3 * NS + 2 + 2 + 2 + 1;
   static constexpr int kOffMisc = kOffBar + kNumBars * 8;
   static constexpr int kOffList = kOffMisc + 16;
-  // FINE: the union of key tiles (uint16); PACK: the key list sorted by tile
-  // kind (uint16) followed by four counts
-  static constexpr int kOffBitmap = kOffList + (FINE ? kFineMaxTiles * 2 : PACK ? kPackMax * 2 + 16 : 0);
+  // FINE: the union of key tiles (uint16)
+  static constexpr int kOffBitmap = kOffList + (FINE ? kFineMaxTiles * 2 : 0);
   static constexpr int kBytes = kOffBitmap + (FINE ? kFineMaxTiles / 8 : 0);
   static constexpr int kSmem = kBytes + 1024;  // room to align the base to 1024
   static constexpr uint32_t kTmemCols = 512;   // S_A | S_B | O_A | O_B
@@ -102,44 +92,7 @@ struct AttnParams {
   const uint32_t* tile_valid;  // [ntiles][4]
   unsigned int* status;
   uint64_t wait_limit_ns;
-  // natural layout (NAT): [B, N, Hh, D] in and out; tile = one ph x pw tile
-  int B, T, H, W, N, TW, ph, pw;
-  const float* fp8_scales;  // F8: [3][B][Hh] scales of Q, K, V
-  FastDiv div_tile_frame, div_TW, div_pw;  // by TH*TW, TW, pw
-  // edge-tile packing (PACK): the partial tiles at the grid's right edge
-  // (kind 1), bottom edge (2) and corner (3), in decreasing size
-  int TH;
-  int pk_on;       // some edge kind exists and block indices fit 15 bits
-  int pk_kind[3];  // kind of each slot (0: absent)
-  int pk_rows[3];  // token rows of a tile of that kind
-  int pk_step[3];  // the same rounded up to 8 (row offset step inside a packed tile)
 };
-
-// Tensor maps of the edge kinds (boxes of their exact size), indexed kind - 1.
-struct EdgeMaps {
-  CUtensorMap k[3], v[3];
-};
-
-// Set bits [lo, hi) of a 128-bit mask (0 <= lo <= hi <= 128).
-__device__ __forceinline__ void set_rows(uint32_t (&m)[4], int lo, int hi) {
-#pragma unroll
-  for (int w = 0; w < 4; ++w) {
-    const int a = max(lo, 32 * w), e = min(hi, 32 * w + 32);
-    if (e > a) m[w] |= (e - a == 32 ? kFull : ((1u << (e - a)) - 1u)) << (a - 32 * w);
-  }
-}
-
-// Composition of the next packed tile of edge pieces: take as many pieces of
-// each kind as fit in 128 rows, largest kind first; r[] = pieces left.
-__device__ __forceinline__ void next_bin(const AttnParams& p, int (&r)[3], int (&a)[3]) {
-  int cap = kTile;
-#pragma unroll
-  for (int e = 0; e < 3; ++e) {
-    a[e] = p.pk_step[e] > 0 ? min(r[e], cap / p.pk_step[e]) : 0;
-    cap -= a[e] * p.pk_step[e];
-    r[e] -= a[e];
-  }
-}
 
 // Set bits [lo, lo+len) of a 128-bit mask; lo is a multiple of len, len | 128.
 __device__ __forceinline__ void set_bits(uint32_t (&m)[4], int lo, int len) {
@@ -159,14 +112,11 @@ __device__ __forceinline__ void cta_end_sync() {
   asm volatile("bar.sync 2, 384;" ::: "memory");
 }
 
-template <int D, bool FINE, bool NAT, bool F8 = false, bool PACK = false>
+template <int D, bool FINE>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmk,
-                    const __grid_constant__ CUtensorMap tmv, const AttnParams p,
-                    const __grid_constant__ EdgeMaps em) {
-  using Cfg = AttnCfg<D, FINE, F8, PACK>;
-  static_assert(!PACK || (NAT && !FINE), "edge packing: natural-layout tiles");
-  static_assert(!F8 || (NAT && D == 128), "the e4m3 path reads the natural layout, D = 128");
+                    const __grid_constant__ CUtensorMap tmv, const AttnParams p) {
+  using Cfg = AttnCfg<D, FINE>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
@@ -177,7 +127,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* v_full = k_full + Cfg::NS;
   uint64_t* kv_empty = v_full + Cfg::NS;
   uint64_t* s_full = kv_empty + Cfg::NS;  // [2]: S_A, S_B written
-  uint64_t* p_half = s_full + 2;          // [2]: keys 0..63 of P_A, P_B written (bf16)
+  uint64_t* p_half = s_full + 2;          // [2]: keys 0..63 of P_A, P_B written
   uint64_t* p_ready = p_half + 2;         // [2]: P_A, P_B written (128 arrivals each)
   uint64_t* o_final = p_ready + 2;        // every MMA done
   uint32_t* misc = reinterpret_cast<uint32_t*>(smem + Cfg::kOffMisc);  // tmem, abort, count, skip
@@ -185,20 +135,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint32_t* bitmap = reinterpret_cast<uint32_t*>(smem + Cfg::kOffBitmap);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  static_assert(!(NAT && FINE), "natural-layout tiles are whole ph x pw tiles");
   const int qt = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
   const int64_t bh_row = ((int64_t)b * p.Hh + h) * p.Npad;
-  // natural layout: tile kt of (b, h) is the ph x pw tile (t, i, j); TMA
-  // coordinates {channel, head, x0, y0, frame}; the part past the grid edge
-  // reads as zero (the empty slots of the tile layout)
-  auto nat_coords = [&](int kt, int& x0, int& y0, int& fr) {
-    const int t = (int)p.div_tile_frame.div((uint32_t)kt);
-    const int r = kt - t * (int)p.div_tile_frame.d;
-    const int i = (int)p.div_TW.div((uint32_t)r);
-    x0 = (r - i * p.TW) * p.pw;
-    y0 = i * p.ph;
-    fr = b * p.T + t;
-  };
   const int64_t list = p.per_head ? (int64_t)b * p.Hh + h : 0;
   const WaitCtx wc{p.status, reinterpret_cast<volatile int*>(&misc[1]), p.wait_limit_ns};
 
@@ -286,102 +224,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     n = (int)misc[2];
   }
 
-  // ------------------------------------------- edge packing: sort the list by kind
-  // Full tiles first (list order), then the edge pieces grouped by kind in
-  // decreasing size; every role replays the same packing of those pieces
-  // (next_bin), so no per-tile schedule is stored.
-  uint16_t* plist = tlist;
-  int* pcnt = reinterpret_cast<int*>(smem + Cfg::kOffList + kPackMax * 2);  // nF, c0, c1, c2
-  bool packed = false;
-  int nF = 0, pc[3] = {0, 0, 0};
-  if constexpr (PACK) {
-    packed = p.pk_on && n > 0 && n <= kPackMax;
-    if (packed) {
-      if (warp == 2) {
-        const int TT = (int)p.div_tile_frame.d;
-        auto kind_of = [&](int c) {
-          const int rr = c % TT, i = rr / p.TW, jj = rr - i * p.TW;
-          const int right = (jj == p.TW - 1 && p.W - jj * p.pw < p.pw) ? 1 : 0;
-          const int bottom = (i == p.TH - 1 && p.H - i * p.ph < p.ph) ? 2 : 0;
-          return right | bottom;
-        };
-        int cF = 0, ce[3] = {0, 0, 0};
-        for (int base = 0; base < n; base += 32) {
-          const int i = base + lane;
-          int kind = -1;
-          if (i < n) {
-            const int c = __ldg(p.col_idx + rs + i);
-            kind = (c >= 0 && (int64_t)c < p.nblocks) ? kind_of(c) : 0;
-          }
-          cF += __popc(__ballot_sync(kFull, kind == 0));
-#pragma unroll
-          for (int e = 0; e < 3; ++e)
-            ce[e] += __popc(__ballot_sync(kFull, kind > 0 && kind == p.pk_kind[e]));
-        }
-        int wF = 0, we[3] = {0, 0, 0};
-        const int start[3] = {cF, cF + ce[0], cF + ce[0] + ce[1]};
-        const uint32_t lt = (1u << lane) - 1u;
-        bool bad = false;
-        for (int base = 0; base < n; base += 32) {
-          const int i = base + lane;
-          int kind = -1;
-          uint16_t val = 0;
-          if (i < n) {
-            const int c = __ldg(p.col_idx + rs + i);
-            const bool ok = c >= 0 && (int64_t)c < p.nblocks;
-            bad |= !ok;
-            kind = ok ? kind_of(c) : 0;
-            val = ok ? (uint16_t)c : kPackBad;
-          }
-          const uint32_t bF = __ballot_sync(kFull, kind == 0);
-          int pos = kind == 0 ? wF + __popc(bF & lt) : 0;
-          wF += __popc(bF);
-#pragma unroll
-          for (int e = 0; e < 3; ++e) {
-            const uint32_t be = __ballot_sync(kFull, kind > 0 && kind == p.pk_kind[e]);
-            if (kind > 0 && kind == p.pk_kind[e]) pos = start[e] + we[e] + __popc(be & lt);
-            we[e] += __popc(be);
-          }
-          if (i < n) plist[pos] = val;
-        }
-        if (__any_sync(kFull, bad) && lane == 0) atomicOr(p.status, kStatusBadBlocklist);
-        if (lane == 0) {
-          pcnt[0] = cF;
-          pcnt[1] = ce[0];
-          pcnt[2] = ce[1];
-          pcnt[3] = ce[2];
-        }
-      }
-      // stale rows of a packed tile are masked, but P = 0 times a value must
-      // stay 0: start every V stage at zero (finite)
-      for (int i = threadIdx.x; i < Cfg::NS * Cfg::kKVBytes / 16; i += kThreads)
-        reinterpret_cast<uint4*>(smem + Cfg::kOffV)[i] = make_uint4(0u, 0u, 0u, 0u);
-      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-      __syncthreads();
-      nF = pcnt[0];
-      pc[0] = pcnt[1];
-      pc[1] = pcnt[2];
-      pc[2] = pcnt[3];
-      // packed tiles: the full ones plus the bins of edge pieces
-      int r[3] = {pc[0], pc[1], pc[2]}, a[3];
-      int nb = 0;
-      while (r[0] + r[1] + r[2] > 0) {
-        next_bin(p, r, a);
-        ++nb;
-      }
-      n = nF + nb;
-    }
-  }
-
   auto tile_of = [&](int j, bool& ok) -> int {
     if (FINE) {
       ok = true;
       return tlist[j];
-    }
-    if (PACK && packed) {  // a full tile of the sorted list (j < nF)
-      const uint16_t c = plist[j];
-      ok = c != kPackBad;
-      return ok ? c : 0;
     }
     const int c = __ldg(p.col_idx + rs + j);
     ok = (c >= 0 && (int64_t)c < p.nblocks);
@@ -396,95 +242,29 @@ __global__ void __launch_bounds__(kThreads, 1)
       // the whole warp runs the loop (warp-uniform operands); one lane issues
       if (elect_one()) {
         mbar_arrive_expect_tx(q_full, Cfg::kQBytes);
-        if constexpr (NAT) {
-          int x0, y0, fr;
-          nat_coords(qt, x0, y0, fr);
-          for (int c = 0; c < Cfg::kChunks; ++c)
-            tma_load_5d(sQ + c * Cfg::kPanel, &tmq, q_full, c * Cfg::kChunkElems, h, x0, y0, fr);
-        } else {
-          for (int c = 0; c < Cfg::kChunks; ++c)
-            tma_load_2d(sQ + c * Cfg::kPanel, &tmq, q_full, c * 64,
-                        (int)(bh_row + (int64_t)qt * kTile));
-        }
+        for (int c = 0; c < Cfg::kChunks; ++c)
+          tma_load_2d(sQ + c * Cfg::kPanel, &tmq, q_full, c * 64,
+                      (int)(bh_row + (int64_t)qt * kTile));
       }
       __syncwarp();
       int issued = 0;
-      // packed bins: pieces left per kind, their region starts and cursors
-      int prem[3] = {pc[0], pc[1], pc[2]};
-      const int pstart[3] = {nF, nF + pc[0], nF + pc[0] + pc[1]};
-      int pptr[3] = {0, 0, 0};
-      (void)prem;
-      (void)pstart;
-      (void)pptr;
       for (int j = 0; j < n; ++j) {
         const int st = j % Cfg::NS;
         const uint32_t ph = (j / Cfg::NS) & 1;
         if (!__all_sync(kFull, bounded_wait(&kv_empty[st], ph ^ 1, wc))) break;
-        if constexpr (PACK) {
-          if (packed && j >= nF) {
-            // a bin of edge pieces: each piece's exact box at 8-row offsets
-            int a[3];
-            next_bin(p, prem, a);
-            if (elect_one()) {
-              uint8_t* sK = smem + Cfg::kOffK + st * Cfg::kKVBytes;
-              uint8_t* sV = smem + Cfg::kOffV + st * Cfg::kKVBytes;
-              uint32_t bytes = 0;
-#pragma unroll
-              for (int e = 0; e < 3; ++e) bytes += a[e] * p.pk_rows[e] * 128 * Cfg::kChunks;
-              mbar_arrive_expect_tx(&k_full[st], bytes);
-              mbar_arrive_expect_tx(&v_full[st], bytes);
-              int off = 0;
-#pragma unroll
-              for (int e = 0; e < 3; ++e) {
-                for (int m = 0; m < a[e]; ++m) {
-                  const int kt = plist[pstart[e] + pptr[e] + m];
-                  int x0, y0, fr;
-                  nat_coords(kt, x0, y0, fr);
-                  const CUtensorMap* mk = &em.k[p.pk_kind[e] - 1];
-                  const CUtensorMap* mv = &em.v[p.pk_kind[e] - 1];
-                  for (int c = 0; c < Cfg::kChunks; ++c) {
-                    tma_load_5d(sK + c * Cfg::kPanel + off * 128, mk, &k_full[st],
-                                c * Cfg::kChunkElems, h, x0, y0, fr);
-                    tma_load_5d(sV + c * Cfg::kPanel + off * 128, mv, &v_full[st],
-                                c * Cfg::kChunkElems, h, x0, y0, fr);
-                  }
-                  off += p.pk_step[e];
-                }
-              }
-            }
-#pragma unroll
-            for (int e = 0; e < 3; ++e) pptr[e] += a[e];
-            __syncwarp();
-            issued = j + 1;
-            continue;
-          }
-        }
         bool ok;
         const int kt = tile_of(j, ok);
         const int krow = (int)(bh_row + (int64_t)kt * kTile);
         if (elect_one()) {
-          if (!ok && !PACK) atomicOr(p.status, kStatusBadBlocklist);
+          if (!ok) atomicOr(p.status, kStatusBadBlocklist);
           uint8_t* sK = smem + Cfg::kOffK + st * Cfg::kKVBytes;
           uint8_t* sV = smem + Cfg::kOffV + st * Cfg::kKVBytes;
-          if constexpr (NAT) {
-            int x0, y0, fr;
-            nat_coords(kt, x0, y0, fr);
-            mbar_arrive_expect_tx(&k_full[st], Cfg::kKVBytes);
-            for (int c = 0; c < Cfg::kChunks; ++c)
-              tma_load_5d(sK + c * Cfg::kPanel, &tmk, &k_full[st], c * Cfg::kChunkElems, h, x0, y0,
-                          fr);
-            mbar_arrive_expect_tx(&v_full[st], Cfg::kKVBytes);
-            for (int c = 0; c < Cfg::kChunks; ++c)
-              tma_load_5d(sV + c * Cfg::kPanel, &tmv, &v_full[st], c * Cfg::kChunkElems, h, x0, y0,
-                          fr);
-          } else {
-            mbar_arrive_expect_tx(&k_full[st], Cfg::kKVBytes);
-            for (int c = 0; c < Cfg::kChunks; ++c)
-              tma_load_2d(sK + c * Cfg::kPanel, &tmk, &k_full[st], c * 64, krow);
-            mbar_arrive_expect_tx(&v_full[st], Cfg::kKVBytes);
-            for (int c = 0; c < Cfg::kChunks; ++c)
-              tma_load_2d(sV + c * Cfg::kPanel, &tmv, &v_full[st], c * 64, krow);
-          }
+          mbar_arrive_expect_tx(&k_full[st], Cfg::kKVBytes);
+          for (int c = 0; c < Cfg::kChunks; ++c)
+            tma_load_2d(sK + c * Cfg::kPanel, &tmk, &k_full[st], c * 64, krow);
+          mbar_arrive_expect_tx(&v_full[st], Cfg::kKVBytes);
+          for (int c = 0; c < Cfg::kChunks; ++c)
+            tma_load_2d(sV + c * Cfg::kPanel, &tmv, &v_full[st], c * 64, krow);
         }
         __syncwarp();
         issued = j + 1;
@@ -505,8 +285,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       // -------------------------------------------------------- MMA issuer
       // the whole warp runs the loop (descriptors stay warp-uniform); the
       // elected lane issues the tcgen05 instructions
-      constexpr uint32_t idesc_qk = F8 ? idesc_e4m3(128, 128, 0) : idesc_bf16(128, 128, 0);
-      constexpr uint32_t idesc_pv = F8 ? idesc_e4m3(128, D, 1) : idesc_bf16(128, D, 1);
+      constexpr uint32_t idesc_qk = idesc_bf16(128, 128, 0);
+      constexpr uint32_t idesc_pv = idesc_bf16(128, D, 1);
       const uint64_t qd = sdesc_sw128(smem_u32(sQ), 16, 1024);
       const uint64_t kd0 = sdesc_sw128(smem_u32(smem + Cfg::kOffK), 16, 1024);
       const uint64_t vd0 = sdesc_sw128(smem_u32(smem + Cfg::kOffV), Cfg::kPanel, 1024);
@@ -517,32 +297,12 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int kk = 0; kk < D / Cfg::kKeysPerMma; ++kk) {
             // K step kk: 32 bytes along the 128-byte swizzle row, then the next panel
             const uint32_t off = (kk >> 2) * Cfg::kPanel + (kk & 3) * 32;
-            if constexpr (F8)
-              mma_ss_f8(tdst, sdesc_add(qd, off), sdesc_add(kd, off), idesc_qk, kk > 0);
-            else
-              mma_ss(tdst, sdesc_add(qd, off), sdesc_add(kd, off), idesc_qk, kk > 0);
+            mma_ss(tdst, sdesc_add(qd, off), sdesc_add(kd, off), idesc_qk, kk > 0);
           }
         }
         __syncwarp();
       };
-      auto issue_pv = [&](int st, uint32_t tP, uint32_t tO, uint32_t acc) {
-        const uint64_t vd = sdesc_add(vd0, st * Cfg::kKVBytes);
-        if (elect_one()) {
-#pragma unroll
-          for (int kk = 0; kk < kTile / Cfg::kKeysPerMma; ++kk) {
-            // K step kk: the next kKeysPerMma keys = 8 TMEM columns of P and
-            // kKeysPerMma 128-byte rows of V
-            if constexpr (F8)
-              mma_ts_f8(tO, tP + kk * 8, sdesc_add(vd, kk * Cfg::kKeysPerMma * 128), idesc_pv,
-                        (acc | (uint32_t)kk) != 0);
-            else
-              mma_ts(tO, tP + kk * 8, sdesc_add(vd, kk * Cfg::kKeysPerMma * 128), idesc_pv,
-                     (acc | (uint32_t)kk) != 0);
-          }
-        }
-        __syncwarp();
-      };
-      // bf16: O_g (+)= P(keys 64 * half .. + 63) . V(same keys)
+      // O_g (+)= P(keys 64 * half .. + 63) . V(same keys)
       auto issue_pv_half = [&](int st, int g, int half, uint32_t acc) {
         const uint64_t vd = sdesc_add(vd0, st * Cfg::kKVBytes + half * 64 * 128);
         const uint32_t tP = tbase + g * 128 + 64 + half * 32, tO = tbase + 256 + g * 128;
@@ -561,54 +321,30 @@ __global__ void __launch_bounds__(kThreads, 1)
       auto wait = [&](uint64_t* bar, uint32_t parity) {
         return __all_sync(kFull, bounded_wait(bar, parity, wc));
       };
-      if constexpr (!F8) {
-        // group g takes tiles g, g + 2, ...; QK of tile j+2 follows PV of
-        // tile j, so each group's next S is ready as soon as its PV is done;
-        // P is handed over in two halves
-        auto qk = [&](int t) {
-          const int st = t % Cfg::NS;
-          if (!wait(&k_full[st], (t / Cfg::NS) & 1)) return false;
-          tc_fence_after();
-          issue_qk(st, tbase + (t & 1) * 128);
-          commit(&s_full[t & 1]);
-          return true;
-        };
-        bool alive = wait(q_full, 0) && qk(0) && (n < 2 || qk(1));
-        for (int j = 0; alive && j < n; ++j) {
-          const int g = j & 1, st = j % Cfg::NS;
-          if (!wait(&p_half[g], (j >> 1) & 1) || !wait(&v_full[st], (j / Cfg::NS) & 1)) break;
-          tc_fence_after();
-          issue_pv_half(st, g, 0, j >= 2);
-          if (!wait(&p_ready[g], (j >> 1) & 1)) break;
-          tc_fence_after();
-          issue_pv_half(st, g, 1, 1);
-          commit(&kv_empty[st]);
-          if (j + 2 < n && !qk(j + 2)) break;
-        }
-        commit(o_final);
-      } else {
-      bool alive = wait(q_full, 0) && wait(&k_full[0], 0);
-      if (alive) {
+      // group g takes tiles g, g + 2, ...; QK of tile j+2 follows PV of
+      // tile j, so each group's next S is ready as soon as its PV is done;
+      // P is handed over in two halves
+      auto qk = [&](int t) {
+        const int st = t % Cfg::NS;
+        if (!wait(&k_full[st], (t / Cfg::NS) & 1)) return false;
         tc_fence_after();
-        issue_qk(0, tbase);
-        commit(&s_full[0]);
-      }
+        issue_qk(st, tbase + (t & 1) * 128);
+        commit(&s_full[t & 1]);
+        return true;
+      };
+      bool alive = wait(q_full, 0) && qk(0) && (n < 2 || qk(1));
       for (int j = 0; alive && j < n; ++j) {
-        if (j + 1 < n) {
-          const int st1 = (j + 1) % Cfg::NS;
-          if (!wait(&k_full[st1], ((j + 1) / Cfg::NS) & 1)) break;
-          tc_fence_after();
-          issue_qk(st1, tbase + ((j + 1) & 1) * 128);
-          commit(&s_full[(j + 1) & 1]);
-        }
         const int g = j & 1, st = j % Cfg::NS;
-        if (!wait(&p_ready[g], (j >> 1) & 1) || !wait(&v_full[st], (j / Cfg::NS) & 1)) break;
+        if (!wait(&p_half[g], (j >> 1) & 1) || !wait(&v_full[st], (j / Cfg::NS) & 1)) break;
         tc_fence_after();
-        issue_pv(st, tbase + g * 128 + 64, tbase + 256 + g * 128, j >= 2);
+        issue_pv_half(st, g, 0, j >= 2);
+        if (!wait(&p_ready[g], (j >> 1) & 1)) break;
+        tc_fence_after();
+        issue_pv_half(st, g, 1, 1);
         commit(&kv_empty[st]);
+        if (j + 2 < n && !qk(j + 2)) break;
       }
       commit(o_final);
-      }
     }
     cta_end_sync();
     if (warp == 1) {
@@ -625,11 +361,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t lane_off = (uint32_t)(q4 * 32) << 16;
     const uint32_t tS = tbase + g * 128 + lane_off;
     const uint32_t tO = tbase + 256 + g * 128 + lane_off;
-    // e4m3: S holds q8.k8; the scores are S * sq * sk
-    const float sqk = F8 ? p.fp8_scales[(int64_t)b * p.Hh + h] *
-                               p.fp8_scales[((int64_t)p.B + b) * p.Hh + h]
-                         : 1.f;
-    const float sl2 = p.scale_log2 * sqk;
+    const float sl2 = p.scale_log2;
     const float thr = 8.0f / sl2;  // rescale O when the max grows by more than 2^8
     RowState rs;
     int64_t fptr = 0, fend = 0;
@@ -647,29 +379,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
     bool alive = true;
-    int srem[3] = {pc[0], pc[1], pc[2]};  // packed bins: pieces left per kind
-    int scur = nF;                        // next bin index to replay
-    (void)srem;
-    (void)scur;
     for (int j = g; j < n; j += 2) {
       uint32_t vm[4] = {0u, 0u, 0u, 0u};
-      if (PACK && packed && j >= nF) {
-        // rows of this bin's pieces: [off, off + rows) of each
-        int a[3];
-        while (scur < j) {
-          next_bin(p, srem, a);
-          ++scur;
-        }
-        next_bin(p, srem, a);
-        ++scur;
-        int off = 0;
-#pragma unroll
-        for (int e = 0; e < 3; ++e)
-          for (int m = 0; m < a[e]; ++m) {
-            set_rows(vm, off, off + p.pk_rows[e]);
-            off += p.pk_step[e];
-          }
-      } else {
+      {
         bool ok;
         const int kt = tile_of(j, ok);
         const uint4 tv = __ldg(reinterpret_cast<const uint4*>(p.tile_valid) + kt);
@@ -713,93 +425,32 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int i = 0; i < 128; ++i) s[i] = __uint_as_float(r128[i]);
       }
-      if constexpr (!F8) {
-        float corr;
-        uint64_t neg_ms2;
-        // full key tiles take a copy of the step without masking
-        const bool need = (vm[0] & vm[1] & vm[2] & vm[3]) == kFull
-                              ? softmax_max<128, false>(s, vm, rs, sl2, thr, corr, neg_ms2)
-                              : softmax_max<128, true>(s, vm, rs, sl2, thr, corr, neg_ms2);
-        uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};
-        {
-          uint32_t pk[32];
-          softmax_exp<0, 64>(s, sl2, neg_ms2, pk, acc);
-          tmem_st32(tS + 64, pk);
-        }
-        // O of this group holds every earlier PV of the group (S(j) was
-        // written after the group's previous PV); it is rescaled before this
-        // tile's first PV, once half of s is no longer live
-        if (j >= 2 && __any_sync(kFull, need)) tmem_scale<D>(tO, corr);
-        tc_fence_before();
-        mbar_arrive(&p_half[g]);
-        {
-          uint32_t pk[32];
-          softmax_exp<64, 64>(s, sl2, neg_ms2, pk, acc);
-          tmem_st32(tS + 96, pk);
-        }
-        softmax_sum(rs, acc);
-        tc_fence_before();
-        mbar_arrive(&p_ready[g]);
-        continue;
-      } else {
-        // e4m3: P rounded to e4m3, four keys to a TMEM column, in one hand-off
-        if ((vm[0] & vm[1] & vm[2] & vm[3]) != kFull) {
-#pragma unroll
-          for (int w = 0; w < 4; ++w)
-#pragma unroll
-            for (int i = 0; i < 32; ++i)
-              if (!((vm[w] >> i) & 1u)) s[w * 32 + i] = -INFINITY;
-        }
-        // row max: 8 independent chains of 3-input max, then a small tree
-        float m8[8];
-#pragma unroll
-        for (int c = 0; c < 8; ++c) m8[c] = fmax3f(s[c], s[c + 8], s[c + 16]);
-#pragma unroll
-        for (int i = 24; i < 120; i += 16)
-#pragma unroll
-          for (int c = 0; c < 8; ++c) m8[c] = fmax3f(m8[c], s[i + c], s[i + 8 + c]);
-#pragma unroll
-        for (int c = 0; c < 8; ++c) m8[c] = fmaxf(m8[c], s[120 + c]);
-        const float mx = fmax3f(fmax3f(m8[0], m8[1], m8[2]), fmax3f(m8[3], m8[4], m8[5]),
-                                fmaxf(m8[6], m8[7]));
-        const float m_new = fmaxf(rs.m, mx);
-        const bool need = m_new > rs.m + thr;
-        float corr = 1.f;
-        if (need) {
-          corr = ex2_approx((rs.m - m_new) * sl2);
-          rs.m = m_new;
-          rs.l *= corr;
-        }
-        const float ms = (rs.m == -INFINITY) ? 0.f : rs.m * sl2;
+      float corr;
+      uint64_t neg_ms2;
+      // full key tiles take a copy of the step without masking
+      const bool need = (vm[0] & vm[1] & vm[2] & vm[3]) == kFull
+                            ? softmax_max<128, false>(s, vm, rs, sl2, thr, corr, neg_ms2)
+                            : softmax_max<128, true>(s, vm, rs, sl2, thr, corr, neg_ms2);
+      uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};
+      {
         uint32_t pk[32];
-        float l8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};  // independent partial sums
-        // P as e4m3 bytes, four keys to a word (P <= 2^8 < 448)
-#pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          const float p0 = ex2_approx(fmaf(s[4 * i], sl2, -ms));
-          const float p1 = ex2_approx(fmaf(s[4 * i + 1], sl2, -ms));
-          const float p2 = ex2_approx(fmaf(s[4 * i + 2], sl2, -ms));
-          const float p3 = ex2_approx(fmaf(s[4 * i + 3], sl2, -ms));
-          l8[i & 7] += (p0 + p1) + (p2 + p3);
-          pk[i] = pack_e4m3x2(p0, p1) | (pack_e4m3x2(p2, p3) << 16);
-        }
-        rs.l += ((l8[0] + l8[1]) + (l8[2] + l8[3])) + ((l8[4] + l8[5]) + (l8[6] + l8[7]));
-        // O of this group holds every earlier PV of the group: S(j) was written
-        // after the group's previous PV in the tensor cores' issue order.
-        if (j >= 2 && __any_sync(kFull, need)) {
-#pragma unroll
-          for (int c = 0; c < D / 32; ++c) {
-            uint32_t o32[32];
-            tmem_ld32(tO + c * 32, o32);
-#pragma unroll
-            for (int i = 0; i < 32; ++i) o32[i] = __float_as_uint(__uint_as_float(o32[i]) * corr);
-            tmem_st32(tO + c * 32, o32);
-          }
-        }
-        tmem_st32(tS + 64, *reinterpret_cast<uint32_t(*)[32]>(&pk[0]));
-        tc_fence_before();
-        mbar_arrive(&p_ready[g]);
+        softmax_exp<0, 64>(s, sl2, neg_ms2, pk, acc);
+        tmem_st32(tS + 64, pk);
       }
+      // O of this group holds every earlier PV of the group (S(j) was
+      // written after the group's previous PV); it is rescaled before this
+      // tile's first PV, once half of s is no longer live
+      if (j >= 2 && __any_sync(kFull, need)) tmem_scale<D>(tO, corr);
+      tc_fence_before();
+      mbar_arrive(&p_half[g]);
+      {
+        uint32_t pk[32];
+        softmax_exp<64, 64>(s, sl2, neg_ms2, pk, acc);
+        tmem_st32(tS + 96, pk);
+      }
+      softmax_sum(rs, acc);
+      tc_fence_before();
+      mbar_arrive(&p_ready[g]);
     }
     // ---------------------------------------------------------- epilogue
     if (alive && n > 0) {
@@ -822,24 +473,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t qw = (row < 32) ? tq.x : (row < 64) ? tq.y : (row < 96) ? tq.z : tq.w;
     const bool qvalid = (qw >> (row & 31)) & 1u;
     const bool has = alive && n > 0 && qvalid && l > 0.f;
-    // e4m3: O holds P.v8; the values are O * sv
-    const float sv = F8 ? p.fp8_scales[(2 * (int64_t)p.B + b) * p.Hh + h] : 1.f;
-    const float inv_l = has ? sv / l : 0.f;
+    const float inv_l = has ? 1.f / l : 0.f;
     const float wa = a * inv_l, wb = bb * inv_l;
-    int64_t orow = bh_row + (int64_t)qt * kTile + row;  // slot row, or natural token row
-    int64_t lrow = orow;                                 // LSE index
-    if constexpr (NAT) {
-      // slot (a, c) of tile (t, i, j) is token (t, y0 + a, x0 + c); empty slots
-      // (past the grid edge) are not stored
-      int x0, y0, fr;
-      nat_coords(qt, x0, y0, fr);
-      const int a = (int)p.div_pw.div((uint32_t)row);
-      const int y = y0 + a, x = x0 + (row - a * p.pw);
-      const int t = fr - b * p.T;
-      const int64_t n = ((int64_t)t * p.H + y) * p.W + x;
-      orow = ((int64_t)b * p.N + n) * p.Hh + h;
-      lrow = ((int64_t)b * p.Hh + h) * p.N + n;
-    }
+    const int64_t orow = bh_row + (int64_t)qt * kTile + row;  // slot row = LSE index
     // group g stores columns [g*D/2, (g+1)*D/2) of its rows
     uint4* dst = reinterpret_cast<uint4*>(p.o + orow * D + g * (D / 2));
     const uint32_t oA = tbase + 256 + lane_off + g * (D / 2);
@@ -859,13 +495,13 @@ __global__ void __launch_bounds__(kThreads, 1)
             has ? __uint_as_float(xa[2 * i + 1]) * wa + __uint_as_float(xb[2 * i + 1]) * wb : 0.f;
         w16[i] = pack_bf16x2(v0, v1);
       }
-      if (!NAT || qvalid) {
+      {
 #pragma unroll
         for (int i = 0; i < 4; ++i)
           dst[c * 4 + i] = make_uint4(w16[4 * i], w16[4 * i + 1], w16[4 * i + 2], w16[4 * i + 3]);
       }
     }
-    if (g == 0 && p.lse && (!NAT || qvalid)) p.lse[lrow] = has ? m * p.scale + logf(l) : -INFINITY;
+    if (g == 0 && p.lse) p.lse[orow] = has ? m * p.scale + logf(l) : -INFINITY;
     tc_fence_before();
     cta_end_sync();
   }
@@ -897,17 +533,14 @@ bool make_tmap(CUtensorMap* m, const void* ptr, int64_t rows, int D) {
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int D, bool FINE, bool NAT = false, bool F8 = false, bool PACK = false>
+template <int D, bool FINE>
 cudaError_t launch_t(const CUtensorMap& q, const CUtensorMap& k, const CUtensorMap& v,
-                     const AttnParams& p, dim3 grid, cudaStream_t st,
-                     const EdgeMaps* em = nullptr) {
-  using Cfg = AttnCfg<D, FINE, F8, PACK>;
-  auto kern = attn_fwd_kernel<D, FINE, NAT, F8, PACK>;
+                     const AttnParams& p, dim3 grid, cudaStream_t st) {
+  using Cfg = AttnCfg<D, FINE>;
+  auto kern = attn_fwd_kernel<D, FINE>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::kSmem);
   if (e != cudaSuccess) return e;
-  EdgeMaps none;
-  memset(&none, 0, sizeof(none));
-  kern<<<grid, kThreads, Cfg::kSmem, st>>>(q, k, v, p, em ? *em : none);
+  kern<<<grid, kThreads, Cfg::kSmem, st>>>(q, k, v, p);
   return cudaGetLastError();
 }
 
@@ -934,46 +567,7 @@ AttnParams make_params(const bsa_plan_s& plan, const int32_t* row_ptr, const int
   p.tile_valid = plan.d_tile_valid;
   p.status = plan.d_status;
   p.wait_limit_ns = plan.wait_limit_ns;
-  p.B = g.B;
-  p.fp8_scales = nullptr;
-  p.T = g.T;
-  p.H = g.H;
-  p.W = g.W;
-  p.N = g.T * g.P;
-  p.ph = g.ph > 0 ? g.ph : 1;
-  p.pw = g.pw > 0 ? g.pw : 1;
-  p.TW = (g.W + p.pw - 1) / p.pw;
-  const int TH = (g.H + p.ph - 1) / p.ph;
-  p.div_tile_frame = FastDiv((uint32_t)(TH * p.TW));
-  p.div_TW = FastDiv((uint32_t)p.TW);
-  p.div_pw = FastDiv((uint32_t)p.pw);
-  p.TH = TH;
-  p.pk_on = 0;
-  for (int e = 0; e < 3; ++e) p.pk_kind[e] = p.pk_rows[e] = p.pk_step[e] = 0;
   return p;
-}
-
-
-
-// Natural layout [B, N, Hh, D] bf16 seen as 5-D {D, Hh, W, H, B*T}; boxes of
-// 64 channels x 1 head x pw x ph x 1 frame (one pooling tile, 128 rows of
-// 128 bytes), 128-byte swizzle.  Boxes reaching past W or H read zeros.
-bool make_tmap_tiles(CUtensorMap* m, const void* ptr, const Geometry& g, bool e4m3 = false,
-                     int box_w = 0, int box_h = 0) {
-  auto fn = encode_fn();
-  if (!fn) return false;
-  const cuuint64_t esz = e4m3 ? 1 : 2;
-  const cuuint64_t row = (cuuint64_t)g.Hh * g.D * esz;  // bytes per token
-  cuuint64_t dims[5] = {(cuuint64_t)g.D, (cuuint64_t)g.Hh, (cuuint64_t)g.W, (cuuint64_t)g.H,
-                        (cuuint64_t)g.B * g.T};
-  cuuint64_t strides[4] = {(cuuint64_t)g.D * esz, row, row * g.W, row * g.W * g.H};
-  cuuint32_t box[5] = {(cuuint32_t)(128 / esz), 1, (cuuint32_t)(box_w > 0 ? box_w : g.pw),
-                       (cuuint32_t)(box_h > 0 ? box_h : g.ph), 1};
-  cuuint32_t estr[5] = {1, 1, 1, 1, 1};
-  return fn(m, e4m3 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5,
-            const_cast<void*>(ptr), dims, strides, box,
-            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 }  // namespace
