@@ -152,6 +152,17 @@ def test_attn_e4m3_small_all_tokens(over):
     assert err.mean() <= MEAN_ABS_E4M3, err.mean()
 
 
+@pytest.mark.parametrize("T", [256, 300])
+def test_attn_e4m3_lists_at_and_past_the_bin_limit(T):
+    # 6 x 10 frames: one 60-token corner tile each, two to a packed MMA tile;
+    # every block kept: 128 packed tiles (the most a list buffer holds) at
+    # T = 256, and an unpacked list at T = 300
+    w = small_workload(CONFIGS[2], T=T, H=6, W=10, Hh=1, draft_sparsity=0, field_grid=(16, 2, 3))
+    *_, err = _e4m3_case(w, q_blocks=[0, 1, T // 2, T - 1])
+    assert err.max() <= MAX_ABS_E4M3, err.max()
+    assert err.mean() <= MEAN_ABS_E4M3, err.mean()
+
+
 @pytest.mark.parametrize("cid", [2, 5])
 def test_attn_e4m3_full_size_sampled(cid):
     w = CONFIGS[cid]

@@ -304,7 +304,23 @@ def _attn_case_var(w, rp, ci):
                       [(b, h) for b in range(w.B) for h in range(w.Hh)])
 
 
-def test_attn_empty_rows_and_out_of_range_blocks():
+def test_attn_per_head_lists_frame_layout():
+    # per-head lists of 128-slot blocks on the frame layout (each frame's
+    # last block is partly empty): the persistent kernel's slot mode
+    w = small_workload(CONFIGS[2], T=3, Hh=2, D=128, field_grid=(3, 4, 7))
+    nb = 3 * 13
+    rng = np.random.default_rng(7)
+    k = 9
+    rows = [np.sort(rng.choice(nb, size=k, replace=False)) for _ in range(w.B * w.Hh * nb)]
+    rp = (np.arange(len(rows) + 1) * k).astype(np.int32)
+    ci = np.concatenate(rows).astype(np.int32)
+    _attn_case(w, "frame", 128, rp, ci, True)
+
+
+@pytest.mark.parametrize("per_head", [False, True])
+def test_attn_empty_rows_and_out_of_range_blocks(per_head):
+    # one (batch, head): the same CSR serves as a shared list (the paired
+    # kernel) and as per-head lists (the persistent kernel's slot mode)
     w = small_workload(CONFIGS[2], T=1, Hh=1, D=128, field_grid=(1, 4, 7))
     q, k, v = make_qkv(w)
     plan = bsa.Plan(1, 1, 128, 1, 30, 52, bsa.LAYOUT_TILE, 8, 16, 128)
@@ -320,7 +336,7 @@ def test_attn_empty_rows_and_out_of_range_blocks():
     o = torch.empty_like(qs)
     lse = torch.empty(qs.shape[:3], dtype=torch.float32, device="cuda")
     bsa.bsa_attn_fwd(plan, qs, ks, vs, torch.from_numpy(rp).cuda(), torch.from_numpy(ci).cuda(),
-                     False, 1 / math.sqrt(128), o, lse)
+                     per_head, 1 / math.sqrt(128), o, lse)
     with pytest.raises(bsa.BsaError) as ei:
         bsa.bsa_poll_status(plan)
     assert ei.value.status == 6
@@ -334,7 +350,7 @@ def test_attn_empty_rows_and_out_of_range_blocks():
     rp_ok = np.concatenate([[0], np.cumsum([len(r) for r in lists_ok])]).astype(np.int32)
     ci_ok = np.array([c for r in lists_ok for c in r], dtype=np.int32)
     O, L = oracle.masked_attention(*(oracle.reorder_fwd(to_np64(x), perm, Np) for x in (q, k, v)),
-                                   valid, 128, rp_ok, ci_ok, False, 1 / math.sqrt(128))
+                                   valid, 128, rp_ok, ci_ok, per_head, 1 / math.sqrt(128))
     compare_attention(o, lse, O, L, valid, 128, list(range(16)), [(0, 0)])
     bsa.bsa_poll_status(plan)   # status was cleared by the previous poll
 
