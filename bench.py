@@ -44,6 +44,8 @@ sys.path.insert(0, ROOT)
 
 from synth import CONFIGS, make_qkv  # noqa: E402
 
+NOMINAL_BF16_TFLOPS = 2250.0  # B200 dense bf16, NVIDIA's figure (context only)
+
 METRIC = "bsattn ms/call + attended TFLOP/s (% BF16 peak), Wan-1.3B-shape 6× length LVSA"
 
 # DRAM bytes per launch of the LVSA step kernel at the full Wan-1.3B 6x
@@ -595,6 +597,8 @@ def main():
             "kernel": dominant}
     if extra.get("traffic_source"):
         roof["traffic_source"] = extra["traffic_source"]
+    # against NVIDIA's nominal dense bf16 figure for B200 (2.25 PFLOP/s), for context
+    roof["frac_of_nominal_dense_bf16"] = dom_tflops / NOMINAL_BF16_TFLOPS
     if sustained:
         roof["frac_of_sustained"] = dom_tflops / sustained
         peak_mhz = _peak_sm_mhz(pk)
