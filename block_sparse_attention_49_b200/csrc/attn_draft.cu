@@ -1,5 +1,10 @@
-// Draft attention on the natural layout, persistent: one CTA per SM walks
-// its share of the query tiles and keeps its pipelines running across them.
+// Block-sparse attention on per-head lists of 128-slot blocks, persistent:
+// one CTA per SM walks its share of the query tiles and keeps its pipelines
+// running across them.  Three forms of the same body:
+//   natural layout (bf16): the draft path without reorders;
+//   natural layout, e4m3 tiles (template flag F8): the 8-bit draft path;
+//   slot mode: [B, Hh, Npad, D] slot tensors of any plan (bsa_attn_fwd with
+//   per-head lists).
 //
 // What it computes (Draft Attention article: the sparse mask from the draft
 // map guides full-resolution block-sparse attention; the reorder that makes
@@ -11,34 +16,34 @@
 // Why persistent: a draft row keeps a few dozen key tiles (34 of 336 at 90 %
 // sparsity), so a CTA per query tile spends a share of its life on set-up
 // and on loads that no earlier work hides.  Here the next tile's list,
-// query tile and first key tiles load while the current tile finishes.
-// Measured on the Wan-14B-like draft workload (keep 4 to 34 blocks per
-// row): 0.67 ms + 0.080 ms per kept block, against 0.74 ms + 0.078 ms with
-// a CTA per query tile.  The remaining per-tile cost is the tile's own
-// ramp: its first softmax waits for its first QK, and its epilogue (the
-// two groups' merge and the stores) runs on the softmax warps before the
-// next tile's softmax can start.
+// query tile and first key tiles load while the current tile finishes.  The
+// remaining per-tile cost is the tile's own ramp: its first softmax waits
+// for its first QK, and its epilogue (the two groups' merge and the stores)
+// runs on the softmax warps before the next tile's softmax can start.
 //
 // Roles (12 warps; tile i = the i-th query tile of this CTA):
 //   warp 0      TMA producer of Q (after the last QK of tile i-1) and of K
-//               into a 3-deep ring; warp 3 of V into a 2-deep ring (K is
-//               needed a softmax earlier than V).  Edge tiles (partial tiles
-//               at the grid's right and bottom edges) are packed several to
-//               a 128-row MMA tile, each piece loaded with a box of its
-//               exact size.
-//   warp 1      MMA issuer: S = Q K^T into the group's S buffer, O += P V;
-//               the first PV of tile i waits until tile i-1's output has
-//               been read out of tensor memory.
-//   warp 2      scheduler: the key list of tile i, sorted by tile kind for
-//               packing, into one of two list buffers.
+//               into a ring (3 deep, 4 for e4m3); warp 3 of V into a ring
+//               (2 deep, 4 for e4m3): K is needed a softmax earlier than V.
+//               On the natural layout, edge tiles (partial tiles at the
+//               grid's right and bottom edges) are packed several to a
+//               128-row MMA tile, each piece loaded with a box of its exact
+//               size.
+//   warp 1      MMA issuer: a group's PV in two halves as its P halves
+//               arrive, then that group's next QK; the first PV of tile i
+//               waits until tile i-1's output has been read out of tensor
+//               memory.
+//   warp 2      scheduler: the key list of tile i, sorted by tile kind, with
+//               the row mask and piece counts of each packed tile, into one
+//               of two list buffers.
 //   warps 4-7   softmax group A (key tiles 0, 2, 4, ... of a query tile),
 //   warps 8-11  group B (1, 3, 5, ...): one row per thread, running max and
-//               sum, P as bf16 over its S; then the epilogue of the tile:
-//               the two groups' partial results merged (a split-key
-//               combine), normalised and stored to the tokens.
+//               sum, P (bf16, or e4m3 four keys to a column) over its S;
+//               then the epilogue of the tile: the two groups' partial
+//               results merged (a split-key combine), normalised and stored.
 // Tensor memory: S_A | S_B | O_A | O_B (512 columns).  The arithmetic per
-// tile is that of bsa_attn_fwd, so on a grid without partial tiles the
-// result is identical, bit for bit, to the reorder path.
+// tile is that of bsa_attn_fwd's block-list kernel, so on a grid without
+// partial tiles the natural and slot forms give identical bits.
 // Every wait is bounded; a wait that runs out records a timeout in the
 // plan's status word and the CTA leaves without trapping.
 #include <cuda_bf16.h>
