@@ -276,8 +276,10 @@ bsa_status bsa_draft_mask_natural_e4m3(bsa_plan_t plan, const void* q, const voi
  * accumulation; the scores are S * sq * sk; P is rounded to e4m3 (it stays
  * below 2^8); O is multiplied by sv.  Requires D = 128 and a TILE plan with
  * pool_h * pool_w = 128.  o: bf16 natural layout; lse as for
- * bsa_attn_fwd_natural.  Result within the e4m3 rounding of Q, K, V and P
- * of the exact attention (see the tests for the bound used). */
+ * bsa_attn_fwd_natural, of the scores scale * S * sq * sk (the dequantized
+ * inputs; P's rounding does not enter it).  Result within the e4m3 rounding
+ * of Q, K, V and P of the exact attention (see the tests for the bound
+ * used). */
 bsa_status bsa_attn_fwd_natural_e4m3(bsa_plan_t plan, const void* q8, const void* k8,
                                      const void* v8, const float* scales, const int32_t* row_ptr,
                                      const int32_t* col_idx, int per_head_lists, float scale,
