@@ -35,8 +35,8 @@ namespace {
 
 constexpr int kTile = 128;
 constexpr int kThreads = 384;
-constexpr int kPairMaxBlocks = 32768;   // blocks a list may name (membership bitmaps)
-constexpr int kPairMaxTiles = 4096;     // key tiles in the union of two rows
+constexpr int kPairMaxTiles = 4096;     // blocks of the plan: a row may name all of them, so
+                                        // the union of two rows and the bitmaps fit this
 
 template <int D>
 struct PairCfg {
@@ -53,8 +53,8 @@ struct PairCfg {
   static constexpr int kNumBars = 1 + 4 * NS + 2 + 2 + 2 + 1;
   static constexpr int kOffMisc = kOffBar + kNumBars * 8;
   static constexpr int kOffList = kOffMisc + 16;                  // union: (block << 2) | rows
-  static constexpr int kOffBits = kOffList + kPairMaxTiles * 4;   // [2][kPairMaxBlocks / 32]
-  static constexpr int kBytes = kOffBits + 2 * (kPairMaxBlocks / 32) * 4;
+  static constexpr int kOffBits = kOffList + kPairMaxTiles * 4;   // [2][kPairMaxTiles / 32]
+  static constexpr int kBytes = kOffBits + 2 * (kPairMaxTiles / 32) * 4;
   static constexpr int kSmem = kBytes + 1024;
   static_assert(kSmem <= 232448, "shared memory budget");
 };
@@ -127,7 +127,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     prefetch_tmap(&tmk);
     prefetch_tmap(&tmv);
   }
-  for (int i = threadIdx.x; i < 2 * words; i += kThreads) bits[(i / words) * (kPairMaxBlocks / 32) + i % words] = 0u;
+  for (int i = threadIdx.x; i < 2 * words; i += kThreads) bits[(i / words) * (kPairMaxTiles / 32) + i % words] = 0u;
   __syncthreads();
   if (misc[3]) return;
   if (warp == 1) {
@@ -147,7 +147,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int64_t i = a + threadIdx.x; i < e; i += kThreads) {
       const int c = __ldg(p.col_idx + i);
       if (c >= 0 && (int64_t)c < p.nblocks)
-        atomicOr(&bits[g * (kPairMaxBlocks / 32) + (c >> 5)], 1u << (c & 31));
+        atomicOr(&bits[g * (kPairMaxTiles / 32) + (c >> 5)], 1u << (c & 31));
       else
         atomicOr(p.status, kStatusBadBlocklist);
     }
@@ -160,7 +160,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int w0 = 0; w0 < words; w0 += 32) {
       const int w = w0 + lane;
       const uint32_t b0 = w < words ? bits[w] : 0u;
-      const uint32_t b1 = w < words ? bits[kPairMaxBlocks / 32 + w] : 0u;
+      const uint32_t b1 = w < words ? bits[kPairMaxTiles / 32 + w] : 0u;
       const uint32_t u = b0 | b1;
       const int mine = __popc(u);
       int pos = mine;
@@ -455,7 +455,8 @@ cudaError_t launch_pair_t(const CUtensorMap& q, const CUtensorMap& k, const CUte
 }  // namespace
 
 bool attn_pair_applies(const Geometry& g, int per_head) {
-  return !per_head && g.block == kTile && g.nblocks <= kPairMaxBlocks;
+  // a row may name every block: the union of two rows must fit the list
+  return !per_head && g.block == kTile && g.nblocks <= kPairMaxTiles;
 }
 
 bsa_status launch_attn_pair(const bsa_plan_s& plan, const void* q, const void* k, const void* v,

@@ -304,6 +304,22 @@ def _attn_case_var(w, rp, ci):
                       [(b, h) for b in range(w.B) for h in range(w.Hh)])
 
 
+@pytest.mark.parametrize("T", [315, 330])
+def test_attn_shared_list_at_and_past_4096_blocks(T):
+    # 13 blocks a frame: 4095 blocks run on the paired kernel, 4290 on the
+    # block-list kernel (the paired kernel's union holds 4096).  Rows 0 and 1
+    # name every block, so their union is the whole plan.
+    w = small_workload(CONFIGS[2], T=T, Hh=1, D=64, field_grid=(8, 4, 7))
+    nb = T * 13
+    rng = np.random.default_rng(T)
+    rows = [np.arange(nb), np.arange(nb)]
+    rows += [np.unique(np.concatenate([[r], rng.choice(nb, size=2, replace=False)]))
+             for r in range(2, nb)]
+    rp = np.concatenate([[0], np.cumsum([len(r) for r in rows])]).astype(np.int32)
+    ci = np.concatenate(rows).astype(np.int32)
+    _attn_case(w, "frame", 128, rp, ci, False, q_blocks=[0, 1, 2, 2000, nb - 1])
+
+
 def test_attn_per_head_lists_frame_layout():
     # per-head lists of 128-slot blocks on the frame layout (each frame's
     # last block is partly empty): the persistent kernel's slot mode
