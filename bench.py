@@ -329,7 +329,7 @@ def kernel_table(args):
             emit(cid, "reorder_fwd (tile layout, Q K V)", timed(lambda: att.gather(q, k, v)),
                  3 * 2 * tok_bytes)
             nb = att.plan.nblocks
-            pooled = 2 * w.B * w.Hh * nb * w.D * 8
+            pooled = 2 * w.B * w.Hh * nb * w.D * 4
             emit(cid, "draft_mask (pool + score/top-k)", timed(att.mask),
                  2 * tok_bytes + 2 * pooled + 4 * att.col_idx.numel(),
                  note=f"k = {att.keep} of {nb} blocks per row")
@@ -414,7 +414,7 @@ def hbm_kernels(cid: int):
     att = DraftAttention(w.B, w.Hh, w.D, w.T, w.H, w.W, w.draft_ph or 8, w.draft_pw or 16,
                          w.draft_sparsity or 90)
     nb = att.plan.nblocks
-    pooled = 2 * w.B * w.Hh * nb * w.D * 8
+    pooled = 2 * w.B * w.Hh * nb * w.D * 4
     for _ in range(2):
         bsa.bsa_reorder_fwd(fr, q, fq, k, fk, v, fv)
         bsa.bsa_reorder_inv(fr, fq, out)
@@ -432,10 +432,10 @@ def hbm_kernels(cid: int):
         "algo_bytes_per_launch": {
             "reorder_fwd_kernel (Q K V, either layout)": 3 * 2 * tok,
             "reorder_inv_kernel (O, either layout)": 2 * tok,
-            "draft_pool_kernel (tile-layout Q K slots read, pooled fp64 written)":
+            "draft_pool_kernel (tile-layout Q K slots read, pooled fp32 written)":
                 2 * w.B * w.Hh * att.plan.Npad * w.D * 2 + pooled,
-            "draft_pool_nat_kernel (natural Q K read, pooled fp64 written)": 2 * tok + pooled,
-            "draft_score_topk_kernel (pooled fp64 read, lists written)":
+            "draft_pool_kernel natural (natural Q K read, pooled fp32 written)": 2 * tok + pooled,
+            "draft_score_reg_kernel (pooled fp32 read, lists written)":
                 pooled + 4 * att.col_idx.numel(),
             "e4m3_amax_kernel (Q K V read)": 3 * tok,
             "e4m3_convert_kernel (Q K V read, codes written)": 3 * tok + 3 * tok // 2},
@@ -737,7 +737,7 @@ def draft_step_setup(w, q, k, v, out):
     torch.cuda.synchronize()
     flops = draft_attended_flops(w, att.col_idx.cpu().numpy(), att.keep)
     tok_bytes = w.B * w.N * w.Hh * w.D * 2
-    pooled = 2 * w.B * w.Hh * att.plan.nblocks * w.D * 8
+    pooled = 2 * w.B * w.Hh * att.plan.nblocks * w.D * 4
     extra = {
         "metric": f"bsattn ms/call + attended TFLOP/s (% BF16 peak), {w.name}, draft attention",
         "poll": lambda: bsa.bsa_poll_status(att.plan),

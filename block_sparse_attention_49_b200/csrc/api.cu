@@ -245,7 +245,7 @@ bsa_status bsa_draft_mask(bsa_plan_t plan, const void* q_slots, const void* k_sl
     return set_error(BSA_ERR_UNSUPPORTED, "block list longer than 2^31 entries");
   cudaError_t e = launch_draft_mask(g, plan->d_tile_valid, q_slots, k_slots, keep,
                                     plan->draft_pooling, row_ptr, kv_idx, draft_map,
-                                    reinterpret_cast<double*>(workspace), plan->d_status,
+                                    reinterpret_cast<float*>(workspace), plan->d_status,
                                     plan->wait_limit_ns, reinterpret_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? BSA_OK : cuda_error(e, "draft_mask launch");
 }
@@ -336,7 +336,7 @@ bsa_status bsa_draft_mask_natural(bsa_plan_t plan, const void* q, const void* k,
   if ((int64_t)g.B * g.Hh * g.nblocks * keep >= (1ll << 31))
     return set_error(BSA_ERR_UNSUPPORTED, "block list longer than 2^31 entries");
   cudaError_t e = launch_draft_mask(g, plan->d_tile_valid, q, k, keep, plan->draft_pooling, row_ptr,
-                                    kv_idx, draft_map, reinterpret_cast<double*>(workspace),
+                                    kv_idx, draft_map, reinterpret_cast<float*>(workspace),
                                     plan->d_status, plan->wait_limit_ns,
                                     reinterpret_cast<cudaStream_t>(stream), /*natural=*/true);
   return e == cudaSuccess ? BSA_OK : cuda_error(e, "draft_mask_natural launch");
@@ -375,7 +375,7 @@ bsa_status bsa_draft_mask_natural_e4m3(bsa_plan_t plan, const void* q, const voi
   if (e != cudaSuccess) return cuda_error(e, "amax reset");
   bool recorded = false;
   e = launch_draft_mask(g, plan->d_tile_valid, q, k, keep, plan->draft_pooling, row_ptr, kv_idx,
-                        draft_map, reinterpret_cast<double*>(workspace), plan->d_status,
+                        draft_map, reinterpret_cast<float*>(workspace), plan->d_status,
                         plan->wait_limit_ns, s, /*natural=*/true, plan->d_amax, &recorded);
   if (e != cudaSuccess) return cuda_error(e, "draft_mask_natural_e4m3 launch");
   e = launch_quantize_e4m3(g, plan->d_amax, q, k, v, q8, k8, v8, scales, s, recorded);

@@ -89,7 +89,7 @@ cudaError_t launch_reorder_inv(const Geometry& g, const void* x_slots, void* x_n
                                cudaStream_t st);
 cudaError_t launch_draft_mask(const Geometry& g, const uint32_t* tile_valid, const void* q,
                               const void* k, int keep, int pooling, int32_t* row_ptr,
-                              int32_t* kv_idx, float* draft_map, double* ws, unsigned int* status,
+                              int32_t* kv_idx, float* draft_map, float* ws, unsigned int* status,
                               uint64_t wait_limit_ns, cudaStream_t st, bool natural = false,
                               uint32_t* amax = nullptr, bool* amax_recorded = nullptr);
 

@@ -95,7 +95,7 @@ class DraftAttention(_Base):
         self.draft_map = (torch.empty(rows * self.plan.nblocks, dtype=torch.float32,
                                       device=device) if want_map else None)
         nbytes = bsa_draft_workspace_bytes(self.plan)
-        self.workspace = torch.empty((nbytes + 7) // 8, dtype=torch.float64, device=device)
+        self.workspace = torch.empty((nbytes + 3) // 4, dtype=torch.float32, device=device)
         self._alloc_slots(device)
 
     def mask(self):

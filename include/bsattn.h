@@ -148,7 +148,7 @@ int64_t bsa_lvsa_nnz(bsa_plan_t plan, int C);
  * k = ceil(Nb*(100 - sparsity_pct)/100), i.e. never sparser than asked. */
 int bsa_draft_keep_count(bsa_plan_t plan, int sparsity_pct);
 
-/* Scratch bytes bsa_draft_mask needs (the pooled Q and K in fp64). */
+/* Scratch bytes bsa_draft_mask needs (the pooled Q and K in fp32). */
 size_t bsa_draft_workspace_bytes(bsa_plan_t plan);
 
 /* Draft mask (Draft Attention article: average pooling of Q and K over each
@@ -156,11 +156,12 @@ size_t bsa_draft_workspace_bytes(bsa_plan_t plan);
  * sparse mask keeping the important blocks at the stated sparsity).
  * Requires a TILE plan.  q_slots, k_slots: slot layout (output of
  * bsa_reorder_fwd).  For every (b, head, query block i):
- *   qbar_i, kbar_j = mean over the tile's tokens inside the grid (fp64,
- *     sequential sum in row-major tile order, one IEEE division), or their
- *     maximum with bsa_plan_set_draft_pooling(BSA_POOL_MAX);
+ *   qbar_i, kbar_j = mean over the tile's tokens inside the grid (fp64
+ *     sequential sum in row-major tile order, one IEEE division, rounded
+ *     once to fp32), or their maximum with
+ *     bsa_plan_set_draft_pooling(BSA_POOL_MAX);
  *   L[i][j] = sum_c qbar_i[c]*kbar_j[c], sequential over c, each product and
- *     sum rounded to fp64 (no fused multiply-add);
+ *     sum rounded to fp32 (no fused multiply-add);
  *   keep the k = bsa_draft_keep_count() blocks j with the largest L[i][j],
  *     ties to the lower j, written ascending.
  * Outputs (device): kv_idx int32[B*Hh*Nb*k]; row_ptr int32[B*Hh*Nb+1] (may be
@@ -179,10 +180,10 @@ bsa_status bsa_draft_mask(bsa_plan_t plan, const void* q_slots, const void* k_sl
  * only input and output buffers, or a caller held to a fixed memory budget
  * where an extra allocation could fail or stall the device mid-step.
  * Same arguments, outputs and results as bsa_draft_mask, minus the workspace:
- * the fp64 scratch lives in a 32 MiB array inside the library
+ * the fp32 scratch lives in a 32 MiB array inside the library
  * (bsa_draft_noalloc_max_scratch_bytes()), held by every GPU that loads the
  * library until the process exits.  Problems needing more scratch than that
- * (2*B*Hh*Nb*D*8 bytes) return BSA_ERR_UNSUPPORTED.  The first call made on a
+ * (2*B*Hh*Nb*D*4 bytes) return BSA_ERR_UNSUPPORTED.  The first call made on a
  * device looks up that array's device address (one cudaGetSymbolAddress);
  * make that first call before any stream capture.  All calls on a device
  * share the array: calls whose kernels overlap on the GPU race on it, calls

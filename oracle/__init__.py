@@ -17,7 +17,9 @@ what the method computes, written from the pages:
   reorder makes the selected blocks contiguous; quantization is named as the
   next step.
 
-All floating point is fp64.  bf16 inputs convert to fp64 exactly.
+Floating point is fp64 (bf16 inputs convert to fp64 exactly), except where
+a float decides an integer in the kernel's precision: the draft logits that
+rank the key blocks are fp32, and the e4m3 scales and divisions are fp32.
 
 Readings of points the pages leave open:
 * window extension order: a right and a left pointer take turns, right
@@ -32,8 +34,10 @@ Readings of points the pages leave open:
   partially filled); sums run sequentially in row-major (a, then b) order and
   the mean is one IEEE division; max pooling takes the maximum over the same
   tokens;
-* draft logits are a sequential multiply-then-add chain over the channels,
-  each operation rounded to fp64 (no fused multiply-add);
+* draft logits are a sequential multiply-then-add chain over the channels
+  of the pooled values rounded to fp32, each operation rounded to fp32 (no
+  fused multiply-add): the pages fix no precision for the draft map, and
+  the top-k that the logits decide is taken in the kernel's precision;
 * top-k per query-block row keeps k = ceil(Nb*(100-p)/100) blocks ranked by
   (logit descending, block index ascending), returned in ascending order;
 * a query with no allowed valid key gets O = 0 and LSE = -inf; pad query
@@ -284,22 +288,28 @@ def draft_pool(x_nat: np.ndarray, T: int, H: int, W: int, ph: int, pw: int,
 
 
 def draft_logits(qbar: np.ndarray, kbar: np.ndarray) -> np.ndarray:
-    """Low-resolution logits L[b,h,i,j] = <qbar_i, kbar_j>, fp64.
+    """Low-resolution logits L[b,h,i,j] = <qbar_i, kbar_j>, in fp32.
 
-    Sequential over channels c = 0..D-1: acc = acc + qbar[i,c]*kbar[j,c], the
-    product and the sum each rounded (no fused multiply-add).
+    The pages fix no precision for the draft map; the top-k decision is taken
+    in the kernel's precision, fp32.  The pooled values are rounded once to
+    fp32 (nearest, ties to even); then, sequentially over channels
+    c = 0..D-1, acc = acc + qbar[i,c]*kbar[j,c] with the product and the sum
+    each rounded to fp32 (no fused multiply-add).  numpy's float32 multiply
+    and add are single IEEE operations.  Returns float32.
     """
-    B, Hh, Nb, D = qbar.shape
-    acc = np.zeros((B, Hh, Nb, kbar.shape[2]), dtype=np.float64)
+    q32 = np.asarray(qbar, dtype=np.float32)
+    k32 = np.asarray(kbar, dtype=np.float32)
+    B, Hh, Nb, D = q32.shape
+    acc = np.zeros((B, Hh, Nb, k32.shape[2]), dtype=np.float32)
     for c in range(D):
-        prod = qbar[:, :, :, c][..., :, None] * kbar[:, :, :, c][..., None, :]
+        prod = q32[:, :, :, c][..., :, None] * k32[:, :, :, c][..., None, :]
         acc = acc + prod
     return acc
 
 
 def draft_map(logits: np.ndarray, D: int) -> np.ndarray:
     """The draft attention map softmax(L / sqrt(D)) over key blocks (fp64)."""
-    z = logits / math.sqrt(D)
+    z = np.asarray(logits, dtype=np.float64) / math.sqrt(D)
     z = z - z.max(axis=-1, keepdims=True)
     e = np.exp(z)
     return e / e.sum(axis=-1, keepdims=True)

@@ -69,7 +69,7 @@ def test_noalloc_matches_workspace_version_on_two_calls_in_a_row():
 def test_noalloc_rejects_problems_above_its_scratch():
     cap = bsa.bsa_draft_noalloc_max_scratch_bytes()
     assert cap == 32 << 20
-    # 40 heads on a 21 x 60 x 104 grid in 8 x 16 tiles: 1344 blocks, 110 MB of scratch
+    # 40 heads on a 21 x 60 x 104 grid in 8 x 16 tiles: 1344 blocks, 55 MB of scratch
     plan = bsa.Plan(1, 40, 128, 21, 60, 104, bsa.LAYOUT_TILE, 8, 16, 128)
     assert bsa.bsa_draft_workspace_bytes(plan) > cap
     buf = torch.empty(16, dtype=torch.int32, device="cuda")
