@@ -329,7 +329,8 @@ def kernel_table(args):
             emit(cid, "reorder_fwd (tile layout, Q K V)", timed(lambda: att.gather(q, k, v)),
                  3 * 2 * tok_bytes)
             nb = att.plan.nblocks
-            pooled = 2 * w.B * w.Hh * nb * w.D * 4
+            pooled = 2 * w.B * w.Hh * nb * w.D * 8      # fp64 draft logits (the default)
+            pooled32 = pooled // 2
             emit(cid, "draft_mask (pool + score/top-k)", timed(att.mask),
                  2 * tok_bytes + 2 * pooled + 4 * att.col_idx.numel(),
                  note=f"k = {att.keep} of {nb} blocks per row")
@@ -356,6 +357,19 @@ def kernel_table(args):
                 emit(cid, "draft pipeline, natural layout (mask, attention)",
                      timed(lambda: att.fused(q, k, v, out)),
                      flops=draft_attended_flops(w, kv_host, att.keep))
+                # the optional fp32 draft logits (their own lists)
+                att32 = DraftAttention(w.B, w.Hh, w.D, w.T, w.H, w.W, w.draft_ph, w.draft_pw,
+                                       w.draft_sparsity, precision=bsa.DRAFT_FP32)
+                emit(cid, "draft_mask_natural, fp32 logits",
+                     timed(lambda: bsa.bsa_draft_mask_natural(att32.plan, q, k, att32.sparsity,
+                                                              att32.row_ptr, att32.col_idx, None,
+                                                              att32.workspace)),
+                     2 * tok_bytes + 2 * pooled32 + 4 * att32.col_idx.numel())
+                emit(cid, "draft pipeline, natural layout, fp32 logits (mask, attention)",
+                     timed(lambda: att32.fused(q, k, v, out)),
+                     flops=draft_attended_flops(w, att32.col_idx.cpu().numpy(), att32.keep))
+                bsa.bsa_poll_status(att32.plan)
+                del att32
                 if w.D == 128:
                     # 8-bit attention: e4m3 Q, K, V (read twice, written at 1 byte)
                     emit(cid, "quantize_e4m3 (Q K V, per-head scales)",
@@ -375,9 +389,10 @@ def kernel_table(args):
 
 
 def draft_pipelines(heads: int):
-    """Runs the three draft pipelines (with reorders, on the natural layout,
-    8-bit) twice each on `heads` heads of the 40-head draft workload: a fixed
-    launch sequence for profilers.  Prints one line."""
+    """Runs the draft pipelines (with reorders, on the natural layout, 8-bit,
+    and on the natural layout with fp32 draft logits) twice each on `heads`
+    heads of the 40-head draft workload: a fixed launch sequence for
+    profilers.  Prints one line."""
     import block_sparse_attention_49_b200 as bsa
     from block_sparse_attention_49_b200.pipeline import DraftAttention
     from synth import small_workload
@@ -385,13 +400,17 @@ def draft_pipelines(heads: int):
     w = small_workload(CONFIGS[5], Hh=heads)
     q, k, v = make_qkv(w, device="cuda")
     att = DraftAttention(w.B, w.Hh, w.D, w.T, w.H, w.W, w.draft_ph, w.draft_pw, w.draft_sparsity)
+    att32 = DraftAttention(w.B, w.Hh, w.D, w.T, w.H, w.W, w.draft_ph, w.draft_pw,
+                           w.draft_sparsity, precision=bsa.DRAFT_FP32)
     out = torch.empty_like(q)
     for _ in range(2):
         att(q, k, v, out)
         att.fused(q, k, v, out)
         att.fused_e4m3(q, k, v, out)
+        att32.fused(q, k, v, out)
     torch.cuda.synchronize()
     bsa.bsa_poll_status(att.plan)
+    bsa.bsa_poll_status(att32.plan)
     print(json.dumps({"draft_pipelines": w.name, "heads": heads}), flush=True)
 
 
@@ -414,7 +433,7 @@ def hbm_kernels(cid: int):
     att = DraftAttention(w.B, w.Hh, w.D, w.T, w.H, w.W, w.draft_ph or 8, w.draft_pw or 16,
                          w.draft_sparsity or 90)
     nb = att.plan.nblocks
-    pooled = 2 * w.B * w.Hh * nb * w.D * 4
+    pooled = 2 * w.B * w.Hh * nb * w.D * 8
     for _ in range(2):
         bsa.bsa_reorder_fwd(fr, q, fq, k, fk, v, fv)
         bsa.bsa_reorder_inv(fr, fq, out)
@@ -432,10 +451,10 @@ def hbm_kernels(cid: int):
         "algo_bytes_per_launch": {
             "reorder_fwd_kernel (Q K V, either layout)": 3 * 2 * tok,
             "reorder_inv_kernel (O, either layout)": 2 * tok,
-            "draft_pool_kernel (tile-layout Q K slots read, pooled fp32 written)":
+            "draft_pool_kernel (tile-layout Q K slots read, pooled fp64 written)":
                 2 * w.B * w.Hh * att.plan.Npad * w.D * 2 + pooled,
-            "draft_pool_kernel natural (natural Q K read, pooled fp32 written)": 2 * tok + pooled,
-            "draft_score_reg_kernel (pooled fp32 read, lists written)":
+            "draft_pool_kernel natural (natural Q K read, pooled fp64 written)": 2 * tok + pooled,
+            "draft_score_reg_kernel (pooled fp64 read, lists written)":
                 pooled + 4 * att.col_idx.numel(),
             "e4m3_amax_kernel (Q K V read)": 3 * tok,
             "e4m3_convert_kernel (Q K V read, codes written)": 3 * tok + 3 * tok // 2},
@@ -737,7 +756,7 @@ def draft_step_setup(w, q, k, v, out):
     torch.cuda.synchronize()
     flops = draft_attended_flops(w, att.col_idx.cpu().numpy(), att.keep)
     tok_bytes = w.B * w.N * w.Hh * w.D * 2
-    pooled = 2 * w.B * w.Hh * att.plan.nblocks * w.D * 4
+    pooled = 2 * w.B * w.Hh * att.plan.nblocks * w.D * 8
     extra = {
         "metric": f"bsattn ms/call + attended TFLOP/s (% BF16 peak), {w.name}, draft attention",
         "poll": lambda: bsa.bsa_poll_status(att.plan),

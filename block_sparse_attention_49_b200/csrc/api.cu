@@ -219,7 +219,7 @@ int bsa_draft_keep_count(bsa_plan_t plan, int sparsity_pct) {
 }
 
 size_t bsa_draft_workspace_bytes(bsa_plan_t plan) {
-  return plan ? draft_workspace_bytes(plan->g) : 0;
+  return plan ? draft_workspace_bytes(plan->g, plan->draft_precision) : 0;
 }
 
 bsa_status bsa_draft_mask(bsa_plan_t plan, const void* q_slots, const void* k_slots,
@@ -235,7 +235,7 @@ bsa_status bsa_draft_mask(bsa_plan_t plan, const void* q_slots, const void* k_sl
   if ((st = check_ptr(k_slots, "k_slots")) != BSA_OK) return st;
   if ((st = check_ptr(workspace, "workspace")) != BSA_OK) return st;
   if (!kv_idx) return set_error(BSA_ERR_INVALID_ARG, "kv_idx is NULL");
-  if (workspace_bytes < draft_workspace_bytes(g))
+  if (workspace_bytes < draft_workspace_bytes(g, plan->draft_precision))
     return set_error(BSA_ERR_INVALID_ARG, "workspace too small");
   if (g.nblocks > 18000) return set_error(BSA_ERR_UNSUPPORTED, "draft mask supports up to 18000 blocks");
   if ((int64_t)g.B * g.Hh * g.Npad >= (1ll << 31))
@@ -244,9 +244,8 @@ bsa_status bsa_draft_mask(bsa_plan_t plan, const void* q_slots, const void* k_sl
   if ((int64_t)g.B * g.Hh * g.nblocks * keep >= (1ll << 31))
     return set_error(BSA_ERR_UNSUPPORTED, "block list longer than 2^31 entries");
   cudaError_t e = launch_draft_mask(g, plan->d_tile_valid, q_slots, k_slots, keep,
-                                    plan->draft_pooling, row_ptr, kv_idx, draft_map,
-                                    reinterpret_cast<float*>(workspace), plan->d_status,
-                                    plan->wait_limit_ns, reinterpret_cast<cudaStream_t>(stream));
+                                    plan->draft_pooling, plan->draft_precision, row_ptr, kv_idx,
+                                    draft_map, workspace, reinterpret_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? BSA_OK : cuda_error(e, "draft_mask launch");
 }
 
@@ -327,7 +326,7 @@ bsa_status bsa_draft_mask_natural(bsa_plan_t plan, const void* q, const void* k,
   if ((st = check_ptr(k, "k")) != BSA_OK) return st;
   if ((st = check_ptr(workspace, "workspace")) != BSA_OK) return st;
   if (!kv_idx) return set_error(BSA_ERR_INVALID_ARG, "kv_idx is NULL");
-  if (workspace_bytes < draft_workspace_bytes(g))
+  if (workspace_bytes < draft_workspace_bytes(g, plan->draft_precision))
     return set_error(BSA_ERR_INVALID_ARG, "workspace too small");
   if (g.nblocks > 18000) return set_error(BSA_ERR_UNSUPPORTED, "draft mask supports up to 18000 blocks");
   if ((int64_t)g.B * g.Hh * g.Npad >= (1ll << 31))
@@ -335,9 +334,8 @@ bsa_status bsa_draft_mask_natural(bsa_plan_t plan, const void* q, const void* k,
   const int keep = bsa_draft_keep_count(plan, sparsity_pct);
   if ((int64_t)g.B * g.Hh * g.nblocks * keep >= (1ll << 31))
     return set_error(BSA_ERR_UNSUPPORTED, "block list longer than 2^31 entries");
-  cudaError_t e = launch_draft_mask(g, plan->d_tile_valid, q, k, keep, plan->draft_pooling, row_ptr,
-                                    kv_idx, draft_map, reinterpret_cast<float*>(workspace),
-                                    plan->d_status, plan->wait_limit_ns,
+  cudaError_t e = launch_draft_mask(g, plan->d_tile_valid, q, k, keep, plan->draft_pooling,
+                                    plan->draft_precision, row_ptr, kv_idx, draft_map, workspace,
                                     reinterpret_cast<cudaStream_t>(stream), /*natural=*/true);
   return e == cudaSuccess ? BSA_OK : cuda_error(e, "draft_mask_natural launch");
 }
@@ -360,7 +358,7 @@ bsa_status bsa_draft_mask_natural_e4m3(bsa_plan_t plan, const void* q, const voi
   if (!scales || (reinterpret_cast<uintptr_t>(scales) & 3u))
     return set_error(BSA_ERR_ALIGNMENT, "scales is NULL or not 4-byte aligned");
   if (!kv_idx) return set_error(BSA_ERR_INVALID_ARG, "kv_idx is NULL");
-  if (workspace_bytes < draft_workspace_bytes(g))
+  if (workspace_bytes < draft_workspace_bytes(g, plan->draft_precision))
     return set_error(BSA_ERR_INVALID_ARG, "workspace too small");
   if (g.nblocks > 18000) return set_error(BSA_ERR_UNSUPPORTED, "draft mask supports up to 18000 blocks");
   if ((int64_t)g.B * g.Hh * g.Npad >= (1ll << 31))
@@ -374,9 +372,9 @@ bsa_status bsa_draft_mask_natural_e4m3(bsa_plan_t plan, const void* q, const voi
   cudaError_t e = cudaMemsetAsync(plan->d_amax, 0, sizeof(uint32_t) * 3 * g.B * g.Hh, s);
   if (e != cudaSuccess) return cuda_error(e, "amax reset");
   bool recorded = false;
-  e = launch_draft_mask(g, plan->d_tile_valid, q, k, keep, plan->draft_pooling, row_ptr, kv_idx,
-                        draft_map, reinterpret_cast<float*>(workspace), plan->d_status,
-                        plan->wait_limit_ns, s, /*natural=*/true, plan->d_amax, &recorded);
+  e = launch_draft_mask(g, plan->d_tile_valid, q, k, keep, plan->draft_pooling,
+                        plan->draft_precision, row_ptr, kv_idx, draft_map, workspace, s,
+                        /*natural=*/true, plan->d_amax, &recorded);
   if (e != cudaSuccess) return cuda_error(e, "draft_mask_natural_e4m3 launch");
   e = launch_quantize_e4m3(g, plan->d_amax, q, k, v, q8, k8, v8, scales, s, recorded);
   return e == cudaSuccess ? BSA_OK : cuda_error(e, "quantize_e4m3 launch");
@@ -448,6 +446,14 @@ bsa_status bsa_plan_set_draft_pooling(bsa_plan_t plan, int pooling) {
   if (pooling != BSA_POOL_MEAN && pooling != BSA_POOL_MAX)
     return set_error(BSA_ERR_INVALID_ARG, "unknown pooling");
   plan->draft_pooling = pooling;
+  return BSA_OK;
+}
+
+bsa_status bsa_plan_set_draft_precision(bsa_plan_t plan, int precision) {
+  if (!plan) return set_error(BSA_ERR_INVALID_ARG, "plan is NULL");
+  if (precision != BSA_DRAFT_FP64 && precision != BSA_DRAFT_FP32)
+    return set_error(BSA_ERR_INVALID_ARG, "unknown draft precision");
+  plan->draft_precision = precision;
   return BSA_OK;
 }
 

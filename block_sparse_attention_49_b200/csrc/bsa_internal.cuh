@@ -68,6 +68,7 @@ struct bsa_plan_s {
   int lvsa_anchors = BSA_ANCHORS_ROTATING;  // bsa_plan_set_lvsa_variant
   int lvsa_window = BSA_WINDOW_ALTERNATE;
   int draft_pooling = BSA_POOL_MEAN;        // bsa_plan_set_draft_pooling
+  int draft_precision = BSA_DRAFT_FP64;     // bsa_plan_set_draft_precision
   uint32_t* d_amax = nullptr;               // [3][B][Hh] scratch of bsa_quantize_e4m3
 };
 
@@ -88,10 +89,10 @@ cudaError_t launch_reorder_fwd(const Geometry& g, const void* const x[3], void* 
 cudaError_t launch_reorder_inv(const Geometry& g, const void* x_slots, void* x_nat,
                                cudaStream_t st);
 cudaError_t launch_draft_mask(const Geometry& g, const uint32_t* tile_valid, const void* q,
-                              const void* k, int keep, int pooling, int32_t* row_ptr,
-                              int32_t* kv_idx, float* draft_map, float* ws, unsigned int* status,
-                              uint64_t wait_limit_ns, cudaStream_t st, bool natural = false,
-                              uint32_t* amax = nullptr, bool* amax_recorded = nullptr);
+                              const void* k, int keep, int pooling, int precision,
+                              int32_t* row_ptr, int32_t* kv_idx, float* draft_map, void* ws,
+                              cudaStream_t st, bool natural = false, uint32_t* amax = nullptr,
+                              bool* amax_recorded = nullptr);
 
 // e4m3 quantization of natural-layout Q, K, V (scales [3][B][Hh]).
 // qk_amax_ready: amax_ws already holds the maxima of Q and K (and zero for V).
@@ -138,7 +139,7 @@ int edge_kinds(const Geometry& g, int kind[3], int rows[3], int bw[3], int bh[3]
 cudaError_t launch_selftest_timeout(unsigned int* status, uint64_t limit_ns, cudaStream_t st);
 
 // Size bookkeeping shared by the API and the draft kernels.
-size_t draft_workspace_bytes(const Geometry& g);
-int draft_rows_per_cta(int64_t nblocks);
+size_t draft_workspace_bytes(const Geometry& g, int precision);
+int draft_rows_per_cta(int64_t nblocks, int precision);
 
 }  // namespace bsa

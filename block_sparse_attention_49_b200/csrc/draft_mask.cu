@@ -35,7 +35,6 @@ namespace {
 
 constexpr int kScoreThreads = 256;
 constexpr int kKeyChunk = 32;  // key blocks staged in shared memory per step
-constexpr int kRegCand = 16;   // top-k candidates per lane held in registers (Nb <= 512)
 constexpr unsigned kFullMaskScore = 0xffffffffu;
 
 // ---------------------------------------------------------------------------
@@ -60,10 +59,12 @@ struct PoolParams {
   int use_max;
   const uint32_t* tile_valid;
   uint32_t* amax;  // [3][B][Hh] float bits, or null
-  float* ws;
+  // pooled Q then K: fp32 always; with F64 first the fp64 values, then the
+  // fp32 copies, then the fp32 2-norms (rounded up) of the fp64 values
+  void* ws;
 };
 
-template <int D, bool NAT, bool MAXP, bool AMAX>
+template <int D, bool NAT, bool MAXP, bool AMAX, bool F64>
 __global__ void __launch_bounds__(kPoolThreads, 4)
     draft_pool_kernel(const uint4* __restrict__ q, const uint4* __restrict__ k, const PoolParams p) {
   constexpr int kTPG = D / 8;  // threads per group
@@ -95,6 +96,7 @@ __global__ void __launch_bounds__(kPoolThreads, 4)
 #pragma unroll
   for (int e = 0; e < 8; ++e) acc[e] = use_max ? -INFINITY : 0.0;
   float mabs = 0.f;
+  double ss = 0.0;  // F64: this thread's share of the squared 2-norm
   int cnt = 0;
   // rows [0, len) from `rowp`, in order, four loads ahead of the additions
   auto run = [&](const uint4* rowp, int len) {
@@ -148,15 +150,41 @@ __global__ void __launch_bounds__(kPoolThreads, 4)
         }
       }
     }
-    float* dst = p.ws + ((int64_t)which * p.groups_per_tensor +
-                         ((int64_t)b * p.Hh + h) * p.nblocks + blk) * D + sub * 8;
+    const int64_t at = ((int64_t)which * p.groups_per_tensor +
+                        ((int64_t)b * p.Hh + h) * p.nblocks + blk) * D + sub * 8;
     const double dc = (double)cnt;
-    float o[8];
+    double o[8];
 #pragma unroll
-    for (int e = 0; e < 8; ++e)
-      o[e] = __double2float_rn(cnt ? (use_max ? acc[e] : __ddiv_rn(acc[e], dc)) : 0.0);
-    reinterpret_cast<float4*>(dst)[0] = make_float4(o[0], o[1], o[2], o[3]);
-    reinterpret_cast<float4*>(dst)[1] = make_float4(o[4], o[5], o[6], o[7]);
+    for (int e = 0; e < 8; ++e) o[e] = cnt ? (use_max ? acc[e] : __ddiv_rn(acc[e], dc)) : 0.0;
+    const int64_t n_all = 2 * p.groups_per_tensor * D;  // values of Q and K
+    float* ws32 = static_cast<float*>(p.ws);
+    if (F64) {
+      double2* dst = reinterpret_cast<double2*>(static_cast<double*>(p.ws) + at);
+#pragma unroll
+      for (int e = 0; e < 4; ++e) dst[e] = make_double2(o[2 * e], o[2 * e + 1]);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) ss = fma(o[e], o[e], ss);
+      ws32 = reinterpret_cast<float*>(static_cast<double*>(p.ws) + n_all);
+    }
+    float4* dst = reinterpret_cast<float4*>(ws32 + at);
+    dst[0] = make_float4(__double2float_rn(o[0]), __double2float_rn(o[1]),
+                         __double2float_rn(o[2]), __double2float_rn(o[3]));
+    dst[1] = make_float4(__double2float_rn(o[4]), __double2float_rn(o[5]),
+                         __double2float_rn(o[6]), __double2float_rn(o[7]));
+  }
+  if (F64) {
+    // 2-norm of the unit's fp64 values, an upper bound: the squares' sum in
+    // fp64 (relative error below D * 2^-53), its square root grown by 2^-40
+    // and rounded up to fp32.  Lanes of a group are kTPG consecutive lanes.
+#pragma unroll
+    for (int o = kTPG / 2; o > 0; o >>= 1) ss += __shfl_xor_sync(kFullMaskScore, ss, o);
+    if (live && sub == 0) {
+      float* norms = reinterpret_cast<float*>(static_cast<double*>(p.ws) +
+                                              2 * p.groups_per_tensor * D) +
+                     2 * p.groups_per_tensor * D;
+      norms[(int64_t)which * p.groups_per_tensor + ((int64_t)b * p.Hh + h) * p.nblocks + blk] =
+          __double2float_ru(sqrt(ss) * (1.0 + 0x1p-40));
+    }
   }
   if (AMAX) {
     // max |x| of the group's tile: lanes of a group are kTPG consecutive lanes
@@ -170,7 +198,8 @@ __global__ void __launch_bounds__(kPoolThreads, 4)
 
 template <int D>
 cudaError_t launch_pool(const Geometry& g, const uint32_t* tile_valid, const void* q, const void* k,
-                        int use_max, bool natural, float* ws, uint32_t* amax, cudaStream_t st) {
+                        int use_max, bool natural, bool f64, void* ws, uint32_t* amax,
+                        cudaStream_t st) {
   PoolParams p;
   p.B = g.B;
   p.Hh = g.Hh;
@@ -193,13 +222,18 @@ cudaError_t launch_pool(const Geometry& g, const uint32_t* tile_valid, const voi
   const unsigned grid = (unsigned)((threads + kPoolThreads - 1) / kPoolThreads);
   auto qq = reinterpret_cast<const uint4*>(q);
   auto kk = reinterpret_cast<const uint4*>(k);
-  auto pick = [&](auto nat) {
-    constexpr bool NAT = decltype(nat)::value;
+  auto pick = [&](auto nat, auto wide) {
+    constexpr bool NAT = decltype(nat)::value, F64 = decltype(wide)::value;
     if (use_max)
-      return amax ? draft_pool_kernel<D, NAT, true, true> : draft_pool_kernel<D, NAT, true, false>;
-    return amax ? draft_pool_kernel<D, NAT, false, true> : draft_pool_kernel<D, NAT, false, false>;
+      return amax ? draft_pool_kernel<D, NAT, true, true, F64>
+                  : draft_pool_kernel<D, NAT, true, false, F64>;
+    return amax ? draft_pool_kernel<D, NAT, false, true, F64>
+                : draft_pool_kernel<D, NAT, false, false, F64>;
   };
-  auto kern = natural ? pick(std::true_type{}) : pick(std::false_type{});
+  auto kern = natural ? (f64 ? pick(std::true_type{}, std::true_type{})
+                             : pick(std::true_type{}, std::false_type{}))
+                      : (f64 ? pick(std::false_type{}, std::true_type{})
+                             : pick(std::false_type{}, std::false_type{}));
   kern<<<grid, kPoolThreads, 0, st>>>(qq, kk, p);
   return cudaGetLastError();
 }
@@ -215,30 +249,37 @@ __device__ __forceinline__ float key_value(uint32_t k) {
   return __uint_as_float((k >> 31) ? (k & 0x7fffffffu) : ~k);
 }
 
-// grid: (ceil(nblocks / R), Hh, B); R query rows per CTA.
-template <int D>
+__device__ __forceinline__ float mul_rn(float a, float b) { return __fmul_rn(a, b); }
+__device__ __forceinline__ double mul_rn(double a, double b) { return __dmul_rn(a, b); }
+__device__ __forceinline__ float add_rn(float a, float b) { return __fadd_rn(a, b); }
+__device__ __forceinline__ double add_rn(double a, double b) { return __dadd_rn(a, b); }
+
+// grid: (ceil(nblocks / R), Hh, B); R query rows per CTA.  Rows of more than
+// 512 key blocks: the logits of R rows in shared memory.
+template <int D, typename T>
 __global__ void __launch_bounds__(kScoreThreads)
-    draft_score_topk_kernel(const float* __restrict__ qbar, const float* __restrict__ kbar,
-                            int Hh, int nblocks, int R, int keep, int32_t* __restrict__ row_ptr,
+    draft_score_topk_kernel(const T* __restrict__ qbar, const T* __restrict__ kbar, int Hh,
+                            int nblocks, int R, int keep, int32_t* __restrict__ row_ptr,
                             int32_t* __restrict__ kv_idx, float* __restrict__ draft_map) {
+  using T2 = typename std::conditional<std::is_same<T, double>::value, double2, float2>::type;
   constexpr int kWarps = kScoreThreads / 32;
-  constexpr int kKStride = D + 2;  // even: 8-byte loads of two channels, no bank conflicts
-  extern __shared__ float2 shf2[];
-  float* sq = reinterpret_cast<float*>(shf2);  // [kWarps][D][2]: rows w and w + kWarps
-  float* sk = sq + 2 * kWarps * D;             // [kKeyChunk][kKStride]
-  float* sl = sk + kKeyChunk * kKStride;       // [R][nblocks] logits
+  constexpr int kKStride = D + 2;  // even: two-channel loads, no bank conflicts
+  extern __shared__ double4 shd4[];
+  T* sq = reinterpret_cast<T*>(shd4);      // [kWarps][D][2]: rows w and w + kWarps
+  T* sk = sq + 2 * kWarps * D;             // [kKeyChunk][kKStride]
+  T* sl = sk + kKeyChunk * kKStride;       // [R][nblocks] logits
   uint8_t* sel = reinterpret_cast<uint8_t*>(sl + (int64_t)R * nblocks);  // [R][nblocks]
   const int h = blockIdx.y, b = blockIdx.z;
   const int64_t bh = (int64_t)b * Hh + h;
   const int r0 = blockIdx.x * R;
   const int rows = min(R, nblocks - r0);  // R <= 2 * kWarps
-  const float* qb = qbar + (bh * nblocks + r0) * D;
-  const float* kb = kbar + bh * nblocks * D;
+  const T* qb = qbar + (bh * nblocks + r0) * D;
+  const T* kb = kbar + bh * nblocks * D;
   // warp w carries rows w and w + kWarps: their values at channel c sit side
-  // by side (one broadcast 8-byte load); missing rows read zeros
+  // by side (one broadcast load); missing rows read zeros
   for (int i = threadIdx.x; i < 2 * kWarps * D; i += kScoreThreads) {
     const int r = i / D, c = i - r * D;
-    sq[((r % kWarps) * D + c) * 2 + r / kWarps] = r < rows ? qb[i] : 0.f;
+    sq[((r % kWarps) * D + c) * 2 + r / kWarps] = r < rows ? qb[i] : T(0);
   }
   for (int i = threadIdx.x; i < rows * nblocks; i += kScoreThreads) sel[i] = 0;
 
@@ -246,13 +287,13 @@ __global__ void __launch_bounds__(kScoreThreads)
   // key chunks: the next chunk is loaded into registers while the current
   // one is used, then stored to shared memory (padded stride: no conflicts)
   constexpr int kPer = kKeyChunk * D / kScoreThreads;
-  float pre[kPer];
+  T pre[kPer];
   auto load_chunk = [&](int j0) {
 #pragma unroll
     for (int u = 0; u < kPer; ++u) {
       const int idx = threadIdx.x + u * kScoreThreads;
       const int jj = idx / D, c = idx - jj * D;
-      pre[u] = (j0 + jj < nblocks) ? kb[(int64_t)(j0 + jj) * D + c] : 0.f;
+      pre[u] = (j0 + jj < nblocks) ? kb[(int64_t)(j0 + jj) * D + c] : T(0);
     }
   };
   load_chunk(0);
@@ -271,17 +312,17 @@ __global__ void __launch_bounds__(kScoreThreads)
     // lane = key block within the chunk.  Each logit is still the sequential
     // multiply-then-add over c.
     if (lane < nj && warp < rows) {
-      const float2* kk = reinterpret_cast<const float2*>(sk + lane * kKStride);
-      const float2* qq = reinterpret_cast<const float2*>(sq) + warp * D;
-      float acc_a = 0.f, acc_b = 0.f;
+      const T2* kk = reinterpret_cast<const T2*>(sk + lane * kKStride);
+      const T2* qq = reinterpret_cast<const T2*>(sq) + warp * D;
+      T acc_a = T(0), acc_b = T(0);
 #pragma unroll 4
       for (int c2 = 0; c2 < D / 2; ++c2) {
-        const float2 kc = kk[c2];
-        const float2 q0 = qq[2 * c2], q1 = qq[2 * c2 + 1];
-        acc_a = __fadd_rn(acc_a, __fmul_rn(q0.x, kc.x));
-        acc_b = __fadd_rn(acc_b, __fmul_rn(q0.y, kc.x));
-        acc_a = __fadd_rn(acc_a, __fmul_rn(q1.x, kc.y));
-        acc_b = __fadd_rn(acc_b, __fmul_rn(q1.y, kc.y));
+        const T2 kc = kk[c2];
+        const T2 q0 = qq[2 * c2], q1 = qq[2 * c2 + 1];
+        acc_a = add_rn(acc_a, mul_rn(q0.x, kc.x));
+        acc_b = add_rn(acc_b, mul_rn(q0.y, kc.x));
+        acc_a = add_rn(acc_a, mul_rn(q1.x, kc.y));
+        acc_b = add_rn(acc_b, mul_rn(q1.y, kc.y));
       }
       sl[(int64_t)warp * nblocks + j0 + lane] = acc_a;
       if (warp + kWarps < rows) sl[(int64_t)(warp + kWarps) * nblocks + j0 + lane] = acc_b;
@@ -292,68 +333,32 @@ __global__ void __launch_bounds__(kScoreThreads)
   // top-k per row, one warp per row: k rounds of a warp-wide arg-max (larger
   // logit first, then the lower block index)
   for (int r = warp; r < rows; r += kWarps) {
-    const float* L = sl + (int64_t)r * nblocks;
+    const T* L = sl + (int64_t)r * nblocks;
     uint8_t* sr = sel + (int64_t)r * nblocks;
-    if (nblocks <= 32 * kRegCand) {
-      // candidates j = lane + 32u held in registers as order-preserving
-      // keys; `avail` marks the ones not yet taken.  A round takes the
-      // largest key, then the lowest index among equal keys (two warp
-      // reductions).
-      uint32_t key[kRegCand];
-      uint32_t avail = 0u;
-#pragma unroll
-      for (int u = 0; u < kRegCand; ++u) {
-        const int j = lane + 32 * u;
-        key[u] = j < nblocks ? order_key(L[j]) : 0u;
-        if (j < nblocks) avail |= 1u << u;
-      }
-      const uint32_t start = avail;
-      for (int it = 0; it < keep; ++it) {
-        uint32_t bk = 0u;
-        int bu = -1;
-#pragma unroll
-        for (int u = 0; u < kRegCand; ++u)
-          if (((avail >> u) & 1u) && (bu < 0 || key[u] > bk)) {
-            bk = key[u];
-            bu = u;
-          }
-        const uint32_t top = __reduce_max_sync(0xffffffffu, bk);
-        const uint32_t idx = (bu >= 0 && bk == top) ? (uint32_t)(lane + 32 * bu) : 0xffffffffu;
-        const uint32_t win = __reduce_min_sync(0xffffffffu, idx);
-        if (win != 0xffffffffu && (int)(win & 31u) == lane) avail &= ~(1u << (win >> 5));
+    for (int it = 0; it < keep; ++it) {
+      T best = T(0);
+      int bidx = 0x7fffffff;
+      for (int j = lane; j < nblocks; j += 32) {
+        if (sr[j]) continue;
+        const T v = L[j];
+        if (bidx == 0x7fffffff || v > best) {  // j ascends: equal values keep the lower j
+          best = v;
+          bidx = j;
+        }
       }
 #pragma unroll
-      for (int u = 0; u < kRegCand; ++u) {
-        const int j = lane + 32 * u;
-        if (j < nblocks) sr[j] = (((start & ~avail) >> u) & 1u) ? 1 : 0;
+      for (int o = 16; o > 0; o >>= 1) {
+        const T ov = __shfl_xor_sync(0xffffffffu, best, o);
+        const int oi = __shfl_xor_sync(0xffffffffu, bidx, o);
+        const bool take = (oi != 0x7fffffff) &&
+                          (bidx == 0x7fffffff || ov > best || (ov == best && oi < bidx));
+        if (take) {
+          best = ov;
+          bidx = oi;
+        }
       }
+      if (lane == 0 && bidx != 0x7fffffff) sr[bidx] = 1;
       __syncwarp();
-    } else {
-      for (int it = 0; it < keep; ++it) {
-        float best = -FLT_MAX;
-        int bidx = 0x7fffffff;
-        for (int j = lane; j < nblocks; j += 32) {
-          if (sr[j]) continue;
-          const float v = L[j];
-          if (bidx == 0x7fffffff || v > best || (v == best && j < bidx)) {
-            best = v;
-            bidx = j;
-          }
-        }
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) {
-          const float ov = __shfl_xor_sync(0xffffffffu, best, o);
-          const int oi = __shfl_xor_sync(0xffffffffu, bidx, o);
-          const bool take = (oi != 0x7fffffff) &&
-                            (bidx == 0x7fffffff || ov > best || (ov == best && oi < bidx));
-          if (take) {
-            best = ov;
-            bidx = oi;
-          }
-        }
-        if (lane == 0 && bidx != 0x7fffffff) sr[bidx] = 1;
-        __syncwarp();
-      }
     }
     // ascending output
     const int64_t grow = bh * nblocks + r0 + r;
@@ -395,17 +400,19 @@ __global__ void __launch_bounds__(kScoreThreads)
 //
 // A warp owns R whole query-block rows; lane l accumulates the logits of key
 // blocks j = l + 32u (u < U) of each row, so a row's top-k runs straight out
-// of registers and no logit ever goes to shared memory.  Rows are held in
-// pairs, one fp32 pair per key, and updated with the two-wide fp32 multiply
-// and add (each lane of the pair rounded on its own, so every logit is still
-// the sequential multiply-then-add chain over c = 0..D-1).  The CTA's warps
-// share the pooled keys, staged CK channels at a time in a two-stage
-// cp.async ring as [channel quad][key][4] (a lane reads four channels of one
-// key with one 16-byte load; a warp's loads are contiguous); the pooled query
-// values are staged as [channel][row], so a row pair is one broadcast load.
+// of registers and no logit ever goes to shared memory.  Every logit is the
+// sequential multiply-then-add chain over c = 0..D-1, each operation rounded
+// to the logit's precision.
+//   fp32: rows are held in pairs, one fp32 pair per key, updated with the
+//     two-wide fp32 multiply and add (each lane of the pair rounded on its
+//     own); keys staged 16 channels at a time as [channel quad][key][4].
+//   fp64: one double per (row, key); keys staged 8 channels at a time as
+//     [channel pair][key][2].
+// Either way a lane reads one key's channels with one 16-byte load and a
+// warp's loads are contiguous; the pooled query values are staged as
+// [channel][row] and read by broadcast.
 // ---------------------------------------------------------------------------
 constexpr int kRegScoreWarps = 4;
-constexpr int kRegScoreCK = 16;  // channels per stage
 
 __device__ __forceinline__ void cp_async4(void* dst, const void* src, bool valid) {
   asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;" ::"r"(smem_u32(dst)), "l"(src),
@@ -426,21 +433,43 @@ __device__ __forceinline__ void cp_async_wait() {
 template <int U>
 struct RegScoreCfg {
   static constexpr int R = 4;                          // rows per warp (pairs)
+  static constexpr int CK = 16;                        // channels per stage
   static constexpr int kRows = R * kRegScoreWarps;     // rows per CTA
   static constexpr int NK = 32 * U;                    // keys, padded
-  static constexpr int kStageK = kRegScoreCK * NK;     // floats per K stage
-  static constexpr int kStageQ = kRegScoreCK * kRows;  // floats per Q stage
+  static constexpr int kStageK = CK * NK;              // floats per K stage
+  static constexpr int kStageQ = CK * kRows;           // floats per Q stage
   static constexpr size_t kSmem = 2 * (size_t)(kStageK + kStageQ) * sizeof(float);
+  // the fp64 refinement's per-warp list of (logit, block) in the same space
+  static_assert(kRegScoreWarps * NK * 12 <= (int)kSmem, "refinement list fits");
 };
 
-// grid: (ceil(nblocks / kRows), Hh, B)
-template <int D, int U>
+// |fp32 logit - fp64 logit| <= kErrBound * |qbar| * |kbar| + 2^-100 for the
+// sequential unfused chains of D products: gamma_D(fp32) on the fp32 chain
+// (of inputs within 2^-24 of the fp64 ones: (1 + 2^-24)^2 - 1 on each
+// product) plus gamma_D(fp64) on the fp64 chain, where gamma_n = n u / (1 -
+// n u) (Higham, "Accuracy and Stability of Numerical Algorithms", sections
+// 3.1 and 3.5), and sum |q_c k_c| <= |q| |k|; doubled as a margin.  The
+// absolute term covers fp32 underflow.
+template <int D>
+struct ErrBound {
+  static constexpr double u32 = 0x1p-24, u64 = 0x1p-53;
+  static constexpr double g32 = D * u32 / (1.0 - D * u32), g64 = D * u64 / (1.0 - D * u64);
+  static constexpr double value = 2.0 * (g32 * (1.0 + u32) * (1.0 + u32) + 2.0 * u32 + u32 * u32 + g64);
+};
+
+// grid: (ceil(nblocks / kRows), Hh, B).  CERT: the plan's precision is fp64;
+// the fp32 logits pick the blocks that are certain under the error bound,
+// and only the ones within it of the k-th logit get their fp64 logits (from
+// q64 / k64), so the lists are those of the fp64 chains.
+template <int D, int U, bool CERT>
 __global__ void __launch_bounds__(32 * kRegScoreWarps, U <= 12 ? 4 : 3)
     draft_score_reg_kernel(const float* __restrict__ qbar, const float* __restrict__ kbar,
                            int Hh, int nblocks, int keep, int32_t* __restrict__ row_ptr,
-                           int32_t* __restrict__ kv_idx, float* __restrict__ draft_map) {
+                           int32_t* __restrict__ kv_idx, float* __restrict__ draft_map,
+                           const double* __restrict__ q64, const double* __restrict__ k64,
+                           const float* __restrict__ qnorm, const float* __restrict__ knorm) {
   using Cfg = RegScoreCfg<U>;
-  constexpr int R = Cfg::R, RP = R / 2, CK = kRegScoreCK, NK = Cfg::NK;
+  constexpr int R = Cfg::R, RP = R / 2, CK = Cfg::CK, NK = Cfg::NK;
   constexpr int kThreads = 32 * kRegScoreWarps;
   static_assert(D % CK == 0 && CK % 4 == 0 && R % 2 == 0, "staging shape");
   extern __shared__ float4 shf4[];
@@ -510,7 +539,7 @@ __global__ void __launch_bounds__(32 * kRegScoreWarps, U <= 12 ? 4 : 3)
         }
       }
     }
-    __syncthreads();  // the next issue() overwrites this stage
+    __syncthreads();  // the next issue() overwrites this stage (or the refinement lists)
   }
 
   // top-k of each row (larger logit first, then the lower block index).
@@ -530,15 +559,15 @@ __global__ void __launch_bounds__(32 * kRegScoreWarps, U <= 12 ? 4 : 3)
       key[r][u] = (row_in && lane + 32 * u < nblocks) ? order_key((r & 1) ? hi : lo) : 0u;
     }
   }
-  uint32_t T[R];
+  uint32_t Tk[R];
 #pragma unroll
-  for (int r = 0; r < R; ++r) T[r] = 0u;
+  for (int r = 0; r < R; ++r) Tk[r] = 0u;
 #pragma unroll 1
   for (int bit = 31; bit >= 0; --bit) {
     unsigned tot[R];
 #pragma unroll
     for (int r = 0; r < R; ++r) {
-      const uint32_t cand = T[r] | (1u << bit);
+      const uint32_t cand = Tk[r] | (1u << bit);
       unsigned c = 0;
 #pragma unroll
       for (int u = 0; u < U; ++u) c += key[r][u] >= cand ? 1u : 0u;
@@ -546,24 +575,136 @@ __global__ void __launch_bounds__(32 * kRegScoreWarps, U <= 12 ? 4 : 3)
     }
 #pragma unroll
     for (int r = 0; r < R; ++r)
-      if (tot[r] >= (unsigned)keep) T[r] |= 1u << bit;
+      if (tot[r] >= (unsigned)keep) Tk[r] |= 1u << bit;
+  }
+  float kmax = 0.f;  // CERT: the largest key-block norm of this (b, head)
+  if constexpr (CERT) {
+#pragma unroll
+    for (int u = 0; u < U; ++u)
+      if (lane + 32 * u < nblocks) kmax = fmaxf(kmax, knorm[bh * nblocks + lane + 32 * u]);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) kmax = fmaxf(kmax, __shfl_xor_sync(kFullMaskScore, kmax, o));
   }
   const uint32_t below = (1u << lane) - 1u;
 #pragma unroll
   for (int r = 0; r < R; ++r) {
     const int row = r0 + warp * R + r;
     if (row >= nblocks) break;  // warp-uniform
-    unsigned c_gt = 0;
-#pragma unroll
-    for (int u = 0; u < U; ++u) c_gt += key[r][u] > T[r] ? 1u : 0u;
-    int eq_left = keep - (int)__reduce_add_sync(kFullMaskScore, c_gt);
     uint32_t taken = 0u;
+    bool by_index = true;
+    if constexpr (CERT) {
+      // blocks whose fp32 logit lies more than twice the bound above the
+      // k-th one are in, more than twice below it out, whatever the fp64
+      // logits; the rest (the band) is decided on the fp64 logits unless
+      // all of it is needed
+      const double t = (double)key_value(Tk[r]);
+      const double e = ErrBound<D>::value * (double)qnorm[bh * nblocks + row] * (double)kmax + 0x1p-100;
+      double lo = t - 2.0 * e, hi = t + 2.0 * e;
+      if (!(lo > -INFINITY && hi < INFINITY)) {  // overflow or NaN: decide all in fp64
+        lo = -INFINITY;
+        hi = INFINITY;
+      }
+      uint32_t band = 0u;
 #pragma unroll
-    for (int u = 0; u < U; ++u) {  // block order: u, then lane
-      const bool eq = key[r][u] == T[r];
-      const uint32_t bal = __ballot_sync(kFullMaskScore, eq);
-      if (key[r][u] > T[r] || (eq && __popc(bal & below) < eq_left)) taken |= 1u << u;
-      eq_left -= __popc(bal);
+      for (int u = 0; u < U; ++u) {
+        if (key[r][u] == 0u) continue;
+        const double L = (double)key_value(key[r][u]);
+        if (L > hi)
+          taken |= 1u << u;
+        else if (L >= lo)
+          band |= 1u << u;
+      }
+      const int need = keep - (int)__reduce_add_sync(kFullMaskScore, (unsigned)__popc(taken));
+      const int nband = (int)__reduce_add_sync(kFullMaskScore, (unsigned)__popc(band));
+      if (nband == need) {
+        taken |= band;
+      } else {
+        // the band's fp64 logits, one block at a time: lanes form the D
+        // rounded products, then every lane adds them in channel order
+        by_index = false;
+        double* sv = reinterpret_cast<double*>(shf4) + warp * NK;
+        int* sj = reinterpret_cast<int*>(reinterpret_cast<double*>(shf4) + kRegScoreWarps * NK) +
+                  warp * NK;
+        const double* qr = q64 + (bh * nblocks + row) * D;
+        int cnt = 0;
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+          uint32_t bb = __ballot_sync(kFullMaskScore, (band >> u) & 1u);
+          while (bb) {
+            const int j = (__ffs(bb) - 1) + 32 * u;
+            bb &= bb - 1;
+            const double* kr = k64 + (bh * nblocks + j) * D;
+            double pr[D / 32];
+#pragma unroll
+            for (int m = 0; m < D / 32; ++m) pr[m] = __dmul_rn(qr[lane + 32 * m], kr[lane + 32 * m]);
+            double L64 = 0.0;
+#pragma unroll
+            for (int c = 0; c < D; ++c)
+              L64 = __dadd_rn(L64, __shfl_sync(kFullMaskScore, pr[c >> 5], c & 31));
+            if (lane == 0) {
+              sv[cnt] = L64;
+              sj[cnt] = j;
+            }
+            ++cnt;
+          }
+        }
+        __syncwarp();
+        // `need` rounds of a warp-wide arg-max over the list: larger fp64
+        // logit, then the lower block index
+        for (int it = 0; it < need; ++it) {
+          double best = 0.0;
+          int bj = 0x7fffffff, be = -1;
+          for (int x = lane; x < cnt; x += 32) {
+            const int j = sj[x];
+            if (j < 0) continue;
+            const double v = sv[x];
+            if (be < 0 || v > best || (v == best && j < bj)) {
+              best = v;
+              bj = j;
+              be = x;
+            }
+          }
+#pragma unroll
+          for (int o = 16; o > 0; o >>= 1) {
+            const double ov = __shfl_xor_sync(kFullMaskScore, best, o);
+            const int oj = __shfl_xor_sync(kFullMaskScore, bj, o);
+            const int oe = __shfl_xor_sync(kFullMaskScore, be, o);
+            if (oe >= 0 && (be < 0 || ov > best || (ov == best && oj < bj))) {
+              best = ov;
+              bj = oj;
+              be = oe;
+            }
+          }
+          if (be >= 0) {
+            if (lane == (bj & 31)) taken |= 1u << (bj >> 5);
+            if (lane == 0) sj[be] = -1;
+          }
+          __syncwarp();
+        }
+      }
+    }
+    if (by_index) {
+      uint32_t tie = 0u;
+      unsigned c_gt = 0;
+      if constexpr (!CERT) {
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+          if (key[r][u] > Tk[r]) {
+            taken |= 1u << u;
+            ++c_gt;
+          } else if (key[r][u] == Tk[r]) {
+            tie |= 1u << u;
+          }
+        }
+        int eq_left = keep - (int)__reduce_add_sync(kFullMaskScore, c_gt);
+#pragma unroll
+        for (int u = 0; u < U; ++u) {  // block order: u, then lane
+          const bool eq = (tie >> u) & 1u;
+          const uint32_t bal = __ballot_sync(kFullMaskScore, eq);
+          if (eq && __popc(bal & below) < eq_left) taken |= 1u << u;
+          eq_left -= __popc(bal);
+        }
+      }
     }
     // ascending output: j = 32u + lane grows with (u, lane)
     const int64_t grow = bh * nblocks + row;
@@ -584,9 +725,21 @@ __global__ void __launch_bounds__(32 * kRegScoreWarps, U <= 12 ? 4 : 3)
       if (grow == (int64_t)gridDim.z * Hh * nblocks - 1) row_ptr[grow + 1] = (int32_t)((grow + 1) * keep);
     }
     if (draft_map) {
-      double lv[U];  // the logits back from their keys (the map is exact to them)
+      double lv[U];
 #pragma unroll
-      for (int u = 0; u < U; ++u) lv[u] = (double)key_value(key[r][u]);
+      for (int u = 0; u < U; ++u) {
+        if (!(lane + 32 * u < nblocks)) {
+          lv[u] = 0.0;
+        } else if constexpr (CERT) {  // the map of the fp64 logits
+          const double* qr = q64 + (bh * nblocks + row) * D;
+          const double* kr = k64 + (bh * nblocks + lane + 32 * u) * D;
+          double a = 0.0;
+          for (int c = 0; c < D; ++c) a = __dadd_rn(a, __dmul_rn(qr[c], kr[c]));
+          lv[u] = a;
+        } else {  // fp32 logits come back from their keys (exactly)
+          lv[u] = (double)key_value(key[r][u]);
+        }
+      }
       double mx = -DBL_MAX;
 #pragma unroll
       for (int u = 0; u < U; ++u)
@@ -608,38 +761,70 @@ __global__ void __launch_bounds__(32 * kRegScoreWarps, U <= 12 ? 4 : 3)
   }
 }
 
+// The pooled values in the workspace.  FP32: [fp32 Q | fp32 K].  FP64:
+// [fp64 Q | fp64 K][fp32 Q | fp32 K][norms of Q | norms of K].
+struct DraftWs {
+  const double *q64 = nullptr, *k64 = nullptr;
+  const float *q32, *k32, *qn = nullptr, *kn = nullptr;
+  DraftWs(const Geometry& g, const void* ws, bool f64) {
+    const int64_t n = (int64_t)g.B * g.Hh * g.nblocks;  // units per tensor
+    const float* w32 = static_cast<const float*>(ws);
+    if (f64) {
+      q64 = static_cast<const double*>(ws);
+      k64 = q64 + n * g.D;
+      w32 = reinterpret_cast<const float*>(q64 + 2 * n * g.D);
+      qn = w32 + 2 * n * g.D;
+      kn = qn + n;
+    }
+    q32 = w32;
+    k32 = w32 + n * g.D;
+  }
+};
+
 template <int D, int U>
-cudaError_t launch_score_reg(const Geometry& g, const float* ws, int keep, int32_t* row_ptr,
+cudaError_t launch_score_reg(const Geometry& g, const DraftWs& w, int keep, int32_t* row_ptr,
                              int32_t* kv_idx, float* draft_map, cudaStream_t st) {
   using Cfg = RegScoreCfg<U>;
-  auto kern = draft_score_reg_kernel<D, U>;
+  const bool cert = w.q64 != nullptr;
+  auto kern = cert ? draft_score_reg_kernel<D, U, true> : draft_score_reg_kernel<D, U, false>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)Cfg::kSmem);
   if (e != cudaSuccess) return e;
-  const int64_t groups = (int64_t)g.B * g.Hh * g.nblocks;
   const dim3 grid((unsigned)((g.nblocks + Cfg::kRows - 1) / Cfg::kRows), (unsigned)g.Hh,
                   (unsigned)g.B);
-  kern<<<grid, 32 * kRegScoreWarps, Cfg::kSmem, st>>>(ws, ws + groups * D, g.Hh, (int)g.nblocks,
-                                                       keep, row_ptr, kv_idx, draft_map);
+  kern<<<grid, 32 * kRegScoreWarps, Cfg::kSmem, st>>>(w.q32, w.k32, g.Hh, (int)g.nblocks, keep,
+                                                       row_ptr, kv_idx, draft_map, w.q64, w.k64,
+                                                       w.qn, w.kn);
+  return cudaGetLastError();
+}
+
+template <int D, typename T>
+cudaError_t launch_score_rows(const Geometry& g, const T* qb, const T* kb, int keep,
+                              int32_t* row_ptr, int32_t* kv_idx, float* draft_map,
+                              cudaStream_t st) {
+  const int R = draft_rows_per_cta(g.nblocks, sizeof(T) == 8 ? BSA_DRAFT_FP64 : BSA_DRAFT_FP32);
+  const size_t smem = (size_t)(2 * (kScoreThreads / 32) * D + kKeyChunk * (D + 2) +
+                               (int64_t)R * g.nblocks) * sizeof(T) +
+                      (size_t)R * g.nblocks;
+  auto kern = draft_score_topk_kernel<D, T>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  const dim3 grid((unsigned)((g.nblocks + R - 1) / R), (unsigned)g.Hh, (unsigned)g.B);
+  kern<<<grid, kScoreThreads, smem, st>>>(qb, kb, g.Hh, (int)g.nblocks, R, keep, row_ptr, kv_idx,
+                                          draft_map);
   return cudaGetLastError();
 }
 
 template <int D>
-cudaError_t launch_t(const Geometry& g, const uint32_t* tile_valid, const void* q, const void* k,
-                     int keep, int pooling, bool natural, int32_t* row_ptr, int32_t* kv_idx,
-                     float* draft_map, float* ws, unsigned int* status, uint64_t wait_limit_ns,
-                     cudaStream_t st, uint32_t* amax, bool* amax_recorded) {
-  const int use_max = pooling == BSA_POOL_MAX ? 1 : 0;
-  cudaError_t e = launch_pool<D>(g, tile_valid, q, k, use_max, natural, ws, amax, st);
-  if (e != cudaSuccess) return e;
-  if (amax_recorded) *amax_recorded = amax != nullptr;
+cudaError_t launch_score(const Geometry& g, const DraftWs& w, int keep, int32_t* row_ptr,
+                         int32_t* kv_idx, float* draft_map, cudaStream_t st) {
   // rows of up to 512 key blocks: logits in registers
   // (one kernel per 32-block width U: no padded keys beyond the next 32)
   if (g.nblocks <= 512) {
     switch ((g.nblocks + 31) / 32) {
 #define BSA_SCORE_U(u) \
   case u:              \
-    return launch_score_reg<D, u>(g, ws, keep, row_ptr, kv_idx, draft_map, st);
+    return launch_score_reg<D, u>(g, w, keep, row_ptr, kv_idx, draft_map, st);
       BSA_SCORE_U(1) BSA_SCORE_U(2) BSA_SCORE_U(3) BSA_SCORE_U(4) BSA_SCORE_U(5) BSA_SCORE_U(6)
       BSA_SCORE_U(7) BSA_SCORE_U(8) BSA_SCORE_U(9) BSA_SCORE_U(10) BSA_SCORE_U(11)
       BSA_SCORE_U(12) BSA_SCORE_U(13) BSA_SCORE_U(14) BSA_SCORE_U(15) BSA_SCORE_U(16)
@@ -648,45 +833,52 @@ cudaError_t launch_t(const Geometry& g, const uint32_t* tile_valid, const void* 
         break;
     }
   }
-  const int R = draft_rows_per_cta(g.nblocks);
-  const size_t smem = (size_t)(2 * (kScoreThreads / 32) * D + kKeyChunk * (D + 2) +
-                               (int64_t)R * g.nblocks) * sizeof(float) +
-                      (size_t)R * g.nblocks;
-  auto kern = draft_score_topk_kernel<D>;
-  e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  // longer rows: logits in shared memory, in the plan's precision
+  if (w.q64)
+    return launch_score_rows<D, double>(g, w.q64, w.k64, keep, row_ptr, kv_idx, draft_map, st);
+  return launch_score_rows<D, float>(g, w.q32, w.k32, keep, row_ptr, kv_idx, draft_map, st);
+}
+
+template <int D>
+cudaError_t launch_t(const Geometry& g, const uint32_t* tile_valid, const void* q, const void* k,
+                     int keep, int pooling, int precision, bool natural, int32_t* row_ptr,
+                     int32_t* kv_idx, float* draft_map, void* ws, cudaStream_t st, uint32_t* amax,
+                     bool* amax_recorded) {
+  const int use_max = pooling == BSA_POOL_MAX ? 1 : 0;
+  const bool f64 = precision == BSA_DRAFT_FP64;
+  cudaError_t e = launch_pool<D>(g, tile_valid, q, k, use_max, natural, f64, ws, amax, st);
   if (e != cudaSuccess) return e;
-  const dim3 grid((unsigned)((g.nblocks + R - 1) / R), (unsigned)g.Hh, (unsigned)g.B);
-  const int64_t groups = (int64_t)g.B * g.Hh * g.nblocks;
-  kern<<<grid, kScoreThreads, smem, st>>>(ws, ws + groups * D, g.Hh, (int)g.nblocks, R, keep,
-                                          row_ptr, kv_idx, draft_map);
-  return cudaGetLastError();
+  if (amax_recorded) *amax_recorded = amax != nullptr;
+  return launch_score<D>(g, DraftWs(g, ws, f64), keep, row_ptr, kv_idx, draft_map, st);
 }
 
 }  // namespace
 
-int draft_rows_per_cta(int64_t nblocks) {
+int draft_rows_per_cta(int64_t nblocks, int precision) {
   // logits + selection flags of R rows within ~150 KB of shared memory; at
   // most two rows per warp of the scoring kernel
   static_assert(2 * (kScoreThreads / 32) >= 16, "two rows per warp");
+  const int64_t per = precision == BSA_DRAFT_FP64 ? 9 : 5;
   int64_t R = 16;
-  while (R > 1 && R * nblocks * 5 > 150 * 1024) R >>= 1;
+  while (R > 1 && R * nblocks * per > 150 * 1024) R >>= 1;
   return (int)R;
 }
 
-size_t draft_workspace_bytes(const Geometry& g) {
-  return (size_t)2 * g.B * g.Hh * g.nblocks * g.D * sizeof(float);
+size_t draft_workspace_bytes(const Geometry& g, int precision) {
+  const size_t n = (size_t)g.B * g.Hh * g.nblocks;  // units per tensor
+  if (precision == BSA_DRAFT_FP64) return 2 * n * g.D * (sizeof(double) + sizeof(float)) + 2 * n * sizeof(float);
+  return 2 * n * g.D * sizeof(float);
 }
 
 cudaError_t launch_draft_mask(const Geometry& g, const uint32_t* tile_valid, const void* q,
-                              const void* k, int keep, int pooling, int32_t* row_ptr,
-                              int32_t* kv_idx, float* draft_map, float* ws, unsigned int* status,
-                              uint64_t wait_limit_ns, cudaStream_t st, bool natural,
-                              uint32_t* amax, bool* amax_recorded) {
+                              const void* k, int keep, int pooling, int precision,
+                              int32_t* row_ptr, int32_t* kv_idx, float* draft_map, void* ws,
+                              cudaStream_t st, bool natural, uint32_t* amax, bool* amax_recorded) {
   if (g.D == 128)
-    return launch_t<128>(g, tile_valid, q, k, keep, pooling, natural, row_ptr, kv_idx, draft_map,
-                         ws, status, wait_limit_ns, st, amax, amax_recorded);
-  return launch_t<64>(g, tile_valid, q, k, keep, pooling, natural, row_ptr, kv_idx, draft_map, ws,
-                      status, wait_limit_ns, st, amax, amax_recorded);
+    return launch_t<128>(g, tile_valid, q, k, keep, pooling, precision, natural, row_ptr, kv_idx,
+                         draft_map, ws, st, amax, amax_recorded);
+  return launch_t<64>(g, tile_valid, q, k, keep, pooling, precision, natural, row_ptr, kv_idx,
+                      draft_map, ws, st, amax, amax_recorded);
 }
 
 }  // namespace bsa
@@ -703,9 +895,9 @@ cudaError_t launch_draft_mask(const Geometry& g, const uint32_t* tile_valid, con
 // and K) taken from the file-scope device array below instead of a caller
 // workspace.
 //
-// The array is kNoAllocScratchBytes (32 MiB) on every GPU that loads this
+// The array is kNoAllocScratchBytes (48 MiB) on every GPU that loads this
 // library, held until the process exits; problems whose scratch would exceed
-// it (2*B*Hh*Nb*D*8 bytes) are rejected.  Every call on a device shares the
+// it (bsa_draft_workspace_bytes) are rejected.  Every call on a device shares the
 // one array, so calls whose kernels overlap on the GPU (on different streams,
 // or from different host threads) race on it; calls in order on one stream
 // are safe.  The array keeps the last call's contents: nothing needs clearing,
@@ -716,19 +908,19 @@ cudaError_t launch_draft_mask(const Geometry& g, const uint32_t* tile_valid, con
 namespace bsa {
 namespace {
 
-constexpr size_t kNoAllocScratchBytes = 32u << 20;
+constexpr size_t kNoAllocScratchBytes = 48u << 20;
 constexpr int kMaxDevices = 64;
 
-static __device__ __align__(256) float g_noalloc_scratch[kNoAllocScratchBytes / sizeof(float)];
+static __device__ __align__(256) double g_noalloc_scratch[kNoAllocScratchBytes / sizeof(double)];
 
 // Device address of g_noalloc_scratch on the current device.  Looked up once
 // per device, on the first call made with that device current, and cached
 // for the life of the process: after cudaDeviceReset the cached address no
 // longer names live memory, so the entry point must not be called again in
 // that process.
-cudaError_t noalloc_scratch_address(float** out) {
+cudaError_t noalloc_scratch_address(void** out) {
   static std::mutex mu;
-  static float* addr[kMaxDevices] = {};
+  static void* addr[kMaxDevices] = {};
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
@@ -738,7 +930,7 @@ cudaError_t noalloc_scratch_address(float** out) {
     void* p = nullptr;
     e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
     if (e != cudaSuccess) return e;
-    addr[dev] = reinterpret_cast<float*>(p);
+    addr[dev] = p;
   }
   *out = addr[dev];
   return cudaSuccess;
@@ -763,11 +955,11 @@ extern "C" bsa_status bsa_draft_mask_noalloc(bsa_plan_t plan, const void* q_slot
     return set_error(BSA_ERR_INVALID_ARG, "q_slots / k_slots / kv_idx is NULL");
   if (!aligned16(q_slots) || !aligned16(k_slots))
     return set_error(BSA_ERR_ALIGNMENT, "q_slots / k_slots not 16-byte aligned");
-  const size_t need = draft_workspace_bytes(g);
+  const size_t need = draft_workspace_bytes(g, plan->draft_precision);
   if (need > kNoAllocScratchBytes)
     return set_error(BSA_ERR_UNSUPPORTED,
                      "draft scratch of " + std::to_string(need) +
-                         " bytes exceeds the 32 MiB static scratch of bsa_draft_mask_noalloc; "
+                         " bytes exceeds the 48 MiB static scratch of bsa_draft_mask_noalloc; "
                          "use bsa_draft_mask with a caller workspace");
   if (g.nblocks > 18000) return set_error(BSA_ERR_UNSUPPORTED, "draft mask supports up to 18000 blocks");
   if ((int64_t)g.B * g.Hh * g.Npad >= (1ll << 31))
@@ -782,11 +974,11 @@ extern "C" bsa_status bsa_draft_mask_noalloc(bsa_plan_t plan, const void* q_slot
     return set_error(BSA_ERR_INVALID_ARG,
                      "the current device is not the plan's: the static scratch of one device "
                      "cannot serve a plan of another");
-  float* scratch = nullptr;
+  void* scratch = nullptr;
   e = noalloc_scratch_address(&scratch);
   if (e != cudaSuccess) return cuda_error(e, "cudaGetSymbolAddress(scratch)");
-  e = launch_draft_mask(g, plan->d_tile_valid, q_slots, k_slots, keep, plan->draft_pooling, row_ptr,
-                        kv_idx, draft_map, scratch, plan->d_status, plan->wait_limit_ns,
+  e = launch_draft_mask(g, plan->d_tile_valid, q_slots, k_slots, keep, plan->draft_pooling,
+                        plan->draft_precision, row_ptr, kv_idx, draft_map, scratch,
                         reinterpret_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? BSA_OK : cuda_error(e, "draft_mask_noalloc launch");
 }

@@ -15,12 +15,14 @@ import math
 
 import torch
 
-from . import (ANCHORS_ROTATING, LAYOUT_FRAME, LAYOUT_TILE, POOL_MEAN, WINDOW_ALTERNATE, Plan,
+from . import (ANCHORS_ROTATING, DRAFT_FP64, LAYOUT_FRAME, LAYOUT_TILE, POOL_MEAN,
+               WINDOW_ALTERNATE, Plan,
                bsa_attn_fwd, bsa_attn_fwd_natural, bsa_attn_fwd_natural_e4m3,
                bsa_draft_keep_count, bsa_draft_mask, bsa_draft_mask_natural,
                bsa_draft_mask_natural_e4m3,
                bsa_draft_workspace_bytes, bsa_quantize_e4m3,
                bsa_lvsa_attn_fwd, bsa_lvsa_mask, bsa_lvsa_nnz, bsa_plan_set_draft_pooling,
+               bsa_plan_set_draft_precision,
                bsa_plan_set_lvsa_variant, bsa_reorder_fwd, bsa_reorder_inv)
 
 
@@ -80,12 +82,14 @@ class LvsaAttention(_Base):
 
 class DraftAttention(_Base):
     """Draft-mask block-sparse attention on the tile layout.  `pooling`:
-    POOL_MEAN (the article's average) or POOL_MAX."""
+    POOL_MEAN (the article's average) or POOL_MAX; `precision`: DRAFT_FP64
+    or DRAFT_FP32 draft logits."""
 
     def __init__(self, B, Hh, D, T, H, W, pool_h, pool_w, sparsity_pct, device="cuda",
-                 scale=None, want_map=False, pooling=POOL_MEAN):
+                 scale=None, want_map=False, pooling=POOL_MEAN, precision=DRAFT_FP64):
         self.plan = Plan(B, Hh, D, T, H, W, LAYOUT_TILE, pool_h, pool_w, pool_h * pool_w)
         bsa_plan_set_draft_pooling(self.plan, pooling)
+        bsa_plan_set_draft_precision(self.plan, precision)
         self.sparsity = sparsity_pct
         self.scale = scale if scale is not None else 1.0 / math.sqrt(D)
         self.keep = bsa_draft_keep_count(self.plan, sparsity_pct)
@@ -95,7 +99,7 @@ class DraftAttention(_Base):
         self.draft_map = (torch.empty(rows * self.plan.nblocks, dtype=torch.float32,
                                       device=device) if want_map else None)
         nbytes = bsa_draft_workspace_bytes(self.plan)
-        self.workspace = torch.empty((nbytes + 3) // 4, dtype=torch.float32, device=device)
+        self.workspace = torch.empty((nbytes + 7) // 8, dtype=torch.float64, device=device)
         self._alloc_slots(device)
 
     def mask(self):

@@ -85,6 +85,9 @@ typedef enum {
 /* Draft pooling (bsa_plan_set_draft_pooling). */
 typedef enum { BSA_POOL_MEAN = 0, BSA_POOL_MAX = 1 } bsa_pooling;
 
+/* Precision of the draft logits (bsa_plan_set_draft_precision). */
+typedef enum { BSA_DRAFT_FP64 = 0, BSA_DRAFT_FP32 = 1 } bsa_draft_precision;
+
 typedef struct bsa_plan_s* bsa_plan_t;
 
 /* Create a plan for batch B, Hh heads, head dim D, latent grid T x H x W.
@@ -119,6 +122,18 @@ bsa_status bsa_plan_set_lvsa_variant(bsa_plan_t plan, int anchors, int window_or
  * pooling first and preferring the average at high sparsity. */
 bsa_status bsa_plan_set_draft_pooling(bsa_plan_t plan, int pooling);
 
+/* Choose the precision of the draft logits of bsa_draft_mask,
+ * bsa_draft_mask_noalloc and bsa_draft_mask_natural(_e4m3) with this plan
+ * (default FP64).  The Draft Attention article fixes none.  FP64: the pooled
+ * values and the logits in fp64.  FP32: the pooled values (still summed in
+ * fp64) rounded once to fp32 and the logits' products and sums rounded to
+ * fp32, about twice as fast to score; the block lists can differ from FP64
+ * where two logits agree to fp32 precision.  Either way the evaluation order
+ * is fixed (below), so the lists are reproducible bit for bit.  The
+ * workspace size (bsa_draft_workspace_bytes) follows the precision.  Takes
+ * effect for calls issued after it; BSA_ERR_INVALID_ARG for unknown values. */
+bsa_status bsa_plan_set_draft_precision(bsa_plan_t plan, int precision);
+
 /* Geometry queries (return -1 for a NULL plan). */
 int64_t bsa_padded_tokens(bsa_plan_t plan);   /* Npad                          */
 int64_t bsa_num_blocks(bsa_plan_t plan);      /* blocks per (b, head): Nb      */
@@ -148,7 +163,8 @@ int64_t bsa_lvsa_nnz(bsa_plan_t plan, int C);
  * k = ceil(Nb*(100 - sparsity_pct)/100), i.e. never sparser than asked. */
 int bsa_draft_keep_count(bsa_plan_t plan, int sparsity_pct);
 
-/* Scratch bytes bsa_draft_mask needs (the pooled Q and K in fp32). */
+/* Scratch bytes bsa_draft_mask needs (the pooled Q and K in the plan's
+ * draft precision: 2*B*Hh*Nb*D*8 bytes for FP64, *4 for FP32). */
 size_t bsa_draft_workspace_bytes(bsa_plan_t plan);
 
 /* Draft mask (Draft Attention article: average pooling of Q and K over each
@@ -157,11 +173,12 @@ size_t bsa_draft_workspace_bytes(bsa_plan_t plan);
  * Requires a TILE plan.  q_slots, k_slots: slot layout (output of
  * bsa_reorder_fwd).  For every (b, head, query block i):
  *   qbar_i, kbar_j = mean over the tile's tokens inside the grid (fp64
- *     sequential sum in row-major tile order, one IEEE division, rounded
- *     once to fp32), or their maximum with
+ *     sequential sum in row-major tile order, one IEEE division; rounded
+ *     once to fp32 in FP32 precision), or their maximum with
  *     bsa_plan_set_draft_pooling(BSA_POOL_MAX);
  *   L[i][j] = sum_c qbar_i[c]*kbar_j[c], sequential over c, each product and
- *     sum rounded to fp32 (no fused multiply-add);
+ *     sum rounded to the plan's draft precision (fp64 by default; no fused
+ *     multiply-add);
  *   keep the k = bsa_draft_keep_count() blocks j with the largest L[i][j],
  *     ties to the lower j, written ascending.
  * Outputs (device): kv_idx int32[B*Hh*Nb*k]; row_ptr int32[B*Hh*Nb+1] (may be
@@ -180,10 +197,10 @@ bsa_status bsa_draft_mask(bsa_plan_t plan, const void* q_slots, const void* k_sl
  * only input and output buffers, or a caller held to a fixed memory budget
  * where an extra allocation could fail or stall the device mid-step.
  * Same arguments, outputs and results as bsa_draft_mask, minus the workspace:
- * the fp32 scratch lives in a 32 MiB array inside the library
+ * the scratch lives in a 48 MiB array inside the library
  * (bsa_draft_noalloc_max_scratch_bytes()), held by every GPU that loads the
  * library until the process exits.  Problems needing more scratch than that
- * (2*B*Hh*Nb*D*4 bytes) return BSA_ERR_UNSUPPORTED.  The first call made on a
+ * (bsa_draft_workspace_bytes) return BSA_ERR_UNSUPPORTED.  The first call made on a
  * device looks up that array's device address (one cudaGetSymbolAddress);
  * make that first call before any stream capture.  All calls on a device
  * share the array: calls whose kernels overlap on the GPU race on it, calls
@@ -196,7 +213,7 @@ bsa_status bsa_draft_mask_noalloc(bsa_plan_t plan, const void* q_slots, const vo
                                   int sparsity_pct, int32_t* row_ptr, int32_t* kv_idx,
                                   float* draft_map, void* stream);
 
-/* Scratch capacity of bsa_draft_mask_noalloc, in bytes (32 MiB). */
+/* Scratch capacity of bsa_draft_mask_noalloc, in bytes (48 MiB). */
 size_t bsa_draft_noalloc_max_scratch_bytes(void);
 
 /* Reorder (Draft Attention article, reorder paragraph): gather natural-layout

@@ -17,9 +17,10 @@ what the method computes, written from the pages:
   reorder makes the selected blocks contiguous; quantization is named as the
   next step.
 
-Floating point is fp64 (bf16 inputs convert to fp64 exactly), except where
-a float decides an integer in the kernel's precision: the draft logits that
-rank the key blocks are fp32, and the e4m3 scales and divisions are fp32.
+All floating point is fp64 (bf16 inputs convert to fp64 exactly), except
+where a float decides an integer in the kernel's precision: the e4m3 scales
+and divisions are fp32, and so are the draft logits of the library's
+optional fp32 draft precision (draft_logits(..., precision="fp32")).
 
 Readings of points the pages leave open:
 * window extension order: a right and a left pointer take turns, right
@@ -34,10 +35,10 @@ Readings of points the pages leave open:
   partially filled); sums run sequentially in row-major (a, then b) order and
   the mean is one IEEE division; max pooling takes the maximum over the same
   tokens;
-* draft logits are a sequential multiply-then-add chain over the channels
-  of the pooled values rounded to fp32, each operation rounded to fp32 (no
-  fused multiply-add): the pages fix no precision for the draft map, and
-  the top-k that the logits decide is taken in the kernel's precision;
+* draft logits are a sequential multiply-then-add chain over the channels,
+  each operation rounded to fp64 (no fused multiply-add); the optional fp32
+  precision rounds the pooled values once to fp32 and every operation to
+  fp32 (the pages fix no precision for the draft map);
 * top-k per query-block row keeps k = ceil(Nb*(100-p)/100) blocks ranked by
   (logit descending, block index ascending), returned in ascending order;
 * a query with no allowed valid key gets O = 0 and LSE = -inf; pad query
@@ -287,22 +288,26 @@ def draft_pool(x_nat: np.ndarray, T: int, H: int, W: int, ph: int, pw: int,
         np.transpose(pooled, (0, 4, 1, 2, 3, 5)).reshape(B, Hh, T * TH * TW, D))
 
 
-def draft_logits(qbar: np.ndarray, kbar: np.ndarray) -> np.ndarray:
-    """Low-resolution logits L[b,h,i,j] = <qbar_i, kbar_j>, in fp32.
+def draft_logits(qbar: np.ndarray, kbar: np.ndarray, precision: str = "fp64") -> np.ndarray:
+    """Low-resolution logits L[b,h,i,j] = <qbar_i, kbar_j>.
 
-    The pages fix no precision for the draft map; the top-k decision is taken
-    in the kernel's precision, fp32.  The pooled values are rounded once to
-    fp32 (nearest, ties to even); then, sequentially over channels
-    c = 0..D-1, acc = acc + qbar[i,c]*kbar[j,c] with the product and the sum
-    each rounded to fp32 (no fused multiply-add).  numpy's float32 multiply
-    and add are single IEEE operations.  Returns float32.
+    Sequential over channels c = 0..D-1: acc = acc + qbar[i,c]*kbar[j,c],
+    the product and the sum each rounded (no fused multiply-add), starting
+    from acc = 0.
+    precision "fp64" (default): everything in fp64.
+    precision "fp32": the pooled values are first rounded to fp32 (nearest,
+    ties to even), and every product and sum is rounded to fp32; numpy's
+    float32 multiply and add are single IEEE operations.  Returns float32.
     """
-    q32 = np.asarray(qbar, dtype=np.float32)
-    k32 = np.asarray(kbar, dtype=np.float32)
-    B, Hh, Nb, D = q32.shape
-    acc = np.zeros((B, Hh, Nb, k32.shape[2]), dtype=np.float32)
+    if precision not in ("fp64", "fp32"):
+        raise ValueError(f"unknown precision {precision!r}")
+    dt = np.float64 if precision == "fp64" else np.float32
+    qv = np.asarray(qbar, dtype=dt)
+    kv = np.asarray(kbar, dtype=dt)
+    B, Hh, Nb, D = qv.shape
+    acc = np.zeros((B, Hh, Nb, kv.shape[2]), dtype=dt)
     for c in range(D):
-        prod = q32[:, :, :, c][..., :, None] * k32[:, :, :, c][..., None, :]
+        prod = qv[:, :, :, c][..., :, None] * kv[:, :, :, c][..., None, :]
         acc = acc + prod
     return acc
 
@@ -332,11 +337,12 @@ def draft_topk(logits: np.ndarray, k: int) -> np.ndarray:
     return out.reshape(*lead, Nq, k)
 
 
-def draft_blocks(q_nat, k_nat, T, H, W, ph, pw, sparsity_pct, mode: str = "mean"):
+def draft_blocks(q_nat, k_nat, T, H, W, ph, pw, sparsity_pct, mode: str = "mean",
+                 precision: str = "fp64"):
     """Full draft-mask pipeline: pool -> logits -> top-k.  int32 [B,Hh,Nb,k]."""
     qbar = draft_pool(q_nat, T, H, W, ph, pw, mode)
     kbar = draft_pool(k_nat, T, H, W, ph, pw, mode)
-    L = draft_logits(qbar, kbar)
+    L = draft_logits(qbar, kbar, precision)
     return draft_topk(L, draft_keep_count(L.shape[-1], sparsity_pct))
 
 

@@ -46,29 +46,39 @@ CASES = [
 
 @pytest.mark.parametrize("over", CASES)
 @pytest.mark.parametrize("pooling", [bsa.POOL_MEAN, bsa.POOL_MAX])
-def test_draft_mask_natural_bit_exact(over, pooling):
+@pytest.mark.parametrize("precision", [bsa.DRAFT_FP64, bsa.DRAFT_FP32])
+def test_draft_mask_natural_bit_exact(over, pooling, precision):
     over = dict(over)
     w = small_workload(CONFIGS[over.pop("cid")], **over)
     ph, pw, sp = w.draft_ph, w.draft_pw, w.draft_sparsity
     q, k, _ = make_qkv(w, device="cuda")
     plan = bsa.Plan(w.B, w.Hh, w.D, w.T, w.H, w.W, bsa.LAYOUT_TILE, ph, pw, ph * pw)
     bsa.bsa_plan_set_draft_pooling(plan, pooling)
+    bsa.bsa_plan_set_draft_precision(plan, precision)
     keep = bsa.bsa_draft_keep_count(plan, sp)
     nb = plan.nblocks
     rows = w.B * w.Hh * nb
     rp = torch.empty(rows + 1, dtype=torch.int32, device="cuda")
     kv = torch.empty(rows * keep, dtype=torch.int32, device="cuda")
-    ws = torch.full(((bsa.bsa_draft_workspace_bytes(plan) + 3) // 4,), float("nan"),
-                    dtype=torch.float32, device="cuda")
+    dt, npdt = ((torch.float64, np.float64) if precision == bsa.DRAFT_FP64
+                else (torch.float32, np.float32))
+    nbytes = bsa.bsa_draft_workspace_bytes(plan)
+    # fp32: the pooled values; fp64: the pooled values, their fp32 copies
+    # and one norm per pooled vector
+    assert nbytes == (2 * rows * w.D * 4 if precision == bsa.DRAFT_FP32
+                      else 2 * rows * w.D * 12 + 2 * rows * 4)
+    ws = torch.full((nbytes // np.dtype(npdt).itemsize,), float("nan"), dtype=dt, device="cuda")
     bsa.bsa_draft_mask_natural(plan, q, k, sp, rp, kv, None, ws)
     bsa.bsa_poll_status(plan)
     mode = "max" if pooling == bsa.POOL_MAX else "mean"
     qbar = oracle.draft_pool(to_np64(q), w.T, w.H, w.W, ph, pw, mode)
     kbar = oracle.draft_pool(to_np64(k), w.T, w.H, w.W, ph, pw, mode)
     got = ws.cpu().numpy()[:2 * rows * w.D].reshape(2, w.B, w.Hh, nb, w.D)
-    np.testing.assert_array_equal(got[0], qbar.astype(np.float32))   # fp64 sum, one rounding
-    np.testing.assert_array_equal(got[1], kbar.astype(np.float32))
-    ref = oracle.draft_topk(oracle.draft_logits(qbar, kbar), oracle.draft_keep_count(nb, sp))
+    # the fp64 sum and division, rounded once to fp32 in FP32 precision
+    np.testing.assert_array_equal(got[0], qbar.astype(npdt))
+    np.testing.assert_array_equal(got[1], kbar.astype(npdt))
+    prec = "fp64" if precision == bsa.DRAFT_FP64 else "fp32"
+    ref = oracle.draft_topk(oracle.draft_logits(qbar, kbar, prec), oracle.draft_keep_count(nb, sp))
     np.testing.assert_array_equal(kv.cpu().numpy().reshape(w.B, w.Hh, nb, keep), ref)
 
 

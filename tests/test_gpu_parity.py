@@ -166,12 +166,16 @@ DRAFT_CASES = [
 
 
 @pytest.mark.parametrize("over", DRAFT_CASES)
-def test_draft_mask_bit_exact(over):
+@pytest.mark.parametrize("precision", [bsa.DRAFT_FP64, bsa.DRAFT_FP32])
+def test_draft_mask_bit_exact(over, precision):
     over = dict(over)
     w = small_workload(CONFIGS[over.pop("cid")], **over)
     ph, pw, sp = w.draft_ph, w.draft_pw, w.draft_sparsity
     q, k, _ = make_qkv(w)
     plan = bsa.Plan(w.B, w.Hh, w.D, w.T, w.H, w.W, bsa.LAYOUT_TILE, ph, pw, ph * pw)
+    bsa.bsa_plan_set_draft_precision(plan, precision)
+    npdt = np.float64 if precision == bsa.DRAFT_FP64 else np.float32
+    prec = "fp64" if precision == bsa.DRAFT_FP64 else "fp32"
     perm, Np = oracle.tile_layout_perm(w.T, w.H, w.W, ph, pw)
     qs, ks = _slots_gpu(q, perm, plan.Npad), _slots_gpu(k, perm, plan.Npad)
     keep = bsa.bsa_draft_keep_count(plan, sp)
@@ -181,8 +185,8 @@ def test_draft_mask_bit_exact(over):
     kv = torch.empty(rows * keep, dtype=torch.int32, device="cuda")
     want_map = w.Hh * nb * nb <= 4_000_000
     dm = torch.empty(rows * nb, dtype=torch.float32, device="cuda") if want_map else None
-    ws = torch.full(((bsa.bsa_draft_workspace_bytes(plan) + 3) // 4,), float("nan"),
-                    dtype=torch.float32, device="cuda")
+    ws = torch.full((bsa.bsa_draft_workspace_bytes(plan) // np.dtype(npdt).itemsize,),
+                    float("nan"), dtype=torch.from_numpy(np.zeros(1, npdt)).dtype, device="cuda")
     bsa.bsa_draft_mask(plan, qs, ks, sp, rp, kv, dm, ws)
     bsa.bsa_poll_status(plan)
 
@@ -190,10 +194,9 @@ def test_draft_mask_bit_exact(over):
     qbar = oracle.draft_pool(qn, w.T, w.H, w.W, ph, pw)
     kbar = oracle.draft_pool(kn, w.T, w.H, w.W, ph, pw)
     got_pool = ws.cpu().numpy()[:2 * rows * w.D].reshape(2, w.B, w.Hh, nb, w.D)
-    # bit-exact: the fp64 sum and division, rounded once to fp32
-    np.testing.assert_array_equal(got_pool[0], qbar.astype(np.float32))
-    np.testing.assert_array_equal(got_pool[1], kbar.astype(np.float32))
-    L = oracle.draft_logits(qbar, kbar)
+    np.testing.assert_array_equal(got_pool[0], qbar.astype(npdt))   # bit-exact
+    np.testing.assert_array_equal(got_pool[1], kbar.astype(npdt))
+    L = oracle.draft_logits(qbar, kbar, prec)
     ref = oracle.draft_topk(L, oracle.draft_keep_count(nb, sp))
     np.testing.assert_array_equal(kv.cpu().numpy().reshape(w.B, w.Hh, nb, keep), ref)
     np.testing.assert_array_equal(rp.cpu().numpy(), np.arange(rows + 1) * keep)
@@ -204,6 +207,76 @@ def test_draft_mask_bit_exact(over):
     if keep < nb:
         srt = -np.sort(-L, axis=-1)
         assert np.isfinite(srt[..., keep - 1] - srt[..., keep]).all()
+
+
+def test_draft_mask_logits_equal_in_fp32_but_not_in_fp64():
+    # Eight 2 x 2 tiles in one row of a 2 x 16 grid, one head, D = 64.  Every
+    # query tile pools to q = (1, 2^-20, 0, ...); key tile j to (a_j, d_j, 0,
+    # ...), so L[i][j] = a_j + 2^-20 d_j exactly in fp64:
+    #   L = 0.5, 2, 1, 3, 1 + 2^-39, 1 + 2^-40, 4, 0.125.
+    # Keeping 5 of 8 takes blocks 1, 3, 6 and two of the three logits that
+    # round to 1.0 in fp32.  fp64 ranks them by value (blocks 4, 5); fp32
+    # sees a tie and takes the lower indices (blocks 2, 4).
+    T, H, W, D, ph, pw = 1, 2, 16, 64, 2, 2
+    a = [0.5, 2.0, 1.0, 3.0, 1.0, 1.0, 4.0, 0.125]
+    d = [0.0, 0.0, 0.0, 0.0, 2.0 ** -19, 2.0 ** -20, 0.0, 0.0]
+    q = torch.zeros((1, T * H * W, 1, D), dtype=torch.bfloat16)
+    k = torch.zeros_like(q)
+    for y in range(H):
+        for x in range(W):
+            n, j = y * W + x, x // pw
+            q[0, n, 0, 0], q[0, n, 0, 1] = 1.0, 2.0 ** -20
+            k[0, n, 0, 0], k[0, n, 0, 1] = a[j], d[j]
+    qn, kn = to_np64(q), to_np64(k)
+    qbar = oracle.draft_pool(qn, T, H, W, ph, pw)
+    kbar = oracle.draft_pool(kn, T, H, W, ph, pw)
+    L64 = oracle.draft_logits(qbar, kbar)
+    assert L64[0, 0, 0, 5] == 1.0 + 2.0 ** -40 and L64[0, 0, 0, 4] == 1.0 + 2.0 ** -39
+    want = {bsa.DRAFT_FP64: [1, 3, 4, 5, 6], bsa.DRAFT_FP32: [1, 2, 3, 4, 6]}
+    for precision, prec in ((bsa.DRAFT_FP64, "fp64"), (bsa.DRAFT_FP32, "fp32")):
+        ref = oracle.draft_topk(oracle.draft_logits(qbar, kbar, prec), 5)
+        assert (ref == np.array(want[precision])).all()
+        plan = bsa.Plan(1, 1, D, T, H, W, bsa.LAYOUT_TILE, ph, pw, ph * pw)
+        bsa.bsa_plan_set_draft_precision(plan, precision)
+        assert bsa.bsa_draft_keep_count(plan, 40) == 5
+        perm, Np = oracle.tile_layout_perm(T, H, W, ph, pw)
+        qs, ks = _slots_gpu(q, perm, plan.Npad), _slots_gpu(k, perm, plan.Npad)
+        rp = torch.empty(9, dtype=torch.int32, device="cuda")
+        kv = torch.empty(8 * 5, dtype=torch.int32, device="cuda")
+        ws = torch.empty(bsa.bsa_draft_workspace_bytes(plan), dtype=torch.uint8, device="cuda")
+        bsa.bsa_draft_mask(plan, qs, ks, 40, rp, kv, None, ws)
+        bsa.bsa_poll_status(plan)
+        got = kv.cpu().numpy().reshape(8, 5)
+        assert (got == np.array(want[precision])[None, :]).all(), (precision, got)
+
+
+@pytest.mark.parametrize("precision", [bsa.DRAFT_FP64, bsa.DRAFT_FP32])
+def test_draft_mask_all_logits_equal(precision):
+    # constant Q and K: every logit of a row is the same, so the kept blocks
+    # are the lowest indices (in fp64 every block of the row is within the
+    # fp32 error bound of the k-th and gets its fp64 logit)
+    T, H, W, D, ph, pw = 1, 4, 8, 64, 2, 2
+    q = torch.full((1, T * H * W, 1, D), 0.5, dtype=torch.bfloat16)
+    k = torch.full_like(q, -0.25)
+    plan = bsa.Plan(1, 1, D, T, H, W, bsa.LAYOUT_TILE, ph, pw, ph * pw)
+    bsa.bsa_plan_set_draft_precision(plan, precision)
+    keep = bsa.bsa_draft_keep_count(plan, 60)
+    nb = plan.nblocks
+    perm, Np = oracle.tile_layout_perm(T, H, W, ph, pw)
+    qs, ks = _slots_gpu(q, perm, plan.Npad), _slots_gpu(k, perm, plan.Npad)
+    rp = torch.empty(nb + 1, dtype=torch.int32, device="cuda")
+    kv = torch.empty(nb * keep, dtype=torch.int32, device="cuda")
+    dm = torch.empty(nb * nb, dtype=torch.float32, device="cuda")
+    ws = torch.empty(bsa.bsa_draft_workspace_bytes(plan), dtype=torch.uint8, device="cuda")
+    bsa.bsa_draft_mask(plan, qs, ks, 60, rp, kv, dm, ws)
+    bsa.bsa_poll_status(plan)
+    prec = "fp64" if precision == bsa.DRAFT_FP64 else "fp32"
+    qbar = oracle.draft_pool(to_np64(q), T, H, W, ph, pw)
+    kbar = oracle.draft_pool(to_np64(k), T, H, W, ph, pw)
+    ref = oracle.draft_topk(oracle.draft_logits(qbar, kbar, prec), keep)
+    assert (ref == np.arange(keep)).all()
+    np.testing.assert_array_equal(kv.cpu().numpy().reshape(1, 1, nb, keep), ref)
+    np.testing.assert_allclose(dm.cpu().numpy(), 1.0 / nb, rtol=1e-6)
 
 
 # ------------------------------------------------------------------ attention

@@ -219,12 +219,12 @@ def test_draft_max_pool_bit_exact(over, noalloc):
     if noalloc:
         bsa.bsa_draft_mask_noalloc(plan, qs, ks, sp, rp, kv, None)
     else:
-        ws = torch.full(((bsa.bsa_draft_workspace_bytes(plan) + 3) // 4,), float("nan"),
-                        dtype=torch.float32, device="cuda")
+        ws = torch.full(((bsa.bsa_draft_workspace_bytes(plan) + 7) // 8,), float("nan"),
+                        dtype=torch.float64, device="cuda")
         bsa.bsa_draft_mask(plan, qs, ks, sp, rp, kv, None, ws)
         got = ws.cpu().numpy()[:2 * rows * w.D].reshape(2, w.B, w.Hh, nb, w.D)
-        np.testing.assert_array_equal(got[0], qbar.astype(np.float32))
-        np.testing.assert_array_equal(got[1], kbar.astype(np.float32))
+        np.testing.assert_array_equal(got[0], qbar)
+        np.testing.assert_array_equal(got[1], kbar)
     bsa.bsa_poll_status(plan)
     ref = oracle.draft_topk(oracle.draft_logits(qbar, kbar), oracle.draft_keep_count(nb, sp))
     np.testing.assert_array_equal(kv.cpu().numpy().reshape(w.B, w.Hh, nb, keep), ref)

@@ -318,6 +318,14 @@ def test_topk_ties_go_to_lower_index_and_bruteforce():
     assert (oracle.draft_topk(L, 9) == np.arange(9)).all()
 
 
+def test_logits_match_library_dot():
+    rng = np.random.default_rng(7)
+    a = rng.standard_normal((1, 2, 11, 32))
+    b = rng.standard_normal((1, 2, 13, 32))
+    np.testing.assert_allclose(oracle.draft_logits(a, b), np.einsum("bhic,bhjc->bhij", a, b),
+                               rtol=1e-13, atol=1e-13)
+
+
 def test_logits_match_library_dot_within_the_fp32_bound():
     # Recursive summation of D rounded products: |fl(L) - L| <= gamma_D *
     # sum_c |q_c k_c| with gamma_D = D u / (1 - D u), u = 2^-24 (Higham,
@@ -326,7 +334,7 @@ def test_logits_match_library_dot_within_the_fp32_bound():
     rng = np.random.default_rng(7)
     a = rng.standard_normal((1, 2, 11, 32))
     b = rng.standard_normal((1, 2, 13, 32))
-    got = oracle.draft_logits(a, b)
+    got = oracle.draft_logits(a, b, "fp32")
     assert got.dtype == np.float32
     a32, b32 = (x.astype(np.float32).astype(np.float64) for x in (a, b))
     exact = np.einsum("bhic,bhjc->bhij", a32, b32)
@@ -334,8 +342,8 @@ def test_logits_match_library_dot_within_the_fp32_bound():
     gamma = 32 * u / (1 - 32 * u)
     bound = gamma * np.einsum("bhic,bhjc->bhij", np.abs(a32), np.abs(b32))
     assert (np.abs(got.astype(np.float64) - exact) <= bound).all()
-    # and it is not the fp64 dot: some logit differs from it
-    assert (got.astype(np.float64) != np.einsum("bhic,bhjc->bhij", a, b)).any()
+    # and it is not the fp64 chain: some logit differs from it
+    assert (got.astype(np.float64) != oracle.draft_logits(a, b)).any()
 
 
 # ---------------------------------------------------------------------------
@@ -690,6 +698,24 @@ def test_pool_sums_in_row_major_order():
     assert ((2.0 ** -53 + 1.0) + 2.0 ** -53) / 4 != got     # the other order differs
 
 
+def test_logits_are_sequential_and_unfused():
+    # channel 0 first: acc = -(1 + 2^-29); channel 1 adds the rounded product
+    # x*x with x = 1 + 2^-30, i.e. 1 + 2^-29 (the exact square carries an
+    # extra 2^-60), so the sum is exactly 0.  A fused multiply-add would keep
+    # 2^-60; the reversed order would give the same 0 here, so a second
+    # case pins the order: 1, then 2^-53 twice, rounds back to 1 each time.
+    x = 1.0 + 2.0 ** -30
+    q = np.array([1.0, x]).reshape(1, 1, 1, 2)
+    k = np.array([-(1.0 + 2.0 ** -29), x]).reshape(1, 1, 1, 2)
+    assert oracle.draft_logits(q, k)[0, 0, 0, 0] == 0.0
+    # the exact value a fused multiply-add would round: 2^-60, not 0
+    assert Fraction(x) * Fraction(x) - Fraction(1.0 + 2.0 ** -29) == Fraction(1, 2 ** 60)
+    q = np.ones((1, 1, 1, 3))
+    k = np.array([1.0, 2.0 ** -53, 2.0 ** -53]).reshape(1, 1, 1, 3)
+    assert oracle.draft_logits(q, k)[0, 0, 0, 0] == 1.0                 # c = 0, 1, 2
+    assert (2.0 ** -53 + 2.0 ** -53) + 1.0 == 1.0 + 2.0 ** -52           # reversed differs
+
+
 def test_logits_are_fp32_sequential_and_unfused():
     # channel 0 first: acc = -(1 + 2^-11); channel 1 adds the rounded product
     # x*x with x = 1 + 2^-12: the exact square 1 + 2^-11 + 2^-24 lies half an
@@ -699,23 +725,23 @@ def test_logits_are_fp32_sequential_and_unfused():
     assert Fraction(x) * Fraction(x) - Fraction(1.0 + 2.0 ** -11) == Fraction(1, 2 ** 24)
     q = np.array([1.0, x]).reshape(1, 1, 1, 2)
     k = np.array([-(1.0 + 2.0 ** -11), x]).reshape(1, 1, 1, 2)
-    assert oracle.draft_logits(q, k)[0, 0, 0, 0] == 0.0
+    assert oracle.draft_logits(q, k, "fp32")[0, 0, 0, 0] == 0.0
     # the products are rounded to fp32, not fp64: x*x alone
-    one = oracle.draft_logits(np.array([x]).reshape(1, 1, 1, 1), np.array([x]).reshape(1, 1, 1, 1))
+    one = oracle.draft_logits(np.array([x]).reshape(1, 1, 1, 1), np.array([x]).reshape(1, 1, 1, 1), "fp32")
     assert one[0, 0, 0, 0] == 1.0 + 2.0 ** -11 and x * x != 1.0 + 2.0 ** -11
     # order: 1, then 2^-24 twice, rounds back to 1 each time (half an ulp,
     # ties to even); the reversed order gives 1 + 2^-23
     q = np.ones((1, 1, 1, 3))
     k = np.array([1.0, 2.0 ** -24, 2.0 ** -24]).reshape(1, 1, 1, 3)
-    assert oracle.draft_logits(q, k)[0, 0, 0, 0] == 1.0
+    assert oracle.draft_logits(q, k, "fp32")[0, 0, 0, 0] == 1.0
     assert np.float32(np.float32(2.0 ** -24) + np.float32(2.0 ** -24)) + np.float32(1.0) == \
         np.float32(1.0 + 2.0 ** -23)
     # the pooled values are rounded to the nearest fp32 before the products:
     # 1 + 3*2^-25 is 0.75 ulp above 1 and rounds up, 1 + 2^-30 rounds down
     ones = np.ones((1, 1, 1, 1))
-    assert oracle.draft_logits(np.full((1, 1, 1, 1), 1.0 + 3 * 2.0 ** -25), ones)[0, 0, 0, 0] == \
+    assert oracle.draft_logits(np.full((1, 1, 1, 1), 1.0 + 3 * 2.0 ** -25), ones, "fp32")[0, 0, 0, 0] == \
         1.0 + 2.0 ** -23
-    assert oracle.draft_logits(np.full((1, 1, 1, 1), 1.0 + 2.0 ** -30), ones)[0, 0, 0, 0] == 1.0
+    assert oracle.draft_logits(np.full((1, 1, 1, 1), 1.0 + 2.0 ** -30), ones, "fp32")[0, 0, 0, 0] == 1.0
 
 
 def test_lvsa_block_csr_literal_table_two_blocks_per_frame():

@@ -3,7 +3,7 @@
 Some callers cannot allocate device memory of their own (a plugin whose host
 program owns every allocation and passes only input and output buffers; a
 caller on a fixed memory budget).  bsa_draft_mask_noalloc computes what
-bsa_draft_mask computes, with its scratch in a fixed 32 MiB array inside the
+bsa_draft_mask computes, with its scratch in a fixed 48 MiB array inside the
 library instead of a caller workspace.  Here it is called through the C ABI
 twice in a row, on two different problems, and each time its outputs must
 equal those of bsa_draft_mask on the same inputs (block lists bit for bit,
@@ -68,8 +68,8 @@ def test_noalloc_matches_workspace_version_on_two_calls_in_a_row():
 
 def test_noalloc_rejects_problems_above_its_scratch():
     cap = bsa.bsa_draft_noalloc_max_scratch_bytes()
-    assert cap == 32 << 20
-    # 40 heads on a 21 x 60 x 104 grid in 8 x 16 tiles: 1344 blocks, 55 MB of scratch
+    assert cap == 48 << 20
+    # 40 heads on a 21 x 60 x 104 grid in 8 x 16 tiles: 1344 blocks, 165 MB of scratch
     plan = bsa.Plan(1, 40, 128, 21, 60, 104, bsa.LAYOUT_TILE, 8, 16, 128)
     assert bsa.bsa_draft_workspace_bytes(plan) > cap
     buf = torch.empty(16, dtype=torch.int32, device="cuda")
@@ -80,4 +80,4 @@ def test_noalloc_rejects_problems_above_its_scratch():
         bsa.bsa_draft_mask_noalloc(plan, x.data_ptr(), x.data_ptr(), 90, buf.data_ptr(),
                                    buf.data_ptr(), None)
     assert ei.value.status == 2
-    assert "32 MiB" in bsa.bsa_last_error()
+    assert "48 MiB" in bsa.bsa_last_error()
