@@ -457,6 +457,94 @@ struct ErrBound {
   static constexpr double value = 2.0 * (g32 * (1.0 + u32) * (1.0 + u32) + 2.0 * u32 + u32 * u32 + g64);
 };
 
+// The fp64 logit of query block `qr` and key block `kr` (D values each),
+// computed by the whole warp: lanes form the rounded products, then every
+// lane adds them in channel order.
+template <int D>
+__device__ __forceinline__ double warp_logit64(const double* qr, const double* kr, int lane) {
+  double pr[D / 32];
+#pragma unroll
+  for (int m = 0; m < D / 32; ++m) pr[m] = __dmul_rn(qr[lane + 32 * m], kr[lane + 32 * m]);
+  double L = 0.0;
+#pragma unroll
+  for (int c = 0; c < D; ++c) L = __dadd_rn(L, __shfl_sync(kFullMaskScore, pr[c >> 5], c & 31));
+  return L;
+}
+
+// Ranks a row's band (bit u of `band`: key block lane + 32u) on the fp64
+// logits and adds the `need` largest (then lowest block index) to `taken`.
+// sv / sj: this warp's list space in shared memory (NK entries).  Kept out
+// of line: it runs for few rows, and its registers stay out of the scorer's.
+template <int D, int U>
+__device__ __noinline__ uint32_t rank_band64(const double* __restrict__ qr,
+                                            const double* __restrict__ khead, uint32_t band,
+                                            int need, uint32_t taken, int lane, double* sv,
+                                            int* sj) {
+  int cnt = 0;
+#pragma unroll 1
+  for (int u = 0; u < U; ++u) {
+    uint32_t bb = __ballot_sync(kFullMaskScore, (band >> u) & 1u);
+    while (bb) {
+      const int j = (__ffs(bb) - 1) + 32 * u;
+      bb &= bb - 1;
+      const double L = warp_logit64<D>(qr, khead + (int64_t)j * D, lane);
+      if (lane == 0) {
+        sv[cnt] = L;
+        sj[cnt] = j;
+      }
+      ++cnt;
+    }
+  }
+  __syncwarp();
+  for (int it = 0; it < need; ++it) {
+    double best = 0.0;
+    int bj = 0x7fffffff, be = -1;
+    for (int x = lane; x < cnt; x += 32) {
+      const int j = sj[x];
+      if (j < 0) continue;
+      const double v = sv[x];
+      if (be < 0 || v > best || (v == best && j < bj)) {
+        best = v;
+        bj = j;
+        be = x;
+      }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      const double ov = __shfl_xor_sync(kFullMaskScore, best, o);
+      const int oj = __shfl_xor_sync(kFullMaskScore, bj, o);
+      const int oe = __shfl_xor_sync(kFullMaskScore, be, o);
+      if (oe >= 0 && (be < 0 || ov > best || (ov == best && oj < bj))) {
+        best = ov;
+        bj = oj;
+        be = oe;
+      }
+    }
+    if (be >= 0) {
+      if (lane == (bj & 31)) taken |= 1u << (bj >> 5);
+      if (lane == 0) sj[be] = -1;
+    }
+    __syncwarp();
+  }
+  return taken;
+}
+
+// The fp64 logits of one row for the draft map (lane's keys lane + 32u).
+template <int D, int U>
+__device__ __noinline__ void row_logits64(const double* __restrict__ qr,
+                                          const double* __restrict__ khead, int nblocks, int lane,
+                                          double* lv) {
+#pragma unroll 1
+  for (int u = 0; u < U; ++u) {
+    double a = 0.0;
+    if (lane + 32 * u < nblocks) {
+      const double* kr = khead + (int64_t)(lane + 32 * u) * D;
+      for (int c = 0; c < D; ++c) a = __dadd_rn(a, __dmul_rn(qr[c], kr[c]));
+    }
+    lv[u] = a;
+  }
+}
+
 // grid: (ceil(nblocks / kRows), Hh, B).  CERT: the plan's precision is fp64;
 // the fp32 logits pick the blocks that are certain under the error bound,
 // and only the ones within it of the k-th logit get their fp64 logits (from
@@ -599,7 +687,9 @@ __global__ void __launch_bounds__(32 * kRegScoreWarps, U <= 12 ? 4 : 3)
       // all of it is needed
       const double t = (double)key_value(Tk[r]);
       const double e = ErrBound<D>::value * (double)qnorm[bh * nblocks + row] * (double)kmax + 0x1p-100;
-      double lo = t - 2.0 * e, hi = t + 2.0 * e;
+      // bounds rounded outwards to fp32: compared with the fp32 logits they
+      // keep every block the fp64 bounds would put in the band
+      float lo = __double2float_rd(t - 2.0 * e), hi = __double2float_ru(t + 2.0 * e);
       if (!(lo > -INFINITY && hi < INFINITY)) {  // overflow or NaN: decide all in fp64
         lo = -INFINITY;
         hi = INFINITY;
@@ -608,7 +698,7 @@ __global__ void __launch_bounds__(32 * kRegScoreWarps, U <= 12 ? 4 : 3)
 #pragma unroll
       for (int u = 0; u < U; ++u) {
         if (key[r][u] == 0u) continue;
-        const double L = (double)key_value(key[r][u]);
+        const float L = key_value(key[r][u]);
         if (L > hi)
           taken |= 1u << u;
         else if (L >= lo)
@@ -616,71 +706,15 @@ __global__ void __launch_bounds__(32 * kRegScoreWarps, U <= 12 ? 4 : 3)
       }
       const int need = keep - (int)__reduce_add_sync(kFullMaskScore, (unsigned)__popc(taken));
       const int nband = (int)__reduce_add_sync(kFullMaskScore, (unsigned)__popc(band));
+      by_index = false;
       if (nband == need) {
         taken |= band;
       } else {
-        // the band's fp64 logits, one block at a time: lanes form the D
-        // rounded products, then every lane adds them in channel order
-        by_index = false;
         double* sv = reinterpret_cast<double*>(shf4) + warp * NK;
         int* sj = reinterpret_cast<int*>(reinterpret_cast<double*>(shf4) + kRegScoreWarps * NK) +
                   warp * NK;
-        const double* qr = q64 + (bh * nblocks + row) * D;
-        int cnt = 0;
-#pragma unroll
-        for (int u = 0; u < U; ++u) {
-          uint32_t bb = __ballot_sync(kFullMaskScore, (band >> u) & 1u);
-          while (bb) {
-            const int j = (__ffs(bb) - 1) + 32 * u;
-            bb &= bb - 1;
-            const double* kr = k64 + (bh * nblocks + j) * D;
-            double pr[D / 32];
-#pragma unroll
-            for (int m = 0; m < D / 32; ++m) pr[m] = __dmul_rn(qr[lane + 32 * m], kr[lane + 32 * m]);
-            double L64 = 0.0;
-#pragma unroll
-            for (int c = 0; c < D; ++c)
-              L64 = __dadd_rn(L64, __shfl_sync(kFullMaskScore, pr[c >> 5], c & 31));
-            if (lane == 0) {
-              sv[cnt] = L64;
-              sj[cnt] = j;
-            }
-            ++cnt;
-          }
-        }
-        __syncwarp();
-        // `need` rounds of a warp-wide arg-max over the list: larger fp64
-        // logit, then the lower block index
-        for (int it = 0; it < need; ++it) {
-          double best = 0.0;
-          int bj = 0x7fffffff, be = -1;
-          for (int x = lane; x < cnt; x += 32) {
-            const int j = sj[x];
-            if (j < 0) continue;
-            const double v = sv[x];
-            if (be < 0 || v > best || (v == best && j < bj)) {
-              best = v;
-              bj = j;
-              be = x;
-            }
-          }
-#pragma unroll
-          for (int o = 16; o > 0; o >>= 1) {
-            const double ov = __shfl_xor_sync(kFullMaskScore, best, o);
-            const int oj = __shfl_xor_sync(kFullMaskScore, bj, o);
-            const int oe = __shfl_xor_sync(kFullMaskScore, be, o);
-            if (oe >= 0 && (be < 0 || ov > best || (ov == best && oj < bj))) {
-              best = ov;
-              bj = oj;
-              be = oe;
-            }
-          }
-          if (be >= 0) {
-            if (lane == (bj & 31)) taken |= 1u << (bj >> 5);
-            if (lane == 0) sj[be] = -1;
-          }
-          __syncwarp();
-        }
+        taken = rank_band64<D, U>(q64 + (bh * nblocks + row) * D, k64 + bh * nblocks * D, band,
+                                  need, taken, lane, sv, sj);
       }
     }
     if (by_index) {
@@ -726,19 +760,13 @@ __global__ void __launch_bounds__(32 * kRegScoreWarps, U <= 12 ? 4 : 3)
     }
     if (draft_map) {
       double lv[U];
+      if constexpr (CERT) {  // the map of the fp64 logits
+        row_logits64<D, U>(q64 + (bh * nblocks + row) * D, k64 + bh * nblocks * D, nblocks, lane,
+                           lv);
+      } else {  // fp32 logits come back from their keys (exactly)
 #pragma unroll
-      for (int u = 0; u < U; ++u) {
-        if (!(lane + 32 * u < nblocks)) {
-          lv[u] = 0.0;
-        } else if constexpr (CERT) {  // the map of the fp64 logits
-          const double* qr = q64 + (bh * nblocks + row) * D;
-          const double* kr = k64 + (bh * nblocks + lane + 32 * u) * D;
-          double a = 0.0;
-          for (int c = 0; c < D; ++c) a = __dadd_rn(a, __dmul_rn(qr[c], kr[c]));
-          lv[u] = a;
-        } else {  // fp32 logits come back from their keys (exactly)
-          lv[u] = (double)key_value(key[r][u]);
-        }
+        for (int u = 0; u < U; ++u)
+          lv[u] = lane + 32 * u < nblocks ? (double)key_value(key[r][u]) : 0.0;
       }
       double mx = -DBL_MAX;
 #pragma unroll
