@@ -433,7 +433,8 @@ def hbm_kernels(cid: int):
     att = DraftAttention(w.B, w.Hh, w.D, w.T, w.H, w.W, w.draft_ph or 8, w.draft_pw or 16,
                          w.draft_sparsity or 90)
     nb = att.plan.nblocks
-    pooled = 2 * w.B * w.Hh * nb * w.D * 8
+    pooled = 2 * w.B * w.Hh * nb * w.D * 8    # fp64 pooled Q and K
+    norms = 2 * w.B * w.Hh * nb * 4
     for _ in range(2):
         bsa.bsa_reorder_fwd(fr, q, fq, k, fk, v, fv)
         bsa.bsa_reorder_inv(fr, fq, out)
@@ -451,11 +452,12 @@ def hbm_kernels(cid: int):
         "algo_bytes_per_launch": {
             "reorder_fwd_kernel (Q K V, either layout)": 3 * 2 * tok,
             "reorder_inv_kernel (O, either layout)": 2 * tok,
-            "draft_pool_kernel (tile-layout Q K slots read, pooled fp64 written)":
-                2 * w.B * w.Hh * att.plan.Npad * w.D * 2 + pooled,
-            "draft_pool_kernel natural (natural Q K read, pooled fp64 written)": 2 * tok + pooled,
-            "draft_score_reg_kernel (pooled fp64 read, lists written)":
-                pooled + 4 * att.col_idx.numel(),
+            "draft_pool_kernel (tile-layout Q K slots read; fp64 values, fp32 copies, norms written)":
+                2 * w.B * w.Hh * att.plan.Npad * w.D * 2 + pooled + pooled // 2 + norms,
+            "draft_pool_kernel natural (natural Q K read; fp64 values, fp32 copies, norms written)":
+                2 * tok + pooled + pooled // 2 + norms,
+            "draft_score_reg_kernel (fp32 copies and norms read, lists written)":
+                pooled // 2 + norms + 4 * att.col_idx.numel(),
             "e4m3_amax_kernel (Q K V read)": 3 * tok,
             "e4m3_convert_kernel (Q K V read, codes written)": 3 * tok + 3 * tok // 2},
         "slots": {"frame_Npad": fr.Npad, "tile_Npad": att.plan.Npad}}), flush=True)
