@@ -42,9 +42,12 @@ def _outputs(plan, keep):
     return rp, kv, dm
 
 
-def test_noalloc_matches_workspace_version_on_two_calls_in_a_row():
+@pytest.mark.parametrize("precision", [bsa.DRAFT_FP64, bsa.DRAFT_FP32])
+def test_noalloc_matches_workspace_version_on_two_calls_in_a_row(precision):
     cases = [_case(21, 30, 52, 12, 128, 8, 16, 90, seed=1),   # Wan-1.3B-like native grid
              _case(3, 20, 36, 4, 64, 4, 8, 75, seed=2)]       # smaller, other head dim
+    for plan, _, _, _ in cases:
+        bsa.bsa_plan_set_draft_precision(plan, precision)
     got = []
     for plan, q, k, sp in cases:
         keep = bsa.bsa_draft_keep_count(plan, sp)
