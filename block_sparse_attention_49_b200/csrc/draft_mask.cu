@@ -8,16 +8,20 @@
 // layout (each block = one pool_h x pool_w tile):
 //  pool:  qbar/kbar[b,h,blk,:] = mean of the tile's tokens: the sum runs
 //         in fp64, sequentially over the tile's tokens in row-major order,
-//         is divided once by the token count and rounded once to fp32.
-//         With max pooling (which the article's authors tried before
-//         settling on the average) it is the channel-wise maximum instead,
-//         exact in any order.  16-byte loads, four rows ahead; HBM bound.
-//  score_topk: for a group of query-block rows of one (b, head), the fp32
-//         logits L[i][j] = sum_c qbar_i[c]*kbar_j[c] (sequential over c, the
-//         product and the sum each rounded to fp32, no fused multiply-add),
-//         then per row the k largest, ties to the lower j, by k rounds of a
-//         warp-wide arg-max; written ascending.  Optionally the draft map
+//         and is divided once by the token count.  With max pooling (which
+//         the article's authors tried before settling on the average) it is
+//         the channel-wise maximum instead, exact in any order.  Written as
+//         fp32 (rounded once), and in the default fp64 precision also as
+//         fp64 with an upper bound of each vector's 2-norm.  16-byte loads,
+//         four rows ahead; HBM bound.
+//  score: for a group of query-block rows of one (b, head), the logits
+//         L[i][j] = sum_c qbar_i[c]*kbar_j[c], sequential over c, the
+//         product and the sum each rounded (no fused multiply-add), in the
+//         plan's precision; per row the k largest, ties to the lower j,
+//         written ascending.  Optionally the draft map
 //         softmax_j(L[i][j]/sqrt(D)), evaluated in fp64 and stored as fp32.
+//         The fp64 lists come out of fp32 logits and a proven bound on their
+//         distance to the fp64 ones (see draft_score_reg_kernel).
 // With this fixed evaluation order the selection is reproducible bit for bit
 // by any implementation that follows the same order.
 #include <cuda_bf16.h>
@@ -398,19 +402,18 @@ __global__ void __launch_bounds__(kScoreThreads)
 // ---------------------------------------------------------------------------
 // Scoring with the logits in registers (up to 512 key blocks per row).
 //
-// A warp owns R whole query-block rows; lane l accumulates the logits of key
-// blocks j = l + 32u (u < U) of each row, so a row's top-k runs straight out
-// of registers and no logit ever goes to shared memory.  Every logit is the
-// sequential multiply-then-add chain over c = 0..D-1, each operation rounded
-// to the logit's precision.
-//   fp32: rows are held in pairs, one fp32 pair per key, updated with the
-//     two-wide fp32 multiply and add (each lane of the pair rounded on its
-//     own); keys staged 16 channels at a time as [channel quad][key][4].
-//   fp64: one double per (row, key); keys staged 8 channels at a time as
-//     [channel pair][key][2].
-// Either way a lane reads one key's channels with one 16-byte load and a
-// warp's loads are contiguous; the pooled query values are staged as
-// [channel][row] and read by broadcast.
+// A warp owns R whole query-block rows; lane l accumulates the fp32 logits
+// of key blocks j = l + 32u (u < U) of each row, so a row's top-k runs
+// straight out of registers and no logit ever goes to shared memory.  Every
+// logit is the sequential multiply-then-add chain over c = 0..D-1, each
+// operation rounded to fp32.  Rows are held in pairs, one fp32 pair per key,
+// updated with the two-wide fp32 multiply and add (each lane of the pair
+// rounded on its own).  Keys are staged 16 channels at a time as [channel
+// quad][key][4], so a lane reads four channels of one key with one 16-byte
+// load and a warp's loads are contiguous; the pooled query values are
+// staged as [channel][row] and read by broadcast.  For the default fp64
+// lists the fp32 logits decide every block that lies clearly above or below
+// the k-th, and the rest get their fp64 logits (CERT).
 // ---------------------------------------------------------------------------
 constexpr int kRegScoreWarps = 4;
 
