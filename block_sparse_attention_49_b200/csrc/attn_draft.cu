@@ -25,10 +25,10 @@
 //   warp 0      TMA producer of Q (after the last QK of tile i-1) and of K
 //               into a ring (3 deep, 4 for e4m3); warp 3 of V into a ring
 //               (2 deep, 4 for e4m3): K is needed a softmax earlier than V.
-//               On the natural layout, edge tiles (partial tiles at the
-//               grid's right and bottom edges) are packed several to a
-//               128-row MMA tile, each piece loaded with a box of its exact
-//               size.
+//               On the tile layout (natural tensors, or the slots of a
+//               TILE plan), edge tiles (partial tiles at the grid's right
+//               and bottom edges) are packed several to a 128-row MMA
+//               tile, each piece loaded with a box of its exact size.
 //   warp 1      MMA issuer: a group's PV in two halves as its P halves
 //               arrive, then that group's next QK; the first PV of tile i
 //               waits until tile i-1's output has been read out of tensor
@@ -41,9 +41,8 @@
 //               sum, P (bf16, or e4m3 four keys to a column) over its S;
 //               then the epilogue of the tile: the two groups' partial
 //               results merged (a split-key combine), normalised and stored.
-// Tensor memory: S_A | S_B | O_A | O_B (512 columns).  The arithmetic per
-// tile is that of bsa_attn_fwd's block-list kernel, so on a grid without
-// partial tiles the natural and slot forms give identical bits.
+// Tensor memory: S_A | S_B | O_A | O_B (512 columns).  The natural and slot
+// forms pack the same tiles in the same order, so they give identical bits.
 // Every wait is bounded; a wait that runs out records a timeout in the
 // plan's status word and the CTA leaves without trapping.
 #include <cuda_bf16.h>
@@ -446,12 +445,22 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
               for (int e = 0; e < 3; ++e) {
                 for (int m = 0; m < a[e]; ++m) {
-                  int x0, y0, fr;
-                  nat_coords(ent[pstart[e] + pptr[e] + m], b, x0, y0, fr);
+                  const int kt = ent[pstart[e] + pptr[e] + m];
                   const CUtensorMap* mx = isK ? &em.k[p.pk_kind[e] - 1] : &em.v[p.pk_kind[e] - 1];
-                  for (int c = 0; c < Cfg::kChunks; ++c)
-                    tma_load_5d(dst + c * Cfg::kPanel + off * 128, mx, &full[st],
-                                c * Cfg::kChunkElems, h, x0, y0, fr);
+                  if (p.slot) {
+                    // the piece's valid slots: a box of its exact size in the
+                    // [tile][row][column] view of the slot tensor
+                    const int tile = (int)(((int64_t)b * p.Hh + h) * p.nblocks + kt);
+                    for (int c = 0; c < Cfg::kChunks; ++c)
+                      tma_load_4d(dst + c * Cfg::kPanel + off * 128, mx, &full[st],
+                                  c * Cfg::kChunkElems, 0, 0, tile);
+                  } else {
+                    int x0, y0, fr;
+                    nat_coords(kt, b, x0, y0, fr);
+                    for (int c = 0; c < Cfg::kChunks; ++c)
+                      tma_load_5d(dst + c * Cfg::kPanel + off * 128, mx, &full[st],
+                                  c * Cfg::kChunkElems, h, x0, y0, fr);
+                  }
                   off += p.pk_step[e];
                 }
               }
@@ -853,6 +862,23 @@ bool make_slot_tmap(CUtensorMap* m, const void* ptr, int64_t rows, int D) {
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// Slot tensors of a TILE plan (128 slots = one ph x pw tile, row-major) as a
+// 4-D [B*Hh*nblocks][ph][pw][D] tensor; boxes of 64 channels x box_w x box_h,
+// 128-byte swizzle: the valid slots of an edge tile, in row-major order.
+bool make_slot_edge_tmap(CUtensorMap* m, const void* ptr, const Geometry& g, int box_w, int box_h) {
+  auto fn = draft_encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[4] = {(cuuint64_t)g.D, (cuuint64_t)g.pw, (cuuint64_t)g.ph,
+                        (cuuint64_t)g.B * g.Hh * g.nblocks};
+  cuuint64_t strides[3] = {(cuuint64_t)g.D * 2, (cuuint64_t)g.pw * g.D * 2,
+                           (cuuint64_t)kTile * g.D * 2};
+  cuuint32_t box[4] = {64, (cuuint32_t)box_w, (cuuint32_t)box_h, 1};
+  cuuint32_t estr[4] = {1, 1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(ptr), dims, strides, box,
+            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 int draft_sm_count() {
   static int n[64] = {};
   int dev = 0;
@@ -942,7 +968,7 @@ bsa_status launch_attn_draft(const bsa_plan_s& plan, const void* q, const void* 
   p.wait_limit_ns = plan.wait_limit_ns;
   DraftEdgeMaps em;
   memset(&em, 0, sizeof(em));
-  if (slot) {
+  if (slot && g.layout != BSA_LAYOUT_TILE) {
     // key tiles as stored (empty slots masked), no packing; the tile-grid
     // divisors are unused
     p.div_tile_frame = FastDiv(1u);
@@ -953,6 +979,7 @@ bsa_status launch_attn_draft(const bsa_plan_s& plan, const void* q, const void* 
     if (e != cudaSuccess) return cuda_error(e, "draft attention launch");
     return BSA_OK;
   }
+  // the tile layout (natural tensors or their slots): edge tiles packed
   p.div_tile_frame = FastDiv((uint32_t)(g.TH * g.TW));
   p.div_TW = FastDiv((uint32_t)g.TW);
   p.div_pw = FastDiv((uint32_t)g.pw);
@@ -963,9 +990,11 @@ bsa_status launch_attn_draft(const bsa_plan_s& plan, const void* q, const void* 
       p.pk_kind[i] = kind[i];
       p.pk_rows[i] = rows[i];
       p.pk_step[i] = (rows[i] + 7) / 8 * 8;
-      if (!make_draft_tmap(&em.k[kind[i] - 1], k, g, bw[i], bh[i], f8) ||
-          !make_draft_tmap(&em.v[kind[i] - 1], v, g, bw[i], bh[i], f8))
-        return set_error(BSA_ERR_CUDA, "cuTensorMapEncodeTiled (5-D edge boxes) failed");
+      const bool ok = slot ? make_slot_edge_tmap(&em.k[kind[i] - 1], k, g, bw[i], bh[i]) &&
+                                 make_slot_edge_tmap(&em.v[kind[i] - 1], v, g, bw[i], bh[i])
+                           : make_draft_tmap(&em.k[kind[i] - 1], k, g, bw[i], bh[i], f8) &&
+                                 make_draft_tmap(&em.v[kind[i] - 1], v, g, bw[i], bh[i], f8);
+      if (!ok) return set_error(BSA_ERR_CUDA, "cuTensorMapEncodeTiled (edge boxes) failed");
     }
     p.pk_on = 1;
   }
