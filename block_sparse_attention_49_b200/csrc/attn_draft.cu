@@ -157,7 +157,9 @@ __device__ __forceinline__ void next_bin(const DraftParams& p, int (&r)[3], int 
 
 __device__ __forceinline__ void end_sync() { asm volatile("bar.sync 2, 384;" ::: "memory"); }
 
-template <int D, bool F8>
+// SLOT: slot tensors (p.slot); a template flag, so the natural-layout
+// kernel carries none of the slot paths' code.
+template <int D, bool F8, bool SLOT>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_draft_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmk,
                       const __grid_constant__ CUtensorMap tmv, const DraftParams p,
@@ -409,7 +411,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (!__all_sync(kAll, bounded_wait(q_empty, (uint32_t)(i & 1) ^ 1u, wc))) break;
           if (elect_one()) {
             mbar_arrive_expect_tx(q_full, Cfg::kTileBytes);
-            if (p.slot) {
+            if constexpr (SLOT) {
               const int row0 = (int)(((int64_t)b * p.Hh + h) * p.Npad + (int64_t)qt * kTile);
               for (int c = 0; c < Cfg::kChunks; ++c)
                 tma_load_2d(sQ + c * Cfg::kPanel, &tmq, q_full, c * Cfg::kChunkElems, row0);
@@ -447,7 +449,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 for (int m = 0; m < a[e]; ++m) {
                   const int kt = ent[pstart[e] + pptr[e] + m];
                   const CUtensorMap* mx = isK ? &em.k[p.pk_kind[e] - 1] : &em.v[p.pk_kind[e] - 1];
-                  if (p.slot) {
+                  if constexpr (SLOT) {
                     // the piece's valid slots: a box of its exact size in the
                     // [tile][row][column] view of the slot tensor
                     const int tile = (int)(((int64_t)b * p.Hh + h) * p.nblocks + kt);
@@ -480,7 +482,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             if (elect_one()) {
               mbar_arrive_expect_tx(&full[st], Cfg::kTileBytes);
-              if (p.slot) {
+              if constexpr (SLOT) {
                 const int row0 = (int)(((int64_t)b * p.Hh + h) * p.Npad + (int64_t)kt * kTile);
                 for (int c = 0; c < Cfg::kChunks; ++c)
                   tma_load_2d(dst + c * Cfg::kPanel, tmx, &full[st], c * Cfg::kChunkElems, row0);
@@ -756,7 +758,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const float l = lA * a + lB * bb;
       bool qvalid;
       int64_t orow, lrow;
-      if (p.slot) {
+      if constexpr (SLOT) {
         // slot tensors: row `row` of tile qt; an empty slot is written as 0
         // (LSE -inf) like every slot of the layout
         const uint4 tq = __ldg(reinterpret_cast<const uint4*>(p.tile_valid) + qt);
@@ -777,7 +779,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         orow = ((int64_t)b * p.N + ntok) * p.Hh + h;
         lrow = ((int64_t)b * p.Hh + h) * p.N + ntok;
       }
-      const bool write = qvalid || p.slot;
+      const bool write = qvalid || SLOT;
       const bool has = n > 0 && qvalid && l > 0.f;
       const float inv_l = has ? sv / l : 0.f;
       const float wa = a * inv_l, wb = bb * inv_l;
@@ -896,7 +898,7 @@ template <int D, bool F8 = false>
 cudaError_t launch_draft_t(const CUtensorMap& q, const CUtensorMap& k, const CUtensorMap& v,
                            const DraftParams& p, const DraftEdgeMaps& em, cudaStream_t st) {
   using Cfg = DraftCfg<D, F8>;
-  auto kern = attn_draft_kernel<D, F8>;
+  auto kern = p.slot ? attn_draft_kernel<D, F8, true> : attn_draft_kernel<D, F8, false>;
   cudaError_t e =
       cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::kSmem);
   if (e != cudaSuccess) return e;
