@@ -20,9 +20,10 @@ from typing import Optional
 __all__ = [
     "BsaError", "Plan", "LAYOUT_FRAME", "LAYOUT_TILE", "lib_path", "load",
     "ANCHORS_ROTATING", "ANCHORS_FIXED", "ANCHORS_NONE", "WINDOW_DISTANCE", "WINDOW_ALTERNATE",
-    "POOL_MEAN", "POOL_MAX", "DRAFT_FP64", "DRAFT_FP32",
+    "POOL_MEAN", "POOL_MAX", "DRAFT_FP64", "DRAFT_FP32", "PADS_WRITE", "PADS_KEEP",
     "bsa_plan_create", "bsa_plan_destroy", "bsa_plan_set_lvsa_variant",
-    "bsa_plan_set_draft_pooling", "bsa_plan_set_draft_precision", "bsa_padded_tokens",
+    "bsa_plan_set_draft_pooling", "bsa_plan_set_draft_precision", "bsa_plan_set_reorder_pads",
+    "bsa_padded_tokens",
     "bsa_num_blocks",
     "bsa_block_size", "bsa_lvsa_mask", "bsa_lvsa_nnz", "bsa_draft_keep_count",
     "bsa_draft_workspace_bytes", "bsa_draft_mask", "bsa_draft_mask_noalloc",
@@ -38,6 +39,7 @@ ANCHORS_ROTATING, ANCHORS_FIXED, ANCHORS_NONE = 0, 1, 2
 WINDOW_DISTANCE, WINDOW_ALTERNATE = 0, 1
 POOL_MEAN, POOL_MAX = 0, 1
 DRAFT_FP64, DRAFT_FP32 = 0, 1
+PADS_WRITE, PADS_KEEP = 0, 1
 
 STATUS = {0: "BSA_OK", 1: "BSA_ERR_INVALID_ARG", 2: "BSA_ERR_UNSUPPORTED",
           3: "BSA_ERR_ALIGNMENT", 4: "BSA_ERR_CUDA", 5: "BSA_ERR_TIMEOUT",
@@ -56,6 +58,7 @@ _SIGS = {
     "bsa_plan_set_lvsa_variant": (_c_int, [_c_p, _c_int, _c_int]),
     "bsa_plan_set_draft_pooling": (_c_int, [_c_p, _c_int]),
     "bsa_plan_set_draft_precision": (_c_int, [_c_p, _c_int]),
+    "bsa_plan_set_reorder_pads": (_c_int, [_c_p, _c_int]),
     "bsa_padded_tokens": (_c_i64, [_c_p]),
     "bsa_num_blocks": (_c_i64, [_c_p]),
     "bsa_block_size": (_c_int, [_c_p]),
@@ -399,6 +402,10 @@ def bsa_plan_set_draft_pooling(plan: Plan, pooling: int):
 def bsa_plan_set_draft_precision(plan: Plan, precision: int):
     _check(load().bsa_plan_set_draft_precision(plan.handle, int(precision)),
            "bsa_plan_set_draft_precision")
+
+
+def bsa_plan_set_reorder_pads(plan: Plan, pads: int):
+    _check(load().bsa_plan_set_reorder_pads(plan.handle, int(pads)), "bsa_plan_set_reorder_pads")
 
 
 def bsa_set_wait_limit_ns(plan: Plan, ns: int):

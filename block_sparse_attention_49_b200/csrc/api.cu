@@ -266,7 +266,8 @@ bsa_status bsa_reorder_fwd(bsa_plan_t plan, const void* x0, void* y0, const void
   for (int i = nt + 1; i < 3; ++i)
     if (xs[i] || ys[i])
       return set_error(BSA_ERR_INVALID_ARG, "tensor pair 2 given without pair 1");
-  cudaError_t e = launch_reorder_fwd(plan->g, xs, ys, nt, reinterpret_cast<cudaStream_t>(stream));
+  cudaError_t e = launch_reorder_fwd(plan->g, xs, ys, nt, plan->reorder_pads == BSA_PADS_WRITE,
+                                     reinterpret_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? BSA_OK : cuda_error(e, "reorder_fwd launch");
 }
 
@@ -446,6 +447,14 @@ bsa_status bsa_plan_set_draft_pooling(bsa_plan_t plan, int pooling) {
   if (pooling != BSA_POOL_MEAN && pooling != BSA_POOL_MAX)
     return set_error(BSA_ERR_INVALID_ARG, "unknown pooling");
   plan->draft_pooling = pooling;
+  return BSA_OK;
+}
+
+bsa_status bsa_plan_set_reorder_pads(bsa_plan_t plan, int pads) {
+  if (!plan) return set_error(BSA_ERR_INVALID_ARG, "plan is NULL");
+  if (pads != BSA_PADS_WRITE && pads != BSA_PADS_KEEP)
+    return set_error(BSA_ERR_INVALID_ARG, "unknown pad mode");
+  plan->reorder_pads = pads;
   return BSA_OK;
 }
 

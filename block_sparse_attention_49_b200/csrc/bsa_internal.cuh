@@ -69,6 +69,7 @@ struct bsa_plan_s {
   int lvsa_window = BSA_WINDOW_ALTERNATE;
   int draft_pooling = BSA_POOL_MEAN;        // bsa_plan_set_draft_pooling
   int draft_precision = BSA_DRAFT_FP64;     // bsa_plan_set_draft_precision
+  int reorder_pads = BSA_PADS_WRITE;        // bsa_plan_set_reorder_pads
   uint32_t* d_amax = nullptr;               // [3][B][Hh] scratch of bsa_quantize_e4m3
 };
 
@@ -85,7 +86,7 @@ cudaError_t launch_lvsa_mask(const Geometry& g, int C, int T_per, int s, int alt
                              int32_t* frame_sets, int32_t* row_ptr, int32_t* col_idx,
                              unsigned int* status, cudaStream_t st);
 cudaError_t launch_reorder_fwd(const Geometry& g, const void* const x[3], void* const y[3],
-                               int nt, cudaStream_t st);
+                               int nt, bool write_pads, cudaStream_t st);
 cudaError_t launch_reorder_inv(const Geometry& g, const void* x_slots, void* x_nat,
                                cudaStream_t st);
 cudaError_t launch_draft_mask(const Geometry& g, const uint32_t* tile_valid, const void* q,

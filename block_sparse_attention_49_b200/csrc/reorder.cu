@@ -94,7 +94,7 @@ struct Ptrs3 {
 // Input chunk = ((b*N + n)*Hh + h)*cpr + c.
 __global__ void __launch_bounds__(kThreads)
     reorder_fwd_kernel(Ptrs3 ptr, SlotMap map, uint32_t N, uint32_t Hh, uint32_t cpr_log2,
-                       uint32_t total, FastDiv div_Npad, FastDiv div_Hh) {
+                       uint32_t total, FastDiv div_Npad, FastDiv div_Hh, uint32_t write_pads) {
   const uint4* __restrict__ src = ptr.x[blockIdx.y];
   uint4* __restrict__ dst = ptr.y[blockIdx.y];
   const uint32_t cmask = (1u << cpr_log2) - 1u;
@@ -102,24 +102,25 @@ __global__ void __launch_bounds__(kThreads)
   for (uint32_t base = blockIdx.x * kThreads + threadIdx.x; base < total;
        base += stride * kUnroll) {
     uint4 v[kUnroll];
+    bool put[kUnroll];  // a token's slot, or an empty slot when pads are written
 #pragma unroll
     for (int u = 0; u < kUnroll; ++u) {
       const uint32_t idx = base + u * stride;
       v[u] = make_uint4(0u, 0u, 0u, 0u);
+      put[u] = false;
       if (idx < total) {
         uint32_t bh, slot, b, h;
         div_Npad.divmod(idx >> cpr_log2, bh, slot);
         div_Hh.divmod(bh, b, h);
         const int32_t n = map.token_of(slot);
+        put[u] = n >= 0 || write_pads;
         if (n >= 0)
           v[u] = __ldg(src + ((((int64_t)b * N + n) * Hh + h) << cpr_log2) + (idx & cmask));
       }
     }
 #pragma unroll
-    for (int u = 0; u < kUnroll; ++u) {
-      const uint32_t idx = base + u * stride;
-      if (idx < total) dst[idx] = v[u];
-    }
+    for (int u = 0; u < kUnroll; ++u)
+      if (put[u]) dst[base + u * stride] = v[u];
   }
 }
 
@@ -171,7 +172,7 @@ unsigned grid_for(uint64_t total) {
 }  // namespace
 
 cudaError_t launch_reorder_fwd(const Geometry& g, const void* const x[3], void* const y[3], int nt,
-                               cudaStream_t st) {
+                               bool write_pads, cudaStream_t st) {
   const SlotMap map = make_map(g);
   Ptrs3 p;
   for (int i = 0; i < 3; ++i) {
@@ -183,7 +184,8 @@ cudaError_t launch_reorder_fwd(const Geometry& g, const void* const x[3], void* 
   const dim3 grid(grid_for(total), (unsigned)nt);
   reorder_fwd_kernel<<<grid, kThreads, 0, st>>>(p, map, (uint32_t)(g.T * g.P), (uint32_t)g.Hh,
                                                 cpr_log2, (uint32_t)total,
-                                                FastDiv((uint32_t)g.Npad), FastDiv((uint32_t)g.Hh));
+                                                FastDiv((uint32_t)g.Npad), FastDiv((uint32_t)g.Hh),
+                                                write_pads ? 1u : 0u);
   return cudaGetLastError();
 }
 

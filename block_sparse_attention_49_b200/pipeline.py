@@ -15,14 +15,14 @@ import math
 
 import torch
 
-from . import (ANCHORS_ROTATING, DRAFT_FP64, LAYOUT_FRAME, LAYOUT_TILE, POOL_MEAN,
-               WINDOW_ALTERNATE, Plan,
+from . import (ANCHORS_ROTATING, DRAFT_FP64, LAYOUT_FRAME, LAYOUT_TILE, PADS_KEEP, PADS_WRITE,
+               POOL_MEAN, WINDOW_ALTERNATE, Plan,
                bsa_attn_fwd, bsa_attn_fwd_natural, bsa_attn_fwd_natural_e4m3,
                bsa_draft_keep_count, bsa_draft_mask, bsa_draft_mask_natural,
                bsa_draft_mask_natural_e4m3,
                bsa_draft_workspace_bytes, bsa_quantize_e4m3,
                bsa_lvsa_attn_fwd, bsa_lvsa_mask, bsa_lvsa_nnz, bsa_plan_set_draft_pooling,
-               bsa_plan_set_draft_precision,
+               bsa_plan_set_draft_precision, bsa_plan_set_reorder_pads,
                bsa_plan_set_lvsa_variant, bsa_reorder_fwd, bsa_reorder_inv)
 
 
@@ -33,13 +33,21 @@ class _Base:
         mk = lambda: torch.empty(shape, dtype=torch.bfloat16, device=device)
         self.q_s, self.k_s, self.v_s, self.o_s = mk(), mk(), mk(), mk()
         self.lse = torch.empty((p.B, p.Hh, p.Npad), dtype=torch.float32, device=device)
+        self._pads_zero = False  # the empty slots of q_s, k_s, v_s hold zeros
 
     def attend(self, per_head: bool):
         bsa_attn_fwd(self.plan, self.q_s, self.k_s, self.v_s, self.row_ptr, self.col_idx,
                      per_head, self.scale, self.o_s, self.lse)
 
     def gather(self, q, k, v):
-        bsa_reorder_fwd(self.plan, q, self.q_s, k, self.k_s, v, self.v_s)
+        # the slot buffers' empty slots are zeroed by the first gather; later
+        # ones write only the tokens (nothing else writes those slots)
+        bsa_plan_set_reorder_pads(self.plan, PADS_KEEP if self._pads_zero else PADS_WRITE)
+        try:
+            bsa_reorder_fwd(self.plan, q, self.q_s, k, self.k_s, v, self.v_s)
+        finally:
+            bsa_plan_set_reorder_pads(self.plan, PADS_WRITE)
+        self._pads_zero = True
 
     def scatter(self, out):
         bsa_reorder_inv(self.plan, self.o_s, out)

@@ -85,6 +85,9 @@ typedef enum {
 /* Draft pooling (bsa_plan_set_draft_pooling). */
 typedef enum { BSA_POOL_MEAN = 0, BSA_POOL_MAX = 1 } bsa_pooling;
 
+/* Empty slots written by bsa_reorder_fwd (bsa_plan_set_reorder_pads). */
+typedef enum { BSA_PADS_WRITE = 0, BSA_PADS_KEEP = 1 } bsa_reorder_pads;
+
 /* Precision of the draft logits (bsa_plan_set_draft_precision). */
 typedef enum { BSA_DRAFT_FP64 = 0, BSA_DRAFT_FP32 = 1 } bsa_draft_precision;
 
@@ -223,6 +226,16 @@ size_t bsa_draft_noalloc_max_scratch_bytes(void);
  * pair), x2/y2 only together with x1/y1; otherwise BSA_ERR_INVALID_ARG. */
 bsa_status bsa_reorder_fwd(bsa_plan_t plan, const void* x0, void* y0, const void* x1,
                            void* y1, const void* x2, void* y2, void* stream);
+
+/* Whether bsa_reorder_fwd with this plan writes the empty slots (default
+ * WRITE: zeros).  KEEP leaves them untouched and writes only the slots that
+ * hold tokens: for callers whose slot buffers already hold zeros there, for
+ * example buffers that an earlier call with WRITE filled and that nothing
+ * has written since (the other entry points only read the empty slots).
+ * The attention reads empty key slots, masked, so they must hold finite
+ * values.  Takes effect for calls issued after it; BSA_ERR_INVALID_ARG for
+ * unknown values. */
+bsa_status bsa_plan_set_reorder_pads(bsa_plan_t plan, int pads);
 
 /* Inverse reorder: slot layout [B, Hh, Npad, D] -> natural layout
  * [B, N, Hh, D], bit for bit; empty slots are dropped. */

@@ -115,6 +115,35 @@ def test_reorder_bit_exact(over, layout, blk):
     assert torch.equal(back.cpu().view(torch.int16), k.view(torch.int16))
 
 
+@pytest.mark.parametrize("layout", ["frame", "tile"])
+def test_reorder_keep_pads_writes_only_token_slots(layout):
+    # BSA_PADS_KEEP: the slots holding tokens get the tokens bit for bit;
+    # every empty slot keeps what the buffer held (here 7.0)
+    w = small_workload(CONFIGS[2], T=3, H=13, W=37, Hh=2, field_grid=(3, 4, 7))
+    q, _, _ = make_qkv(w)
+    if layout == "frame":
+        plan = bsa.Plan(w.B, w.Hh, w.D, w.T, w.H, w.W, bsa.LAYOUT_FRAME, block=128)
+        perm, Np = oracle.frame_layout_perm(w.T, w.H, w.W, 128)
+    else:
+        plan = bsa.Plan(w.B, w.Hh, w.D, w.T, w.H, w.W, bsa.LAYOUT_TILE, 8, 16, 128)
+        perm, Np = oracle.tile_layout_perm(w.T, w.H, w.W, 8, 16)
+    bsa.bsa_plan_set_reorder_pads(plan, bsa.PADS_KEEP)
+    y = torch.full((w.B, w.Hh, plan.Npad, w.D), 7.0, dtype=torch.bfloat16, device="cuda")
+    bsa.bsa_reorder_fwd(plan, q.cuda(), y)
+    bsa.bsa_poll_status(plan)
+    valid = np.zeros(plan.Npad, dtype=bool)
+    valid[:Np] = oracle.slot_valid(perm, Np)
+    ref = oracle.reorder_fwd(q.view(torch.int16).numpy(), perm, Np)
+    got = y.cpu().view(torch.int16).numpy()
+    np.testing.assert_array_equal(got[:, :, :Np][:, :, valid[:Np]], ref[:, :, valid[:Np]])
+    seven = torch.tensor(7.0, dtype=torch.bfloat16).view(torch.int16).item()
+    assert (got[:, :, ~valid] == seven).all() and (~valid).any()
+    # WRITE (the default) zeroes them again
+    bsa.bsa_plan_set_reorder_pads(plan, bsa.PADS_WRITE)
+    bsa.bsa_reorder_fwd(plan, q.cuda(), y)
+    assert (y.cpu().view(torch.int16).numpy()[:, :, ~valid] == 0).all()
+
+
 def test_reorder_rejects_a_third_pair_without_the_second():
     plan = bsa.Plan(1, 1, 64, 8, 8, 8, bsa.LAYOUT_FRAME, block=64)
     x = torch.zeros((1, 512, 1, 64), dtype=torch.bfloat16, device="cuda")

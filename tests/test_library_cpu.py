@@ -71,6 +71,7 @@ def test_null_plan_is_rejected(lib):
     assert lib.bsa_plan_set_lvsa_variant(None, 0, 0) == 1
     assert lib.bsa_plan_set_draft_pooling(None, 0) == 1
     assert lib.bsa_plan_set_draft_precision(None, 0) == 1
+    assert lib.bsa_plan_set_reorder_pads(None, 0) == 1
     assert lib.bsa_lvsa_attn_fwd(None, 4, 4, 0, None, None, None, 1.0, None, None, None) == 1
     assert lib.bsa_attn_fwd_natural(None, None, None, None, None, None, 1, 1.0, None, None,
                                     None) == 1
