@@ -698,6 +698,35 @@ def test_pool_sums_in_row_major_order():
     assert ((2.0 ** -53 + 1.0) + 2.0 ** -53) / 4 != got     # the other order differs
 
 
+def test_fp32_and_fp64_logits_within_the_certification_bound():
+    # The GPU takes the fp64 draft lists from fp32 logits wherever they are
+    # further than twice e = c |q| max|k| + 2^-100 from the k-th logit, with
+    # c = 2 (gamma_D(fp32) (1 + u32)^2 + 2 u32 + u32^2 + gamma_D(fp64)),
+    # gamma_n = n u / (1 - n u) (Higham, "Accuracy and Stability of Numerical
+    # Algorithms", sections 3.1 and 3.5).  The two oracles' logits must be
+    # that close on every pair, here on random rows, on rows spread over
+    # many binades, and on nearly cancelling rows.
+    rng = np.random.default_rng(17)
+    D = 128
+    u32, u64 = 2.0 ** -24, 2.0 ** -53
+    g32, g64 = D * u32 / (1 - D * u32), D * u64 / (1 - D * u64)
+    c = 2.0 * (g32 * (1 + u32) ** 2 + 2 * u32 + u32 * u32 + g64)
+    cases = [rng.standard_normal((2, 40, D)),
+             rng.standard_normal((2, 40, D)) * np.exp2(rng.integers(-30, 30, size=(2, 40, D)))]
+    base = rng.standard_normal((1, 40, D))
+    cases.append(np.concatenate([base, -base + 1e-7 * rng.standard_normal((1, 40, D))]))
+    for x in cases:
+        q, k = x[0][None, None], x[1][None, None]
+        L64 = oracle.draft_logits(q, k)[0, 0]
+        L32 = oracle.draft_logits(q, k, "fp32")[0, 0].astype(np.float64)
+        qn = np.sqrt((x[0] ** 2).sum(-1))
+        kn = np.sqrt((x[1] ** 2).sum(-1))
+        e = c * qn[:, None] * kn.max() + 2.0 ** -100
+        assert (np.abs(L32 - L64) <= e).all()
+        assert (np.abs(L32 - L64) <= c * qn[:, None] * kn[None, :] + 2.0 ** -100).all()
+        assert (L32 != L64).any()      # the precisions do differ
+
+
 def test_logits_are_sequential_and_unfused():
     # channel 0 first: acc = -(1 + 2^-29); channel 1 adds the rounded product
     # x*x with x = 1 + 2^-30, i.e. 1 + 2^-29 (the exact square carries an
