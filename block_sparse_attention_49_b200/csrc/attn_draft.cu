@@ -939,8 +939,7 @@ bsa_status launch_attn_draft(const bsa_plan_s& plan, const void* q, const void* 
         !make_draft_tmap(&tv, v, g, g.pw, g.ph, f8))
       return set_error(BSA_ERR_CUDA, "cuTensorMapEncodeTiled (5-D) failed");
   }
-  DraftParams p;
-  memset(&p, 0, sizeof(p));
+  DraftParams p{};  // every field zero (the divisors 1) until set below
   p.slot = slot ? 1 : 0;
   p.Npad = g.Npad;
   p.fp8_scales = fp8_scales;
