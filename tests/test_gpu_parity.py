@@ -279,6 +279,47 @@ def test_draft_mask_logits_equal_in_fp32_but_not_in_fp64():
         assert (got == np.array(want[precision])[None, :]).all(), (precision, got)
 
 
+def test_draft_mask_fp32_overflow_decided_in_fp64():
+    # pooled values 2^66 and 2^66 (1 + j/64): every product overflows fp32,
+    # so the fp32 logits are all +inf and tie, while the fp64 ones are
+    # distinct.  The fp64 lists then come from the fp64 logits of every
+    # block (the overflow path of the certification): blocks 8..15; fp32
+    # precision keeps the lowest indices, 0..7.
+    T, H, W, D, ph, pw = 1, 4, 16, 64, 2, 2
+    q = torch.full((1, T * H * W, 1, D), 2.0 ** 66, dtype=torch.bfloat16)
+    k = torch.zeros_like(q)
+    for y in range(H):
+        for x in range(W):
+            j = (y // ph) * (W // pw) + x // pw
+            k[0, y * W + x, 0, :] = 2.0 ** 66 * (1 + j / 64)
+    qbar = oracle.draft_pool(to_np64(q), T, H, W, ph, pw)
+    kbar = oracle.draft_pool(to_np64(k), T, H, W, ph, pw)
+    L64 = oracle.draft_logits(qbar, kbar)
+    with np.errstate(over="ignore"):
+        L32 = oracle.draft_logits(qbar, kbar, "fp32")
+    assert np.isinf(L32).all() and np.isfinite(L64).all()
+    for precision, L, want in ((bsa.DRAFT_FP64, L64, np.arange(8, 16)),
+                               (bsa.DRAFT_FP32, L32, np.arange(8))):
+        ref = oracle.draft_topk(L, 8)
+        assert (ref == want).all()
+        plan = bsa.Plan(1, 1, D, T, H, W, bsa.LAYOUT_TILE, ph, pw, ph * pw)
+        bsa.bsa_plan_set_draft_precision(plan, precision)
+        assert plan.nblocks == 16 and bsa.bsa_draft_keep_count(plan, 50) == 8
+        perm, Np = oracle.tile_layout_perm(T, H, W, ph, pw)
+        qs, ks = _slots_gpu(q, perm, plan.Npad), _slots_gpu(k, perm, plan.Npad)
+        rp = torch.empty(17, dtype=torch.int32, device="cuda")
+        kv = torch.empty(16 * 8, dtype=torch.int32, device="cuda")
+        dm = (torch.empty(16 * 16, dtype=torch.float32, device="cuda")
+              if precision == bsa.DRAFT_FP64 else None)
+        ws = torch.empty(bsa.bsa_draft_workspace_bytes(plan), dtype=torch.uint8, device="cuda")
+        bsa.bsa_draft_mask(plan, qs, ks, 50, rp, kv, dm, ws)
+        bsa.bsa_poll_status(plan)
+        np.testing.assert_array_equal(kv.cpu().numpy().reshape(1, 1, 16, 8), ref)
+        if dm is not None:
+            np.testing.assert_allclose(dm.cpu().numpy().reshape(1, 1, 16, 16),
+                                       oracle.draft_map(L64, D), rtol=1e-6, atol=1e-12)
+
+
 @pytest.mark.parametrize("precision", [bsa.DRAFT_FP64, bsa.DRAFT_FP32])
 def test_draft_mask_all_logits_equal(precision):
     # constant Q and K: every logit of a row is the same, so the kept blocks
