@@ -230,20 +230,29 @@ def test_attn_natural_rejects_unsupported_plans():
     assert ei.value.status == 2
 
 
-def test_draft_mask_many_blocks_takes_the_shared_memory_selection():
+@pytest.mark.parametrize("precision", [bsa.DRAFT_FP64, bsa.DRAFT_FP32])
+def test_draft_mask_many_blocks_takes_the_shared_memory_selection(precision):
     # 2 x 64 x 64 grid with 2 x 2 tiles: 2048 blocks per row, more than the
-    # register-held candidates of the top-k, so the other selection path runs
+    # register-held logits of the scorer, so the shared-memory kernel runs
+    # (in the plan's precision); the draft map is checked too
     w = small_workload(CONFIGS[1], T=2, H=64, W=64, Hh=1, D=64, qk="iid", draft_ph=2, draft_pw=2,
                        draft_sparsity=95)
     q, k, _ = make_qkv(w, device="cuda")
     plan = bsa.Plan(w.B, w.Hh, w.D, w.T, w.H, w.W, bsa.LAYOUT_TILE, 2, 2, 4)
+    bsa.bsa_plan_set_draft_precision(plan, precision)
     nb = plan.nblocks
     assert nb == 2048
     keep = bsa.bsa_draft_keep_count(plan, 95)
     kv = torch.empty(nb * keep, dtype=torch.int32, device="cuda")
-    ws = torch.empty(((bsa.bsa_draft_workspace_bytes(plan) + 7) // 8,), dtype=torch.float64,
-                     device="cuda")
-    bsa.bsa_draft_mask_natural(plan, q, k, 95, None, kv, None, ws)
+    dm = torch.empty(nb * nb, dtype=torch.float32, device="cuda")
+    ws = torch.empty(bsa.bsa_draft_workspace_bytes(plan), dtype=torch.uint8, device="cuda")
+    bsa.bsa_draft_mask_natural(plan, q, k, 95, None, kv, dm, ws)
     bsa.bsa_poll_status(plan)
-    ref = oracle.draft_blocks(to_np64(q), to_np64(k), w.T, w.H, w.W, 2, 2, 95)
+    prec = "fp64" if precision == bsa.DRAFT_FP64 else "fp32"
+    qbar = oracle.draft_pool(to_np64(q), w.T, w.H, w.W, 2, 2)
+    kbar = oracle.draft_pool(to_np64(k), w.T, w.H, w.W, 2, 2)
+    L = oracle.draft_logits(qbar, kbar, prec)
+    ref = oracle.draft_topk(L, keep)
     np.testing.assert_array_equal(kv.cpu().numpy().reshape(1, 1, nb, keep), ref)
+    np.testing.assert_allclose(dm.cpu().numpy().reshape(1, 1, nb, nb), oracle.draft_map(L, w.D),
+                               rtol=1e-5, atol=1e-7)
