@@ -45,7 +45,7 @@ constexpr unsigned kFullMaskScore = 0xffffffffu;
 // Pooling.  One group of D/8 threads per unit (Q or K, tile, batch, head);
 // each thread owns 8 channels: eight independent fp64 chains, each the
 // sequential sum over the tile's tokens in row-major order, stored as fp32.  Token rows are
-// read with 16-byte loads, four rows ahead of the additions.  Units are
+// read with 16-byte streaming loads (no L1 allocation), four rows ahead of the additions.  Units are
 // ordered heads fastest, so the groups of a warp read neighbouring 256-byte
 // rows of one token.  At most 64 registers a thread: four 256-thread CTAs fit
 // on an SM, so a 12-head Wan-1.3B-like problem runs in one wave.
@@ -108,7 +108,7 @@ __global__ void __launch_bounds__(kPoolThreads, 4)
       uint4 v[kAhead];
 #pragma unroll
       for (int u = 0; u < kAhead; ++u)
-        if (c0 + u < len) v[u] = __ldg(rowp + (int64_t)(c0 + u) * row_step);
+        if (c0 + u < len) v[u] = ld_stream_v4(rowp + (int64_t)(c0 + u) * row_step);
 #pragma unroll
       for (int u = 0; u < kAhead; ++u) {
         if (c0 + u >= len) break;
@@ -638,7 +638,11 @@ __global__ void __launch_bounds__(32 * kRegScoreWarps, U <= 12 ? 4 : 3)
   // with at least k keys >= T), for the warp's R rows side by side; then
   // every key above T is taken, and of the keys equal to T the ones with the
   // lowest block indices.  Blocks past the grid (and rows past it) hold key
-  // 0, below every real key.
+  // 0, below every real key.  With fp32 lists the search stops once every
+  // row has exactly k keys >= its prefix Tk: those k keys are the selection
+  // whatever the remaining bits, and the tie rule on Tk takes all of them.
+  // (The fp64 lists' kernel runs every bit: stopping early measured slower
+  // there, although the result is the same.)
   uint32_t key[R][U];
 #pragma unroll
   for (int r = 0; r < R; ++r) {
@@ -651,10 +655,20 @@ __global__ void __launch_bounds__(32 * kRegScoreWarps, U <= 12 ? 4 : 3)
     }
   }
   uint32_t Tk[R];
+  unsigned nge[R];  // keys >= Tk[r]; rows past the grid count as settled
 #pragma unroll
-  for (int r = 0; r < R; ++r) Tk[r] = 0u;
+  for (int r = 0; r < R; ++r) {
+    Tk[r] = 0u;
+    nge[r] = r0 + warp * R + r < nblocks ? 32u * U : (unsigned)keep;
+  }
 #pragma unroll 1
   for (int bit = 31; bit >= 0; --bit) {
+    if constexpr (!CERT) {
+      bool settled = true;
+#pragma unroll
+      for (int r = 0; r < R; ++r) settled = settled && nge[r] == (unsigned)keep;
+      if (settled) break;  // warp-uniform: the counts are warp sums
+    }
     unsigned tot[R];
 #pragma unroll
     for (int r = 0; r < R; ++r) {
@@ -666,7 +680,10 @@ __global__ void __launch_bounds__(32 * kRegScoreWarps, U <= 12 ? 4 : 3)
     }
 #pragma unroll
     for (int r = 0; r < R; ++r)
-      if (tot[r] >= (unsigned)keep) Tk[r] |= 1u << bit;
+      if (tot[r] >= (unsigned)keep) {
+        Tk[r] |= 1u << bit;
+        nge[r] = tot[r];
+      }
   }
   float kmax = 0.f;  // CERT: the largest key-block norm of this (b, head)
   if constexpr (CERT) {
@@ -688,7 +705,7 @@ __global__ void __launch_bounds__(32 * kRegScoreWarps, U <= 12 ? 4 : 3)
       // k-th one are in, more than twice below it out, whatever the fp64
       // logits; the rest (the band) is decided on the fp64 logits unless
       // all of it is needed
-      const double t = (double)key_value(Tk[r]);
+      const double t = (double)key_value(Tk[r]);  // the k-th largest fp32 logit
       const double e = ErrBound<D>::value * (double)qnorm[bh * nblocks + row] * (double)kmax + 0x1p-100;
       // bounds rounded outwards to fp32: compared with the fp32 logits they
       // keep every block the fp64 bounds would put in the band

@@ -25,6 +25,16 @@ __device__ __forceinline__ bool elect_one() {
   return pred != 0;
 }
 
+// 16 bytes of read-only global data that is read once: no L1 line is
+// allocated for it, and L2 fetches the surrounding 128-byte line.
+__device__ __forceinline__ uint4 ld_stream_v4(const uint4* p) {
+  uint4 r;
+  asm volatile("ld.global.nc.L1::no_allocate.L2::128B.v4.u32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
+               : "l"(p));
+  return r;
+}
+
 // ---------------------------------------------------------------- mbarrier
 __device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
   asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count)
