@@ -191,6 +191,12 @@ DRAFT_CASES = [
     dict(cid=2),
     dict(cid=1, T=3, H=5, W=7, Hh=3, D=128, qk="iid", draft_ph=4, draft_pw=4, draft_sparsity=70),
     dict(cid=5),
+    # rows of exactly 32 blocks (no padded keys): keep = the whole row, where
+    # the threshold search is settled before its first bit, and keep = 1
+    dict(cid=1, T=2, H=16, W=32, Hh=2, D=128, qk="iid", draft_ph=4, draft_pw=8, draft_sparsity=0),
+    dict(cid=1, T=2, H=16, W=32, Hh=2, D=128, qk="iid", draft_ph=4, draft_pw=8, draft_sparsity=97),
+    # 64 blocks, half kept, head dim 64
+    dict(cid=1, T=4, H=16, W=32, Hh=2, D=64, qk="iid", draft_ph=4, draft_pw=8, draft_sparsity=50),
 ]
 
 
