@@ -99,9 +99,12 @@ __device__ __forceinline__ float quotient_for_e4m3(float x, float s, float r) {
   return safe ? y : __fdiv_rn(x, s);
 }
 
-// grid-stride over the 8-value groups of one tensor (blockIdx.y); the group
-// count of a tensor is below 2^31 (the plan checks it), so 32-bit indices
-// and magic-number division give (b, h) of a group
+// grid-stride over pairs of 8-value groups of one tensor (blockIdx.y): the
+// two groups of a pair lie in one token row, so they share the index
+// arithmetic and the scale loads, and their 16 codes go out in one 16-byte
+// store (the e4m3 buffers are 16-byte aligned: the entry points check it).
+// The group count of a tensor is below 2^31 (the plan checks it), so 32-bit
+// indices and magic-number division give (b, h) of a group
 template <int D>
 __global__ void __launch_bounds__(kThreads)
     e4m3_convert_kernel(const uint4* __restrict__ q, const uint4* __restrict__ k,
@@ -116,22 +119,27 @@ __global__ void __launch_bounds__(kThreads)
   const float* sc = scales + (int64_t)which * B * Hh;
   const float* rc = recips + (int64_t)which * B * Hh;
   const uint32_t stride = gridDim.x * kThreads;
-  for (uint32_t r = blockIdx.x * kThreads + threadIdx.x; r < per; r += stride) {
+  const uint32_t per2 = per >> 1;  // pairs of groups (a row holds 8 or 16 groups)
+  for (uint32_t r2 = blockIdx.x * kThreads + threadIdx.x; r2 < per2; r2 += stride) {
+    const uint32_t r = r2 << 1;
     const uint32_t row = r >> kShift;                  // (b * N + n) * Hh + h
     const uint32_t bn = div_Hh.div(row);
     const int h = (int)(row - bn * (uint32_t)Hh);
     const int b = (int)div_batch.div(r);               // r / (N * Hh * D / 8)
     const float s = __ldg(sc + b * Hh + h), rs = __ldg(rc + b * Hh + h);
-    const uint4 u = __ldg(x + r);
-    const __nv_bfloat162* pv = reinterpret_cast<const __nv_bfloat162*>(&u);
-    uint32_t w[2];
+    const uint4 u0 = __ldg(x + r), u1 = __ldg(x + r + 1);
+    uint32_t w[4];
 #pragma unroll
-    for (int i = 0; i < 2; ++i) {
-      const float2 f0 = __bfloat1622float2(pv[2 * i]), f1 = __bfloat1622float2(pv[2 * i + 1]);
-      w[i] = e4m3x2(quotient_for_e4m3(f0.x, s, rs), quotient_for_e4m3(f0.y, s, rs)) |
-             (e4m3x2(quotient_for_e4m3(f1.x, s, rs), quotient_for_e4m3(f1.y, s, rs)) << 16);
+    for (int g = 0; g < 2; ++g) {
+      const __nv_bfloat162* pv = reinterpret_cast<const __nv_bfloat162*>(g ? &u1 : &u0);
+#pragma unroll
+      for (int i = 0; i < 2; ++i) {
+        const float2 f0 = __bfloat1622float2(pv[2 * i]), f1 = __bfloat1622float2(pv[2 * i + 1]);
+        w[2 * g + i] = e4m3x2(quotient_for_e4m3(f0.x, s, rs), quotient_for_e4m3(f0.y, s, rs)) |
+                       (e4m3x2(quotient_for_e4m3(f1.x, s, rs), quotient_for_e4m3(f1.y, s, rs)) << 16);
+      }
     }
-    y[r] = make_uint2(w[0], w[1]);
+    reinterpret_cast<uint4*>(y)[r2] = make_uint4(w[0], w[1], w[2], w[3]);
   }
 }
 
